@@ -1,0 +1,200 @@
+/*
+ * zt_q4_oracle.c -- the plain, slow CPU oracle for the q4f16 dequantizing
+ * matrix-vector product.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path may link,
+ * load or call this file; only the tests, the smoke check and the bench's
+ * CPU-baseline leg do.  It shares no code, header, table or constant generator
+ * with the CUDA library: every step here is written out from the definition.
+ *
+ * What it computes (all arithmetic in IEEE double):
+ *
+ *   The pages (Zero-TVM forum write-up, section "完整的推理流水线") name the
+ *   compute core "int4 反量化矩阵乘法" -- an int4 dequantizing matrix product --
+ *   with a plain variant, and an f32-output variant for the LM head "for
+ *   sampling stability"; the same page's performance section names the
+ *   weights "Phi-3-mini-q4f16_1": 4-bit weights, fp16 scales, fp16
+ *   activations.  The pages do not spell out the bit format.  This library
+ *   fixes it as follows (the plainest reading consistent with the pages):
+ *
+ *     weights   W is N x K (out x in).  qw is uint32 [N][K/8]; element (n,k)
+ *               is bits 4*(k%8) .. 4*(k%8)+3 of qw[n][k/8]  (low nibble first)
+ *     scales    fp16 [N][K/32], one per group of 32 consecutive k
+ *     dequant   w[n][k] = (q[n][k] - 7) * s[n][k/32]
+ *     product   y[m][n] = sum_k w[n][k] * x[m][k], summed in plain k order
+ *
+ *   fused FFN ("fused_ffn.wgsl": gate, up and SiLU in one pass, section
+ *   "内核融合"): weight rows [0,N) are gate, rows [N,2N) are up;
+ *   out[m][n] = SiLU(g) * u with SiLU(g) = g / (1 + exp(-g)).
+ *
+ *   LM head + greedy sampling (section "完整的推理流水线": f32 LM head and "a
+ *   simple argmax dispatch"): logits = y kept in double; argmax = the lowest
+ *   index among the maxima, NaN treated as -infinity.
+ *
+ * Every function computes each output row with the same fixed sequence of
+ * operations, so the optional OpenMP split over rows (threads > 1) returns
+ * bit-identical results to the single-threaded run.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define ZTO_GROUP 32   /* k values per fp16 scale */
+#define ZTO_ZERO 7     /* the zero point subtracted from every 4-bit code */
+
+/* IEEE-754 binary16 bit pattern -> double, written out from the format:
+ * 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double zto_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1F;
+    int frac = h & 0x3FF;
+    double v;
+    if (expo == 0) {
+        v = ldexp((double)frac, -24);                 /* zero / subnormal */
+    } else if (expo == 31) {
+        v = frac ? NAN : INFINITY;                    /* inf / NaN */
+    } else {
+        v = ldexp((double)(1024 + frac), expo - 25);  /* normal */
+    }
+    return sign ? -v : v;
+}
+
+/* The 4-bit code of element (n,k): the (k%8)-th nibble, counted from the
+ * least significant end, of word qw[n][k/8]. */
+static int zto_code(const uint32_t *qw, int64_t K, int64_t n, int64_t k)
+{
+    uint32_t word = qw[n * (K / 8) + k / 8];
+    return (int)((word >> (4 * (k % 8))) & 0xFu);
+}
+
+/* Dequantized weight w[n][k] = (q - 7) * s, exact in double. */
+static double zto_weight(const uint32_t *qw, const uint16_t *scales, int64_t K,
+                         int64_t n, int64_t k)
+{
+    double s = zto_half_to_double(scales[n * (K / ZTO_GROUP) + k / ZTO_GROUP]);
+    return (double)(zto_code(qw, K, n, k) - ZTO_ZERO) * s;
+}
+
+/* One dot product: sum over k = 0..K-1, in that order, of w[n][k] * x[m][k]. */
+static double zto_row_dot(const uint32_t *qw, const uint16_t *scales,
+                          const uint16_t *x, int64_t K, int64_t m, int64_t n)
+{
+    double acc = 0.0;
+    for (int64_t k = 0; k < K; ++k)
+        acc += zto_weight(qw, scales, K, n, k) * zto_half_to_double(x[m * K + k]);
+    return acc;
+}
+
+static int zto_shape_ok(int M, int N, int K)
+{
+    return M >= 1 && N >= 1 && K >= ZTO_GROUP && K % ZTO_GROUP == 0;
+}
+
+/* Unpack codes: q[n][k] (one byte each, 0..15) from qw[n][K/8]. */
+int zto_unpack(const uint32_t *qw, int N, int K, uint8_t *q)
+{
+    if (!qw || !q || N < 1 || K < 8 || K % 8) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (uint8_t)zto_code(qw, K, n, k);
+    return 0;
+}
+
+/* Pack codes 0..15 into words, low nibble first. Codes above 15 are an error. */
+int zto_pack(const uint8_t *q, int N, int K, uint32_t *qw)
+{
+    if (!qw || !q || N < 1 || K < 8 || K % 8) return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t w = 0; w < K / 8; ++w) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j) {
+                uint8_t c = q[n * K + 8 * w + j];
+                if (c > 15) return -1;
+                word |= (uint32_t)c << (4 * j);
+            }
+            qw[n * (K / 8) + w] = word;
+        }
+    }
+    return 0;
+}
+
+/* y[m][i] = sum_k w[row_i][k] x[m][k].  rows == NULL computes every row
+ * (n_rows must equal N and row_i = i); otherwise only the listed rows, and y is
+ * [M][n_rows].  Output in double, no rounding to fp16. */
+int zto_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+             int M, int N, int K, const int32_t *rows, int n_rows,
+             double *y, int threads)
+{
+    if (!qw || !scales || !x || !y || !zto_shape_ok(M, N, K)) return -1;
+    if (!rows) n_rows = N;
+    for (int i = 0; rows && i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= N) return -1;
+    if (threads < 1) threads = 1;
+#pragma omp parallel for schedule(static) num_threads(threads)
+    for (int i = 0; i < n_rows; ++i) {
+        int64_t n = rows ? rows[i] : i;
+        for (int64_t m = 0; m < M; ++m)
+            y[m * n_rows + i] = zto_row_dot(qw, scales, x, K, m, n);
+    }
+    return 0;
+}
+
+/* SiLU(g) = g * sigmoid(g) = g / (1 + exp(-g)). */
+double zto_silu(double g)
+{
+    return g / (1.0 + exp(-g));
+}
+
+/* Fused gate/up + SiLU.  qw and scales hold 2N rows: rows 0..N-1 are the gate
+ * projection, rows N..2N-1 the up projection.  out[m][i] = SiLU(g) * u with
+ * g = dot(gate row n), u = dot(up row n), n = rows[i] (or i), all in double. */
+int zto_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                     int M, int N, int K, const int32_t *rows, int n_rows,
+                     double *out, int threads)
+{
+    if (!qw || !scales || !x || !out || !zto_shape_ok(M, N, K)) return -1;
+    if (!rows) n_rows = N;
+    for (int i = 0; rows && i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= N) return -1;
+    if (threads < 1) threads = 1;
+#pragma omp parallel for schedule(static) num_threads(threads)
+    for (int i = 0; i < n_rows; ++i) {
+        int64_t n = rows ? rows[i] : i;
+        for (int64_t m = 0; m < M; ++m) {
+            double g = zto_row_dot(qw, scales, x, K, m, n);
+            double u = zto_row_dot(qw, scales, x, K, m, n + N);
+            out[m * n_rows + i] = zto_silu(g) * u;
+        }
+    }
+    return 0;
+}
+
+/* Greedy sampling over one row of logits: the lowest index among the maxima.
+ * NaN compares as -infinity, so a row of NaNs (or of -inf) returns 0. */
+int32_t zto_argmax(const double *v, int N)
+{
+    int32_t best = 0;
+    double best_v = isnan(v[0]) ? -INFINITY : v[0];
+    for (int32_t n = 1; n < N; ++n) {
+        double c = isnan(v[n]) ? -INFINITY : v[n];
+        if (c > best_v) {   /* strict: an equal later value never wins */
+            best_v = c;
+            best = n;
+        }
+    }
+    return best;
+}
+
+/* LM head: logits[m][n] (double, never rounded to fp16) and argmax[m]. */
+int zto_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                      int M, int N, int K, double *logits, int32_t *argmax,
+                      int threads)
+{
+    if (!qw || !scales || !x || !logits || !argmax || !zto_shape_ok(M, N, K)) return -1;
+    int rc = zto_gemv(qw, scales, x, M, N, K, NULL, N, logits, threads);
+    if (rc) return rc;
+    for (int64_t m = 0; m < M; ++m)
+        argmax[m] = zto_argmax(logits + m * N, N);
+    return 0;
+}

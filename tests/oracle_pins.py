@@ -1,0 +1,295 @@
+"""Pins that tie the oracle to something other than itself.
+
+Each ``pin_*`` function takes an ``oracle.Oracle`` and raises AssertionError
+when the oracle disagrees with what the format, the mathematics or a library
+routine fixes.  ``test_oracle.py`` runs them against the real oracle (all must
+pass) and ``test_oracle_mutants.py`` runs them against deliberately broken
+copies of it (each copy must fail at least one).
+
+Independent routes used here, none of which calls the oracle's own helpers:
+
+* fp16 decoding -- numpy's float16 -> float64 conversion (library routine);
+* nibble order  -- a word's hexadecimal digits read least-significant first
+  (string formatting, no shifts or masks);
+* sums          -- exact rational arithmetic (``fractions.Fraction``) or
+  numpy's float64 matrix product on a dense matrix built by the hex route;
+* SiLU          -- closed values: SiLU(0) = 0, SiLU(ln 3) = (3/4) ln 3,
+  SiLU(g) - SiLU(-g) = g, SiLU(g) -> g as g -> +inf;
+* argmax        -- hand-built logit vectors.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                      "q4_worked_examples.txt")
+
+
+# ---------------------------------------------------------------- helpers --
+def codes_by_hex(qw: np.ndarray) -> np.ndarray:
+    """4-bit codes of packed words, by reading each word's hex digits from the
+    least significant end (low nibble first)."""
+    qw = np.asarray(qw, dtype=np.uint32)
+    N, W = qw.shape
+    out = np.empty((N, 8 * W), dtype=np.uint8)
+    for n in range(N):
+        digits = "".join(format(int(w), "08x")[::-1] for w in qw[n])
+        out[n] = [int(c, 16) for c in digits]
+    return out
+
+
+def dense_weights(qw: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """W[n][k] = (q - 7) * s as float64, codes by the hex route."""
+    q = codes_by_hex(qw).astype(np.float64)
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)
+    return (q - 7.0) * np.repeat(s, 32, axis=1)
+
+
+def exact_dot(qrow, srow, xrow) -> Fraction:
+    """sum_k (q_k - 7) * s_{k//32} * x_k in exact rationals."""
+    tot = Fraction(0)
+    for k, c in enumerate(qrow):
+        tot += (int(c) - 7) * Fraction(float(srow[k // 32])) * Fraction(float(xrow[k]))
+    return tot
+
+
+def small_problem(seed: int, N: int, K: int, M: int = 1):
+    g = np.random.default_rng([seed, 12345])
+    qw = g.integers(0, 2**32, size=(N, K // 8), dtype=np.uint32)
+    s = g.uniform(0.005, 0.02, size=(N, K // 32)).astype(np.float16)
+    x = g.standard_normal((M, K)).astype(np.float16)
+    return qw, s, x
+
+
+def parse_golden(path: str = GOLDEN):
+    cases, cur = [], None
+    with open(path) as fh:
+        for raw in fh:
+            line = raw.split("#", 1)[0].strip()
+            if not line:
+                continue
+            tok = line.split()
+            if tok[0] == "case":
+                cur = {"name": tok[1], "kind": tok[2]}
+            elif tok[0] == "end":
+                cases.append(cur)
+                cur = None
+            else:
+                cur[tok[0]] = tok[1:]
+    out = []
+    for c in cases:
+        K, N, M = int(c["K"][0]), int(c["N"][0]), int(c["M"][0])
+        rows = 2 * N if c["kind"] == "gate_up" else N
+        d = {
+            "name": c["name"], "kind": c["kind"], "K": K, "N": N, "M": M,
+            "qw": np.array([int(v, 16) for v in c["qw"]], dtype=np.uint32).reshape(rows, K // 8),
+            "scales": np.array([int(v, 16) for v in c["scales"]], dtype=np.uint16)
+                        .view(np.float16).reshape(rows, K // 32),
+            "x": np.array([int(v, 16) for v in c["x"]], dtype=np.uint16)
+                   .view(np.float16).reshape(M, K),
+            "y": np.array([float(v) for v in c["y"]], dtype=np.float64).reshape(M, N),
+        }
+        if "argmax" in c:
+            d["argmax"] = np.array([int(v) for v in c["argmax"]], dtype=np.int32)
+        out.append(d)
+    return out
+
+
+# ------------------------------------------------------------------- pins --
+def pin_half_decode(o):
+    """Every one of the 65536 fp16 bit patterns decodes as numpy decodes it."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = o.half_to_double(bits)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "NaN patterns decode differently"
+    assert np.array_equal(got[~nan], ref[~nan]), "finite/inf fp16 decode mismatch"
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan])), "sign of zero"
+
+
+def pin_pack_words(o):
+    """Hand-written words: codes are stored low nibble first."""
+    q = np.array([[1, 2, 3, 4, 5, 6, 7, 8],
+                  [15, 0, 0, 0, 0, 0, 0, 0],
+                  [0, 0, 0, 0, 0, 0, 0, 15],
+                  [0, 1, 2, 3, 4, 5, 6, 7]], dtype=np.uint8)
+    want = np.array([[0x87654321], [0x0000000F], [0xF0000000], [0x76543210]], dtype=np.uint32)
+    got = o.pack(q)
+    assert np.array_equal(got, want), f"pack: {[hex(int(v)) for v in got.ravel()]}"
+    assert np.array_equal(o.unpack(want, 8), q), "unpack of hand-written words"
+
+
+def pin_unpack_matches_hex(o):
+    qw, _, _ = small_problem(1, 5, 96)
+    assert np.array_equal(o.unpack(qw, 96), codes_by_hex(qw)), "unpack vs hex digits"
+
+
+def pin_roundtrip(o):
+    qw, _, _ = small_problem(2, 7, 256)
+    q = o.unpack(qw, 256)
+    assert np.array_equal(o.pack(q), qw), "pack(unpack(qw)) != qw"
+    g = np.random.default_rng(3)
+    q2 = g.integers(0, 16, size=(3, 64), dtype=np.uint8)
+    assert np.array_equal(o.unpack(o.pack(q2), 64), q2), "unpack(pack(q)) != q"
+
+
+def pin_zero_x(o):
+    qw, s, x = small_problem(4, 9, 128, M=2)
+    y = o.gemv(qw, s, np.zeros_like(x))
+    assert np.all(y == 0.0), "zero activations must give exactly zero"
+
+
+def pin_scale_doubling(o):
+    qw, s, x = small_problem(5, 6, 256, M=3)
+    s2 = (s.astype(np.float32) * 2).astype(np.float16)          # exact in fp16
+    assert np.array_equal(s2.astype(np.float64), 2 * s.astype(np.float64))
+    assert np.array_equal(o.gemv(qw, s2, x), 2.0 * o.gemv(qw, s, x)), "y(2s) != 2 y(s)"
+
+
+def pin_all_ones(o):
+    """x = 1: y_n = sum_g s_ng * (sum_{k in g} q_nk - 224), exact."""
+    N, K = 16, 256
+    qw, s, _ = small_problem(6, N, K)
+    x = np.ones((1, K), dtype=np.float16)
+    q = codes_by_hex(qw)
+    y = o.gemv(qw, s, x)
+    for n in range(N):
+        want = sum(Fraction(float(s[n, g])) * (int(q[n, 32 * g:32 * g + 32].sum()) - 224)
+                   for g in range(K // 32))
+        assert Fraction(float(y[0, n])) == want, f"all-ones closed form, row {n}"
+
+
+def pin_one_hot(o):
+    """x = e_k: y_n = (q_nk - 7) * s_n,k/32, exactly, for every k."""
+    N, K = 4, 64
+    qw, s, _ = small_problem(7, N, K)
+    q = codes_by_hex(qw)
+    for k in range(K):
+        x = np.zeros((1, K), dtype=np.float16)
+        x[0, k] = 1.0
+        y = o.gemv(qw, s, x)[0]
+        want = (q[:, k].astype(np.float64) - 7.0) * s[:, k // 32].astype(np.float64)
+        assert np.array_equal(y, want), f"one-hot k={k}"
+
+
+def pin_brute_force_tiny(o):
+    """K = 32, N = 3, M = 2 against exact rationals."""
+    qw, s, x = small_problem(8, 3, 32, M=2)
+    q = codes_by_hex(qw)
+    y = o.gemv(qw, s, x)
+    for m in range(2):
+        for n in range(3):
+            exact = exact_dot(q[n], s[n], x[m])
+            mag = sum(abs((int(c) - 7) * float(s[n, k // 32]) * float(x[m, k]))
+                      for k, c in enumerate(q[n]))
+            assert abs(float(y[m, n]) - float(exact)) <= 1e-14 * mag, f"brute force m={m} n={n}"
+
+
+def pin_numpy_dense(o):
+    """The double matvec against numpy's W @ x^T on a hex-route dense W."""
+    qw, s, x = small_problem(9, 64, 512, M=3)
+    W = dense_weights(qw, s)
+    ref = (W @ x.astype(np.float64).T).T
+    y = o.gemv(qw, s, x)
+    mag = np.abs(W) @ np.abs(x.astype(np.float64)).T
+    assert np.all(np.abs(y - ref) <= 1e-13 * mag.T), "oracle vs numpy dense matvec"
+
+
+def pin_row_subset(o):
+    """A row subset returns exactly the listed rows of the full product."""
+    qw, s, x = small_problem(10, 20, 128, M=2)
+    full = o.gemv(qw, s, x)
+    rows = np.array([19, 0, 7, 7, 3], dtype=np.int32)
+    assert np.array_equal(o.gemv(qw, s, x, rows=rows), full[:, rows]), "row subset"
+
+
+def pin_threads_identical(o):
+    qw, s, x = small_problem(11, 33, 256, M=2)
+    assert np.array_equal(o.gemv(qw, s, x, threads=1), o.gemv(qw, s, x, threads=4))
+
+
+def pin_silu_closed_values(o):
+    assert o.silu(0.0) == 0.0
+    assert math.isclose(o.silu(math.log(3.0)), 0.75 * math.log(3.0), rel_tol=1e-15)
+    for g in (0.3, 1.7, 5.0, 11.0):
+        assert math.isclose(o.silu(g) - o.silu(-g), g, rel_tol=1e-14), f"odd part at {g}"
+    assert o.silu(200.0) == 200.0
+    assert abs(o.silu(-200.0)) < 1e-80
+
+
+def pin_gate_up(o):
+    """Gate rows come first: a constant large gate g makes out = g * u."""
+    N, K, M = 3, 64, 2
+    g = np.random.default_rng(13)
+    qw_up = g.integers(0, 2**32, size=(N, K // 8), dtype=np.uint32)
+    s_up = g.uniform(0.005, 0.02, size=(N, K // 32)).astype(np.float16)
+    qw_gate = np.full((N, K // 8), 0xFFFFFFFF, dtype=np.uint32)   # codes 15 -> w = 8 s
+    s_gate = np.full((N, K // 32), 1.0, dtype=np.float16)
+    x = np.ones((M, K), dtype=np.float16)
+    x[1] = 2.0
+    qw = np.concatenate([qw_gate, qw_up])
+    s = np.concatenate([s_gate, s_up])
+    out = o.gate_up_silu(qw, s, x)
+    Wup = dense_weights(qw_up, s_up)
+    for m in range(M):
+        gate = 8.0 * K * float(x[m, 0])             # 512 or 1024: SiLU(g) == g in double
+        u = Wup @ x[m].astype(np.float64)
+        assert np.allclose(out[m], gate * u, rtol=1e-13, atol=0), f"gate/up order m={m}"
+    # mirrored gate (q -> 14 - q turns g into -g): out(g) - out(-g) = g * u
+    qg = g.integers(0, 15, size=(N, K), dtype=np.uint8)
+    qw_g = np.array([[sum(int(qg[n, 8 * w + j]) << (4 * j) for j in range(8))
+                      for w in range(K // 8)] for n in range(N)], dtype=np.uint32)
+    qw_gm = np.array([[sum((14 - int(qg[n, 8 * w + j])) << (4 * j) for j in range(8))
+                       for w in range(K // 8)] for n in range(N)], dtype=np.uint32)
+    s_g = g.uniform(0.005, 0.02, size=(N, K // 32)).astype(np.float16)
+    xr = g.standard_normal((1, K)).astype(np.float16) * np.float16(8)
+    a = o.gate_up_silu(np.concatenate([qw_g, qw_up]), np.concatenate([s_g, s_up]), xr)[0]
+    b = o.gate_up_silu(np.concatenate([qw_gm, qw_up]), np.concatenate([s_g, s_up]), xr)[0]
+    gv = dense_weights(qw_g, s_g) @ xr[0].astype(np.float64)
+    uv = Wup @ xr[0].astype(np.float64)
+    assert np.allclose(a - b, gv * uv, rtol=1e-12, atol=1e-12), "SiLU odd-part identity"
+
+
+def pin_argmax(o):
+    assert o.argmax([1.0, 3.0, 3.0, 2.0]) == 1, "ties go to the lowest index"
+    assert o.argmax([5.0, 5.0]) == 0
+    assert o.argmax([float("nan"), -1.0, float("nan")]) == 1, "NaN is -inf"
+    assert o.argmax([float("nan"), float("nan")]) == 0, "all NaN -> 0"
+    assert o.argmax([-float("inf"), -float("inf"), -3.0]) == 2
+    assert o.argmax([0.0, -0.0, 1e-300]) == 2
+
+
+def pin_lmhead_duplicate_rows(o):
+    """An exact duplicate of the top row at a lower index takes the argmax."""
+    qw, s, x = small_problem(14, 40, 128, M=2)
+    logits, am = o.lmhead_argmax(qw, s, x)
+    for m in range(2):
+        top = int(np.argmax(logits[m]))
+        assert am[m] == top
+        qw2, s2 = qw.copy(), s.copy()
+        dup = 3 if top != 3 else 5
+        lo = min(dup, top)
+        qw2[dup], s2[dup] = qw[top], s[top]
+        _, am2 = o.lmhead_argmax(qw2, s2, x[m:m + 1])
+        assert am2[0] == lo, f"duplicate top row: want {lo}, got {am2[0]}"
+
+
+def pin_golden(o):
+    for c in parse_golden():
+        if c["kind"] == "gemv":
+            y = o.gemv(c["qw"], c["scales"], c["x"])
+            assert np.array_equal(y, c["y"]), f"golden {c['name']}: {y} vs {c['y']}"
+        elif c["kind"] == "gate_up":
+            y = o.gate_up_silu(c["qw"], c["scales"], c["x"])
+            assert np.allclose(y, c["y"], rtol=1e-14, atol=0), f"golden {c['name']}"
+        elif c["kind"] == "lm_head":
+            logits, am = o.lmhead_argmax(c["qw"], c["scales"], c["x"])
+            assert np.array_equal(logits, c["y"]), f"golden {c['name']} logits"
+            assert np.array_equal(am, c["argmax"]), f"golden {c['name']} argmax"
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

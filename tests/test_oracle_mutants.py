@@ -1,0 +1,56 @@
+"""Mutation gate for the oracle's pins (CPU only).
+
+Each mutant is a copy of the oracle's C source with one plausible mistake
+planted in it (the kind of defect that gives fluent wrong numbers instead of a
+crash).  The copy is compiled into a temporary directory and the pins are run
+against it: at least one pin must fail, or the pins would not have caught that
+mistake in the real oracle either.
+"""
+import os
+
+import pytest
+
+import oracle as oracle_pkg
+import oracle_pins as P
+
+# (name, text in the oracle source, replacement)
+MUTANTS = [
+    ("nibble_order_reversed", "(word >> (4 * (k % 8)))", "(word >> (4 * (7 - k % 8)))"),
+    ("scale_group_off_by_one", "scales[n * (K / ZTO_GROUP) + k / ZTO_GROUP]",
+     "scales[n * (K / ZTO_GROUP) + (k / ZTO_GROUP + 1) % (K / ZTO_GROUP)]"),
+    ("zero_point_8", "#define ZTO_ZERO 7", "#define ZTO_ZERO 8"),
+    ("gate_up_swapped",
+     "double g = zto_row_dot(qw, scales, x, K, m, n);",
+     "double g = zto_row_dot(qw, scales, x, K, m, n + N);"),
+    ("argmax_highest_index_on_tie", "if (c > best_v) {", "if (c >= best_v) {"),
+    ("dropped_k_tail", "for (int64_t k = 0; k < K; ++k)\n        acc +=",
+     "for (int64_t k = 0; k < K - 1; ++k)\n        acc +="),
+    ("half_exponent_bias", "expo - 25", "expo - 24"),
+    ("half_subnormal_scale", "ldexp((double)frac, -24)", "ldexp((double)frac, -25)"),
+    ("silu_sign", "return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
+    ("argmax_leading_nan_wins", "double best_v = isnan(v[0]) ? -INFINITY : v[0];",
+     "double best_v = v[0];"),
+    ("pack_high_nibble_first", "word |= (uint32_t)c << (4 * j);",
+     "word |= (uint32_t)c << (4 * (7 - j));"),
+    ("x_row_stride", "zto_half_to_double(x[m * K + k])", "zto_half_to_double(x[k])"),
+    ("sampled_rows_ignored", "int64_t n = rows ? rows[i] : i;\n        for (int64_t m = 0; m < M; ++m)\n            y[",
+     "int64_t n = i;\n        for (int64_t m = 0; m < M; ++m)\n            y["),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    with open(oracle_pkg.SOURCE) as fh:
+        src = fh.read()
+    assert src.count(old) == 1, f"mutation site for {name} must occur exactly once"
+    mutated = tmp_path / f"mutant_{name}.c"
+    mutated.write_text(src.replace(old, new))
+    lib = oracle_pkg.compile_oracle(str(mutated), str(tmp_path / f"lib_{name}.so"))
+    mutant = oracle_pkg.Oracle(lib)
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"
