@@ -1,0 +1,135 @@
+/*
+ * zt_q4.h -- C ABI of the q4f16 dequantizing GEMV library for NVIDIA B200
+ * (sm_100a): the int4 group-quantized matrix-vector products that dominate
+ * single-token LLM decode.
+ *
+ * Source of the operations: the Zero-TVM forum write-up ("Zero-TVM：手写 WGSL
+ * 着色器在浏览器中运行 Phi-3-mini，挑战编译器霸权"), section "完整的推理流水线"
+ * (int4 反量化矩阵乘法 -- the int4 dequantizing matrix product, with an f32-output
+ * variant for the LM head; greedy argmax sampling) and section "内核融合"
+ * (fused_ffn: gate, up and SiLU in one pass).  Its performance section names the
+ * weights "Phi-3-mini-q4f16_1".  The pages give no bit layout; this library
+ * fixes the format below and every entry point uses it.
+ *
+ * FORMAT ("q4f16", group 32)
+ *   W is n_rows x K (output features x input features), row-major.
+ *   qw      uint32 [n_rows][K/8].  Element (n,k) is the 4-bit code in bits
+ *           4*(k%8) .. 4*(k%8)+3 of qw[n][k/8] (low nibble first), 0..15.
+ *   scales  IEEE binary16 bit patterns [n_rows][K/32]: one scale per 32 k.
+ *   dequant w[n][k] = (code - 7) * scales[n][k/32]   (zero point 7).
+ *   x       IEEE binary16 [M][K], M = number of tokens (1..16).
+ *   Products are exact and accumulate in fp32; fp16 outputs are rounded once,
+ *   to nearest even, at the store.
+ *
+ * CONVENTIONS (all compute entry points)
+ *   - Pointers named qw, scales, x, y, logits, argmax, workspace are DEVICE
+ *     pointers owned by the caller; the library never allocates, frees or
+ *     keeps them after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is launched asynchronously on it; no entry point
+ *     synchronizes.  Errors inside a kernel surface at the caller's next
+ *     synchronization, as for any CUDA launch.
+ *   - Every argument is checked on the host BEFORE anything is launched; a
+ *     call that returns a negative status launched nothing and wrote nothing.
+ *   - Shapes: 1 <= M <= 16, N >= 1, K >= 32, K % 32 == 0, and the products
+ *     n_rows*K and M*K fit in int64 (n_rows = N, or 2N for gate/up).
+ *   - Alignment: qw and x 16 bytes; scales and y 2 bytes; logits and argmax
+ *     4 bytes; workspace 16 bytes.
+ *   - Inputs and outputs must not overlap.
+ *   - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef ZT_Q4_H
+#define ZT_Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZT_API __attribute__((visibility("default")))
+#else
+#define ZT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define ZT_OK                    0
+#define ZT_ERR_INVALID_ARG      -1  /* null pointer, M/N/K out of range, K % 32 */
+#define ZT_ERR_MISALIGNED       -2  /* a pointer violates its alignment rule */
+#define ZT_ERR_WORKSPACE        -3  /* workspace smaller than the query says */
+#define ZT_ERR_LAUNCH           -4  /* the CUDA launch failed (error not cleared) */
+#define ZT_ERR_UNSUPPORTED      -5  /* shape valid but beyond this build's limits */
+#define ZT_ERR_DEVICE           -6  /* no usable sm_100 device / attribute query failed */
+
+/*
+ * y[m][n] = sum_k (q[n][k] - 7) * s[n][k/32] * x[m][k]        (fp16 out)
+ *
+ * The plain projection (Zero-TVM write-up, "完整的推理流水线": the baseline,
+ * subgroup-reduce and rows x4 / rows x8 variants of the int4 dequantizing
+ * matrix product -- one kernel here, with warp-shuffle K reduction and
+ * row tiling chosen from the shape).
+ *   qw [N][K/8], scales [N][K/32], x [M][K], y [M][N] (fp16 bit patterns).
+ * Returns ZT_OK or a negative status.
+ */
+ZT_API int zt_q4_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+               uint16_t *y, int M, int N, int K, void *stream);
+
+/*
+ * Fused FFN input projection (Zero-TVM write-up, "内核融合": fused_ffn.wgsl,
+ * gate, up and SiLU in one pass):
+ *   g = gate row n . x_m,  u = up row n . x_m   (both fp32, never rounded)
+ *   y[m][n] = fp16( SiLU(g) * u ),  SiLU(g) = g / (1 + exp(-g)).
+ *   qw [2N][K/8] and scales [2N][K/32]: rows 0..N-1 are gate, N..2N-1 up.
+ *   x [M][K], y [M][N].
+ */
+ZT_API int zt_q4_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                       uint16_t *y, int M, int N, int K, void *stream);
+
+/*
+ * Bytes of device workspace zt_q4_lmhead_argmax needs for these shapes
+ * (per-CTA partial maxima; 0 if the shapes are invalid).  The value depends
+ * only on (M, N, K), never on the device.
+ */
+ZT_API size_t zt_q4_lmhead_workspace_bytes(int M, int N, int K);
+
+/*
+ * LM head with f32 logits and greedy argmax (Zero-TVM write-up,
+ * "完整的推理流水线": the f32-output dequantizing matrix product "for sampling
+ * stability", and greedy decoding as an argmax dispatch):
+ *   logits[m][n] = sum_k (q[n][k] - 7) * s[n][k/32] * x[m][k]   (f32, not rounded to fp16)
+ *   argmax[m]    = the lowest n among the maxima of logits[m][*]; NaN counts as
+ *                  -infinity (a row of NaN gives 0).
+ *   qw [N][K/8], scales [N][K/32], x [M][K], logits [M][N] f32, argmax [M] int32.
+ *   workspace: device scratch of at least zt_q4_lmhead_workspace_bytes(M,N,K)
+ *   bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *   matter.  Two launches on `stream` (logits + per-CTA maxima, then the
+ *   final reduction); no device-side waits, no float atomics: the result is
+ *   deterministic.
+ */
+ZT_API int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                        float *logits, int32_t *argmax, void *workspace, size_t ws_bytes,
+                        int M, int N, int K, void *stream);
+
+/*
+ * Host-side layout helpers (HOST pointers, synchronous, no CUDA calls).
+ * pack:   q uint8 [N][K] codes 0..15  ->  qw uint32 [N][K/8], low nibble first.
+ *         A code above 15 is ZT_ERR_INVALID_ARG (qw is then unspecified).
+ * unpack: qw [N][K/8] -> q [N][K].
+ * K % 8 == 0 and K >= 8 for both.
+ */
+ZT_API int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw);
+ZT_API int zt_q4_unpack_host(const uint32_t *qw, int N, int K, uint8_t *q);
+
+/* Static English text for a status code (never NULL). */
+ZT_API const char *zt_q4_strerror(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+ZT_API int zt_q4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZT_Q4_H */

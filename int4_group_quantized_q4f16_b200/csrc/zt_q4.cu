@@ -1,0 +1,240 @@
+// zt_q4.cu -- the C ABI of the q4f16 dequantizing GEMV library (see
+// include/zt_q4.h for the contract of every entry point).
+//
+// Host side only: argument checks, launch-shape selection and launches.  Every
+// check runs before the first CUDA call, so a rejected call launches nothing.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <mutex>
+#include <unordered_map>
+
+#include "q4_gemv.cuh"
+#include "zt_q4.h"
+
+namespace {
+
+using namespace zt;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_shapes(int M, int N, int K, int row_mult)
+{
+    if (M < 1 || M > 16 || N < 1 || K < kGroup || K % kGroup) return ZT_ERR_INVALID_ARG;
+    if ((int64_t)N * row_mult > INT_MAX) return ZT_ERR_INVALID_ARG;
+    return ZT_OK;
+}
+
+// Launch shape for a given K: WK warps split K (one 32-group chunk each), WR
+// warps split rows, at most 8 warps per CTA.
+void pick_warps(int G, int &wk, int &wr)
+{
+    wk = std::min(kMaxWarps, (G + 31) / 32);
+    wr = std::max(1, kMaxWarps / wk);
+}
+
+int smallest_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
+
+// rows per warp for each padded batch size (R * MT <= 32)
+int rows_per_warp(int mt) { return mt <= 4 ? 4 : 2; }
+
+struct OccKey {
+    const void *fn;
+    int dev, threads;
+    size_t smem;
+    bool operator==(const OccKey &o) const
+    {
+        return fn == o.fn && dev == o.dev && threads == o.threads && smem == o.smem;
+    }
+};
+struct OccHash {
+    size_t operator()(const OccKey &k) const
+    {
+        return std::hash<const void *>()(k.fn) ^ (size_t)k.dev * 131 ^ (size_t)k.threads * 7919 ^
+               k.smem * 104729;
+    }
+};
+
+std::mutex g_mu;
+std::unordered_map<OccKey, int, OccHash> g_occ;   // resident CTAs per SM, or -1 if unusable
+std::unordered_map<int, int> g_sms;               // device -> SM count
+
+// resident CTAs per SM for (kernel, block, smem) on the current device,
+// opting the kernel in to that much dynamic shared memory on first use
+int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it_s = g_sms.find(dev);
+    if (it_s == g_sms.end()) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            return -1;
+        it_s = g_sms.emplace(dev, n).first;
+    }
+    sms = it_s->second;
+    OccKey key{fn, dev, threads, smem};
+    auto it = g_occ.find(key);
+    if (it != g_occ.end()) return it->second;
+    int occ = -1;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) == cudaSuccess && nb > 0)
+            occ = nb;
+    }
+    g_occ.emplace(key, occ);
+    return occ;
+}
+
+template <int R, int MT, int EPI>
+int launch_one(Q4Args a, cudaStream_t st, int *grid_out)
+{
+    constexpr int V = R * MT;
+    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;
+    const int threads = a.wk * a.wr * 32;
+    const size_t smem = q4_smem_bytes(a.M, a.G, a.wk, a.wr, V);
+    if (smem > 227 * 1024) return ZT_ERR_UNSUPPORTED;
+    const void *fn = reinterpret_cast<const void *>(&q4_gemv_kernel<R, MT, EPI>);
+    int sms = 0;
+    const int occ = resident_ctas(fn, threads, smem, sms);
+    if (occ < 1) return ZT_ERR_DEVICE;
+    a.n_tiles = (a.N + a.wr * ROUT - 1) / (a.wr * ROUT);
+    const int grid = std::max(1, std::min({a.n_tiles, sms * occ, kMaxCtas}));
+    if (grid_out) *grid_out = grid;
+    q4_gemv_kernel<R, MT, EPI><<<grid, threads, smem, st>>>(a);
+    return cudaPeekAtLastError() == cudaSuccess ? ZT_OK : ZT_ERR_LAUNCH;
+}
+
+template <int EPI>
+int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, void *out, float *ws_val,
+              int *ws_idx, int M, int N, int K, void *stream, int *grid_out)
+{
+    Q4Args a;
+    a.qw = reinterpret_cast<const uint4 *>(qw);
+    a.scales = reinterpret_cast<const __half *>(scales);
+    a.x = reinterpret_cast<const __half *>(x);
+    a.out = out;
+    a.ws_val = ws_val;
+    a.ws_idx = ws_idx;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.G = K / kGroup;
+    pick_warps(a.G, a.wk, a.wr);
+    a.n_tiles = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int mt = smallest_mt(M);
+    const int r = rows_per_warp(mt);
+    (void)r;
+    switch (mt) {
+    case 1: return launch_one<4, 1, EPI>(a, st, grid_out);
+    case 2: return launch_one<4, 2, EPI>(a, st, grid_out);
+    case 4: return launch_one<4, 4, EPI>(a, st, grid_out);
+    case 8: return launch_one<2, 8, EPI>(a, st, grid_out);
+    default: return launch_one<2, 16, EPI>(a, st, grid_out);
+    }
+}
+
+size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + sizeof(int)); }
+
+}  // namespace
+
+extern "C" {
+
+int zt_q4_version(void) { return (1 << 16) | 0; }
+
+const char *zt_q4_strerror(int status)
+{
+    switch (status) {
+    case ZT_OK: return "success";
+    case ZT_ERR_INVALID_ARG: return "invalid argument (null pointer, or M/N/K out of range, or K % 32 != 0)";
+    case ZT_ERR_MISALIGNED: return "pointer misaligned (qw and x need 16 bytes, workspace 16, logits/argmax 4, scales/y 2)";
+    case ZT_ERR_WORKSPACE: return "workspace smaller than zt_q4_lmhead_workspace_bytes()";
+    case ZT_ERR_LAUNCH: return "CUDA kernel launch failed";
+    case ZT_ERR_UNSUPPORTED: return "shape is valid but exceeds this build's limits (activations must fit in shared memory: M*K*4.125 bytes)";
+    case ZT_ERR_DEVICE: return "no usable CUDA device, or a device attribute query failed";
+    default: return "unknown status";
+    }
+}
+
+int zt_q4_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M, int N,
+               int K, void *stream)
+{
+    if (!qw || !scales || !x || !y) return ZT_ERR_INVALID_ARG;
+    int rc = check_shapes(M, N, K, 1);
+    if (rc) return rc;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(y, 2)) return ZT_ERR_MISALIGNED;
+    return launch_q4<kEpiF16>(qw, scales, x, y, nullptr, nullptr, M, N, K, stream, nullptr);
+}
+
+int zt_q4_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M,
+                       int N, int K, void *stream)
+{
+    if (!qw || !scales || !x || !y) return ZT_ERR_INVALID_ARG;
+    int rc = check_shapes(M, N, K, 2);
+    if (rc) return rc;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(y, 2)) return ZT_ERR_MISALIGNED;
+    return launch_q4<kEpiGateUp>(qw, scales, x, y, nullptr, nullptr, M, N, K, stream, nullptr);
+}
+
+size_t zt_q4_lmhead_workspace_bytes(int M, int N, int K)
+{
+    if (check_shapes(M, N, K, 1) != ZT_OK) return 0;
+    return lmhead_ws_bytes(M);
+}
+
+int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, float *logits,
+                        int32_t *argmax, void *workspace, size_t ws_bytes, int M, int N, int K, void *stream)
+{
+    if (!qw || !scales || !x || !logits || !argmax || !workspace) return ZT_ERR_INVALID_ARG;
+    int rc = check_shapes(M, N, K, 1);
+    if (rc) return rc;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(logits, 4) ||
+        !aligned(argmax, 4) || !aligned(workspace, 16))
+        return ZT_ERR_MISALIGNED;
+    if (ws_bytes < lmhead_ws_bytes(M)) return ZT_ERR_WORKSPACE;
+    float *ws_val = reinterpret_cast<float *>(workspace);
+    int *ws_idx = reinterpret_cast<int *>(ws_val + (size_t)kMaxCtas * M);
+    int grid = 0;
+    rc = launch_q4<kEpiLogits>(qw, scales, x, logits, ws_val, ws_idx, M, N, K, stream, &grid);
+    if (rc) return rc;
+    q4_argmax_reduce_kernel<<<M, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ws_val, ws_idx, grid, M,
+                                                                                   argmax);
+    return cudaPeekAtLastError() == cudaSuccess ? ZT_OK : ZT_ERR_LAUNCH;
+}
+
+int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)
+{
+    if (!q || !qw || N < 1 || K < 8 || K % 8) return ZT_ERR_INVALID_ARG;
+    const int64_t W = K / 8;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t *src = q + n * (int64_t)K;
+        for (int64_t w = 0; w < W; ++w) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t c = src[8 * w + j];
+                if (c > 15u) return ZT_ERR_INVALID_ARG;
+                word |= c << (4 * j);
+            }
+            qw[n * W + w] = word;
+        }
+    }
+    return ZT_OK;
+}
+
+int zt_q4_unpack_host(const uint32_t *qw, int N, int K, uint8_t *q)
+{
+    if (!q || !qw || N < 1 || K < 8 || K % 8) return ZT_ERR_INVALID_ARG;
+    const int64_t W = K / 8;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t w = 0; w < W; ++w) {
+            const uint32_t word = qw[n * W + w];
+            for (int j = 0; j < 8; ++j) q[n * (int64_t)K + 8 * w + j] = (uint8_t)((word >> (4 * j)) & 0xFu);
+        }
+    return ZT_OK;
+}
+
+}  // extern "C"

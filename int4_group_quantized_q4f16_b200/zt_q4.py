@@ -1,0 +1,165 @@
+"""Thin ctypes binding of ``libzt_q4.so`` (declared in ``include/zt_q4.h``).
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every step of the computation runs in the library's kernels.  Importing
+this module loads the library and fails loudly when it is missing -- there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libzt_q4.so")
+
+ZT_OK = 0
+ZT_ERR_INVALID_ARG = -1
+ZT_ERR_MISALIGNED = -2
+ZT_ERR_WORKSPACE = -3
+ZT_ERR_LAUNCH = -4
+ZT_ERR_UNSUPPORTED = -5
+ZT_ERR_DEVICE = -6
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+class ZtError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: status {status}: {strerror(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m int4_group_quantized_q4f16_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.zt_q4_gemv.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P]
+    lib.zt_q4_gate_up_silu.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P]
+    lib.zt_q4_lmhead_workspace_bytes.argtypes = [_I, _I, _I]
+    lib.zt_q4_lmhead_workspace_bytes.restype = ctypes.c_size_t
+    lib.zt_q4_lmhead_argmax.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _P]
+    lib.zt_q4_pack_host.argtypes = [_P, _I, _I, _P]
+    lib.zt_q4_unpack_host.argtypes = [_P, _I, _I, _P]
+    lib.zt_q4_strerror.argtypes = [_I]
+    lib.zt_q4_strerror.restype = ctypes.c_char_p
+    lib.zt_q4_version.argtypes = []
+    for f in (lib.zt_q4_gemv, lib.zt_q4_gate_up_silu, lib.zt_q4_lmhead_argmax,
+              lib.zt_q4_pack_host, lib.zt_q4_unpack_host, lib.zt_q4_version):
+        f.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def strerror(status: int) -> str:
+    return lib.zt_q4_strerror(int(status)).decode()
+
+
+def version() -> Tuple[int, int]:
+    v = lib.zt_q4_version()
+    return v >> 16, v & 0xFFFF
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != ZT_OK:
+        raise ZtError(rc, what)
+
+
+# ------------------------------------------------------------ host layout --
+def pack_host(q: np.ndarray) -> np.ndarray:
+    """codes uint8 [N][K] (0..15) -> packed uint32 [N][K/8], low nibble first."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    N, K = q.shape
+    qw = np.empty((N, K // 8), dtype=np.uint32)
+    _check(lib.zt_q4_pack_host(q.ctypes.data, N, K, qw.ctypes.data), "zt_q4_pack_host")
+    return qw
+
+
+def unpack_host(qw: np.ndarray, K: int) -> np.ndarray:
+    qw = np.ascontiguousarray(qw, dtype=np.uint32)
+    N = qw.shape[0]
+    q = np.empty((N, K), dtype=np.uint8)
+    _check(lib.zt_q4_unpack_host(qw.ctypes.data, N, K, q.ctypes.data), "zt_q4_unpack_host")
+    return q
+
+
+# ---------------------------------------------------------- device calls --
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dims(qw, scales, x, rows_mult: int):
+    torch = _torch()
+    for t, name in ((qw, "qw"), (scales, "scales"), (x, "x")):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if qw.dtype not in (torch.int32, torch.uint32):
+        raise TypeError("qw must hold 32-bit words (int32 or uint32)")
+    if scales.dtype != torch.float16 or x.dtype != torch.float16:
+        raise TypeError("scales and x must be float16")
+    x2 = x if x.dim() == 2 else x.view(1, -1)
+    M, K = x2.shape
+    n_rows = qw.shape[0]
+    if qw.dim() != 2 or qw.shape[1] * 8 != K or scales.shape != (n_rows, K // 32):
+        raise ValueError(f"shape mismatch: qw {tuple(qw.shape)}, scales {tuple(scales.shape)}, x {tuple(x.shape)}")
+    if n_rows % rows_mult:
+        raise ValueError("gate/up weights need an even number of rows")
+    return M, n_rows // rows_mult, K
+
+
+def gemv(qw, scales, x, y=None, stream=None):
+    """y[M][N] fp16 = dequant(qw, scales) @ x^T (torch CUDA tensors)."""
+    torch = _torch()
+    M, N, K = _dims(qw, scales, x, 1)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check(lib.zt_q4_gemv(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(),
+                          M, N, K, _stream_handle(stream)), "zt_q4_gemv")
+    return y
+
+
+def gate_up_silu(qw, scales, x, y=None, stream=None):
+    """y[M][N] fp16 = SiLU(gate . x) * (up . x); qw has 2N rows, gate first."""
+    torch = _torch()
+    M, N, K = _dims(qw, scales, x, 2)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check(lib.zt_q4_gate_up_silu(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(),
+                                  M, N, K, _stream_handle(stream)), "zt_q4_gate_up_silu")
+    return y
+
+
+def lmhead_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.zt_q4_lmhead_workspace_bytes(M, N, K))
+
+
+def lmhead_argmax(qw, scales, x, logits=None, argmax=None, workspace=None, stream=None):
+    """(logits f32 [M][N], argmax int32 [M]); workspace is a uint8 CUDA tensor."""
+    torch = _torch()
+    M, N, K = _dims(qw, scales, x, 1)
+    if logits is None:
+        logits = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if argmax is None:
+        argmax = torch.empty((M,), dtype=torch.int32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((lmhead_workspace_bytes(M, N, K),), dtype=torch.uint8, device=x.device)
+    _check(lib.zt_q4_lmhead_argmax(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), logits.data_ptr(),
+                                   argmax.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                   M, N, K, _stream_handle(stream)), "zt_q4_lmhead_argmax")
+    return logits, argmax

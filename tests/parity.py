@@ -1,0 +1,83 @@
+"""Helpers for the GPU parity tests: move seeded inputs to the device, call the
+library through its binding, and compare with the oracle.
+
+Tolerances (the stated bar): fp16 outputs relative L2 error <= 1e-3, f32
+logits <= 1e-5, argmax exact unless the oracle's top-2 logits are within 1e-3.
+On top of that, every fp16 output must lie within one fp16 ulp of the
+correctly rounded oracle value: the kernels form exact products and
+accumulate in fp32, so the only visible difference is on which side of a
+rounding boundary an fp32 sum falls.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+F16_REL_L2 = 1e-3
+F32_REL_L2 = 1e-5
+ARGMAX_GAP = 1e-3
+
+
+def dev(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint32:
+        a = a.view(np.int32)
+    return torch.from_numpy(a).cuda()
+
+
+def host(t) -> np.ndarray:
+    import torch
+    t = t.detach().cpu()
+    if t.dtype == torch.int32:
+        return t.numpy()
+    return t.numpy()
+
+
+def rel_l2(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(got - ref)
+    return float(num / den) if den > 0 else float(num)
+
+
+def assert_f16_matches(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    got = np.asarray(got, dtype=np.float16)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite fp16 output"
+    r = rel_l2(got, ref)
+    assert r <= F16_REL_L2, f"{what}: rel L2 {r:.3e} > {F16_REL_L2}"
+    ref16 = ref.astype(np.float16)
+    ulp = np.spacing(np.abs(ref16)).astype(np.float64)
+    err = np.abs(got.astype(np.float64) - ref16.astype(np.float64))
+    bad = err > ulp
+    assert not bad.any(), (f"{what}: {int(bad.sum())} outputs more than 1 fp16 ulp from the "
+                           f"rounded oracle, e.g. index {np.argwhere(bad)[0].tolist()}")
+
+
+def assert_f32_matches(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    r = rel_l2(got, ref)
+    assert r <= F32_REL_L2, f"{what}: rel L2 {r:.3e} > {F32_REL_L2}"
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    assert np.max(np.abs(got - ref)) <= 1e-4 * rms + 1e-30, f"{what}: element error too large"
+
+
+def check_argmax(am_gpu: np.ndarray, logits_ref: np.ndarray, exact_dups=None):
+    """argmax exact, unless the oracle's top-2 are within ARGMAX_GAP: then the
+    GPU's index must be one of the near-maximal ones.  `exact_dups[m]` lists
+    rows known to be exact copies of the top row: then the lowest one must win."""
+    for m in range(logits_ref.shape[0]):
+        row = logits_ref[m]
+        best = int(np.argmax(row))              # numpy: first occurrence = lowest index
+        top = row[best]
+        near = np.flatnonzero(row >= top - ARGMAX_GAP)
+        if exact_dups is not None and exact_dups[m]:
+            assert int(am_gpu[m]) == best, f"row {m}: exact duplicate tie must give lowest index {best}"
+        elif len(near) == 1:
+            assert int(am_gpu[m]) == best, f"row {m}: argmax {am_gpu[m]} != {best}"
+        else:
+            assert int(am_gpu[m]) in set(near.tolist()), f"row {m}: {am_gpu[m]} not near-max"

@@ -1,0 +1,116 @@
+"""The C-ABI library on the host: it loads, exports every symbol the header
+declares, rejects bad arguments before touching the GPU, and its host layout
+helpers agree with the oracle.  No compute call runs here (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from int4_group_quantized_q4f16_b200 import build as zt_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zt_q4.h")
+
+
+@pytest.fixture(scope="module")
+def zt():
+    zt_build.build()
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    return zt_q4
+
+
+def declared_symbols(path):
+    text = open(path).read()
+    return sorted(set(re.findall(r"ZT_API\s+[\w\s\*]*?\b(zt_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    syms = declared_symbols(HEADER)
+    for want in ("zt_q4_gemv", "zt_q4_gate_up_silu", "zt_q4_lmhead_argmax",
+                 "zt_q4_lmhead_workspace_bytes", "zt_q4_pack_host", "zt_q4_unpack_host",
+                 "zt_q4_strerror", "zt_q4_version"):
+        assert want in syms
+
+
+def test_library_exports_every_declared_symbol(zt):
+    for path in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if path.endswith(".h"):
+            for sym in declared_symbols(os.path.join(ROOT, "include", path)):
+                assert hasattr(zt.lib, sym), f"{sym} declared in {path} but not exported"
+
+
+def test_strerror_and_version(zt):
+    for code in (0, -1, -2, -3, -4, -5, -6, 12345):
+        assert isinstance(zt.strerror(code), str) and zt.strerror(code)
+    assert zt.version()[0] == 1
+
+
+FAKE = 0x10000  # 64 KiB-aligned fake address: never dereferenced (checks fail first)
+
+
+@pytest.mark.parametrize("fn", ["zt_q4_gemv", "zt_q4_gate_up_silu"])
+def test_bad_arguments_rejected(zt, fn):
+    f = getattr(zt.lib, fn)
+    ok = (FAKE, FAKE, FAKE, FAKE)
+    # null pointers
+    for i in range(4):
+        ptrs = list(ok)
+        ptrs[i] = None
+        assert f(*ptrs, 1, 64, 64, None) == zt.ZT_ERR_INVALID_ARG
+    # shapes
+    for M, N, K in ((0, 64, 64), (17, 64, 64), (-1, 64, 64), (1, 0, 64), (1, 64, 0),
+                    (1, 64, 16), (1, 64, 48), (1, 64, 100), (1, -5, 64)):
+        assert f(*ok, M, N, K, None) == zt.ZT_ERR_INVALID_ARG, (M, N, K)
+    # misalignment: qw and x need 16 bytes, scales and y 2
+    assert f(FAKE + 8, FAKE, FAKE, FAKE, 1, 64, 64, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE + 1, FAKE, FAKE, 1, 64, 64, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE + 4, FAKE, 1, 64, 64, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, FAKE + 1, 1, 64, 64, None) == zt.ZT_ERR_MISALIGNED
+
+
+def test_gate_up_row_count_overflow(zt):
+    assert zt.lib.zt_q4_gate_up_silu(FAKE, FAKE, FAKE, FAKE, 1, 2**30 + 1, 64, None) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_lmhead_arguments(zt):
+    f = zt.lib.zt_q4_lmhead_argmax
+    ws = zt.lmhead_workspace_bytes(1, 1000, 256)
+    assert ws > 0
+    assert zt.lmhead_workspace_bytes(0, 1000, 256) == 0
+    assert zt.lmhead_workspace_bytes(1, 1000, 100) == 0
+    assert zt.lmhead_workspace_bytes(16, 1000, 256) >= ws
+    assert zt.lmhead_workspace_bytes(1, 10, 256) == zt.lmhead_workspace_bytes(1, 10**6, 8192)
+    args = [FAKE] * 6
+    for i in range(6):
+        a = list(args)
+        a[i] = None
+        assert f(*a, ws, 1, 1000, 256, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(*args, ws - 1, 1, 1000, 256, None) == zt.ZT_ERR_WORKSPACE
+    assert f(*args, 0, 1, 1000, 256, None) == zt.ZT_ERR_WORKSPACE
+    a = list(args)
+    a[3] = FAKE + 2          # logits need 4 bytes
+    assert f(*a, ws, 1, 1000, 256, None) == zt.ZT_ERR_MISALIGNED
+    a = list(args)
+    a[5] = FAKE + 8          # workspace needs 16
+    assert f(*a, ws, 1, 1000, 256, None) == zt.ZT_ERR_MISALIGNED
+    assert f(*args, ws, 17, 1000, 256, None) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_pack_unpack_host_matches_oracle(zt, oracle):
+    g = np.random.default_rng(21)
+    qw = g.integers(0, 2**32, size=(13, 40), dtype=np.uint32)
+    q = zt.unpack_host(qw, 320)
+    assert np.array_equal(q, oracle.unpack(qw, 320))
+    assert np.array_equal(zt.pack_host(q), qw)
+    assert np.array_equal(zt.pack_host(q), oracle.pack(q))
+
+
+def test_pack_host_rejects_codes_above_15(zt):
+    q = np.zeros((2, 16), dtype=np.uint8)
+    q[1, 5] = 16
+    with pytest.raises(zt.ZtError):
+        zt.pack_host(q)
+    rc = zt.lib.zt_q4_pack_host(None, 2, 16, None)
+    assert rc == zt.ZT_ERR_INVALID_ARG
