@@ -59,7 +59,7 @@ extern "C" {
 #define ZT_ERR_INVALID_ARG      -1  /* null pointer, M/N/K out of range, K % 32 */
 #define ZT_ERR_MISALIGNED       -2  /* a pointer violates its alignment rule */
 #define ZT_ERR_WORKSPACE        -3  /* workspace smaller than the query says */
-#define ZT_ERR_LAUNCH           -4  /* the CUDA launch failed (error not cleared) */
+#define ZT_ERR_LAUNCH           -4  /* the CUDA launch failed (see zt_q4_last_cuda_error) */
 #define ZT_ERR_UNSUPPORTED      -5  /* shape valid but beyond this build's limits */
 #define ZT_ERR_DEVICE           -6  /* no usable sm_100 device / attribute query failed */
 
@@ -124,6 +124,13 @@ ZT_API int zt_q4_unpack_host(const uint32_t *qw, int N, int K, uint8_t *q);
 
 /* Static English text for a status code (never NULL). */
 ZT_API const char *zt_q4_strerror(int status);
+
+/*
+ * Name of the last CUDA runtime error a library call met on the calling host
+ * thread (e.g. "cudaErrorInvalidResourceHandle"), or "" if none.  Diagnostics
+ * for ZT_ERR_LAUNCH / ZT_ERR_DEVICE; static storage, never NULL.
+ */
+ZT_API const char *zt_q4_last_cuda_error(void);
 
 /* Library ABI version, (major << 16) | minor. */
 ZT_API int zt_q4_version(void);

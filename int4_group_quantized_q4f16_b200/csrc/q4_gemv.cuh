@@ -7,18 +7,21 @@
 // One templated kernel covers all of them; the epilogue differs.
 //
 // Work decomposition (CUDA cores; the path is HBM-bound at M = 1):
-//   * A CTA is WK x WR warps.  The WK warps split K: warp kw, lane l owns the
-//     groups g = 32*kw + l, + 32*WK, ...  A group is exactly one 16-byte chunk
-//     of packed codes, so a warp reads 512 contiguous bytes per row: fully
-//     coalesced 128-bit loads straight from HBM.
-//   * Each warp computes R weight rows at once, so every activation value it
-//     fetches from shared memory is reused R times (the pages' rows x4 / x8
-//     tiling).
+//   * Persistent grid: one CTA of 16 warps per SM (or as many as fit), each
+//     CTA stages the activations once into shared memory.
+//   * A warp owns a tile of R weight rows over the whole of K and needs no
+//     block-wide synchronisation: lane l handles the groups g = l, l + 32, ...
+//     A group is exactly one 16-byte chunk of packed codes, so each load
+//     instruction of a warp reads 512 contiguous bytes of one row: fully
+//     coalesced 128-bit loads straight from HBM, U groups x R rows in flight
+//     per lane.
+//   * Every activation value a lane fetches from shared memory serves R rows
+//     (the pages' rows x4 / rows x8 tiling).
 //   * Lane partials are combined with a transposing warp-shuffle butterfly
-//     (the pages' subgroup reduction) and the WK warps through shared memory,
-//     in a fixed order: results are deterministic.
-//   * The grid is persistent (SM count x resident CTAs); CTAs stride over
-//     row tiles.
+//     (the pages' subgroup reduction) in a fixed order, so results are
+//     deterministic and identical rows give identical outputs.
+//   * Tiles are dealt to CTAs first, then to warps, so consecutive tiles land
+//     on different SMs.
 //
 // Arithmetic (exact products, no conversion instructions):
 //   For a binary32 bit pattern below 2^24 the value is exactly
@@ -44,8 +47,6 @@
 namespace zt {
 
 constexpr int kGroup = 32;                 // k values per scale
-constexpr int kMaxWarps = 8;               // per CTA
-constexpr int kThreadsMax = kMaxWarps * 32;
 constexpr int kMaxCtas = 4096;             // grid cap (sizes the LM-head workspace)
 
 enum EpiKind : int { kEpiF16 = 0, kEpiGateUp = 1, kEpiLogits = 2 };
@@ -58,8 +59,7 @@ struct Q4Args {
     float *ws_val;          // Logits: per-CTA maximum   [gridDim.x][M]
     int *ws_idx;            // Logits: per-CTA arg-max   [gridDim.x][M]
     int M, N, K, G;         // N = output features; G = K / 32
-    int wk, wr;             // warps along K, warps along rows (wk * wr <= 8)
-    int n_tiles;            // row tiles of wr * (outputs per warp) outputs
+    int n_tiles;            // warp tiles (of R weight rows = R or R/2 outputs)
 };
 
 // exponent (of 2) applied to x for the code at position j = k % 8 of its word
@@ -115,6 +115,19 @@ __device__ __forceinline__ void warp_transpose_reduce(float (&v)[V], int lane, i
     }
 }
 
+// Inverse of warp_transpose_reduce's lane -> value map: the value number a lane holds.
+template <int V>
+__device__ __forceinline__ int lane_vid(int lane)
+{
+    int vid = 0;
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+        const int half = V >> (s + 1);
+        if (half >= 1 && (lane & (16 >> s))) vid += half;
+    }
+    return vid;
+}
+
 // greater value wins; equal values -> lower index; NaN counts as -inf
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi)
 {
@@ -123,156 +136,185 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi)
     return v > bv || (v == bv && i < bi);
 }
 
+constexpr int kWarps = 16;                 // per CTA
+constexpr int kThreads = kWarps * 32;
+
 // Dynamic shared memory layout (bytes):
 //   xs   float [M][G][32]  pre-scaled activations, float4 slots XOR-swizzled by g&7
 //   xg   float [M][G]      7 * X_g * 2^-59
-//   red  float [wr][wk][V] per-warp partial sums
-//   bv   float [256], bi int [256]   (Logits: per-thread running maxima)
-__host__ __device__ inline size_t q4_smem_bytes(int M, int G, int wk, int wr, int V)
+//   bv   float [kThreads], bi int [kThreads]   (Logits: per-lane running maxima)
+__host__ __device__ inline size_t q4_smem_bytes(int M, int G)
 {
-    return (size_t)M * G * 32 * 4 + (size_t)M * G * 4 + (size_t)wr * wk * V * 4 +
-           (size_t)kThreadsMax * 8;
+    return (size_t)M * G * 32 * 4 + (size_t)M * G * 4 + (size_t)kThreads * 8;
 }
 
-template <int R, int MT, int EPI>
-__global__ void __launch_bounds__(kThreadsMax) q4_gemv_kernel(const Q4Args a)
+// Stage x once per CTA: xs = x * 2^(90 - 4p(k)) (exact), xg = 7 * X_g * 2^-59.
+// Each thread converts 8 consecutive k (one 16-byte load); the 4 threads of a
+// group add their partial sums with two shuffles (fixed order).
+__device__ __forceinline__ void stage_activations(const __half *__restrict__ x, float *xs, float *xg, int M,
+                                                  int K, int G)
+{
+    const int K8 = K >> 3;
+    for (int m = 0; m < M; ++m) {
+        for (int base = 0; base < K8; base += kThreads) {
+            const int kk = base + threadIdx.x;        // uniform trip count: shuffles see full warps
+            float part = 0.f;
+            if (kk < K8) {
+                const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)m * K + 8 * kk);
+                const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __half22float2(h[j]);
+                    v[2 * j] = f.x;
+                    v[2 * j + 1] = f.y;
+                }
+                part = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+                const int g = kk >> 2, c0 = (kk & 3) * 2;
+                float4 *dst = reinterpret_cast<float4 *>(xs + ((size_t)m * G + g) * 32);
+                dst[c0 ^ (g & 7)] = make_float4(v[0] * pow2f(xscale_exp(0)), v[1] * pow2f(xscale_exp(1)),
+                                                v[2] * pow2f(xscale_exp(2)), v[3] * pow2f(xscale_exp(3)));
+                dst[(c0 + 1) ^ (g & 7)] = make_float4(v[4] * pow2f(xscale_exp(4)), v[5] * pow2f(xscale_exp(5)),
+                                                      v[6] * pow2f(xscale_exp(6)), v[7] * pow2f(xscale_exp(7)));
+            }
+            part += __shfl_xor_sync(0xffffffffu, part, 1);
+            part += __shfl_xor_sync(0xffffffffu, part, 2);
+            if (kk < K8 && (kk & 3) == 0) xg[(size_t)m * G + (kk >> 2)] = part * (7.0f * pow2f(-59));
+        }
+    }
+}
+
+template <int R, int MT, int U, int EPI>
+__global__ void __launch_bounds__(kThreads, 1) q4_gemv_kernel(const Q4Args a)
 {
     constexpr int V = R * MT;                                // partial sums per lane
-    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;    // outputs per warp
+    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;    // outputs per warp tile
     static_assert(V <= 32 && (V & (V - 1)) == 0, "R*MT must be a power of two <= 32");
     static_assert(EPI != kEpiGateUp || (R % 2 == 0), "gate/up needs an even row count");
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int M = a.M, K = a.K, G = a.G, N = a.N, wk = a.wk, wr = a.wr;
+    const int M = a.M, G = a.G, N = a.N;
     float *xs = reinterpret_cast<float *>(smem_raw);
     float *xg = xs + (size_t)M * G * 32;
-    float *red = xg + (size_t)M * G;
-    float *bvs = red + wr * wk * V;
-    int *bis = reinterpret_cast<int *>(bvs + kThreadsMax);
+    float *bvs = xg + (size_t)M * G;
+    int *bis = reinterpret_cast<int *>(bvs + kThreads);
 
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
-    const int kw = warp % wk;
-    const int wri = warp / wk;
-    const int nthreads = blockDim.x;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
 
-    // ---- stage pre-scaled activations once per CTA ----
-    for (int idx = tid; idx < M * K; idx += nthreads) {
-        const int m = idx / K, k = idx - m * K;
-        const int g = k >> 5, c = (k & 31) >> 2, e = k & 3;
-        const float v = __half2float(a.x[idx]) * pow2f(xscale_exp(k & 7));
-        xs[(((size_t)m * G + g) * 8 + (c ^ (g & 7))) * 4 + e] = v;
-    }
-    for (int idx = tid; idx < M * G; idx += nthreads) {
-        const __half *xp = a.x + (size_t)idx * kGroup;   // (m, g) -> x[m][32g ...]
-        float s = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < kGroup; ++j) s += __half2float(xp[j]);
-        xg[idx] = s * (7.0f * pow2f(-59));
-    }
+    stage_activations(a.x, xs, xg, M, a.K, G);
     __syncthreads();
 
+    const int vid = lane_vid<V>(lane);
+    const bool rep = (lane & (32 / V - 1)) == 0;      // one lane per distinct value
+    const int my_r = vid / MT, my_m = vid - (vid / MT) * MT;
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
-    const int rows_per_tile = wr * ROUT;
-    const int n_out = wr * V / (EPI == kEpiGateUp ? 2 : 1);   // outputs per tile (incl. m)
 
-    for (int tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
-        const int obase = tile * rows_per_tile + wri * ROUT;   // first output row of this warp
-
-        // weight rows of this warp (clamped: rows past N are loaded but never stored)
-        int wrow[R];
+    for (int tile = blockIdx.x + gridDim.x * warp; tile < a.n_tiles; tile += gridDim.x * kWarps) {
+        const int obase = tile * ROUT;                    // first output row of the tile
+        const uint4 *rowp[R];
+        const __half *srow[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
+            int row;
             if (EPI == kEpiGateUp) {
                 const int o = min(obase + (r % ROUT), N - 1);
-                wrow[r] = (r < ROUT) ? o : N + o;
+                row = (r < ROUT) ? o : N + o;
             } else {
-                wrow[r] = min(obase + r, N - 1);
+                row = min(obase + r, N - 1);              // rows past N are loaded, never stored
             }
+            rowp[r] = a.qw + (size_t)row * G;
+            srow[r] = a.scales + (size_t)row * G;
         }
 
         float part[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) part[i] = 0.f;
 
-        for (int g = kw * 32 + lane; g < G; g += wk * 32) {
-            uint4 w[R];
-            float s[R];
+        for (int g0 = lane; g0 < G; g0 += 32 * U) {
+            uint4 w[U][R];
+            float s[U][R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) w[r] = ldg_stream(a.qw + (size_t)wrow[r] * G + g);
+            for (int u = 0; u < U; ++u) {
+                const int g = g0 + 32 * u;
 #pragma unroll
-            for (int r = 0; r < R; ++r) s[r] = __half2float(a.scales[(size_t)wrow[r] * G + g]);
+                for (int r = 0; r < R; ++r) w[u][r] = (g < G) ? ldg_stream(rowp[r] + g) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m < M) {
-                    const float4 *xv4 = reinterpret_cast<const float4 *>(xs + ((size_t)m * G + g) * 32);
-                    const int sw = g & 7;
-                    float4 xv[8];
+            for (int u = 0; u < U; ++u) {
+                const int g = g0 + 32 * u;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) xv[c] = xv4[c ^ sw];
-                    const float xgm = xg[m * G + g];
+                for (int r = 0; r < R; ++r) s[u][r] = (g < G) ? __half2float(srow[r][g]) : 0.f;
+            }
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        float2 acc = make_float2(0.f, 0.f);
-                        acc = word_dot(w[r].x, xv[0], xv[1], acc);
-                        acc = word_dot(w[r].y, xv[2], xv[3], acc);
-                        acc = word_dot(w[r].z, xv[4], xv[5], acc);
-                        acc = word_dot(w[r].w, xv[6], xv[7], acc);
-                        part[r * MT + m] = fmaf(s[r], (acc.x + acc.y) - xgm, part[r * MT + m]);
+            for (int u = 0; u < U; ++u) {
+                const int g = g0 + 32 * u;
+                if (g < G) {
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        if (m < M) {
+                            const float4 *xv4 = reinterpret_cast<const float4 *>(xs + ((size_t)m * G + g) * 32);
+                            const int sw = g & 7;
+                            float4 xv[8];
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) xv[c] = xv4[c ^ sw];
+                            const float xgm = xg[m * G + g];
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                float2 acc = make_float2(0.f, 0.f);
+                                acc = word_dot(w[u][r].x, xv[0], xv[1], acc);
+                                acc = word_dot(w[u][r].y, xv[2], xv[3], acc);
+                                acc = word_dot(w[u][r].z, xv[4], xv[5], acc);
+                                acc = word_dot(w[u][r].w, xv[6], xv[7], acc);
+                                part[r * MT + m] = fmaf(s[u][r], (acc.x + acc.y) - xgm, part[r * MT + m]);
+                            }
+                        }
                     }
                 }
             }
         }
 
-        int vid;
-        warp_transpose_reduce<V>(part, lane, vid);
-        if ((lane & (32 / V - 1)) == 0) red[(wri * wk + kw) * V + vid] = part[0];
-        __syncthreads();
-
-        if (tid < n_out) {
-            // output (wri_o, r, m) of this tile
-            constexpr int VO = ROUT * MT;
-            const int wri_o = tid / VO, vo = tid - wri_o * VO;
-            const int r = vo / MT, m = vo - r * MT;
-            const int n = tile * rows_per_tile + wri_o * ROUT + r;
-            const float *rp = red + wri_o * wk * V;
-            float t0 = 0.f, t1 = 0.f;
-            for (int k2 = 0; k2 < wk; ++k2) {
-                t0 += rp[k2 * V + r * MT + m];
-                if (EPI == kEpiGateUp) t1 += rp[k2 * V + (r + ROUT) * MT + m];
+        int v_unused;
+        warp_transpose_reduce<V>(part, lane, v_unused);
+        const float y = part[0] * pow2f(59);              // this lane's value: (row my_r, m my_m)
+        if (EPI == kEpiGateUp) {
+            const float u = __shfl_xor_sync(0xffffffffu, y, 16);   // the up row's value
+            const int n = obase + my_r;
+            if (rep && vid < V / 2 && n < N && my_m < M) {
+                const float silu = y / (1.0f + expf(-y));
+                reinterpret_cast<__half *>(a.out)[(size_t)my_m * N + n] = __float2half_rn(silu * u);
             }
-            if (n < N && m < M) {
-                const float y = t0 * pow2f(59);
+        } else {
+            const int n = obase + my_r;
+            if (rep && n < N && my_m < M) {
                 if (EPI == kEpiF16) {
-                    reinterpret_cast<__half *>(a.out)[(size_t)m * N + n] = __float2half_rn(y);
-                } else if (EPI == kEpiGateUp) {
-                    const float u = t1 * pow2f(59);
-                    const float silu = y / (1.0f + expf(-y));
-                    reinterpret_cast<__half *>(a.out)[(size_t)m * N + n] = __float2half_rn(silu * u);
+                    reinterpret_cast<__half *>(a.out)[(size_t)my_m * N + n] = __float2half_rn(y);
                 } else {
-                    reinterpret_cast<float *>(a.out)[(size_t)m * N + n] = y;
+                    reinterpret_cast<float *>(a.out)[(size_t)my_m * N + n] = y;
                     if (better(y, n, best_v, best_i)) { best_v = isnan(y) ? -INFINITY : y; best_i = n; }
                 }
             }
         }
-        __syncthreads();   // red[] is reused by the next tile
     }
 
     if (EPI == kEpiLogits) {
-        // per-CTA maximum for each m; thread t always handled m = t % MT
-        bvs[tid] = best_v;
-        bis[tid] = best_i;
+        // per-CTA maximum for each m over all its lanes' running maxima
+        bvs[threadIdx.x] = best_v;
+        bis[threadIdx.x] = best_i;
         __syncthreads();
-        if (tid < M) {
+        if (threadIdx.x < M) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
-            const int lim = min(n_out, nthreads);
-            for (int t = tid; t < lim; t += MT)
-                if (better(bvs[t], bis[t], bv, bi)) { bv = bvs[t]; bi = bis[t]; }
-            a.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-            a.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
+            for (int t = 0; t < kThreads; ++t) {
+                const int tv = lane_vid<V>(t & 31);
+                if (tv - (tv / MT) * MT == (int)threadIdx.x && better(bvs[t], bis[t], bv, bi)) {
+                    bv = bvs[t];
+                    bi = bis[t];
+                }
+            }
+            a.ws_val[(size_t)blockIdx.x * M + threadIdx.x] = bv;
+            a.ws_idx[(size_t)blockIdx.x * M + threadIdx.x] = bi;
         }
     }
 }

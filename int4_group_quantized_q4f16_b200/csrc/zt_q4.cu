@@ -27,18 +27,7 @@ int check_shapes(int M, int N, int K, int row_mult)
     return ZT_OK;
 }
 
-// Launch shape for a given K: WK warps split K (one 32-group chunk each), WR
-// warps split rows, at most 8 warps per CTA.
-void pick_warps(int G, int &wk, int &wr)
-{
-    wk = std::min(kMaxWarps, (G + 31) / 32);
-    wr = std::max(1, kMaxWarps / wk);
-}
-
 int smallest_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
-
-// rows per warp for each padded batch size (R * MT <= 32)
-int rows_per_warp(int mt) { return mt <= 4 ? 4 : 2; }
 
 struct OccKey {
     const void *fn;
@@ -57,6 +46,22 @@ struct OccHash {
     }
 };
 
+// last CUDA error seen by a library call on this host thread (diagnostics only)
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// Launch status: clear a stale non-sticky error left by an earlier, unrelated
+// runtime call before launching (so it is not blamed on this launch), then
+// read and clear the launch's own error.
+void clear_stale_error() { (void)cudaGetLastError(); }
+
+int launch_status()
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) return ZT_OK;
+    g_last_cuda_error = e;
+    return ZT_ERR_LAUNCH;
+}
+
 std::mutex g_mu;
 std::unordered_map<OccKey, int, OccHash> g_occ;   // resident CTAs per SM, or -1 if unusable
 std::unordered_map<int, int> g_sms;               // device -> SM count
@@ -66,13 +71,20 @@ std::unordered_map<int, int> g_sms;               // device -> SM count
 int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        return -1;
+    }
     std::lock_guard<std::mutex> lk(g_mu);
     auto it_s = g_sms.find(dev);
     if (it_s == g_sms.end()) {
         int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess || n < 1) {
+            g_last_cuda_error = e;
             return -1;
+        }
         it_s = g_sms.emplace(dev, n).first;
     }
     sms = it_s->second;
@@ -80,32 +92,37 @@ int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
     auto it = g_occ.find(key);
     if (it != g_occ.end()) return it->second;
     int occ = -1;
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) {
         int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem) == cudaSuccess && nb > 0)
-            occ = nb;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem);
+        if (e == cudaSuccess && nb > 0) occ = nb;
+    }
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return -1;   // not cached: a later call may succeed
     }
     g_occ.emplace(key, occ);
     return occ;
 }
 
-template <int R, int MT, int EPI>
+template <int R, int MT, int U, int EPI>
 int launch_one(Q4Args a, cudaStream_t st, int *grid_out)
 {
-    constexpr int V = R * MT;
     constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;
-    const int threads = a.wk * a.wr * 32;
-    const size_t smem = q4_smem_bytes(a.M, a.G, a.wk, a.wr, V);
+    const size_t smem = q4_smem_bytes(a.M, a.G);
     if (smem > 227 * 1024) return ZT_ERR_UNSUPPORTED;
-    const void *fn = reinterpret_cast<const void *>(&q4_gemv_kernel<R, MT, EPI>);
+    const void *fn = reinterpret_cast<const void *>(&q4_gemv_kernel<R, MT, U, EPI>);
     int sms = 0;
-    const int occ = resident_ctas(fn, threads, smem, sms);
+    const int occ = resident_ctas(fn, kThreads, smem, sms);
     if (occ < 1) return ZT_ERR_DEVICE;
-    a.n_tiles = (a.N + a.wr * ROUT - 1) / (a.wr * ROUT);
+    a.n_tiles = (a.N + ROUT - 1) / ROUT;
     const int grid = std::max(1, std::min({a.n_tiles, sms * occ, kMaxCtas}));
     if (grid_out) *grid_out = grid;
-    q4_gemv_kernel<R, MT, EPI><<<grid, threads, smem, st>>>(a);
-    return cudaPeekAtLastError() == cudaSuccess ? ZT_OK : ZT_ERR_LAUNCH;
+    clear_stale_error();
+    q4_gemv_kernel<R, MT, U, EPI><<<grid, kThreads, smem, st>>>(a);
+    return launch_status();
 }
 
 template <int EPI>
@@ -123,18 +140,15 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     a.N = N;
     a.K = K;
     a.G = K / kGroup;
-    pick_warps(a.G, a.wk, a.wr);
     a.n_tiles = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int mt = smallest_mt(M);
-    const int r = rows_per_warp(mt);
-    (void)r;
-    switch (mt) {
-    case 1: return launch_one<4, 1, EPI>(a, st, grid_out);
-    case 2: return launch_one<4, 2, EPI>(a, st, grid_out);
-    case 4: return launch_one<4, 4, EPI>(a, st, grid_out);
-    case 8: return launch_one<2, 8, EPI>(a, st, grid_out);
-    default: return launch_one<2, 16, EPI>(a, st, grid_out);
+    // rows per warp tile R, groups in flight per lane U, padded batch MT
+    switch (smallest_mt(M)) {
+    case 1: return launch_one<4, 1, 2, EPI>(a, st, grid_out);
+    case 2: return launch_one<4, 2, 1, EPI>(a, st, grid_out);
+    case 4: return launch_one<4, 4, 1, EPI>(a, st, grid_out);
+    case 8: return launch_one<2, 8, 1, EPI>(a, st, grid_out);
+    default: return launch_one<2, 16, 1, EPI>(a, st, grid_out);
     }
 }
 
@@ -146,6 +160,11 @@ extern "C" {
 
 int zt_q4_version(void) { return (1 << 16) | 0; }
 
+const char *zt_q4_last_cuda_error(void)
+{
+    return g_last_cuda_error == cudaSuccess ? "" : cudaGetErrorName(g_last_cuda_error);
+}
+
 const char *zt_q4_strerror(int status)
 {
     switch (status) {
@@ -154,7 +173,7 @@ const char *zt_q4_strerror(int status)
     case ZT_ERR_MISALIGNED: return "pointer misaligned (qw and x need 16 bytes, workspace 16, logits/argmax 4, scales/y 2)";
     case ZT_ERR_WORKSPACE: return "workspace smaller than zt_q4_lmhead_workspace_bytes()";
     case ZT_ERR_LAUNCH: return "CUDA kernel launch failed";
-    case ZT_ERR_UNSUPPORTED: return "shape is valid but exceeds this build's limits (activations must fit in shared memory: M*K*4.125 bytes)";
+    case ZT_ERR_UNSUPPORTED: return "shape is valid but exceeds this build's limits (staged activations must fit in shared memory: M*K*4.125 + 4096 bytes <= 227 KiB)";
     case ZT_ERR_DEVICE: return "no usable CUDA device, or a device attribute query failed";
     default: return "unknown status";
     }
@@ -203,7 +222,7 @@ int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16
     if (rc) return rc;
     q4_argmax_reduce_kernel<<<M, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ws_val, ws_idx, grid, M,
                                                                                    argmax);
-    return cudaPeekAtLastError() == cudaSuccess ? ZT_OK : ZT_ERR_LAUNCH;
+    return launch_status();
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)

@@ -31,7 +31,8 @@ _I = ctypes.c_int
 class ZtError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: status {status}: {strerror(status)}")
+        cuda = lib.zt_q4_last_cuda_error().decode() if status in (ZT_ERR_LAUNCH, ZT_ERR_DEVICE) else ""
+        super().__init__(f"{what}: status {status}: {strerror(status)}" + (f" [{cuda}]" if cuda else ""))
 
 
 def _load() -> ctypes.CDLL:
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_strerror.argtypes = [_I]
     lib.zt_q4_strerror.restype = ctypes.c_char_p
     lib.zt_q4_version.argtypes = []
+    lib.zt_q4_last_cuda_error.argtypes = []
+    lib.zt_q4_last_cuda_error.restype = ctypes.c_char_p
     for f in (lib.zt_q4_gemv, lib.zt_q4_gate_up_silu, lib.zt_q4_lmhead_argmax,
               lib.zt_q4_pack_host, lib.zt_q4_unpack_host, lib.zt_q4_version):
         f.restype = ctypes.c_int

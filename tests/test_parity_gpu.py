@@ -186,7 +186,10 @@ def test_lmhead_seed_sweep_with_planted_ties(zt, oracle):
             s16[0] += 1                              # one fp16 ulp in group 0
             s[near] = s16.view(np.float16)
             dups = [lo < top]
-        logits, am = run_lmhead(zt, qw, s, x)
+        try:
+            logits, am = run_lmhead(zt, qw, s, x)
+        except zt.ZtError as e:
+            raise AssertionError(f"seed {seed}: {e}") from e
         ref, _ = oracle.lmhead_argmax(qw, s, x, threads=8)
         assert rel_l2(logits, ref) <= 1e-5, f"seed {seed}"
         check_argmax(am, ref, exact_dups=dups if seed % 100 == 99 else None)
