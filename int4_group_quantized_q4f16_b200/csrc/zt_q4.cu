@@ -66,8 +66,11 @@ std::mutex g_mu;
 std::unordered_map<OccKey, int, OccHash> g_occ;   // resident CTAs per SM, or -1 if unusable
 std::unordered_map<int, int> g_sms;               // device -> SM count
 
-// resident CTAs per SM for (kernel, block, smem) on the current device,
-// opting the kernel in to that much dynamic shared memory on first use
+std::unordered_map<uint64_t, bool> g_optin;      // (kernel, device) opted in to the max smem
+
+// Resident CTAs per SM for (kernel, block, smem) on the current device.  On
+// first use of a kernel on a device its dynamic shared memory limit is raised
+// once to the device's opt-in maximum, so every later launch of any size fits.
 int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
 {
     int dev = 0;
@@ -88,23 +91,30 @@ int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
         it_s = g_sms.emplace(dev, n).first;
     }
     sms = it_s->second;
+    const uint64_t fkey = (uint64_t)(uintptr_t)fn * 64u + (uint64_t)dev;
+    if (g_optin.find(fkey) == g_optin.end()) {
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = e;
+            (void)cudaGetLastError();
+            return -1;
+        }
+        g_optin.emplace(fkey, true);
+    }
     OccKey key{fn, dev, threads, smem};
     auto it = g_occ.find(key);
     if (it != g_occ.end()) return it->second;
-    int occ = -1;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) {
-        int nb = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem);
-        if (e == cudaSuccess && nb > 0) occ = nb;
-    }
+    int nb = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, smem);
     if (e != cudaSuccess) {
         g_last_cuda_error = e;
         (void)cudaGetLastError();
-        return -1;   // not cached: a later call may succeed
+        return -1;
     }
-    g_occ.emplace(key, occ);
-    return occ;
+    g_occ.emplace(key, nb > 0 ? nb : -1);
+    return nb > 0 ? nb : -1;
 }
 
 template <int R, int MT, int U, int EPI>
