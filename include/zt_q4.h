@@ -37,6 +37,13 @@
  *     4 bytes; workspace 16 bytes.
  *   - Inputs and outputs must not overlap.
  *   - Thread safety: calls on different streams may run concurrently.
+ *   - Launch overlap: the kernels use programmatic dependent launch.  A call
+ *     may start streaming qw and scales from HBM before the kernel ahead of it
+ *     on the stream has finished; it reads x (and writes its outputs) only
+ *     after that kernel completes.  So x may be produced by the preceding
+ *     kernel, but qw and scales must not be written by a preceding kernel
+ *     that itself triggers dependent launches early (weights are meant to be
+ *     static; ordinary kernels, copies and the library's own calls are safe).
  */
 #ifndef ZT_Q4_H
 #define ZT_Q4_H
@@ -124,6 +131,16 @@ ZT_API int zt_q4_unpack_host(const uint32_t *qw, int N, int K, uint8_t *q);
 
 /* Static English text for a status code (never NULL). */
 ZT_API const char *zt_q4_strerror(int status);
+
+/*
+ * Read (and, if `clear` != 0, reset) the current device's error word: the OR
+ * of codes that kernels record when one of their bounded waits expires
+ * (1: a consumer waited > 2 s for data, 2: the producer waited > 2 s for a free
+ * stage, 4: copies were still in flight at exit).  0 means no kernel gave up.
+ * Synchronous (device-wide copy); for diagnostics and tests.  `out` is a HOST
+ * pointer.
+ */
+ZT_API int zt_q4_device_errors(unsigned int *out, int clear);
 
 /*
  * Name of the last CUDA runtime error a library call met on the calling host

@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(256) q4_argmax_reduce_kernel(const float *ws_v
 {
     __shared__ float sv[256];
     __shared__ int si[256];
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the first pass may still be running
     const int m = blockIdx.x;
     float bv = -INFINITY;
     int bi = 0x7fffffff;

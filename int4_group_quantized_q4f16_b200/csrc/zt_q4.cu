@@ -12,7 +12,12 @@
 #include <unordered_map>
 
 #include "q4_gemv.cuh"
+#include "q4_stream.cuh"
 #include "zt_q4.h"
+
+// Device error word: bounded waits that expire OR a code in here (read with
+// zt_q4_device_errors).  One per device, zero at load.
+__device__ unsigned int g_zt_device_errors = 0;
 
 namespace {
 
@@ -63,6 +68,7 @@ int launch_status()
 }
 
 std::mutex g_mu;
+std::unordered_map<int, unsigned int *> g_err_ptr;   // device -> &g_zt_device_errors
 std::unordered_map<OccKey, int, OccHash> g_occ;   // resident CTAs per SM, or -1 if unusable
 std::unordered_map<int, int> g_sms;               // device -> SM count
 
@@ -135,6 +141,83 @@ int launch_one(Q4Args a, cudaStream_t st, int *grid_out)
     return launch_status();
 }
 
+// Address of the device error word on the current device (cached).
+unsigned int *device_error_word()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_err_ptr.find(dev);
+    if (it != g_err_ptr.end()) return it->second;
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_zt_device_errors);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    g_err_ptr.emplace(dev, reinterpret_cast<unsigned int *>(p));
+    return reinterpret_cast<unsigned int *>(p);
+}
+
+// shared memory per CTA for 2 and for 1 resident CTA per SM (228 KiB per SM,
+// 1 KiB reserved per CTA)
+constexpr size_t kSmemTwoPerSm = 113 * 1024;
+constexpr size_t kSmemOnePerSm = 227 * 1024;
+
+// Launch the streaming kernel; ZT_ERR_UNSUPPORTED if its ring does not fit.
+template <int MT, int EPI>
+int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
+{
+    StreamArgs a;
+    a.qw = reinterpret_cast<const uint8_t *>(q.qw);
+    a.scales = q.scales;
+    a.x = q.x;
+    a.out = q.out;
+    a.ws_val = q.ws_val;
+    a.ws_idx = q.ws_idx;
+    a.M = q.M;
+    a.N = q.N;
+    a.K = q.K;
+    a.G = q.G;
+    a.scales_tma = (q.K % 256 == 0) && aligned(q.scales, 16);
+    const size_t fixed = stream_smem_bytes(q.M, q.G, 0);
+    int stages = 0;
+    for (size_t budget : {kSmemTwoPerSm, kSmemOnePerSm}) {
+        stages = budget > fixed ? (int)std::min<size_t>(kMaxStages, (budget - fixed) / kStageBytes) : 0;
+        if (stages >= 2) break;
+    }
+    if (stages < 2) return ZT_ERR_UNSUPPORTED;
+    a.stages = stages;
+    a.err = device_error_word();
+    if (!a.err) return ZT_ERR_DEVICE;
+    const size_t smem = stream_smem_bytes(q.M, q.G, stages);
+    const void *fn = reinterpret_cast<const void *>(&q4_stream_kernel<MT, EPI>);
+    int sms = 0;
+    const int occ = resident_ctas(fn, kSThreads, smem, sms);
+    if (occ < 1) return ZT_ERR_DEVICE;
+    const int grid = std::max(1, std::min({sms * occ, q.N, kMaxCtas}));
+    if (grid_out) *grid_out = grid;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kSThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    clear_stale_error();
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_stream_kernel<MT, EPI>, a);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    return ZT_OK;
+}
+
 template <int EPI>
 int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, void *out, float *ws_val,
               int *ws_idx, int M, int N, int K, void *stream, int *grid_out)
@@ -152,7 +235,18 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     a.G = K / kGroup;
     a.n_tiles = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // rows per warp tile R, groups in flight per lane U, padded batch MT
+    // Small batch: the TMA-streaming kernel when its ring fits in shared memory.
+    if (M <= 4) {
+        int rc = ZT_ERR_UNSUPPORTED;
+        switch (smallest_mt(M)) {
+        case 1: rc = launch_stream<1, EPI>(a, st, grid_out); break;
+        case 2: rc = launch_stream<2, EPI>(a, st, grid_out); break;
+        default: rc = launch_stream<4, EPI>(a, st, grid_out); break;
+        }
+        if (rc != ZT_ERR_UNSUPPORTED) return rc;
+    }
+    // Otherwise the register-pipelined kernel: rows per warp tile R, groups in
+    // flight per lane U, padded batch MT.
     switch (smallest_mt(M)) {
     case 1: return launch_one<4, 1, 2, EPI>(a, st, grid_out);
     case 2: return launch_one<4, 2, 1, EPI>(a, st, grid_out);
@@ -169,6 +263,24 @@ size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + s
 extern "C" {
 
 int zt_q4_version(void) { return (1 << 16) | 0; }
+
+int zt_q4_device_errors(unsigned int *out, int clear)
+{
+    if (!out) return ZT_ERR_INVALID_ARG;
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_zt_device_errors, sizeof(v));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_zt_device_errors, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_DEVICE;
+    }
+    *out = v;
+    return ZT_OK;
+}
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -230,9 +342,25 @@ int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16
     int grid = 0;
     rc = launch_q4<kEpiLogits>(qw, scales, x, logits, ws_val, ws_idx, M, N, K, stream, &grid);
     if (rc) return rc;
-    q4_argmax_reduce_kernel<<<M, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ws_val, ws_idx, grid, M,
-                                                                                   argmax);
-    return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(M);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    clear_stale_error();
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_argmax_reduce_kernel, (const float *)ws_val, (const int *)ws_idx,
+                                             grid, M, argmax);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    return ZT_OK;
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)
