@@ -133,16 +133,6 @@ ZT_API int zt_q4_unpack_host(const uint32_t *qw, int N, int K, uint8_t *q);
 ZT_API const char *zt_q4_strerror(int status);
 
 /*
- * Read (and, if `clear` != 0, reset) the current device's error word: the OR
- * of codes that kernels record when one of their bounded waits expires
- * (1: a consumer waited > 2 s for data, 2: the producer waited > 2 s for a free
- * stage, 4: copies were still in flight at exit).  0 means no kernel gave up.
- * Synchronous (device-wide copy); for diagnostics and tests.  `out` is a HOST
- * pointer.
- */
-ZT_API int zt_q4_device_errors(unsigned int *out, int clear);
-
-/*
  * Name of the last CUDA runtime error a library call met on the calling host
  * thread (e.g. "cudaErrorInvalidResourceHandle"), or "" if none.  Diagnostics
  * for ZT_ERR_LAUNCH / ZT_ERR_DEVICE; static storage, never NULL.

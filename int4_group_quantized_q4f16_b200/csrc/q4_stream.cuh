@@ -6,30 +6,31 @@
 // variants and the f32-output LM head) and its fused FFN (section "内核融合",
 // fused_ffn: gate, up and SiLU in one pass).  Arithmetic is the exact-product
 // scheme of q4_gemv.cuh (codes masked in place and read as subnormal floats,
-// pre-scaled activations, fp32 accumulation); only the data movement differs.
+// pre-scaled activations, fp32 accumulation); this file is about feeding it
+// from HBM at full rate.
 //
-// Data movement (one CTA = 1 producer warp + 8 consumer warps, 2 CTAs per SM):
+// Data movement (CTA = 8 warps; persistent grid sized from occupancy):
 //   * Each CTA owns a contiguous, balanced range of output rows, so every SM
-//     streams the same number of bytes and all finish together.
-//   * The rows are cut into tiles of 32 weight rows and each tile into chunks
-//     of 1024 k.  One (tile, chunk) item = 32 row pieces of 512 contiguous
-//     bytes of codes + 64 bytes of scales, moved by the producer with 1D TMA
-//     bulk copies (cp.async.bulk, no multicast) into a ring of S stages in
-//     shared memory, completion tracked by an mbarrier per stage.  With S - 1
-//     stages in flight per CTA the memory system sees tens of KB outstanding
-//     per SM without spending registers on it.
-//   * A consumer warp owns 4 weight rows of the tile; lane l reads group l of
-//     the chunk (16 bytes, conflict-free) and the 32 pre-scaled activations
-//     of that group once for all 4 rows.  Lane partials are combined by a
-//     warp-shuffle butterfly after the tile's last chunk.
+//     streams the same number of bytes.
+//   * The range is cut into tiles of 4 weight rows (rows x4; for the fused FFN
+//     2 gate + 2 up rows) and K into chunks of 32 groups (1024 k, one group
+//     per lane).  The 8 warps form WR x WK: WR warps deal the tiles, WK warps
+//     split the chunks of a tile (WK > 1 when the CTA has few rows, e.g. the
+//     3072-row projections), chosen on the host to balance items per warp.
+//   * Every warp owns a private ring of S stages in shared memory and fills
+//     it with 16-byte cp.async copies (LDGSTS, L2 only): lane l copies group l
+//     of each of the tile's 4 rows, lanes 0..3 the chunk's 64 bytes of scales.
+//     S - 1 items per warp are in flight while one is computed, i.e. tens of
+//     KB per SM without registers.  cp.async.wait_group is a hardware wait:
+//     the kernel contains no spin loops.
+//   * The pre-scaled activations of a group are read once from shared memory
+//     for all 4 rows of a tile.  Lane partials are combined by a warp-shuffle
+//     butterfly; WK > 1 partials meet in shared memory and are summed in a
+//     fixed order at the end: results are deterministic.
 //   * Programmatic dependent launch: the kernel lets the next kernel on the
-//     stream launch at once, and its producer starts streaming weights before
-//     the previous kernel has finished; only the activations are read after
-//     griddepcontrol.wait.  Consequence (stated in the C header): qw and scales
-//     must not be produced by a kernel that triggers dependent launches early.
-//   * Every wait on an mbarrier is bounded by a time limit; on expiry the
-//     kernel records an error code in a device word, drains its own copies in
-//     flight (again bounded) and returns.
+//     stream launch at once; each warp issues its first S - 1 weight copies
+//     before griddepcontrol.wait, so weights stream while the previous kernel
+//     finishes.  Activations are read and outputs written only after the wait.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -39,115 +40,71 @@
 
 namespace zt {
 
-constexpr int kSC = 8;                              // consumer warps per CTA
-constexpr int kSThreads = (kSC + 1) * 32;           // + one producer warp
-constexpr int kSR = 4;                              // weight rows per consumer warp per tile
-constexpr int kTileRows = kSC * kSR;                // weight rows per tile
-constexpr int kKC = 1024;                           // k per chunk: one group per lane
-constexpr int kChunkW = kKC / 2;                    // bytes of codes per row per chunk
-constexpr int kChunkS = kKC / 16;                   // bytes of scales per row per chunk
-constexpr int kStageBytes = kTileRows * (kChunkW + kChunkS);
-constexpr int kMaxStages = 8;
-constexpr int kBarBytes = 256;                      // barriers + flags at the front of smem
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
-
-// device error codes (OR-ed into StreamArgs::err)
-constexpr unsigned kErrFullTimeout = 1u;            // a consumer gave up waiting for data
-constexpr unsigned kErrEmptyTimeout = 2u;           // the producer gave up waiting for a free stage
-constexpr unsigned kErrDrainTimeout = 4u;           // copies still in flight at exit
+constexpr int kAW = 8;                              // warps per CTA
+constexpr int kAThreads = kAW * 32;
+constexpr int kAR = 4;                              // weight rows per tile
+constexpr int kAChunkG = 32;                        // groups per chunk (one per lane)
+constexpr int kARowBytes = kAChunkG * 16;           // codes of one row of a chunk: 512 B
+constexpr int kAScaleBytes = kAChunkG * 2;          // scales of one row of a chunk: 64 B
+constexpr int kAStage = kAR * (kARowBytes + kAScaleBytes);   // 2304 B per warp per stage
+constexpr int kAMaxStages = 8;
 
 struct StreamArgs {
-    const uint8_t *qw;          // packed codes, [rows][K/2] bytes
+    const uint4 *qw;            // [rows][G] 16-byte chunks
     const __half *scales;       // [rows][G]
     const __half *x;            // [M][K]
     void *out;                  // fp16 [M][N] or f32 [M][N]
     float *ws_val;              // Logits: per-CTA maximum [gridDim.x][M]
     int *ws_idx;
-    unsigned int *err;          // device error word
     int M, N, K, G;
-    int stages;                 // ring depth S (2..kMaxStages)
-    int scales_tma;             // 1: scales ride in the stage; 0: read from global
+    int stages;                 // ring depth S per warp (2..kAMaxStages)
+    int wk;                     // warps splitting K (1, 2, 4, 8); WR = 8 / wk
+    int max_tiles;              // tiles of the largest CTA range (sizes the WK > 1 buffer)
+    int scales_async;           // 1: scales copied with cp.async; 0: read from global
 };
 
-__host__ __device__ inline size_t stream_smem_bytes(int M, int G, int stages)
+__host__ __device__ inline size_t stream_smem_bytes(int M, int G, int stages, int wk, int max_tiles, int V)
 {
-    return (size_t)kBarBytes + (size_t)stages * kStageBytes + (size_t)M * G * 32 * 4 +
-           (((size_t)M * G * 4 + 15) & ~(size_t)15) + (size_t)kSC * 32 * 8;
+    const size_t ring = (size_t)kAW * stages * kAStage;
+    const size_t xs = (size_t)M * G * 32 * 4;
+    const size_t xg = ((size_t)M * G * 4 + 15) & ~(size_t)15;
+    const size_t red = wk > 1 ? (size_t)max_tiles * wk * V * 4 : 0;
+    return ring + xs + xg + ((red + 15) & ~(size_t)15) + (size_t)kAThreads * 8;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
 {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_dyn(int pending)
 {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long global_ns()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait for the phase of `bar` with parity `parity` to complete; false after
-// kWaitLimitNs without completion.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    for (;;) {
-#pragma unroll 1
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+    // wait_group takes an immediate: dispatch the ring depths in use
+    switch (pending) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<5>(); break;
+    default: cp_async_wait<6>(); break;
     }
-}
-
-// 1D bulk copy global -> this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
 }
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSC * 32) : "memory"); }
 
-// x staging for the consumer warps (same values as stage_activations).
-__device__ __forceinline__ void stage_x_consumers(const __half *__restrict__ x, float *xs, float *xg, int M, int K,
-                                                  int G, int tid)
+// Stage x for the whole CTA (same values as stage_activations in q4_gemv.cuh).
+__device__ __forceinline__ void stage_x_cta(const __half *__restrict__ x, float *xs, float *xg, int M, int K, int G)
 {
     const int K8 = K >> 3;
     for (int m = 0; m < M; ++m) {
-        for (int base = 0; base < K8; base += kSC * 32) {
-            const int kk = base + tid;
+        for (int base = 0; base < K8; base += kAThreads) {
+            const int kk = base + threadIdx.x;
             float part = 0.f;
             if (kk < K8) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)m * K + 8 * kk);
@@ -175,169 +132,135 @@ __device__ __forceinline__ void stage_x_consumers(const __half *__restrict__ x, 
 }
 
 template <int MT, int EPI>
-__global__ void __launch_bounds__(kSThreads, 2) q4_stream_kernel(const StreamArgs a)
+__global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArgs a)
 {
-    constexpr int R = kSR;
+    constexpr int R = kAR;
     constexpr int V = R * MT;
-    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;          // outputs per consumer warp
-    constexpr int TOUT = kSC * ROUT;                               // outputs per tile
+    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;          // outputs per tile
     static_assert(V <= 32 && (V & (V - 1)) == 0, "R*MT must be a power of two <= 32");
 
     extern __shared__ __align__(128) unsigned char smem[];
-    const int S = a.stages;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + kMaxStages;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kMaxStages);
-    unsigned char *stage0 = smem + kBarBytes;
-    float *xs = reinterpret_cast<float *>(stage0 + (size_t)S * kStageBytes);
-    float *xg = xs + (size_t)a.M * a.G * 32;
-    float *bvs = xg + (((size_t)a.M * a.G + 3) & ~(size_t)3);
-    int *bis = reinterpret_cast<int *>(bvs + kSC * 32);
-
-    const int M = a.M, N = a.N, K = a.K, G = a.G;
+    const int M = a.M, N = a.N, G = a.G, S = a.stages, wk = a.wk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    unsigned char *ring = smem + (size_t)warp * S * kAStage;
+    float *xs = reinterpret_cast<float *>(smem + (size_t)kAW * S * kAStage);
+    float *xg = xs + (size_t)M * G * 32;
+    float *red = xg + (((size_t)M * G + 3) & ~(size_t)3);
+    const size_t red_floats = wk > 1 ? (size_t)a.max_tiles * wk * V : 0;
+    float *bvs = red + ((red_floats + 3) & ~(size_t)3);
+    int *bis = reinterpret_cast<int *>(bvs + kAThreads);
 
-    // this CTA's output rows [o_begin, o_end)
-    const int o_begin = (int)(((long long)N * blockIdx.x) / gridDim.x);
-    const int o_end = (int)(((long long)N * (blockIdx.x + 1)) / gridDim.x);
-    const int n_tiles = (o_end - o_begin + TOUT - 1) / TOUT;
-    const int n_chunks = (K + kKC - 1) / kKC;
-    const int n_items = n_tiles * n_chunks;
-
-    if (tid == 0) {
-        for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSC);
-        }
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
     pdl_launch_dependents();
 
-    if (warp == kSC) {
-        // ------------------------------------------------------ producer --
-        if (lane == 0) {
-            const size_t row_bytes = (size_t)K / 2;
-            int issued = 0;
-            for (int i = 0; i < n_items; ++i) {
-                const int s = i % S;
-                if (i >= S && !mbar_wait_bounded(&empty[s], ((i / S) - 1) & 1)) {
-                    atomicOr(a.err, kErrEmptyTimeout);
-                    *abort_flag = 1;
-                    break;
-                }
-                if (*abort_flag) break;
-                const int t = i / n_chunks, c = i - t * n_chunks;
-                const int o0 = o_begin + t * TOUT;
-                const int rows = min(TOUT, o_end - o0);
-                const int kcount = min(kKC, K - c * kKC);
-                const uint32_t wbytes = (uint32_t)kcount / 2, sbytes = (uint32_t)kcount / 16;
-                const int halves = (EPI == kEpiGateUp) ? 2 : 1;
-                const uint32_t total = (uint32_t)(halves * rows) * (wbytes + (a.scales_tma ? sbytes : 0u));
-                unsigned char *sw = stage0 + (size_t)s * kStageBytes;
-                unsigned char *ss = sw + kTileRows * kChunkW;
-                mbar_arrive_expect_tx(&full[s], total);
-                for (int h = 0; h < halves; ++h) {
-                    for (int r = 0; r < rows; ++r) {
-                        const int slot = h * TOUT + r;
-                        const size_t wrow = (size_t)(h * N + o0 + r);
-                        bulk_g2s(sw + (size_t)slot * kChunkW, a.qw + wrow * row_bytes + (size_t)c * (kKC / 2), wbytes,
-                                 &full[s]);
-                        if (a.scales_tma)
-                            bulk_g2s(ss + (size_t)slot * kChunkS, a.scales + wrow * G + (size_t)c * (kKC / 32), sbytes,
-                                     &full[s]);
-                    }
-                }
-                issued = i + 1;
+    // this CTA's outputs [o_begin, o_end), tiles of ROUT outputs, chunks of 32 groups
+    const int o_begin = (int)(((long long)N * blockIdx.x) / gridDim.x);
+    const int o_end = (int)(((long long)N * (blockIdx.x + 1)) / gridDim.x);
+    const int n_tiles = (o_end - o_begin + ROUT - 1) / ROUT;
+    const int n_chunks = (G + kAChunkG - 1) / kAChunkG;
+    const int wr_n = kAW / wk;
+    const int my_wk = warp % wk, my_wr = warp / wk;
+    const int my_tiles = my_wr < n_tiles ? (n_tiles - my_wr + wr_n - 1) / wr_n : 0;
+    const int my_chunks = my_wk < n_chunks ? (n_chunks - my_wk + wk - 1) / wk : 0;
+    const int n_items = my_tiles * my_chunks;
+
+    // weight row of slot r of a tile starting at output o0 (clamped; rows past
+    // the CTA's range are copied but never stored)
+    auto weight_row = [&](int o0, int r) -> size_t {
+        if (EPI == kEpiGateUp) {
+            const int o = min(o0 + (r % ROUT), N - 1);
+            return (size_t)((r < ROUT) ? o : N + o);
+        }
+        return (size_t)min(o0 + r, N - 1);
+    };
+
+    auto issue = [&](int j) {
+        if (j < n_items) {
+            const int t = my_wr + wr_n * (j / my_chunks);
+            const int c = my_wk + wk * (j - (j / my_chunks) * my_chunks);
+            const int o0 = o_begin + t * ROUT;
+            unsigned char *st = ring + (size_t)(j % S) * kAStage;
+            const int g = c * kAChunkG + lane;
+            const int kc = min(kAChunkG, G - c * kAChunkG);        // groups in this chunk
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const size_t wrow = weight_row(o0, r);
+                if (lane < kc) cp_async16(st + r * kARowBytes + lane * 16, a.qw + wrow * G + g);
+                if (a.scales_async && lane < kc / 8)
+                    cp_async16(st + R * kARowBytes + r * kAScaleBytes + lane * 16,
+                               a.scales + wrow * G + c * kAChunkG + lane * 8);
             }
-            // drain: every copy this CTA issued must land before it exits
-            for (int i = max(0, issued - S); i < issued; ++i) {
-                if (!mbar_wait_bounded(&full[i % S], (i / S) & 1)) {
-                    atomicOr(a.err, kErrDrainTimeout);
-                    break;
+        }
+        cp_async_commit();     // always one group per item slot, so wait counts stay uniform
+    };
+
+    // prologue: weights stream before the previous kernel has finished
+    for (int j = 0; j < S - 1; ++j) issue(j);
+
+    pdl_wait();
+    stage_x_cta(a.x, xs, xg, M, a.K, G);
+    __syncthreads();
+
+    const int vid = lane_vid<V>(lane);
+    const bool rep = (lane & (32 / V - 1)) == 0;
+    const int my_r = vid / MT, my_m = vid - (vid / MT) * MT;
+    float best_v = -INFINITY;
+    int best_i = 0x7fffffff;
+    float part[V];
+
+    for (int j = 0; j < n_items; ++j) {
+        cp_async_wait_dyn(S - 2);          // item j's group has landed
+        __syncwarp();
+        const int tl = j / my_chunks, cl = j - (j / my_chunks) * my_chunks;
+        const int t = my_wr + wr_n * tl;
+        const int c = my_wk + wk * cl;
+        const int o0 = o_begin + t * ROUT;
+        if (cl == 0) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) part[v] = 0.f;
+        }
+        const int g = c * kAChunkG + lane;
+        if (g < G) {
+            const unsigned char *st = ring + (size_t)(j % S) * kAStage;
+            float sc[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                sc[r] = a.scales_async
+                            ? __half2float(reinterpret_cast<const __half *>(st + R * kARowBytes + r * kAScaleBytes)[lane])
+                            : __half2float(a.scales[weight_row(o0, r) * G + g]);
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m < M) {
+                    const float4 *xv4 = reinterpret_cast<const float4 *>(xs + ((size_t)m * G + g) * 32);
+                    const int swz = g & 7;
+                    float4 xv[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) xv[q] = xv4[q ^ swz];
+                    const float xgm = xg[m * G + g];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(st + r * kARowBytes + lane * 16);
+                        float2 acc = make_float2(0.f, 0.f);
+                        acc = word_dot(w.x, xv[0], xv[1], acc);
+                        acc = word_dot(w.y, xv[2], xv[3], acc);
+                        acc = word_dot(w.z, xv[4], xv[5], acc);
+                        acc = word_dot(w.w, xv[6], xv[7], acc);
+                        part[r * MT + m] = fmaf(sc[r], (acc.x + acc.y) - xgm, part[r * MT + m]);
+                    }
                 }
             }
         }
-    } else {
-        // ----------------------------------------------------- consumers --
-        pdl_wait();                                   // activations may come from the previous kernel
-        stage_x_consumers(a.x, xs, xg, M, K, G, tid);
-        consumers_sync();
+        __syncwarp();                      // the stage is free again (scales were read by all lanes)
+        issue(j + S - 1);
 
-        const int vid = lane_vid<V>(lane);
-        const bool rep = (lane & (32 / V - 1)) == 0;
-        const int my_r = vid / MT, my_m = vid - (vid / MT) * MT;
-        float best_v = -INFINITY;
-        int best_i = 0x7fffffff;
-        float part[V];
-
-        for (int i = 0; i < n_items; ++i) {
-            const int s = i % S;
-            if (*abort_flag) break;
-            if (!mbar_wait_bounded(&full[s], (i / S) & 1)) {
-                atomicOr(a.err, kErrFullTimeout);
-                *abort_flag = 1;
-                break;
-            }
-            const int t = i / n_chunks, c = i - t * n_chunks;
-            const int o0 = o_begin + t * TOUT;
-            const int rows = min(TOUT, o_end - o0);
-            if (c == 0) {
-#pragma unroll
-                for (int v = 0; v < V; ++v) part[v] = 0.f;
-            }
-            const int g = c * 32 + lane;
-            if (warp * ROUT < rows && g < G) {
-                const unsigned char *sw = stage0 + (size_t)s * kStageBytes;
-                const __half *ss = reinterpret_cast<const __half *>(sw + kTileRows * kChunkW);
-                int slot[R];
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-                    slot[r] = (EPI == kEpiGateUp) ? (r < ROUT ? warp * ROUT + r : TOUT + warp * ROUT + (r - ROUT))
-                                                  : warp * R + r;
-                uint4 w[R];
-                float sc[R];
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    w[r] = *reinterpret_cast<const uint4 *>(sw + (size_t)slot[r] * kChunkW + lane * 16);
-                    if (a.scales_tma) {
-                        sc[r] = __half2float(ss[slot[r] * (kChunkS / 2) + lane]);
-                    } else {
-                        const int orow = min(o0 + (slot[r] % TOUT), N - 1);
-                        const size_t wrow = (size_t)((slot[r] >= TOUT ? N : 0) + orow);
-                        sc[r] = __half2float(a.scales[wrow * G + g]);
-                    }
-                }
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (m < M) {
-                        const float4 *xv4 = reinterpret_cast<const float4 *>(xs + ((size_t)m * G + g) * 32);
-                        const int swz = g & 7;
-                        float4 xv[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) xv[q] = xv4[q ^ swz];
-                        const float xgm = xg[m * G + g];
-#pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            float2 acc = make_float2(0.f, 0.f);
-                            acc = word_dot(w[r].x, xv[0], xv[1], acc);
-                            acc = word_dot(w[r].y, xv[2], xv[3], acc);
-                            acc = word_dot(w[r].z, xv[4], xv[5], acc);
-                            acc = word_dot(w[r].w, xv[6], xv[7], acc);
-                            part[r * MT + m] = fmaf(sc[r], (acc.x + acc.y) - xgm, part[r * MT + m]);
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-
-            if (c == n_chunks - 1) {
-                int v_unused;
-                warp_transpose_reduce<V>(part, lane, v_unused);
+        if (cl == my_chunks - 1) {
+            int v_unused;
+            warp_transpose_reduce<V>(part, lane, v_unused);
+            if (wk > 1) {
+                if (rep) red[((size_t)t * wk + my_wk) * V + vid] = part[0];
+            } else {
                 const float y = part[0] * pow2f(59);
-                const int n = o0 + warp * ROUT + my_r;
+                const int n = o0 + my_r;
                 if (EPI == kEpiGateUp) {
                     const float u = __shfl_xor_sync(0xffffffffu, y, 16);
                     if (rep && vid < V / 2 && n < o_end && my_m < M) {
@@ -357,24 +280,67 @@ __global__ void __launch_bounds__(kSThreads, 2) q4_stream_kernel(const StreamArg
                 }
             }
         }
+    }
+    cp_async_wait<0>();
 
-        if (EPI == kEpiLogits) {
-            bvs[tid] = best_v;
-            bis[tid] = best_i;
-            consumers_sync();
-            if (tid < M) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-                for (int t = 0; t < kSC * 32; ++t) {
-                    const int tv = lane_vid<V>(t & 31);
-                    if (tv - (tv / MT) * MT == tid && better(bvs[t], bis[t], bv, bi)) {
-                        bv = bvs[t];
-                        bi = bis[t];
+    if (wk > 1) {
+        // partials of the WK warps of each tile meet here; fixed summation order
+        __syncthreads();
+        constexpr int VO = ROUT * MT;
+        for (int idx = tid; idx < n_tiles * VO; idx += kAThreads) {
+            const int t = idx / VO, vo = idx - (idx / VO) * VO;
+            const int r = vo / MT, m = vo - (vo / MT) * MT;
+            const int n = o_begin + t * ROUT + r;
+            const float *rp = red + (size_t)t * wk * V;
+            float y = 0.f, u = 0.f;
+            for (int k2 = 0; k2 < wk; ++k2) {
+                y += rp[k2 * V + r * MT + m];
+                if (EPI == kEpiGateUp) u += rp[k2 * V + (r + ROUT) * MT + m];
+            }
+            y *= pow2f(59);
+            if (n < o_end && m < M) {
+                if (EPI == kEpiF16) {
+                    reinterpret_cast<__half *>(a.out)[(size_t)m * N + n] = __float2half_rn(y);
+                } else if (EPI == kEpiGateUp) {
+                    u *= pow2f(59);
+                    const float silu = y / (1.0f + expf(-y));
+                    reinterpret_cast<__half *>(a.out)[(size_t)m * N + n] = __float2half_rn(silu * u);
+                } else {
+                    reinterpret_cast<float *>(a.out)[(size_t)m * N + n] = y;
+                    if (better(y, n, best_v, best_i)) {
+                        best_v = isnan(y) ? -INFINITY : y;
+                        best_i = n;
                     }
                 }
-                a.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-                a.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
             }
+        }
+    }
+
+    if (EPI == kEpiLogits) {
+        // per-CTA maximum per m.  Thread t holds maxima for m = (its vid) % MT
+        // when the warp epilogue ran (wk == 1), or for m = idx % MT when the
+        // shared-memory epilogue did (idx = t + 256 i, and 256 % MT == 0).
+        bvs[tid] = best_v;
+        bis[tid] = best_i;
+        __syncthreads();
+        if (tid < M) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int t = 0; t < kAThreads; ++t) {
+                int tm;
+                if (wk > 1) {
+                    tm = t % MT;
+                } else {
+                    const int tv = lane_vid<V>(t & 31);
+                    tm = tv - (tv / MT) * MT;
+                }
+                if (tm == tid && better(bvs[t], bis[t], bv, bi)) {
+                    bv = bvs[t];
+                    bi = bis[t];
+                }
+            }
+            a.ws_val[(size_t)blockIdx.x * M + tid] = bv;
+            a.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
         }
     }
 }

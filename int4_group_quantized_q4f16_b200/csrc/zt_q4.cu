@@ -15,10 +15,6 @@
 #include "q4_stream.cuh"
 #include "zt_q4.h"
 
-// Device error word: bounded waits that expire OR a code in here (read with
-// zt_q4_device_errors).  One per device, zero at load.
-__device__ unsigned int g_zt_device_errors = 0;
-
 namespace {
 
 using namespace zt;
@@ -68,7 +64,6 @@ int launch_status()
 }
 
 std::mutex g_mu;
-std::unordered_map<int, unsigned int *> g_err_ptr;   // device -> &g_zt_device_errors
 std::unordered_map<OccKey, int, OccHash> g_occ;   // resident CTAs per SM, or -1 if unusable
 std::unordered_map<int, int> g_sms;               // device -> SM count
 
@@ -141,36 +136,41 @@ int launch_one(Q4Args a, cudaStream_t st, int *grid_out)
     return launch_status();
 }
 
-// Address of the device error word on the current device (cached).
-unsigned int *device_error_word()
-{
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-    std::lock_guard<std::mutex> lk(g_mu);
-    auto it = g_err_ptr.find(dev);
-    if (it != g_err_ptr.end()) return it->second;
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_zt_device_errors);
-    if (e != cudaSuccess) {
-        g_last_cuda_error = e;
-        (void)cudaGetLastError();
-        return nullptr;
-    }
-    g_err_ptr.emplace(dev, reinterpret_cast<unsigned int *>(p));
-    return reinterpret_cast<unsigned int *>(p);
-}
-
 // shared memory per CTA for 2 and for 1 resident CTA per SM (228 KiB per SM,
 // 1 KiB reserved per CTA)
 constexpr size_t kSmemTwoPerSm = 113 * 1024;
 constexpr size_t kSmemOnePerSm = 227 * 1024;
 
-// Launch the streaming kernel; ZT_ERR_UNSUPPORTED if its ring does not fit.
+// Warps splitting K for the streaming kernel: minimise the items of the
+// busiest warp (tiles per row-warp x chunks per K-warp); ties -> smaller WK.
+int pick_wk(int max_tiles, int n_chunks)
+{
+    int best = 1;
+    long best_cost = -1;
+    for (int wk = 1; wk <= kAW; wk *= 2) {
+        if (wk > n_chunks) break;
+        const int wr = kAW / wk;
+        const long cost = (long)((max_tiles + wr - 1) / wr) * ((n_chunks + wk - 1) / wk);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = wk;
+        }
+    }
+    return best;
+}
+
+// Launch the streaming kernel; ZT_ERR_UNSUPPORTED if its rings and staged
+// activations do not fit in shared memory.
 template <int MT, int EPI>
 int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
 {
+    constexpr int V = kAR * MT;
+    constexpr int ROUT = (EPI == kEpiGateUp) ? kAR / 2 : kAR;
+    const void *fn = reinterpret_cast<const void *>(&q4_stream_kernel<MT, EPI>);
+    int sms = 0;
+    if (resident_ctas(fn, kAThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
     StreamArgs a;
-    a.qw = reinterpret_cast<const uint8_t *>(q.qw);
+    a.qw = q.qw;
     a.scales = q.scales;
     a.x = q.x;
     a.out = q.out;
@@ -180,42 +180,43 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
     a.N = q.N;
     a.K = q.K;
     a.G = q.G;
-    a.scales_tma = (q.K % 256 == 0) && aligned(q.scales, 16);
-    const size_t fixed = stream_smem_bytes(q.M, q.G, 0);
-    int stages = 0;
-    for (size_t budget : {kSmemTwoPerSm, kSmemOnePerSm}) {
-        stages = budget > fixed ? (int)std::min<size_t>(kMaxStages, (budget - fixed) / kStageBytes) : 0;
-        if (stages >= 2) break;
+    a.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+    const int n_chunks = (q.G + kAChunkG - 1) / kAChunkG;
+    for (int cps = 2; cps >= 1; --cps) {
+        const int grid = std::max(1, std::min({sms * cps, q.N, kMaxCtas}));
+        const int rows_max = (q.N + grid - 1) / grid;
+        a.max_tiles = (rows_max + ROUT - 1) / ROUT;
+        a.wk = pick_wk(a.max_tiles, n_chunks);
+        const size_t fixed = stream_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, V);
+        const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
+        const size_t per_stage = (size_t)kAW * kAStage;
+        const int stages = budget > fixed ? (int)std::min<size_t>(kAMaxStages, (budget - fixed) / per_stage) : 0;
+        if (stages < 2) continue;
+        a.stages = stages;
+        const size_t smem = stream_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, V);
+        const int occ = resident_ctas(fn, kAThreads, smem, sms);
+        if (occ < cps) continue;
+        if (grid_out) *grid_out = grid;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kAThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        clear_stale_error();
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_stream_kernel<MT, EPI>, a);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = e;
+            (void)cudaGetLastError();
+            return ZT_ERR_LAUNCH;
+        }
+        return ZT_OK;
     }
-    if (stages < 2) return ZT_ERR_UNSUPPORTED;
-    a.stages = stages;
-    a.err = device_error_word();
-    if (!a.err) return ZT_ERR_DEVICE;
-    const size_t smem = stream_smem_bytes(q.M, q.G, stages);
-    const void *fn = reinterpret_cast<const void *>(&q4_stream_kernel<MT, EPI>);
-    int sms = 0;
-    const int occ = resident_ctas(fn, kSThreads, smem, sms);
-    if (occ < 1) return ZT_ERR_DEVICE;
-    const int grid = std::max(1, std::min({sms * occ, q.N, kMaxCtas}));
-    if (grid_out) *grid_out = grid;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kSThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    clear_stale_error();
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_stream_kernel<MT, EPI>, a);
-    if (e != cudaSuccess) {
-        g_last_cuda_error = e;
-        (void)cudaGetLastError();
-        return ZT_ERR_LAUNCH;
-    }
-    return ZT_OK;
+    return ZT_ERR_UNSUPPORTED;
 }
 
 template <int EPI>
@@ -263,24 +264,6 @@ size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + s
 extern "C" {
 
 int zt_q4_version(void) { return (1 << 16) | 0; }
-
-int zt_q4_device_errors(unsigned int *out, int clear)
-{
-    if (!out) return ZT_ERR_INVALID_ARG;
-    unsigned int v = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(&v, g_zt_device_errors, sizeof(v));
-    if (e == cudaSuccess && clear) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_zt_device_errors, &zero, sizeof(zero));
-    }
-    if (e != cudaSuccess) {
-        g_last_cuda_error = e;
-        (void)cudaGetLastError();
-        return ZT_ERR_DEVICE;
-    }
-    *out = v;
-    return ZT_OK;
-}
 
 const char *zt_q4_last_cuda_error(void)
 {

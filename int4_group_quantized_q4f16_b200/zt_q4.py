@@ -51,8 +51,6 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_strerror.argtypes = [_I]
     lib.zt_q4_strerror.restype = ctypes.c_char_p
     lib.zt_q4_version.argtypes = []
-    lib.zt_q4_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint), _I]
-    lib.zt_q4_device_errors.restype = ctypes.c_int
     lib.zt_q4_last_cuda_error.argtypes = []
     lib.zt_q4_last_cuda_error.restype = ctypes.c_char_p
     for f in (lib.zt_q4_gemv, lib.zt_q4_gate_up_silu, lib.zt_q4_lmhead_argmax,
@@ -76,13 +74,6 @@ def version() -> Tuple[int, int]:
 def _check(rc: int, what: str) -> None:
     if rc != ZT_OK:
         raise ZtError(rc, what)
-
-
-def device_errors(clear: bool = False) -> int:
-    """The current device's error word (0: no kernel's bounded wait expired)."""
-    v = ctypes.c_uint(0)
-    _check(lib.zt_q4_device_errors(ctypes.byref(v), int(bool(clear))), "zt_q4_device_errors")
-    return int(v.value)
 
 
 # ------------------------------------------------------------ host layout --

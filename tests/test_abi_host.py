@@ -30,7 +30,7 @@ def test_header_declares_the_abi():
     syms = declared_symbols(HEADER)
     for want in ("zt_q4_gemv", "zt_q4_gate_up_silu", "zt_q4_lmhead_argmax",
                  "zt_q4_lmhead_workspace_bytes", "zt_q4_pack_host", "zt_q4_unpack_host",
-                 "zt_q4_strerror", "zt_q4_version", "zt_q4_device_errors",
+                 "zt_q4_strerror", "zt_q4_version",
                  "zt_q4_last_cuda_error"):
         assert want in syms
 
@@ -40,10 +40,6 @@ def test_library_exports_every_declared_symbol(zt):
         if path.endswith(".h"):
             for sym in declared_symbols(os.path.join(ROOT, "include", path)):
                 assert hasattr(zt.lib, sym), f"{sym} declared in {path} but not exported"
-
-
-def test_device_errors_rejects_null(zt):
-    assert zt.lib.zt_q4_device_errors(None, 0) == zt.ZT_ERR_INVALID_ARG
 
 
 def test_strerror_and_version(zt):
