@@ -90,6 +90,36 @@ __device__ __forceinline__ float2 word_dot(uint32_t w, const float4 &xa, const f
     return acc;
 }
 
+// sum over the 32 codes of one group (16 bytes) of q_k * x''_k, scaled by 2^-59
+__device__ __forceinline__ float group_dot(const uint4 &w, const float4 (&xv)[8])
+{
+#ifdef ZT_SCALAR_FMA
+    float acc0 = 0.f, acc1 = 0.f;
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t u = ws[i], h = u >> 12;
+        const float4 xa = xv[2 * i], xb = xv[2 * i + 1];
+        acc0 = fmaf(bits_f(u & 0xFu), xa.x, acc0);
+        acc1 = fmaf(bits_f(u & 0xF0u), xa.y, acc1);
+        acc0 = fmaf(bits_f(u & 0xF00u), xa.z, acc0);
+        acc1 = fmaf(bits_f(u & 0xF000u), xa.w, acc1);
+        acc0 = fmaf(bits_f(u & 0xF0000u), xb.x, acc0);
+        acc1 = fmaf(bits_f(u & 0xF00000u), xb.y, acc1);
+        acc0 = fmaf(bits_f(h & 0xF000u), xb.z, acc0);
+        acc1 = fmaf(bits_f(h & 0xF0000u), xb.w, acc1);
+    }
+    return acc0 + acc1;
+#else
+    float2 acc = make_float2(0.f, 0.f);
+    acc = word_dot(w.x, xv[0], xv[1], acc);
+    acc = word_dot(w.y, xv[2], xv[3], acc);
+    acc = word_dot(w.z, xv[4], xv[5], acc);
+    acc = word_dot(w.w, xv[6], xv[7], acc);
+    return acc.x + acc.y;
+#endif
+}
+
 // Transposing butterfly over the 32 lanes of a warp: on return every lane holds
 // in v[0] the warp-wide sum of value number `vid` (a function of the lane id).
 template <int V>

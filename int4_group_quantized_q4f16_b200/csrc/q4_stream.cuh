@@ -63,9 +63,10 @@ struct StreamArgs {
     int scales_async;           // 1: scales copied with cp.async; 0: read from global
 };
 
-__host__ __device__ inline size_t stream_smem_bytes(int M, int G, int stages, int wk, int max_tiles, int V)
+// R = weight rows per tile, V = R * MT partial sums per lane
+__host__ __device__ inline size_t stream_smem_bytes(int M, int G, int stages, int wk, int max_tiles, int R, int V)
 {
-    const size_t ring = (size_t)kAW * stages * kAStage;
+    const size_t ring = (size_t)kAW * stages * R * (kARowBytes + kAScaleBytes);
     const size_t xs = (size_t)M * G * 32 * 4;
     const size_t xg = ((size_t)M * G * 4 + 15) & ~(size_t)15;
     const size_t red = wk > 1 ? (size_t)max_tiles * wk * V * 4 : 0;
@@ -131,19 +132,19 @@ __device__ __forceinline__ void stage_x_cta(const __half *__restrict__ x, float 
     }
 }
 
-template <int MT, int EPI>
+template <int MT, int EPI, int R = kAR>
 __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArgs a)
 {
-    constexpr int R = kAR;
     constexpr int V = R * MT;
     constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;          // outputs per tile
+    constexpr int STAGE = R * (kARowBytes + kAScaleBytes);
     static_assert(V <= 32 && (V & (V - 1)) == 0, "R*MT must be a power of two <= 32");
 
     extern __shared__ __align__(128) unsigned char smem[];
     const int M = a.M, N = a.N, G = a.G, S = a.stages, wk = a.wk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    unsigned char *ring = smem + (size_t)warp * S * kAStage;
-    float *xs = reinterpret_cast<float *>(smem + (size_t)kAW * S * kAStage);
+    unsigned char *ring = smem + (size_t)warp * S * STAGE;
+    float *xs = reinterpret_cast<float *>(smem + (size_t)kAW * S * STAGE);
     float *xg = xs + (size_t)M * G * 32;
     float *red = xg + (((size_t)M * G + 3) & ~(size_t)3);
     const size_t red_floats = wk > 1 ? (size_t)a.max_tiles * wk * V : 0;
@@ -162,39 +163,53 @@ __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArg
     const int my_tiles = my_wr < n_tiles ? (n_tiles - my_wr + wr_n - 1) / wr_n : 0;
     const int my_chunks = my_wk < n_chunks ? (n_chunks - my_wk + wk - 1) / wk : 0;
     const int n_items = my_tiles * my_chunks;
+    const bool scales_async = a.scales_async != 0;
 
-    // weight row of slot r of a tile starting at output o0 (clamped; rows past
-    // the CTA's range are copied but never stored)
-    auto weight_row = [&](int o0, int r) -> size_t {
-        if (EPI == kEpiGateUp) {
-            const int o = min(o0 + (r % ROUT), N - 1);
-            return (size_t)((r < ROUT) ? o : N + o);
+    // Issue side: item counters advance without divisions.  Rows past the
+    // CTA's range are clamped (copied, never stored).
+    int is_tl = 0, is_cl = 0, is_stage = 0, is_left = n_items;
+    const uint4 *is_w[R];
+    const __half *is_s[R];
+    auto set_rows = [&](const uint4 **wp, const __half **sp, int tl) {
+        const int o0 = o_begin + (my_wr + wr_n * tl) * ROUT;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            int row;
+            if (EPI == kEpiGateUp) {
+                const int o = min(o0 + (r % ROUT), N - 1);
+                row = (r < ROUT) ? o : N + o;
+            } else {
+                row = min(o0 + r, N - 1);
+            }
+            wp[r] = a.qw + (size_t)row * G;
+            sp[r] = a.scales + (size_t)row * G;
         }
-        return (size_t)min(o0 + r, N - 1);
     };
-
-    auto issue = [&](int j) {
-        if (j < n_items) {
-            const int t = my_wr + wr_n * (j / my_chunks);
-            const int c = my_wk + wk * (j - (j / my_chunks) * my_chunks);
-            const int o0 = o_begin + t * ROUT;
-            unsigned char *st = ring + (size_t)(j % S) * kAStage;
+    if (n_items > 0) set_rows(is_w, is_s, 0);
+    auto issue_next = [&]() {
+        if (is_left > 0) {
+            const int c = my_wk + wk * is_cl;
+            unsigned char *st = ring + (size_t)is_stage * STAGE;
             const int g = c * kAChunkG + lane;
-            const int kc = min(kAChunkG, G - c * kAChunkG);        // groups in this chunk
+            const int kc = min(kAChunkG, G - c * kAChunkG);
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const size_t wrow = weight_row(o0, r);
-                if (lane < kc) cp_async16(st + r * kARowBytes + lane * 16, a.qw + wrow * G + g);
-                if (a.scales_async && lane < kc / 8)
-                    cp_async16(st + R * kARowBytes + r * kAScaleBytes + lane * 16,
-                               a.scales + wrow * G + c * kAChunkG + lane * 8);
+                if (lane < kc) cp_async16(st + r * kARowBytes + lane * 16, is_w[r] + g);
+                if (scales_async && lane < (kc >> 3))
+                    cp_async16(st + R * kARowBytes + r * kAScaleBytes + lane * 16, is_s[r] + c * kAChunkG + lane * 8);
+            }
+            --is_left;
+            if (++is_cl == my_chunks) {
+                is_cl = 0;
+                if (++is_tl < my_tiles) set_rows(is_w, is_s, is_tl);
             }
         }
-        cp_async_commit();     // always one group per item slot, so wait counts stay uniform
+        cp_async_commit();     // one group per item slot, so wait counts stay uniform
+        if (++is_stage == S) is_stage = 0;
     };
 
     // prologue: weights stream before the previous kernel has finished
-    for (int j = 0; j < S - 1; ++j) issue(j);
+    for (int j = 0; j < S - 1; ++j) issue_next();
 
     pdl_wait();
     stage_x_cta(a.x, xs, xg, M, a.K, G);
@@ -206,11 +221,14 @@ __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArg
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
     float part[V];
+    const __half *cs_s[R];
+    const uint4 *cs_w_unused[R];
+    int tl = 0, cl = 0, stage = 0;
+    if (n_items > 0 && !scales_async) set_rows(cs_w_unused, cs_s, 0);
 
     for (int j = 0; j < n_items; ++j) {
         cp_async_wait_dyn(S - 2);          // item j's group has landed
         __syncwarp();
-        const int tl = j / my_chunks, cl = j - (j / my_chunks) * my_chunks;
         const int t = my_wr + wr_n * tl;
         const int c = my_wk + wk * cl;
         const int o0 = o_begin + t * ROUT;
@@ -220,14 +238,13 @@ __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArg
         }
         const int g = c * kAChunkG + lane;
         if (g < G) {
-            const unsigned char *st = ring + (size_t)(j % S) * kAStage;
+            const unsigned char *st = ring + (size_t)stage * STAGE;
             float sc[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                sc[r] = a.scales_async
+            for (int r = 0; r < R; ++r)
+                sc[r] = scales_async
                             ? __half2float(reinterpret_cast<const __half *>(st + R * kARowBytes + r * kAScaleBytes)[lane])
-                            : __half2float(a.scales[weight_row(o0, r) * G + g]);
-            }
+                            : __half2float(cs_s[r][g]);
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m < M) {
@@ -240,18 +257,14 @@ __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArg
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(st + r * kARowBytes + lane * 16);
-                        float2 acc = make_float2(0.f, 0.f);
-                        acc = word_dot(w.x, xv[0], xv[1], acc);
-                        acc = word_dot(w.y, xv[2], xv[3], acc);
-                        acc = word_dot(w.z, xv[4], xv[5], acc);
-                        acc = word_dot(w.w, xv[6], xv[7], acc);
-                        part[r * MT + m] = fmaf(sc[r], (acc.x + acc.y) - xgm, part[r * MT + m]);
+                        part[r * MT + m] = fmaf(sc[r], group_dot(w, xv) - xgm, part[r * MT + m]);
                     }
                 }
             }
         }
         __syncwarp();                      // the stage is free again (scales were read by all lanes)
-        issue(j + S - 1);
+        issue_next();
+        if (++stage == S) stage = 0;
 
         if (cl == my_chunks - 1) {
             int v_unused;
@@ -279,6 +292,11 @@ __global__ void __launch_bounds__(kAThreads, 2) q4_stream_kernel(const StreamArg
                     }
                 }
             }
+        }
+        if (++cl == my_chunks) {
+            cl = 0;
+            ++tl;
+            if (!scales_async && tl < my_tiles) set_rows(cs_w_unused, cs_s, tl);
         }
     }
     cp_async_wait<0>();

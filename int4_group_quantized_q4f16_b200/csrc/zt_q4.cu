@@ -187,13 +187,13 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
         const int rows_max = (q.N + grid - 1) / grid;
         a.max_tiles = (rows_max + ROUT - 1) / ROUT;
         a.wk = pick_wk(a.max_tiles, n_chunks);
-        const size_t fixed = stream_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, V);
+        const size_t fixed = stream_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, kAR, V);
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const size_t per_stage = (size_t)kAW * kAStage;
         const int stages = budget > fixed ? (int)std::min<size_t>(kAMaxStages, (budget - fixed) / per_stage) : 0;
         if (stages < 2) continue;
         a.stages = stages;
-        const size_t smem = stream_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, V);
+        const size_t smem = stream_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, kAR, V);
         const int occ = resident_ctas(fn, kAThreads, smem, sms);
         if (occ < cps) continue;
         if (grid_out) *grid_out = grid;
