@@ -13,6 +13,7 @@
 
 #include "q4_gemv.cuh"
 #include "q4_stream.cuh"
+#include "q4_mma.cuh"
 #include "zt_q4.h"
 
 namespace {
@@ -219,6 +220,65 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
     return ZT_ERR_UNSUPPORTED;
 }
 
+// Launch the tensor-core kernel; ZT_ERR_UNSUPPORTED if its rings and staged
+// activations do not fit in shared memory.
+template <int NT, int EPI>
+int launch_mma(const Q4Args &q, cudaStream_t st, int *grid_out)
+{
+    constexpr int ROUT = (EPI == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;
+    const void *fn = reinterpret_cast<const void *>(&q4_mma_kernel<NT, EPI>);
+    int sms = 0;
+    if (resident_ctas(fn, kMThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
+    MmaArgs a;
+    a.qw = q.qw;
+    a.scales = q.scales;
+    a.x = q.x;
+    a.out = q.out;
+    a.ws_val = q.ws_val;
+    a.ws_idx = q.ws_idx;
+    a.M = q.M;
+    a.N = q.N;
+    a.K = q.K;
+    a.G = q.G;
+    a.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+    const int n_chunks = (q.G + kMChunkG - 1) / kMChunkG;
+    for (int cps = 2; cps >= 1; --cps) {
+        const int grid = std::max(1, std::min({sms * cps, q.N, kMaxCtas}));
+        const int rows_max = (q.N + grid - 1) / grid;
+        a.max_tiles = (rows_max + ROUT - 1) / ROUT;
+        a.wk = pick_wk(a.max_tiles, n_chunks);
+        const size_t fixed = mma_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, NT);
+        const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
+        const size_t per_stage = (size_t)kMW * kMStage;
+        const int stages = budget > fixed ? (int)std::min<size_t>(kMMaxStages, (budget - fixed) / per_stage) : 0;
+        if (stages < 2) continue;
+        a.stages = stages;
+        const size_t smem = mma_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, NT);
+        const int occ = resident_ctas(fn, kMThreads, smem, sms);
+        if (occ < cps) continue;
+        if (grid_out) *grid_out = grid;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kMThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        clear_stale_error();
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_mma_kernel<NT, EPI>, a);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = e;
+            (void)cudaGetLastError();
+            return ZT_ERR_LAUNCH;
+        }
+        return ZT_OK;
+    }
+    return ZT_ERR_UNSUPPORTED;
+}
+
 template <int EPI>
 int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, void *out, float *ws_val,
               int *ws_idx, int M, int N, int K, void *stream, int *grid_out)
@@ -236,7 +296,12 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     a.G = K / kGroup;
     a.n_tiles = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // Small batch: the TMA-streaming kernel when its ring fits in shared memory.
+    // The tensor-core kernel whenever its rings and activations fit.
+    {
+        const int rc = (M <= 8) ? launch_mma<1, EPI>(a, st, grid_out) : launch_mma<2, EPI>(a, st, grid_out);
+        if (rc != ZT_ERR_UNSUPPORTED) return rc;
+    }
+    // Small batch: the CUDA-core streaming kernel when its ring fits.
     if (M <= 4) {
         int rc = ZT_ERR_UNSUPPORTED;
         switch (smallest_mt(M)) {
