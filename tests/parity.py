@@ -3,10 +3,14 @@ library through its binding, and compare with the oracle.
 
 Tolerances (the stated bar): fp16 outputs relative L2 error <= 1e-3, f32
 logits <= 1e-5, argmax exact unless the oracle's top-2 logits are within 1e-3.
-On top of that, every fp16 output must lie within one fp16 ulp of the
-correctly rounded oracle value: the kernels form exact products and
-accumulate in fp32, so the only visible difference is on which side of a
-rounding boundary an fp32 sum falls.
+
+On top of that, every element is checked against a bound derived from the
+kernels' arithmetic: the products are exact and they are summed in fp32
+(tensor-core accumulation included), so an output can differ from the exact
+value by at most the fp32 accumulation error, bounded here generously by
+2^-14 * sum_k |w_k x_k| (the worst case of K <= 16384 fp32 additions is
+K * 2^-24), plus one ulp of the final fp16 rounding.  sum_k |w_k x_k| comes
+from the oracle itself (codes 7 + |q - 7| against |x|).
 """
 from __future__ import annotations
 
@@ -41,7 +45,18 @@ def rel_l2(got, ref) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
-def assert_f16_matches(got: np.ndarray, ref: np.ndarray, what: str = ""):
+ACC_BOUND = 2.0 ** -14
+
+
+def abs_products(oracle, qw, scales, x, rows=None) -> np.ndarray:
+    """sum_k |w_nk| |x_mk| in double, by the oracle: codes 7 + |q - 7| and |x|."""
+    q = oracle.unpack(qw, qw.shape[1] * 8).astype(np.int16)
+    qa = (7 + np.abs(q - 7)).astype(np.uint8)
+    xa = np.abs(np.asarray(x, dtype=np.float16))
+    return oracle.gemv(oracle.pack(qa), scales, xa, rows=rows, threads=8)
+
+
+def assert_f16_matches(got: np.ndarray, ref: np.ndarray, what: str = "", absprod=None):
     got = np.asarray(got, dtype=np.float16)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
@@ -50,10 +65,13 @@ def assert_f16_matches(got: np.ndarray, ref: np.ndarray, what: str = ""):
     assert r <= F16_REL_L2, f"{what}: rel L2 {r:.3e} > {F16_REL_L2}"
     ref16 = ref.astype(np.float16)
     ulp = np.spacing(np.abs(ref16)).astype(np.float64)
-    err = np.abs(got.astype(np.float64) - ref16.astype(np.float64))
-    bad = err > ulp
-    assert not bad.any(), (f"{what}: {int(bad.sum())} outputs more than 1 fp16 ulp from the "
-                           f"rounded oracle, e.g. index {np.argwhere(bad)[0].tolist()}")
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    bound = ulp + (ACC_BOUND * np.asarray(absprod, dtype=np.float64) if absprod is not None else 0.0)
+    bad = err > bound
+    if bad.any():
+        i = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} outputs outside the element bound, e.g. {list(i)}: "
+                             f"got {float(got[i])!r}, exact {float(ref[i])!r}, bound {float(bound[i]):.3g}")
 
 
 def assert_f32_matches(got: np.ndarray, ref: np.ndarray, what: str = ""):

@@ -5,8 +5,8 @@ import pytest
 
 from int4_group_quantized_q4f16_b200 import synth
 import oracle_pins as P
-from parity import (assert_f16_matches, assert_f32_matches, check_argmax, dev, host,
-                    rel_l2)
+from parity import (ACC_BOUND, abs_products, assert_f16_matches, assert_f32_matches, check_argmax, dev,
+                    host, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +37,8 @@ def run_lmhead(zt, qw, s, x):
 def test_single_gemv_seed0(zt, oracle):
     """M=1, K=256, N=512, seed 0: the small single-GEMV workload."""
     qw, s, x = synth.problem(0, 512, 256, M=1)
-    assert_f16_matches(run_gemv(zt, qw, s, x), oracle.gemv(qw, s, x), "gemv 512x256")
+    assert_f16_matches(run_gemv(zt, qw, s, x), oracle.gemv(qw, s, x), "gemv 512x256",
+                       abs_products(oracle, qw, s, x))
 
 
 SHAPES = [(1, 1, 32), (1, 33, 96), (2, 7, 64), (1, 1000, 1024), (3, 100, 352),
@@ -48,7 +49,8 @@ SHAPES = [(1, 1, 32), (1, 33, 96), (2, 7, 64), (1, 1000, 1024), (3, 100, 352),
 @pytest.mark.parametrize("M,N,K", SHAPES)
 def test_gemv_shapes(zt, oracle, M, N, K):
     qw, s, x = synth.problem(M * 1000 + N + K, N, K, M=M)
-    assert_f16_matches(run_gemv(zt, qw, s, x), oracle.gemv(qw, s, x), f"gemv M{M} N{N} K{K}")
+    assert_f16_matches(run_gemv(zt, qw, s, x), oracle.gemv(qw, s, x), f"gemv M{M} N{N} K{K}",
+                       abs_products(oracle, qw, s, x))
 
 
 @pytest.mark.parametrize("K", [32, 96, 256, 1056])
@@ -130,7 +132,20 @@ def test_gate_up(zt, oracle, M, N, K):
     rows = np.unique(np.concatenate([np.arange(min(N, 64)), np.arange(max(0, N - 64), N),
                                      np.random.default_rng(N).integers(0, N, 64)])).astype(np.int32)
     ref = oracle.gate_up_silu(qw, s, x, rows=rows, threads=8)
-    assert_f16_matches(got[:, rows], ref, f"gate_up M{M} N{N} K{K}")
+    assert_f16_matches(got[:, rows], ref, f"gate_up M{M} N{N} K{K}", gate_up_bound(oracle, qw, s, x, rows))
+
+
+def gate_up_bound(oracle, qw, s, x, rows):
+    """Element bound for SiLU(g) u: with |dg| <= eg, |du| <= eu (accumulation
+    errors as for a plain projection) the product moves by at most
+    |SiLU'| eg |u| + |SiLU(g)| eu + eg eu, and |SiLU'| <= 1.1."""
+    N = qw.shape[0] // 2
+    g = oracle.gemv(qw, s, x, rows=rows, threads=8)
+    u = oracle.gemv(qw, s, x, rows=rows + N, threads=8)
+    eg = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows)
+    eu = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows + N)
+    silu = g / (1.0 + np.exp(-g))
+    return (1.1 * eg * np.abs(u) + np.abs(silu) * eu + eg * eu) / ACC_BOUND
 
 
 def test_gate_up_order_pinned(zt, oracle):
@@ -143,7 +158,8 @@ def test_gate_up_order_pinned(zt, oracle):
     s = np.concatenate([np.full((N, K // 32), 0.0625, dtype=np.float16), s_up])
     x = np.ones((1, K), dtype=np.float16)
     got = run_gate_up(zt, qw, s, x)
-    assert_f16_matches(got, oracle.gate_up_silu(qw, s, x), "gate order")
+    assert_f16_matches(got, oracle.gate_up_silu(qw, s, x), "gate order",
+                       gate_up_bound(oracle, qw, s, x, np.arange(N, dtype=np.int32)))
 
 
 # ------------------------------------------------------------ LM head ----
@@ -229,7 +245,9 @@ def test_decode_layer_shapes_sampled(zt, oracle, model):
             if p.kind == "gemv":
                 got = run_gemv(zt, qw, s, x)
                 ref = oracle.gemv(qw, s, x, rows=rows, threads=8)
+                bound = abs_products(oracle, qw, s, x, rows=rows)
             else:
                 got = run_gate_up(zt, qw, s, x)
                 ref = oracle.gate_up_silu(qw, s, x, rows=rows, threads=8)
-            assert_f16_matches(got[:, rows], ref, f"{model} layer {li} {p.name}")
+                bound = gate_up_bound(oracle, qw, s, x, rows)
+            assert_f16_matches(got[:, rows], ref, f"{model} layer {li} {p.name}", bound)
