@@ -23,20 +23,23 @@
 //     (q0 * 2^-24, q4 * 2^-24), and (w & 0x00F000F0) is (16 q1 * 2^-24,
 //     16 q5 * 2^-24): one logic instruction dequantizes two codes, with no
 //     bias to subtract.
-//   * mma.sync.m16n8k16 (f16 x f16 -> f32) forms the exact products q * x *
-//     2^-24 (4-bit times 11-bit significands) and accumulates in fp32.  The
+//   * mma.sync.m16n8k16 (f16 x f16 -> f32) forms the products q * x * 2^-24
+//     exactly (4-bit times 11-bit significands) and accumulates in fp32.  The
 //     k axis inside a group is permuted consistently on the A and B sides (a
 //     dot product does not depend on the order of its terms), so that each
 //     thread's codes come from one 32-bit word: thread t of a quad owns word t
 //     (codes 8t..8t+7) of the group; step 0 of the group takes codes
 //     {0,4 | 2,6} of it (mask 0x000F000F on w and w >> 8), step 1 codes
-//     {1,5 | 3,7} (mask 0x00F000F0, carrying a factor 16).  The activations are
-//     staged once per CTA in that same order.
+//     {1,5 | 3,7} (mask 0x00F000F0, which carries a factor 16).  The
+//     activations are staged once per CTA in that order, and those meeting
+//     step 1 are staged divided by 16 -- exact for |x| >= 2^-10 (smaller ones
+//     are rounded to fp16 after the division, an absolute error below 2^-25
+//     per value).  So both steps accumulate into one fp32 tile.
 //   * Zero point: sum_k (q_k - 7) x_k = sum_k q_k x_k - 7 X_g; the -7 X_g term
 //     (X_g = sum of the group's activations, per column) enters as the C
-//     operand of the step-0 mma.  Step 1's factor 16 is removed with the scale:
-//     acc += s * D0 + (s / 16) * D1, in fp32, and the final 2^24 is an exact
-//     power-of-two multiply.
+//     operand of the group's first mma.  The group's result is scaled once:
+//     acc += s * D, in fp32, and the final 2^24 is an exact power-of-two
+//     multiply.
 //
 // Layout (mma tile = 16 weight rows x 8 columns of x):
 //   * A warp tile is 16 weight rows (for the fused FFN: 8 gate rows + the 8 up
@@ -84,12 +87,13 @@ struct MmaArgs {
 };
 
 // Per-CTA shared memory: rings, permuted activations (n-stride G*64 + 32
-// bytes), -7*X_g table [G][8*NT] f32, WK > 1 partials, LM-head maxima.
+// bytes), C-operand table [G][NT][4 quad threads][c0 c1 c0 c1] f32 (= -7 X_g
+// 2^-24 of columns 8nt + 2t, + 1), WK > 1 partials, LM-head maxima.
 __host__ __device__ inline size_t mma_smem_bytes(int M, int G, int stages, int wk, int max_tiles, int NT)
 {
     const size_t ring = (size_t)kMW * stages * kMStage;
     const size_t xp = (size_t)M * ((size_t)G * 64 + 32);
-    const size_t x7 = (size_t)G * 8 * NT * 4;
+    const size_t x7 = (size_t)G * NT * 64;
     const size_t red = wk > 1 ? (size_t)max_tiles * wk * kMTileRows * 8 * NT * 4 : 0;
     const size_t best = (size_t)kMThreads * 2 * NT * 8;
     return ring + ((xp + 15) & ~(size_t)15) + x7 + red + best;
@@ -107,12 +111,17 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 
 // Stage x in mma-B order: for column n and group g, 64 bytes = for t = 0..3:
 // step 0 (x[8t], x[8t+4], x[8t+2], x[8t+6]), step 1 (x[8t+1], x[8t+5],
-// x[8t+3], x[8t+7]) (k relative to 32g).  x7[g][n] = -7 * X_g * 2^-24.
+// x[8t+3], x[8t+7]) / 16 (k relative to 32g).  The C table holds, for each
+// (g, n-tile, quad thread t), (c, c', c, c') with c = -7 X_g 2^-24 of column
+// 8 nt + 2t and c' of the next column (zero for columns >= M).
 __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsigned char *xp, float *x7, int M,
                                             int K, int G, int NT)
 {
     const int K8 = K >> 3;
     const size_t nstride = (size_t)G * 64 + 32;
+    const __half2 sixteenth = __float2half2_rn(0.0625f);
+    for (int i = threadIdx.x; i < G * NT * 16; i += kMThreads) x7[i] = 0.f;
+    __syncthreads();
     for (int m = 0; m < M; ++m) {
         for (int base = 0; base < K8; base += kMThreads) {
             const int kk = base + threadIdx.x;      // (g = kk / 4, t = kk % 4)
@@ -123,8 +132,12 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
                 uint4 o;
                 o.x = __byte_perm(v01, v45, 0x5410);   // (x0, x4)
                 o.y = __byte_perm(v23, v67, 0x5410);   // (x2, x6)
-                o.z = __byte_perm(v01, v45, 0x7632);   // (x1, x5)
-                o.w = __byte_perm(v23, v67, 0x7632);   // (x3, x7)
+                uint32_t h15 = __byte_perm(v01, v45, 0x7632);   // (x1, x5)
+                uint32_t h37 = __byte_perm(v23, v67, 0x7632);   // (x3, x7)
+                __half2 q15 = __hmul2(*reinterpret_cast<__half2 *>(&h15), sixteenth);
+                __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
+                o.z = *reinterpret_cast<uint32_t *>(&q15);
+                o.w = *reinterpret_cast<uint32_t *>(&q37);
                 *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = o;
                 const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
                 float v[8];
@@ -138,12 +151,15 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
             }
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
-            if (kk < K8 && (kk & 3) == 0) x7[(size_t)(kk >> 2) * 8 * NT + m] = part * (-7.0f * pow2f(-24));
+            if (kk < K8 && (kk & 3) == 0) {
+                const float c = part * (-7.0f * pow2f(-24));
+                const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+                float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+                cv[e] = c;
+                cv[2 + e] = c;
+            }
         }
     }
-    // columns M .. 8*NT-1 of the table are zero
-    for (int i = threadIdx.x; i < G * 8 * NT; i += kMThreads)
-        if (i % (8 * NT) >= M) x7[i] = 0.f;
 }
 
 template <int NT, int EPI>
@@ -159,7 +175,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
     unsigned char *xp = smem + (size_t)kMW * S * kMStage;
     const size_t nstride = (size_t)G * 64 + 32;
     float *x7 = reinterpret_cast<float *>(xp + (((size_t)M * nstride + 15) & ~(size_t)15));
-    float *red = x7 + (size_t)G * 8 * NT;
+    float *red = x7 + (size_t)G * NT * 16;
     const size_t red_floats = wk > 1 ? (size_t)a.max_tiles * wk * kMTileRows * 8 * NT : 0;
     float *bvs = red + red_floats;
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
@@ -190,32 +206,43 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
     };
 
     // ---------------------------------------------------------- issue side --
+    // Lane l copies pieces p = l + 32 i (i < 4) of an item: tile row
+    // r = l / 8 + 4 i, group l % 8 of the chunk.  Its source rows change per
+    // tile only; per item just the chunk offset moves.
+    const int pg = lane & 7;
     int is_tl = 0, is_cl = 0, is_stage = 0, is_left = n_items;
+    const uint4 *src_w[4];
+    bool ok_w[4];
+    const __half *src_s = a.scales;
+    bool ok_s = false;
+    auto set_tile = [&](int tl) {
+        const int o0 = o_begin + (my_wr + wr_n * tl) * ROUT;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int row = slot_row(o0, (lane >> 3) + 4 * i, ok_w[i]);
+            src_w[i] = a.qw + (size_t)row * G + pg;
+        }
+        if (lane < kMTileRows) {
+            const int row = slot_row(o0, lane, ok_s);
+            src_s = a.scales + (size_t)row * G;
+        }
+    };
+    if (n_items > 0) set_tile(0);
     auto issue_next = [&]() {
         if (is_left > 0) {
-            const int t = my_wr + wr_n * is_tl;
             const int c = my_wk + wk * is_cl;
-            const int o0 = o_begin + t * ROUT;
-            const int kc = min(kMChunkG, G - c * kMChunkG);
-            unsigned char *st = ring + (size_t)is_stage * kMStage;
+            const bool full = (c + 1) * kMChunkG <= G;
+            const int kc = full ? kMChunkG : G - c * kMChunkG;
+            unsigned char *st = ring + (size_t)is_stage * kMStage + (lane >> 3) * kMRowStride + pg * 16;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int p = lane + 32 * i;           // piece: (row p / 8, group p % 8)
-                const int r = p >> 3, gl = p & 7;
-                bool valid;
-                const int row = slot_row(o0, r, valid);
-                if (valid && gl < kc)
-                    cp_async16(st + r * kMRowStride + gl * 16, a.qw + (size_t)row * G + c * kMChunkG + gl);
-            }
-            if (scales_async && lane < kMTileRows) {
-                bool valid;
-                const int row = slot_row(o0, lane, valid);
-                if (valid) cp_async16(st + kMScaleOff + lane * 16, a.scales + (size_t)row * G + c * kMChunkG);
-            }
+            for (int i = 0; i < 4; ++i)
+                if (ok_w[i] && pg < kc) cp_async16(st + 4 * i * kMRowStride, src_w[i] + c * kMChunkG);
+            if (scales_async && ok_s && lane < kMTileRows)
+                cp_async16(ring + (size_t)is_stage * kMStage + kMScaleOff + lane * 16, src_s + c * kMChunkG);
             --is_left;
             if (++is_cl == my_chunks) {
                 is_cl = 0;
-                ++is_tl;
+                if (++is_tl < my_tiles) set_tile(is_tl);
             }
         }
         cp_async_commit();
@@ -276,12 +303,14 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
             sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
         }
         const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+        const unsigned char *wrow0 = st + qg * kMRowStride + qt * 4;
+        const unsigned char *wrow1 = wrow0 + 8 * kMRowStride;
 #pragma unroll
         for (int gl = 0; gl < kMChunkG; ++gl) {
             if (gl < kc) {
                 const int g = c * kMChunkG + gl;
-                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(st + qg * kMRowStride + gl * 16 + qt * 4);
-                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(st + (qg + 8) * kMRowStride + gl * 16 + qt * 4);
+                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wrow0 + gl * 16);
+                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wrow1 + gl * 16);
                 const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
                 const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
                 const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
@@ -289,25 +318,17 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
                 const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
                 const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
                 const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
-                const float2 sp0 = make_float2(s0, s0), sp1 = make_float2(s1, s1);
-                const float2 sq0 = make_float2(s0 * 0.0625f, s0 * 0.0625f), sq1 = make_float2(s1 * 0.0625f, s1 * 0.0625f);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint2 b0 = *reinterpret_cast<const uint2 *>(xb[nt] + (size_t)g * 64);
-                    const uint2 b1 = *reinterpret_cast<const uint2 *>(xb[nt] + (size_t)g * 64 + 8);
-                    const float2 cz = *reinterpret_cast<const float2 *>(x7 + (size_t)g * 8 * NT + 8 * nt + 2 * qt);
-                    float d0[4], d1[4];
-                    mma_16816(d0, A0, b0.x, b0.y, cz.x, cz.y, cz.x, cz.y);
-                    mma_16816(d1, A1, b1.x, b1.y, 0.f, 0.f, 0.f, 0.f);
-                    float2 lo = make_float2(acc[nt][0], acc[nt][1]), hi = make_float2(acc[nt][2], acc[nt][3]);
-                    lo = __ffma2_rn(make_float2(d0[0], d0[1]), sp0, lo);
-                    hi = __ffma2_rn(make_float2(d0[2], d0[3]), sp1, hi);
-                    lo = __ffma2_rn(make_float2(d1[0], d1[1]), sq0, lo);
-                    hi = __ffma2_rn(make_float2(d1[2], d1[3]), sq1, hi);
-                    acc[nt][0] = lo.x;
-                    acc[nt][1] = lo.y;
-                    acc[nt][2] = hi.x;
-                    acc[nt][3] = hi.y;
+                    const uint4 bb = *reinterpret_cast<const uint4 *>(xb[nt] + (size_t)g * 64);
+                    const float4 cz = *reinterpret_cast<const float4 *>(x7 + (((size_t)g * NT + nt) * 4 + qt) * 4);
+                    float d[4];
+                    mma_16816(d, A0, bb.x, bb.y, cz.x, cz.y, cz.z, cz.w);
+                    mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                    acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                    acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                    acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                    acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
                 }
             }
         }
