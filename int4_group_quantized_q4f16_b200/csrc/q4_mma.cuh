@@ -99,10 +99,29 @@ __host__ __device__ inline size_t mma_smem_bytes(int M, int G, int stages, int w
     return ring + ((xp + 15) & ~(size_t)15) + x7 + red + best;
 }
 
+// Shared-memory loads by 32-bit shared-window address (keeps address math
+// 32-bit and the loads explicit LDS).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void cp_async16_u32(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
                                           float c0, float c1, float c2, float c3)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%10,%11,%12,%13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
@@ -228,17 +247,19 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
         }
     };
     if (n_items > 0) set_tile(0);
+    const uint32_t ring_u = smem_u32(ring);
+    const uint32_t piece_u = ring_u + (lane >> 3) * kMRowStride + pg * 16;   // + stage, + 4 i rows
+    const uint32_t scale_u = ring_u + kMScaleOff + lane * 16;
     auto issue_next = [&]() {
         if (is_left > 0) {
             const int c = my_wk + wk * is_cl;
             const bool full = (c + 1) * kMChunkG <= G;
             const int kc = full ? kMChunkG : G - c * kMChunkG;
-            unsigned char *st = ring + (size_t)is_stage * kMStage + (lane >> 3) * kMRowStride + pg * 16;
+            const uint32_t so = (uint32_t)is_stage * kMStage;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok_w[i] && pg < kc) cp_async16(st + 4 * i * kMRowStride, src_w[i] + c * kMChunkG);
-            if (scales_async && ok_s && lane < kMTileRows)
-                cp_async16(ring + (size_t)is_stage * kMStage + kMScaleOff + lane * 16, src_s + c * kMChunkG);
+                if (ok_w[i] && pg < kc) cp_async16_u32(piece_u + so + 4 * i * kMRowStride, src_w[i] + c * kMChunkG);
+            if (scales_async && ok_s && lane < kMTileRows) cp_async16_u32(scale_u + so, src_s + c * kMChunkG);
             --is_left;
             if (++is_cl == my_chunks) {
                 is_cl = 0;
@@ -256,9 +277,12 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
     __syncthreads();
 
     // B-operand column of this lane (columns >= M read column M-1: ignored)
-    const unsigned char *xb[NT];
+    uint32_t xb[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) xb[nt] = xp + (size_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
+    for (int nt = 0; nt < NT; ++nt) xb[nt] = smem_u32(xp) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
+    const uint32_t x7_u = smem_u32(x7) + qt * 16;
+    const uint32_t wq_u = ring_u + qg * kMRowStride + qt * 4;          // + stage + row block + group
+    const uint32_t sc_u = ring_u + kMScaleOff + qg * 16;
 
     float acc[NT][4];
     float best_v[2 * NT];
@@ -283,12 +307,12 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
         }
-        const unsigned char *st = ring + (size_t)stage * kMStage;
+        const uint32_t so = (uint32_t)stage * kMStage;
         // scales of rows qg and qg + 8 for the item's 8 groups
         uint4 sg, sg8;
         if (scales_async) {
-            sg = *reinterpret_cast<const uint4 *>(st + kMScaleOff + qg * 16);
-            sg8 = *reinterpret_cast<const uint4 *>(st + kMScaleOff + (qg + 8) * 16);
+            sg = lds_u128(sc_u + so);
+            sg8 = lds_u128(sc_u + so + 8 * 16);
         } else {
             bool v0, v1;
             const int r0 = slot_row(o0, qg, v0), r1 = slot_row(o0, qg + 8, v1);
@@ -303,14 +327,14 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
             sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
         }
         const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-        const unsigned char *wrow0 = st + qg * kMRowStride + qt * 4;
-        const unsigned char *wrow1 = wrow0 + 8 * kMRowStride;
+        const uint32_t wrow0 = wq_u + so;
+        const uint32_t xb0 = (uint32_t)(c * kMChunkG) * 64u;                   // + xb[nt] + gl * 64
+        const uint32_t x70 = x7_u + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
 #pragma unroll
         for (int gl = 0; gl < kMChunkG; ++gl) {
             if (gl < kc) {
-                const int g = c * kMChunkG + gl;
-                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wrow0 + gl * 16);
-                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wrow1 + gl * 16);
+                const uint32_t w0 = lds_u32(wrow0 + gl * 16);
+                const uint32_t w1 = lds_u32(wrow0 + 8 * kMRowStride + gl * 16);
                 const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
                 const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
                 const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
@@ -320,8 +344,10 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
                 const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 bb = *reinterpret_cast<const uint4 *>(xb[nt] + (size_t)g * 64);
-                    const float4 cz = *reinterpret_cast<const float4 *>(x7 + (((size_t)g * NT + nt) * 4 + qt) * 4);
+                    const uint4 bb = lds_u128(xb[nt] + xb0 + gl * 64);
+                    const uint4 czu = lds_u128(x70 + (gl * NT + nt) * 64);
+                    const float4 cz = make_float4(__uint_as_float(czu.x), __uint_as_float(czu.y),
+                                                  __uint_as_float(czu.z), __uint_as_float(czu.w));
                     float d[4];
                     mma_16816(d, A0, bb.x, bb.y, cz.x, cz.y, cz.z, cz.w);
                     mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
