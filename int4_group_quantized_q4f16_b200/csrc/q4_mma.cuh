@@ -181,8 +181,12 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
     }
 }
 
+#ifndef ZT_MMA_MIN_CTAS
+#define ZT_MMA_MIN_CTAS 2
+#endif
+
 template <int NT, int EPI>
-__global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
+__global__ void __launch_bounds__(kMThreads, ZT_MMA_MIN_CTAS) q4_mma_kernel(const MmaArgs a)
 {
     constexpr int ROUT = (EPI == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;   // outputs per tile
     extern __shared__ __align__(128) unsigned char smem[];
@@ -276,13 +280,17 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
     stage_x_mma(a.x, xp, x7, M, a.K, G, NT);
     __syncthreads();
 
-    // B-operand column of this lane (columns >= M read column M-1: ignored)
-    uint32_t xb[NT];
+    // Byte offsets from the start of shared memory; loads index the shared
+    // array directly, so the compiler sees shared-space, 32-bit addressing.
+    const uint32_t *smw = reinterpret_cast<const uint32_t *>(smem);
+    const uint4 *smq = reinterpret_cast<const uint4 *>(smem);
+    const uint32_t ring_o = (uint32_t)(ring - smem);
+    uint32_t xb[NT];       // B-operand column of this lane (columns >= M read column M-1: ignored)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) xb[nt] = smem_u32(xp) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
-    const uint32_t x7_u = smem_u32(x7) + qt * 16;
-    const uint32_t wq_u = ring_u + qg * kMRowStride + qt * 4;          // + stage + row block + group
-    const uint32_t sc_u = ring_u + kMScaleOff + qg * 16;
+    for (int nt = 0; nt < NT; ++nt) xb[nt] = (uint32_t)(xp - smem) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
+    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
+    const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
+    const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
 
     float acc[NT][4];
     float best_v[2 * NT];
@@ -311,8 +319,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
         // scales of rows qg and qg + 8 for the item's 8 groups
         uint4 sg, sg8;
         if (scales_async) {
-            sg = lds_u128(sc_u + so);
-            sg8 = lds_u128(sc_u + so + 8 * 16);
+            sg = smq[(sc_o + so) >> 4];
+            sg8 = smq[(sc_o + so + 8 * 16) >> 4];
         } else {
             bool v0, v1;
             const int r0 = slot_row(o0, qg, v0), r1 = slot_row(o0, qg + 8, v1);
@@ -327,36 +335,40 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_mma_kernel(const MmaArgs a)
             sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
         }
         const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-        const uint32_t wrow0 = wq_u + so;
+        const uint32_t wrow0 = wq_o + so;
         const uint32_t xb0 = (uint32_t)(c * kMChunkG) * 64u;                   // + xb[nt] + gl * 64
-        const uint32_t x70 = x7_u + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
+        const uint32_t x70 = x7_o + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
+        auto step = [&](int gl) {
+            const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
+            const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
+            const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+            const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
+            const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
+            const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+            const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+            const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+            const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
 #pragma unroll
-        for (int gl = 0; gl < kMChunkG; ++gl) {
-            if (gl < kc) {
-                const uint32_t w0 = lds_u32(wrow0 + gl * 16);
-                const uint32_t w1 = lds_u32(wrow0 + 8 * kMRowStride + gl * 16);
-                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
-                const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
-                const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 bb = lds_u128(xb[nt] + xb0 + gl * 64);
-                    const uint4 czu = lds_u128(x70 + (gl * NT + nt) * 64);
-                    const float4 cz = make_float4(__uint_as_float(czu.x), __uint_as_float(czu.y),
-                                                  __uint_as_float(czu.z), __uint_as_float(czu.w));
-                    float d[4];
-                    mma_16816(d, A0, bb.x, bb.y, cz.x, cz.y, cz.z, cz.w);
-                    mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                    acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                    acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                    acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                    acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
-                }
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint4 bb = smq[(xb[nt] + xb0 + gl * 64) >> 4];
+                const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
+                float d[4];
+                mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y), __uint_as_float(czu.z),
+                          __uint_as_float(czu.w));
+                mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
             }
+        };
+        if (kc == kMChunkG) {
+#pragma unroll
+            for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
+        } else {
+#pragma unroll
+            for (int gl = 0; gl < kMChunkG; ++gl)
+                if (gl < kc) step(gl);
         }
         __syncwarp();
         issue_next();
