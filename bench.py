@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the q4f16 dequantizing GEMV hot path on B200.
+
+One step = one Phi-3-mini-shaped decode weight pass at M = 1: 32 layers of
+{qkv 3072->9216, o 3072->3072, gate_up 3072->2x8192 with SiLU(gate)*up,
+down 8192->3072} plus the LM head 3072->32064 (f32 logits + argmax), on
+seeded synthetic q4 weights (2.1 GB, larger than L2, so no flush is needed
+between steps).  The step runs as a CUDA graph of 130 launches of this
+library's kernels.
+
+Prints one JSON line (rank 0).  Metric: effective HBM GB/s of the pass
+(algorithmic bytes / time); the line also carries us per pass, the roofline
+of the dominant kernel, the CPU oracle baseline, an end-to-end figure with
+host<->device copies, the SM clocks seen, and the launch count.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+--impl reference times the float64 CPU oracle on the same workload (a bounded
+sample per step) on the host cores.  With N > 1 (torchrun) every rank runs
+its own replica (the path does not shard; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from int4_group_quantized_q4f16_b200 import synth  # noqa: E402
+
+METRIC = "q4 dequant-GEMV effective HBM GB/s & % of B200 peak; us per decode weight pass"
+NOMINAL_HBM_GBS = 8000.0
+WORKLOAD = ("Phi-3-mini decode weight pass, M=1: 32 x (qkv 3072->9216, o 3072->3072, "
+            "gate_up 3072->2x8192 +SiLU*up, down 8192->3072) + LM head 3072->32064 f32+argmax; "
+            "q4 group-32 weights, seed 0")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--layers", type=int, default=32)
+    return p.parse_args()
+
+
+def projections(layers: int):
+    """(layer, Proj) for every launch of the pass, LM head last."""
+    out = [(l, p) for l in range(layers) for p in synth.phi3_mini_layer()]
+    out.append((0, synth.phi3_mini_lm_head()))
+    return out
+
+
+def alg_bytes(p: synth.Proj, M: int = 1) -> int:
+    """Algorithmic bytes of one call: codes + scales + x + outputs."""
+    out_bytes = 4 if p.kind == "lm_head" else 2
+    return p.weight_bytes() + M * p.K * 2 + M * p.n_out * out_bytes + (4 * M if p.kind == "lm_head" else 0)
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int4_group_quantized_q4f16_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi samples (200 ms) during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        mhz, max_mhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                max_mhz = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max_mhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------- distributed ----
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def dist_max(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------- CPU side ----
+def cpu_oracle_sample(seed: int, layers: int, threads: int):
+    """Time the float64 oracle on `layers` full layers of the pass (all four
+    projections each).  Returns (algorithmic bytes, seconds)."""
+    import oracle
+    o = oracle.get()
+    nbytes, secs = 0, 0.0
+    for l in range(layers):
+        for p in synth.phi3_mini_layer():
+            qw, s, x = synth.proj_inputs(seed, l, p)
+            t0 = time.perf_counter()
+            if p.kind == "gemv":
+                o.gemv(qw, s, x, threads=threads)
+            else:
+                o.gate_up_silu(qw, s, x, threads=threads)
+            secs += time.perf_counter() - t0
+            nbytes += alg_bytes(p)
+    return nbytes, secs
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step = one layer of the pass on
+    the host cores (a bounded sample of the same workload)."""
+    if rank != 0:
+        return
+    cores = host_cores()
+    for _ in range(args.warmup):
+        cpu_oracle_sample(args.seed, 1, cores)
+    nbytes, secs = 0, 0.0
+    for _ in range(args.steps):
+        b, s = cpu_oracle_sample(args.seed, 1, cores)
+        nbytes += b
+        secs += s
+    gbs = nbytes / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_per_step": "layer 0: qkv, o, gate_up+SiLU, down (63.8 MB)"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "one Phi-3-mini layer (4 projections, 63.8 MB of q4 weights) per step"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU side ----
+def build_pass(args, device):
+    """Allocate the pass on the device: weights, activations, outputs."""
+    import torch
+    calls = []
+    for l, p in projections(args.layers):
+        qw, s, x = synth.proj_inputs(args.seed, l, p)
+        d = {
+            "p": p, "layer": l,
+            "qw": torch.from_numpy(qw.view(np.int32)).to(device),
+            "s": torch.from_numpy(s).to(device),
+            "x": torch.from_numpy(x).to(device),
+        }
+        if p.kind == "lm_head":
+            from int4_group_quantized_q4f16_b200 import zt_q4
+            d["y"] = torch.empty((1, p.n_out), dtype=torch.float32, device=device)
+            d["am"] = torch.empty((1,), dtype=torch.int32, device=device)
+            d["ws"] = torch.empty((zt_q4.lmhead_workspace_bytes(1, p.n_out, p.K),), dtype=torch.uint8,
+                                  device=device)
+        else:
+            d["y"] = torch.empty((1, p.n_out), dtype=torch.float16, device=device)
+        calls.append(d)
+    return calls
+
+
+def launch(zt_q4, d, stream):
+    p = d["p"]
+    if p.kind == "gemv":
+        zt_q4.gemv(d["qw"], d["s"], d["x"], d["y"], stream=stream)
+    elif p.kind == "gate_up":
+        zt_q4.gate_up_silu(d["qw"], d["s"], d["x"], d["y"], stream=stream)
+    else:
+        zt_q4.lmhead_argmax(d["qw"], d["s"], d["x"], d["y"], d["am"], d["ws"], stream=stream)
+
+
+def launches_per_step(calls) -> int:
+    return sum(2 if d["p"].kind == "lm_head" else 1 for d in calls)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from int4_group_quantized_q4f16_b200 import zt_q4
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    calls = build_pass(args, device)
+    total_bytes = sum(alg_bytes(d["p"]) for d in calls)
+    stream = torch.cuda.Stream(device=device)
+
+    # capture the pass once; replays are the steps
+    with torch.cuda.stream(stream):
+        for d in calls:
+            launch(zt_q4, d, stream)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for d in calls:
+                launch(zt_q4, d, stream)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K replays, barrier + sync on both sides ----
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.4)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    clock_info = clocks.stop() if clocks else None
+    ms_max = dist_max(ms, world, device)
+    ms_per_step = ms_max / args.steps
+    value = total_bytes * world * args.steps / (ms_max / 1e3) / 1e9
+
+    # ---- per-launch durations of the dominant kernel (same stream) ----
+    evs = []
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for d in calls:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                launch(zt_q4, d, stream)
+                b.record(stream)
+                evs.append((d, a, b))
+    torch.cuda.synchronize()
+    proj = [(alg_bytes(d["p"]), a.elapsed_time(b)) for d, a, b in evs if d["p"].kind != "lm_head"]
+    kb = sum(x for x, _ in proj) / len(proj)
+    kms = sum(t for _, t in proj) / len(proj)
+    achieved = kb / (kms / 1e3) / 1e9
+    per_kind = {}
+    for d, a, b in evs:
+        per_kind.setdefault(d["p"].name, []).append(a.elapsed_time(b) * 1e3)
+    per_kind_us = {k: round(sum(v) / len(v), 3) for k, v in per_kind.items()}
+
+    # ---- end to end through the public API: H2D x, pass, D2H outputs ----
+    xs_host = [torch.empty_like(d["x"], device="cpu").pin_memory() for d in calls]
+    for h, d in zip(xs_host, calls):
+        h.copy_(d["x"].cpu())
+    ys_host = [torch.empty_like(d["y"], device="cpu").pin_memory() for d in calls]
+    am_host = torch.empty((1,), dtype=torch.int32).pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h in xs_host)
+    d2h = sum(h.numel() * h.element_size() for h in ys_host) + 4
+
+    def e2e_step():
+        for h, d in zip(xs_host, calls):
+            d["x"].copy_(h, non_blocking=True)
+        graph.replay()
+        for h, d in zip(ys_host, calls):
+            h.copy_(d["y"], non_blocking=True)
+        am_host.copy_(calls[-1]["am"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        dist_barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world, device)
+    e2e_value = total_bytes * world * args.steps / (e2e_ms / 1e3) / 1e9
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1:
+        cores = host_cores()
+        nb, secs = cpu_oracle_sample(args.seed, 4, cores)
+        cpu = {"value": round(nb / secs / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"layers 0-3 of the pass (16 projections, {nb / 1e6:.1f} MB), float64 oracle, "
+                         f"OpenMP over rows, {secs:.1f} s"}
+
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peaks = json.load(fh)
+    except (OSError, ValueError):
+        pass
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "q4_mma_traffic.json")) as fh:
+            tr = json.load(fh)
+        if tr.get("kernel_sources_sha") == kernel_sources_sha():
+            traffic = round(tr["dram_bytes_per_algorithmic_byte"] * kb)
+    except (OSError, ValueError, KeyError):
+        pass
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16xf16->f32 (int4 codes, fp16 scales)",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 1, "layers": args.layers, "launches_per_step": launches_per_step(calls),
+                       "bytes_per_step": total_bytes, "l2": "inputs larger than L2 (2.1 GB per step, L2 126 MB)",
+                       "parallelism": f"replicas x{world}"},
+            "us_per_pass": round(ms_per_step * 1e3, 2),
+            "pct_of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS * 100, 2),
+            "pct_of_measured_peak": round(value / world / peak * 100, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "kernel": "q4_mma_kernel (128 projection launches per step)",
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                         else "fallback 6.65 TB/s",
+                         "bytes_per_launch": round(kb), "us_per_launch": round(kms * 1e3, 3)},
+            "per_projection_us": per_kind_us,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step(calls) * args.steps,
+            "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    graph.reset()
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
