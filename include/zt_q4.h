@@ -120,6 +120,30 @@ ZT_API int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const
                         int M, int N, int K, void *stream);
 
 /*
+ * zt_q4_lmhead_argmax without a caller-supplied workspace, for callers that
+ * cannot allocate device memory: a plug-in running inside a host framework
+ * that owns every device allocation, code being recorded into a CUDA graph
+ * (where cudaMalloc is not allowed), or a latency-critical decode loop that
+ * must not allocate (cudaMalloc can synchronize the device).  There is no
+ * counterpart on the pages; it is an interface convenience of this library.
+ *
+ * Same arguments, results and checks as zt_q4_lmhead_argmax, minus the
+ * workspace: the per-CTA maxima go to one static 512 KiB device array inside
+ * the library (enough for every legal shape, M <= 16; a shape needing more
+ * would return ZT_ERR_WORKSPACE).  Every GPU that loads the library holds that
+ * array until the process exits.  Allocates nothing: no cudaMalloc/cudaFree.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call on a device shares the array.  Calls whose kernels can
+ *     overlap on the GPU (different streams without ordering) race on it and
+ *     give wrong argmax; serialize them (one stream, or events).
+ *   - Nothing in the array needs to start at zero: each call writes every
+ *     entry it later reads.
+ */
+ZT_API int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                                       float *logits, int32_t *argmax, int M, int N, int K, void *stream);
+
+/*
  * Host-side layout helpers (HOST pointers, synchronous, no CUDA calls).
  * pack:   q uint8 [N][K] codes 0..15  ->  qw uint32 [N][K/8], low nibble first.
  *         A code above 15 is ZT_ERR_INVALID_ARG (qw is then unspecified).

@@ -324,6 +324,37 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
 
 size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + sizeof(int)); }
 
+// Scratch of zt_q4_lmhead_argmax_noalloc: one per device, for the whole life
+// of the library.  Sized for the largest LM-head workspace (M = 16).
+constexpr size_t kNoAllocScratchBytes = (size_t)kMaxCtas * 16 * (sizeof(float) + sizeof(int));   // 512 KiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::unordered_map<int, void *> g_noalloc_ptr;   // device -> device address of g_noalloc_scratch
+
+// Device address of the scratch array on the current device, looked up once
+// per device (a host-side `g_noalloc_scratch` is only a stand-in, not a device
+// address, so it must never be passed to a kernel directly).
+void *noalloc_scratch()
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_noalloc_ptr.find(dev);
+    if (it != g_noalloc_ptr.end()) return it->second;
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    g_noalloc_ptr.emplace(dev, ptr);
+    return ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -409,6 +440,18 @@ int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16
         return ZT_ERR_LAUNCH;
     }
     return ZT_OK;
+}
+
+int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, float *logits,
+                                int32_t *argmax, int M, int N, int K, void *stream)
+{
+    if (!qw || !scales || !x || !logits || !argmax) return ZT_ERR_INVALID_ARG;
+    const int rc = check_shapes(M, N, K, 1);
+    if (rc) return rc;
+    if (lmhead_ws_bytes(M) > kNoAllocScratchBytes) return ZT_ERR_WORKSPACE;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return ZT_ERR_DEVICE;
+    return zt_q4_lmhead_argmax(qw, scales, x, logits, argmax, scratch, kNoAllocScratchBytes, M, N, K, stream);
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)

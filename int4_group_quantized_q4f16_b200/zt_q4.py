@@ -46,6 +46,8 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_lmhead_workspace_bytes.argtypes = [_I, _I, _I]
     lib.zt_q4_lmhead_workspace_bytes.restype = ctypes.c_size_t
     lib.zt_q4_lmhead_argmax.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _P]
+    lib.zt_q4_lmhead_argmax_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _P]
+    lib.zt_q4_lmhead_argmax_noalloc.restype = ctypes.c_int
     lib.zt_q4_pack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_unpack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_strerror.argtypes = [_I]
@@ -165,4 +167,19 @@ def lmhead_argmax(qw, scales, x, logits=None, argmax=None, workspace=None, strea
     _check(lib.zt_q4_lmhead_argmax(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), logits.data_ptr(),
                                    argmax.data_ptr(), workspace.data_ptr(), workspace.numel(),
                                    M, N, K, _stream_handle(stream)), "zt_q4_lmhead_argmax")
+    return logits, argmax
+
+
+def lmhead_argmax_noalloc(qw, scales, x, logits=None, argmax=None, stream=None):
+    """lmhead_argmax through the entry point that allocates no device memory
+    (its scratch is a static array in the library; see include/zt_q4.h)."""
+    torch = _torch()
+    M, N, K = _dims(qw, scales, x, 1)
+    if logits is None:
+        logits = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    if argmax is None:
+        argmax = torch.empty((M,), dtype=torch.int32, device=x.device)
+    _check(lib.zt_q4_lmhead_argmax_noalloc(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), logits.data_ptr(),
+                                           argmax.data_ptr(), M, N, K, _stream_handle(stream)),
+           "zt_q4_lmhead_argmax_noalloc")
     return logits, argmax
