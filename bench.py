@@ -322,12 +322,16 @@ def run_ours(args, world, rank, local):
     value = total_bytes * world * args.steps / (ms_max / 1e3) / 1e9
 
     # ---- per-launch durations of the dominant kernel (same stream) ----
-    # A second graph brackets every launch with timing events (which also
-    # keeps consecutive launches from overlapping), replayed twice.
+    # Each launch is bracketed by timing events (which also keeps consecutive
+    # launches from overlapping).  A fixed-length GPU delay is queued first so
+    # that the host has enqueued the whole pass before the GPU reaches it: the
+    # events then time kernels, not host launch latency.
+    per = {}
     evs = []
     with torch.cuda.stream(stream):
-        tgraph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(tgraph, stream=stream):
+        for rep in range(3):
+            torch.cuda._sleep(40_000_000)
+            evs = []
             for d in calls:
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
@@ -335,11 +339,6 @@ def run_ours(args, world, rank, local):
                 launch(zt_q4, d, stream)
                 b.record(stream)
                 evs.append((d, a, b))
-        tgraph.replay()
-        stream.synchronize()
-        per = {}
-        for _ in range(3):
-            tgraph.replay()
             stream.synchronize()
             for i, (d, a, b) in enumerate(evs):
                 per.setdefault(i, []).append(a.elapsed_time(b))
@@ -351,7 +350,6 @@ def run_ours(args, world, rank, local):
     for i, (d, _, _) in enumerate(evs):
         per_kind.setdefault(d["p"].name, []).append(statistics.median(per[i]) * 1e3)
     per_kind_us = {k: round(sum(v) / len(v), 3) for k, v in per_kind.items()}
-    tgraph.reset()
 
     # ---- end to end through the public API: H2D x, pass, D2H outputs ----
     x_host = xbuf.cpu().pin_memory()
