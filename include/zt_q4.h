@@ -144,6 +144,54 @@ ZT_API int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scale
                                        float *logits, int32_t *argmax, int M, int N, int K, void *stream);
 
 /*
+ * A DECODE WEIGHT PASS in one launch: a list of projections run in order by one
+ * persistent kernel (Zero-TVM write-up, "完整的推理流水线": per decoder layer the
+ * QKV, output, fused FFN and down projections, then the f32 LM head; this is
+ * that sequence of int4 dequantizing products with the weights streamed back to
+ * back).  Each projection computes exactly what the single-call entry point of
+ * its kind computes (zt_q4_gemv, zt_q4_gate_up_silu, zt_q4_lmhead_argmax), with
+ * the same arguments and the same checks; M (tokens, 1..16) is shared.
+ *
+ * Ordering: a projection with `wait` != 0 reads its x only after every earlier
+ * projection of the list has completed on the whole GPU (so x may be an earlier
+ * projection's output); without `wait`, x must not be written by the list.  A
+ * projection that writes a buffer an earlier projection reads needs `wait` too.
+ * The weights of later projections stream while earlier ones compute.
+ *
+ * `wait` on any projection makes the launch cooperative (all CTAs resident);
+ * the wait is bounded: after 2 s a CTA records bit 1 in the error word, stops
+ * and exits (outputs are then incomplete); read it with zt_q4_pass_errors.
+ *
+ * workspace: device memory, 16-byte aligned, at least
+ * zt_q4_pass_workspace_bytes(projs, n, M) bytes: barrier counters, the error
+ * word, and the per-CTA maxima of each LM head.  Its contents on entry do not
+ * matter (the call clears what it needs on `stream`).  Launches: one pass
+ * kernel, plus one argmax reduction per LM-head projection.
+ * projs is a HOST array of n entries (1..ZT_Q4_PASS_MAX), read during the call.
+ */
+#define ZT_Q4_GEMV 0
+#define ZT_Q4_GATE_UP_SILU 1
+#define ZT_Q4_LM_HEAD 2
+#define ZT_Q4_PASS_MAX 160
+
+typedef struct zt_q4_proj {
+    const uint32_t *qw;       /* [n_rows][K/8], n_rows = N (2N for GATE_UP_SILU) */
+    const uint16_t *scales;   /* [n_rows][K/32] fp16 */
+    const uint16_t *x;        /* [M][K] fp16 */
+    void *out;                /* fp16 [M][N], or f32 [M][N] logits for LM_HEAD */
+    int32_t *argmax;          /* LM_HEAD: [M]; ignored otherwise */
+    int kind;                 /* ZT_Q4_GEMV, ZT_Q4_GATE_UP_SILU or ZT_Q4_LM_HEAD */
+    int N, K;
+    int wait;                 /* read x only after all earlier projections completed */
+} zt_q4_proj;
+
+ZT_API size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M);
+ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronous read of a finished pass's error word (0: no bounded wait expired). */
+ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
+
+/*
  * Host-side layout helpers (HOST pointers, synchronous, no CUDA calls).
  * pack:   q uint8 [N][K] codes 0..15  ->  qw uint32 [N][K/8], low nibble first.
  *         A code above 15 is ZT_ERR_INVALID_ARG (qw is then unspecified).

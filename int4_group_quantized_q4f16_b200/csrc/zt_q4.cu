@@ -14,6 +14,7 @@
 #include "q4_gemv.cuh"
 #include "q4_stream.cuh"
 #include "q4_mma.cuh"
+#include "q4_pass.cuh"
 #include "zt_q4.h"
 
 namespace {
@@ -220,40 +221,46 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
     return ZT_ERR_UNSUPPORTED;
 }
 
-// Launch the tensor-core kernel; ZT_ERR_UNSUPPORTED if its rings and staged
-// activations do not fit in shared memory.
-template <int NT, int EPI>
-int launch_mma(const Q4Args &q, cudaStream_t st, int *grid_out)
+// Fill the per-projection launch fields that depend on the grid.
+void pass_fill(PassArgs &a, int grid, int NT, int &red_floats_max)
 {
-    constexpr int ROUT = (EPI == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;
-    const void *fn = reinterpret_cast<const void *>(&q4_mma_kernel<NT, EPI>);
+    red_floats_max = 0;
+    for (int i = 0; i < a.n; ++i) {
+        PassProj &p = a.p[i];
+        const int rout = (p.kind == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;
+        const int rows_max = (p.N + grid - 1) / grid;
+        p.max_tiles = (rows_max + rout - 1) / rout;
+        p.wk = pick_wk(p.max_tiles, (p.G + kMChunkG - 1) / kMChunkG);
+        const int red = p.wk > 1 ? p.max_tiles * p.wk * kMTileRows * 8 * NT : 0;
+        red_floats_max = std::max(red_floats_max, red);
+    }
+}
+
+// Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
+// some projection waits on earlier ones (all CTAs must be co-resident).
+// ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
+template <int NT>
+int launch_pass(PassArgs &a, bool cooperative, cudaStream_t st, int *grid_out)
+{
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT>);
     int sms = 0;
     if (resident_ctas(fn, kMThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
-    MmaArgs a;
-    a.qw = q.qw;
-    a.scales = q.scales;
-    a.x = q.x;
-    a.out = q.out;
-    a.ws_val = q.ws_val;
-    a.ws_idx = q.ws_idx;
-    a.M = q.M;
-    a.N = q.N;
-    a.K = q.K;
-    a.G = q.G;
-    a.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
-    const int n_chunks = (q.G + kMChunkG - 1) / kMChunkG;
+    a.g_max = 0;
+    for (int i = 0; i < a.n; ++i) a.g_max = std::max(a.g_max, a.p[i].G);
+    int min_n = a.p[0].N;
+    for (int i = 1; i < a.n; ++i) min_n = std::min(min_n, a.p[i].N);
     for (int cps = 2; cps >= 1; --cps) {
-        const int grid = std::max(1, std::min({sms * cps, q.N, kMaxCtas}));
-        const int rows_max = (q.N + grid - 1) / grid;
-        a.max_tiles = (rows_max + ROUT - 1) / ROUT;
-        a.wk = pick_wk(a.max_tiles, n_chunks);
-        const size_t fixed = mma_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, NT);
+        const int grid = std::max(1, std::min({sms * cps, cooperative ? sms * cps : min_n, kMaxCtas}));
+        int red_floats = 0;
+        pass_fill(a, grid, NT, red_floats);
+        a.red_floats = red_floats;
+        const size_t fixed = pass_smem_bytes(a.M, a.g_max, 0, red_floats, NT);
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const size_t per_stage = (size_t)kMW * kMStage;
         const int stages = budget > fixed ? (int)std::min<size_t>(kMMaxStages, (budget - fixed) / per_stage) : 0;
         if (stages < 2) continue;
         a.stages = stages;
-        const size_t smem = mma_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, NT);
+        const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, red_floats, NT);
         const int occ = resident_ctas(fn, kMThreads, smem, sms);
         if (occ < cps) continue;
         if (grid_out) *grid_out = grid;
@@ -263,12 +270,17 @@ int launch_mma(const Q4Args &q, cudaStream_t st, int *grid_out)
         cfg.dynamicSmemBytes = smem;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        if (cooperative) {
+            attr[0].id = cudaLaunchAttributeCooperative;
+            attr[0].val.cooperative = 1;
+        } else {
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+        }
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         clear_stale_error();
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_mma_kernel<NT, EPI>, a);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT>, a);
         if (e != cudaSuccess) {
             g_last_cuda_error = e;
             (void)cudaGetLastError();
@@ -277,6 +289,30 @@ int launch_mma(const Q4Args &q, cudaStream_t st, int *grid_out)
         return ZT_OK;
     }
     return ZT_ERR_UNSUPPORTED;
+}
+
+// One projection through the pass kernel (no waits, launched with PDL).
+int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out)
+{
+    static thread_local PassArgs a;    // ~13 KB: kept off the stack
+    a.n = 1;
+    a.M = q.M;
+    a.counters = nullptr;
+    a.error = nullptr;
+    PassProj &p = a.p[0];
+    p.qw = q.qw;
+    p.scales = q.scales;
+    p.x = q.x;
+    p.out = q.out;
+    p.ws_val = q.ws_val;
+    p.ws_idx = q.ws_idx;
+    p.N = q.N;
+    p.K = q.K;
+    p.G = q.G;
+    p.kind = kind;
+    p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+    p.wait = 0;
+    return (q.M <= 8) ? launch_pass<1>(a, false, st, grid_out) : launch_pass<2>(a, false, st, grid_out);
 }
 
 template <int EPI>
@@ -298,7 +334,7 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // The tensor-core kernel whenever its rings and activations fit.
     {
-        const int rc = (M <= 8) ? launch_mma<1, EPI>(a, st, grid_out) : launch_mma<2, EPI>(a, st, grid_out);
+        const int rc = launch_single_pass(a, EPI, st, grid_out);
         if (rc != ZT_ERR_UNSUPPORTED) return rc;
     }
     // Small batch: the CUDA-core streaming kernel when its ring fits.
@@ -452,6 +488,118 @@ int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scales, cons
     void *scratch = noalloc_scratch();
     if (!scratch) return ZT_ERR_DEVICE;
     return zt_q4_lmhead_argmax(qw, scales, x, logits, argmax, scratch, kNoAllocScratchBytes, M, N, K, stream);
+}
+
+static size_t pass_ws_layout(const zt_q4_proj *projs, int n, int M, size_t *err_off, size_t *lm_off)
+{
+    const size_t counters = ((size_t)n * 4 + 15) & ~(size_t)15;
+    if (err_off) *err_off = counters;
+    if (lm_off) *lm_off = counters + 16;
+    size_t bytes = counters + 16;
+    for (int i = 0; i < n; ++i)
+        if (projs[i].kind == ZT_Q4_LM_HEAD) bytes += lmhead_ws_bytes(M);
+    return bytes;
+}
+
+size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M)
+{
+    if (!projs || n < 1 || n > ZT_Q4_PASS_MAX || M < 1 || M > 16) return 0;
+    return pass_ws_layout(projs, n, M, nullptr, nullptr);
+}
+
+int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!projs || !workspace || n < 1 || n > ZT_Q4_PASS_MAX || M < 1 || M > 16) return ZT_ERR_INVALID_ARG;
+    bool cooperative = false;
+    for (int i = 0; i < n; ++i) {
+        const zt_q4_proj &q = projs[i];
+        if (!q.qw || !q.scales || !q.x || !q.out) return ZT_ERR_INVALID_ARG;
+        if (q.kind != ZT_Q4_GEMV && q.kind != ZT_Q4_GATE_UP_SILU && q.kind != ZT_Q4_LM_HEAD) return ZT_ERR_INVALID_ARG;
+        if (q.kind == ZT_Q4_LM_HEAD && !q.argmax) return ZT_ERR_INVALID_ARG;
+        const int rc = check_shapes(M, q.N, q.K, q.kind == ZT_Q4_GATE_UP_SILU ? 2 : 1);
+        if (rc) return rc;
+        if (!aligned(q.qw, 16) || !aligned(q.x, 16) || !aligned(q.scales, 2) ||
+            !aligned(q.out, q.kind == ZT_Q4_LM_HEAD ? 4 : 2) || (q.argmax && !aligned(q.argmax, 4)))
+            return ZT_ERR_MISALIGNED;
+        if (i > 0 && q.wait) cooperative = true;
+    }
+    if (!aligned(workspace, 16)) return ZT_ERR_MISALIGNED;
+    size_t err_off = 0, lm_off = 0;
+    if (ws_bytes < pass_ws_layout(projs, n, M, &err_off, &lm_off)) return ZT_ERR_WORKSPACE;
+
+    static thread_local PassArgs a;    // ~13 KB: kept off the stack
+    unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
+    a.n = n;
+    a.M = M;
+    a.counters = cooperative ? reinterpret_cast<unsigned int *>(ws) : nullptr;
+    a.error = reinterpret_cast<unsigned int *>(ws + err_off);
+    size_t lm = lm_off;
+    for (int i = 0; i < n; ++i) {
+        const zt_q4_proj &q = projs[i];
+        PassProj &p = a.p[i];
+        p.qw = reinterpret_cast<const uint4 *>(q.qw);
+        p.scales = reinterpret_cast<const __half *>(q.scales);
+        p.x = reinterpret_cast<const __half *>(q.x);
+        p.out = q.out;
+        p.N = q.N;
+        p.K = q.K;
+        p.G = q.K / kGroup;
+        p.kind = q.kind == ZT_Q4_GEMV ? kEpiF16 : q.kind == ZT_Q4_GATE_UP_SILU ? kEpiGateUp : kEpiLogits;
+        p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+        p.wait = (i > 0 && q.wait) ? 1 : 0;
+        p.ws_val = nullptr;
+        p.ws_idx = nullptr;
+        if (q.kind == ZT_Q4_LM_HEAD) {
+            p.ws_val = reinterpret_cast<float *>(ws + lm);
+            p.ws_idx = reinterpret_cast<int *>(ws + lm) + (size_t)kMaxCtas * M;
+            lm += lmhead_ws_bytes(M);
+        }
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    clear_stale_error();
+    cudaError_t e = cudaMemsetAsync(ws, 0, err_off + 16, st);   // counters + error bits
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    int grid = 0;
+    const int rc = (M <= 8) ? launch_pass<1>(a, cooperative, st, &grid) : launch_pass<2>(a, cooperative, st, &grid);
+    if (rc) return rc;
+    for (int i = 0; i < n; ++i) {
+        if (projs[i].kind != ZT_Q4_LM_HEAD) continue;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(M);
+        cfg.blockDim = dim3(256);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, q4_argmax_reduce_kernel, (const float *)a.p[i].ws_val,
+                               (const int *)a.p[i].ws_idx, grid, M, projs[i].argmax);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = e;
+            (void)cudaGetLastError();
+            return ZT_ERR_LAUNCH;
+        }
+    }
+    return ZT_OK;
+}
+
+int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out)
+{
+    if (!workspace || !out || n < 1 || n > ZT_Q4_PASS_MAX) return ZT_ERR_INVALID_ARG;
+    const size_t err_off = ((size_t)n * 4 + 15) & ~(size_t)15;
+    const cudaError_t e = cudaMemcpy(out, reinterpret_cast<const unsigned char *>(workspace) + err_off,
+                                     sizeof(unsigned int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_DEVICE;
+    }
+    return ZT_OK;
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)

@@ -35,6 +35,19 @@ class ZtError(RuntimeError):
         super().__init__(f"{what}: status {status}: {strerror(status)}" + (f" [{cuda}]" if cuda else ""))
 
 
+ZT_Q4_GEMV = 0
+ZT_Q4_GATE_UP_SILU = 1
+ZT_Q4_LM_HEAD = 2
+ZT_Q4_PASS_MAX = 160
+
+
+class ZtProj(ctypes.Structure):
+    """struct zt_q4_proj of include/zt_q4.h"""
+    _fields_ = [("qw", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("argmax", ctypes.c_void_p), ("kind", ctypes.c_int),
+                ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -48,6 +61,12 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_lmhead_argmax.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _P]
     lib.zt_q4_lmhead_argmax_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _P]
     lib.zt_q4_lmhead_argmax_noalloc.restype = ctypes.c_int
+    lib.zt_q4_pass_workspace_bytes.argtypes = [ctypes.POINTER(ZtProj), _I, _I]
+    lib.zt_q4_pass_workspace_bytes.restype = ctypes.c_size_t
+    lib.zt_q4_pass.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
+    lib.zt_q4_pass.restype = ctypes.c_int
+    lib.zt_q4_pass_errors.argtypes = [_P, _I, ctypes.POINTER(ctypes.c_uint)]
+    lib.zt_q4_pass_errors.restype = ctypes.c_int
     lib.zt_q4_pack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_unpack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_strerror.argtypes = [_I]
@@ -183,3 +202,46 @@ def lmhead_argmax_noalloc(qw, scales, x, logits=None, argmax=None, stream=None):
                                            argmax.data_ptr(), M, N, K, _stream_handle(stream)),
            "zt_q4_lmhead_argmax_noalloc")
     return logits, argmax
+
+
+class Pass:
+    """A decode weight pass: a list of projections run by one persistent kernel.
+
+    Each entry is a dict with torch CUDA tensors: kind ("gemv", "gate_up",
+    "lm_head"), qw, scales, x, out (and argmax for "lm_head"), and optional
+    wait (read x only after all earlier projections completed).  The
+    ctypes array and the workspace are built once; run() only launches."""
+
+    KINDS = {"gemv": ZT_Q4_GEMV, "gate_up": ZT_Q4_GATE_UP_SILU, "lm_head": ZT_Q4_LM_HEAD}
+
+    def __init__(self, projs, workspace=None):
+        torch = _torch()
+        if not 1 <= len(projs) <= ZT_Q4_PASS_MAX:
+            raise ValueError(f"a pass has 1..{ZT_Q4_PASS_MAX} projections")
+        self._keep = projs
+        arr = (ZtProj * len(projs))()
+        M = None
+        for i, p in enumerate(projs):
+            kind = self.KINDS[p["kind"]]
+            m, n, k = _dims(p["qw"], p["scales"], p["x"], 2 if kind == ZT_Q4_GATE_UP_SILU else 1)
+            if M is None:
+                M = m
+            elif m != M:
+                raise ValueError("all projections of a pass share M")
+            am = p.get("argmax")
+            arr[i] = ZtProj(p["qw"].data_ptr(), p["scales"].data_ptr(), p["x"].data_ptr(), p["out"].data_ptr(),
+                            am.data_ptr() if am is not None else None, kind, n, k, int(bool(p.get("wait", 0))))
+        self.arr, self.n, self.M = arr, len(projs), M
+        nbytes = int(lib.zt_q4_pass_workspace_bytes(arr, self.n, M))
+        if workspace is None:
+            workspace = torch.empty((nbytes,), dtype=torch.uint8, device=projs[0]["x"].device)
+        self.workspace = workspace
+
+    def run(self, stream=None):
+        _check(lib.zt_q4_pass(self.arr, self.n, self.M, self.workspace.data_ptr(), self.workspace.numel(),
+                              _stream_handle(stream)), "zt_q4_pass")
+
+    def errors(self) -> int:
+        v = ctypes.c_uint(0)
+        _check(lib.zt_q4_pass_errors(self.workspace.data_ptr(), self.n, ctypes.byref(v)), "zt_q4_pass_errors")
+        return int(v.value)

@@ -115,3 +115,29 @@ def test_pack_host_rejects_codes_above_15(zt):
         zt.pack_host(q)
     rc = zt.lib.zt_q4_pack_host(None, 2, 16, None)
     assert rc == zt.ZT_ERR_INVALID_ARG
+
+
+def test_pass_arguments_rejected(zt):
+    P = zt.ZtProj
+    ok = P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0)
+    arr = (P * 1)(ok)
+    ws = zt.lib.zt_q4_pass_workspace_bytes(arr, 1, 1)
+    assert ws > 0
+    f = zt.lib.zt_q4_pass
+    assert f(None, 1, 1, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(arr, 0, 1, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(arr, zt.ZT_Q4_PASS_MAX + 1, 1, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(arr, 1, 17, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(arr, 1, 1, None, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(arr, 1, 1, FAKE, ws - 1, None) == zt.ZT_ERR_WORKSPACE
+    assert f(arr, 1, 1, FAKE + 8, ws, None) == zt.ZT_ERR_MISALIGNED
+    for bad in (P(FAKE, FAKE, FAKE, FAKE, None, 7, 64, 64, 0),              # unknown kind
+                P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_LM_HEAD, 64, 64, 0),  # LM head without argmax
+                P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 48, 0),     # K % 32
+                P(None, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0)):
+        assert f((P * 2)(ok, bad), 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG
+    mis = P(FAKE, FAKE, FAKE + 8, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0)
+    assert f((P * 1)(mis), 1, 1, FAKE, ws, None) == zt.ZT_ERR_MISALIGNED
+    lm = P(FAKE, FAKE, FAKE, FAKE, FAKE, zt.ZT_Q4_LM_HEAD, 64, 64, 0)
+    assert zt.lib.zt_q4_pass_workspace_bytes((P * 2)(ok, lm), 2, 1) > ws
+    assert zt.lib.zt_q4_pass_errors(None, 1, None) == zt.ZT_ERR_INVALID_ARG

@@ -1,0 +1,112 @@
+"""GPU parity of the one-launch decode weight pass (zt_q4_pass) against the
+oracle, element by element, on independent and on chained projection lists."""
+import numpy as np
+import pytest
+
+from int4_group_quantized_q4f16_b200 import synth
+from parity import (abs_products, assert_f16_matches, assert_f32_matches, check_argmax, dev, host)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def zt():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    return zt_q4
+
+
+def _proj(kind, N, K, M, seed, proj_id):
+    import torch
+    rows = 2 * N if kind == "gate_up" else N
+    qw, s, x = synth.problem(seed, rows, K, M=M, proj=proj_id)
+    d = {"kind": kind, "qw": dev(qw), "scales": dev(s), "x": dev(x), "host": (qw, s, x), "N": N}
+    if kind == "lm_head":
+        d["out"] = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        d["argmax"] = torch.empty((M,), dtype=torch.int32, device="cuda")
+    else:
+        d["out"] = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    return d
+
+
+def _check_against_oracle(oracle, d, x_host=None):
+    qw, s, x = d["host"]
+    if x_host is not None:
+        x = x_host
+    got = host(d["out"])
+    if d["kind"] == "gemv":
+        assert_f16_matches(got, oracle.gemv(qw, s, x, threads=8), "pass gemv", abs_products(oracle, qw, s, x))
+    elif d["kind"] == "gate_up":
+        ref = oracle.gate_up_silu(qw, s, x, threads=8)
+        N = d["N"]
+        rows = np.arange(N, dtype=np.int32)
+        g = oracle.gemv(qw, s, x, rows=rows, threads=8)
+        u = oracle.gemv(qw, s, x, rows=rows + N, threads=8)
+        eg = 2.0 ** -14 * abs_products(oracle, qw, s, x, rows=rows)
+        eu = 2.0 ** -14 * abs_products(oracle, qw, s, x, rows=rows + N)
+        silu = g / (1.0 + np.exp(-g))
+        bound = (1.1 * eg * np.abs(u) + np.abs(silu) * eu + eg * eu) / 2.0 ** -14
+        assert_f16_matches(got, ref, "pass gate_up", bound)
+    else:
+        ref, _ = oracle.lmhead_argmax(qw, s, x, threads=8)
+        assert_f32_matches(got, ref, "pass lm head")
+        check_argmax(host(d["argmax"]), ref)
+
+
+@pytest.mark.parametrize("M", [1, 3, 12])
+def test_pass_independent_mixed(zt, oracle, M):
+    """qkv/o/gate_up/down-like projections of two layers + an LM head, no waits."""
+    import torch
+    shapes = [("gemv", 640, 1024), ("gemv", 300, 1024), ("gate_up", 512, 1024), ("gemv", 256, 2048),
+              ("gemv", 700, 512), ("gate_up", 96, 256), ("lm_head", 3000, 1024)]
+    projs = [_proj(k, N, K, M, 11 + i, i) for i, (k, N, K) in enumerate(shapes)]
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for d in projs:
+        _check_against_oracle(oracle, d)
+    # a second run of the same pass gives identical results
+    before = [host(d["out"]).copy() for d in projs]
+    p.run()
+    torch.cuda.synchronize()
+    for b, d in zip(before, projs):
+        assert np.array_equal(b.view(np.uint8), host(d["out"]).view(np.uint8))
+
+
+def test_pass_chained_waits(zt, oracle):
+    """x of projection i+1 is the output of projection i (wait set): every
+    stage is checked against the oracle on the stage's actual input."""
+    import torch
+    M = 2
+    dims = [1024, 2048, 512, 1024, 3072, 256]
+    projs = []
+    for i in range(len(dims) - 1):
+        d = _proj("gemv", dims[i + 1], dims[i], M, 40 + i, i)
+        projs.append(d)
+    gu = _proj("gate_up", 1024, dims[-1], M, 60, 9)
+    projs.append(gu)
+    lm = _proj("lm_head", 5000, 1024, M, 61, 10)
+    projs.append(lm)
+    for i in range(1, len(projs)):
+        projs[i]["x"] = projs[i - 1]["out"]
+        projs[i]["wait"] = 1
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    _check_against_oracle(oracle, projs[0])
+    for i in range(1, len(projs)):
+        _check_against_oracle(oracle, projs[i], x_host=host(projs[i - 1]["out"]).astype(np.float16))
+
+
+def test_pass_matches_single_calls(zt):
+    """One projection through the pass equals the single-call entry point bit for bit."""
+    import torch
+    d = _proj("gemv", 4097, 3072, 1, 5, 0)
+    zt.Pass([d]).run()
+    single = zt.gemv(d["qw"], d["scales"], d["x"])
+    torch.cuda.synchronize()
+    assert np.array_equal(host(d["out"]).view(np.uint16), host(single).view(np.uint16))
