@@ -48,13 +48,16 @@ struct PassProj {
     int wait;                   // wait for all earlier projections before reading x
 };
 
+// PMAX bounds the list: 1 for the single-call entry points (a small kernel
+// parameter block), kPassMax for zt_q4_pass.
+template <int PMAX>
 struct PassArgs {
     int n, M, stages;
     int g_max;                  // largest G of the list (sizes the activation area)
     int red_floats;             // largest WK partial buffer of the list
     unsigned int *counters;     // [n], zero at launch (needed only when some wait != 0)
     unsigned int *error;        // error bits
-    PassProj p[kPassMax];
+    PassProj p[PMAX];
 };
 
 __host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int red_floats, int NT)
@@ -127,8 +130,8 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *counter, unsign
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs a)
+template <int NT, int PMAX>
+__global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int M = a.M, S = a.stages;

@@ -222,7 +222,8 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
 }
 
 // Fill the per-projection launch fields that depend on the grid.
-void pass_fill(PassArgs &a, int grid, int NT, int &red_floats_max)
+template <int PMAX>
+void pass_fill(PassArgs<PMAX> &a, int grid, int NT, int &red_floats_max)
 {
     red_floats_max = 0;
     for (int i = 0; i < a.n; ++i) {
@@ -239,10 +240,10 @@ void pass_fill(PassArgs &a, int grid, int NT, int &red_floats_max)
 // Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
 // some projection waits on earlier ones (all CTAs must be co-resident).
 // ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
-template <int NT>
-int launch_pass(PassArgs &a, bool cooperative, cudaStream_t st, int *grid_out)
+template <int NT, int PMAX>
+int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_out)
 {
-    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT>);
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX>);
     int sms = 0;
     if (resident_ctas(fn, kMThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
     a.g_max = 0;
@@ -280,7 +281,7 @@ int launch_pass(PassArgs &a, bool cooperative, cudaStream_t st, int *grid_out)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         clear_stale_error();
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT>, a);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX>, a);
         if (e != cudaSuccess) {
             g_last_cuda_error = e;
             (void)cudaGetLastError();
@@ -294,7 +295,7 @@ int launch_pass(PassArgs &a, bool cooperative, cudaStream_t st, int *grid_out)
 // One projection through the pass kernel (no waits, launched with PDL).
 int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out)
 {
-    static thread_local PassArgs a;    // ~13 KB: kept off the stack
+    PassArgs<1> a;
     a.n = 1;
     a.M = q.M;
     a.counters = nullptr;
@@ -312,7 +313,7 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.kind = kind;
     p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
     p.wait = 0;
-    return (q.M <= 8) ? launch_pass<1>(a, false, st, grid_out) : launch_pass<2>(a, false, st, grid_out);
+    return (q.M <= 8) ? launch_pass<1, 1>(a, false, st, grid_out) : launch_pass<2, 1>(a, false, st, grid_out);
 }
 
 template <int EPI>
@@ -527,7 +528,7 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
     size_t err_off = 0, lm_off = 0;
     if (ws_bytes < pass_ws_layout(projs, n, M, &err_off, &lm_off)) return ZT_ERR_WORKSPACE;
 
-    static thread_local PassArgs a;    // ~13 KB: kept off the stack
+    static thread_local PassArgs<kPassMax> a;    // ~13 KB: kept off the stack
     unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
     a.n = n;
     a.M = M;
@@ -564,7 +565,8 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         return ZT_ERR_LAUNCH;
     }
     int grid = 0;
-    const int rc = (M <= 8) ? launch_pass<1>(a, cooperative, st, &grid) : launch_pass<2>(a, cooperative, st, &grid);
+    const int rc = (M <= 8) ? launch_pass<1, kPassMax>(a, cooperative, st, &grid)
+                            : launch_pass<2, kPassMax>(a, cooperative, st, &grid);
     if (rc) return rc;
     for (int i = 0; i < n; ++i) {
         if (projs[i].kind != ZT_Q4_LM_HEAD) continue;
