@@ -106,52 +106,74 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // step 0 (x[8t], x[8t+4], x[8t+2], x[8t+6]), step 1 (x[8t+1], x[8t+5],
 // x[8t+3], x[8t+7]) / 16 (k relative to 32g).  The C table holds, for each
 // (g, n-tile, quad thread t), (c, c', c, c') with c = -7 X_g 2^-24 of column
-// 8 nt + 2t and c' of the next column (zero for columns >= M).
+// 8 nt + 2t and c' of the next column (zero for columns >= M).  Thread i of
+// the CTA takes 8 activations of one column per round; the 4 threads of a
+// group are adjacent lanes.  Callers synchronise before reading.
+__device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool valid, unsigned char *xp,
+                                            float *x7, size_t nstride, int NT)
+{
+    const __half2 sixteenth = __float2half2_rn(0.0625f);
+    float part = 0.f;
+    if (valid) {
+        const uint32_t v01 = raw.x, v23 = raw.y, v45 = raw.z, v67 = raw.w;   // half pairs
+        uint4 o;
+        o.x = __byte_perm(v01, v45, 0x5410);   // (x0, x4)
+        o.y = __byte_perm(v23, v67, 0x5410);   // (x2, x6)
+        uint32_t h15 = __byte_perm(v01, v45, 0x7632);   // (x1, x5)
+        uint32_t h37 = __byte_perm(v23, v67, 0x7632);   // (x3, x7)
+        __half2 q15 = __hmul2(*reinterpret_cast<__half2 *>(&h15), sixteenth);
+        __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
+        o.z = *reinterpret_cast<uint32_t *>(&q15);
+        o.w = *reinterpret_cast<uint32_t *>(&q37);
+        *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = o;
+        const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(h[j]);
+            v[2 * j] = f.x;
+            v[2 * j + 1] = f.y;
+        }
+        part = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    }
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if (valid && (kk & 3) == 0) {
+        const float c = part * (-7.0f * pow2f(-24));
+        const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+        float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+        cv[e] = c;
+        cv[2 + e] = c;
+    }
+}
+
 __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsigned char *xp, float *x7, int M,
                                             int K, int G, int NT)
 {
-    const int K8 = K >> 3;
+    const int K8 = K >> 3;                     // a multiple of 4: groups never straddle a column
+    const int total = M * K8;
     const size_t nstride = (size_t)G * 64 + 32;
-    const __half2 sixteenth = __float2half2_rn(0.0625f);
-    for (int i = threadIdx.x; i < G * NT * 16; i += kMThreads) x7[i] = 0.f;
-    __syncthreads();
-    for (int m = 0; m < M; ++m) {
-        for (int base = 0; base < K8; base += kMThreads) {
-            const int kk = base + threadIdx.x;      // (g = kk / 4, t = kk % 4)
-            float part = 0.f;
-            if (kk < K8) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(x + (size_t)m * K + 8 * kk);
-                const uint32_t v01 = raw.x, v23 = raw.y, v45 = raw.z, v67 = raw.w;   // half pairs
-                uint4 o;
-                o.x = __byte_perm(v01, v45, 0x5410);   // (x0, x4)
-                o.y = __byte_perm(v23, v67, 0x5410);   // (x2, x6)
-                uint32_t h15 = __byte_perm(v01, v45, 0x7632);   // (x1, x5)
-                uint32_t h37 = __byte_perm(v23, v67, 0x7632);   // (x3, x7)
-                __half2 q15 = __hmul2(*reinterpret_cast<__half2 *>(&h15), sixteenth);
-                __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
-                o.z = *reinterpret_cast<uint32_t *>(&q15);
-                o.w = *reinterpret_cast<uint32_t *>(&q37);
-                *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = o;
-                const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
-                float v[8];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = __half22float2(h[j]);
-                    v[2 * j] = f.x;
-                    v[2 * j + 1] = f.y;
-                }
-                part = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-            }
-            part += __shfl_xor_sync(0xffffffffu, part, 1);
-            part += __shfl_xor_sync(0xffffffffu, part, 2);
-            if (kk < K8 && (kk & 3) == 0) {
-                const float c = part * (-7.0f * pow2f(-24));
-                const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
-                float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
-                cv[e] = c;
-                cv[2 + e] = c;
-            }
-        }
+    // C entries of the padding columns M .. 8 NT - 1 are zero
+    const int pad = 8 * NT - M;
+    for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
+        const int g = j / pad, m = M + (j - (j / pad) * pad);
+        const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+        float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+        cv[e] = 0.f;
+        cv[2 + e] = 0.f;
+    }
+    // two rounds per iteration: both loads in flight before either is used.
+    // L2-coherent loads: x may be an output of an earlier phase of the same launch.
+    for (int base = 0; base < total; base += 2 * kMThreads) {
+        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+        const bool v0 = i0 < total, v1 = i1 < total;
+        const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
+        const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
+        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+        if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * K + 8 * k0));
+        if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * K + 8 * k1));
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT);
+        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT);
     }
 }
 

@@ -9,18 +9,20 @@
 // point of the library runs through this kernel.
 //
 // Why one launch for many projections: each projection streams 5..56 MB,
-// i.e. 1..9 us of HBM time, comparable to what a kernel boundary costs
-// (block launch, ring start-up, activation staging, tail).  Here a CTA stays
-// resident for the whole list: its warps' cp.async streams run straight from
-// one projection's weights into the next one's, so HBM never idles at a
-// projection boundary.  Only the activations of a projection that consumes an
-// earlier projection's output wait, on a grid-wide counter.
+// i.e. 1..9 us of HBM time, comparable to what a boundary costs (activation
+// staging, reductions, tail: ~3 us measured per projection when every CTA
+// takes a slice of every projection).  So the list is cut into PHASES at the
+// projections that must wait for earlier outputs; the projections inside a
+// phase are independent, and their rows, concatenated, are split into one
+// contiguous, byte-balanced range per CTA.  A CTA then meets only the two or
+// three projection boundaries inside its own range, and its warps' cp.async
+// streams run straight from one projection's weights into the next one's --
+// across phase boundaries too, since weights never depend on earlier outputs.
 //
-// Cross-CTA waits: a projection marked `wait` reads its activations only after
-// every CTA has finished every earlier projection (counters[p] counts the CTAs
-// done with projection p; each CTA handles the projections in order).  Such a
-// launch is cooperative (all CTAs co-resident) and the wait is bounded: after
-// 2 s the CTA records an error bit, stops, lets its own copies land and exits.
+// Cross-CTA waits: phase k > 0 starts only when every CTA has finished phase
+// k - 1 (counters[k-1] counts them).  Such a launch is cooperative (all CTAs
+// co-resident) and the wait is bounded: after 2 s the CTA records an error
+// bit, stops, lets its own copies land and exits.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -41,32 +43,45 @@ struct PassProj {
     void *out;                  // fp16 [M][N] (gemv, gate/up) or f32 [M][N] (LM head)
     float *ws_val;              // LM head: per-CTA maximum [gridDim.x][M]
     int *ws_idx;                //          per-CTA arg-max
+    long long base;             // byte offset of the projection's rows within its phase
+    long long phase_bytes;      // HBM bytes of the whole phase
     int N, K, G, kind;          // kind: kEpiF16 / kEpiGateUp / kEpiLogits
-    int wk;                     // warps splitting K (1, 2, 4, 8)
-    int max_tiles;              // tiles of the largest CTA range
+    int row_bytes;              // HBM bytes per output (codes + scales of its weight rows)
     int scales_async;           // scales copied by cp.async (16-byte aligned rows)
-    int wait;                   // wait for all earlier projections before reading x
+    int phase;                  // index of the projection's phase
+    int wait;                   // starts a phase: wait for all earlier projections
 };
 
 // PMAX bounds the list: 1 for the single-call entry points (a small kernel
 // parameter block), kPassMax for zt_q4_pass.
 template <int PMAX>
 struct PassArgs {
-    int n, M, stages;
+    int n, M, stages, phases;
     int g_max;                  // largest G of the list (sizes the activation area)
-    int red_floats;             // largest WK partial buffer of the list
-    unsigned int *counters;     // [n], zero at launch (needed only when some wait != 0)
+    unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
     PassProj p[PMAX];
 };
 
-__host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int red_floats, int NT)
+// WK > 1 partial buffer: at most kRedTiles / NT tiles x WK warps per segment
+constexpr int kRedFloats = 4096;            // 16 KB: (tiles * wk) * 16 rows * 8 NT cols <= this
+
+// One projection's rows in one CTA, with the CTA's warp layout for them.
+struct PassSeg {
+    int p, o_begin, o_end, phase;           // rows [o_begin, o_end) of projection p
+    int n_tiles, n_chunks, wkl, rout;       // warp tiles, K chunks, log2 of the K-splitting warps
+};
+
+// Shared memory per CTA: rings, permuted activations (n-stride G*64 + 32
+// bytes), C-operand table, WK partials, LM-head maxima, segment list, flags.
+__host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int n, int NT)
 {
     const size_t ring = (size_t)kMW * stages * kMStage;
     const size_t xp = (size_t)M * ((size_t)g_max * 64 + 32);
     const size_t x7 = (size_t)g_max * NT * 64;
     const size_t best = (size_t)kMThreads * 2 * NT * 8;
-    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)red_floats * 4 + best + 16;
+    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)kRedFloats * 4 + best + (size_t)n * sizeof(PassSeg) +
+           (kMW + 4) * sizeof(int);
 }
 
 // Per-projection geometry of one warp.
@@ -74,20 +89,43 @@ struct PassGeo {
     int o_begin, o_end, rout, n_tiles, n_chunks, wk, wr_n, my_wk, my_wr, my_tiles, my_chunks, n_items;
 };
 
-__device__ __forceinline__ PassGeo pass_geo(const PassProj &P, int warp)
+static_assert(kMW == 8, "warp layout below assumes 8 warps");
+static_assert(kPassMax <= kMThreads, "one thread per projection builds the segment list");
+
+// log2 of the warps splitting K for a segment: minimise the items of the
+// busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
+// K-warps, with the partial buffer bounded (tiles * WK * 16 * 8 NT <= kRedFloats).
+__device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT)
+{
+    int best = 0, best_cost = -1;
+#pragma unroll
+    for (int wkl = 0; wkl <= 3; ++wkl) {
+        const int wk = 1 << wkl;
+        if (wk > n_chunks) break;
+        if (wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > kRedFloats) break;
+        const int cost = ((n_tiles + (kMW >> wkl) - 1) >> (3 - wkl)) * ((n_chunks + wk - 1) >> wkl);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = wkl;
+        }
+    }
+    return best;
+}
+
+__device__ __forceinline__ PassGeo pass_geo(const PassSeg &sg, int warp)
 {
     PassGeo g;
-    g.o_begin = (int)(((long long)P.N * blockIdx.x) / gridDim.x);
-    g.o_end = (int)(((long long)P.N * (blockIdx.x + 1)) / gridDim.x);
-    g.rout = (P.kind == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;
-    g.n_tiles = (g.o_end - g.o_begin + g.rout - 1) / g.rout;
-    g.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
-    g.wk = P.wk;
-    g.wr_n = kMW / P.wk;
-    g.my_wk = warp % P.wk;
-    g.my_wr = warp / P.wk;
-    g.my_tiles = g.my_wr < g.n_tiles ? (g.n_tiles - g.my_wr + g.wr_n - 1) / g.wr_n : 0;
-    g.my_chunks = g.my_wk < g.n_chunks ? (g.n_chunks - g.my_wk + g.wk - 1) / g.wk : 0;
+    g.o_begin = sg.o_begin;
+    g.o_end = sg.o_end;
+    g.rout = sg.rout;
+    g.n_tiles = sg.n_tiles;
+    g.n_chunks = sg.n_chunks;
+    g.wk = 1 << sg.wkl;
+    g.wr_n = kMW >> sg.wkl;
+    g.my_wk = warp & (g.wk - 1);
+    g.my_wr = warp >> sg.wkl;
+    g.my_tiles = g.my_wr < g.n_tiles ? (g.n_tiles - g.my_wr + g.wr_n - 1) >> (3 - sg.wkl) : 0;
+    g.my_chunks = g.my_wk < g.n_chunks ? (g.n_chunks - g.my_wk + g.wk - 1) >> sg.wkl : 0;
     g.n_items = g.my_tiles * g.my_chunks;
     return g;
 }
@@ -134,7 +172,7 @@ template <int NT, int PMAX>
 __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
-    const int M = a.M, S = a.stages;
+    const int M = a.M, S = a.stages, n = a.n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qg = lane >> 2, qt = lane & 3;       // mma quad row / thread in quad
 
@@ -143,12 +181,63 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const size_t xp_bytes = ((size_t)M * ((size_t)a.g_max * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
     float *red = x7 + (size_t)a.g_max * NT * 16;
-    float *bvs = red + a.red_floats;
+    float *bvs = red + kRedFloats;
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bis + kMThreads * 2 * NT);
+    PassSeg *segs = reinterpret_cast<PassSeg *>(bis + kMThreads * 2 * NT);
+    int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
+    volatile int *abort_flag = wcount + kMW;
 
-    if (tid == 0) *abort_flag = 0;
     pdl_launch_dependents();
+
+    // ---- this CTA's segments: per phase, its byte-balanced share of the
+    //      phase's concatenated rows (a row belongs to the CTA whose share
+    //      holds the row's first byte).  Thread p looks at projection p. ----
+    {
+        PassSeg mine{};
+        bool has = false;
+        if (tid < n) {
+            const PassProj &P = a.p[tid];
+            const long long lo = P.phase_bytes * blockIdx.x / gridDim.x;
+            const long long hi = P.phase_bytes * (blockIdx.x + 1) / gridDim.x;
+            const long long rb = P.row_bytes, end = P.base + (long long)P.N * rb;
+            if (hi > P.base && lo < end) {
+                const int o0 = lo > P.base ? (int)((lo - P.base + rb - 1) / rb) : 0;
+                const int o1 = hi < end ? (int)((hi - P.base + rb - 1) / rb) : P.N;
+                if (o1 > o0) {
+                    has = true;
+                    mine.p = tid;
+                    mine.o_begin = o0;
+                    mine.o_end = o1;
+                    mine.phase = P.phase;
+                    mine.rout = P.kind == kEpiGateUp ? kMTileRows / 2 : kMTileRows;
+                    mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
+                    mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
+                    mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT);
+                }
+            }
+            if (!has && P.kind == kEpiLogits) {
+                // an LM head this CTA has no rows of still gets a (neutral) partial maximum
+                for (int m = 0; m < M; ++m) {
+                    P.ws_val[(size_t)blockIdx.x * M + m] = -INFINITY;
+                    P.ws_idx[(size_t)blockIdx.x * M + m] = 0x7fffffff;
+                }
+            }
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, has);
+        if (lane == 0) wcount[warp] = __popc(ball);
+        if (tid == 0) *abort_flag = 0;
+        __syncthreads();
+        if (has) {
+            int idx = __popc(ball & ((1u << lane) - 1u));
+            for (int w = 0; w < warp; ++w) idx += wcount[w];
+            segs[idx] = mine;
+        }
+    }
+    int nseg = 0;
+#pragma unroll
+    for (int w = 0; w < kMW; ++w) nseg += wcount[w];
+    __syncthreads();
+    const int nphase = a.phases;
 
     // Byte offsets from the start of shared memory; loads index the shared
     // array directly, so the compiler sees shared-space, 32-bit addressing.
@@ -158,21 +247,21 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const uint32_t ring_u = smem_u32(ring);
 
     // ---------------------------------------------------------- issue side --
-    // The warp's items of all projections form one stream (projection, tile,
+    // The warp's items of all segments form one stream (segment, tile,
     // chunk); lane l copies pieces p = l + 32 i (i < 4) of an item: tile row
-    // r = l / 8 + 4 i, group l % 8 of the chunk.
+    // r = l / 8 + 4 i, group l % 8 of the chunk.  It runs ahead of the
+    // compute side by S - 1 items, across segment and phase boundaries.
     const int pg = lane & 7;
     const uint32_t piece_u = ring_u + (lane >> 3) * kMRowStride + pg * 16;   // + stage, + 4 i rows
     const uint32_t scale_u = ring_u + kMScaleOff + lane * 16;
-    int is_p = 0, is_tl = 0, is_cl = 0, is_stage = 0;
-    PassGeo ig = pass_geo(a.p[0], warp);
-    int is_left = ig.n_items;                       // items of projection is_p still to issue
+    int is_s = 0, is_tl = 0, is_cl = 0, is_stage = 0, is_left = 0;
+    PassGeo ig{};
     const uint4 *src_w[4];
     bool ok_w[4];
     const __half *src_s = nullptr;
     bool ok_s = false;
     auto set_tile = [&](int tl) {
-        const PassProj &P = a.p[is_p];
+        const PassProj &P = a.p[segs[is_s].p];
         const int o0 = ig.o_begin + (ig.my_wr + ig.wr_n * tl) * ig.rout;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -185,20 +274,25 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             src_s = P.scales + (size_t)row * P.G;
         }
     };
-    // move the issue pointer to the next projection that has items for this warp
+    // move the issue pointer to the next segment that has items for this warp
     auto advance = [&]() {
-        while (is_left == 0 && ++is_p < a.n) {
-            ig = pass_geo(a.p[is_p], warp);
+        while (is_left == 0 && is_s < nseg) {
+            if (++is_s >= nseg) break;
+            ig = pass_geo(segs[is_s], warp);
             is_tl = is_cl = 0;
             is_left = ig.n_items;
         }
         if (is_left > 0) set_tile(is_tl);
     };
-    if (is_left > 0) set_tile(0);
-    else advance();
+    if (nseg > 0) {
+        ig = pass_geo(segs[0], warp);
+        is_left = ig.n_items;
+        if (is_left > 0) set_tile(0);
+        else advance();
+    }
     auto issue_next = [&]() {
         if (is_left > 0 && !*abort_flag) {
-            const PassProj &P = a.p[is_p];
+            const PassProj &P = a.p[segs[is_s].p];
             const int c = ig.my_wk + ig.wk * is_cl;
             const bool full = (c + 1) * kMChunkG <= P.G;
             const int kc = full ? kMChunkG : P.G - c * kMChunkG;
@@ -219,7 +313,6 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         if (++is_stage == S) is_stage = 0;
     };
 
-    __syncthreads();           // abort flag initialised
     // prologue: the first weights stream before the previous kernel has finished
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
@@ -227,146 +320,152 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
     const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
     const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
-    int stage = 0;
+    int stage = 0, cs = 0;
 
-    for (int cp = 0; cp < a.n; ++cp) {
-        const PassProj &P = a.p[cp];
-        const PassGeo g = pass_geo(P, warp);
-        const int G = P.G;
-        if (P.wait && cp > 0) {
-            if (tid == 0 && !wait_counter(&a.counters[cp - 1], gridDim.x)) {
+    for (int ph = 0; ph < nphase; ++ph) {
+        if (ph > 0) {
+            if (tid == 0 && !wait_counter(&a.counters[ph - 1], gridDim.x)) {
                 atomicOr(a.error, kErrWaitExpired);
                 *abort_flag = 1;
             }
             __syncthreads();
+            if (*abort_flag) break;
         }
-        if (*abort_flag) break;
-        stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
-        __syncthreads();
+        for (; cs < nseg && segs[cs].phase == ph; ++cs) {
+            const PassSeg sgm = segs[cs];
+            const PassProj &P = a.p[sgm.p];
+            const PassGeo g = pass_geo(sgm, warp);
+            const int G = P.G;
+            stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
+            __syncthreads();
 
-        const size_t nstride = (size_t)G * 64 + 32;
-        uint32_t xb[NT];       // B-operand column of this lane (columns >= M read column M-1: ignored)
+            const size_t nstride = (size_t)G * 64 + 32;
+            uint32_t xb[NT];   // B-operand column of this lane (columns >= M read column M-1: ignored)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) xb[nt] = (uint32_t)(xp - smem) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
+            for (int nt = 0; nt < NT; ++nt)
+                xb[nt] = (uint32_t)(xp - smem) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
 
-        float acc[NT][4];
-        float best_v[2 * NT];
-        int best_i[2 * NT];
+            float acc[NT][4];
+            float best_v[2 * NT];
+            int best_i[2 * NT];
 #pragma unroll
-        for (int i = 0; i < 2 * NT; ++i) {
-            best_v[i] = -INFINITY;
-            best_i[i] = 0x7fffffff;
-        }
-        int tl = 0, cl = 0;
-        for (int j = 0; j < g.n_items; ++j) {
-            cp_async_wait_dyn(S - 2);
-            __syncwarp();
-            const int t = g.my_wr + g.wr_n * tl;
-            const int c = g.my_wk + g.wk * cl;
-            const int o0 = g.o_begin + t * g.rout;
-            const int kc = min(kMChunkG, G - c * kMChunkG);
-            if (cl == 0) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+            for (int i = 0; i < 2 * NT; ++i) {
+                best_v[i] = -INFINITY;
+                best_i[i] = 0x7fffffff;
             }
-            const uint32_t so = (uint32_t)stage * kMStage;
-            uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
-            if (P.scales_async) {
-                sg = smq[(sc_o + so) >> 4];
-                sg8 = smq[(sc_o + so + 8 * 16) >> 4];
-            } else {
-                bool v0, v1;
-                const int r0 = pass_slot_row(P, g, o0, qg, v0), r1 = pass_slot_row(P, g, o0, qg + 8, v1);
-                uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
-                const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
-                for (int gl = 0; gl < kc; ++gl) {
-                    u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
-                    u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+            int tl = 0, cl = 0;
+            for (int j = 0; j < g.n_items; ++j) {
+                cp_async_wait_dyn(S - 2);
+                __syncwarp();
+                const int t = g.my_wr + g.wr_n * tl;
+                const int c = g.my_wk + g.wk * cl;
+                const int o0 = g.o_begin + t * g.rout;
+                const int kc = min(kMChunkG, G - c * kMChunkG);
+                if (cl == 0) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
                 }
-                sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-                sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-            }
-            const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-            const uint32_t wrow0 = wq_o + so;
-            const uint32_t xb0 = (uint32_t)(c * kMChunkG) * 64u;                   // + xb[nt] + gl * 64
-            const uint32_t x70 = x7_o + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
-            auto step = [&](int gl) {
-                const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
-                const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
-                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
-                const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
-                const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 bb = smq[(xb[nt] + xb0 + gl * 64) >> 4];
-                    const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
-                    float d[4];
-                    mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
-                              __uint_as_float(czu.z), __uint_as_float(czu.w));
-                    mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                    acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                    acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                    acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                    acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                const uint32_t so = (uint32_t)stage * kMStage;
+                uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
+                if (P.scales_async) {
+                    sg = smq[(sc_o + so) >> 4];
+                    sg8 = smq[(sc_o + so + 8 * 16) >> 4];
+                } else {
+                    bool v0, v1;
+                    const int r0 = pass_slot_row(P, g, o0, qg, v0), r1 = pass_slot_row(P, g, o0, qg + 8, v1);
+                    uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
+                    const unsigned short *p0 =
+                        reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
+                    const unsigned short *p1 =
+                        reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
+                    for (int gl = 0; gl < kc; ++gl) {
+                        u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
+                        u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                    }
+                    sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+                    sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
                 }
-            };
-            if (kc == kMChunkG) {
-#pragma unroll
-                for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
-            } else {
-#pragma unroll
-                for (int gl = 0; gl < kMChunkG; ++gl)
-                    if (gl < kc) step(gl);
-            }
-            __syncwarp();
-            issue_next();
-            if (++stage == S) stage = 0;
-
-            if (cl == g.my_chunks - 1) {
-                if (g.wk > 1) {
-                    // this warp's partial of tile t: [16 rows][8*NT columns]
-                    float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
+                const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+                const uint32_t wrow0 = wq_o + so;
+                const uint32_t xb0 = (uint32_t)(c * kMChunkG) * 64u;                   // + xb[nt] + gl * 64
+                const uint32_t x70 = x7_o + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
+                auto step = [&](int gl) {
+                    const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
+                    const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
+                    const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                    const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
+                    const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
+                    const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+                    const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+                    const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+                    const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
-                        rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
-                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
-                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                        const uint4 bb = smq[(xb[nt] + xb0 + gl * 64) >> 4];
+                        const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
+                        float d[4];
+                        mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
+                                  __uint_as_float(czu.z), __uint_as_float(czu.w));
+                        mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                        acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                        acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                        acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                        acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
                     }
+                };
+                if (kc == kMChunkG) {
+#pragma unroll
+                    for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
                 } else {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
+                    for (int gl = 0; gl < kMChunkG; ++gl)
+                        if (gl < kc) step(gl);
+                }
+                __syncwarp();
+                issue_next();
+                if (++stage == S) stage = 0;
+
+                if (cl == g.my_chunks - 1) {
+                    if (g.wk > 1) {
+                        // this warp's partial of tile t: [16 rows][8*NT columns]
+                        float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int m = 8 * nt + 2 * qt + e;
-                            if (m >= M) continue;
-                            if (P.kind == kEpiGateUp) {
-                                const int n = o0 + qg;
-                                if (n < g.o_end) {
-                                    const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
-                                    const float silu = gv / (1.0f + expf(-gv));
-                                    reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + n] = __float2half_rn(silu * u);
-                                }
-                            } else {
+                        for (int nt = 0; nt < NT; ++nt) {
+                            rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
+                            rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
+                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
+                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                        }
+                    } else {
 #pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    const int n = o0 + qg + 8 * h;
-                                    if (n >= g.o_end) continue;
-                                    const float y = acc[nt][2 * h + e] * pow2f(24);
-                                    if (P.kind == kEpiF16) {
-                                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + n] = __float2half_rn(y);
-                                    } else {
-                                        reinterpret_cast<float *>(P.out)[(size_t)m * P.N + n] = y;
-                                        if (better(y, n, best_v[2 * nt + e], best_i[2 * nt + e])) {
-                                            best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
-                                            best_i[2 * nt + e] = n;
+                        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int m = 8 * nt + 2 * qt + e;
+                                if (m >= M) continue;
+                                if (P.kind == kEpiGateUp) {
+                                    const int nn = o0 + qg;
+                                    if (nn < g.o_end) {
+                                        const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
+                                        const float silu = gv / (1.0f + expf(-gv));
+                                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(silu * u);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        const int nn = o0 + qg + 8 * h;
+                                        if (nn >= g.o_end) continue;
+                                        const float y = acc[nt][2 * h + e] * pow2f(24);
+                                        if (P.kind == kEpiF16) {
+                                            reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(y);
+                                        } else {
+                                            reinterpret_cast<float *>(P.out)[(size_t)m * P.N + nn] = y;
+                                            if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
+                                                best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
+                                                best_i[2 * nt + e] = nn;
+                                            }
                                         }
                                     }
                                 }
@@ -374,81 +473,82 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         }
                     }
                 }
-            }
-            if (++cl == g.my_chunks) {
-                cl = 0;
-                ++tl;
-            }
-        }
-
-        if (g.wk > 1) {
-            // WK partials of each tile meet here; fixed summation order
-            __syncthreads();
-            const int VO = g.rout * 8 * NT;                   // (output row, column) pairs per tile
-            for (int idx = tid; idx < g.n_tiles * VO; idx += kMThreads) {
-                const int t = idx / VO, vo = idx - (idx / VO) * VO;
-                const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
-                const int n = g.o_begin + t * g.rout + r;
-                if (n >= g.o_end || m >= M) continue;
-                const float *rp = red + (size_t)t * g.wk * kMTileRows * 8 * NT;
-                float y = 0.f, u = 0.f;
-                for (int k2 = 0; k2 < g.wk; ++k2) {
-                    y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
-                    if (P.kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                if (++cl == g.my_chunks) {
+                    cl = 0;
+                    ++tl;
                 }
-                y *= pow2f(24);
-                if (P.kind == kEpiF16) {
-                    reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + n] = __float2half_rn(y);
-                } else if (P.kind == kEpiGateUp) {
-                    u *= pow2f(24);
-                    const float silu = y / (1.0f + expf(-y));
-                    reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + n] = __float2half_rn(silu * u);
-                } else {
-                    reinterpret_cast<float *>(P.out)[(size_t)m * P.N + n] = y;
-                    // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
-                    if (better(y, n, best_v[0], best_i[0])) {
-                        best_v[0] = isnan(y) ? -INFINITY : y;
-                        best_i[0] = n;
+            }
+
+            if (g.wk > 1) {
+                // WK partials of each tile meet here; fixed summation order
+                __syncthreads();
+                const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
+                for (int idx = tid; idx < g.n_tiles * VO; idx += kMThreads) {
+                    const int t = idx / VO, vo = idx - (idx / VO) * VO;
+                    const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
+                    const int nn = g.o_begin + t * g.rout + r;
+                    if (nn >= g.o_end || m >= M) continue;
+                    const float *rp = red + (size_t)t * g.wk * kMTileRows * 8 * NT;
+                    float y = 0.f, u = 0.f;
+                    for (int k2 = 0; k2 < g.wk; ++k2) {
+                        y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
+                        if (P.kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                    }
+                    y *= pow2f(24);
+                    if (P.kind == kEpiF16) {
+                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(y);
+                    } else if (P.kind == kEpiGateUp) {
+                        u *= pow2f(24);
+                        const float silu = y / (1.0f + expf(-y));
+                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(silu * u);
+                    } else {
+                        reinterpret_cast<float *>(P.out)[(size_t)m * P.N + nn] = y;
+                        // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
+                        if (better(y, nn, best_v[0], best_i[0])) {
+                            best_v[0] = isnan(y) ? -INFINITY : y;
+                            best_i[0] = nn;
+                        }
                     }
                 }
             }
-        }
 
-        if (P.kind == kEpiLogits) {
+            if (P.kind == kEpiLogits) {
 #pragma unroll
-            for (int i = 0; i < 2 * NT; ++i) {
-                bvs[tid * 2 * NT + i] = best_v[i];
-                bis[tid * 2 * NT + i] = best_i[i];
-            }
-            __syncthreads();
-            if (tid < M) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-                for (int th = 0; th < kMThreads; ++th) {
-                    for (int i = 0; i < 2 * NT; ++i) {
-                        int tm;
-                        if (g.wk > 1) {
-                            if (i != 0) continue;
-                            tm = th % (8 * NT);
-                        } else {
-                            tm = 8 * (i >> 1) + 2 * (th & 3) + (i & 1);
-                        }
-                        if (tm == tid && better(bvs[th * 2 * NT + i], bis[th * 2 * NT + i], bv, bi)) {
-                            bv = bvs[th * 2 * NT + i];
-                            bi = bis[th * 2 * NT + i];
+                for (int i = 0; i < 2 * NT; ++i) {
+                    bvs[tid * 2 * NT + i] = best_v[i];
+                    bis[tid * 2 * NT + i] = best_i[i];
+                }
+                __syncthreads();
+                if (tid < M) {
+                    float bv = -INFINITY;
+                    int bi = 0x7fffffff;
+                    for (int th = 0; th < kMThreads; ++th) {
+                        for (int i = 0; i < 2 * NT; ++i) {
+                            int tm;
+                            if (g.wk > 1) {
+                                if (i != 0) continue;
+                                tm = th % (8 * NT);
+                            } else {
+                                tm = 8 * (i >> 1) + 2 * (th & 3) + (i & 1);
+                            }
+                            if (tm == tid && better(bvs[th * 2 * NT + i], bis[th * 2 * NT + i], bv, bi)) {
+                                bv = bvs[th * 2 * NT + i];
+                                bi = bis[th * 2 * NT + i];
+                            }
                         }
                     }
+                    P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
+                    P.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
                 }
-                P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-                P.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
             }
+            __syncthreads();   // the activation area and partial buffers are free again
         }
-
-        // done with this projection: the activation area may be restaged and,
-        // if a later projection waits on it, the CTA's outputs are published
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && a.counters != nullptr) atomicAdd(&a.counters[cp], 1u);
+        if (ph + 1 < nphase) {
+            // publish this CTA's outputs of the phase, then count it done
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicAdd(&a.counters[ph], 1u);
+        }
     }
     cp_async_wait<0>();
 }

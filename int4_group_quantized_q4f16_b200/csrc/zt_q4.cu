@@ -221,22 +221,6 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
     return ZT_ERR_UNSUPPORTED;
 }
 
-// Fill the per-projection launch fields that depend on the grid.
-template <int PMAX>
-void pass_fill(PassArgs<PMAX> &a, int grid, int NT, int &red_floats_max)
-{
-    red_floats_max = 0;
-    for (int i = 0; i < a.n; ++i) {
-        PassProj &p = a.p[i];
-        const int rout = (p.kind == kEpiGateUp) ? kMTileRows / 2 : kMTileRows;
-        const int rows_max = (p.N + grid - 1) / grid;
-        p.max_tiles = (rows_max + rout - 1) / rout;
-        p.wk = pick_wk(p.max_tiles, (p.G + kMChunkG - 1) / kMChunkG);
-        const int red = p.wk > 1 ? p.max_tiles * p.wk * kMTileRows * 8 * NT : 0;
-        red_floats_max = std::max(red_floats_max, red);
-    }
-}
-
 // Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
 // some projection waits on earlier ones (all CTAs must be co-resident).
 // ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
@@ -248,20 +232,31 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
     if (resident_ctas(fn, kMThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
     a.g_max = 0;
     for (int i = 0; i < a.n; ++i) a.g_max = std::max(a.g_max, a.p[i].G);
-    int min_n = a.p[0].N;
-    for (int i = 1; i < a.n; ++i) min_n = std::min(min_n, a.p[i].N);
+    // Phases: a new one at every projection that waits.  Each CTA takes a
+    // byte-balanced share of each phase's concatenated rows.
+    long long rows = 0;      // a CTA with no rows of a list without waits would only idle
+    long long phase_bytes[kPassMax];
+    a.phases = 0;
+    for (int i = 0; i < a.n; ++i) {
+        PassProj &p = a.p[i];
+        if (i == 0 || p.wait) phase_bytes[a.phases++] = 0;
+        p.phase = a.phases - 1;
+        p.row_bytes = (p.K / 2 + p.K / 16) * (p.kind == kEpiGateUp ? 2 : 1);
+        p.base = phase_bytes[p.phase];
+        phase_bytes[p.phase] += (long long)p.N * p.row_bytes;
+        rows += p.N;
+    }
+    for (int i = 0; i < a.n; ++i) a.p[i].phase_bytes = phase_bytes[a.p[i].phase];
     for (int cps = 2; cps >= 1; --cps) {
-        const int grid = std::max(1, std::min({sms * cps, cooperative ? sms * cps : min_n, kMaxCtas}));
-        int red_floats = 0;
-        pass_fill(a, grid, NT, red_floats);
-        a.red_floats = red_floats;
-        const size_t fixed = pass_smem_bytes(a.M, a.g_max, 0, red_floats, NT);
+        const int grid = (int)std::max<long long>(
+            1, std::min<long long>({(long long)sms * cps, cooperative ? (long long)sms * cps : rows, kMaxCtas}));
+        const size_t fixed = pass_smem_bytes(a.M, a.g_max, 0, a.n, NT);
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const size_t per_stage = (size_t)kMW * kMStage;
         const int stages = budget > fixed ? (int)std::min<size_t>(kMMaxStages, (budget - fixed) / per_stage) : 0;
         if (stages < 2) continue;
         a.stages = stages;
-        const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, red_floats, NT);
+        const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, a.n, NT);
         const int occ = resident_ctas(fn, kMThreads, smem, sms);
         if (occ < cps) continue;
         if (grid_out) *grid_out = grid;
