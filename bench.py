@@ -47,9 +47,10 @@ from int4_group_quantized_q4f16_b200 import synth  # noqa: E402
 
 METRIC = "q4 dequant-GEMV effective HBM GB/s & % of B200 peak; us per decode weight pass"
 NOMINAL_HBM_GBS = 8000.0
-WORKLOAD = ("Phi-3-mini decode weight pass, M=1: 32 x (qkv 3072->9216, o 3072->3072, "
+def workload(layers: int, seed: int) -> str:
+    return (f"Phi-3-mini decode weight pass, M=1: {layers} x (qkv 3072->9216, o 3072->3072, "
             "gate_up 3072->2x8192 +SiLU*up, down 8192->3072) + LM head 3072->32064 f32+argmax; "
-            "q4 group-32 weights, seed 0")
+            f"q4 group-32 weights, seed {seed}")
 
 
 def parse_args():
@@ -220,7 +221,7 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_per_step": "layer 0: qkv, o, gate_up+SiLU, down (63.8 MB)"},
+        "config": {"workload": workload(32, args.seed), "sample_per_step": "layer 0: qkv, o, gate_up+SiLU, down (63.8 MB)"},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": "one Phi-3-mini layer (4 projections, 63.8 MB of q4 weights) per step"},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -494,17 +495,17 @@ def run_ours(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16xf16->f32 (int4 codes, fp16 scales)",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": 1, "layers": args.layers, "launches_per_step": 2,
+            "config": {"workload": workload(args.layers, args.seed), "M": 1, "layers": args.layers, "launches_per_step": 2,
                        "entry_point": "zt_q4_pass (one persistent kernel over independent projections) + argmax reduction",
                        "graph": graph is not None,
-                       "bytes_per_step": total_bytes, "l2": "inputs larger than L2 (2.1 GB per step, L2 126 MB)",
+                       "bytes_per_step": total_bytes, "l2": f"inputs larger than L2 ({total_bytes / 1e9:.2f} GB per step, L2 126 MB)",
                        "parallelism": f"replicas x{world}"},
             "us_per_pass": round(ms_per_step * 1e3, 2),
             "pct_of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS * 100, 2),
             "pct_of_measured_peak": round(value / world / peak * 100, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "kernel": "q4_pass_kernel (one launch per step over the 129 projections)",
+                         "kernel": f"q4_pass_kernel (one launch per step over the {len(calls)} projections)",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                          else "fallback 6.65 TB/s",
                          "bytes_per_launch": round(kb), "us_per_launch": round(kms * 1e3, 3)},

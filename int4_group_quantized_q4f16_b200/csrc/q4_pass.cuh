@@ -56,15 +56,19 @@ struct PassProj {
 // parameter block), kPassMax for zt_q4_pass.
 template <int PMAX>
 struct PassArgs {
-    int n, M, stages, phases;
+    int n, M, phases;
     int g_max;                  // largest G of the list (sizes the activation area)
     unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
     PassProj p[PMAX];
 };
 
-// WK > 1 partial buffer: at most kRedTiles / NT tiles x WK warps per segment
-constexpr int kRedFloats = 4096;            // 16 KB: (tiles * wk) * 16 rows * 8 NT cols <= this
+// WK > 1 partial buffer: (tiles x WK) warp tiles of 16 rows x 8 NT columns
+// per segment.  The LM head's per-thread maxima reuse it once a segment's
+// partial sums have been read.
+constexpr int kRedFloats = 2048;            // 8 KB
+static_assert(kMThreads * 2 * 2 * 8 <= kRedFloats * 4, "LM-head maxima must fit the partial buffer");
+constexpr int kPassMaxStages = 4;           // ring depths 2..4 are instantiated
 
 // One projection's rows in one CTA, with the CTA's warp layout for them.
 struct PassSeg {
@@ -73,20 +77,19 @@ struct PassSeg {
 };
 
 // Shared memory per CTA: rings, permuted activations (n-stride G*64 + 32
-// bytes), C-operand table, WK partials, LM-head maxima, segment list, flags.
+// bytes), C-operand table, WK partials / LM-head maxima, segment list, flags.
 __host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int n, int NT)
 {
     const size_t ring = (size_t)kMW * stages * kMStage;
     const size_t xp = (size_t)M * ((size_t)g_max * 64 + 32);
     const size_t x7 = (size_t)g_max * NT * 64;
-    const size_t best = (size_t)kMThreads * 2 * NT * 8;
-    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)kRedFloats * 4 + best + (size_t)n * sizeof(PassSeg) +
+    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)kRedFloats * 4 + (size_t)n * sizeof(PassSeg) +
            (kMW + 4) * sizeof(int);
 }
 
-// Per-projection geometry of one warp.
+// Per-segment geometry of one warp.
 struct PassGeo {
-    int o_begin, o_end, rout, n_tiles, n_chunks, wk, wr_n, my_wk, my_wr, my_tiles, my_chunks, n_items;
+    int o_begin, o_end, rout, n_tiles, n_chunks, wk, wr_n, my_wk, my_wr, my_tiles, my_chunks;
 };
 
 static_assert(kMW == 8, "warp layout below assumes 8 warps");
@@ -126,21 +129,29 @@ __device__ __forceinline__ PassGeo pass_geo(const PassSeg &sg, int warp)
     g.my_wr = warp >> sg.wkl;
     g.my_tiles = g.my_wr < g.n_tiles ? (g.n_tiles - g.my_wr + g.wr_n - 1) >> (3 - sg.wkl) : 0;
     g.my_chunks = g.my_wk < g.n_chunks ? (g.n_chunks - g.my_wk + g.wk - 1) >> sg.wkl : 0;
-    g.n_items = g.my_tiles * g.my_chunks;
+    if (g.my_chunks == 0) g.my_tiles = 0;
     return g;
 }
 
 // weight row of tile slot r (0..15) of the tile starting at output o0
-__device__ __forceinline__ int pass_slot_row(const PassProj &P, const PassGeo &g, int o0, int r, bool &valid)
+__device__ __forceinline__ int pass_slot_row(int kind, int N, int o_end, int o0, int r, bool &valid)
 {
-    if (P.kind == kEpiGateUp) {
+    if (kind == kEpiGateUp) {
         const int o = o0 + (r & 7);
-        valid = o < g.o_end;
-        return (r < 8 ? 0 : P.N) + min(o, P.N - 1);
+        valid = o < o_end;
+        return (r < 8 ? 0 : N) + min(o, N - 1);
     }
     const int o = o0 + r;
-    valid = o < g.o_end;
-    return min(o, P.N - 1);
+    valid = o < o_end;
+    return min(o, N - 1);
+}
+
+// groups in the last chunk this warp reads of a segment (8 unless G % 8 != 0
+// and that chunk is the projection's last)
+__device__ __forceinline__ int pass_last_kc(const PassGeo &g, int G)
+{
+    const int c_last = g.my_wk + g.wk * (g.my_chunks - 1);
+    return min(kMChunkG, G - c_last * kMChunkG);
 }
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned int *p)
@@ -168,11 +179,12 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *counter, unsign
     }
 }
 
-template <int NT, int PMAX>
+template <int NT, int PMAX, int S>
 __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
+    static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     extern __shared__ __align__(128) unsigned char smem[];
-    const int M = a.M, S = a.stages, n = a.n;
+    const int M = a.M, n = a.n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qg = lane >> 2, qt = lane & 3;       // mma quad row / thread in quad
 
@@ -181,9 +193,9 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const size_t xp_bytes = ((size_t)M * ((size_t)a.g_max * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
     float *red = x7 + (size_t)a.g_max * NT * 16;
-    float *bvs = red + kRedFloats;
+    float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
-    PassSeg *segs = reinterpret_cast<PassSeg *>(bis + kMThreads * 2 * NT);
+    PassSeg *segs = reinterpret_cast<PassSeg *>(red + kRedFloats);
     int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
     volatile int *abort_flag = wcount + kMW;
 
@@ -239,88 +251,97 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     __syncthreads();
     const int nphase = a.phases;
 
-    // Byte offsets from the start of shared memory; loads index the shared
-    // array directly, so the compiler sees shared-space, 32-bit addressing.
-    const uint32_t *smw = reinterpret_cast<const uint32_t *>(smem);
-    const uint4 *smq = reinterpret_cast<const uint4 *>(smem);
-    const uint32_t ring_o = (uint32_t)(ring - smem);
     const uint32_t ring_u = smem_u32(ring);
 
     // ---------------------------------------------------------- issue side --
     // The warp's items of all segments form one stream (segment, tile,
-    // chunk); lane l copies pieces p = l + 32 i (i < 4) of an item: tile row
-    // r = l / 8 + 4 i, group l % 8 of the chunk.  It runs ahead of the
-    // compute side by S - 1 items, across segment and phase boundaries.
+    // chunk); lane l copies pieces l + 32 i (i < 4) of an item: tile row
+    // l / 8 + 4 i, group l % 8 of the chunk.  The stream runs S - 1 items
+    // ahead of the math, across segment and phase boundaries (weights never
+    // depend on outputs).  Per item it only advances pointers; segment and
+    // tile changes recompute them.
     const int pg = lane & 7;
     const uint32_t piece_u = ring_u + (lane >> 3) * kMRowStride + pg * 16;   // + stage, + 4 i rows
     const uint32_t scale_u = ring_u + kMScaleOff + lane * 16;
-    int is_s = 0, is_tl = 0, is_cl = 0, is_stage = 0, is_left = 0;
+    int is_s = -1;                  // segment being issued
+    int is_tiles = 0;               // tiles left after the current one
+    int is_chunks = 0;              // chunks left in the current tile (0: stream ended)
+    int is_kc_last = kMChunkG;      // groups of the tile's last chunk
+    int is_step = 0;                // uint4 per chunk step (WK chunks of 8 groups)
+    uint32_t is_so = 0;             // ring stage offset
+    int is_o0 = 0, is_rstep = 0;    // current tile's first output, outputs per tile step
     PassGeo ig{};
     const uint4 *src_w[4];
     bool ok_w[4];
     const __half *src_s = nullptr;
     bool ok_s = false;
-    auto set_tile = [&](int tl) {
+    auto set_tile = [&]() {
         const PassProj &P = a.p[segs[is_s].p];
-        const int o0 = ig.o_begin + (ig.my_wr + ig.wr_n * tl) * ig.rout;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = pass_slot_row(P, ig, o0, (lane >> 3) + 4 * i, ok_w[i]);
-            src_w[i] = P.qw + (size_t)row * P.G + pg;
+            const int row = pass_slot_row(P.kind, P.N, ig.o_end, is_o0, (lane >> 3) + 4 * i, ok_w[i]);
+            src_w[i] = P.qw + (size_t)row * P.G + ig.my_wk * kMChunkG + pg;
         }
         ok_s = false;
-        if (lane < kMTileRows) {
-            const int row = pass_slot_row(P, ig, o0, lane, ok_s);
-            src_s = P.scales + (size_t)row * P.G;
-        }
+        const int row = pass_slot_row(P.kind, P.N, ig.o_end, is_o0, lane & 15, ok_s);
+        ok_s = ok_s && lane < kMTileRows && P.scales_async;
+        src_s = P.scales + (size_t)row * P.G + ig.my_wk * kMChunkG;
+        is_chunks = ig.my_chunks;
     };
-    // move the issue pointer to the next segment that has items for this warp
-    auto advance = [&]() {
-        while (is_left == 0 && is_s < nseg) {
-            if (++is_s >= nseg) break;
+    // move to the next segment that has items for this warp (or end the stream)
+    auto next_segment = [&]() {
+        is_chunks = 0;
+        while (++is_s < nseg) {
             ig = pass_geo(segs[is_s], warp);
-            is_tl = is_cl = 0;
-            is_left = ig.n_items;
-        }
-        if (is_left > 0) set_tile(is_tl);
-    };
-    if (nseg > 0) {
-        ig = pass_geo(segs[0], warp);
-        is_left = ig.n_items;
-        if (is_left > 0) set_tile(0);
-        else advance();
-    }
-    auto issue_next = [&]() {
-        if (is_left > 0 && !*abort_flag) {
+            if (ig.my_tiles == 0) continue;
             const PassProj &P = a.p[segs[is_s].p];
-            const int c = ig.my_wk + ig.wk * is_cl;
-            const bool full = (c + 1) * kMChunkG <= P.G;
-            const int kc = full ? kMChunkG : P.G - c * kMChunkG;
-            const uint32_t so = (uint32_t)is_stage * kMStage;
+            is_tiles = ig.my_tiles - 1;
+            is_kc_last = pass_last_kc(ig, P.G);
+            is_step = ig.wk * kMChunkG;
+            is_rstep = ig.wr_n * ig.rout;
+            is_o0 = ig.o_begin + ig.my_wr * ig.rout;
+            set_tile();
+            return;
+        }
+    };
+    next_segment();
+    auto issue_next = [&]() {
+        if (is_chunks > 0) {
+            const int kc = is_chunks == 1 ? is_kc_last : kMChunkG;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok_w[i] && pg < kc) cp_async16_u32(piece_u + so + 4 * i * kMRowStride, src_w[i] + c * kMChunkG);
-            if (P.scales_async && ok_s && lane < kMTileRows) cp_async16_u32(scale_u + so, src_s + c * kMChunkG);
-            --is_left;
-            if (++is_cl == ig.my_chunks) {
-                is_cl = 0;
-                ++is_tl;
-                if (is_left > 0) set_tile(is_tl);
+                if (ok_w[i] && pg < kc) cp_async16_u32(piece_u + is_so + 4 * i * kMRowStride, src_w[i]);
+            if (ok_s) cp_async16_u32(scale_u + is_so, src_s);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) src_w[i] += is_step;
+            src_s += is_step;
+            if (--is_chunks == 0) {
+                if (is_tiles > 0) {
+                    --is_tiles;
+                    is_o0 += is_rstep;
+                    set_tile();
+                } else {
+                    next_segment();
+                }
             }
-            if (is_left == 0) advance();
         }
         cp_async_commit();     // one group per item slot, so wait counts stay uniform
-        if (++is_stage == S) is_stage = 0;
+        is_so = (is_so + kMStage == (uint32_t)(S * kMStage)) ? 0u : is_so + kMStage;
     };
 
     // prologue: the first weights stream before the previous kernel has finished
+#pragma unroll
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
 
+    const uint32_t ring_o = (uint32_t)(ring - smem);
     const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
     const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
     const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
-    int stage = 0, cs = 0;
+    const uint32_t *smw = reinterpret_cast<const uint32_t *>(smem);
+    const uint4 *smq = reinterpret_cast<const uint4 *>(smem);
+    uint32_t so = 0;                // ring stage offset of the next item to compute
+    int cs = 0;
 
     for (int ph = 0; ph < nphase; ++ph) {
         if (ph > 0) {
@@ -335,17 +356,20 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const PassSeg sgm = segs[cs];
             const PassProj &P = a.p[sgm.p];
             const PassGeo g = pass_geo(sgm, warp);
-            const int G = P.G;
+            const int G = P.G, N = P.N, kind = P.kind;
+            const bool sasync = P.scales_async;
+            void *const out = P.out;
             stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
             __syncthreads();
 
-            const size_t nstride = (size_t)G * 64 + 32;
+            const uint32_t nstride = (uint32_t)G * 64u + 32u;
             uint32_t xb[NT];   // B-operand column of this lane (columns >= M read column M-1: ignored)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-                xb[nt] = (uint32_t)(xp - smem) + (uint32_t)(min(qg + 8 * nt, M - 1) * nstride) + qt * 16;
+                xb[nt] = (uint32_t)(xp - smem) + (uint32_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
+            const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
+            const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = xstep * NT;
 
-            float acc[NT][4];
             float best_v[2 * NT];
             int best_i[2 * NT];
 #pragma unroll
@@ -353,129 +377,132 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 best_v[i] = -INFINITY;
                 best_i[i] = 0x7fffffff;
             }
-            int tl = 0, cl = 0;
-            for (int j = 0; j < g.n_items; ++j) {
-                cp_async_wait_dyn(S - 2);
-                __syncwarp();
+            for (int tl = 0; tl < g.my_tiles; ++tl) {
                 const int t = g.my_wr + g.wr_n * tl;
-                const int c = g.my_wk + g.wk * cl;
                 const int o0 = g.o_begin + t * g.rout;
-                const int kc = min(kMChunkG, G - c * kMChunkG);
-                if (cl == 0) {
+                float acc[NT][4];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-                }
-                const uint32_t so = (uint32_t)stage * kMStage;
-                uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
-                if (P.scales_async) {
-                    sg = smq[(sc_o + so) >> 4];
-                    sg8 = smq[(sc_o + so + 8 * 16) >> 4];
-                } else {
-                    bool v0, v1;
-                    const int r0 = pass_slot_row(P, g, o0, qg, v0), r1 = pass_slot_row(P, g, o0, qg + 8, v1);
-                    uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                    const unsigned short *p0 =
-                        reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
-                    const unsigned short *p1 =
-                        reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
-                    for (int gl = 0; gl < kc; ++gl) {
-                        u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
-                        u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+                uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
+                uint32_t coff = xoff * NT;                            // C-table bytes
+                for (int cl = 0; cl < g.my_chunks; ++cl) {
+                    cp_async_wait<S - 2>();
+                    __syncwarp();
+                    const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
+                    uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
+                    if (sasync) {
+                        sg = smq[(sc_o + so) >> 4];
+                        sg8 = smq[(sc_o + so + 8 * 16) >> 4];
+                    } else {
+                        bool v0, v1;
+                        const int c = g.my_wk + g.wk * cl;
+                        const int r0 = pass_slot_row(kind, N, g.o_end, o0, qg, v0);
+                        const int r1 = pass_slot_row(kind, N, g.o_end, o0, qg + 8, v1);
+                        uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
+                        const unsigned short *p0 =
+                            reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
+                        const unsigned short *p1 =
+                            reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
+                        for (int gl = 0; gl < kc; ++gl) {
+                            u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
+                            u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                        }
+                        sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+                        sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
                     }
-                    sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-                    sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-                }
-                const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-                const uint32_t wrow0 = wq_o + so;
-                const uint32_t xb0 = (uint32_t)(c * kMChunkG) * 64u;                   // + xb[nt] + gl * 64
-                const uint32_t x70 = x7_o + (uint32_t)(c * kMChunkG) * (NT * 64u);    // + (gl * NT + nt) * 64
-                auto step = [&](int gl) {
-                    const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
-                    const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
-                    const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                    const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu, w1s & 0x000F000Fu};
-                    const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u, w1s & 0x00F000F0u};
-                    const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                    const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                    const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                    const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
+                    const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+                    const uint32_t wrow0 = wq_o + so;
+                    const uint32_t x70 = x7_o + coff;                 // + (gl * NT + nt) * 64
+                    uint32_t xbc[NT];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint4 bb = smq[(xb[nt] + xb0 + gl * 64) >> 4];
-                        const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
-                        float d[4];
-                        mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
-                                  __uint_as_float(czu.z), __uint_as_float(czu.w));
-                        mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                        acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                        acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                        acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                        acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
-                    }
-                };
-                if (kc == kMChunkG) {
-#pragma unroll
-                    for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
-                } else {
-#pragma unroll
-                    for (int gl = 0; gl < kMChunkG; ++gl)
-                        if (gl < kc) step(gl);
-                }
-                __syncwarp();
-                issue_next();
-                if (++stage == S) stage = 0;
-
-                if (cl == g.my_chunks - 1) {
-                    if (g.wk > 1) {
-                        // this warp's partial of tile t: [16 rows][8*NT columns]
-                        float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
+                    for (int nt = 0; nt < NT; ++nt) xbc[nt] = xb[nt] + xoff;   // + gl * 64
+                    auto step = [&](int gl) {
+                        const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
+                        const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
+                        const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                        const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
+                                                w1s & 0x000F000Fu};
+                        const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
+                                                w1s & 0x00F000F0u};
+                        const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+                        const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+                        const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+                        const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
-                            rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
-                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
-                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                            const uint4 bb = smq[(xbc[nt] + gl * 64) >> 4];
+                            const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
+                            float d[4];
+                            mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
+                                      __uint_as_float(czu.z), __uint_as_float(czu.w));
+                            mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                            acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                            acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                            acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                            acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
                         }
+                    };
+                    if (kc == kMChunkG) {
+#pragma unroll
+                        for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
                     } else {
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
+                        for (int gl = 0; gl < kMChunkG; ++gl)
+                            if (gl < kc) step(gl);
+                    }
+                    __syncwarp();
+                    issue_next();
+                    so = (so + kMStage == (uint32_t)(S * kMStage)) ? 0u : so + kMStage;
+                    xoff += xstep;
+                    coff += cstep;
+                }
+
+                // ---- tile epilogue ----
+                if (g.wk > 1) {
+                    // this warp's partial of tile t: [16 rows][8*NT columns]
+                    float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int m = 8 * nt + 2 * qt + e;
-                                if (m >= M) continue;
-                                if (P.kind == kEpiGateUp) {
-                                    const int nn = o0 + qg;
-                                    if (nn < g.o_end) {
-                                        const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
-                                        const float silu = gv / (1.0f + expf(-gv));
-                                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(silu * u);
-                                    }
-                                } else {
+                    for (int nt = 0; nt < NT; ++nt) {
+                        rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
+                        rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
+                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
+                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                    }
+                } else {
 #pragma unroll
-                                    for (int h = 0; h < 2; ++h) {
-                                        const int nn = o0 + qg + 8 * h;
-                                        if (nn >= g.o_end) continue;
-                                        const float y = acc[nt][2 * h + e] * pow2f(24);
-                                        if (P.kind == kEpiF16) {
-                                            reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(y);
-                                        } else {
-                                            reinterpret_cast<float *>(P.out)[(size_t)m * P.N + nn] = y;
-                                            if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
-                                                best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
-                                                best_i[2 * nt + e] = nn;
-                                            }
+                    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int m = 8 * nt + 2 * qt + e;
+                            if (m >= M) continue;
+                            if (kind == kEpiGateUp) {
+                                const int nn = o0 + qg;
+                                if (nn < g.o_end) {
+                                    const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
+                                    const float silu = gv / (1.0f + expf(-gv));
+                                    reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
+                                }
+                            } else {
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int nn = o0 + qg + 8 * h;
+                                    if (nn >= g.o_end) continue;
+                                    const float y = acc[nt][2 * h + e] * pow2f(24);
+                                    if (kind == kEpiF16) {
+                                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                                    } else {
+                                        reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
+                                        if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
+                                            best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
+                                            best_i[2 * nt + e] = nn;
                                         }
                                     }
                                 }
                             }
                         }
                     }
-                }
-                if (++cl == g.my_chunks) {
-                    cl = 0;
-                    ++tl;
                 }
             }
 
@@ -492,17 +519,17 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     float y = 0.f, u = 0.f;
                     for (int k2 = 0; k2 < g.wk; ++k2) {
                         y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
-                        if (P.kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                        if (kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
                     }
                     y *= pow2f(24);
-                    if (P.kind == kEpiF16) {
-                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(y);
-                    } else if (P.kind == kEpiGateUp) {
+                    if (kind == kEpiF16) {
+                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                    } else if (kind == kEpiGateUp) {
                         u *= pow2f(24);
                         const float silu = y / (1.0f + expf(-y));
-                        reinterpret_cast<__half *>(P.out)[(size_t)m * P.N + nn] = __float2half_rn(silu * u);
+                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
                     } else {
-                        reinterpret_cast<float *>(P.out)[(size_t)m * P.N + nn] = y;
+                        reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
                         // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
                         if (better(y, nn, best_v[0], best_i[0])) {
                             best_v[0] = isnan(y) ? -INFINITY : y;
@@ -512,7 +539,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 }
             }
 
-            if (P.kind == kEpiLogits) {
+            if (kind == kEpiLogits) {
+                __syncthreads();   // the maxima overwrite the partial buffer
 #pragma unroll
                 for (int i = 0; i < 2 * NT; ++i) {
                     bvs[tid * 2 * NT + i] = best_v[i];

@@ -224,12 +224,50 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
 // Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
 // some projection waits on earlier ones (all CTAs must be co-resident).
 // ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
+constexpr int kNotResident = 1;   // launch_pass_s: this shape does not reach the wanted residency
+
+template <int NT, int PMAX, int S>
+int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps)
+{
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S>);
+    int sms = 0;
+    if (resident_ctas(fn, kMThreads, smem, sms) < cps) return kNotResident;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kMThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (cooperative) {
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    clear_stale_error();
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S>, a);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    return ZT_OK;
+}
+
+// Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
+// some projection waits on earlier ones (all CTAs must be co-resident).
+// Two CTAs per SM when the rings (2..4 stages) and the staged activations
+// fit in half the SM's shared memory, else one.  ZT_ERR_UNSUPPORTED if
+// neither fits.
 template <int NT, int PMAX>
 int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_out)
 {
-    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX>);
     int sms = 0;
-    if (resident_ctas(fn, kMThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2>), kMThreads, 0, sms) < 1)
+        return ZT_ERR_DEVICE;
     a.g_max = 0;
     for (int i = 0; i < a.n; ++i) a.g_max = std::max(a.g_max, a.p[i].G);
     // Phases: a new one at every projection that waits.  Each CTA takes a
@@ -253,36 +291,18 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         const size_t fixed = pass_smem_bytes(a.M, a.g_max, 0, a.n, NT);
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const size_t per_stage = (size_t)kMW * kMStage;
-        const int stages = budget > fixed ? (int)std::min<size_t>(kMMaxStages, (budget - fixed) / per_stage) : 0;
+        const int stages = budget > fixed ? (int)std::min<size_t>(kPassMaxStages, (budget - fixed) / per_stage) : 0;
         if (stages < 2) continue;
-        a.stages = stages;
         const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, a.n, NT);
-        const int occ = resident_ctas(fn, kMThreads, smem, sms);
-        if (occ < cps) continue;
-        if (grid_out) *grid_out = grid;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(kMThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        if (cooperative) {
-            attr[0].id = cudaLaunchAttributeCooperative;
-            attr[0].val.cooperative = 1;
-        } else {
-            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[0].val.programmaticStreamSerializationAllowed = 1;
+        int rc;
+        switch (stages) {
+        case 2: rc = launch_pass_s<NT, PMAX, 2>(a, cooperative, st, grid, smem, cps); break;
+        case 3: rc = launch_pass_s<NT, PMAX, 3>(a, cooperative, st, grid, smem, cps); break;
+        default: rc = launch_pass_s<NT, PMAX, 4>(a, cooperative, st, grid, smem, cps); break;
         }
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        clear_stale_error();
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX>, a);
-        if (e != cudaSuccess) {
-            g_last_cuda_error = e;
-            (void)cudaGetLastError();
-            return ZT_ERR_LAUNCH;
-        }
-        return ZT_OK;
+        if (rc == kNotResident) continue;
+        if (rc == ZT_OK && grid_out) *grid_out = grid;
+        return rc;
     }
     return ZT_ERR_UNSUPPORTED;
 }
