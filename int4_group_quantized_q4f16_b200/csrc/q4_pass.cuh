@@ -28,6 +28,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "q4_mma.cuh"
 
 namespace zt {
@@ -179,10 +181,13 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *counter, unsign
     }
 }
 
-template <int NT, int PMAX, int S>
+// NT: n-tiles of 8 activation columns (M <= 8 NT); ONE: M == 1, so the mma's
+// odd columns are never read and their accumulation is skipped; S: ring depth.
+template <int NT, int PMAX, int S, bool ONE>
 __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
+    static_assert(!ONE || NT == 1, "one column fits one n-tile");
     extern __shared__ __align__(128) unsigned char smem[];
     const int M = a.M, n = a.n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -271,7 +276,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     uint32_t is_so = 0;             // ring stage offset
     int is_o0 = 0, is_rstep = 0;    // current tile's first output, outputs per tile step
     PassGeo ig{};
-    const uint4 *src_w[4];
+    const uint4 *src_w[4];          // the next chunk's source, per piece
     bool ok_w[4];
     const __half *src_s = nullptr;
     bool ok_s = false;
@@ -338,8 +343,6 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
     const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
     const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
-    const uint32_t *smw = reinterpret_cast<const uint32_t *>(smem);
-    const uint4 *smq = reinterpret_cast<const uint4 *>(smem);
     uint32_t so = 0;                // ring stage offset of the next item to compute
     int cs = 0;
 
@@ -370,133 +373,143 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
             const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = xstep * NT;
 
-            float best_v[2 * NT];
-            int best_i[2 * NT];
+            // The segment's tiles; LOG: the LM head's epilogue (f32 logits and
+            // running maxima) -- compiled apart so that the other projections'
+            // loop does not carry the maxima.
+            auto run_segment = [&](auto log_tag) {
+                constexpr bool LOG = decltype(log_tag)::value;
+                float best_v[2 * NT];
+                int best_i[2 * NT];
 #pragma unroll
-            for (int i = 0; i < 2 * NT; ++i) {
-                best_v[i] = -INFINITY;
-                best_i[i] = 0x7fffffff;
-            }
-            for (int tl = 0; tl < g.my_tiles; ++tl) {
-                const int t = g.my_wr + g.wr_n * tl;
-                const int o0 = g.o_begin + t * g.rout;
-                float acc[NT][4];
+                for (int i = 0; i < 2 * NT; ++i) {
+                    best_v[i] = -INFINITY;
+                    best_i[i] = 0x7fffffff;
+                }
+                for (int tl = 0; tl < g.my_tiles; ++tl) {
+                    const int t = g.my_wr + g.wr_n * tl;
+                    const int o0 = g.o_begin + t * g.rout;
+                    float acc[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-                uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
-                uint32_t coff = xoff * NT;                            // C-table bytes
-                for (int cl = 0; cl < g.my_chunks; ++cl) {
-                    cp_async_wait<S - 2>();
-                    __syncwarp();
-                    const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
-                    uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
-                    if (sasync) {
-                        sg = smq[(sc_o + so) >> 4];
-                        sg8 = smq[(sc_o + so + 8 * 16) >> 4];
-                    } else {
-                        bool v0, v1;
-                        const int c = g.my_wk + g.wk * cl;
-                        const int r0 = pass_slot_row(kind, N, g.o_end, o0, qg, v0);
-                        const int r1 = pass_slot_row(kind, N, g.o_end, o0, qg + 8, v1);
-                        uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                        const unsigned short *p0 =
-                            reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
-                        const unsigned short *p1 =
-                            reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
-                        for (int gl = 0; gl < kc; ++gl) {
-                            u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
-                            u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+                    uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
+                    uint32_t coff = xoff * NT;                            // C-table bytes
+                    for (int cl = 0; cl < g.my_chunks; ++cl) {
+                        cp_async_wait<S - 2>();
+                        __syncwarp();
+                        const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
+                        uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
+                        if (sasync) {
+                            const unsigned char *sp = smem + sc_o + so;
+                            sg = *reinterpret_cast<const uint4 *>(sp);
+                            sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
+                        } else {
+                            bool v0, v1;
+                            const int c = g.my_wk + g.wk * cl;
+                            const int r0 = pass_slot_row(kind, N, g.o_end, o0, qg, v0);
+                            const int r1 = pass_slot_row(kind, N, g.o_end, o0, qg + 8, v1);
+                            uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
+                            const unsigned short *p0 =
+                                reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
+                            const unsigned short *p1 =
+                                reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
+                            for (int gl = 0; gl < kc; ++gl) {
+                                u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
+                                u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                            }
+                            sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+                            sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
                         }
-                        sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-                        sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-                    }
-                    const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-                    const uint32_t wrow0 = wq_o + so;
-                    const uint32_t x70 = x7_o + coff;                 // + (gl * NT + nt) * 64
-                    uint32_t xbc[NT];
+                        const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+                        // shared-memory pointers of the item; the unrolled groups add constants
+                        const unsigned char *wp = smem + wq_o + so;
+                        const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64
+                        const unsigned char *bp[NT];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) xbc[nt] = xb[nt] + xoff;   // + gl * 64
-                    auto step = [&](int gl) {
-                        const uint32_t w0 = smw[(wrow0 + gl * 16) >> 2];
-                        const uint32_t w1 = smw[(wrow0 + 8 * kMRowStride + gl * 16) >> 2];
-                        const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                        const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
-                                                w1s & 0x000F000Fu};
-                        const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
-                                                w1s & 0x00F000F0u};
-                        const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                        const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                        const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                        const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
+                        for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
+                        auto step = [&](int gl) {
+                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wp + gl * 16);
+                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wp + 8 * kMRowStride + gl * 16);
+                            const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                            const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
+                                                    w1s & 0x000F000Fu};
+                            const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
+                                                    w1s & 0x00F000F0u};
+                            const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+                            const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+                            const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+                            const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
+                                const uint4 czu = *reinterpret_cast<const uint4 *>(cp + (gl * NT + nt) * 64);
+                                float d[4];
+                                mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
+                                          __uint_as_float(czu.z), __uint_as_float(czu.w));
+                                mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                                acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                                acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                                if (!ONE) {
+                                    acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                                    acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                                }
+                            }
+                        };
+                        if (kc == kMChunkG) {
+#pragma unroll
+                            for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
+                        } else {
+#pragma unroll
+                            for (int gl = 0; gl < kMChunkG; ++gl)
+                                if (gl < kc) step(gl);
+                        }
+                        __syncwarp();
+                        issue_next();
+                        so = (so + kMStage == (uint32_t)(S * kMStage)) ? 0u : so + kMStage;
+                        xoff += xstep;
+                        coff += cstep;
+                    }
+
+                    // ---- tile epilogue ----
+                    if (g.wk > 1) {
+                        // this warp's partial of tile t: [16 rows][8*NT columns]
+                        float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
-                            const uint4 bb = smq[(xbc[nt] + gl * 64) >> 4];
-                            const uint4 czu = smq[(x70 + (gl * NT + nt) * 64) >> 4];
-                            float d[4];
-                            mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
-                                      __uint_as_float(czu.z), __uint_as_float(czu.w));
-                            mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                            acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                            acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                            acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                            acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                            rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
+                            rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
+                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
+                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
                         }
-                    };
-                    if (kc == kMChunkG) {
-#pragma unroll
-                        for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
                     } else {
 #pragma unroll
-                        for (int gl = 0; gl < kMChunkG; ++gl)
-                            if (gl < kc) step(gl);
-                    }
-                    __syncwarp();
-                    issue_next();
-                    so = (so + kMStage == (uint32_t)(S * kMStage)) ? 0u : so + kMStage;
-                    xoff += xstep;
-                    coff += cstep;
-                }
-
-                // ---- tile epilogue ----
-                if (g.wk > 1) {
-                    // this warp's partial of tile t: [16 rows][8*NT columns]
-                    float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
+                        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
-                        rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
-                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
-                        rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
-                    }
-                } else {
+                            for (int e = 0; e < 2; ++e) {
+                                const int m = 8 * nt + 2 * qt + e;
+                                if (m >= M) continue;
+                                if (kind == kEpiGateUp) {
+                                    const int nn = o0 + qg;
+                                    if (nn < g.o_end) {
+                                        const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
+                                        const float silu = gv / (1.0f + expf(-gv));
+                                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
+                                    }
+                                } else {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int m = 8 * nt + 2 * qt + e;
-                            if (m >= M) continue;
-                            if (kind == kEpiGateUp) {
-                                const int nn = o0 + qg;
-                                if (nn < g.o_end) {
-                                    const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
-                                    const float silu = gv / (1.0f + expf(-gv));
-                                    reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
-                                }
-                            } else {
-#pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    const int nn = o0 + qg + 8 * h;
-                                    if (nn >= g.o_end) continue;
-                                    const float y = acc[nt][2 * h + e] * pow2f(24);
-                                    if (kind == kEpiF16) {
-                                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
-                                    } else {
-                                        reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
-                                        if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
-                                            best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
-                                            best_i[2 * nt + e] = nn;
+                                    for (int h = 0; h < 2; ++h) {
+                                        const int nn = o0 + qg + 8 * h;
+                                        if (nn >= g.o_end) continue;
+                                        const float y = acc[nt][2 * h + e] * pow2f(24);
+                                        if constexpr (!LOG) {
+                                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                                        } else {
+                                            reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
+                                            if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
+                                                best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
+                                                best_i[2 * nt + e] = nn;
+                                            }
                                         }
                                     }
                                 }
@@ -504,71 +517,73 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         }
                     }
                 }
-            }
 
-            if (g.wk > 1) {
-                // WK partials of each tile meet here; fixed summation order
-                __syncthreads();
-                const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
-                for (int idx = tid; idx < g.n_tiles * VO; idx += kMThreads) {
-                    const int t = idx / VO, vo = idx - (idx / VO) * VO;
-                    const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
-                    const int nn = g.o_begin + t * g.rout + r;
-                    if (nn >= g.o_end || m >= M) continue;
-                    const float *rp = red + (size_t)t * g.wk * kMTileRows * 8 * NT;
-                    float y = 0.f, u = 0.f;
-                    for (int k2 = 0; k2 < g.wk; ++k2) {
-                        y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
-                        if (kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
-                    }
-                    y *= pow2f(24);
-                    if (kind == kEpiF16) {
-                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
-                    } else if (kind == kEpiGateUp) {
-                        u *= pow2f(24);
-                        const float silu = y / (1.0f + expf(-y));
-                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
-                    } else {
-                        reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
-                        // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
-                        if (better(y, nn, best_v[0], best_i[0])) {
-                            best_v[0] = isnan(y) ? -INFINITY : y;
-                            best_i[0] = nn;
+                if (g.wk > 1) {
+                    // WK partials of each tile meet here; fixed summation order
+                    __syncthreads();
+                    const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
+                    for (int idx = tid; idx < g.n_tiles * VO; idx += kMThreads) {
+                        const int t = idx / VO, vo = idx - (idx / VO) * VO;
+                        const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
+                        const int nn = g.o_begin + t * g.rout + r;
+                        if (nn >= g.o_end || m >= M) continue;
+                        const float *rp = red + (size_t)t * g.wk * kMTileRows * 8 * NT;
+                        float y = 0.f, u = 0.f;
+                        for (int k2 = 0; k2 < g.wk; ++k2) {
+                            y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
+                            if (kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                        }
+                        y *= pow2f(24);
+                        if constexpr (LOG) {
+                            reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
+                            // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
+                            if (better(y, nn, best_v[0], best_i[0])) {
+                                best_v[0] = isnan(y) ? -INFINITY : y;
+                                best_i[0] = nn;
+                            }
+                        } else if (kind == kEpiF16) {
+                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                        } else {
+                            u *= pow2f(24);
+                            const float silu = y / (1.0f + expf(-y));
+                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
                         }
                     }
                 }
-            }
 
-            if (kind == kEpiLogits) {
-                __syncthreads();   // the maxima overwrite the partial buffer
+                if constexpr (LOG) {
+                    __syncthreads();   // the maxima overwrite the partial buffer
 #pragma unroll
-                for (int i = 0; i < 2 * NT; ++i) {
-                    bvs[tid * 2 * NT + i] = best_v[i];
-                    bis[tid * 2 * NT + i] = best_i[i];
-                }
-                __syncthreads();
-                if (tid < M) {
-                    float bv = -INFINITY;
-                    int bi = 0x7fffffff;
-                    for (int th = 0; th < kMThreads; ++th) {
-                        for (int i = 0; i < 2 * NT; ++i) {
-                            int tm;
-                            if (g.wk > 1) {
-                                if (i != 0) continue;
-                                tm = th % (8 * NT);
-                            } else {
-                                tm = 8 * (i >> 1) + 2 * (th & 3) + (i & 1);
-                            }
-                            if (tm == tid && better(bvs[th * 2 * NT + i], bis[th * 2 * NT + i], bv, bi)) {
-                                bv = bvs[th * 2 * NT + i];
-                                bi = bis[th * 2 * NT + i];
+                    for (int i = 0; i < 2 * NT; ++i) {
+                        bvs[tid * 2 * NT + i] = best_v[i];
+                        bis[tid * 2 * NT + i] = best_i[i];
+                    }
+                    __syncthreads();
+                    if (tid < M) {
+                        float bv = -INFINITY;
+                        int bi = 0x7fffffff;
+                        for (int th = 0; th < kMThreads; ++th) {
+                            for (int i = 0; i < 2 * NT; ++i) {
+                                int tm;
+                                if (g.wk > 1) {
+                                    if (i != 0) continue;
+                                    tm = th % (8 * NT);
+                                } else {
+                                    tm = 8 * (i >> 1) + 2 * (th & 3) + (i & 1);
+                                }
+                                if (tm == tid && better(bvs[th * 2 * NT + i], bis[th * 2 * NT + i], bv, bi)) {
+                                    bv = bvs[th * 2 * NT + i];
+                                    bi = bis[th * 2 * NT + i];
+                                }
                             }
                         }
+                        P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
+                        P.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
                     }
-                    P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-                    P.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
                 }
-            }
+            };
+            if (kind == kEpiLogits) run_segment(std::true_type{});
+            else run_segment(std::false_type{});
             __syncthreads();   // the activation area and partial buffers are free again
         }
         if (ph + 1 < nphase) {

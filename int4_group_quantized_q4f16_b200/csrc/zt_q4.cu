@@ -226,10 +226,10 @@ int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
 // ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
 constexpr int kNotResident = 1;   // launch_pass_s: this shape does not reach the wanted residency
 
-template <int NT, int PMAX, int S>
+template <int NT, int PMAX, int S, bool ONE>
 int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps)
 {
-    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S>);
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S, ONE>);
     int sms = 0;
     if (resident_ctas(fn, kMThreads, smem, sms) < cps) return kNotResident;
     cudaLaunchConfig_t cfg = {};
@@ -248,7 +248,7 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     clear_stale_error();
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S, ONE>, a);
     if (e != cudaSuccess) {
         g_last_cuda_error = e;
         (void)cudaGetLastError();
@@ -262,11 +262,11 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
 // Two CTAs per SM when the rings (2..4 stages) and the staged activations
 // fit in half the SM's shared memory, else one.  ZT_ERR_UNSUPPORTED if
 // neither fits.
-template <int NT, int PMAX>
+template <int NT, int PMAX, bool ONE>
 int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_out)
 {
     int sms = 0;
-    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2>), kMThreads, 0, sms) < 1)
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2, ONE>), kMThreads, 0, sms) < 1)
         return ZT_ERR_DEVICE;
     a.g_max = 0;
     for (int i = 0; i < a.n; ++i) a.g_max = std::max(a.g_max, a.p[i].G);
@@ -296,9 +296,9 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, a.n, NT);
         int rc;
         switch (stages) {
-        case 2: rc = launch_pass_s<NT, PMAX, 2>(a, cooperative, st, grid, smem, cps); break;
-        case 3: rc = launch_pass_s<NT, PMAX, 3>(a, cooperative, st, grid, smem, cps); break;
-        default: rc = launch_pass_s<NT, PMAX, 4>(a, cooperative, st, grid, smem, cps); break;
+        case 2: rc = launch_pass_s<NT, PMAX, 2, ONE>(a, cooperative, st, grid, smem, cps); break;
+        case 3: rc = launch_pass_s<NT, PMAX, 3, ONE>(a, cooperative, st, grid, smem, cps); break;
+        default: rc = launch_pass_s<NT, PMAX, 4, ONE>(a, cooperative, st, grid, smem, cps); break;
         }
         if (rc == kNotResident) continue;
         if (rc == ZT_OK && grid_out) *grid_out = grid;
@@ -328,7 +328,8 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.kind = kind;
     p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
     p.wait = 0;
-    return (q.M <= 8) ? launch_pass<1, 1>(a, false, st, grid_out) : launch_pass<2, 1>(a, false, st, grid_out);
+    if (q.M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
+    return (q.M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
 
 template <int EPI>
@@ -580,8 +581,9 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         return ZT_ERR_LAUNCH;
     }
     int grid = 0;
-    const int rc = (M <= 8) ? launch_pass<1, kPassMax>(a, cooperative, st, &grid)
-                            : launch_pass<2, kPassMax>(a, cooperative, st, &grid);
+    const int rc = M == 1   ? launch_pass<1, kPassMax, true>(a, cooperative, st, &grid)
+                   : M <= 8 ? launch_pass<1, kPassMax, false>(a, cooperative, st, &grid)
+                            : launch_pass<2, kPassMax, false>(a, cooperative, st, &grid);
     if (rc) return rc;
     for (int i = 0; i < n; ++i) {
         if (projs[i].kind != ZT_Q4_LM_HEAD) continue;
