@@ -482,7 +482,7 @@ def run_ours(args, world, rank, local):
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
     traffic = None
     try:
-        with open(os.path.join(ROOT, "profiles", "q4_mma_traffic.json")) as fh:
+        with open(os.path.join(ROOT, "profiles", "q4_pass_traffic.json")) as fh:
             tr = json.load(fh)
         if tr.get("kernel_sources_sha") == kernel_sources_sha():
             traffic = round(tr["dram_bytes_per_algorithmic_byte"] * kb)

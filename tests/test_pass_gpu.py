@@ -113,3 +113,79 @@ def test_pass_matches_single_calls(zt):
     single = zt.gemv(d["qw"], d["scales"], d["x"])
     torch.cuda.synchronize()
     assert np.array_equal(host(d["out"]).view(np.uint16), host(single).view(np.uint16))
+
+
+def test_pass_phases_mixed(zt, oracle):
+    """Phases of several independent projections, each later phase reading
+    outputs of earlier ones (wait set only on a phase's first projection);
+    an LM head in the middle; a ragged K (G % 8 != 0, scales not 16-byte
+    aligned rows) whose input is itself an earlier output."""
+    import torch
+    M = 2
+    a = _proj("gemv", 1056, 1024, M, 70, 0, scale_shift=2)        # -> x of c (K = 1056: 33 groups)
+    b = _proj("gemv", 768, 1024, M, 71, 1, scale_shift=2)         # -> x of d
+    lm = _proj("lm_head", 1000, 1024, M, 72, 2)
+    c = _proj("gemv", 2048, 1056, M, 73, 3, scale_shift=2)
+    d = _proj("gate_up", 256, 768, M, 74, 4, scale_shift=2)
+    e = _proj("gemv", 100, 2048, M, 75, 5, scale_shift=2)
+    f = _proj("gemv", 64, 256, M, 76, 6, scale_shift=2)
+    c["x"], d["x"], e["x"], f["x"] = a["out"], b["out"], c["out"], d["out"]
+    c["wait"] = 1          # phase 1: c, d
+    e["wait"] = 1          # phase 2: e, f
+    projs = [a, b, lm, c, d, e, f]
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for q in (a, b, lm):
+        _check_against_oracle(oracle, q)
+    for q, src in ((c, a), (d, b), (e, c), (f, d)):
+        _check_against_oracle(oracle, q, x_host=host(src["out"]).astype(np.float16))
+
+
+def test_pass_many_small_projections(zt, oracle):
+    """150 small projections (8..70 outputs, K from one group to a ragged 33
+    groups): every CTA's share spans many segments."""
+    import torch
+    rng = np.random.default_rng(5)
+    kinds = ["gemv", "gemv", "gate_up", "gemv"]
+    Ks = [32, 96, 288, 1056, 256]
+    projs = []
+    for i in range(150):
+        kind = kinds[i % 4]
+        projs.append(_proj(kind, int(rng.integers(8, 71)), Ks[i % 5], 1, 300 + i, i % 5))
+    projs[77] = _proj("lm_head", 333, 96, 1, 999, 4)
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for d in projs:
+        _check_against_oracle(oracle, d)
+
+
+@pytest.mark.parametrize("M", [2, 5, 8, 9, 16])
+def test_pass_batch_sweep(zt, oracle, M):
+    """M = 2..16: the single-column kernel is not used, one or two n-tiles."""
+    import torch
+    shapes = [("gemv", 300, 1024), ("gate_up", 200, 1024), ("lm_head", 777, 512), ("gemv", 64, 3072)]
+    projs = [_proj(k, N, K, M, 500 + i, i) for i, (k, N, K) in enumerate(shapes)]
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for d in projs:
+        _check_against_oracle(oracle, d)
+
+
+@pytest.mark.parametrize("N", [1, 3, 17])
+def test_pass_fewer_rows_than_ctas(zt, oracle, N):
+    """A list smaller than the grid: CTAs without rows still write neutral
+    LM-head partial maxima."""
+    import torch
+    projs = [_proj("gemv", N, 256, 1, 600 + N, 0), _proj("lm_head", N, 256, 1, 601 + N, 1)]
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for d in projs:
+        _check_against_oracle(oracle, d)
