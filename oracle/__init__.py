@@ -11,7 +11,9 @@ Each wrapper names the passage the C function follows:
 * dequantizing matrix product and f32 LM head -- Zero-TVM forum write-up,
   section "完整的推理流水线" (int4 反量化矩阵乘法; f32 output for the LM head);
 * fused gate/up + SiLU -- same write-up, section "内核融合" (fused_ffn.wgsl);
-* greedy argmax -- same write-up, section "完整的推理流水线" (贪婪解码采样).
+* greedy argmax -- same write-up, section "完整的推理流水线" (贪婪解码采样);
+* residual add + RMSNorm -- same write-up, section "内核融合" (add_norm.wgsl),
+  read as the standard RMSNorm on the fp16 residual stream.
 
 Format reading (the pages name "q4f16_1" but give no bit layout): group of 32
 along K, fp16 scale per group, 8 codes per uint32 low nibble first,
@@ -89,8 +91,11 @@ class Oracle:
         lib.zto_argmax.argtypes = [_P, _I]
         lib.zto_argmax.restype = ctypes.c_int32
         lib.zto_lmhead_argmax.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P, _I]
+        lib.zto_double_to_half.argtypes = [ctypes.c_double]
+        lib.zto_double_to_half.restype = ctypes.c_uint16
+        lib.zto_add_rmsnorm.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
         for f in (lib.zto_unpack, lib.zto_pack, lib.zto_gemv,
-                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax):
+                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm):
             f.restype = ctypes.c_int
         self._lib = lib
 
@@ -99,6 +104,12 @@ class Oracle:
         h = _u16(h)
         f = self._lib.zto_half_to_double
         return np.array([f(int(v)) for v in h.ravel()], dtype=np.float64).reshape(h.shape)
+
+    def double_to_half(self, v) -> np.ndarray:
+        """double -> fp16 bit patterns (uint16), round to nearest even."""
+        v = np.asarray(v, dtype=np.float64)
+        f = self._lib.zto_double_to_half
+        return np.array([f(float(a)) for a in v.ravel()], dtype=np.uint16).reshape(v.shape)
 
     def unpack(self, qw: np.ndarray, K: int) -> np.ndarray:
         qw = np.ascontiguousarray(qw, dtype=np.uint32)
@@ -159,6 +170,25 @@ class Oracle:
         if rc:
             raise ValueError("zto_gate_up_silu rejected its arguments")
         return out
+
+    def add_rmsnorm(self, residual, delta, gamma, eps: float):
+        """(h, x) as fp16 arrays [M][K]: h = fp16(residual + delta),
+        x = fp16(h * gamma / sqrt(mean_k h^2 + eps)); delta may be None."""
+        r = _u16(np.atleast_2d(residual))
+        M, K = r.shape
+        d = _u16(np.atleast_2d(delta)) if delta is not None else None
+        if d is not None and d.shape != r.shape:
+            raise ValueError("delta must have the residual's shape")
+        g = _u16(gamma).ravel()
+        if g.size != K:
+            raise ValueError("gamma must have K entries")
+        h = np.empty((M, K), dtype=np.uint16)
+        x = np.empty((M, K), dtype=np.uint16)
+        rc = self._lib.zto_add_rmsnorm(_ptr(r), _ptr(d) if d is not None else None, _ptr(g), M, K,
+                                       float(eps), _ptr(h), _ptr(x))
+        if rc:
+            raise ValueError("zto_add_rmsnorm rejected its arguments")
+        return h.view(np.float16), x.view(np.float16)
 
     def silu(self, g: float) -> float:
         return self._lib.zto_silu(float(g))

@@ -31,6 +31,12 @@
  *   simple argmax dispatch"): logits = y kept in double; argmax = the lowest
  *   index among the maxima, NaN treated as -infinity.
  *
+ *   residual add + RMSNorm ("add_norm.wgsl": the residual connection and
+ *   RMSNorm in one step, section "内核融合"; the pages give no formula, so
+ *   the standard RMSNorm is read): per row m, h = fp16(residual + delta)
+ *   (the residual stream stays fp16), x = fp16(h * gamma / sqrt(mean_k h^2 +
+ *   eps)).  x is then the input of the next projection.
+ *
  * Every function computes each output row with the same fixed sequence of
  * operations, so the optional OpenMP split over rows (threads > 1) returns
  * bit-identical results to the single-threaded run.
@@ -196,5 +202,66 @@ int zto_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16_t
     if (rc) return rc;
     for (int64_t m = 0; m < M; ++m)
         argmax[m] = zto_argmax(logits + m * N, N);
+    return 0;
+}
+
+/* double -> IEEE-754 binary16 bit pattern, round to nearest, ties to even,
+ * written out from the format: in the binade [2^e, 2^(e+1)) (e >= -14; below
+ * that the subnormal spacing 2^-24 continues) representable values are
+ * spaced 2^(e-10), so the value is rounded to an integer count of spacings.
+ * Values that round above 65504 (the largest finite) become infinity; NaN
+ * becomes the quiet NaN 0x7E00. */
+uint16_t zto_double_to_half(double v)
+{
+    const uint16_t sign = signbit(v) ? 0x8000 : 0;
+    if (isnan(v)) return 0x7E00;
+    const double a = fabs(v);
+    if (isinf(a)) return sign | 0x7C00;
+    if (a == 0.0) return sign;
+    int E;
+    (void)frexp(a, &E);                 /* a in [2^(E-1), 2^E) */
+    int e = E - 1;
+    if (e < -14) e = -14;               /* subnormals share the spacing of binade -14 */
+    const double units = ldexp(a, 10 - e);          /* a / 2^(e-10), exact */
+    double r = floor(units);
+    const double frac = units - r;                  /* exact */
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    if (ldexp(r, e - 10) > 65504.0) return sign | 0x7C00;
+    int64_t ri = (int64_t)r;
+    if (ri == 2048) {                   /* rounded up into the next binade */
+        ri = 1024;
+        e += 1;
+    }
+    if (ri < 1024) return sign | (uint16_t)ri;      /* subnormal (e == -14) */
+    return sign | (uint16_t)((e + 15) << 10) | (uint16_t)(ri - 1024);
+}
+
+/* Residual add + RMSNorm over rows of [M][K] fp16:
+ *   h[m][k] = fp16(residual[m][k] + delta[m][k])     (delta == NULL: h = residual)
+ *   r[m]    = 1 / sqrt((sum_k h[m][k]^2) / K + eps)   (k in plain order, double)
+ *   x[m][k] = fp16(h[m][k] * r[m] * gamma[k])
+ * h_out (may be NULL) receives h, x_out receives x (fp16 bit patterns). */
+int zto_add_rmsnorm(const uint16_t *residual, const uint16_t *delta, const uint16_t *gamma,
+                    int M, int K, double eps, uint16_t *h_out, uint16_t *x_out)
+{
+    if (!residual || !gamma || !x_out || M < 1 || K < 1 || !(eps >= 0.0)) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double h = zto_half_to_double(residual[m * K + k]);
+            if (delta) h += zto_half_to_double(delta[m * K + k]);   /* exact: two fp16 values */
+            const uint16_t hb = zto_double_to_half(h);
+            if (h_out) h_out[m * K + k] = hb;
+            const double hd = zto_half_to_double(hb);
+            ss += hd * hd;
+        }
+        const double r = 1.0 / sqrt(ss / (double)K + eps);
+        for (int64_t k = 0; k < K; ++k) {
+            double h = zto_half_to_double(residual[m * K + k]);
+            if (delta) h += zto_half_to_double(delta[m * K + k]);
+            const double hd = zto_half_to_double(zto_double_to_half(h));
+            x_out[m * K + k] = zto_double_to_half(hd * r * zto_half_to_double(gamma[k]));
+        }
+    }
     return 0;
 }

@@ -292,4 +292,105 @@ def pin_golden(o):
             assert np.array_equal(am, c["argmax"]), f"golden {c['name']} argmax"
 
 
+# ------------------------------------------------ residual add + RMSNorm ----
+# add_norm.wgsl (Zero-TVM write-up, section "内核融合"): the residual add and
+# RMSNorm in one step; read as h = fp16(residual + delta),
+# x = fp16(h * gamma / sqrt(mean h^2 + eps)).
+
+def _f16(v):
+    return np.asarray(v, dtype=np.float64).astype(np.float16)
+
+
+def pin_double_to_half_is_ieee_round_to_nearest_even(o):
+    """Against numpy's double -> binary16 conversion, including exact ties
+    (midpoints of adjacent fp16 values), subnormals and the overflow edge."""
+    rng = np.random.default_rng(17)
+    v = rng.standard_normal(4000) * 10.0 ** rng.integers(-8, 5, 4000)
+    a = rng.integers(0, 0x7BFF, 2000, dtype=np.uint16).view(np.float16).astype(np.float64)
+    b = (rng.integers(0, 0x7BFF, 2000, dtype=np.uint16) ).view(np.float16).astype(np.float64)
+    nxt = np.nextafter(a.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+    ties = (a + nxt) / 2.0                        # exact in double
+    edge = np.array([0.0, -0.0, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14, 65504.0,
+                     65519.0, 65520.0, 65536.0, 1e30, -65520.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11])
+    vals = np.concatenate([v, -v, ties, -ties, b, edge])
+    with np.errstate(over="ignore"):
+        ref = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(o.double_to_half(vals), ref)
+
+
+def pin_rmsnorm_constant_row_gives_gamma(o):
+    """A constant row c with eps = 0 normalises to exactly +-1: x = +-gamma
+    (gamma varies with k, so a wrong gamma index shows)."""
+    K = 64
+    gamma = _f16(np.linspace(-3.0, 5.0, K))
+    for c in (1.5, -0.375, 96.0):
+        h, x = o.add_rmsnorm(_f16(np.full((1, K), c)), None, gamma, 0.0)
+        assert np.array_equal(h, _f16(np.full((1, K), c)))
+        assert np.array_equal(x[0].astype(np.float64), np.sign(c) * gamma.astype(np.float64))
+
+
+def pin_rmsnorm_closed_form_ones_and_sevens(o):
+    """K = 32: sixteen 1s and sixteen 7s: mean h^2 = (16 + 784) / 32 = 25, so
+    with eps = 0 and gamma = 5 the output is h itself.  The row is split as
+    residual + delta (both exact in fp16)."""
+    h = np.array([1.0] * 16 + [7.0] * 16)
+    res = _f16(h - 0.5)
+    dlt = _f16(np.full(32, 0.5))
+    got_h, x = o.add_rmsnorm(res[None, :], dlt[None, :], _f16(np.full(32, 5.0)), 0.0)
+    assert np.array_equal(got_h[0].astype(np.float64), h)
+    assert np.array_equal(x[0].astype(np.float64), h)
+
+
+def pin_rmsnorm_eps_inside_sqrt(o):
+    """h = 2^-7 everywhere, eps = 3 * 2^-14: mean h^2 + eps = 2^-12, its root
+    2^-6, so x = gamma / 2 exactly."""
+    K = 32
+    gamma = _f16(np.arange(1, K + 1) * 0.25)
+    _, x = o.add_rmsnorm(_f16(np.full((1, K), 2.0 ** -7)), None, gamma, 3 * 2.0 ** -14)
+    assert np.array_equal(x[0].astype(np.float64), gamma.astype(np.float64) / 2)
+
+
+def pin_rmsnorm_scale_invariant(o):
+    """eps = 0: scaling the residual by 2^j scales sum h^2 by 4^j and the root
+    by 2^j, all exactly, so x does not change."""
+    rng = np.random.default_rng(3)
+    res = _f16(rng.standard_normal((2, 96)))
+    gamma = _f16(rng.uniform(0.5, 2.0, 96))
+    _, x0 = o.add_rmsnorm(res, None, gamma, 0.0)
+    for j in (-3, 4):
+        _, xj = o.add_rmsnorm(_f16(res.astype(np.float64) * 2.0 ** j), None, gamma, 0.0)
+        assert np.array_equal(x0.view(np.uint16), xj.view(np.uint16))
+
+
+def pin_rmsnorm_residual_rounded_to_fp16(o):
+    """h is the fp16 sum: 1 + 2^-11 is a tie between 1 and 1 + 2^-10 and goes
+    to the even 1; (1 + 2^-10) + 2^-11 goes up to 1 + 2^-9.  delta = -residual
+    gives +0 and, with eps > 0, x = 0."""
+    K = 32
+    res = _f16(np.array([1.0] * 16 + [1.0 + 2.0 ** -10] * 16))
+    dlt = _f16(np.full(K, 2.0 ** -11))
+    h, _ = o.add_rmsnorm(res[None, :], dlt[None, :], _f16(np.ones(K)), 1e-5)
+    assert np.array_equal(h[0].astype(np.float64), np.array([1.0] * 16 + [1.0 + 2.0 ** -9] * 16))
+    h, x = o.add_rmsnorm(res[None, :], (-res)[None, :], _f16(np.ones(K)), 1e-5)
+    assert np.array_equal(h.view(np.uint16), np.zeros((1, K), dtype=np.uint16))
+    assert np.array_equal(x.view(np.uint16), np.zeros((1, K), dtype=np.uint16))
+
+
+def pin_rmsnorm_rows_independent(o):
+    """Each row is normalised by its own mean square: a batch equals its rows
+    one at a time, and rows of different scale keep their own result."""
+    rng = np.random.default_rng(4)
+    res = _f16(rng.standard_normal((3, 64)) * np.array([[0.01], [1.0], [300.0]]))
+    dlt = _f16(rng.standard_normal((3, 64)))
+    gamma = _f16(rng.uniform(0.5, 2.0, 64))
+    h, x = o.add_rmsnorm(res, dlt, gamma, 1e-5)
+    for m in range(3):
+        hm, xm = o.add_rmsnorm(res[m:m + 1], dlt[m:m + 1], gamma, 1e-5)
+        assert np.array_equal(hm.view(np.uint16), h[m:m + 1].view(np.uint16))
+        assert np.array_equal(xm.view(np.uint16), x[m:m + 1].view(np.uint16))
+    # |x| has unit mean square before gamma: sum (x / gamma)^2 / K ~ 1 in every row
+    ms = np.mean((x.astype(np.float64) / gamma.astype(np.float64)) ** 2, axis=1)
+    assert np.all(np.abs(ms - 1.0) < 2e-3), ms
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -33,6 +33,16 @@ MUTANTS = [
     ("pack_high_nibble_first", "word |= (uint32_t)c << (4 * j);",
      "word |= (uint32_t)c << (4 * (7 - j));"),
     ("x_row_stride", "zto_half_to_double(x[m * K + k])", "zto_half_to_double(x[k])"),
+    ("rmsnorm_eps_outside_sqrt", "1.0 / sqrt(ss / (double)K + eps)", "1.0 / (sqrt(ss / (double)K) + eps)"),
+    ("rmsnorm_sum_not_mean", "1.0 / sqrt(ss / (double)K + eps)", "1.0 / sqrt(ss + eps)"),
+    ("rmsnorm_gamma_dropped", "hd * r * zto_half_to_double(gamma[k])", "hd * r"),
+    ("rmsnorm_gamma_reversed", "hd * r * zto_half_to_double(gamma[k])", "hd * r * zto_half_to_double(gamma[K - 1 - k])"),
+    ("rmsnorm_delta_ignored_in_h", "if (h_out) h_out[m * K + k] = hb;",
+     "if (h_out) h_out[m * K + k] = residual[m * K + k];"),
+    ("rmsnorm_rows_share_one_sum", "    for (int64_t m = 0; m < M; ++m) {\n        double ss = 0.0;",
+     "    double ss = 0.0;\n    for (int64_t m = 0; m < M; ++m) {"),
+    ("half_rounding_ties_away", "(frac == 0.5 && fmod(r, 2.0) != 0.0)", "(frac == 0.5)"),
+    ("half_subnormal_spacing", "if (e < -14) e = -14;", "if (e < -15) e = -15;"),
     ("sampled_rows_ignored", "int64_t n = rows ? rows[i] : i;\n        for (int64_t m = 0; m < M; ++m)\n            y[",
      "int64_t n = i;\n        for (int64_t m = 0; m < M; ++m)\n            y["),
 ]
