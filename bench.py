@@ -357,6 +357,43 @@ def run_ours(args, world, rank, local):
     chained_us = c0.elapsed_time(c1) / ch_steps * 1e3
     assert zchain.errors() == 0, "a bounded wait of the chained pass expired"
 
+    # ---- the pass with residual add + RMSNorm prologues on every qkv and
+    # gate_up projection (x computed while staging), for comparison ----
+    def make_norm_pass():
+        projs, gen = [], torch.Generator(device=device).manual_seed(args.seed)
+        for d in calls:
+            e = {"kind": d["p"].kind, "qw": d["qw"], "scales": d["s"], "x": d["x"], "out": d["y"]}
+            if d["p"].kind == "lm_head":
+                e["argmax"] = d["am"]
+            if d["p"].name in ("qkv", "gate_up"):
+                K = d["p"].K
+                e["norm"] = {"residual": torch.randn((1, K), generator=gen, device=device).half(),
+                             "delta": torch.randn((1, K), generator=gen, device=device).half(),
+                             "gamma": torch.rand((K,), generator=gen, device=device).half() + 0.5,
+                             "eps": 1e-5}
+            projs.append(e)
+        return zt_q4.Pass(projs)
+
+    def time_pass(pz, steps):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                pz.run(stream)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(steps):
+                pz.run(stream)
+            t1.record(stream)
+            stream.synchronize()
+        return t0.elapsed_time(t1) / steps * 1e3
+
+    znorm = make_norm_pass()
+    nm_steps = max(1, min(args.steps, 200))
+    # the plain pass and the pass with prologues, back to back, same length
+    plain_us_short = time_pass(zpass, nm_steps)
+    norm_us = time_pass(znorm, nm_steps)
+    assert znorm.errors() == 0
+
     # ---- the same pass as 130 separate calls (graph + PDL), for comparison ----
     def capture(fn):
         with torch.cuda.stream(stream):
@@ -509,6 +546,10 @@ def run_ours(args, world, rank, local):
                          "duration": "mean of the event-bracketed zt_q4_pass calls of the timed region "
                                      "(pass kernel + argmax reduction)"},
             "chained_us_per_pass": round(chained_us, 2),
+            "add_rmsnorm_prologue": {"us_per_pass": round(norm_us, 2), "plain_us_per_pass": round(plain_us_short, 2),
+                                     "steps": nm_steps,
+                                     "what": "64 residual add + RMSNorm prologues (every qkv and gate_up), x computed "
+                                             "while staging; timed back to back with the plain pass"},
             "per_call_graph_us_per_pass": round(per_call_us, 2),
             "per_projection_us_isolated": per_kind_us,
             "cpu_baseline": cpu,

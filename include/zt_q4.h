@@ -174,15 +174,43 @@ ZT_API int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scale
 #define ZT_Q4_LM_HEAD 2
 #define ZT_Q4_PASS_MAX 160
 
+/*
+ * Optional prologue of a pass projection: residual add + RMSNorm (Zero-TVM
+ * write-up, "内核融合": add_norm.wgsl joins the residual connection and the
+ * RMSNorm layer normalisation; the pages give no formula, the standard RMSNorm
+ * on the fp16 residual stream is read).  The projection's x is then not read;
+ * instead, per row m (token) of [M][K]:
+ *
+ *   h[m][k] = fp16(residual[m][k] + delta[m][k])      (delta NULL: h = residual)
+ *   x[m][k] = fp16(h[m][k] * gamma[k] / sqrt(sum_k h[m][k]^2 / K + eps))
+ *
+ * (h * gamma * r in fp32, the sum of squares in fp32, one rounding to fp16 at
+ * the end, so an element can differ from the exactly rounded value by one
+ * fp16 ulp.)  The kernel computes x while staging the projection's
+ * activations -- no separate launch, x never goes through HBM.  h and x can be
+ * written out (residual_out, x_out), once, by one CTA.  All pointers are
+ * device memory, 16-byte aligned; residual_out must not overlap residual or
+ * delta; a later projection that reads residual_out needs `wait`.
+ */
+typedef struct zt_q4_norm {
+    const uint16_t *residual; /* [M][K] fp16 */
+    const uint16_t *delta;    /* [M][K] fp16, or NULL */
+    const uint16_t *gamma;    /* [K] fp16 */
+    uint16_t *residual_out;   /* [M][K] fp16 receives h, or NULL */
+    uint16_t *x_out;          /* [M][K] fp16 receives x, or NULL */
+    float eps;                /* >= 0, finite */
+} zt_q4_norm;
+
 typedef struct zt_q4_proj {
     const uint32_t *qw;       /* [n_rows][K/8], n_rows = N (2N for GATE_UP_SILU) */
     const uint16_t *scales;   /* [n_rows][K/32] fp16 */
-    const uint16_t *x;        /* [M][K] fp16 */
+    const uint16_t *x;        /* [M][K] fp16 (ignored, may be NULL, when norm is set) */
     void *out;                /* fp16 [M][N], or f32 [M][N] logits for LM_HEAD */
     int32_t *argmax;          /* LM_HEAD: [M]; ignored otherwise */
     int kind;                 /* ZT_Q4_GEMV, ZT_Q4_GATE_UP_SILU or ZT_Q4_LM_HEAD */
     int N, K;
     int wait;                 /* read x only after all earlier projections completed */
+    const zt_q4_norm *norm;   /* HOST pointer to the prologue, or NULL (read during the call) */
 } zt_q4_proj;
 
 ZT_API size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M);

@@ -177,4 +177,96 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
     }
 }
 
+// Residual add + RMSNorm ahead of a projection (the pages' add_norm step:
+// residual connection and RMSNorm in one kernel), staged like stage_x_mma:
+//   h = fp16(res + dlt) (dlt may be null), r = 1 / sqrt(sum_k h^2 / K + eps)
+//   per row, x = fp16(h * r * gamma).
+// Pass 1 writes h into the activation area (plain order) and sums squares
+// (fp32, fixed order: per-thread strided sums, warp butterfly, warps in
+// order); pass 2 turns each thread's own 16 bytes of h into x in the mma-B
+// order.  res_out / x_out (plain [M][K] fp16) are written when non-null.
+// scratch: kMW + M floats of shared memory.  All threads of the CTA call it.
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
+{
+    __half2 r = __hadd2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dlt, const __half *gamma, float eps,
+                                             __half *res_out, __half *x_out, unsigned char *xp, float *x7,
+                                             float *scratch, int M, int K, int G, int NT)
+{
+    const int K8 = K >> 3;
+    const size_t nstride = (size_t)G * 64 + 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int m = 0; m < M; ++m) {
+        float part = 0.f;
+        for (int kk = threadIdx.x; kk < K8; kk += kMThreads) {
+            uint4 h = __ldcg(reinterpret_cast<const uint4 *>(res + (size_t)m * K + 8 * kk));
+            if (dlt) {
+                const uint4 d = __ldcg(reinterpret_cast<const uint4 *>(dlt + (size_t)m * K + 8 * kk));
+                h.x = hadd2_u32(h.x, d.x);
+                h.y = hadd2_u32(h.y, d.y);
+                h.z = hadd2_u32(h.z, d.z);
+                h.w = hadd2_u32(h.w, d.w);
+            }
+            *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = h;
+            if (res_out) *reinterpret_cast<uint4 *>(res_out + (size_t)m * K + 8 * kk) = h;
+            const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(hh[j]);
+                part = fmaf(f.x, f.x, part);
+                part = fmaf(f.y, f.y, part);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) scratch[warp] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float ss = 0.f;
+            for (int w = 0; w < kMW; ++w) ss += scratch[w];
+            scratch[kMW + m] = 1.0f / sqrtf(ss / (float)K + eps);
+        }
+        __syncthreads();
+    }
+    const int total = M * K8;
+    const int pad = 8 * NT - M;
+    for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
+        const int g = j / pad, m = M + (j - (j / pad) * pad);
+        const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+        float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+        cv[e] = 0.f;
+        cv[2 + e] = 0.f;
+    }
+    auto normalise = [&](int m, int kk) {
+        const uint4 h = *reinterpret_cast<const uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16);
+        const uint4 g = __ldcg(reinterpret_cast<const uint4 *>(gamma + 8 * kk));
+        const float r = scratch[kMW + m];
+        const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
+        const __half2 *gg = reinterpret_cast<const __half2 *>(&g);
+        uint4 x;
+        __half2 *xx = reinterpret_cast<__half2 *>(&x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 hf = __half22float2(hh[j]), gf = __half22float2(gg[j]);
+            xx[j] = __floats2half2_rn(hf.x * r * gf.x, hf.y * r * gf.y);
+        }
+        if (x_out) *reinterpret_cast<uint4 *>(x_out + (size_t)m * K + 8 * kk) = x;
+        return x;
+    };
+    for (int base = 0; base < total; base += 2 * kMThreads) {
+        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+        const bool v0 = i0 < total, v1 = i1 < total;
+        const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
+        const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
+        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+        if (v0) r0 = normalise(m0, k0);
+        if (v1) r1 = normalise(m1, k1);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT);
+        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT);
+    }
+}
+
 }  // namespace zt

@@ -52,6 +52,12 @@ struct PassProj {
     int scales_async;           // scales copied by cp.async (16-byte aligned rows)
     int phase;                  // index of the projection's phase
     int wait;                   // starts a phase: wait for all earlier projections
+    // residual add + RMSNorm prologue (norm != 0): x = fp16(h * gamma / rms(h)),
+    // h = fp16(res + dlt); res_out / x_out receive h / x (the CTA holding row 0)
+    const __half *res, *dlt, *gamma;
+    __half *res_out, *x_out;
+    float eps;
+    int norm;
 };
 
 // PMAX bounds the list: 1 for the single-call entry points (a small kernel
@@ -362,7 +368,13 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const int G = P.G, N = P.N, kind = P.kind;
             const bool sasync = P.scales_async;
             void *const out = P.out;
-            stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
+            if (P.norm) {
+                const bool writer = sgm.o_begin == 0;   // exactly one CTA holds row 0
+                stage_x_norm(P.res, P.dlt, P.gamma, P.eps, writer ? P.res_out : nullptr,
+                             writer ? P.x_out : nullptr, xp, x7, red, M, P.K, G, NT);
+            } else {
+                stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
+            }
             __syncthreads();
 
             const uint32_t nstride = (uint32_t)G * 64u + 32u;

@@ -328,6 +328,10 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.kind = kind;
     p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
     p.wait = 0;
+    p.norm = 0;
+    p.res = p.dlt = p.gamma = nullptr;
+    p.res_out = p.x_out = nullptr;
+    p.eps = 0.f;
     if (q.M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
     return (q.M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
@@ -412,7 +416,7 @@ void *noalloc_scratch()
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 0; }
+int zt_q4_version(void) { return (1 << 16) | 1; }
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -530,11 +534,24 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
     bool cooperative = false;
     for (int i = 0; i < n; ++i) {
         const zt_q4_proj &q = projs[i];
-        if (!q.qw || !q.scales || !q.x || !q.out) return ZT_ERR_INVALID_ARG;
+        if (!q.qw || !q.scales || !q.out || (!q.x && !q.norm)) return ZT_ERR_INVALID_ARG;
         if (q.kind != ZT_Q4_GEMV && q.kind != ZT_Q4_GATE_UP_SILU && q.kind != ZT_Q4_LM_HEAD) return ZT_ERR_INVALID_ARG;
         if (q.kind == ZT_Q4_LM_HEAD && !q.argmax) return ZT_ERR_INVALID_ARG;
         const int rc = check_shapes(M, q.N, q.K, q.kind == ZT_Q4_GATE_UP_SILU ? 2 : 1);
         if (rc) return rc;
+        if (q.norm) {
+            const zt_q4_norm &nm = *q.norm;
+            if (!nm.residual || !nm.gamma || !(nm.eps >= 0.f) || nm.eps > 3.0e38f) return ZT_ERR_INVALID_ARG;
+            if (!aligned(nm.residual, 16) || !aligned(nm.delta, 16) || !aligned(nm.gamma, 16) ||
+                !aligned(nm.residual_out, 16) || !aligned(nm.x_out, 16))
+                return ZT_ERR_MISALIGNED;
+            const uintptr_t bytes = (uintptr_t)M * (uintptr_t)q.K * 2;
+            auto overlap = [bytes](const void *a, const void *b) {
+                const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+                return a && b && pa < pb + bytes && pb < pa + bytes;
+            };
+            if (overlap(nm.residual_out, nm.residual) || overlap(nm.residual_out, nm.delta)) return ZT_ERR_INVALID_ARG;
+        }
         if (!aligned(q.qw, 16) || !aligned(q.x, 16) || !aligned(q.scales, 2) ||
             !aligned(q.out, q.kind == ZT_Q4_LM_HEAD ? 4 : 2) || (q.argmax && !aligned(q.argmax, 4)))
             return ZT_ERR_MISALIGNED;
@@ -564,6 +581,13 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         p.kind = q.kind == ZT_Q4_GEMV ? kEpiF16 : q.kind == ZT_Q4_GATE_UP_SILU ? kEpiGateUp : kEpiLogits;
         p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
         p.wait = (i > 0 && q.wait) ? 1 : 0;
+        p.norm = q.norm ? 1 : 0;
+        p.res = q.norm ? reinterpret_cast<const __half *>(q.norm->residual) : nullptr;
+        p.dlt = q.norm ? reinterpret_cast<const __half *>(q.norm->delta) : nullptr;
+        p.gamma = q.norm ? reinterpret_cast<const __half *>(q.norm->gamma) : nullptr;
+        p.res_out = q.norm ? reinterpret_cast<__half *>(q.norm->residual_out) : nullptr;
+        p.x_out = q.norm ? reinterpret_cast<__half *>(q.norm->x_out) : nullptr;
+        p.eps = q.norm ? q.norm->eps : 0.f;
         p.ws_val = nullptr;
         p.ws_idx = nullptr;
         if (q.kind == ZT_Q4_LM_HEAD) {

@@ -41,11 +41,18 @@ ZT_Q4_LM_HEAD = 2
 ZT_Q4_PASS_MAX = 160
 
 
+class ZtNorm(ctypes.Structure):
+    """struct zt_q4_norm of include/zt_q4.h (residual add + RMSNorm prologue)"""
+    _fields_ = [("residual", ctypes.c_void_p), ("delta", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("residual_out", ctypes.c_void_p), ("x_out", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 class ZtProj(ctypes.Structure):
     """struct zt_q4_proj of include/zt_q4.h"""
     _fields_ = [("qw", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("argmax", ctypes.c_void_p), ("kind", ctypes.c_int),
-                ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int)]
+                ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int),
+                ("norm", ctypes.POINTER(ZtNorm))]
 
 
 def _load() -> ctypes.CDLL:
@@ -209,8 +216,11 @@ class Pass:
 
     Each entry is a dict with torch CUDA tensors: kind ("gemv", "gate_up",
     "lm_head"), qw, scales, x, out (and argmax for "lm_head"), and optional
-    wait (read x only after all earlier projections completed).  The
-    ctypes array and the workspace are built once; run() only launches."""
+    wait (read x only after all earlier projections completed).  An optional
+    "norm" dict turns on the residual add + RMSNorm prologue (x is then not
+    read and may be omitted): residual, gamma, eps, and optionally delta,
+    residual_out, x_out.  The ctypes arrays and the workspace are built once;
+    run() only launches."""
 
     KINDS = {"gemv": ZT_Q4_GEMV, "gate_up": ZT_Q4_GATE_UP_SILU, "lm_head": ZT_Q4_LM_HEAD}
 
@@ -220,21 +230,39 @@ class Pass:
             raise ValueError(f"a pass has 1..{ZT_Q4_PASS_MAX} projections")
         self._keep = projs
         arr = (ZtProj * len(projs))()
+        self._norms = []
         M = None
         for i, p in enumerate(projs):
             kind = self.KINDS[p["kind"]]
-            m, n, k = _dims(p["qw"], p["scales"], p["x"], 2 if kind == ZT_Q4_GATE_UP_SILU else 1)
+            nm = p.get("norm")
+            xs = p.get("x") if nm is None else nm["residual"]
+            m, n, k = _dims(p["qw"], p["scales"], xs, 2 if kind == ZT_Q4_GATE_UP_SILU else 1)
             if M is None:
                 M = m
             elif m != M:
                 raise ValueError("all projections of a pass share M")
             am = p.get("argmax")
-            arr[i] = ZtProj(p["qw"].data_ptr(), p["scales"].data_ptr(), p["x"].data_ptr(), p["out"].data_ptr(),
-                            am.data_ptr() if am is not None else None, kind, n, k, int(bool(p.get("wait", 0))))
+            norm_ptr = None
+            if nm is not None:
+                def ptr(key, numel):
+                    t = nm.get(key)
+                    if t is None:
+                        return None
+                    if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float16 or t.numel() != numel:
+                        raise ValueError(f"norm {key} must be a contiguous CUDA float16 tensor of {numel} elements")
+                    return t.data_ptr()
+                z = ZtNorm(ptr("residual", m * k), ptr("delta", m * k), ptr("gamma", k),
+                           ptr("residual_out", m * k), ptr("x_out", m * k), float(nm.get("eps", 1e-5)))
+                self._norms.append(z)
+                norm_ptr = ctypes.pointer(z)
+            x = p.get("x")
+            arr[i] = ZtProj(p["qw"].data_ptr(), p["scales"].data_ptr(), x.data_ptr() if x is not None else None,
+                            p["out"].data_ptr(), am.data_ptr() if am is not None else None, kind, n, k,
+                            int(bool(p.get("wait", 0))), norm_ptr)
         self.arr, self.n, self.M = arr, len(projs), M
         nbytes = int(lib.zt_q4_pass_workspace_bytes(arr, self.n, M))
         if workspace is None:
-            workspace = torch.empty((nbytes,), dtype=torch.uint8, device=projs[0]["x"].device)
+            workspace = torch.empty((nbytes,), dtype=torch.uint8, device=projs[0]["out"].device)
         self.workspace = workspace
 
     def run(self, stream=None):

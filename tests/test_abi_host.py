@@ -141,3 +141,31 @@ def test_pass_arguments_rejected(zt):
     lm = P(FAKE, FAKE, FAKE, FAKE, FAKE, zt.ZT_Q4_LM_HEAD, 64, 64, 0)
     assert zt.lib.zt_q4_pass_workspace_bytes((P * 2)(ok, lm), 2, 1) > ws
     assert zt.lib.zt_q4_pass_errors(None, 1, None) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_pass_norm_arguments_rejected(zt):
+    """The add + RMSNorm prologue's checks run before any launch."""
+    import ctypes
+    P, Nm = zt.ZtProj, zt.ZtNorm
+    f = zt.lib.zt_q4_pass
+
+    def call(nm, x=None):
+        proj = P(FAKE, FAKE, x, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0, ctypes.pointer(nm) if nm else None)
+        return f((P * 1)(proj), 1, 1, FAKE, 1 << 20, None)
+
+    for bad in (Nm(None, None, FAKE, None, None, 1e-5),                 # no residual
+                Nm(FAKE, None, None, None, None, 1e-5),                 # no gamma
+                Nm(FAKE, None, FAKE, None, None, -1e-5),               # negative eps
+                Nm(FAKE, None, FAKE, None, None, float("nan")),
+                Nm(FAKE, None, FAKE, None, None, float("inf")),
+                Nm(FAKE, None, FAKE, FAKE + 64, None, 1e-5),            # residual_out overlaps residual
+                Nm(FAKE, FAKE + 4096, FAKE, FAKE + 4096 + 112, None, 1e-5)):   # ... overlaps delta
+        assert call(bad) == zt.ZT_ERR_INVALID_ARG
+    for bad in (Nm(FAKE + 2, None, FAKE, None, None, 1e-5),
+                Nm(FAKE, FAKE + 8, FAKE, None, None, 1e-5),
+                Nm(FAKE, None, FAKE + 8, None, None, 1e-5),
+                Nm(FAKE, None, FAKE, FAKE + 4100, None, 1e-5),
+                Nm(FAKE, None, FAKE, None, FAKE + 2, 1e-5)):
+        assert call(bad) == zt.ZT_ERR_MISALIGNED
+    # without a prologue x is required
+    assert call(None, x=None) == zt.ZT_ERR_INVALID_ARG
