@@ -13,7 +13,10 @@ Each wrapper names the passage the C function follows:
 * fused gate/up + SiLU -- same write-up, section "内核融合" (fused_ffn.wgsl);
 * greedy argmax -- same write-up, section "完整的推理流水线" (贪婪解码采样);
 * residual add + RMSNorm -- same write-up, section "内核融合" (add_norm.wgsl),
-  read as the standard RMSNorm on the fp16 residual stream.
+  read as the standard RMSNorm on the fp16 residual stream;
+* rotary position embedding -- same write-up, section "完整的推理流水线" (RoPE
+  computed in place in the fused QKV kernel), read as the standard rotation
+  of feature pairs (i, i + d/2) within each head.
 
 Format reading (the pages name "q4f16_1" but give no bit layout): group of 32
 along K, fp16 scale per group, 8 codes per uint32 low nibble first,
@@ -94,8 +97,9 @@ class Oracle:
         lib.zto_double_to_half.argtypes = [ctypes.c_double]
         lib.zto_double_to_half.restype = ctypes.c_uint16
         lib.zto_add_rmsnorm.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
+        lib.zto_gemv_rope.argtypes = [_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_double, _P, _I]
         for f in (lib.zto_unpack, lib.zto_pack, lib.zto_gemv,
-                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm):
+                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm, lib.zto_gemv_rope):
             f.restype = ctypes.c_int
         self._lib = lib
 
@@ -189,6 +193,24 @@ class Oracle:
         if rc:
             raise ValueError("zto_add_rmsnorm rejected its arguments")
         return h.view(np.float16), x.view(np.float16)
+
+    def gemv_rope(self, qw, scales, x, pos, head_dim: int, theta: float, threads: int = 1) -> np.ndarray:
+        """y = W x (double), then feature pairs (i, i + d/2) of every head turned
+        by pos[m] * theta^(-2i/d)."""
+        qw = np.ascontiguousarray(qw, dtype=np.uint32)
+        s = _u16(scales)
+        x = _u16(np.atleast_2d(x))
+        N, K = qw.shape[0], qw.shape[1] * 8
+        M = x.shape[0]
+        pos = np.ascontiguousarray(pos, dtype=np.int32).ravel()
+        if pos.size != M:
+            raise ValueError("one position per token")
+        out = np.empty((M, N), dtype=np.float64)
+        rc = self._lib.zto_gemv_rope(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _ptr(pos), int(head_dim), float(theta),
+                                     _ptr(out), threads)
+        if rc:
+            raise ValueError("zto_gemv_rope rejected its arguments")
+        return out
 
     def silu(self, g: float) -> float:
         return self._lib.zto_silu(float(g))

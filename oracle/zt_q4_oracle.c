@@ -31,6 +31,11 @@
  *   simple argmax dispatch"): logits = y kept in double; argmax = the lowest
  *   index among the maxima, NaN treated as -infinity.
  *
+ *   rotary position embedding (section "完整的推理流水线": RoPE computed in
+ *   place inside the fused QKV kernel; no formula given, the standard
+ *   rotation is read): within each head of d features, feature pair
+ *   (i, i + d/2) of token m turns by pos[m] * theta^(-2i/d).
+ *
  *   residual add + RMSNorm ("add_norm.wgsl": the residual connection and
  *   RMSNorm in one step, section "内核融合"; the pages give no formula, so
  *   the standard RMSNorm is read): per row m, h = fp16(residual + delta)
@@ -261,6 +266,36 @@ int zto_add_rmsnorm(const uint16_t *residual, const uint16_t *delta, const uint1
             if (delta) h += zto_half_to_double(delta[m * K + k]);
             const double hd = zto_half_to_double(zto_double_to_half(h));
             x_out[m * K + k] = zto_double_to_half(hd * r * zto_half_to_double(gamma[k]));
+        }
+    }
+    return 0;
+}
+
+/* Projection + rotary position embedding.  y = W x as zto_gemv (double, all N
+ * rows), then for every head h (d = head_dim features, N % d == 0), every
+ * i < d/2 and every token m, with n = h*d + i, n2 = n + d/2 and
+ * phi = pos[m] * theta^(-2i/d):
+ *   out[m][n]  = y[m][n] cos(phi) - y[m][n2] sin(phi)
+ *   out[m][n2] = y[m][n2] cos(phi) + y[m][n] sin(phi)            */
+int zto_gemv_rope(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                  int M, int N, int K, const int32_t *pos, int head_dim, double theta,
+                  double *out, int threads)
+{
+    if (!qw || !scales || !x || !pos || !out || !zto_shape_ok(M, N, K)) return -1;
+    if (head_dim < 2 || head_dim % 2 || N % head_dim || !(theta > 0.0)) return -1;
+    const int half = head_dim / 2;
+    if (threads < 1) threads = 1;
+#pragma omp parallel for schedule(static) num_threads(threads)
+    for (int p = 0; p < N / 2; ++p) {
+        const int64_t h = p / half, i = p % half;
+        const int64_t n = h * head_dim + i, n2 = n + half;
+        const double inv_freq = pow(theta, -2.0 * (double)i / (double)head_dim);
+        for (int64_t m = 0; m < M; ++m) {
+            const double a = zto_row_dot(qw, scales, x, K, m, n);
+            const double b = zto_row_dot(qw, scales, x, K, m, n2);
+            const double phi = (double)pos[m] * inv_freq;
+            out[m * N + n] = a * cos(phi) - b * sin(phi);
+            out[m * N + n2] = b * cos(phi) + a * sin(phi);
         }
     }
     return 0;

@@ -393,4 +393,73 @@ def pin_rmsnorm_rows_independent(o):
     assert np.all(np.abs(ms - 1.0) < 2e-3), ms
 
 
+# ------------------------------------------------ rotary position embedding ----
+# RoPE computed in place in the fused QKV kernel (Zero-TVM write-up, section
+# "完整的推理流水线"); read as the standard rotation of pairs (i, i + d/2).
+
+def _rope_problem(seed, M, N, K):
+    rng = np.random.default_rng(seed)
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s = rng.uniform(0.005, 0.02, size=(N, K // 32)).astype(np.float16)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    return qw, s, x
+
+
+def pin_rope_position_zero_is_the_projection(o):
+    """pos = 0: cos 0 = 1 and sin 0 = 0 exactly, so every row equals the plain product."""
+    qw, s, x = _rope_problem(21, 2, 96, 64)
+    got = o.gemv_rope(qw, s, x, np.zeros(2, np.int32), 32, 10000.0)
+    assert np.array_equal(got, o.gemv(qw, s, x))
+
+
+def pin_rope_quarter_turns(o):
+    """d = 4, theta = 4 / pi^2: pair 0 (features 0, 2) turns by pos radians and
+    pair 1 (features 1, 3) by pos * theta^(-1/2) = pos * pi / 2.  pos = 1
+    sends pair 1's (a, b) to (-b, a); pos = 2 to (-a, -b); pos = 4 back."""
+    qw, s, x = _rope_problem(22, 1, 8, 64)
+    y = o.gemv(qw, s, x)[0]
+    theta = 4.0 / np.pi ** 2
+    for pos, (ca, cb) in ((1, ((0, -1), (1, 0))), (2, ((-1, 0), (0, -1))), (4, ((1, 0), (0, 1)))):
+        got = o.gemv_rope(qw, s, x, np.array([pos], np.int32), 4, theta)[0]
+        for h in (0, 4):
+            a, b = y[h + 1], y[h + 3]
+            assert abs(got[h + 1] - (ca[0] * a + ca[1] * b)) <= 1e-12 * (abs(a) + abs(b))
+            assert abs(got[h + 3] - (cb[0] * a + cb[1] * b)) <= 1e-12 * (abs(a) + abs(b))
+        # pair 0 turns by pos radians (math library cos / sin of an integer)
+        a, b = y[0], y[2]
+        c, sn = np.cos(float(pos)), np.sin(float(pos))
+        assert abs(got[0] - (a * c - b * sn)) <= 1e-12 * (abs(a) + abs(b))
+        assert abs(got[2] - (b * c + a * sn)) <= 1e-12 * (abs(a) + abs(b))
+
+
+def pin_rope_keeps_pair_lengths(o):
+    """A rotation keeps a^2 + b^2 of every pair; the pairing is (i, i + d/2):
+    pairing neighbours (2i, 2i + 1) instead breaks this for the true pairs."""
+    qw, s, x = _rope_problem(23, 3, 192, 96)
+    d = 96
+    y = o.gemv(qw, s, x)
+    got = o.gemv_rope(qw, s, x, np.array([5, 1000, 31], np.int32), d, 10000.0)
+    for h in range(2):
+        for i in range(d // 2):
+            n, n2 = h * d + i, h * d + i + d // 2
+            r0 = y[:, n] ** 2 + y[:, n2] ** 2
+            r1 = got[:, n] ** 2 + got[:, n2] ** 2
+            assert np.all(np.abs(r1 - r0) <= 1e-12 * r0 + 1e-300)
+    assert not np.allclose(got, y)
+
+
+def pin_rope_frequency_per_pair(o):
+    """With theta = 2^8 and d = 16, pair i turns by pos * 2^(-i): for pos =
+    2^7 pair 7 turns by exactly 1 radian, pair 0 by 128 -- each token uses its
+    own position."""
+    qw, s, x = _rope_problem(24, 2, 16, 32)
+    y = o.gemv(qw, s, x)
+    got = o.gemv_rope(qw, s, x, np.array([128, 0], np.int32), 16, 256.0)
+    for i, phi in ((7, 1.0), (0, 128.0), (3, 16.0)):
+        a, b = y[0, i], y[0, i + 8]
+        assert abs(got[0, i] - (a * np.cos(phi) - b * np.sin(phi))) <= 1e-11 * (abs(a) + abs(b))
+        assert abs(got[0, i + 8] - (b * np.cos(phi) + a * np.sin(phi))) <= 1e-11 * (abs(a) + abs(b))
+    assert np.array_equal(got[1], y[1])          # the second token sits at position 0
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

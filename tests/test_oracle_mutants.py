@@ -43,6 +43,11 @@ MUTANTS = [
      "    double ss = 0.0;\n    for (int64_t m = 0; m < M; ++m) {"),
     ("half_rounding_ties_away", "(frac == 0.5 && fmod(r, 2.0) != 0.0)", "(frac == 0.5)"),
     ("half_subnormal_spacing", "if (e < -14) e = -14;", "if (e < -15) e = -15;"),
+    ("rope_neighbour_pairs", "const int64_t n = h * head_dim + i, n2 = n + half;",
+     "const int64_t n = h * head_dim + 2 * i, n2 = n + 1;"),
+    ("rope_sin_sign", "out[m * N + n] = a * cos(phi) - b * sin(phi);", "out[m * N + n] = a * cos(phi) + b * sin(phi);"),
+    ("rope_frequency_exponent", "pow(theta, -2.0 * (double)i / (double)head_dim)", "pow(theta, -(double)i / (double)head_dim)"),
+    ("rope_first_token_position", "const double phi = (double)pos[m] * inv_freq;", "const double phi = (double)pos[0] * inv_freq;"),
     ("sampled_rows_ignored", "int64_t n = rows ? rows[i] : i;\n        for (int64_t m = 0; m < M; ++m)\n            y[",
      "int64_t n = i;\n        for (int64_t m = 0; m < M; ++m)\n            y["),
 ]
