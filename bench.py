@@ -357,42 +357,62 @@ def run_ours(args, world, rank, local):
     chained_us = c0.elapsed_time(c1) / ch_steps * 1e3
     assert zchain.errors() == 0, "a bounded wait of the chained pass expired"
 
-    # ---- the pass with residual add + RMSNorm prologues on every qkv and
-    # gate_up projection (x computed while staging), for comparison ----
-    def make_norm_pass():
+    # ---- the pass with the decoder layer's fusions, for comparison: every
+    # qkv split into Q/K rows with a RoPE epilogue and V rows (one [1][9216]
+    # output through ld_out), residual add + RMSNorm prologues on Q/K, V and
+    # gate_up (x computed while staging; the V projection normalises the same
+    # residual again) -- 161 projections, one launch ----
+    def make_fused_pass():
         projs, gen = [], torch.Generator(device=device).manual_seed(args.seed)
+        pos = torch.full((1,), 1234, dtype=torch.int32, device=device)
+
+        def norm(K):
+            return {"residual": torch.randn((1, K), generator=gen, device=device).half(),
+                    "delta": torch.randn((1, K), generator=gen, device=device).half(),
+                    "gamma": torch.rand((K,), generator=gen, device=device).half() + 0.5, "eps": 1e-5}
+
         for d in calls:
+            name, K = d["p"].name, d["p"].K
+            if name == "qkv":
+                nm = norm(K)
+                D = d["p"].n_out // 3
+                projs.append({"kind": "gemv", "qw": d["qw"][:2 * D], "scales": d["s"][:2 * D], "out": d["y"],
+                              "ld_out": 3 * D, "norm": nm, "rope": {"pos": pos, "head_dim": 96, "theta": 10000.0}})
+                projs.append({"kind": "gemv", "qw": d["qw"][2 * D:], "scales": d["s"][2 * D:],
+                              "out": d["y"][:, 2 * D:], "ld_out": 3 * D, "norm": nm})
+                continue
             e = {"kind": d["p"].kind, "qw": d["qw"], "scales": d["s"], "x": d["x"], "out": d["y"]}
             if d["p"].kind == "lm_head":
                 e["argmax"] = d["am"]
-            if d["p"].name in ("qkv", "gate_up"):
-                K = d["p"].K
-                e["norm"] = {"residual": torch.randn((1, K), generator=gen, device=device).half(),
-                             "delta": torch.randn((1, K), generator=gen, device=device).half(),
-                             "gamma": torch.rand((K,), generator=gen, device=device).half() + 0.5,
-                             "eps": 1e-5}
+            if name == "gate_up":
+                e["norm"] = norm(K)
             projs.append(e)
-        return zt_q4.Pass(projs)
+        return zt_q4.Pass(projs), len(projs)
 
-    def time_pass(pz, steps):
+    def time_alternating(pa, pb, steps):
+        """Mean us per call of two passes run alternately, each call between
+        its own events, so clock and power drift weigh on both alike."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
         with torch.cuda.stream(stream):
             for _ in range(3):
-                pz.run(stream)
-            t0 = torch.cuda.Event(enable_timing=True)
-            t1 = torch.cuda.Event(enable_timing=True)
-            t0.record(stream)
-            for _ in range(steps):
-                pz.run(stream)
-            t1.record(stream)
+                pa.run(stream)
+                pb.run(stream)
+            for e in ev:
+                e[0].record(stream)
+                pa.run(stream)
+                e[1].record(stream)
+                e[2].record(stream)
+                pb.run(stream)
+                e[3].record(stream)
             stream.synchronize()
-        return t0.elapsed_time(t1) / steps * 1e3
+        ta = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) * 1e3
+        tb = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) * 1e3
+        return ta, tb
 
-    znorm = make_norm_pass()
-    nm_steps = max(1, min(args.steps, 200))
-    # the plain pass and the pass with prologues, back to back, same length
-    plain_us_short = time_pass(zpass, nm_steps)
-    norm_us = time_pass(znorm, nm_steps)
-    assert znorm.errors() == 0
+    zfused, n_fused = make_fused_pass()
+    fz_steps = max(1, min(args.steps, 200))
+    plain_us_short, fused_us = time_alternating(zpass, zfused, fz_steps)
+    assert zfused.errors() == 0
 
     # ---- the same pass as 130 separate calls (graph + PDL), for comparison ----
     def capture(fn):
@@ -546,10 +566,11 @@ def run_ours(args, world, rank, local):
                          "duration": "mean of the event-bracketed zt_q4_pass calls of the timed region "
                                      "(pass kernel + argmax reduction)"},
             "chained_us_per_pass": round(chained_us, 2),
-            "add_rmsnorm_prologue": {"us_per_pass": round(norm_us, 2), "plain_us_per_pass": round(plain_us_short, 2),
-                                     "steps": nm_steps,
-                                     "what": "64 residual add + RMSNorm prologues (every qkv and gate_up), x computed "
-                                             "while staging; timed back to back with the plain pass"},
+            "decode_fusions": {"us_per_pass": round(fused_us, 2), "plain_us_per_pass": round(plain_us_short, 2),
+                               "steps": fz_steps, "projections": n_fused,
+                               "what": "RoPE epilogue on every Q/K, residual add + RMSNorm prologues on Q/K, V and "
+                                       "gate_up (96 norms, x computed while staging); calls alternating with "
+                                       "the plain pass, each between its own events"},
             "per_call_graph_us_per_pass": round(per_call_us, 2),
             "per_projection_us_isolated": per_kind_us,
             "cpu_baseline": cpu,

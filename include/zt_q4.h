@@ -172,7 +172,7 @@ ZT_API int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scale
 #define ZT_Q4_GEMV 0
 #define ZT_Q4_GATE_UP_SILU 1
 #define ZT_Q4_LM_HEAD 2
-#define ZT_Q4_PASS_MAX 160
+#define ZT_Q4_PASS_MAX 192
 
 /*
  * Optional prologue of a pass projection: residual add + RMSNorm (Zero-TVM
@@ -201,16 +201,41 @@ typedef struct zt_q4_norm {
     float eps;                /* >= 0, finite */
 } zt_q4_norm;
 
+/*
+ * Optional epilogue of a ZT_Q4_GEMV pass projection: rotary position
+ * embedding (Zero-TVM write-up, "完整的推理流水线": RoPE is computed in place
+ * inside the fused QKV kernel; the pages give no formula, the standard
+ * rotation is read).  The N output rows form heads of head_dim features; for
+ * head h, i < head_dim / 2, n = h * head_dim + i, n2 = n + head_dim / 2 and
+ * token m at position pos[m]:
+ *
+ *   phi       = pos[m] * theta^(-2 i / head_dim)
+ *   out[m][n]  = fp16(y[n] cos(phi) - y[n2] sin(phi))
+ *   out[m][n2] = fp16(y[n2] cos(phi) + y[n] sin(phi))
+ *
+ * y is the projection's fp32 result (not rounded before the rotation); the
+ * angle, sin, cos and the rotation are taken in double.  Use it for the Q and
+ * K rows of a QKV projection and give the V rows their own plain projection
+ * (same pass, same phase; ld_out lets both write one [M][3 * D] buffer).
+ */
+typedef struct zt_q4_rope {
+    const int32_t *pos;       /* [M] device: position of token m, >= 0 */
+    int head_dim;             /* even; N % head_dim == 0 */
+    float theta;              /* frequency base, > 0 (10000 for Phi-3-mini) */
+} zt_q4_rope;
+
 typedef struct zt_q4_proj {
     const uint32_t *qw;       /* [n_rows][K/8], n_rows = N (2N for GATE_UP_SILU) */
     const uint16_t *scales;   /* [n_rows][K/32] fp16 */
     const uint16_t *x;        /* [M][K] fp16 (ignored, may be NULL, when norm is set) */
-    void *out;                /* fp16 [M][N], or f32 [M][N] logits for LM_HEAD */
+    void *out;                /* fp16 [M][ld_out], or f32 [M][ld_out] logits for LM_HEAD */
     int32_t *argmax;          /* LM_HEAD: [M]; ignored otherwise */
     int kind;                 /* ZT_Q4_GEMV, ZT_Q4_GATE_UP_SILU or ZT_Q4_LM_HEAD */
     int N, K;
     int wait;                 /* read x only after all earlier projections completed */
-    const zt_q4_norm *norm;   /* HOST pointer to the prologue, or NULL (read during the call) */
+    int ld_out;               /* elements between output rows (tokens); 0 means N; else >= N */
+    const zt_q4_norm *norm;   /* HOST pointer to the add + RMSNorm prologue, or NULL */
+    const zt_q4_rope *rope;   /* HOST pointer to the RoPE epilogue (ZT_Q4_GEMV only), or NULL */
 } zt_q4_proj;
 
 ZT_API size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M);

@@ -49,7 +49,7 @@ namespace zt {
 constexpr int kGroup = 32;                 // k values per scale
 constexpr int kMaxCtas = 4096;             // grid cap (sizes the LM-head workspace)
 
-enum EpiKind : int { kEpiF16 = 0, kEpiGateUp = 1, kEpiLogits = 2 };
+enum EpiKind : int { kEpiF16 = 0, kEpiGateUp = 1, kEpiLogits = 2, kEpiRope = 3 };   // RoPE: pass kernel only
 
 struct Q4Args {
     const uint4 *qw;        // [rows][G]: one 16-byte chunk = the 32 codes of one group

@@ -34,7 +34,7 @@
 
 namespace zt {
 
-constexpr int kPassMax = 160;                       // projections per launch
+constexpr int kPassMax = 192;                       // projections per launch
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr unsigned kErrWaitExpired = 1u;
 
@@ -42,23 +42,34 @@ struct PassProj {
     const uint4 *qw;            // [rows][G] 16-byte chunks
     const __half *scales;       // [rows][G]
     const __half *x;            // [M][K]
-    void *out;                  // fp16 [M][N] (gemv, gate/up) or f32 [M][N] (LM head)
-    float *ws_val;              // LM head: per-CTA maximum [gridDim.x][M]
-    int *ws_idx;                //          per-CTA arg-max
-    long long base;             // byte offset of the projection's rows within its phase
-    long long phase_bytes;      // HBM bytes of the whole phase
-    int N, K, G, kind;          // kind: kEpiF16 / kEpiGateUp / kEpiLogits
-    int row_bytes;              // HBM bytes per output (codes + scales of its weight rows)
-    int scales_async;           // scales copied by cp.async (16-byte aligned rows)
-    int phase;                  // index of the projection's phase
-    int wait;                   // starts a phase: wait for all earlier projections
+    void *out;                  // fp16 [M][ldo] (gemv, gate/up, RoPE) or f32 [M][ldo] (LM head)
+    float *ws_val;              // LM head: per-CTA maximum [gridDim.x][M], then the arg-max as int
+                                // at ws_val + kMaxCtas * M (pass_ws_idx)
     // residual add + RMSNorm prologue (norm != 0): x = fp16(h * gamma / rms(h)),
     // h = fp16(res + dlt); res_out / x_out receive h / x (the CTA holding row 0)
     const __half *res, *dlt, *gamma;
     __half *res_out, *x_out;
-    float eps;
+    // RoPE epilogue (kind kEpiRope): pairs (i, i + d/2) of each head of d rows
+    // turned by pos[m] * theta^(-2i/d); N counts pairs
+    const int *pos;
+    long long base;             // byte offset of the projection's rows within its phase
+    long long phase_bytes;      // HBM bytes of the whole phase
+    int N, K, G, kind;          // kind: kEpiF16 / kEpiGateUp / kEpiLogits / kEpiRope (N: outputs, pairs for RoPE)
+    int ldo;                    // elements between output rows
+    int row_bytes;              // HBM bytes per output (codes + scales of its weight rows)
+    int scales_async;           // scales copied by cp.async (16-byte aligned rows)
+    int phase;                  // index of the projection's phase
+    int wait;                   // starts a phase: wait for all earlier projections
     int norm;
+    int rope_d;
+    float eps;
+    float theta;
 };
+
+__device__ __forceinline__ int *pass_ws_idx(const PassProj &P, int M)
+{
+    return reinterpret_cast<int *>(P.ws_val + (size_t)kMaxCtas * M);
+}
 
 // PMAX bounds the list: 1 for the single-call entry points (a small kernel
 // parameter block), kPassMax for zt_q4_pass.
@@ -102,6 +113,7 @@ struct PassGeo {
 
 static_assert(kMW == 8, "warp layout below assumes 8 warps");
 static_assert(kPassMax <= kMThreads, "one thread per projection builds the segment list");
+static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel parameter block");
 
 // log2 of the warps splitting K for a segment: minimise the items of the
 // busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
@@ -141,9 +153,17 @@ __device__ __forceinline__ PassGeo pass_geo(const PassSeg &sg, int warp)
     return g;
 }
 
-// weight row of tile slot r (0..15) of the tile starting at output o0
-__device__ __forceinline__ int pass_slot_row(int kind, int N, int o_end, int o0, int r, bool &valid)
+// weight row of tile slot r (0..15) of the tile starting at output o0.  Gate/up
+// and RoPE tiles hold 8 outputs: slots 0..7 their first rows, 8..15 the
+// partner rows (up rows; the second feature of each RoPE pair).
+__device__ __forceinline__ int pass_slot_row(int kind, int N, int rope_d, int o_end, int o0, int r, bool &valid)
 {
+    if (kind == kEpiRope) {
+        const int o = min(o0 + (r & 7), N - 1), half = rope_d >> 1;
+        valid = o0 + (r & 7) < o_end;
+        const int h = o / half, i = o - h * half;
+        return h * rope_d + i + (r < 8 ? 0 : half);
+    }
     if (kind == kEpiGateUp) {
         const int o = o0 + (r & 7);
         valid = o < o_end;
@@ -185,6 +205,22 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *counter, unsign
         asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
         if (t - t0 > kWaitLimitNs) return false;
     }
+}
+
+// RoPE epilogue of one pair: a, b = the pair's two projections (fp32 sums),
+// turned by pos * theta^(-2i/d) in double and rounded once to fp16.  Out of
+// line: the double-precision pow / sincos stay out of the hot loop's register
+// allocation (inlined, they cost the plain projections ~5 %).
+__device__ __noinline__ void rope_store(__half *out, size_t row_off, int pair, int d, float theta, int pos,
+                                           float a, float b)
+{
+    const int half = d >> 1, h = pair / half, i = pair - h * half;
+    const double phi = (double)pos * pow((double)theta, -2.0 * i / d);
+    double sn, cs;
+    sincos(phi, &sn, &cs);
+    const int n = h * d + i;
+    out[row_off + n] = __double2half((double)a * cs - (double)b * sn);
+    out[row_off + n + half] = __double2half((double)b * cs + (double)a * sn);
 }
 
 // NT: n-tiles of 8 activation columns (M <= 8 NT); ONE: M == 1, so the mma's
@@ -232,7 +268,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     mine.o_begin = o0;
                     mine.o_end = o1;
                     mine.phase = P.phase;
-                    mine.rout = P.kind == kEpiGateUp ? kMTileRows / 2 : kMTileRows;
+                    mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
                     mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT);
@@ -242,7 +278,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 // an LM head this CTA has no rows of still gets a (neutral) partial maximum
                 for (int m = 0; m < M; ++m) {
                     P.ws_val[(size_t)blockIdx.x * M + m] = -INFINITY;
-                    P.ws_idx[(size_t)blockIdx.x * M + m] = 0x7fffffff;
+                    pass_ws_idx(P, M)[(size_t)blockIdx.x * M + m] = 0x7fffffff;
                 }
             }
         }
@@ -290,11 +326,11 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         const PassProj &P = a.p[segs[is_s].p];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = pass_slot_row(P.kind, P.N, ig.o_end, is_o0, (lane >> 3) + 4 * i, ok_w[i]);
+            const int row = pass_slot_row(P.kind, P.N, P.rope_d, ig.o_end, is_o0, (lane >> 3) + 4 * i, ok_w[i]);
             src_w[i] = P.qw + (size_t)row * P.G + ig.my_wk * kMChunkG + pg;
         }
         ok_s = false;
-        const int row = pass_slot_row(P.kind, P.N, ig.o_end, is_o0, lane & 15, ok_s);
+        const int row = pass_slot_row(P.kind, P.N, P.rope_d, ig.o_end, is_o0, lane & 15, ok_s);
         ok_s = ok_s && lane < kMTileRows && P.scales_async;
         src_s = P.scales + (size_t)row * P.G + ig.my_wk * kMChunkG;
         is_chunks = ig.my_chunks;
@@ -365,7 +401,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const PassSeg sgm = segs[cs];
             const PassProj &P = a.p[sgm.p];
             const PassGeo g = pass_geo(sgm, warp);
-            const int G = P.G, N = P.N, kind = P.kind;
+            const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d;
             const bool sasync = P.scales_async;
             void *const out = P.out;
             if (P.norm) {
@@ -419,8 +455,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         } else {
                             bool v0, v1;
                             const int c = g.my_wk + g.wk * cl;
-                            const int r0 = pass_slot_row(kind, N, g.o_end, o0, qg, v0);
-                            const int r1 = pass_slot_row(kind, N, g.o_end, o0, qg + 8, v1);
+                            const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
+                            const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
                             uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
                             const unsigned short *p0 =
                                 reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
@@ -506,8 +542,13 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                                     if (nn < g.o_end) {
                                         const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
                                         const float silu = gv / (1.0f + expf(-gv));
-                                        reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
+                                        reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(silu * u);
                                     }
+                                } else if (!LOG && kind == kEpiRope) {
+                                    const int nn = o0 + qg;
+                                    if (nn < g.o_end)
+                                        rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta,
+                                                   P.pos[m], acc[nt][e] * pow2f(24), acc[nt][2 + e] * pow2f(24));
                                 } else {
 #pragma unroll
                                     for (int h = 0; h < 2; ++h) {
@@ -515,9 +556,9 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                                         if (nn >= g.o_end) continue;
                                         const float y = acc[nt][2 * h + e] * pow2f(24);
                                         if constexpr (!LOG) {
-                                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                                            reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
                                         } else {
-                                            reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
+                                            reinterpret_cast<float *>(out)[(size_t)m * ldo + nn] = y;
                                             if (better(y, nn, best_v[2 * nt + e], best_i[2 * nt + e])) {
                                                 best_v[2 * nt + e] = isnan(y) ? -INFINITY : y;
                                                 best_i[2 * nt + e] = nn;
@@ -543,22 +584,26 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         float y = 0.f, u = 0.f;
                         for (int k2 = 0; k2 < g.wk; ++k2) {
                             y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
-                            if (kind == kEpiGateUp) u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                            if (kind == kEpiGateUp || kind == kEpiRope)
+                                u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
                         }
                         y *= pow2f(24);
                         if constexpr (LOG) {
-                            reinterpret_cast<float *>(out)[(size_t)m * N + nn] = y;
+                            reinterpret_cast<float *>(out)[(size_t)m * ldo + nn] = y;
                             // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
                             if (better(y, nn, best_v[0], best_i[0])) {
                                 best_v[0] = isnan(y) ? -INFINITY : y;
                                 best_i[0] = nn;
                             }
                         } else if (kind == kEpiF16) {
-                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(y);
+                            reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
+                        } else if (kind == kEpiRope) {
+                            rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta, P.pos[m],
+                                       y, u * pow2f(24));
                         } else {
                             u *= pow2f(24);
                             const float silu = y / (1.0f + expf(-y));
-                            reinterpret_cast<__half *>(out)[(size_t)m * N + nn] = __float2half_rn(silu * u);
+                            reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(silu * u);
                         }
                     }
                 }
@@ -590,7 +635,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             }
                         }
                         P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-                        P.ws_idx[(size_t)blockIdx.x * M + tid] = bi;
+                        pass_ws_idx(P, M)[(size_t)blockIdx.x * M + tid] = bi;
                     }
                 }
             };

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <climits>
 #include <cstdint>
 #include <mutex>
@@ -279,7 +280,7 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         PassProj &p = a.p[i];
         if (i == 0 || p.wait) phase_bytes[a.phases++] = 0;
         p.phase = a.phases - 1;
-        p.row_bytes = (p.K / 2 + p.K / 16) * (p.kind == kEpiGateUp ? 2 : 1);
+        p.row_bytes = (p.K / 2 + p.K / 16) * ((p.kind == kEpiGateUp || p.kind == kEpiRope) ? 2 : 1);
         p.base = phase_bytes[p.phase];
         phase_bytes[p.phase] += (long long)p.N * p.row_bytes;
         rows += p.N;
@@ -320,8 +321,7 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.scales = q.scales;
     p.x = q.x;
     p.out = q.out;
-    p.ws_val = q.ws_val;
-    p.ws_idx = q.ws_idx;
+    p.ws_val = q.ws_val;   // the arg-max follows at ws_val + kMaxCtas * M (q.ws_idx)
     p.N = q.N;
     p.K = q.K;
     p.G = q.G;
@@ -332,6 +332,10 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.res = p.dlt = p.gamma = nullptr;
     p.res_out = p.x_out = nullptr;
     p.eps = 0.f;
+    p.ldo = q.N;
+    p.pos = nullptr;
+    p.theta = 0.f;
+    p.rope_d = 0;
     if (q.M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
     return (q.M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
@@ -552,6 +556,14 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
             };
             if (overlap(nm.residual_out, nm.residual) || overlap(nm.residual_out, nm.delta)) return ZT_ERR_INVALID_ARG;
         }
+        if (q.ld_out != 0 && q.ld_out < q.N) return ZT_ERR_INVALID_ARG;
+        if (q.rope) {
+            const zt_q4_rope &rp = *q.rope;
+            if (q.kind != ZT_Q4_GEMV || !rp.pos || rp.head_dim < 2 || rp.head_dim % 2 || q.N % rp.head_dim ||
+                !(rp.theta > 0.f) || rp.theta > 3.0e38f)
+                return ZT_ERR_INVALID_ARG;
+            if (!aligned(rp.pos, 4)) return ZT_ERR_MISALIGNED;
+        }
         if (!aligned(q.qw, 16) || !aligned(q.x, 16) || !aligned(q.scales, 2) ||
             !aligned(q.out, q.kind == ZT_Q4_LM_HEAD ? 4 : 2) || (q.argmax && !aligned(q.argmax, 4)))
             return ZT_ERR_MISALIGNED;
@@ -561,7 +573,7 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
     size_t err_off = 0, lm_off = 0;
     if (ws_bytes < pass_ws_layout(projs, n, M, &err_off, &lm_off)) return ZT_ERR_WORKSPACE;
 
-    static thread_local PassArgs<kPassMax> a;    // ~13 KB: kept off the stack
+    static thread_local PassArgs<kPassMax> a;    // ~32 KB: kept off the stack
     unsigned char *ws = reinterpret_cast<unsigned char *>(workspace);
     a.n = n;
     a.M = M;
@@ -588,11 +600,20 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         p.res_out = q.norm ? reinterpret_cast<__half *>(q.norm->residual_out) : nullptr;
         p.x_out = q.norm ? reinterpret_cast<__half *>(q.norm->x_out) : nullptr;
         p.eps = q.norm ? q.norm->eps : 0.f;
+        p.ldo = q.ld_out ? q.ld_out : q.N;
+        p.pos = nullptr;
+        p.theta = 0.f;
+        p.rope_d = 0;
+        if (q.rope) {
+            p.kind = kEpiRope;
+            p.N = q.N / 2;                    // pairs
+            p.pos = q.rope->pos;
+            p.rope_d = q.rope->head_dim;
+            p.theta = q.rope->theta;
+        }
         p.ws_val = nullptr;
-        p.ws_idx = nullptr;
         if (q.kind == ZT_Q4_LM_HEAD) {
             p.ws_val = reinterpret_cast<float *>(ws + lm);
-            p.ws_idx = reinterpret_cast<int *>(ws + lm) + (size_t)kMaxCtas * M;
             lm += lmhead_ws_bytes(M);
         }
     }
@@ -621,7 +642,7 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         e = cudaLaunchKernelEx(&cfg, q4_argmax_reduce_kernel, (const float *)a.p[i].ws_val,
-                               (const int *)a.p[i].ws_idx, grid, M, projs[i].argmax);
+                               (const int *)(a.p[i].ws_val + (size_t)kMaxCtas * M), grid, M, projs[i].argmax);
         if (e != cudaSuccess) {
             g_last_cuda_error = e;
             (void)cudaGetLastError();

@@ -38,7 +38,7 @@ class ZtError(RuntimeError):
 ZT_Q4_GEMV = 0
 ZT_Q4_GATE_UP_SILU = 1
 ZT_Q4_LM_HEAD = 2
-ZT_Q4_PASS_MAX = 160
+ZT_Q4_PASS_MAX = 192
 
 
 class ZtNorm(ctypes.Structure):
@@ -47,12 +47,17 @@ class ZtNorm(ctypes.Structure):
                 ("residual_out", ctypes.c_void_p), ("x_out", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
+class ZtRope(ctypes.Structure):
+    """struct zt_q4_rope of include/zt_q4.h (rotary position embedding epilogue)"""
+    _fields_ = [("pos", ctypes.c_void_p), ("head_dim", ctypes.c_int), ("theta", ctypes.c_float)]
+
+
 class ZtProj(ctypes.Structure):
     """struct zt_q4_proj of include/zt_q4.h"""
     _fields_ = [("qw", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("argmax", ctypes.c_void_p), ("kind", ctypes.c_int),
-                ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int),
-                ("norm", ctypes.POINTER(ZtNorm))]
+                ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int), ("ld_out", ctypes.c_int),
+                ("norm", ctypes.POINTER(ZtNorm)), ("rope", ctypes.POINTER(ZtRope))]
 
 
 def _load() -> ctypes.CDLL:
@@ -219,8 +224,10 @@ class Pass:
     wait (read x only after all earlier projections completed).  An optional
     "norm" dict turns on the residual add + RMSNorm prologue (x is then not
     read and may be omitted): residual, gamma, eps, and optionally delta,
-    residual_out, x_out.  The ctypes arrays and the workspace are built once;
-    run() only launches."""
+    residual_out, x_out.  An optional "rope" dict (gemv only) rotates the
+    output's feature pairs: pos (int32 [M] CUDA tensor), head_dim, theta.
+    "ld_out" sets the output row stride (default N).  The ctypes arrays and
+    the workspace are built once; run() only launches."""
 
     KINDS = {"gemv": ZT_Q4_GEMV, "gate_up": ZT_Q4_GATE_UP_SILU, "lm_head": ZT_Q4_LM_HEAD}
 
@@ -255,10 +262,19 @@ class Pass:
                            ptr("residual_out", m * k), ptr("x_out", m * k), float(nm.get("eps", 1e-5)))
                 self._norms.append(z)
                 norm_ptr = ctypes.pointer(z)
+            rope_ptr = None
+            rp = p.get("rope")
+            if rp is not None:
+                pos = rp["pos"]
+                if not pos.is_cuda or pos.dtype != torch.int32 or pos.numel() != m or not pos.is_contiguous():
+                    raise ValueError("rope pos must be a contiguous CUDA int32 tensor with one position per token")
+                z = ZtRope(pos.data_ptr(), int(rp["head_dim"]), float(rp.get("theta", 10000.0)))
+                self._norms.append(z)
+                rope_ptr = ctypes.pointer(z)
             x = p.get("x")
             arr[i] = ZtProj(p["qw"].data_ptr(), p["scales"].data_ptr(), x.data_ptr() if x is not None else None,
                             p["out"].data_ptr(), am.data_ptr() if am is not None else None, kind, n, k,
-                            int(bool(p.get("wait", 0))), norm_ptr)
+                            int(bool(p.get("wait", 0))), int(p.get("ld_out", 0)), norm_ptr, rope_ptr)
         self.arr, self.n, self.M = arr, len(projs), M
         nbytes = int(lib.zt_q4_pass_workspace_bytes(arr, self.n, M))
         if workspace is None:

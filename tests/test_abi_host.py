@@ -150,7 +150,7 @@ def test_pass_norm_arguments_rejected(zt):
     f = zt.lib.zt_q4_pass
 
     def call(nm, x=None):
-        proj = P(FAKE, FAKE, x, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0, ctypes.pointer(nm) if nm else None)
+        proj = P(FAKE, FAKE, x, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0, norm=ctypes.pointer(nm) if nm else None)
         return f((P * 1)(proj), 1, 1, FAKE, 1 << 20, None)
 
     for bad in (Nm(None, None, FAKE, None, None, 1e-5),                 # no residual
@@ -169,3 +169,26 @@ def test_pass_norm_arguments_rejected(zt):
         assert call(bad) == zt.ZT_ERR_MISALIGNED
     # without a prologue x is required
     assert call(None, x=None) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_pass_rope_and_ld_out_arguments_rejected(zt):
+    """RoPE epilogue and output-stride checks run before any launch."""
+    import ctypes
+    P, R = zt.ZtProj, zt.ZtRope
+    f = zt.lib.zt_q4_pass
+
+    def call(rope, kind=zt.ZT_Q4_GEMV, N=96, ld_out=0, argmax=None):
+        proj = P(FAKE, FAKE, FAKE, FAKE, argmax, kind, N, 64, 0, ld_out, rope=ctypes.pointer(rope) if rope else None)
+        return f((P * 1)(proj), 1, 1, FAKE, 1 << 20, None)
+
+    good = R(FAKE, 32, 10000.0)
+    for bad in (R(None, 32, 10000.0),             # no positions
+                R(FAKE, 33, 10000.0),             # odd head_dim
+                R(FAKE, 64, 10000.0),             # N % head_dim != 0
+                R(FAKE, 0, 10000.0),
+                R(FAKE, 32, 0.0), R(FAKE, 32, -2.0), R(FAKE, 32, float("nan")), R(FAKE, 32, float("inf"))):
+        assert call(bad) == zt.ZT_ERR_INVALID_ARG
+    assert call(good, kind=zt.ZT_Q4_GATE_UP_SILU) == zt.ZT_ERR_INVALID_ARG       # RoPE is for plain projections
+    assert call(good, kind=zt.ZT_Q4_LM_HEAD, argmax=FAKE) == zt.ZT_ERR_INVALID_ARG
+    assert call(R(FAKE + 2, 32, 10000.0)) == zt.ZT_ERR_MISALIGNED
+    assert call(None, ld_out=95) == zt.ZT_ERR_INVALID_ARG                         # stride below N
