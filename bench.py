@@ -61,6 +61,9 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--sweep-m", action="store_true",
+                   help="instead of the pass: the fused gate_up projection (K 3072, 2 x 8192 rows) at M = 1, 2, 4, "
+                        "8, 16, one JSON line per M")
     return p.parse_args()
 
 
@@ -583,12 +586,52 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep_m(args, local):
+    """The small-batch configuration: gate_up (K 3072, 2 x 8192 rows, SiLU(g)*u)
+    at M = 1, 2, 4, 8, 16 tokens.  Eight copies of the weights (8 x 28.3 MB,
+    larger than L2) are used in turn, so every call streams from HBM."""
+    import torch
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    K, N, copies = 3072, 8192, 8
+    p = synth.Proj("gate_up", "gate_up", K, N, synth.PROJ_GATE_UP)
+    w = []
+    for c in range(copies):
+        qw, s, _ = synth.proj_inputs(args.seed, c, p)
+        w.append((torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)))
+    stream = torch.cuda.Stream(device=device)
+    for M in (1, 2, 4, 8, 16):
+        x = torch.randn((M, K), device=device).half()
+        y = torch.empty((M, N), dtype=torch.float16, device=device)
+        steps = max(args.steps, 8 * copies)
+        with torch.cuda.stream(stream):
+            for i in range(max(args.warmup, 3) * copies):
+                zt_q4.gate_up_silu(w[i % copies][0], w[i % copies][1], x, y, stream=stream)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(steps):
+                zt_q4.gate_up_silu(w[i % copies][0], w[i % copies][1], x, y, stream=stream)
+            b.record(stream)
+            stream.synchronize()
+        us = a.elapsed_time(b) / steps * 1e3
+        nbytes = alg_bytes(p, M)
+        print(json.dumps({"metric": "q4 gate_up GEMV effective HBM GB/s", "value": round(nbytes / us / 1e3, 1),
+                          "unit": "GB/s", "M": M, "us_per_call": round(us, 3), "bytes_per_call": nbytes,
+                          "flops_per_call": 2 * M * 2 * N * K, "steps": steps, "weight_copies": copies,
+                          "config": {"workload": "gate_up K=3072 N=2x8192 +SiLU*up, q4 group-32, single calls"}}),
+              flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.sweep_m:
+            run_sweep_m(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:
