@@ -106,11 +106,13 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // step 0 (x[8t], x[8t+4], x[8t+2], x[8t+6]), step 1 (x[8t+1], x[8t+5],
 // x[8t+3], x[8t+7]) / 16 (k relative to 32g).  The C table holds, for each
 // (g, n-tile, quad thread t), (c, c', c, c') with c = -7 X_g 2^-24 of column
-// 8 nt + 2t and c' of the next column (zero for columns >= M).  Thread i of
+// 8 nt + 2t and c' of the next column (zero for columns >= M).  With a single
+// column (compact) the table holds one entry (c, 0, c, 0) per group, which
+// every lane reads -- the other lanes' columns are never used.  Thread i of
 // the CTA takes 8 activations of one column per round; the 4 threads of a
 // group are adjacent lanes.  Callers synchronise before reading.
 __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool valid, unsigned char *xp,
-                                            float *x7, size_t nstride, int NT)
+                                            float *x7, size_t nstride, int NT, bool compact)
 {
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     float part = 0.f;
@@ -140,10 +142,14 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
     part += __shfl_xor_sync(0xffffffffu, part, 2);
     if (valid && (kk & 3) == 0) {
         const float c = part * (-7.0f * pow2f(-24));
-        const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
-        float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
-        cv[e] = c;
-        cv[2 + e] = c;
+        if (compact) {
+            *reinterpret_cast<float4 *>(x7 + (size_t)(kk >> 2) * 4) = make_float4(c, 0.f, c, 0.f);
+        } else {
+            const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+            float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+            cv[e] = c;
+            cv[2 + e] = c;
+        }
     }
 }
 
@@ -154,7 +160,8 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
     const int total = M * K8;
     const size_t nstride = (size_t)G * 64 + 32;
     // C entries of the padding columns M .. 8 NT - 1 are zero
-    const int pad = 8 * NT - M;
+    const bool compact = M == 1;
+    const int pad = compact ? 0 : 8 * NT - M;
     for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
@@ -172,8 +179,8 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
         if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * K + 8 * k0));
         if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * K + 8 * k1));
-        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT);
-        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
+        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
 }
 
@@ -232,7 +239,8 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         __syncthreads();
     }
     const int total = M * K8;
-    const int pad = 8 * NT - M;
+    const bool compact = M == 1;
+    const int pad = compact ? 0 : 8 * NT - M;
     for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
@@ -264,8 +272,8 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
         if (v0) r0 = normalise(m0, k0);
         if (v1) r1 = normalise(m1, k1);
-        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT);
-        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
+        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
 }
 

@@ -85,8 +85,9 @@ struct PassArgs {
 // WK > 1 partial buffer: (tiles x WK) warp tiles of 16 rows x 8 NT columns
 // per segment.  The LM head's per-thread maxima reuse it once a segment's
 // partial sums have been read.
-constexpr int kRedFloats = 2048;            // 8 KB
-static_assert(kMThreads * 2 * 2 * 8 <= kRedFloats * 4, "LM-head maxima must fit the partial buffer");
+__host__ __device__ constexpr int pass_red_floats(int NT) { return 1024 * NT; }   // 4 KB per n-tile
+static_assert(kMThreads * 2 * 1 * 8 <= pass_red_floats(1) * 4, "LM-head maxima must fit the partial buffer");
+static_assert(kMThreads * 2 * 2 * 8 <= pass_red_floats(2) * 4, "LM-head maxima must fit the partial buffer");
 constexpr int kPassMaxStages = 4;           // ring depths 2..4 are instantiated
 
 // One projection's rows in one CTA, with the CTA's warp layout for them.
@@ -101,8 +102,8 @@ __host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, 
 {
     const size_t ring = (size_t)kMW * stages * kMStage;
     const size_t xp = (size_t)M * ((size_t)g_max * 64 + 32);
-    const size_t x7 = (size_t)g_max * NT * 64;
-    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)kRedFloats * 4 + (size_t)n * sizeof(PassSeg) +
+    const size_t x7 = M == 1 ? (size_t)g_max * 16 : (size_t)g_max * NT * 64;   // compact C table at M = 1
+    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT) * 4 + (size_t)n * sizeof(PassSeg) +
            (kMW + 4) * sizeof(int);
 }
 
@@ -117,7 +118,7 @@ static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel
 
 // log2 of the warps splitting K for a segment: minimise the items of the
 // busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
-// K-warps, with the partial buffer bounded (tiles * WK * 16 * 8 NT <= kRedFloats).
+// K-warps, with the partial buffer bounded (tiles * WK * 16 * 8 NT <= pass_red_floats).
 __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT)
 {
     int best = 0, best_cost = -1;
@@ -125,7 +126,7 @@ __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT)
     for (int wkl = 0; wkl <= 3; ++wkl) {
         const int wk = 1 << wkl;
         if (wk > n_chunks) break;
-        if (wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > kRedFloats) break;
+        if (wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT)) break;
         const int cost = ((n_tiles + (kMW >> wkl) - 1) >> (3 - wkl)) * ((n_chunks + wk - 1) >> wkl);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
@@ -239,10 +240,10 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     unsigned char *xp = smem + (size_t)kMW * S * kMStage;
     const size_t xp_bytes = ((size_t)M * ((size_t)a.g_max * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
-    float *red = x7 + (size_t)a.g_max * NT * 16;
+    float *red = x7 + (ONE ? (size_t)a.g_max * 4 : (size_t)a.g_max * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
-    PassSeg *segs = reinterpret_cast<PassSeg *>(red + kRedFloats);
+    PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT));
     int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
     volatile int *abort_flag = wcount + kMW;
 
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const uint32_t ring_o = (uint32_t)(ring - smem);
     const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
     const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
-    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
+    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? 0 : qt * 16);
     uint32_t so = 0;                // ring stage offset of the next item to compute
     int cs = 0;
 
@@ -419,7 +420,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             for (int nt = 0; nt < NT; ++nt)
                 xb[nt] = (uint32_t)(xp - smem) + (uint32_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
             const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
-            const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = xstep * NT;
+            // per chunk: 64 B of staged x per group; the C table 64 NT B per group (16 B compact)
+            const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = ONE ? xstep / 4 : xstep * NT;
 
             // The segment's tiles; LOG: the LM head's epilogue (f32 logits and
             // running maxima) -- compiled apart so that the other projections'
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 #pragma unroll
                         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
                     uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
-                    uint32_t coff = xoff * NT;                            // C-table bytes
+                    uint32_t coff = ONE ? xoff / 4 : xoff * NT;           // C-table bytes
                     for (int cl = 0; cl < g.my_chunks; ++cl) {
                         cp_async_wait<S - 2>();
                         __syncwarp();
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
                         // shared-memory pointers of the item; the unrolled groups add constants
                         const unsigned char *wp = smem + wq_o + so;
-                        const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64
+                        const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
                         const unsigned char *bp[NT];
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
@@ -491,7 +493,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
                                 const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
-                                const uint4 czu = *reinterpret_cast<const uint4 *>(cp + (gl * NT + nt) * 64);
+                                const uint4 czu =
+                                    *reinterpret_cast<const uint4 *>(cp + (ONE ? gl * 16 : (gl * NT + nt) * 64));
                                 float d[4];
                                 mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
                                           __uint_as_float(czu.z), __uint_as_float(czu.w));
