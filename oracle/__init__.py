@@ -20,7 +20,8 @@ Each wrapper names the passage the C function follows:
 
 Format reading (the pages name "q4f16_1" but give no bit layout): group of 32
 along K, fp16 scale per group, 8 codes per uint32 low nibble first,
-w = (q - 7) * s.
+w = (q - 7) * s.  The group size is read from the scales' shape ([rows][K /
+group]), so groups of 64 or 128 k use the same functions.
 """
 from __future__ import annotations
 
@@ -62,6 +63,14 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _group(K: int, scales: np.ndarray) -> int:
+    """Group size from the scales' shape: [rows][K / group]."""
+    ng = scales.shape[-1]
+    if ng < 1 or K % ng:
+        raise ValueError(f"scales with {ng} groups per row do not divide K = {K}")
+    return K // ng
+
+
 def _u16(a) -> np.ndarray:
     """fp16 (or raw uint16 bit patterns) -> contiguous uint16 bit patterns."""
     a = np.asarray(a)
@@ -87,17 +96,17 @@ class Oracle:
         lib.zto_half_to_double.restype = ctypes.c_double
         lib.zto_unpack.argtypes = [_P, _I, _I, _P]
         lib.zto_pack.argtypes = [_P, _I, _I, _P]
-        lib.zto_gemv.argtypes = [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I]
-        lib.zto_gate_up_silu.argtypes = [_P, _P, _P, _I, _I, _I, _P, _I, _P, _I]
+        lib.zto_gemv.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I]
+        lib.zto_gate_up_silu.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I]
         lib.zto_silu.argtypes = [ctypes.c_double]
         lib.zto_silu.restype = ctypes.c_double
         lib.zto_argmax.argtypes = [_P, _I]
         lib.zto_argmax.restype = ctypes.c_int32
-        lib.zto_lmhead_argmax.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P, _I]
+        lib.zto_lmhead_argmax.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P, _I]
         lib.zto_double_to_half.argtypes = [ctypes.c_double]
         lib.zto_double_to_half.restype = ctypes.c_uint16
         lib.zto_add_rmsnorm.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
-        lib.zto_gemv_rope.argtypes = [_P, _P, _P, _I, _I, _I, _P, _I, ctypes.c_double, _P, _I]
+        lib.zto_gemv_rope.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, ctypes.c_double, _P, _I]
         for f in (lib.zto_unpack, lib.zto_pack, lib.zto_gemv,
                   lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm, lib.zto_gemv_rope):
             f.restype = ctypes.c_int
@@ -150,7 +159,7 @@ class Oracle:
         M = x.shape[0]
         r, nr = self._rows(rows)
         y = np.empty((M, nr if r is not None else N), dtype=np.float64)
-        rc = self._lib.zto_gemv(_ptr(qw), _ptr(s), _ptr(x), M, N, K,
+        rc = self._lib.zto_gemv(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s),
                                 _ptr(r) if r is not None else None, nr, _ptr(y), threads)
         if rc:
             raise ValueError("zto_gemv rejected its arguments")
@@ -168,7 +177,7 @@ class Oracle:
         M = x.shape[0]
         r, nr = self._rows(rows)
         out = np.empty((M, nr if r is not None else N), dtype=np.float64)
-        rc = self._lib.zto_gate_up_silu(_ptr(qw), _ptr(s), _ptr(x), M, N, K,
+        rc = self._lib.zto_gate_up_silu(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s),
                                         _ptr(r) if r is not None else None, nr,
                                         _ptr(out), threads)
         if rc:
@@ -206,8 +215,8 @@ class Oracle:
         if pos.size != M:
             raise ValueError("one position per token")
         out = np.empty((M, N), dtype=np.float64)
-        rc = self._lib.zto_gemv_rope(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _ptr(pos), int(head_dim), float(theta),
-                                     _ptr(out), threads)
+        rc = self._lib.zto_gemv_rope(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s), _ptr(pos), int(head_dim),
+                                     float(theta), _ptr(out), threads)
         if rc:
             raise ValueError("zto_gemv_rope rejected its arguments")
         return out
@@ -228,7 +237,7 @@ class Oracle:
         M = x.shape[0]
         logits = np.empty((M, N), dtype=np.float64)
         am = np.empty((M,), dtype=np.int32)
-        rc = self._lib.zto_lmhead_argmax(_ptr(qw), _ptr(s), _ptr(x), M, N, K,
+        rc = self._lib.zto_lmhead_argmax(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s),
                                          _ptr(logits), _ptr(am), threads)
         if rc:
             raise ValueError("zto_lmhead_argmax rejected its arguments")

@@ -19,7 +19,9 @@
  *
  *     weights   W is N x K (out x in).  qw is uint32 [N][K/8]; element (n,k)
  *               is bits 4*(k%8) .. 4*(k%8)+3 of qw[n][k/8]  (low nibble first)
- *     scales    fp16 [N][K/32], one per group of 32 consecutive k
+ *     scales    fp16 [N][K/32], one per group of 32 consecutive k (the
+ *               functions take the group size: 64 or 128 k per scale, the
+ *               usual GPTQ / AWQ groupings, are the same formula)
  *     dequant   w[n][k] = (q[n][k] - 7) * s[n][k/32]
  *     product   y[m][n] = sum_k w[n][k] * x[m][k], summed in plain k order
  *
@@ -50,7 +52,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#define ZTO_GROUP 32   /* k values per fp16 scale */
+#define ZTO_GROUP 32   /* k values per fp16 scale in the q4f16 format (callers pass it; larger groups also work) */
 #define ZTO_ZERO 7     /* the zero point subtracted from every 4-bit code */
 
 /* IEEE-754 binary16 bit pattern -> double, written out from the format:
@@ -80,26 +82,29 @@ static int zto_code(const uint32_t *qw, int64_t K, int64_t n, int64_t k)
 }
 
 /* Dequantized weight w[n][k] = (q - 7) * s, exact in double. */
-static double zto_weight(const uint32_t *qw, const uint16_t *scales, int64_t K,
+static double zto_weight(const uint32_t *qw, const uint16_t *scales, int64_t K, int64_t group,
                          int64_t n, int64_t k)
 {
-    double s = zto_half_to_double(scales[n * (K / ZTO_GROUP) + k / ZTO_GROUP]);
+    double s = zto_half_to_double(scales[n * (K / group) + k / group]);
     return (double)(zto_code(qw, K, n, k) - ZTO_ZERO) * s;
 }
 
 /* One dot product: sum over k = 0..K-1, in that order, of w[n][k] * x[m][k]. */
 static double zto_row_dot(const uint32_t *qw, const uint16_t *scales,
-                          const uint16_t *x, int64_t K, int64_t m, int64_t n)
+                          const uint16_t *x, int64_t K, int64_t group, int64_t m, int64_t n)
 {
     double acc = 0.0;
     for (int64_t k = 0; k < K; ++k)
-        acc += zto_weight(qw, scales, K, n, k) * zto_half_to_double(x[m * K + k]);
+        acc += zto_weight(qw, scales, K, group, n, k) * zto_half_to_double(x[m * K + k]);
     return acc;
 }
 
-static int zto_shape_ok(int M, int N, int K)
+/* Shapes: K a multiple of 8 (whole words) and of the group size (whole
+ * groups); the format's group is ZTO_GROUP = 32, larger groups share one
+ * scale among group / 32 consecutive blocks of 32. */
+static int zto_shape_ok(int M, int N, int K, int group)
 {
-    return M >= 1 && N >= 1 && K >= ZTO_GROUP && K % ZTO_GROUP == 0;
+    return M >= 1 && N >= 1 && group >= 1 && K >= group && K % group == 0 && K % 8 == 0;
 }
 
 /* Unpack codes: q[n][k] (one byte each, 0..15) from qw[n][K/8]. */
@@ -134,10 +139,10 @@ int zto_pack(const uint8_t *q, int N, int K, uint32_t *qw)
  * (n_rows must equal N and row_i = i); otherwise only the listed rows, and y is
  * [M][n_rows].  Output in double, no rounding to fp16. */
 int zto_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
-             int M, int N, int K, const int32_t *rows, int n_rows,
+             int M, int N, int K, int group, const int32_t *rows, int n_rows,
              double *y, int threads)
 {
-    if (!qw || !scales || !x || !y || !zto_shape_ok(M, N, K)) return -1;
+    if (!qw || !scales || !x || !y || !zto_shape_ok(M, N, K, group)) return -1;
     if (!rows) n_rows = N;
     for (int i = 0; rows && i < n_rows; ++i)
         if (rows[i] < 0 || rows[i] >= N) return -1;
@@ -146,7 +151,7 @@ int zto_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
     for (int i = 0; i < n_rows; ++i) {
         int64_t n = rows ? rows[i] : i;
         for (int64_t m = 0; m < M; ++m)
-            y[m * n_rows + i] = zto_row_dot(qw, scales, x, K, m, n);
+            y[m * n_rows + i] = zto_row_dot(qw, scales, x, K, group, m, n);
     }
     return 0;
 }
@@ -161,10 +166,10 @@ double zto_silu(double g)
  * projection, rows N..2N-1 the up projection.  out[m][i] = SiLU(g) * u with
  * g = dot(gate row n), u = dot(up row n), n = rows[i] (or i), all in double. */
 int zto_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
-                     int M, int N, int K, const int32_t *rows, int n_rows,
+                     int M, int N, int K, int group, const int32_t *rows, int n_rows,
                      double *out, int threads)
 {
-    if (!qw || !scales || !x || !out || !zto_shape_ok(M, N, K)) return -1;
+    if (!qw || !scales || !x || !out || !zto_shape_ok(M, N, K, group)) return -1;
     if (!rows) n_rows = N;
     for (int i = 0; rows && i < n_rows; ++i)
         if (rows[i] < 0 || rows[i] >= N) return -1;
@@ -173,8 +178,8 @@ int zto_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t 
     for (int i = 0; i < n_rows; ++i) {
         int64_t n = rows ? rows[i] : i;
         for (int64_t m = 0; m < M; ++m) {
-            double g = zto_row_dot(qw, scales, x, K, m, n);
-            double u = zto_row_dot(qw, scales, x, K, m, n + N);
+            double g = zto_row_dot(qw, scales, x, K, group, m, n);
+            double u = zto_row_dot(qw, scales, x, K, group, m, n + N);
             out[m * n_rows + i] = zto_silu(g) * u;
         }
     }
@@ -199,11 +204,11 @@ int32_t zto_argmax(const double *v, int N)
 
 /* LM head: logits[m][n] (double, never rounded to fp16) and argmax[m]. */
 int zto_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
-                      int M, int N, int K, double *logits, int32_t *argmax,
+                      int M, int N, int K, int group, double *logits, int32_t *argmax,
                       int threads)
 {
-    if (!qw || !scales || !x || !logits || !argmax || !zto_shape_ok(M, N, K)) return -1;
-    int rc = zto_gemv(qw, scales, x, M, N, K, NULL, N, logits, threads);
+    if (!qw || !scales || !x || !logits || !argmax || !zto_shape_ok(M, N, K, group)) return -1;
+    int rc = zto_gemv(qw, scales, x, M, N, K, group, NULL, N, logits, threads);
     if (rc) return rc;
     for (int64_t m = 0; m < M; ++m)
         argmax[m] = zto_argmax(logits + m * N, N);
@@ -278,10 +283,10 @@ int zto_add_rmsnorm(const uint16_t *residual, const uint16_t *delta, const uint1
  *   out[m][n]  = y[m][n] cos(phi) - y[m][n2] sin(phi)
  *   out[m][n2] = y[m][n2] cos(phi) + y[m][n] sin(phi)            */
 int zto_gemv_rope(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
-                  int M, int N, int K, const int32_t *pos, int head_dim, double theta,
+                  int M, int N, int K, int group, const int32_t *pos, int head_dim, double theta,
                   double *out, int threads)
 {
-    if (!qw || !scales || !x || !pos || !out || !zto_shape_ok(M, N, K)) return -1;
+    if (!qw || !scales || !x || !pos || !out || !zto_shape_ok(M, N, K, group)) return -1;
     if (head_dim < 2 || head_dim % 2 || N % head_dim || !(theta > 0.0)) return -1;
     const int half = head_dim / 2;
     if (threads < 1) threads = 1;
@@ -291,8 +296,8 @@ int zto_gemv_rope(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
         const int64_t n = h * head_dim + i, n2 = n + half;
         const double inv_freq = pow(theta, -2.0 * (double)i / (double)head_dim);
         for (int64_t m = 0; m < M; ++m) {
-            const double a = zto_row_dot(qw, scales, x, K, m, n);
-            const double b = zto_row_dot(qw, scales, x, K, m, n2);
+            const double a = zto_row_dot(qw, scales, x, K, group, m, n);
+            const double b = zto_row_dot(qw, scales, x, K, group, m, n2);
             const double phi = (double)pos[m] * inv_freq;
             out[m * N + n] = a * cos(phi) - b * sin(phi);
             out[m * N + n2] = b * cos(phi) + a * sin(phi);

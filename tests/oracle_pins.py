@@ -462,4 +462,42 @@ def pin_rope_frequency_per_pair(o):
     assert np.array_equal(got[1], y[1])          # the second token sits at position 0
 
 
+# ------------------------------------------------------- group sizes ----
+# q4f16_1 groups 32 k per scale; groups of 64 and 128 (one scale shared by
+# 2 or 4 consecutive blocks of 32) are the same formula.
+
+def pin_group_64_and_128_are_repeated_32(o):
+    """A group-G scale array equals the group-32 array with every scale
+    repeated G / 32 times: the products, the sums and their order are the
+    same, so the results are identical bit for bit (gemv, gate/up, LM head)."""
+    rng = np.random.default_rng(31)
+    K, N, M = 512, 24, 2
+    qw = rng.integers(0, 2 ** 32, size=(2 * N, K // 8), dtype=np.uint64).astype(np.uint32)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    for G in (64, 128):
+        sG = rng.uniform(0.005, 0.02, size=(2 * N, K // G)).astype(np.float16)
+        s32 = np.repeat(sG, G // 32, axis=1)
+        assert np.array_equal(o.gemv(qw, sG, x), o.gemv(qw, s32, x))
+        assert np.array_equal(o.gate_up_silu(qw, sG, x), o.gate_up_silu(qw, s32, x))
+        la, aa = o.lmhead_argmax(qw, sG, x)
+        lb, ab = o.lmhead_argmax(qw, s32, x)
+        assert np.array_equal(la, lb) and np.array_equal(aa, ab)
+
+
+def pin_group_whole_row_brute_force(o):
+    """One scale per row (group = K = 64): y = s * sum_k (q_k - 7) x_k, in
+    exact rationals."""
+    from fractions import Fraction
+    rng = np.random.default_rng(32)
+    K, N = 64, 3
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s = rng.uniform(0.5, 2.0, size=(N, 1)).astype(np.float16)
+    x = rng.standard_normal((1, K)).astype(np.float16)
+    q = codes_by_hex(qw)
+    y = o.gemv(qw, s, x)
+    for n in range(N):
+        exact = Fraction(float(s[n, 0])) * sum(Fraction(int(q[n, k]) - 7) * Fraction(float(x[0, k])) for k in range(K))
+        assert abs(Fraction(y[0, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 200)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -16,12 +16,14 @@ import oracle_pins as P
 # (name, text in the oracle source, replacement)
 MUTANTS = [
     ("nibble_order_reversed", "(word >> (4 * (k % 8)))", "(word >> (4 * (7 - k % 8)))"),
-    ("scale_group_off_by_one", "scales[n * (K / ZTO_GROUP) + k / ZTO_GROUP]",
-     "scales[n * (K / ZTO_GROUP) + (k / ZTO_GROUP + 1) % (K / ZTO_GROUP)]"),
+    ("scale_group_off_by_one", "scales[n * (K / group) + k / group]",
+     "scales[n * (K / group) + (k / group + 1) % (K / group)]"),
+    ("scale_group_fixed_32", "scales[n * (K / group) + k / group]",
+     "scales[n * (K / group) + (k / ZTO_GROUP) % (K / group)]"),
     ("zero_point_8", "#define ZTO_ZERO 7", "#define ZTO_ZERO 8"),
     ("gate_up_swapped",
-     "double g = zto_row_dot(qw, scales, x, K, m, n);",
-     "double g = zto_row_dot(qw, scales, x, K, m, n + N);"),
+     "double g = zto_row_dot(qw, scales, x, K, group, m, n);",
+     "double g = zto_row_dot(qw, scales, x, K, group, m, n + N);"),
     ("argmax_highest_index_on_tie", "if (c > best_v) {", "if (c >= best_v) {"),
     ("dropped_k_tail", "for (int64_t k = 0; k < K; ++k)\n        acc +=",
      "for (int64_t k = 0; k < K - 1; ++k)\n        acc +="),
