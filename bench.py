@@ -417,6 +417,21 @@ def run_ours(args, world, rank, local):
     plain_us_short, fused_us = time_alternating(zpass, zfused, fz_steps)
     assert zfused.errors() == 0
 
+    # ---- the same pass with groups of 128 k per scale (the GPTQ / AWQ
+    # grouping: 1/4 of the scale bytes), alternating with the group-32 pass ----
+    g128 = []
+    g128_bytes = 0
+    for d in calls:
+        sc = d["s"][:, ::4].contiguous()
+        e = {"kind": d["p"].kind, "qw": d["qw"], "scales": sc, "x": d["x"], "out": d["y"], "group": 128}
+        if d["p"].kind == "lm_head":
+            e["argmax"] = d["am"]
+        g128.append(e)
+        g128_bytes += alg_bytes(d["p"]) - d["p"].n_rows * (d["p"].K // 32) * 2 + sc.numel() * 2
+    zg128 = zt_q4.Pass(g128)
+    plain_us_g, g128_us = time_alternating(zpass, zg128, fz_steps)
+    assert zg128.errors() == 0
+
     # ---- the same pass as 130 separate calls (graph + PDL), for comparison ----
     def capture(fn):
         with torch.cuda.stream(stream):
@@ -569,6 +584,11 @@ def run_ours(args, world, rank, local):
                          "duration": "mean of the event-bracketed zt_q4_pass calls of the timed region "
                                      "(pass kernel + argmax reduction)"},
             "chained_us_per_pass": round(chained_us, 2),
+            "group_128": {"us_per_pass": round(g128_us, 2), "plain_us_per_pass": round(plain_us_g, 2),
+                          "GBps": round(g128_bytes / g128_us / 1e3, 1), "bytes_per_pass": g128_bytes,
+                          "steps": fz_steps,
+                          "what": "the same pass with 128 k per scale (scale bytes / 4); calls alternating with the "
+                                  "group-32 pass"},
             "decode_fusions": {"us_per_pass": round(fused_us, 2), "plain_us_per_pass": round(plain_us_short, 2),
                                "steps": fz_steps, "projections": n_fused,
                                "what": "RoPE epilogue on every Q/K, residual add + RMSNorm prologues on Q/K, V and "

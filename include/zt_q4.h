@@ -234,6 +234,8 @@ typedef struct zt_q4_proj {
     int N, K;
     int wait;                 /* read x only after all earlier projections completed */
     int ld_out;               /* elements between output rows (tokens); 0 means N; else >= N */
+    int group;                /* k per fp16 scale: 0 or 32 (the q4f16 format), 64 or 128; K % group == 0;
+                                 scales are then [n_rows][K/group] */
     const zt_q4_norm *norm;   /* HOST pointer to the add + RMSNorm prologue, or NULL */
     const zt_q4_rope *rope;   /* HOST pointer to the RoPE epilogue (ZT_Q4_GEMV only), or NULL */
 } zt_q4_proj;

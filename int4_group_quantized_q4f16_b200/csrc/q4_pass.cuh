@@ -62,6 +62,7 @@ struct PassProj {
     int wait;                   // starts a phase: wait for all earlier projections
     int norm;
     int rope_d;
+    int gsh;                    // log2(group / 32): 0, 1, 2 for 32, 64, 128 k per scale
     float eps;
     float theta;
 };
@@ -208,6 +209,17 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *counter, unsign
     }
 }
 
+// Scales of an item for groups of 64 (gsh 1) or 128 (gsh 2) k: the first 4
+// (or 2) halves of the slot, each repeated so that half j is block j's scale.
+__device__ __forceinline__ uint4 spread_scales(uint4 v, int gsh)
+{
+    if (gsh == 1)
+        return make_uint4(__byte_perm(v.x, 0, 0x1010), __byte_perm(v.x, 0, 0x3232), __byte_perm(v.y, 0, 0x1010),
+                          __byte_perm(v.y, 0, 0x3232));
+    const uint32_t a = __byte_perm(v.x, 0, 0x1010), b = __byte_perm(v.x, 0, 0x3232);
+    return make_uint4(a, a, b, b);
+}
+
 // RoPE epilogue of one pair: a, b = the pair's two projections (fp32 sums),
 // turned by pos * theta^(-2i/d) in double and rounded once to fp16.  Out of
 // line: the double-precision pow / sincos stay out of the hot loop's register
@@ -312,6 +324,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     const uint32_t piece_u = ring_u + (lane >> 3) * kMRowStride + pg * 16;   // + stage, + 4 i rows
     const uint32_t scale_u = ring_u + kMScaleOff + lane * 16;
     int is_s = -1;                  // segment being issued
+    int is_gsh = 0;                 // log2(group / 32) of its projection
     int is_tiles = 0;               // tiles left after the current one
     int is_chunks = 0;              // chunks left in the current tile (0: stream ended)
     int is_kc_last = kMChunkG;      // groups of the tile's last chunk
@@ -333,7 +346,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         ok_s = false;
         const int row = pass_slot_row(P.kind, P.N, P.rope_d, ig.o_end, is_o0, lane & 15, ok_s);
         ok_s = ok_s && lane < kMTileRows && P.scales_async;
-        src_s = P.scales + (size_t)row * P.G + ig.my_wk * kMChunkG;
+        src_s = P.scales + (size_t)row * (P.G >> P.gsh) + ((ig.my_wk * kMChunkG) >> P.gsh);
+        is_gsh = P.gsh;
         is_chunks = ig.my_chunks;
     };
     // move to the next segment that has items for this warp (or end the stream)
@@ -359,10 +373,15 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 if (ok_w[i] && pg < kc) cp_async16_u32(piece_u + is_so + 4 * i * kMRowStride, src_w[i]);
-            if (ok_s) cp_async16_u32(scale_u + is_so, src_s);
+            if (ok_s) {
+                // the item's 8 blocks of 32 share 8, 4 or 2 scales: 16, 8 or 4 bytes per row
+                if (is_gsh == 0) cp_async16_u32(scale_u + is_so, src_s);
+                else if (is_gsh == 1) cp_async8_u32(scale_u + is_so, src_s);
+                else cp_async4_u32(scale_u + is_so, src_s);
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) src_w[i] += is_step;
-            src_s += is_step;
+            src_s += is_step >> is_gsh;
             if (--is_chunks == 0) {
                 if (is_tiles > 0) {
                     --is_tiles;
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const PassSeg sgm = segs[cs];
             const PassProj &P = a.p[sgm.p];
             const PassGeo g = pass_geo(sgm, warp);
-            const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d;
+            const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d, gsh = P.gsh;
             const bool sasync = P.scales_async;
             void *const out = P.out;
             if (P.norm) {
@@ -454,19 +473,25 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             const unsigned char *sp = smem + sc_o + so;
                             sg = *reinterpret_cast<const uint4 *>(sp);
                             sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
+                            if (gsh) {
+                                // one scale per 32-block: repeat each of the 4 (or 2) scales 2 (or 4) times
+                                sg = spread_scales(sg, gsh);
+                                sg8 = spread_scales(sg8, gsh);
+                            }
                         } else {
                             bool v0, v1;
                             const int c = g.my_wk + g.wk * cl;
                             const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
                             const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
                             uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                            const unsigned short *p0 =
-                                reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r0 * G + c * kMChunkG;
-                            const unsigned short *p1 =
-                                reinterpret_cast<const unsigned short *>(P.scales) + (size_t)r1 * G + c * kMChunkG;
+                            const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                       (size_t)r0 * (G >> gsh);
+                            const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                       (size_t)r1 * (G >> gsh);
                             for (int gl = 0; gl < kc; ++gl) {
-                                u0[gl >> 1] |= (uint32_t)p0[gl] << (16 * (gl & 1));
-                                u1[gl >> 1] |= (uint32_t)p1[gl] << (16 * (gl & 1));
+                                const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
+                                u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
+                                u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
                             }
                             sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
                             sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);

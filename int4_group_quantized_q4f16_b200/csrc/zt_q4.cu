@@ -280,7 +280,7 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         PassProj &p = a.p[i];
         if (i == 0 || p.wait) phase_bytes[a.phases++] = 0;
         p.phase = a.phases - 1;
-        p.row_bytes = (p.K / 2 + p.K / 16) * ((p.kind == kEpiGateUp || p.kind == kEpiRope) ? 2 : 1);
+        p.row_bytes = (p.K / 2 + (p.K / 16 >> p.gsh)) * ((p.kind == kEpiGateUp || p.kind == kEpiRope) ? 2 : 1);
         p.base = phase_bytes[p.phase];
         phase_bytes[p.phase] += (long long)p.N * p.row_bytes;
         rows += p.N;
@@ -336,6 +336,7 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     p.pos = nullptr;
     p.theta = 0.f;
     p.rope_d = 0;
+    p.gsh = 0;
     if (q.M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
     return (q.M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
@@ -557,6 +558,8 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
             if (overlap(nm.residual_out, nm.residual) || overlap(nm.residual_out, nm.delta)) return ZT_ERR_INVALID_ARG;
         }
         if (q.ld_out != 0 && q.ld_out < q.N) return ZT_ERR_INVALID_ARG;
+        if (q.group != 0 && q.group != 32 && q.group != 64 && q.group != 128) return ZT_ERR_INVALID_ARG;
+        if (q.group != 0 && q.K % q.group) return ZT_ERR_INVALID_ARG;
         if (q.rope) {
             const zt_q4_rope &rp = *q.rope;
             if (q.kind != ZT_Q4_GEMV || !rp.pos || rp.head_dim < 2 || rp.head_dim % 2 || q.N % rp.head_dim ||
@@ -591,7 +594,8 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         p.K = q.K;
         p.G = q.K / kGroup;
         p.kind = q.kind == ZT_Q4_GEMV ? kEpiF16 : q.kind == ZT_Q4_GATE_UP_SILU ? kEpiGateUp : kEpiLogits;
-        p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+        p.gsh = q.group == 64 ? 1 : q.group == 128 ? 2 : 0;
+        p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16 >> p.gsh);
         p.wait = (i > 0 && q.wait) ? 1 : 0;
         p.norm = q.norm ? 1 : 0;
         p.res = q.norm ? reinterpret_cast<const __half *>(q.norm->residual) : nullptr;

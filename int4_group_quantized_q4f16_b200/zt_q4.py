@@ -57,7 +57,7 @@ class ZtProj(ctypes.Structure):
     _fields_ = [("qw", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
                 ("out", ctypes.c_void_p), ("argmax", ctypes.c_void_p), ("kind", ctypes.c_int),
                 ("N", ctypes.c_int), ("K", ctypes.c_int), ("wait", ctypes.c_int), ("ld_out", ctypes.c_int),
-                ("norm", ctypes.POINTER(ZtNorm)), ("rope", ctypes.POINTER(ZtRope))]
+                ("group", ctypes.c_int), ("norm", ctypes.POINTER(ZtNorm)), ("rope", ctypes.POINTER(ZtRope))]
 
 
 def _load() -> ctypes.CDLL:
@@ -140,7 +140,7 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _dims(qw, scales, x, rows_mult: int):
+def _dims(qw, scales, x, rows_mult: int, group: int = 32):
     torch = _torch()
     for t, name in ((qw, "qw"), (scales, "scales"), (x, "x")):
         if not t.is_cuda or not t.is_contiguous():
@@ -152,7 +152,7 @@ def _dims(qw, scales, x, rows_mult: int):
     x2 = x if x.dim() == 2 else x.view(1, -1)
     M, K = x2.shape
     n_rows = qw.shape[0]
-    if qw.dim() != 2 or qw.shape[1] * 8 != K or scales.shape != (n_rows, K // 32):
+    if qw.dim() != 2 or qw.shape[1] * 8 != K or K % group or scales.shape != (n_rows, K // group):
         raise ValueError(f"shape mismatch: qw {tuple(qw.shape)}, scales {tuple(scales.shape)}, x {tuple(x.shape)}")
     if n_rows % rows_mult:
         raise ValueError("gate/up weights need an even number of rows")
@@ -226,7 +226,8 @@ class Pass:
     read and may be omitted): residual, gamma, eps, and optionally delta,
     residual_out, x_out.  An optional "rope" dict (gemv only) rotates the
     output's feature pairs: pos (int32 [M] CUDA tensor), head_dim, theta.
-    "ld_out" sets the output row stride (default N).  The ctypes arrays and
+    "ld_out" sets the output row stride (default N); "group" the k per scale
+    (32, 64 or 128; scales are [rows][K / group]).  The ctypes arrays and
     the workspace are built once; run() only launches."""
 
     KINDS = {"gemv": ZT_Q4_GEMV, "gate_up": ZT_Q4_GATE_UP_SILU, "lm_head": ZT_Q4_LM_HEAD}
@@ -243,7 +244,8 @@ class Pass:
             kind = self.KINDS[p["kind"]]
             nm = p.get("norm")
             xs = p.get("x") if nm is None else nm["residual"]
-            m, n, k = _dims(p["qw"], p["scales"], xs, 2 if kind == ZT_Q4_GATE_UP_SILU else 1)
+            group = int(p.get("group", 32))
+            m, n, k = _dims(p["qw"], p["scales"], xs, 2 if kind == ZT_Q4_GATE_UP_SILU else 1, group)
             if M is None:
                 M = m
             elif m != M:
@@ -274,7 +276,7 @@ class Pass:
             x = p.get("x")
             arr[i] = ZtProj(p["qw"].data_ptr(), p["scales"].data_ptr(), x.data_ptr() if x is not None else None,
                             p["out"].data_ptr(), am.data_ptr() if am is not None else None, kind, n, k,
-                            int(bool(p.get("wait", 0))), int(p.get("ld_out", 0)), norm_ptr, rope_ptr)
+                            int(bool(p.get("wait", 0))), int(p.get("ld_out", 0)), group, norm_ptr, rope_ptr)
         self.arr, self.n, self.M = arr, len(projs), M
         nbytes = int(lib.zt_q4_pass_workspace_bytes(arr, self.n, M))
         if workspace is None:

@@ -192,3 +192,12 @@ def test_pass_rope_and_ld_out_arguments_rejected(zt):
     assert call(good, kind=zt.ZT_Q4_LM_HEAD, argmax=FAKE) == zt.ZT_ERR_INVALID_ARG
     assert call(R(FAKE + 2, 32, 10000.0)) == zt.ZT_ERR_MISALIGNED
     assert call(None, ld_out=95) == zt.ZT_ERR_INVALID_ARG                         # stride below N
+
+
+def test_pass_group_size_rejected(zt):
+    """Groups other than 32, 64, 128 (0 = 32), or not dividing K, fail before any launch."""
+    P = zt.ZtProj
+    f = zt.lib.zt_q4_pass
+    for group, K in ((16, 256), (96, 384), (256, 512), (128, 320), (64, 96)):
+        proj = P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, K, 0, 0, group)
+        assert f((P * 1)(proj), 1, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG, (group, K)
