@@ -68,9 +68,14 @@ constexpr int kMW = 8;                              // warps per CTA
 constexpr int kMThreads = kMW * 32;
 constexpr int kMTileRows = 16;                      // weight rows per warp tile (mma M)
 constexpr int kMChunkG = 8;                         // groups per item
-constexpr int kMRowStride = kMChunkG * 16 + 16;     // smem bytes per tile row (padded: conflict-free)
-constexpr int kMScaleOff = kMTileRows * kMRowStride;
-constexpr int kMStage = kMScaleOff + kMTileRows * kMChunkG * 2;   // 2560 bytes per warp per stage
+// A ring stage holds an item: codes [16 rows][128 B] with the 128-byte XOR
+// swizzle (16-byte chunk j of row r at r * 128 + (j ^ (r & 7)) * 16 -- the
+// layout a TMA box with 128-byte swizzling writes; the 8 quad rows of an mma
+// then read 8 distinct bank groups), and, in a separate region, the tile's
+// scales [16 rows][16 B].
+constexpr int kMCodeStage = kMTileRows * kMChunkG * 16;   // 2048 bytes
+constexpr int kMScaleStage = kMTileRows * kMChunkG * 2;   // 256 bytes
+constexpr int kMStage = kMCodeStage + kMScaleStage;       // 2304 bytes per warp per stage
 constexpr int kMMaxStages = 8;
 
 // Shared-memory loads by 32-bit shared-window address (keeps address math

@@ -101,7 +101,7 @@ struct PassSeg {
 // bytes), C-operand table, WK partials / LM-head maxima, segment list, flags.
 __host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int n, int NT)
 {
-    const size_t ring = (size_t)kMW * stages * kMStage;
+    const size_t ring = (size_t)kMW * stages * kMStage + 1024;   // + alignment of the code stages
     const size_t xp = (size_t)M * ((size_t)g_max * 64 + 32);
     const size_t x7 = M == 1 ? (size_t)g_max * 16 : (size_t)g_max * NT * 64;   // compact C table at M = 1
     return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT) * 4 + (size_t)n * sizeof(PassSeg) +
@@ -243,13 +243,17 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 {
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     static_assert(!ONE || NT == 1, "one column fits one n-tile");
-    extern __shared__ __align__(128) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem[];
     const int M = a.M, n = a.n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qg = lane >> 2, qt = lane & 3;       // mma quad row / thread in quad
 
-    unsigned char *ring = smem + (size_t)warp * S * kMStage;
-    unsigned char *xp = smem + (size_t)kMW * S * kMStage;
+    // code stages [kMW][S][2048] start on a 1024-byte boundary (128-byte
+    // swizzle), scale stages [kMW][S][256] follow, then the activations
+    unsigned char *codes = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    unsigned char *ring_c = codes + (size_t)warp * S * kMCodeStage;
+    unsigned char *ring_s = codes + (size_t)kMW * S * kMCodeStage + (size_t)warp * S * kMScaleStage;
+    unsigned char *xp = codes + (size_t)kMW * S * kMStage;
     const size_t xp_bytes = ((size_t)M * ((size_t)a.g_max * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
     float *red = x7 + (ONE ? (size_t)a.g_max * 4 : (size_t)a.g_max * NT * 16);
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     __syncthreads();
     const int nphase = a.phases;
 
-    const uint32_t ring_u = smem_u32(ring);
+    const uint32_t ring_cu = smem_u32(ring_c), ring_su = smem_u32(ring_s);
 
     // ---------------------------------------------------------- issue side --
     // The warp's items of all segments form one stream (segment, tile,
@@ -320,16 +324,19 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     // ahead of the math, across segment and phase boundaries (weights never
     // depend on outputs).  Per item it only advances pointers; segment and
     // tile changes recompute them.
-    const int pg = lane & 7;
-    const uint32_t piece_u = ring_u + (lane >> 3) * kMRowStride + pg * 16;   // + stage, + 4 i rows
-    const uint32_t scale_u = ring_u + kMScaleOff + lane * 16;
+    // piece i: row l / 8 + 4 i, chunk pg at swizzled position pg ^ (row & 7);
+    // rows + 8 sit 1024 bytes further with the same swizzle
+    const int pg = lane & 7, l3 = lane >> 3;
+    const uint32_t piece_u0 = ring_cu + l3 * 128 + ((pg ^ l3) << 4);               // rows l3, l3 + 8
+    const uint32_t piece_u1 = ring_cu + (l3 + 4) * 128 + ((pg ^ (l3 + 4)) << 4);   // rows l3 + 4, l3 + 12
+    const uint32_t scale_u = ring_su + lane * 16;
     int is_s = -1;                  // segment being issued
     int is_gsh = 0;                 // log2(group / 32) of its projection
     int is_tiles = 0;               // tiles left after the current one
     int is_chunks = 0;              // chunks left in the current tile (0: stream ended)
     int is_kc_last = kMChunkG;      // groups of the tile's last chunk
     int is_step = 0;                // uint4 per chunk step (WK chunks of 8 groups)
-    uint32_t is_so = 0;             // ring stage offset
+    uint32_t is_st = 0;             // ring stage of the next item to issue
     int is_o0 = 0, is_rstep = 0;    // current tile's first output, outputs per tile step
     PassGeo ig{};
     const uint4 *src_w[4];          // the next chunk's source, per piece
@@ -372,12 +379,13 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const int kc = is_chunks == 1 ? is_kc_last : kMChunkG;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok_w[i] && pg < kc) cp_async16_u32(piece_u + is_so + 4 * i * kMRowStride, src_w[i]);
+                if (ok_w[i] && pg < kc)
+                    cp_async16_u32(((i & 1) ? piece_u1 : piece_u0) + (is_st << 11) + (i >> 1) * 1024, src_w[i]);
             if (ok_s) {
                 // the item's 8 blocks of 32 share 8, 4 or 2 scales: 16, 8 or 4 bytes per row
-                if (is_gsh == 0) cp_async16_u32(scale_u + is_so, src_s);
-                else if (is_gsh == 1) cp_async8_u32(scale_u + is_so, src_s);
-                else cp_async4_u32(scale_u + is_so, src_s);
+                if (is_gsh == 0) cp_async16_u32(scale_u + (is_st << 8), src_s);
+                else if (is_gsh == 1) cp_async8_u32(scale_u + (is_st << 8), src_s);
+                else cp_async4_u32(scale_u + (is_st << 8), src_s);
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) src_w[i] += is_step;
@@ -393,7 +401,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             }
         }
         cp_async_commit();     // one group per item slot, so wait counts stay uniform
-        is_so = (is_so + kMStage == (uint32_t)(S * kMStage)) ? 0u : is_so + kMStage;
+        is_st = (is_st + 1 == (uint32_t)S) ? 0u : is_st + 1;
     };
 
     // prologue: the first weights stream before the previous kernel has finished
@@ -401,11 +409,13 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
 
-    const uint32_t ring_o = (uint32_t)(ring - smem);
-    const uint32_t wq_o = ring_o + qg * kMRowStride + qt * 4;          // + stage + group
-    const uint32_t sc_o = ring_o + kMScaleOff + qg * 16;
+    // row qg's codes: bits 4..6 of this offset hold qg (the stage bases are
+    // multiples of 1024 from a 128-aligned array start), so XOR-ing gl * 16
+    // gives the swizzled chunk of group gl; row qg + 8 is 1024 bytes on
+    const uint32_t wq_o = (uint32_t)(ring_c - smem) + qg * 128 + qt * 4 + (qg << 4);   // + stage * 2048
+    const uint32_t sc_o = (uint32_t)(ring_s - smem) + qg * 16;                          // + stage * 256
     const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? 0 : qt * 16);
-    uint32_t so = 0;                // ring stage offset of the next item to compute
+    uint32_t st = 0;                // ring stage of the next item to compute
     int cs = 0;
 
     for (int ph = 0; ph < nphase; ++ph) {
@@ -470,7 +480,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
                         uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
                         if (sasync) {
-                            const unsigned char *sp = smem + sc_o + so;
+                            const unsigned char *sp = smem + sc_o + (st << 8);
                             sg = *reinterpret_cast<const uint4 *>(sp);
                             sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
                             if (gsh) {
@@ -498,14 +508,15 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         }
                         const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
                         // shared-memory pointers of the item; the unrolled groups add constants
-                        const unsigned char *wp = smem + wq_o + so;
+                        const uint32_t wb = wq_o + (st << 11);
                         const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
                         const unsigned char *bp[NT];
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
                         auto step = [&](int gl) {
-                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wp + gl * 16);
-                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wp + 8 * kMRowStride + gl * 16);
+                            const unsigned char *wa = smem + (wb ^ (uint32_t)(gl << 4));
+                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wa);
+                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wa + 1024);
                             const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
                             const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
                                                     w1s & 0x000F000Fu};
@@ -542,7 +553,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         }
                         __syncwarp();
                         issue_next();
-                        so = (so + kMStage == (uint32_t)(S * kMStage)) ? 0u : so + kMStage;
+                        st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
                         xoff += xstep;
                         coff += cstep;
                     }
