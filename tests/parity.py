@@ -56,6 +56,19 @@ def abs_products(oracle, qw, scales, x, rows=None) -> np.ndarray:
     return oracle.gemv(oracle.pack(qa), scales, xa, rows=rows, threads=8)
 
 
+def gate_up_bound(oracle, qw, s, x, rows):
+    """Element bound for SiLU(g) u: with |dg| <= eg, |du| <= eu (accumulation
+    errors as for a plain projection) the product moves by at most
+    |SiLU'| eg |u| + |SiLU(g)| eu + eg eu, and |SiLU'| <= 1.1."""
+    N = qw.shape[0] // 2
+    g = oracle.gemv(qw, s, x, rows=rows, threads=8)
+    u = oracle.gemv(qw, s, x, rows=rows + N, threads=8)
+    eg = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows)
+    eu = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows + N)
+    silu = g / (1.0 + np.exp(-g))
+    return (1.1 * eg * np.abs(u) + np.abs(silu) * eu + eg * eu) / ACC_BOUND
+
+
 def assert_f16_matches(got: np.ndarray, ref: np.ndarray, what: str = "", absprod=None):
     got = np.asarray(got, dtype=np.float16)
     ref = np.asarray(ref, dtype=np.float64)

@@ -6,7 +6,7 @@ import pytest
 from int4_group_quantized_q4f16_b200 import synth
 import oracle_pins as P
 from parity import (ACC_BOUND, abs_products, assert_f16_matches, assert_f32_matches, check_argmax, dev,
-                    host, rel_l2)
+                    gate_up_bound, host, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -133,19 +133,6 @@ def test_gate_up(zt, oracle, M, N, K):
                                      np.random.default_rng(N).integers(0, N, 64)])).astype(np.int32)
     ref = oracle.gate_up_silu(qw, s, x, rows=rows, threads=8)
     assert_f16_matches(got[:, rows], ref, f"gate_up M{M} N{N} K{K}", gate_up_bound(oracle, qw, s, x, rows))
-
-
-def gate_up_bound(oracle, qw, s, x, rows):
-    """Element bound for SiLU(g) u: with |dg| <= eg, |du| <= eu (accumulation
-    errors as for a plain projection) the product moves by at most
-    |SiLU'| eg |u| + |SiLU(g)| eu + eg eu, and |SiLU'| <= 1.1."""
-    N = qw.shape[0] // 2
-    g = oracle.gemv(qw, s, x, rows=rows, threads=8)
-    u = oracle.gemv(qw, s, x, rows=rows + N, threads=8)
-    eg = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows)
-    eu = ACC_BOUND * abs_products(oracle, qw, s, x, rows=rows + N)
-    silu = g / (1.0 + np.exp(-g))
-    return (1.1 * eg * np.abs(u) + np.abs(silu) * eu + eg * eu) / ACC_BOUND
 
 
 def test_gate_up_order_pinned(zt, oracle):
