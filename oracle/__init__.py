@@ -107,8 +107,11 @@ class Oracle:
         lib.zto_double_to_half.restype = ctypes.c_uint16
         lib.zto_add_rmsnorm.argtypes = [_P, _P, _P, _I, _I, ctypes.c_double, _P, _P]
         lib.zto_gemv_rope.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, ctypes.c_double, _P, _I]
+        lib.zto_dequant_f16.argtypes = [_P, _P, _I, _I, _I, _P]
+        lib.zto_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I]
         for f in (lib.zto_unpack, lib.zto_pack, lib.zto_gemv,
-                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm, lib.zto_gemv_rope):
+                  lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm, lib.zto_gemv_rope,
+                  lib.zto_dequant_f16, lib.zto_gemm_f16w):
             f.restype = ctypes.c_int
         self._lib = lib
 
@@ -163,6 +166,32 @@ class Oracle:
                                 _ptr(r) if r is not None else None, nr, _ptr(y), threads)
         if rc:
             raise ValueError("zto_gemv rejected its arguments")
+        return y
+
+    def dequant_f16(self, qw, scales) -> np.ndarray:
+        """w16[n][k] = fp16((q[n][k] - 7) * s[n][k/group]), round to nearest
+        even, as binary16 bit patterns viewed as float16 [N][K]."""
+        qw = np.ascontiguousarray(qw, dtype=np.uint32)
+        s = _u16(scales)
+        N, K = qw.shape[0], qw.shape[1] * 8
+        w = np.empty((N, K), dtype=np.uint16)
+        if self._lib.zto_dequant_f16(_ptr(qw), _ptr(s), N, K, _group(K, s), _ptr(w)):
+            raise ValueError("zto_dequant_f16 rejected its arguments")
+        return w.view(np.float16)
+
+    def gemm_f16w(self, qw, scales, x, rows=None, threads: int = 1) -> np.ndarray:
+        """y[m][i] = sum_k w16[n_i][k] * x[m][k] in double, w16 as dequant_f16."""
+        qw = np.ascontiguousarray(qw, dtype=np.uint32)
+        s = _u16(scales)
+        x = _u16(np.atleast_2d(x))
+        N, K = qw.shape[0], qw.shape[1] * 8
+        M = x.shape[0]
+        r, nr = self._rows(rows)
+        y = np.empty((M, nr if r is not None else N), dtype=np.float64)
+        rc = self._lib.zto_gemm_f16w(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s),
+                                     _ptr(r) if r is not None else None, nr, _ptr(y), threads)
+        if rc:
+            raise ValueError("zto_gemm_f16w rejected its arguments")
         return y
 
     def gate_up_silu(self, qw, scales, x, rows=None, threads: int = 1) -> np.ndarray:

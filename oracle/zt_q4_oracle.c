@@ -38,6 +38,14 @@
  *   rotation is read): within each head of d features, feature pair
  *   (i, i + d/2) of token m turns by pos[m] * theta^(-2i/d).
  *
+ *   batched prefill (limitations section, item on sequential prefill: the
+ *   project ships batched-prefill shaders without wiring them in; its
+ *   shaders need WebGPU's shader-f16, i.e. they compute in f16): for M
+ *   tokens at once the weights are first dequantized to binary16 the way an
+ *   f16 shader forms them, w16[n][k] = fp16((q[n][k] - 7) * s) -- the
+ *   product is exact in double, so this is one correct rounding -- and then
+ *   y[m][n] = sum_k w16[n][k] * x[m][k] in plain k order.
+ *
  *   residual add + RMSNorm ("add_norm.wgsl": the residual connection and
  *   RMSNorm in one step, section "内核融合"; the pages give no formula, so
  *   the standard RMSNorm is read): per row m, h = fp16(residual + delta)
@@ -301,6 +309,45 @@ int zto_gemv_rope(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
             const double phi = (double)pos[m] * inv_freq;
             out[m * N + n] = a * cos(phi) - b * sin(phi);
             out[m * N + n2] = b * cos(phi) + a * sin(phi);
+        }
+    }
+    return 0;
+}
+
+/* Dequantize to binary16: w16[n][k] = fp16((q[n][k] - 7) * s[n][k/group]),
+ * round to nearest even (zto_double_to_half); the product itself is exact in
+ * double (a 4-bit integer times an 11-bit significand). */
+int zto_dequant_f16(const uint32_t *qw, const uint16_t *scales, int N, int K, int group, uint16_t *w16)
+{
+    if (!qw || !scales || !w16 || !zto_shape_ok(1, N, K, group)) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            w16[n * K + k] = zto_double_to_half(zto_weight(qw, scales, K, group, n, k));
+    return 0;
+}
+
+/* Batched product on the binary16 weights: y[m][i] = sum_k w16[row_i][k] x[m][k]
+ * with w16 as zto_dequant_f16 forms it, summed in double in plain k order.
+ * rows / n_rows / y as in zto_gemv. */
+int zto_gemm_f16w(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                  int M, int N, int K, int group, const int32_t *rows, int n_rows,
+                  double *y, int threads)
+{
+    if (!qw || !scales || !x || !y || !zto_shape_ok(M, N, K, group)) return -1;
+    if (!rows) n_rows = N;
+    for (int i = 0; rows && i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= N) return -1;
+    if (threads < 1) threads = 1;
+#pragma omp parallel for schedule(static) num_threads(threads)
+    for (int i = 0; i < n_rows; ++i) {
+        const int64_t n = rows ? rows[i] : i;
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double w = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));
+                acc += w * zto_half_to_double(x[m * K + k]);
+            }
+            y[m * n_rows + i] = acc;
         }
     }
     return 0;

@@ -500,4 +500,110 @@ def pin_group_whole_row_brute_force(o):
         assert abs(Fraction(y[0, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 200)
 
 
+
+
+# -------------------------------------- batched prefill on fp16 weights ----
+# The limitations section of the Zero-TVM write-up: batched-prefill shaders
+# exist (not wired in), and the shaders compute in f16.  Read as
+# w16 = fp16((q - 7) * s), then y = sum_k w16 x in plain k order.
+
+GOLDEN_F16 = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "q4_dequant_f16.txt")
+
+
+def _golden_f16():
+    ws, ys = [], []
+    with open(GOLDEN_F16) as fh:
+        for raw in fh:
+            tok = raw.split("#", 1)[0].split()
+            if not tok:
+                continue
+            if tok[0] == "w":
+                ws.append((int(tok[1]), int(tok[2], 16), int(tok[3], 16)))
+            elif tok[0] == "y":
+                ys.append((int(tok[1]), int(tok[2]), int(tok[3], 16), int(tok[4], 16), float(tok[5])))
+    return ws, ys
+
+
+def _row_of_codes(code: int, K: int) -> np.ndarray:
+    word = int("".join([format(code, "x")] * 8), 16)       # eight equal hex digits
+    return np.full((1, K // 8), word, dtype=np.uint32)
+
+
+def pin_dequant_f16_golden(o):
+    ws, ys = _golden_f16()
+    for code, sbits, wbits in ws:
+        qw = _row_of_codes(code, 32)
+        s = np.array([[sbits]], dtype=np.uint16).view(np.float16)
+        got = o.dequant_f16(qw, s).view(np.uint16)
+        assert np.all(got == wbits), f"code {code} scale {sbits:#06x}: {got[0, 0]:#06x} vs {wbits:#06x}"
+    for K, code, sbits, xbits, y in ys:
+        qw = _row_of_codes(code, K)
+        s = np.full((1, K // 32), sbits, dtype=np.uint16).view(np.float16)
+        x = np.full((1, K), xbits, dtype=np.uint16).view(np.float16)
+        assert o.gemm_f16w(qw, s, x)[0, 0] == y
+
+
+def pin_dequant_f16_is_numpy_rounding(o):
+    """Against numpy's double -> binary16 conversion of the exact product
+    (codes by the hex route), over random codes and scales from subnormal to
+    large, groups 32 and 64."""
+    rng = np.random.default_rng(41)
+    N, K = 24, 256
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    q = codes_by_hex(qw).astype(np.float64) - 7.0
+    for G in (32, 64):
+        sb = rng.integers(0, 0x7C00, size=(N, K // G), dtype=np.uint16)
+        s = sb.view(np.float16)
+        with np.errstate(over="ignore"):
+            ref = (q * np.repeat(s.astype(np.float64), G, axis=1)).astype(np.float16)
+        assert np.array_equal(o.dequant_f16(qw, s).view(np.uint16), ref.view(np.uint16))
+
+
+def pin_gemm_f16w_exact_when_scales_are_short(o):
+    """Scales with at most 7 significant bits make (q - 7) s exact in fp16
+    (4 + 7 bits), so the fp16-weight product equals the exact one bit for bit."""
+    rng = np.random.default_rng(42)
+    N, K, M = 16, 192, 3
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    mant = rng.integers(64, 128, size=(N, K // 32)).astype(np.float64)
+    s = (mant * 2.0 ** rng.integers(-16, -8, size=(N, K // 32))).astype(np.float16)
+    assert np.array_equal(s.astype(np.float64), mant * 2.0 ** np.round(np.log2(s.astype(np.float64) / mant)))
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    assert np.array_equal(o.gemm_f16w(qw, s, x), o.gemv(qw, s, x))
+
+
+def pin_gemm_f16w_one_hot_and_brute_force(o):
+    """x = e_k picks numpy's fp16 rounding of (q - 7) s at column k; a tiny
+    case summed in exact rationals over numpy-rounded weights."""
+    rng = np.random.default_rng(43)
+    N, K = 5, 64
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s = rng.uniform(0.3, 3.0, size=(N, K // 32)).astype(np.float16)
+    w16 = ((codes_by_hex(qw).astype(np.float64) - 7.0) * np.repeat(s.astype(np.float64), 32, axis=1)).astype(np.float16)
+    eye = np.eye(K, dtype=np.float16)
+    y = o.gemm_f16w(qw, s, eye)                       # y[k][n] = w16[n][k]
+    assert np.array_equal(y.T, w16.astype(np.float64))
+    x = rng.standard_normal((3, K)).astype(np.float16)
+    y = o.gemm_f16w(qw, s, x)
+    for m in range(3):
+        for n in range(N):
+            exact = sum(Fraction(float(w16[n, k])) * Fraction(float(x[m, k])) for k in range(K))
+            assert abs(Fraction(y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 48) + Fraction(1, 2 ** 200)
+
+
+def pin_gemm_f16w_rows_and_tokens(o):
+    """Row subsets and token rows are independent: a subset and a single token
+    return the same numbers as the full product."""
+    rng = np.random.default_rng(44)
+    N, K, M = 40, 96, 4
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s = rng.uniform(0.005, 0.02, size=(N, K // 32)).astype(np.float16)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    full = o.gemm_f16w(qw, s, x)
+    rows = np.array([39, 0, 17, 17, 5], dtype=np.int32)
+    assert np.array_equal(o.gemm_f16w(qw, s, x, rows=rows), full[:, rows])
+    for m in range(M):
+        assert np.array_equal(o.gemm_f16w(qw, s, x[m:m + 1])[0], full[m])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
