@@ -58,6 +58,7 @@
  */
 #include <math.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <stdint.h>
 
 #define ZTO_GROUP 32   /* k values per fp16 scale in the q4f16 format (callers pass it; larger groups also work) */
@@ -328,7 +329,8 @@ int zto_dequant_f16(const uint32_t *qw, const uint16_t *scales, int N, int K, in
 
 /* Batched product on the binary16 weights: y[m][i] = sum_k w16[row_i][k] x[m][k]
  * with w16 as zto_dequant_f16 forms it, summed in double in plain k order.
- * rows / n_rows / y as in zto_gemv. */
+ * Each row's w16 values are formed once into a scratch row and then used for
+ * every token.  rows / n_rows / y as in zto_gemv. */
 int zto_gemm_f16w(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
                   int M, int N, int K, int group, const int32_t *rows, int n_rows,
                   double *y, int threads)
@@ -338,17 +340,24 @@ int zto_gemm_f16w(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
     for (int i = 0; rows && i < n_rows; ++i)
         if (rows[i] < 0 || rows[i] >= N) return -1;
     if (threads < 1) threads = 1;
-#pragma omp parallel for schedule(static) num_threads(threads)
+    int bad = 0;
+#pragma omp parallel for schedule(static) num_threads(threads) reduction(| : bad)
     for (int i = 0; i < n_rows; ++i) {
         const int64_t n = rows ? rows[i] : i;
+        double *w = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!w) {
+            bad = 1;
+            continue;
+        }
+        for (int64_t k = 0; k < K; ++k)
+            w[k] = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));
         for (int64_t m = 0; m < M; ++m) {
             double acc = 0.0;
-            for (int64_t k = 0; k < K; ++k) {
-                const double w = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));
-                acc += w * zto_half_to_double(x[m * K + k]);
-            }
+            for (int64_t k = 0; k < K; ++k)
+                acc += w[k] * zto_half_to_double(x[m * K + k]);
             y[m * n_rows + i] = acc;
         }
+        free(w);
     }
-    return 0;
+    return bad ? -1 : 0;
 }

@@ -52,11 +52,11 @@ MUTANTS = [
     ("rope_frequency_exponent", "pow(theta, -2.0 * (double)i / (double)head_dim)", "pow(theta, -(double)i / (double)head_dim)"),
     ("rope_first_token_position", "const double phi = (double)pos[m] * inv_freq;", "const double phi = (double)pos[0] * inv_freq;"),
     ("gemm_f16w_weights_not_rounded",
-     "const double w = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));",
-     "const double w = zto_weight(qw, scales, K, group, n, k);"),
+     "w[k] = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));",
+     "w[k] = zto_weight(qw, scales, K, group, n, k);"),
     ("dequant_f16_transposed", "w16[n * K + k] = zto_double_to_half", "w16[k * N + n] = zto_double_to_half"),
-    ("gemm_f16w_first_token_for_all", "acc += w * zto_half_to_double(x[m * K + k]);",
-     "acc += w * zto_half_to_double(x[k]);"),
+    ("gemm_f16w_first_token_for_all", "acc += w[k] * zto_half_to_double(x[m * K + k]);",
+     "acc += w[k] * zto_half_to_double(x[k]);"),
     ("gemm_f16w_rows_ignored", "const int64_t n = rows ? rows[i] : i;", "const int64_t n = i;"),
     ("sampled_rows_ignored", "int64_t n = rows ? rows[i] : i;\n        for (int64_t m = 0; m < M; ++m)\n            y[",
      "int64_t n = i;\n        for (int64_t m = 0; m < M; ++m)\n            y["),
