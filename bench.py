@@ -80,10 +80,15 @@ def alg_bytes(p: synth.Proj, M: int = 1) -> int:
     return p.weight_bytes() + M * p.K * 2 + M * p.n_out * out_bytes + (4 * M if p.kind == "lm_head" else 0)
 
 
+PASS_KERNEL_SOURCES = ("q4_gemv.cuh", "q4_mma.cuh", "q4_pass.cuh", "q4_stream.cuh")
+
+
 def kernel_sources_sha() -> str:
+    """Hash of the device sources the pass kernel and the argmax reduction are
+    compiled from; a recorded DRAM traffic figure is used only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int4_group_quantized_q4f16_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in PASS_KERNEL_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
