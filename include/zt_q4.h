@@ -17,7 +17,8 @@
  *           4*(k%8) .. 4*(k%8)+3 of qw[n][k/8] (low nibble first), 0..15.
  *   scales  IEEE binary16 bit patterns [n_rows][K/32]: one scale per 32 k.
  *   dequant w[n][k] = (code - 7) * scales[n][k/32]   (zero point 7).
- *   x       IEEE binary16 [M][K], M = number of tokens (1..16).
+ *   x       IEEE binary16 [M][K], M = number of tokens (1..16; the batched
+ *           prefill entry points below take any M >= 1).
  *   Products are exact and accumulate in fp32; fp16 outputs are rounded once,
  *   to nearest even, at the store.
  *
@@ -31,7 +32,7 @@
  *     synchronization, as for any CUDA launch.
  *   - Every argument is checked on the host BEFORE anything is launched; a
  *     call that returns a negative status launched nothing and wrote nothing.
- *   - Shapes: 1 <= M <= 16, N >= 1, K >= 32, K % 32 == 0, and the products
+ *   - Shapes (decode entry points): 1 <= M <= 16, N >= 1, K >= 32, K % 32 == 0, and the products
  *     n_rows*K and M*K fit in int64 (n_rows = N, or 2N for gate/up).
  *   - Alignment: qw and x 16 bytes; scales and y 2 bytes; logits and argmax
  *     4 bytes; workspace 16 bytes.
@@ -245,6 +246,44 @@ ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, si
 
 /* Synchronous read of a finished pass's error word (0: no bounded wait expired). */
 ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
+
+/*
+ * BATCHED PREFILL (M > 16 tokens; any M >= 1 is accepted)
+ *
+ * Zero-TVM write-up, limitations section: the project ships shaders for
+ * batched prefill (not wired into its decode loop), and its shaders compute
+ * in f16 (WebGPU shader-f16).  For M tokens at once the weights are first
+ * dequantized to binary16 the way an f16 shader forms them,
+ *     w16[n][k] = fp16((code - 7) * scales[n][k/group])   (one rounding, to nearest even),
+ * and then y[m][n] = fp16(sum_k w16[n][k] * x[m][k]) with fp32 accumulation on
+ * the tensor cores (tcgen05, kind::f16).  This is NOT the decode entry points'
+ * arithmetic (they use the exact products (code - 7) * s); the difference is
+ * the rounding of each weight to binary16.
+ *
+ * zt_q4_dequant_f16: w16 (DEVICE, fp16 [N][K], 16-byte aligned) from qw [N][K/8]
+ *     and scales [N][K/group].  group: 0 or 32, 64, 128 (K % group == 0).  HBM-bound
+ *     streaming kernel; a caller that runs many prefill batches may keep w16 and
+ *     call zt_q4_gemm_f16w directly.
+ * zt_q4_gemm_f16w: y fp16 [M][N] = x fp16 [M][K] times w16^T.  err is a DEVICE
+ *     uint32 the kernel ORs bit 0 into if one of its bounded waits (2 s) expired
+ *     (outputs are then incomplete); the caller zeroes it.  w16 and x 16-byte
+ *     aligned, y 2 bytes, err 4.
+ * zt_q4_gemm: both steps; workspace (DEVICE, 16-byte aligned, at least
+ *     zt_q4_gemm_workspace_bytes(N, K) bytes) holds w16 and the error word, which
+ *     the dequant launch clears; read it with zt_q4_gemm_errors (synchronous).
+ *     Two launches on `stream`.
+ * Shapes: 1 <= M <= 2^22, N >= 1, K >= 32, K % 32 == 0, N*K <= 2^40.  Inputs and
+ * outputs must not overlap.  Status codes as elsewhere; ZT_ERR_DEVICE also when the
+ * TMA descriptor encoder is unavailable.
+ */
+ZT_API int zt_q4_dequant_f16(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int group,
+                             void *stream);
+ZT_API int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K,
+                           unsigned int *err, void *stream);
+ZT_API size_t zt_q4_gemm_workspace_bytes(int N, int K);
+ZT_API int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M, int N,
+                      int K, int group, void *workspace, size_t ws_bytes, void *stream);
+ZT_API int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out);
 
 /*
  * Host-side layout helpers (HOST pointers, synchronous, no CUDA calls).

@@ -1,0 +1,297 @@
+// q4_gemm_tc.cuh -- batched (prefill) product on the 5th-generation tensor cores.
+//
+// Zero-TVM write-up, limitations section: the project ships batched-prefill
+// shaders (not wired into its decode loop), and its shaders compute in f16
+// (WebGPU shader-f16).  For M tokens at once the product becomes a real GEMM,
+// so it is split in two launches:
+//
+//   1. q4_dequant_f16_kernel  -- w16[n][k] = fp16((q - 7) * s), one correct
+//      rounding per weight (HBM-bound: 0.5625 B read, 2 B written per weight);
+//   2. q4_gemm_tc_kernel      -- y[m][n] = fp16(sum_k w16[n][k] x[m][k]) with
+//      tcgen05.mma (kind::f16, fp32 accumulator in tensor memory).
+//
+// Dequantizing inside the GEMM would cost ~1.6 instructions per weight for
+// every CTA that touches the weight, several times the tensor-core time of a
+// 128 x 256 tile; writing w16 once and streaming it with TMA keeps the GEMM a
+// plain fp16 contraction.
+//
+// GEMM layout ("swap AB"): the weight rows are the MMA's M dimension (128 per
+// CTA, TMEM lane = weight row) and the tokens its N dimension (BT = 64, 128 or
+// 256 per CTA, TMEM column = token), so a prefill of a few dozen tokens does
+// not pad the 128-row MMA.  Both operands are K-major fp16 tiles of 64 k
+// (one 128-byte row per weight row / token), loaded by TMA with the 128-byte
+// swizzle that the UMMA shared-memory descriptor names.
+//
+// Roles (128 threads): thread 0 issues TMA loads into an S-stage ring, thread
+// 32 issues the MMAs (4 x K=16 per stage) and frees each stage with
+// tcgen05.commit; all four warps then read the accumulator (warp w owns TMEM
+// lanes 32w..32w+31) and store y.  Every mbarrier wait is bounded (2 s of
+// globaltimer); on expiry the thread sets bit 0 of *err, stops issuing, and
+// the CTA still drains its loads and frees its tensor memory.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace zt {
+
+// ------------------------------------------------------------ dequant ----
+// One thread per 16-byte chunk of codes (32 consecutive k of one row).
+// (1024 + q) is the fp16 pattern 0x6400 | q; subtracting 1031 = 0x6407 gives
+// q - 7 exactly, and __hmul2 rounds (q - 7) * s once, to nearest even.
+__device__ __forceinline__ uint32_t dq_pair(uint32_t codes2, __half2 s2)
+{
+    uint32_t v = codes2 | 0x64006400u;
+    __half2 h = *reinterpret_cast<__half2 *>(&v);
+    h = __hmul2(__hsub2(h, __half2half2(__ushort_as_half((unsigned short)0x6407))), s2);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint4 dq_word(uint32_t w, __half2 s2)
+{
+    const uint32_t a = dq_pair(w & 0x000F000Fu, s2);          // k 0, 4
+    const uint32_t b = dq_pair((w >> 4) & 0x000F000Fu, s2);   // k 1, 5
+    const uint32_t c = dq_pair((w >> 8) & 0x000F000Fu, s2);   // k 2, 6
+    const uint32_t d = dq_pair((w >> 12) & 0x000F000Fu, s2);  // k 3, 7
+    uint4 o;
+    o.x = __byte_perm(a, b, 0x5410);   // k 0, 1
+    o.y = __byte_perm(c, d, 0x5410);   // k 2, 3
+    o.z = __byte_perm(a, b, 0x7632);   // k 4, 5
+    o.w = __byte_perm(c, d, 0x7632);   // k 6, 7
+    return o;
+}
+
+// qw as uint4 [N][K/32], scales [N][K/group], w16 as uint4 [N][K/8].
+// gsh = log2(group / 32).  err (may be null) is cleared by thread 0 so the
+// GEMM that follows on the stream starts with a clean error word.
+__global__ void __launch_bounds__(256) q4_dequant_f16_kernel(const uint4 *__restrict__ qw,
+                                                             const __half *__restrict__ scales,
+                                                             uint4 *__restrict__ w16, long long chunks, int cpr,
+                                                             int gsh, unsigned int *err)
+{
+    if (err && blockIdx.x == 0 && threadIdx.x == 0) *err = 0u;
+    const int spr = cpr >> gsh;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < chunks; c += stride) {
+        const long long n = c / cpr;
+        const int j = (int)(c - n * cpr);
+        const uint4 q = ldg_stream(qw + c);
+        const __half2 s2 = __half2half2(scales[n * spr + (j >> gsh)]);
+        uint4 *dst = w16 + 4 * c;
+        dst[0] = dq_word(q.x, s2);
+        dst[1] = dq_word(q.y, s2);
+        dst[2] = dq_word(q.z, s2);
+        dst[3] = dq_word(q.w, s2);
+    }
+}
+
+// --------------------------------------------------------------- GEMM ----
+constexpr int kTcRows = 128;      // weight rows per CTA (MMA M)
+constexpr int kTcK = 64;          // k per stage: one 128-byte swizzle row of fp16
+constexpr int kTcThreads = 128;
+constexpr unsigned kErrTcWait = 1u;
+
+template <int BT>
+struct TcCfg {
+    static constexpr int kABytes = kTcRows * kTcK * 2;                  // 16 KB
+    static constexpr int kBBytes = BT * kTcK * 2;                       // 8, 16 or 32 KB
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (192 * 1024) / kStageBytes;          // 8, 6 or 4
+    static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;    // + alignment + barriers
+    // instruction descriptor, kind::f16: D f32 (bits 4-5 = 1), A and B f16
+    // (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
+    // M >> 4 at bit 24
+    static constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BT >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
+    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M = 128");
+    static_assert((BT & (BT - 1)) == 0 && BT >= 32, "tensor memory is allocated in powers of two >= 32 columns");
+    static_assert(kStages >= 2, "ring depth");
+};
+
+__device__ __forceinline__ unsigned long long tc_now()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of parity `par` of the mbarrier at shared address `bar`
+// to complete; false after 2 s.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t par, bool nap)
+{
+    unsigned long long t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        uint32_t ok;
+        asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                     : "=r"(ok) : "r"(bar), "r"(par) : "memory");
+        if (ok) return true;
+        if (it == 0) t0 = tc_now();
+        else if ((it & 15u) == 0 && tc_now() - t0 > 2000000000ull) return false;
+        if (nap) __nanosleep(256);
+    }
+}
+
+// UMMA shared-memory descriptor for a K-major tile in the 128-byte swizzle:
+// start address >> 4 (bits 0-13), leading byte offset 1 (unused for this
+// layout, bits 16-29), stride byte offset 1024 >> 4 between 8-row groups
+// (bits 32-45), version 1 (bits 46-47), base offset 0 (the tile is 1024-byte
+// aligned), layout 2 = SWIZZLE_128B (bits 61-63).
+__device__ __forceinline__ uint64_t tc_desc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tc_tma_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+// 32 consecutive TMEM columns of this warp's 32 lanes into r[0..31]; the wait
+// names the registers so no use is scheduled before the data has arrived.
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// tma_w: fp16 [N][K] (w16), box 64 x 128; tma_x: fp16 [M][K], box 64 x BT;
+// both 128-byte swizzled, out-of-range rows and k read as zero.
+template <int BT>
+__global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_w,
+                                                                   const __grid_constant__ CUtensorMap tma_x,
+                                                                   __half *__restrict__ y, int M, int N, int K,
+                                                                   unsigned int *err)
+{
+    using C = TcCfg<BT>;
+    constexpr int S = C::kStages;
+    extern __shared__ __align__(128) unsigned char tc_smem[];
+    const uint32_t raw = smem_u32(tc_smem);
+    const uint32_t ring = (raw + 1023u) & ~1023u;                     // swizzle atoms are 1024-byte aligned
+    const uint32_t bars = ring + S * C::kStageBytes;                  // full[S], empty[S], acc
+    const uint32_t slot = bars + (2 * S + 1) * 8;                     // TMEM base written by tcgen05.alloc
+    auto full = [&](int s) { return bars + 8u * s; };
+    auto empty = [&](int s) { return bars + 8u * (S + s); };
+    const uint32_t accb = bars + 8u * (2 * S);
+    volatile uint32_t *consumed_s = reinterpret_cast<volatile uint32_t *>(tc_smem + (slot + 8 - raw));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kTcRows, m0 = blockIdx.y * BT;
+    const int kb_n = (K + kTcK - 1) / kTcK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full(s)) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(empty(s)) : "memory");
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(accb) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        *consumed_s = 0u;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(BT)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    uint32_t tmem;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(slot) : "memory");
+
+    int issued = 0;
+    if (threadIdx.x == 0) {
+        // producer: stage s of round r waits until round r - 1 of s was consumed
+        for (int kb = 0; kb < kb_n; ++kb) {
+            const int s = kb % S, r = kb / S;
+            if (r > 0 && !tc_wait(empty(s), (uint32_t)((r - 1) & 1), false)) {
+                atomicOr(err, kErrTcWait);
+                break;
+            }
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full(s)),
+                         "r"(C::kStageBytes) : "memory");
+            const uint32_t a = ring + s * C::kStageBytes;
+            tc_tma_2d(a, &tma_w, kb * kTcK, n0, full(s));
+            tc_tma_2d(a + C::kABytes, &tma_x, kb * kTcK, m0, full(s));
+            issued = kb + 1;
+        }
+    } else if (threadIdx.x == 32) {
+        // MMA issuer
+        int kb = 0;
+        for (; kb < kb_n; ++kb) {
+            const int s = kb % S, r = kb / S;
+            if (!tc_wait(full(s), (uint32_t)(r & 1), false)) {
+                atomicOr(err, kErrTcWait);
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t a = ring + s * C::kStageBytes;
+            const uint64_t da = tc_desc_sw128(a), db = tc_desc_sw128(a + C::kABytes);
+#pragma unroll
+            for (int j = 0; j < kTcK / 16; ++j) {
+                // K = 16 fp16 = 32 bytes further along the swizzled row: +2 in the address field
+                const uint32_t acc = (kb | j) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                    ::"r"(tmem), "l"(da + 2 * j), "l"(db + 2 * j), "r"(C::kIdesc), "r"(acc));
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(empty(s))
+                         : "memory");
+        }
+        *consumed_s = (uint32_t)kb;
+        // all MMAs issued above complete before this arrives
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(accb)
+                     : "memory");
+    }
+    __syncwarp();
+
+    // epilogue: TMEM lane = weight row n, column = token m
+    const bool ok = tc_wait(accb, 0u, true);
+    if (!ok && lane == 0) atomicOr(err, kErrTcWait);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const int n = n0 + warp * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+    for (int c = 0; c < BT / 32; ++c) {
+        uint32_t r[32];
+        tc_ld32(trow + (uint32_t)(c * 32), r);
+        if (ok && n < N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int m = m0 + c * 32 + j;
+                if (m < M) y[(size_t)m * N + n] = __float2half_rn(__uint_as_float(r[j]));
+            }
+        }
+    }
+
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // loads issued but never consumed (only after an expired wait) land before the CTA exits
+        for (int kb = (int)*consumed_s; kb < issued; ++kb)
+            if (!tc_wait(full(kb % S), (uint32_t)((kb / S) & 1), false)) break;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BT) : "memory");
+    }
+}
+
+}  // namespace zt

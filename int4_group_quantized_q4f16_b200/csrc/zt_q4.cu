@@ -3,6 +3,8 @@
 //
 // Host side only: argument checks, launch-shape selection and launches.  Every
 // check runs before the first CUDA call, so a rejected call launches nothing.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -16,6 +18,7 @@
 #include "q4_stream.cuh"
 #include "q4_mma.cuh"
 #include "q4_pass.cuh"
+#include "q4_gemm_tc.cuh"
 #include "zt_q4.h"
 
 namespace {
@@ -417,11 +420,111 @@ void *noalloc_scratch()
     return ptr;
 }
 
+// ------------------------------------------------ batched (prefill) GEMM ----
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link to the
+// driver library needed).
+PFN_cuTensorMapEncodeTiled_v12000 tma_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        (void)cudaGetLastError();
+    });
+    return fn;
+}
+
+// fp16 [rows][K] row-major, boxes of 64 k x box_rows rows, 128-byte swizzle,
+// out-of-range elements read as zero.
+bool tma_map_f16(CUtensorMap *map, const void *base, int K, long long rows, int box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tma_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int check_gemm_shapes(int M, int N, int K)
+{
+    if (M < 1 || M > (1 << 22) || N < 1 || K < kGroup || K % kGroup) return ZT_ERR_INVALID_ARG;
+    if ((long long)N * K > (1ll << 40)) return ZT_ERR_INVALID_ARG;
+    return ZT_OK;
+}
+
+int group_shift(int K, int group)
+{
+    if (group == 0) group = kGroup;
+    if (group != 32 && group != 64 && group != 128) return -1;
+    if (K % group) return -1;
+    return group == 32 ? 0 : group == 64 ? 1 : 2;
+}
+
+size_t gemm_err_offset(int N, int K) { return ((size_t)N * (size_t)K * 2 + 255) & ~(size_t)255; }
+
+int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int gsh,
+                   unsigned int *err, cudaStream_t st)
+{
+    const void *fn = reinterpret_cast<const void *>(&q4_dequant_f16_kernel);
+    int sms = 0;
+    const int occ = resident_ctas(fn, 256, 0, sms);
+    if (occ < 1) return ZT_ERR_DEVICE;
+    const long long chunks = (long long)N * (K / 32);
+    const long long want = (chunks + 255) / 256;
+    const int grid = (int)std::max(1ll, std::min(want, (long long)sms * occ * 4));
+    clear_stale_error();
+    q4_dequant_f16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(qw),
+                                                  reinterpret_cast<const __half *>(scales),
+                                                  reinterpret_cast<uint4 *>(w16), chunks, K / 32, gsh, err);
+    return launch_status();
+}
+
+template <int BT>
+int launch_gemm_tc_bt(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
+                      cudaStream_t st)
+{
+    using C = TcCfg<BT>;
+    const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<BT>);
+    int sms = 0;
+    if (resident_ctas(fn, kTcThreads, C::kSmem, sms) < 1) return ZT_ERR_DEVICE;
+    CUtensorMap mw, mx;
+    if (!tma_map_f16(&mw, w16, K, N, kTcRows) || !tma_map_f16(&mx, x, K, M, BT)) return ZT_ERR_DEVICE;
+    const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows), (unsigned)((M + BT - 1) / BT));
+    clear_stale_error();
+    q4_gemm_tc_kernel<BT><<<grid, kTcThreads, C::kSmem, st>>>(mw, mx, reinterpret_cast<__half *>(y), M, N, K, err);
+    return launch_status();
+}
+
+// Tokens per CTA: the smallest of 64 / 128 / 256 that covers M, halved while
+// the grid would leave more than a quarter of the SMs idle.
+int launch_gemm_tc(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
+                   cudaStream_t st)
+{
+    int sms = 0;
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_gemm_tc_kernel<256>), kTcThreads, TcCfg<256>::kSmem,
+                      sms) < 1)
+        return ZT_ERR_DEVICE;
+    const long long nt = (N + kTcRows - 1) / kTcRows;
+    int bt = M <= 64 ? 64 : M <= 128 ? 128 : 256;
+    while (bt > 64 && nt * ((M + bt - 1) / bt) * 4 < 3ll * sms) bt /= 2;
+    if (bt == 256) return launch_gemm_tc_bt<256>(w16, x, y, M, N, K, err, st);
+    if (bt == 128) return launch_gemm_tc_bt<128>(w16, x, y, M, N, K, err, st);
+    return launch_gemm_tc_bt<64>(w16, x, y, M, N, K, err, st);
+}
+
 }  // namespace
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 1; }
+int zt_q4_version(void) { return (1 << 16) | 2; }
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -661,6 +764,66 @@ int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out)
     if (!workspace || !out || n < 1 || n > ZT_Q4_PASS_MAX) return ZT_ERR_INVALID_ARG;
     const size_t err_off = ((size_t)n * 4 + 15) & ~(size_t)15;
     const cudaError_t e = cudaMemcpy(out, reinterpret_cast<const unsigned char *>(workspace) + err_off,
+                                     sizeof(unsigned int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_DEVICE;
+    }
+    return ZT_OK;
+}
+
+int zt_q4_dequant_f16(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int group,
+                      void *stream)
+{
+    if (!qw || !scales || !w16) return ZT_ERR_INVALID_ARG;
+    if (check_gemm_shapes(1, N, K) != ZT_OK) return ZT_ERR_INVALID_ARG;
+    const int gsh = group_shift(K, group);
+    if (gsh < 0) return ZT_ERR_INVALID_ARG;
+    if (!aligned(qw, 16) || !aligned(w16, 16) || !aligned(scales, 2)) return ZT_ERR_MISALIGNED;
+    return launch_dequant(qw, scales, w16, N, K, gsh, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
+                    void *stream)
+{
+    if (!w16 || !x || !y || !err) return ZT_ERR_INVALID_ARG;
+    int rc = check_gemm_shapes(M, N, K);
+    if (rc) return rc;
+    if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(err, 4)) return ZT_ERR_MISALIGNED;
+    return launch_gemm_tc(w16, x, y, M, N, K, err, static_cast<cudaStream_t>(stream));
+}
+
+size_t zt_q4_gemm_workspace_bytes(int N, int K)
+{
+    if (check_gemm_shapes(1, N, K) != ZT_OK) return 0;
+    return gemm_err_offset(N, K) + 16;
+}
+
+int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M, int N, int K,
+               int group, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!qw || !scales || !x || !y || !workspace) return ZT_ERR_INVALID_ARG;
+    int rc = check_gemm_shapes(M, N, K);
+    if (rc) return rc;
+    const int gsh = group_shift(K, group);
+    if (gsh < 0) return ZT_ERR_INVALID_ARG;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(scales, 2) || !aligned(y, 2))
+        return ZT_ERR_MISALIGNED;
+    if (ws_bytes < gemm_err_offset(N, K) + 16) return ZT_ERR_WORKSPACE;
+    uint16_t *w16 = static_cast<uint16_t *>(workspace);
+    unsigned int *err = reinterpret_cast<unsigned int *>(static_cast<unsigned char *>(workspace) +
+                                                         gemm_err_offset(N, K));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_dequant(qw, scales, w16, N, K, gsh, err, st);
+    if (rc) return rc;
+    return launch_gemm_tc(w16, x, y, M, N, K, err, st);
+}
+
+int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out)
+{
+    if (!workspace || !out || check_gemm_shapes(1, N, K) != ZT_OK) return ZT_ERR_INVALID_ARG;
+    const cudaError_t e = cudaMemcpy(out, static_cast<const unsigned char *>(workspace) + gemm_err_offset(N, K),
                                      sizeof(unsigned int), cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) {
         g_last_cuda_error = e;

@@ -201,3 +201,63 @@ def test_pass_group_size_rejected(zt):
     for group, K in ((16, 256), (96, 384), (256, 512), (128, 320), (64, 96)):
         proj = P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, K, 0, 0, group)
         assert f((P * 1)(proj), 1, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG, (group, K)
+
+
+# ------------------------------------------------- batched prefill (M > 16) --
+def test_prefill_symbols_declared():
+    syms = declared_symbols(HEADER)
+    for want in ("zt_q4_dequant_f16", "zt_q4_gemm_f16w", "zt_q4_gemm", "zt_q4_gemm_workspace_bytes",
+                 "zt_q4_gemm_errors"):
+        assert want in syms
+
+
+def test_gemm_workspace_bytes(zt):
+    f = zt.lib.zt_q4_gemm_workspace_bytes
+    assert f(9216, 3072) == ((9216 * 3072 * 2 + 255) // 256) * 256 + 16
+    assert f(3, 32) == 256 + 16
+    assert f(0, 3072) == 0 and f(8, 48) == 0 and f(8, 0) == 0
+
+
+def test_gemm_arguments_rejected(zt):
+    """Every check runs before a launch: these calls touch no device memory."""
+    g = zt.lib.zt_q4_gemm
+    ws = zt.gemm_workspace_bytes(256, 64)
+    ok = [FAKE, FAKE, FAKE, FAKE, 40, 256, 64, 32, FAKE, ws, None]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["qw", "scales", "x", "y", "M", "N", "K", "group", "ws", "ws_bytes", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return g(*a)
+
+    for k in ("qw", "scales", "x", "y", "ws"):
+        assert call(**{k: None}) == zt.ZT_ERR_INVALID_ARG
+    assert call(M=0) == zt.ZT_ERR_INVALID_ARG
+    assert call(M=(1 << 22) + 1) == zt.ZT_ERR_INVALID_ARG
+    assert call(N=0) == zt.ZT_ERR_INVALID_ARG
+    assert call(K=48) == zt.ZT_ERR_INVALID_ARG
+    assert call(group=48) == zt.ZT_ERR_INVALID_ARG
+    assert call(group=128) == zt.ZT_ERR_INVALID_ARG          # K = 64 is not a multiple of 128
+    assert call(qw=FAKE + 8) == zt.ZT_ERR_MISALIGNED
+    assert call(x=FAKE + 8) == zt.ZT_ERR_MISALIGNED
+    assert call(ws=FAKE + 8) == zt.ZT_ERR_MISALIGNED
+    assert call(scales=FAKE + 1) == zt.ZT_ERR_MISALIGNED
+    assert call(y=FAKE + 1) == zt.ZT_ERR_MISALIGNED
+    assert call(ws_bytes=ws - 1) == zt.ZT_ERR_WORKSPACE
+
+
+def test_dequant_and_gemm_f16w_arguments_rejected(zt):
+    d = zt.lib.zt_q4_dequant_f16
+    assert d(None, FAKE, FAKE, 8, 64, 32, None) == zt.ZT_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE, 8, 48, 32, None) == zt.ZT_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE, 8, 64, 16, None) == zt.ZT_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE + 8, 8, 64, 32, None) == zt.ZT_ERR_MISALIGNED
+    assert d(FAKE + 4, FAKE, FAKE, 8, 64, 32, None) == zt.ZT_ERR_MISALIGNED
+    f = zt.lib.zt_q4_gemm_f16w
+    assert f(FAKE, FAKE, FAKE, 17, 64, 64, None, None) == zt.ZT_ERR_INVALID_ARG      # no error word
+    assert f(FAKE, FAKE, FAKE, 0, 64, 64, FAKE, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(FAKE + 8, FAKE, FAKE, 17, 64, 64, FAKE, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, 17, 64, 64, FAKE + 2, None) == zt.ZT_ERR_MISALIGNED
+    out = ctypes.c_uint(0)
+    assert zt.lib.zt_q4_gemm_errors(None, 8, 64, ctypes.byref(out)) == zt.ZT_ERR_INVALID_ARG

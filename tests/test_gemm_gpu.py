@@ -1,0 +1,157 @@
+"""GPU parity of the batched (prefill) path: the binary16 dequantization
+(bit-exact against the oracle) and the tensor-core GEMM on those weights
+(element bound: fp32 accumulation, 2^-14 sum |w16 x|, plus one fp16 ulp)
+against the oracle's fp16-weight product (Zero-TVM write-up, limitations
+section: batched-prefill shaders, computing in f16)."""
+import numpy as np
+import pytest
+
+from int4_group_quantized_q4f16_b200 import synth
+from parity import F16_REL_L2, assert_f16_matches, dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def zt():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    return zt_q4
+
+
+def abs_products_f16w(oracle, qw, scales, x, rows=None):
+    """sum_k |w16_nk| |x_mk| by the oracle: |fp16((q - 7) s)| = fp16(|q - 7| |s|),
+    i.e. codes 7 + |q - 7| with |s|, against |x|."""
+    q = oracle.unpack(qw, qw.shape[1] * 8).astype(np.int16)
+    qa = (7 + np.abs(q - 7)).astype(np.uint8)
+    sa = np.abs(np.asarray(scales, dtype=np.float16))
+    xa = np.abs(np.asarray(x, dtype=np.float16))
+    return oracle.gemm_f16w(oracle.pack(qa), sa, xa, rows=rows, threads=8)
+
+
+def _prefill_x(seed, M, K):
+    return np.random.default_rng([seed, 91]).standard_normal((M, K)).astype(np.float16)
+
+
+@pytest.mark.parametrize("N,K,group", [(1, 32, 32), (3, 96, 32), (256, 3072, 32), (1000, 1024, 64),
+                                       (777, 2048, 128), (64, 11008, 32)])
+def test_dequant_f16_bit_exact(zt, oracle, N, K, group):
+    import torch
+    qw, s32, _ = synth.problem(500 + N, N, K, M=1, proj=1)
+    s = s32[:, ::group // 32].copy()
+    w16 = zt.dequant_f16(dev(qw), dev(s))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(w16).view(np.uint16), oracle.dequant_f16(qw, s).view(np.uint16))
+
+
+def test_dequant_f16_edge_scales(zt, oracle):
+    """Subnormal, tiny, huge (overflowing to inf), negative and zero scales."""
+    import torch
+    N, K = 64, 64
+    rng = np.random.default_rng(5)
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    bits = np.concatenate([rng.integers(0, 0x0400, 32), rng.integers(0x7800, 0x7C00, 32),
+                           rng.integers(0x8000, 0xFC00, 32), [0, 0x8000, 0x3C01, 0x3C03] * 8]).astype(np.uint16)
+    s = bits[:N * (K // 32)].reshape(N, K // 32).view(np.float16)
+    w16 = zt.dequant_f16(dev(qw), dev(s))
+    torch.cuda.synchronize()
+    with np.errstate(over="ignore"):
+        assert np.array_equal(host(w16).view(np.uint16), oracle.dequant_f16(qw, s).view(np.uint16))
+
+
+SHAPES = [
+    (17, 128, 64),          # one weight tile, one k block, 17 tokens of a 64-token tile
+    (1, 200, 96),           # M = 1, ragged N, K % 64 == 32
+    (64, 384, 1024),
+    (100, 300, 1056),       # ragged everything
+    (129, 256, 512),        # just past one 128-token tile
+    (256, 1024, 3072),
+    (300, 640, 2048),       # 256-token tiles with a ragged second tile
+    (40, 3072, 8192),       # Phi-3-mini down projection shape, 40 tokens
+]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_gemm_matches_oracle(zt, oracle, M, N, K):
+    import torch
+    qw, s, _ = synth.problem(600 + M, N, K, M=1, proj=0)
+    x = _prefill_x(M + N, M, K)
+    ws = torch.empty((zt.gemm_workspace_bytes(N, K),), dtype=torch.uint8, device="cuda")
+    y = zt.gemm(dev(qw), dev(s), dev(x), workspace=ws)
+    torch.cuda.synchronize()
+    assert zt.gemm_errors(ws, N, K) == 0
+    ref = oracle.gemm_f16w(qw, s, x, threads=8)
+    assert_f16_matches(host(y), ref, f"gemm M{M} N{N} K{K}", abs_products_f16w(oracle, qw, s, x))
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_gemm_groups(zt, oracle, group):
+    import torch
+    M, N, K = 48, 256, 1024
+    qw, s32, _ = synth.problem(700 + group, N, K, M=1, proj=2)
+    s = s32[:, ::group // 32].copy()
+    x = _prefill_x(group, M, K)
+    y = zt.gemm(dev(qw), dev(s), dev(x))
+    torch.cuda.synchronize()
+    assert_f16_matches(host(y), oracle.gemm_f16w(qw, s, x, threads=8), f"gemm group {group}",
+                       abs_products_f16w(oracle, qw, s, x))
+
+
+def test_gemm_full_size_sampled(zt, oracle):
+    """Prefill of 512 tokens through the Phi-3-mini qkv projection (3072 ->
+    9216) and the LM head rows (3072 -> 32064, fp16 out): sampled rows."""
+    import torch
+    for N, seed in ((9216, 1), (32064, 2)):
+        M, K = 512, 3072
+        qw, s, _ = synth.problem(seed, N, K, M=1, proj=0)
+        x = _prefill_x(seed, M, K)
+        y = host(zt.gemm(dev(qw), dev(s), dev(x)))
+        torch.cuda.synchronize()
+        rows = np.unique(np.concatenate([[0, 127, 128, N - 1], np.random.default_rng(seed).integers(0, N, 60)]))
+        rows = rows.astype(np.int32)
+        ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
+        assert_f16_matches(y[:, rows], ref, f"gemm N{N} sampled", abs_products_f16w(oracle, qw, s, x, rows=rows))
+
+
+def test_gemm_f16w_reuses_dequantized_weights(zt):
+    """dequant once + gemm_f16w equals the one-call gemm bit for bit, and
+    repeated calls are bit-identical."""
+    import torch
+    M, N, K = 77, 512, 2048
+    qw, s, _ = synth.problem(9, N, K, M=1, proj=3)
+    x = dev(_prefill_x(9, M, K))
+    qd, sd = dev(qw), dev(s)
+    w16 = zt.dequant_f16(qd, sd)
+    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    a = zt.gemm_f16w(w16, x, err=err)
+    b = zt.gemm(qd, sd, x)
+    c = zt.gemm(qd, sd, x)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(host(a).view(np.uint16), host(b).view(np.uint16))
+    assert np.array_equal(host(b).view(np.uint16), host(c).view(np.uint16))
+
+
+def test_gemm_exact_weights_match_decode_path(zt, oracle):
+    """With 7-bit scales the binary16 weights are exact, so the prefill GEMM
+    and the decode GEMV compute the same exact products: both within their
+    bounds of the exact oracle, for the same 16 tokens."""
+    import torch
+    M, N, K = 16, 384, 1024
+    rng = np.random.default_rng(12)
+    qw = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    mant = rng.integers(64, 128, size=(N, K // 32)).astype(np.float64)
+    s = (mant * 2.0 ** -13).astype(np.float16)
+    x = _prefill_x(12, M, K)
+    y_pre = host(zt.gemm(dev(qw), dev(s), dev(x)))
+    y_dec = host(zt.gemv(dev(qw), dev(s), dev(x)))
+    torch.cuda.synchronize()
+    ref = oracle.gemv(qw, s, x, threads=8)
+    assert np.array_equal(oracle.gemm_f16w(qw, s, x, threads=8), ref)
+    from parity import abs_products
+    bound = abs_products(oracle, qw, s, x)
+    assert_f16_matches(y_pre, ref, "prefill", bound)
+    assert_f16_matches(y_dec, ref, "decode", bound)
+    assert rel_l2(y_pre, y_dec) <= F16_REL_L2
