@@ -61,6 +61,10 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--prefill", action="store_true",
+                   help="instead of the pass: the batched prefill GEMM (binary16 dequant + tensor-core GEMM) on the "
+                        "Phi-3-mini qkv projection (K 3072, N 9216) at M = 128, 512, 2048 tokens, one JSON line per M")
+    p.add_argument("--prefill-m", type=str, default="128,512,2048")
     p.add_argument("--sweep-m", action="store_true",
                    help="instead of the pass: the fused gate_up projection (K 3072, 2 x 8192 rows) at M = 1, 2, 4, "
                         "8, 16, one JSON line per M")
@@ -649,6 +653,80 @@ def run_sweep_m(args, local):
               flush=True)
 
 
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return json.load(fh)
+    except (OSError, ValueError):
+        return {}
+
+
+def run_prefill(args, local):
+    """Batched prefill (M > 16): zt_q4_gemm = dequant to binary16 (HBM-bound)
+    + tcgen05 GEMM (tensor-bound) on the Phi-3-mini qkv projection.  Four
+    weight copies (4 x 28.3 MB of codes + 56.6 MB of w16 each) rotate so the
+    dequant streams from HBM; each timed region is bracketed by CUDA events on
+    the launching stream."""
+    import torch
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    K, N, copies = 3072, 9216, 4
+    p = synth.Proj("qkv", "gemv", K, N, synth.PROJ_QKV)
+    w = []
+    for c in range(copies):
+        qw, s, _ = synth.proj_inputs(args.seed, c, p)
+        qd, sd = torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)
+        ws = torch.empty((zt_q4.gemm_workspace_bytes(N, K),), dtype=torch.uint8, device=device)
+        w.append((qd, sd, ws, ws[:N * K * 2].view(torch.float16).view(N, K)))
+    peaks = measured_peaks()
+    tc_peak = peaks.get("bf16_tflops")
+    hbm_peak = peaks.get("hbm_gbs")
+    stream = torch.cuda.Stream(device=device)
+    err = torch.zeros((1,), dtype=torch.int32, device=device)
+
+    def timed(fn, steps):
+        with torch.cuda.stream(stream):
+            for i in range(max(args.warmup, 3) * copies):
+                fn(i)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(steps):
+                fn(i)
+            b.record(stream)
+            stream.synchronize()
+        return a.elapsed_time(b) / steps * 1e3
+
+    for M in [int(v) for v in args.prefill_m.split(",")]:
+        x = torch.randn((M, K), device=device).half()
+        y = torch.empty((M, N), dtype=torch.float16, device=device)
+        steps = max(min(args.steps, 200), 4 * copies)
+        both = timed(lambda i: zt_q4.gemm(w[i % copies][0], w[i % copies][1], x, y, w[i % copies][2],
+                                          stream=stream), steps)
+        gemm = timed(lambda i: zt_q4.gemm_f16w(w[i % copies][3], x, y, err, stream=stream), steps)
+        deq = timed(lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][3],
+                                                stream=stream), steps)
+        assert int(err.item()) == 0 and all(zt_q4.gemm_errors(c[2], N, K) == 0 for c in w)
+        flops = 2.0 * M * N * K
+        deq_bytes = N * K // 2 + N * (K // 32) * 2 + N * K * 2
+        g_tf = flops / gemm / 1e6
+        line = {"metric": "q4 prefill GEMM TFLOP/s (dequant to binary16 + tcgen05 GEMM)",
+                "value": round(flops / both / 1e6, 1), "unit": "TFLOP/s", "higher_is_better": True, "M": M,
+                "us_per_call": round(both, 2), "gemm_us": round(gemm, 2), "dequant_us": round(deq, 2),
+                "dtype": "f16 x f16 -> f32", "steps": steps, "weight_copies": copies,
+                "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                             "frac": round(g_tf / tc_peak, 4) if tc_peak else None,
+                             "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst; fp16 runs at the bf16 rate)",
+                             "kernel": "q4_gemm_tc_kernel"},
+                "dequant_roofline": {"bound": "hbm", "achieved": round(deq_bytes / deq / 1e3, 1), "peak": hbm_peak,
+                                     "unit": "GB/s", "frac": round(deq_bytes / deq / 1e3 / hbm_peak, 4)
+                                     if hbm_peak else None, "bytes_per_call": deq_bytes},
+                "config": {"workload": f"Phi-3-mini qkv projection 3072->9216 for {M} tokens, q4 group-32, "
+                                       "weights dequantized per call"}}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args)
@@ -657,6 +735,8 @@ def main():
             run_reference(args, world, rank)
         elif args.sweep_m:
             run_sweep_m(args, local)
+        elif args.prefill:
+            run_prefill(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -15,15 +15,16 @@
 // 128 x 256 tile; writing w16 once and streaming it with TMA keeps the GEMM a
 // plain fp16 contraction.
 //
-// GEMM layout ("swap AB"): the weight rows are the MMA's M dimension (128 per
-// CTA, TMEM lane = weight row) and the tokens its N dimension (BT = 64, 128 or
-// 256 per CTA, TMEM column = token), so a prefill of a few dozen tokens does
-// not pad the 128-row MMA.  Both operands are K-major fp16 tiles of 64 k
+// GEMM layout: from 128 tokens on, the tokens are the MMA's M dimension (128
+// or 256 per CTA as one or two 128-row MMAs, TMEM lane = token) and the weight
+// rows its N dimension (64..256 per CTA, TMEM column = weight row).  Below 128
+// tokens the roles swap ("swap AB": weight rows as M, tokens as N = 64 or
+// 128), so a prefill of a few dozen tokens does not pad the 128-row MMA.  Both operands are K-major fp16 tiles of 64 k
 // (one 128-byte row per weight row / token), loaded by TMA with the 128-byte
 // swizzle that the UMMA shared-memory descriptor names.
 //
 // Roles (128 threads): thread 0 issues TMA loads into an S-stage ring, thread
-// 32 issues the MMAs (4 x K=16 per stage) and frees each stage with
+// 32 issues the MMAs (4 or 8 x K=16 per stage) and frees each stage with
 // tcgen05.commit; all four warps then read the accumulator (warp w owns TMEM
 // lanes 32w..32w+31) and store y.  Every mbarrier wait is bounded (2 s of
 // globaltimer); on expiry the thread sets bit 0 of *err, stops issuing, and
@@ -69,41 +70,64 @@ __global__ void __launch_bounds__(256) q4_dequant_f16_kernel(const uint4 *__rest
                                                              uint4 *__restrict__ w16, long long chunks, int cpr,
                                                              int gsh, unsigned int *err)
 {
+    constexpr int U = 4;   // chunks per thread per step: their loads are in flight together
     if (err && blockIdx.x == 0 && threadIdx.x == 0) *err = 0u;
     const int spr = cpr >> gsh;
     const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < chunks; c += stride) {
-        const long long n = c / cpr;
-        const int j = (int)(c - n * cpr);
-        const uint4 q = ldg_stream(qw + c);
-        const __half2 s2 = __half2half2(scales[n * spr + (j >> gsh)]);
-        uint4 *dst = w16 + 4 * c;
-        dst[0] = dq_word(q.x, s2);
-        dst[1] = dq_word(q.y, s2);
-        dst[2] = dq_word(q.z, s2);
-        dst[3] = dq_word(q.w, s2);
+    for (long long c0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; c0 < chunks; c0 += U * stride) {
+        uint4 q[U];
+        __half s[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long c = c0 + u * stride;
+            if (c < chunks) {
+                const long long n = c / cpr;
+                q[u] = ldg_stream(qw + c);
+                s[u] = scales[n * spr + ((int)(c - n * cpr) >> gsh)];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long c = c0 + u * stride;
+            if (c < chunks) {
+                const __half2 s2 = __half2half2(s[u]);
+                uint4 *dst = w16 + 4 * c;
+                dst[0] = dq_word(q[u].x, s2);
+                dst[1] = dq_word(q[u].y, s2);
+                dst[2] = dq_word(q[u].z, s2);
+                dst[3] = dq_word(q[u].w, s2);
+            }
+        }
     }
 }
 
 // --------------------------------------------------------------- GEMM ----
-constexpr int kTcRows = 128;      // weight rows per CTA (MMA M)
+constexpr int kTcMma = 128;       // rows of one MMA (M)
 constexpr int kTcK = 64;          // k per stage: one 128-byte swizzle row of fp16
 constexpr int kTcThreads = 128;
 constexpr unsigned kErrTcWait = 1u;
 
-template <int BT>
+// Operand tiles.  A: AM rows per CTA (128, or 256 as two 128-row MMAs that
+// share the B tile, into two accumulators); B: BN rows per CTA (the MMA N).
+// The 256-row A tile halves the bytes each SM takes in per MMA cycle (the
+// limit of the 128-row tile), at the cost of half as many CTAs.
+template <int AM, int BN>
 struct TcCfg {
-    static constexpr int kABytes = kTcRows * kTcK * 2;                  // 16 KB
-    static constexpr int kBBytes = BT * kTcK * 2;                       // 8, 16 or 32 KB
+    static constexpr int kHalves = AM / kTcMma;
+    static constexpr int kABytes = AM * kTcK * 2;                       // 16 or 32 KB
+    static constexpr int kBBytes = BN * kTcK * 2;                       // 8, 16 or 32 KB
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = (192 * 1024) / kStageBytes;          // 8, 6 or 4
+    static constexpr int kStages = (192 * 1024) / kStageBytes;          // 3..8
+    static constexpr int kTmemCols = kHalves * BN;
     static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;    // + alignment + barriers
     // instruction descriptor, kind::f16: D f32 (bits 4-5 = 1), A and B f16
     // (bits 7-9, 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 at bit 17,
     // M >> 4 at bit 24
-    static constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BT >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
-    static_assert(BT % 16 == 0 && BT >= 16 && BT <= 256, "MMA N for M = 128");
-    static_assert((BT & (BT - 1)) == 0 && BT >= 32, "tensor memory is allocated in powers of two >= 32 columns");
+    static constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kTcMma >> 4) << 24);
+    static_assert(AM == 128 || AM == 256, "one or two MMAs per k step");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
+    static_assert((BN & (BN - 1)) == 0 && BN >= 32, "tensor memory is allocated in powers of two >= 32 columns");
+    static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
     static_assert(kStages >= 2, "ring depth");
 };
 
@@ -170,15 +194,19 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32])
                  : "memory");
 }
 
-// tma_w: fp16 [N][K] (w16), box 64 x 128; tma_x: fp16 [M][K], box 64 x BT;
-// both 128-byte swizzled, out-of-range rows and k read as zero.
-template <int BT>
-__global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_w,
-                                                                   const __grid_constant__ CUtensorMap tma_x,
+// TOKA: the A operand holds tokens (x) and B weight rows (w16): TMEM lane =
+// token m, column = weight row n, so each thread ends with 32 consecutive
+// outputs of one token row and writes them as four 16-byte stores.  Otherwise
+// ("swap AB", for fewer than 128 tokens) A holds weight rows and B tokens.
+// tma_a / tma_b: fp16 [rows][K], boxes 64 x AM and 64 x BN, 128-byte swizzled,
+// out-of-range rows and k read as zero.
+template <int AM, int BN, bool TOKA>
+__global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
+                                                                   const __grid_constant__ CUtensorMap tma_b,
                                                                    __half *__restrict__ y, int M, int N, int K,
                                                                    unsigned int *err)
 {
-    using C = TcCfg<BT>;
+    using C = TcCfg<AM, BN>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(128) unsigned char tc_smem[];
     const uint32_t raw = smem_u32(tc_smem);
@@ -191,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     volatile uint32_t *consumed_s = reinterpret_cast<volatile uint32_t *>(tc_smem + (slot + 8 - raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kTcRows, m0 = blockIdx.y * BT;
+    const int a0 = blockIdx.x * AM, b0 = blockIdx.y * BN;
     const int kb_n = (K + kTcK - 1) / kTcK;
 
     if (threadIdx.x == 0) {
@@ -204,8 +232,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
         *consumed_s = 0u;
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(BT)
-                     : "memory");
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot),
+                     "r"(C::kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -226,8 +254,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full(s)),
                          "r"(C::kStageBytes) : "memory");
             const uint32_t a = ring + s * C::kStageBytes;
-            tc_tma_2d(a, &tma_w, kb * kTcK, n0, full(s));
-            tc_tma_2d(a + C::kABytes, &tma_x, kb * kTcK, m0, full(s));
+            tc_tma_2d(a, &tma_a, kb * kTcK, a0, full(s));
+            tc_tma_2d(a + C::kABytes, &tma_b, kb * kTcK, b0, full(s));
             issued = kb + 1;
         }
     } else if (threadIdx.x == 32) {
@@ -246,10 +274,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
             for (int j = 0; j < kTcK / 16; ++j) {
                 // K = 16 fp16 = 32 bytes further along the swizzled row: +2 in the address field
                 const uint32_t acc = (kb | j) ? 1u : 0u;
-                asm volatile(
-                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                    ::"r"(tmem), "l"(da + 2 * j), "l"(db + 2 * j), "r"(C::kIdesc), "r"(acc));
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h) {
+                    // rows 128h.. of the A tile start 16 KB (1024 in the address field) further
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                        ::"r"(tmem + (uint32_t)(h * BN)), "l"(da + (uint64_t)(h * 1024) + 2 * j), "l"(db + 2 * j),
+                        "r"(C::kIdesc), "r"(acc));
+                }
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(empty(s))
                          : "memory");
@@ -261,21 +294,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     }
     __syncwarp();
 
-    // epilogue: TMEM lane = weight row n, column = token m
-    const bool ok = tc_wait(accb, 0u, true);
+    // epilogue: TMEM lane = A row, column = B row
+    // warp-uniform, so the aligned tensor-memory loads below stay converged
+    const bool ok = __all_sync(0xffffffffu, tc_wait(accb, 0u, true));
     if (!ok && lane == 0) atomicOr(err, kErrTcWait);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const int n = n0 + warp * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const bool vec = TOKA && (N % 8) == 0 && ((reinterpret_cast<uintptr_t>(y) & 15) == 0);
 #pragma unroll 1
-    for (int c = 0; c < BT / 32; ++c) {
-        uint32_t r[32];
-        tc_ld32(trow + (uint32_t)(c * 32), r);
-        if (ok && n < N) {
+    for (int h = 0; h < C::kHalves; ++h) {
+        const int ra = a0 + h * kTcMma + warp * 32 + lane;           // this thread's A row
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(h * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tc_ld32(trow + (uint32_t)(c * 32), r);
+            if (!ok) continue;
+            const int rb = b0 + c * 32;                                 // first B row of these columns
+            if (TOKA) {
+                if (ra < M) {
+                    __half *dst = y + (size_t)ra * N + rb;
+                    if (vec && rb + 32 <= N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int m = m0 + c * 32 + j;
-                if (m < M) y[(size_t)m * N + n] = __float2half_rn(__uint_as_float(r[j]));
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 v;
+                            uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __half2 h2 = __floats2half2_rn(__uint_as_float(r[8 * q + 2 * e]),
+                                                               __uint_as_float(r[8 * q + 2 * e + 1]));
+                                pv[e] = *reinterpret_cast<uint32_t *>(&h2);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + 8 * q) = v;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (rb + j < N) dst[j] = __float2half_rn(__uint_as_float(r[j]));
+                    }
+                }
+            } else if (ra < N) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int m = rb + j;
+                    if (m < M) y[(size_t)m * N + ra] = __float2half_rn(__uint_as_float(r[j]));
+                }
             }
         }
     }
@@ -290,7 +352,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     __syncthreads();
     if (warp == 0) {
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BT) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                     : "memory");
     }
 }
 

@@ -446,7 +446,7 @@ bool tma_map_f16(CUtensorMap *map, const void *base, int K, long long rows, int 
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)box_rows};   // box_rows <= 256
     cuuint32_t estr[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -487,37 +487,49 @@ int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, in
     return launch_status();
 }
 
-template <int BT>
-int launch_gemm_tc_bt(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
-                      cudaStream_t st)
+template <int AM, int BN, bool TOKA>
+int launch_gemm_tc_cfg(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
+                       cudaStream_t st)
 {
-    using C = TcCfg<BT>;
-    const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<BT>);
+    using C = TcCfg<AM, BN>;
+    const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<AM, BN, TOKA>);
     int sms = 0;
     if (resident_ctas(fn, kTcThreads, C::kSmem, sms) < 1) return ZT_ERR_DEVICE;
-    CUtensorMap mw, mx;
-    if (!tma_map_f16(&mw, w16, K, N, kTcRows) || !tma_map_f16(&mx, x, K, M, BT)) return ZT_ERR_DEVICE;
-    const dim3 grid((unsigned)((N + kTcRows - 1) / kTcRows), (unsigned)((M + BT - 1) / BT));
+    const uint16_t *a = TOKA ? x : w16, *b = TOKA ? w16 : x;
+    const int ra = TOKA ? M : N, rb = TOKA ? N : M;
+    CUtensorMap ma, mb;
+    if (!tma_map_f16(&ma, a, K, ra, AM) || !tma_map_f16(&mb, b, K, rb, BN)) return ZT_ERR_DEVICE;
+    const dim3 grid((unsigned)((ra + AM - 1) / AM), (unsigned)((rb + BN - 1) / BN));
     clear_stale_error();
-    q4_gemm_tc_kernel<BT><<<grid, kTcThreads, C::kSmem, st>>>(mw, mx, reinterpret_cast<__half *>(y), M, N, K, err);
+    q4_gemm_tc_kernel<AM, BN, TOKA><<<grid, kTcThreads, C::kSmem, st>>>(ma, mb, reinterpret_cast<__half *>(y), M, N,
+                                                                         K, err);
     return launch_status();
 }
 
-// Tokens per CTA: the smallest of 64 / 128 / 256 that covers M, halved while
-// the grid would leave more than a quarter of the SMs idle.
+// Tile choice.  From 128 tokens on, tokens are the A operand: 256 tokens x
+// 256 weight rows per CTA when that still gives every SM a CTA, else 128
+// tokens x BN weight rows, BN = 256 halved while the grid would leave more
+// than a quarter of the SMs idle.  Below 128 tokens, weight rows are the A
+// operand (128 per CTA) and the tokens a 64- or 128-wide B tile.
 int launch_gemm_tc(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
                    cudaStream_t st)
 {
     int sms = 0;
-    if (resident_ctas(reinterpret_cast<const void *>(&q4_gemm_tc_kernel<256>), kTcThreads, TcCfg<256>::kSmem,
-                      sms) < 1)
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_gemm_tc_kernel<128, 256, true>), kTcThreads,
+                      TcCfg<128, 256>::kSmem, sms) < 1)
         return ZT_ERR_DEVICE;
-    const long long nt = (N + kTcRows - 1) / kTcRows;
-    int bt = M <= 64 ? 64 : M <= 128 ? 128 : 256;
-    while (bt > 64 && nt * ((M + bt - 1) / bt) * 4 < 3ll * sms) bt /= 2;
-    if (bt == 256) return launch_gemm_tc_bt<256>(w16, x, y, M, N, K, err, st);
-    if (bt == 128) return launch_gemm_tc_bt<128>(w16, x, y, M, N, K, err, st);
-    return launch_gemm_tc_bt<64>(w16, x, y, M, N, K, err, st);
+    if (M >= 128) {
+        if (((M + 255) / 256) * (long long)((N + 255) / 256) >= sms)
+            return launch_gemm_tc_cfg<256, 256, true>(w16, x, y, M, N, K, err, st);
+        const long long mt = (M + 127) / 128;
+        int bn = 256;
+        while (bn > 64 && mt * ((N + bn - 1) / bn) * 4 < 3ll * sms) bn /= 2;
+        if (bn == 256) return launch_gemm_tc_cfg<128, 256, true>(w16, x, y, M, N, K, err, st);
+        if (bn == 128) return launch_gemm_tc_cfg<128, 128, true>(w16, x, y, M, N, K, err, st);
+        return launch_gemm_tc_cfg<128, 64, true>(w16, x, y, M, N, K, err, st);
+    }
+    if (M > 64) return launch_gemm_tc_cfg<128, 128, false>(w16, x, y, M, N, K, err, st);
+    return launch_gemm_tc_cfg<128, 64, false>(w16, x, y, M, N, K, err, st);
 }
 
 }  // namespace

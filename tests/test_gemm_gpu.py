@@ -70,6 +70,9 @@ SHAPES = [
     (256, 1024, 3072),
     (300, 640, 2048),       # 256-token tiles with a ragged second tile
     (40, 3072, 8192),       # Phi-3-mini down projection shape, 40 tokens
+    (150, 203, 256),        # tokens as the A operand, N % 8 != 0: element stores
+    (200, 360, 128),        # N % 8 == 0 but the last 32 columns ragged: mixed stores
+    (128, 1024, 3072),      # exactly one 128-token A tile
 ]
 
 
@@ -155,3 +158,21 @@ def test_gemm_exact_weights_match_decode_path(zt, oracle):
     assert_f16_matches(y_pre, ref, "prefill", bound)
     assert_f16_matches(y_dec, ref, "decode", bound)
     assert rel_l2(y_pre, y_dec) <= F16_REL_L2
+
+
+@pytest.mark.parametrize("M,N,K", [(1100, 9000, 256), (600, 16000, 96), (2048, 9216, 3072)])
+def test_gemm_256_row_tiles_sampled(zt, oracle, M, N, K):
+    """Shapes whose grid of 256-row x 256-token tiles covers every SM, so the
+    two-accumulator tile runs (ragged N, M and K included); sampled rows on
+    both halves of several tiles, every token."""
+    import torch
+    qw, s, _ = synth.problem(800 + M, N, K, M=1, proj=1)
+    x = _prefill_x(M, M, K)
+    y = host(zt.gemm(dev(qw), dev(s), dev(x)))
+    torch.cuda.synchronize()
+    edges = [0, 1, 127, 128, 129, 255, 256, 257, 383, 384, N - 129, N - 128, N - 2, N - 1]
+    rows = np.unique(np.concatenate([[r for r in edges if 0 <= r < N],
+                                     np.random.default_rng(M).integers(0, N, 40)])).astype(np.int32)
+    ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
+    assert_f16_matches(y[:, rows], ref, f"gemm 256-row tiles M{M} N{N} K{K}",
+                       abs_products_f16w(oracle, qw, s, x, rows=rows))
