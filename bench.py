@@ -677,13 +677,11 @@ def run_prefill(args, local):
     for c in range(copies):
         qw, s, _ = synth.proj_inputs(args.seed, c, p)
         qd, sd = torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)
-        ws = torch.empty((zt_q4.gemm_workspace_bytes(N, K),), dtype=torch.uint8, device=device)
-        w.append((qd, sd, ws, ws[:N * K * 2].view(torch.float16).view(N, K)))
+        w.append((qd, sd, torch.empty((N, K), dtype=torch.float16, device=device)))
     peaks = measured_peaks()
     tc_peak = peaks.get("bf16_tflops")
     hbm_peak = peaks.get("hbm_gbs")
     stream = torch.cuda.Stream(device=device)
-    err = torch.zeros((1,), dtype=torch.int32, device=device)
 
     def timed(fn, steps):
         with torch.cuda.stream(stream):
@@ -702,12 +700,15 @@ def run_prefill(args, local):
         x = torch.randn((M, K), device=device).half()
         y = torch.empty((M, N), dtype=torch.float16, device=device)
         steps = max(min(args.steps, 200), 4 * copies)
-        both = timed(lambda i: zt_q4.gemm(w[i % copies][0], w[i % copies][1], x, y, w[i % copies][2],
+        ws = [torch.empty((zt_q4.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device=device)
+              for _ in range(copies)]
+        gws = torch.empty((zt_q4.gemm_f16w_workspace_bytes(M, N, K),), dtype=torch.uint8, device=device)
+        both = timed(lambda i: zt_q4.gemm(w[i % copies][0], w[i % copies][1], x, y, ws[i % copies],
                                           stream=stream), steps)
-        gemm = timed(lambda i: zt_q4.gemm_f16w(w[i % copies][3], x, y, err, stream=stream), steps)
-        deq = timed(lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][3],
+        gemm = timed(lambda i: zt_q4.gemm_f16w(w[i % copies][2], x, y, gws, stream=stream), steps)
+        deq = timed(lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][2],
                                                 stream=stream), steps)
-        assert int(err.item()) == 0 and all(zt_q4.gemm_errors(c[2], N, K) == 0 for c in w)
+        assert zt_q4.gemm_f16w_errors(gws) == 0 and all(zt_q4.gemm_errors(c, N, K) == 0 for c in ws)
         flops = 2.0 * M * N * K
         deq_bytes = N * K // 2 + N * (K // 32) * 2 + N * K * 2
         g_tf = flops / gemm / 1e6

@@ -264,23 +264,28 @@ ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
  *     and scales [N][K/group].  group: 0 or 32, 64, 128 (K % group == 0).  HBM-bound
  *     streaming kernel; a caller that runs many prefill batches may keep w16 and
  *     call zt_q4_gemm_f16w directly.
- * zt_q4_gemm_f16w: y fp16 [M][N] = x fp16 [M][K] times w16^T.  err is a DEVICE
- *     uint32 the kernel ORs bit 0 into if one of its bounded waits (2 s) expired
- *     (outputs are then incomplete); the caller zeroes it.  w16 and x 16-byte
- *     aligned, y 2 bytes, err 4.
- * zt_q4_gemm: both steps; workspace (DEVICE, 16-byte aligned, at least
- *     zt_q4_gemm_workspace_bytes(N, K) bytes) holds w16 and the error word, which
- *     the dequant launch clears; read it with zt_q4_gemm_errors (synchronous).
- *     Two launches on `stream`.
+ * zt_q4_gemm_f16w: y fp16 [M][N] = x fp16 [M][K] times w16^T.  workspace (DEVICE,
+ *     16-byte aligned, zt_q4_gemm_f16w_workspace_bytes(M, N, K) bytes) holds an error
+ *     word (cleared by the call, on the stream) and, for shapes whose tiles cover
+ *     few SMs, fp32 partial sums of a split along K, added in a fixed order by a
+ *     second launch (results are deterministic).  Bit 0 of the error word is set if
+ *     one of the kernel's bounded waits (2 s) expired (outputs are then incomplete);
+ *     read it with zt_q4_gemm_f16w_errors.  w16 and x 16-byte aligned, y 2 bytes.
+ * zt_q4_gemm: both steps through one workspace of zt_q4_gemm_workspace_bytes(M, N, K)
+ *     bytes (16-byte aligned): w16 first, then the GEMM's workspace; read its error
+ *     word with zt_q4_gemm_errors.  Two or three launches on `stream`.
+ * The tile plan (and so the workspace size) is a function of (M, N, K) alone.
  * Shapes: 1 <= M <= 2^22, N >= 1, K >= 32, K % 32 == 0, N*K <= 2^40.  Inputs and
  * outputs must not overlap.  Status codes as elsewhere; ZT_ERR_DEVICE also when the
- * TMA descriptor encoder is unavailable.
+ * TMA descriptor encoder is unavailable.  The *_errors calls are synchronous.
  */
 ZT_API int zt_q4_dequant_f16(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int group,
                              void *stream);
+ZT_API size_t zt_q4_gemm_f16w_workspace_bytes(int M, int N, int K);
 ZT_API int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K,
-                           unsigned int *err, void *stream);
-ZT_API size_t zt_q4_gemm_workspace_bytes(int N, int K);
+                           void *workspace, size_t ws_bytes, void *stream);
+ZT_API int zt_q4_gemm_f16w_errors(const void *workspace, unsigned int *out);
+ZT_API size_t zt_q4_gemm_workspace_bytes(int M, int N, int K);
 ZT_API int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M, int N,
                       int K, int group, void *workspace, size_t ws_bytes, void *stream);
 ZT_API int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out);

@@ -36,6 +36,12 @@
 
 namespace zt {
 
+__device__ __forceinline__ float4 ldg_stream_f4(const float *p)
+{
+    const uint4 v = ldg_stream(reinterpret_cast<const uint4 *>(p));
+    return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+
 // ------------------------------------------------------------ dequant ----
 // One thread per 16-byte chunk of codes (32 consecutive k of one row).
 // (1024 + q) is the fp16 pattern 0x6400 | q; subtracting 1031 = 0x6407 gives
@@ -200,10 +206,15 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32])
 // ("swap AB", for fewer than 128 tokens) A holds weight rows and B tokens.
 // tma_a / tma_b: fp16 [rows][K], boxes 64 x AM and 64 x BN, 128-byte swizzled,
 // out-of-range rows and k read as zero.
+//
+// Split K (blockIdx.z = split, kb_per k blocks each): with part != null the
+// CTA writes its fp32 partial tile to part[z][M][N] instead of y, and
+// q4_splitk_reduce_kernel sums the splits in order.
 template <int AM, int BN, bool TOKA>
 __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
                                                                    const __grid_constant__ CUtensorMap tma_b,
-                                                                   __half *__restrict__ y, int M, int N, int K,
+                                                                   __half *__restrict__ y, float *__restrict__ part,
+                                                                   int M, int N, int K, int kb_per,
                                                                    unsigned int *err)
 {
     using C = TcCfg<AM, BN>;
@@ -220,7 +231,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int a0 = blockIdx.x * AM, b0 = blockIdx.y * BN;
-    const int kb_n = (K + kTcK - 1) / kTcK;
+    const int kb_lo = blockIdx.z * kb_per;
+    const int kb_n = min((K + kTcK - 1) / kTcK - kb_lo, kb_per);   // k blocks of this split (>= 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -254,8 +266,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full(s)),
                          "r"(C::kStageBytes) : "memory");
             const uint32_t a = ring + s * C::kStageBytes;
-            tc_tma_2d(a, &tma_a, kb * kTcK, a0, full(s));
-            tc_tma_2d(a + C::kABytes, &tma_b, kb * kTcK, b0, full(s));
+            tc_tma_2d(a, &tma_a, (kb_lo + kb) * kTcK, a0, full(s));
+            tc_tma_2d(a + C::kABytes, &tma_b, (kb_lo + kb) * kTcK, b0, full(s));
             issued = kb + 1;
         }
     } else if (threadIdx.x == 32) {
@@ -300,6 +312,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     if (!ok && lane == 0) atomicOr(err, kErrTcWait);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const bool vec = TOKA && (N % 8) == 0 && ((reinterpret_cast<uintptr_t>(y) & 15) == 0);
+    const bool vecp = TOKA && (N % 4) == 0 && ((reinterpret_cast<uintptr_t>(part) & 15) == 0);
+    float *pz = part ? part + (size_t)blockIdx.z * M * N : nullptr;
 #pragma unroll 1
     for (int h = 0; h < C::kHalves; ++h) {
         const int ra = a0 + h * kTcMma + warp * 32 + lane;           // this thread's A row
@@ -310,7 +324,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
             tc_ld32(trow + (uint32_t)(c * 32), r);
             if (!ok) continue;
             const int rb = b0 + c * 32;                                 // first B row of these columns
-            if (TOKA) {
+            if (pz) {
+                // fp32 partials, [M][N] per split
+                if (TOKA) {
+                    if (ra < M) {
+                        float *dst = pz + (size_t)ra * N + rb;
+                        if (vecp && rb + 32 <= N) {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                *reinterpret_cast<float4 *>(dst + 4 * q) =
+                                    make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                                __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (rb + j < N) dst[j] = __uint_as_float(r[j]);
+                        }
+                    }
+                } else if (ra < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (rb + j < M) pz[(size_t)(rb + j) * N + ra] = __uint_as_float(r[j]);
+                }
+            } else if (TOKA) {
                 if (ra < M) {
                     __half *dst = y + (size_t)ra * N + rb;
                     if (vec && rb + 32 <= N) {
@@ -354,6 +390,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
                      : "memory");
+    }
+}
+
+// y[i] = fp16(sum_z part[z][i]), z = 0 .. splits-1 in order (deterministic);
+// four elements per thread when mn % 4 == 0 and y is 8-byte aligned.
+__global__ void __launch_bounds__(256) q4_splitk_reduce_kernel(const float *__restrict__ part,
+                                                               __half *__restrict__ y, long long mn, int splits)
+{
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if ((mn & 3) == 0 && (reinterpret_cast<uintptr_t>(y) & 7) == 0) {
+        for (long long i = t0; i < mn / 4; i += stride) {
+            float4 a = ldg_stream_f4(part + 4 * i);
+            for (int z = 1; z < splits; ++z) {
+                const float4 b = ldg_stream_f4(part + (size_t)z * mn + 4 * i);
+                a.x += b.x;
+                a.y += b.y;
+                a.z += b.z;
+                a.w += b.w;
+            }
+            const __half2 lo = __floats2half2_rn(a.x, a.y), hi = __floats2half2_rn(a.z, a.w);
+            uint2 v;
+            v.x = *reinterpret_cast<const uint32_t *>(&lo);
+            v.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(y + 4 * i) = v;
+        }
+    } else {
+        for (long long i = t0; i < mn; i += stride) {
+            float a = part[i];
+            for (int z = 1; z < splits; ++z) a += part[(size_t)z * mn + i];
+            y[i] = __float2half_rn(a);
+        }
     }
 }
 

@@ -468,7 +468,79 @@ int group_shift(int K, int group)
     return group == 32 ? 0 : group == 64 ? 1 : 2;
 }
 
-size_t gemm_err_offset(int N, int K) { return ((size_t)N * (size_t)K * 2 + 255) & ~(size_t)255; }
+// Workspace of the GEMM on binary16 weights: the error word (256 bytes
+// reserved), then split-K partials fp32 [splits][M][N].  zt_q4_gemm puts the
+// w16 weights in front of it.
+size_t w16_bytes(int N, int K) { return ((size_t)N * (size_t)K * 2 + 255) & ~(size_t)255; }
+
+// Launch plan, a function of the shape only (computed for the 148 SMs of a
+// B200, so the workspace query needs no device).  From 128 tokens on, tokens
+// are the A operand and weight rows the B operand (AM x BN = 256 x 256,
+// 128 x 256, 128 x 128 or 128 x 64); below 128 tokens weight rows are A (128
+// per CTA) and
+// the tokens a 64- or 128-wide B tile.  K may be split into s <= 8 parts of
+// at least 16 k blocks (fp32 partials, summed in order by a second launch).
+// Among these the plan with the least estimated time wins:
+//   waves x (MMA cycles of one CTA / ingest efficiency + epilogue + fixed)
+//   + the partials' round trip when split,
+// where one k block of an AM x BN tile is AM * BN / 64 MMA cycles and the
+// ingest efficiency is min(1, 70 / (bytes per MMA cycle the tile needs)),
+// 70 bytes per cycle being about what one SM takes in from L2 (measured: the
+// 128 x 256 tile needs 96 and keeps the tensor pipe ~60 % busy), and the
+// partials' round trip is priced at 24 bytes per cycle per SM.  (A 256 x 128
+// tile needs as many bytes per cycle as 128 x 256 but measured slower, so it
+// is not offered.)
+constexpr int kPlanSms = 148;
+struct GemmPlan {
+    int am, bn, splits, kb_per;
+    bool toka;
+};
+
+double plan_cost(int am, int bn, int s, long long M, long long N, long long kb_n, bool toka)
+{
+    const long long ra = toka ? M : N, rb = toka ? N : M;
+    const long long ctas = ((ra + am - 1) / am) * ((rb + bn - 1) / bn) * s;
+    const long long waves = (ctas + kPlanSms - 1) / kPlanSms;
+    const long long kb_per = (kb_n + s - 1) / s;
+    const double need = 8192.0 * (am + bn) / ((double)am * bn);          // bytes per MMA cycle
+    const double eff = std::min(1.0, 70.0 / need);
+    const double mma = (double)am * bn / 64.0 * kb_per / eff;
+    const double epi = (double)am * bn * (s > 1 ? 4 : 2) / 48.0;
+    double cost = (double)waves * (mma + epi + 3000.0);
+    if (s > 1) cost += 2.0 * s * (double)M * N * 4 / (kPlanSms * 24.0);
+    return cost;
+}
+
+GemmPlan gemm_plan(int M, int N, int K)
+{
+    const long long kb_n = (K + kTcK - 1) / kTcK;
+    static const int toka_tiles[][2] = {{256, 256}, {128, 256}, {128, 128}, {128, 64}};
+    static const int swap_tiles[][2] = {{128, 128}, {128, 64}};
+    const bool toka = M >= 128;
+    GemmPlan best{128, 64, 1, (int)kb_n, toka};
+    double best_cost = 1e300;
+    const int n_tiles = toka ? 4 : 2;
+    for (int t = 0; t < n_tiles; ++t) {
+        const int am = toka ? toka_tiles[t][0] : swap_tiles[t][0];
+        const int bn = toka ? toka_tiles[t][1] : swap_tiles[t][1];
+        if (!toka && bn == 128 && M <= 64) continue;        // a 64-wide token tile covers M
+        for (int sp = 1; sp <= 8; ++sp) {
+            if (sp > 1 && kb_n / sp < 16) break;
+            const double c = plan_cost(am, bn, sp, M, N, kb_n, toka);
+            if (c < best_cost) {
+                best_cost = c;
+                best = GemmPlan{am, bn, sp, (int)((kb_n + sp - 1) / sp), toka};
+            }
+        }
+    }
+    return best;
+}
+
+size_t f16w_ws_bytes(int M, int N, int K)
+{
+    const GemmPlan p = gemm_plan(M, N, K);
+    return 256 + (p.splits > 1 ? (size_t)p.splits * M * N * 4 : 0);
+}
 
 int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int gsh,
                    unsigned int *err, cudaStream_t st)
@@ -488,8 +560,8 @@ int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, in
 }
 
 template <int AM, int BN, bool TOKA>
-int launch_gemm_tc_cfg(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
-                       cudaStream_t st)
+int launch_gemm_tc_cfg(const GemmPlan &p, const uint16_t *w16, const uint16_t *x, uint16_t *y, float *part, int M,
+                       int N, int K, unsigned int *err, cudaStream_t st)
 {
     using C = TcCfg<AM, BN>;
     const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<AM, BN, TOKA>);
@@ -499,37 +571,44 @@ int launch_gemm_tc_cfg(const uint16_t *w16, const uint16_t *x, uint16_t *y, int 
     const int ra = TOKA ? M : N, rb = TOKA ? N : M;
     CUtensorMap ma, mb;
     if (!tma_map_f16(&ma, a, K, ra, AM) || !tma_map_f16(&mb, b, K, rb, BN)) return ZT_ERR_DEVICE;
-    const dim3 grid((unsigned)((ra + AM - 1) / AM), (unsigned)((rb + BN - 1) / BN));
+    const dim3 grid((unsigned)((ra + AM - 1) / AM), (unsigned)((rb + BN - 1) / BN), (unsigned)p.splits);
     clear_stale_error();
-    q4_gemm_tc_kernel<AM, BN, TOKA><<<grid, kTcThreads, C::kSmem, st>>>(ma, mb, reinterpret_cast<__half *>(y), M, N,
-                                                                         K, err);
+    q4_gemm_tc_kernel<AM, BN, TOKA><<<grid, kTcThreads, C::kSmem, st>>>(
+        ma, mb, reinterpret_cast<__half *>(y), p.splits > 1 ? part : nullptr, M, N, K, p.kb_per, err);
+    int rc = launch_status();
+    if (rc || p.splits == 1) return rc;
+    const long long mn = (long long)M * N;
+    const int grid_r = (int)std::max(1ll, std::min((mn / 4 + 255) / 256, (long long)sms * 8));
+    q4_splitk_reduce_kernel<<<grid_r, 256, 0, st>>>(part, reinterpret_cast<__half *>(y), mn, p.splits);
     return launch_status();
 }
 
-// Tile choice.  From 128 tokens on, tokens are the A operand: 256 tokens x
-// 256 weight rows per CTA when that still gives every SM a CTA, else 128
-// tokens x BN weight rows, BN = 256 halved while the grid would leave more
-// than a quarter of the SMs idle.  Below 128 tokens, weight rows are the A
-// operand (128 per CTA) and the tokens a 64- or 128-wide B tile.
-int launch_gemm_tc(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
+// ws: the GEMM's workspace (error word, then partials), f16w_ws_bytes long.
+int launch_gemm_tc(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, void *ws,
                    cudaStream_t st)
 {
-    int sms = 0;
-    if (resident_ctas(reinterpret_cast<const void *>(&q4_gemm_tc_kernel<128, 256, true>), kTcThreads,
-                      TcCfg<128, 256>::kSmem, sms) < 1)
-        return ZT_ERR_DEVICE;
-    if (M >= 128) {
-        if (((M + 255) / 256) * (long long)((N + 255) / 256) >= sms)
-            return launch_gemm_tc_cfg<256, 256, true>(w16, x, y, M, N, K, err, st);
-        const long long mt = (M + 127) / 128;
-        int bn = 256;
-        while (bn > 64 && mt * ((N + bn - 1) / bn) * 4 < 3ll * sms) bn /= 2;
-        if (bn == 256) return launch_gemm_tc_cfg<128, 256, true>(w16, x, y, M, N, K, err, st);
-        if (bn == 128) return launch_gemm_tc_cfg<128, 128, true>(w16, x, y, M, N, K, err, st);
-        return launch_gemm_tc_cfg<128, 64, true>(w16, x, y, M, N, K, err, st);
+    const GemmPlan p = gemm_plan(M, N, K);
+    unsigned int *err = static_cast<unsigned int *>(ws);
+    float *part = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + 256);
+    if (p.toka) {
+        if (p.am == 256) return launch_gemm_tc_cfg<256, 256, true>(p, w16, x, y, part, M, N, K, err, st);
+        if (p.bn == 256) return launch_gemm_tc_cfg<128, 256, true>(p, w16, x, y, part, M, N, K, err, st);
+        if (p.bn == 128) return launch_gemm_tc_cfg<128, 128, true>(p, w16, x, y, part, M, N, K, err, st);
+        return launch_gemm_tc_cfg<128, 64, true>(p, w16, x, y, part, M, N, K, err, st);
     }
-    if (M > 64) return launch_gemm_tc_cfg<128, 128, false>(w16, x, y, M, N, K, err, st);
-    return launch_gemm_tc_cfg<128, 64, false>(w16, x, y, M, N, K, err, st);
+    if (p.bn == 128) return launch_gemm_tc_cfg<128, 128, false>(p, w16, x, y, part, M, N, K, err, st);
+    return launch_gemm_tc_cfg<128, 64, false>(p, w16, x, y, part, M, N, K, err, st);
+}
+
+int read_error_word(const void *p, unsigned int *out)
+{
+    const cudaError_t e = cudaMemcpy(out, p, sizeof(unsigned int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_DEVICE;
+    }
+    return ZT_OK;
 }
 
 }  // namespace
@@ -796,20 +875,35 @@ int zt_q4_dequant_f16(const uint32_t *qw, const uint16_t *scales, uint16_t *w16,
     return launch_dequant(qw, scales, w16, N, K, gsh, nullptr, static_cast<cudaStream_t>(stream));
 }
 
-int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, unsigned int *err,
-                    void *stream)
+size_t zt_q4_gemm_f16w_workspace_bytes(int M, int N, int K)
 {
-    if (!w16 || !x || !y || !err) return ZT_ERR_INVALID_ARG;
-    int rc = check_gemm_shapes(M, N, K);
-    if (rc) return rc;
-    if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(err, 4)) return ZT_ERR_MISALIGNED;
-    return launch_gemm_tc(w16, x, y, M, N, K, err, static_cast<cudaStream_t>(stream));
+    if (check_gemm_shapes(M, N, K) != ZT_OK) return 0;
+    return f16w_ws_bytes(M, N, K);
 }
 
-size_t zt_q4_gemm_workspace_bytes(int N, int K)
+int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, void *workspace,
+                    size_t ws_bytes, void *stream)
 {
-    if (check_gemm_shapes(1, N, K) != ZT_OK) return 0;
-    return gemm_err_offset(N, K) + 16;
+    if (!w16 || !x || !y || !workspace) return ZT_ERR_INVALID_ARG;
+    int rc = check_gemm_shapes(M, N, K);
+    if (rc) return rc;
+    if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(workspace, 16)) return ZT_ERR_MISALIGNED;
+    if (ws_bytes < f16w_ws_bytes(M, N, K)) return ZT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    clear_stale_error();
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    return launch_gemm_tc(w16, x, y, M, N, K, workspace, st);
+}
+
+size_t zt_q4_gemm_workspace_bytes(int M, int N, int K)
+{
+    if (check_gemm_shapes(M, N, K) != ZT_OK) return 0;
+    return w16_bytes(N, K) + f16w_ws_bytes(M, N, K);
 }
 
 int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M, int N, int K,
@@ -822,27 +916,25 @@ int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, ui
     if (gsh < 0) return ZT_ERR_INVALID_ARG;
     if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return ZT_ERR_MISALIGNED;
-    if (ws_bytes < gemm_err_offset(N, K) + 16) return ZT_ERR_WORKSPACE;
+    if (ws_bytes < w16_bytes(N, K) + f16w_ws_bytes(M, N, K)) return ZT_ERR_WORKSPACE;
     uint16_t *w16 = static_cast<uint16_t *>(workspace);
-    unsigned int *err = reinterpret_cast<unsigned int *>(static_cast<unsigned char *>(workspace) +
-                                                         gemm_err_offset(N, K));
+    void *gws = static_cast<unsigned char *>(workspace) + w16_bytes(N, K);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = launch_dequant(qw, scales, w16, N, K, gsh, err, st);
+    rc = launch_dequant(qw, scales, w16, N, K, gsh, static_cast<unsigned int *>(gws), st);
     if (rc) return rc;
-    return launch_gemm_tc(w16, x, y, M, N, K, err, st);
+    return launch_gemm_tc(w16, x, y, M, N, K, gws, st);
+}
+
+int zt_q4_gemm_f16w_errors(const void *workspace, unsigned int *out)
+{
+    if (!workspace || !out) return ZT_ERR_INVALID_ARG;
+    return read_error_word(workspace, out);
 }
 
 int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out)
 {
     if (!workspace || !out || check_gemm_shapes(1, N, K) != ZT_OK) return ZT_ERR_INVALID_ARG;
-    const cudaError_t e = cudaMemcpy(out, static_cast<const unsigned char *>(workspace) + gemm_err_offset(N, K),
-                                     sizeof(unsigned int), cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) {
-        g_last_cuda_error = e;
-        (void)cudaGetLastError();
-        return ZT_ERR_DEVICE;
-    }
-    return ZT_OK;
+    return read_error_word(static_cast<const unsigned char *>(workspace) + w16_bytes(N, K), out);
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)

@@ -80,12 +80,16 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_pass_errors.argtypes = [_P, _I, ctypes.POINTER(ctypes.c_uint)]
     lib.zt_q4_pass_errors.restype = ctypes.c_int
     lib.zt_q4_dequant_f16.argtypes = [_P, _P, _P, _I, _I, _I, _P]
-    lib.zt_q4_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
-    lib.zt_q4_gemm_workspace_bytes.argtypes = [_I, _I]
+    lib.zt_q4_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
+    lib.zt_q4_gemm_f16w_workspace_bytes.argtypes = [_I, _I, _I]
+    lib.zt_q4_gemm_f16w_workspace_bytes.restype = ctypes.c_size_t
+    lib.zt_q4_gemm_f16w_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_uint)]
+    lib.zt_q4_gemm_workspace_bytes.argtypes = [_I, _I, _I]
     lib.zt_q4_gemm_workspace_bytes.restype = ctypes.c_size_t
     lib.zt_q4_gemm.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_gemm_errors.argtypes = [_P, _I, _I, ctypes.POINTER(ctypes.c_uint)]
-    for f in (lib.zt_q4_dequant_f16, lib.zt_q4_gemm_f16w, lib.zt_q4_gemm, lib.zt_q4_gemm_errors):
+    for f in (lib.zt_q4_dequant_f16, lib.zt_q4_gemm_f16w, lib.zt_q4_gemm, lib.zt_q4_gemm_errors,
+              lib.zt_q4_gemm_f16w_errors):
         f.restype = ctypes.c_int
     lib.zt_q4_pack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_unpack_host.argtypes = [_P, _I, _I, _P]
@@ -210,9 +214,14 @@ def dequant_f16(qw, scales, w16=None, stream=None):
     return w16
 
 
-def gemm_f16w(w16, x, y=None, err=None, stream=None):
-    """y fp16 [M][N] = x [M][K] @ w16^T on the tensor cores; err: int32 CUDA
-    tensor of one element that the kernel ORs 1 into if a bounded wait expired."""
+def gemm_f16w_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.zt_q4_gemm_f16w_workspace_bytes(M, N, K))
+
+
+def gemm_f16w(w16, x, y=None, workspace=None, stream=None):
+    """y fp16 [M][N] = x [M][K] @ w16^T on the tensor cores; workspace: uint8
+    CUDA tensor of gemm_f16w_workspace_bytes(M, N, K) bytes (error word and
+    split-K partials)."""
     torch = _torch()
     for t, name in ((w16, "w16"), (x, "x")):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float16 or t.dim() != 2:
@@ -222,20 +231,27 @@ def gemm_f16w(w16, x, y=None, err=None, stream=None):
         raise ValueError("x and w16 disagree on K")
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=x.device)
-    if err is None:
-        err = torch.zeros((1,), dtype=torch.int32, device=x.device)
-    _check(lib.zt_q4_gemm_f16w(w16.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, err.data_ptr(),
-                               _stream_handle(stream)), "zt_q4_gemm_f16w")
+    if workspace is None:
+        workspace = torch.empty((gemm_f16w_workspace_bytes(M, N, K),), dtype=torch.uint8, device=x.device)
+    _check(lib.zt_q4_gemm_f16w(w16.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, workspace.data_ptr(),
+                               workspace.numel(), _stream_handle(stream)), "zt_q4_gemm_f16w")
     return y
 
 
-def gemm_workspace_bytes(N: int, K: int) -> int:
-    return int(lib.zt_q4_gemm_workspace_bytes(N, K))
+def gemm_f16w_errors(workspace) -> int:
+    out = ctypes.c_uint(0)
+    _check(lib.zt_q4_gemm_f16w_errors(workspace.data_ptr(), ctypes.byref(out)), "zt_q4_gemm_f16w_errors")
+    return int(out.value)
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.zt_q4_gemm_workspace_bytes(M, N, K))
 
 
 def gemm(qw, scales, x, y=None, workspace=None, stream=None):
-    """Batched prefill: y fp16 [M][N] = x @ fp16(dequant(qw, scales))^T, two
-    launches (dequant into the workspace, then the tensor-core GEMM)."""
+    """Batched prefill: y fp16 [M][N] = x @ fp16(dequant(qw, scales))^T: the
+    dequant into the workspace, then the tensor-core GEMM (and, for shapes
+    split along K, the ordered sum of the partials)."""
     torch = _torch()
     N, K = qw.shape[0], qw.shape[1] * 8
     g = _group_of(K, scales)
@@ -243,7 +259,7 @@ def gemm(qw, scales, x, y=None, workspace=None, stream=None):
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=x.device)
     if workspace is None:
-        workspace = torch.empty((gemm_workspace_bytes(N, K),), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty((gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device=x.device)
     _check(lib.zt_q4_gemm(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, g,
                           workspace.data_ptr(), workspace.numel(), _stream_handle(stream)), "zt_q4_gemm")
     return y

@@ -206,22 +206,33 @@ def test_pass_group_size_rejected(zt):
 # ------------------------------------------------- batched prefill (M > 16) --
 def test_prefill_symbols_declared():
     syms = declared_symbols(HEADER)
-    for want in ("zt_q4_dequant_f16", "zt_q4_gemm_f16w", "zt_q4_gemm", "zt_q4_gemm_workspace_bytes",
-                 "zt_q4_gemm_errors"):
+    for want in ("zt_q4_dequant_f16", "zt_q4_gemm_f16w", "zt_q4_gemm_f16w_workspace_bytes", "zt_q4_gemm_f16w_errors",
+                 "zt_q4_gemm", "zt_q4_gemm_workspace_bytes", "zt_q4_gemm_errors"):
         assert want in syms
 
 
 def test_gemm_workspace_bytes(zt):
-    f = zt.lib.zt_q4_gemm_workspace_bytes
-    assert f(9216, 3072) == ((9216 * 3072 * 2 + 255) // 256) * 256 + 16
-    assert f(3, 32) == 256 + 16
-    assert f(0, 3072) == 0 and f(8, 48) == 0 and f(8, 0) == 0
+    """The plan (and so the workspace) is a function of the shape alone."""
+    f, g = zt.lib.zt_q4_gemm_workspace_bytes, zt.lib.zt_q4_gemm_f16w_workspace_bytes
+    w16 = ((9216 * 3072 * 2 + 255) // 256) * 256
+    assert g(512, 9216, 3072) == 256                      # one wave of 256 x 128 tiles: no split
+    assert f(512, 9216, 3072) == w16 + 256
+    assert g(4096, 16384, 3072) == 256                    # 256 x 256 tiles, many waves
+    assert g(512, 3072, 8192) == 256 + 3 * 512 * 3072 * 4  # 36 tiles: 3 splits of fp32 partials
+    assert g(128, 9216, 8192) == 256 + 4 * 128 * 9216 * 4
+    assert g(40, 3072, 8192) == 256 + 6 * 40 * 3072 * 4    # weight rows as A: 24 tiles, 6 splits
+    assert g(512, 3072, 512) == 256                       # K too short to split
+    assert f(3, 3, 32) == 256 + 256
+    assert f(0, 9216, 3072) == 0 and f(8, 8, 48) == 0 and f(8, 0, 32) == 0 and g(1, 8, 0) == 0
+    for M, N, K in ((17, 128, 64), (300, 640, 2048), (2048, 3072, 8192)):
+        assert f(M, N, K) == ((N * K * 2 + 255) // 256) * 256 + g(M, N, K)
+        assert (g(M, N, K) - 256) % (M * N * 4) == 0 and (g(M, N, K) - 256) // (M * N * 4) <= 8
 
 
 def test_gemm_arguments_rejected(zt):
     """Every check runs before a launch: these calls touch no device memory."""
     g = zt.lib.zt_q4_gemm
-    ws = zt.gemm_workspace_bytes(256, 64)
+    ws = zt.gemm_workspace_bytes(40, 256, 64)
     ok = [FAKE, FAKE, FAKE, FAKE, 40, 256, 64, 32, FAKE, ws, None]
 
     def call(**kw):
@@ -255,9 +266,12 @@ def test_dequant_and_gemm_f16w_arguments_rejected(zt):
     assert d(FAKE, FAKE, FAKE + 8, 8, 64, 32, None) == zt.ZT_ERR_MISALIGNED
     assert d(FAKE + 4, FAKE, FAKE, 8, 64, 32, None) == zt.ZT_ERR_MISALIGNED
     f = zt.lib.zt_q4_gemm_f16w
-    assert f(FAKE, FAKE, FAKE, 17, 64, 64, None, None) == zt.ZT_ERR_INVALID_ARG      # no error word
-    assert f(FAKE, FAKE, FAKE, 0, 64, 64, FAKE, None) == zt.ZT_ERR_INVALID_ARG
-    assert f(FAKE + 8, FAKE, FAKE, 17, 64, 64, FAKE, None) == zt.ZT_ERR_MISALIGNED
-    assert f(FAKE, FAKE, FAKE, 17, 64, 64, FAKE + 2, None) == zt.ZT_ERR_MISALIGNED
+    ws = zt.gemm_f16w_workspace_bytes(17, 64, 64)
+    assert f(FAKE, FAKE, FAKE, 17, 64, 64, None, ws, None) == zt.ZT_ERR_INVALID_ARG     # no workspace
+    assert f(FAKE, FAKE, FAKE, 0, 64, 64, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert f(FAKE + 8, FAKE, FAKE, 17, 64, 64, FAKE, ws, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, 17, 64, 64, FAKE + 8, ws, None) == zt.ZT_ERR_MISALIGNED
+    assert f(FAKE, FAKE, FAKE, 17, 64, 64, FAKE, ws - 1, None) == zt.ZT_ERR_WORKSPACE
     out = ctypes.c_uint(0)
     assert zt.lib.zt_q4_gemm_errors(None, 8, 64, ctypes.byref(out)) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_gemm_f16w_errors(None, ctypes.byref(out)) == zt.ZT_ERR_INVALID_ARG

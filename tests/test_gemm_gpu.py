@@ -81,7 +81,7 @@ def test_gemm_matches_oracle(zt, oracle, M, N, K):
     import torch
     qw, s, _ = synth.problem(600 + M, N, K, M=1, proj=0)
     x = _prefill_x(M + N, M, K)
-    ws = torch.empty((zt.gemm_workspace_bytes(N, K),), dtype=torch.uint8, device="cuda")
+    ws = torch.empty((zt.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
     y = zt.gemm(dev(qw), dev(s), dev(x), workspace=ws)
     torch.cuda.synchronize()
     assert zt.gemm_errors(ws, N, K) == 0
@@ -127,12 +127,12 @@ def test_gemm_f16w_reuses_dequantized_weights(zt):
     x = dev(_prefill_x(9, M, K))
     qd, sd = dev(qw), dev(s)
     w16 = zt.dequant_f16(qd, sd)
-    err = torch.zeros((1,), dtype=torch.int32, device="cuda")
-    a = zt.gemm_f16w(w16, x, err=err)
+    ws = torch.empty((zt.gemm_f16w_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    a = zt.gemm_f16w(w16, x, workspace=ws)
     b = zt.gemm(qd, sd, x)
     c = zt.gemm(qd, sd, x)
     torch.cuda.synchronize()
-    assert int(err.item()) == 0
+    assert zt.gemm_f16w_errors(ws) == 0
     assert np.array_equal(host(a).view(np.uint16), host(b).view(np.uint16))
     assert np.array_equal(host(b).view(np.uint16), host(c).view(np.uint16))
 
@@ -176,3 +176,46 @@ def test_gemm_256_row_tiles_sampled(zt, oracle, M, N, K):
     ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
     assert_f16_matches(y[:, rows], ref, f"gemm 256-row tiles M{M} N{N} K{K}",
                        abs_products_f16w(oracle, qw, s, x, rows=rows))
+
+
+@pytest.mark.parametrize("M,N,K", [(512, 3072, 8192), (128, 9216, 8192), (40, 3072, 8192), (200, 1000, 16448)])
+def test_gemm_split_k(zt, oracle, M, N, K):
+    """Shapes whose tiles cover few SMs run split along K (fp32 partials summed
+    in order by a second launch): the Phi-3-mini down projection at 512 and 40
+    tokens (weight rows as the A operand at 40), 128 tokens over K = 8192, and
+    8 splits with a short last one (K = 16448 = 257 blocks of 64); sampled
+    rows, every token; deterministic."""
+    import torch
+    qw, s, _ = synth.problem(900 + M + N, N, K, M=1, proj=3)
+    x = _prefill_x(N, M, K)
+    ws = torch.empty((zt.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    assert ws.numel() > zt.gemm_workspace_bytes(M, N, K) - 1
+    qd, sd, xd = dev(qw), dev(s), dev(x)
+    y = host(zt.gemm(qd, sd, xd, workspace=ws))
+    y2 = host(zt.gemm(qd, sd, xd, workspace=ws))
+    torch.cuda.synchronize()
+    assert zt.gemm_errors(ws, N, K) == 0
+    assert np.array_equal(y.view(np.uint16), y2.view(np.uint16))
+    rows = np.unique(np.concatenate([[0, 1, 255, 256, N - 1], np.random.default_rng(M).integers(0, N, 50)]))
+    rows = rows.astype(np.int32)
+    ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
+    assert_f16_matches(y[:, rows], ref, f"split-K gemm M{M} N{N} K{K}", abs_products_f16w(oracle, qw, s, x, rows=rows))
+
+
+@pytest.mark.parametrize("M,N,K", [(70, 12288, 256), (128, 12288, 256), (384, 12288, 256), (256, 8192, 4096),
+                                   (384, 8192, 4096), (160, 12288, 4096)])
+def test_gemm_tile_plans(zt, oracle, M, N, K):
+    """Shapes for the remaining tile plans: weight rows as A with a 128-wide
+    token tile; 128 x 128 and 128 x 256 token tiles; 256 x 256 split in three
+    with 160 tokens in a 256-token tile; sampled rows, every token."""
+    import torch
+    qw, s, _ = synth.problem(1000 + M, N, K, M=1, proj=2)
+    x = _prefill_x(M * 3, M, K)
+    ws = torch.empty((zt.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    y = host(zt.gemm(dev(qw), dev(s), dev(x), workspace=ws))
+    torch.cuda.synchronize()
+    assert zt.gemm_errors(ws, N, K) == 0
+    rows = np.unique(np.concatenate([[0, 63, 64, 127, 128, 255, 256, N - 1],
+                                     np.random.default_rng(N).integers(0, N, 40)])).astype(np.int32)
+    ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
+    assert_f16_matches(y[:, rows], ref, f"gemm plan M{M} N{N} K{K}", abs_products_f16w(oracle, qw, s, x, rows=rows))
