@@ -43,7 +43,6 @@ __device__ __forceinline__ float4 ldg_stream_f4(const float *p)
 }
 
 // ------------------------------------------------------------ dequant ----
-// One thread per 16-byte chunk of codes (32 consecutive k of one row).
 // (1024 + q) is the fp16 pattern 0x6400 | q; subtracting 1031 = 0x6407 gives
 // q - 7 exactly, and __hmul2 rounds (q - 7) * s once, to nearest even.
 __device__ __forceinline__ uint32_t dq_pair(uint32_t codes2, __half2 s2)
@@ -68,40 +67,49 @@ __device__ __forceinline__ uint4 dq_word(uint32_t w, __half2 s2)
     return o;
 }
 
-// qw as uint4 [N][K/32], scales [N][K/group], w16 as uint4 [N][K/8].
-// gsh = log2(group / 32).  err (may be null) is cleared by thread 0 so the
-// GEMM that follows on the stream starts with a clean error word.
-__global__ void __launch_bounds__(256) q4_dequant_f16_kernel(const uint4 *__restrict__ qw,
-                                                             const __half *__restrict__ scales,
-                                                             uint4 *__restrict__ w16, long long chunks, int cpr,
-                                                             int gsh, unsigned int *err)
+__device__ __forceinline__ uint32_t ldg_stream_u32(const uint32_t *p)
 {
-    constexpr int U = 4;   // chunks per thread per step: their loads are in flight together
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// One warp per weight row (rows strided over the grid's warps); lane l takes
+// the code words l, l + 32, ...: each load instruction reads 128 contiguous
+// bytes of codes and each store writes 512 contiguous bytes of w16.
+// qw [N][kw] words (kw = K/8), scales [N][K/group], w16 as uint4 [N][kw] (8
+// halves per word).  gsh = log2(group / 32).  err (may be null) is cleared by
+// thread 0 so the GEMM that follows on the stream starts with a clean error
+// word.
+__global__ void __launch_bounds__(256) q4_dequant_f16_kernel(const uint32_t *__restrict__ qw,
+                                                             const __half *__restrict__ scales,
+                                                             uint4 *__restrict__ w16, int N, int kw, int gsh,
+                                                             unsigned int *err)
+{
+    constexpr int U = 4;   // words per lane per step: their loads are in flight together
     if (err && blockIdx.x == 0 && threadIdx.x == 0) *err = 0u;
-    const int spr = cpr >> gsh;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long c0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; c0 < chunks; c0 += U * stride) {
-        uint4 q[U];
-        __half s[U];
+    const int lane = threadIdx.x & 31;
+    const int spr = (kw >> 2) >> gsh;                       // scales per row, K / group
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long n = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += warps) {
+        const uint32_t *src = qw + n * kw;
+        const __half *srow = scales + n * spr;
+        uint4 *dst = w16 + n * kw;
+        for (int w0 = lane; w0 < kw; w0 += 32 * U) {
+            uint32_t q[U];
+            __half sc[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const long long c = c0 + u * stride;
-            if (c < chunks) {
-                const long long n = c / cpr;
-                q[u] = ldg_stream(qw + c);
-                s[u] = scales[n * spr + ((int)(c - n * cpr) >> gsh)];
+            for (int u = 0; u < U; ++u) {
+                const int w = w0 + 32 * u;
+                if (w < kw) {
+                    q[u] = ldg_stream_u32(src + w);
+                    sc[u] = srow[(w >> 2) >> gsh];          // word w holds k = 8w .. 8w + 7
+                }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const long long c = c0 + u * stride;
-            if (c < chunks) {
-                const __half2 s2 = __half2half2(s[u]);
-                uint4 *dst = w16 + 4 * c;
-                dst[0] = dq_word(q[u].x, s2);
-                dst[1] = dq_word(q[u].y, s2);
-                dst[2] = dq_word(q[u].z, s2);
-                dst[3] = dq_word(q[u].w, s2);
+            for (int u = 0; u < U; ++u) {
+                const int w = w0 + 32 * u;
+                if (w < kw) dst[w] = dq_word(q[u], __half2half2(sc[u]));
             }
         }
     }

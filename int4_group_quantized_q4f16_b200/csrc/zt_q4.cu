@@ -549,13 +549,11 @@ int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, in
     int sms = 0;
     const int occ = resident_ctas(fn, 256, 0, sms);
     if (occ < 1) return ZT_ERR_DEVICE;
-    const long long chunks = (long long)N * (K / 32);
-    const long long want = (chunks + 255) / 256;
-    const int grid = (int)std::max(1ll, std::min(want, (long long)sms * occ * 4));
+    const long long want = ((long long)N + 7) / 8;          // 8 warps per block, one row per warp
+    const int grid = (int)std::max(1ll, std::min(want, (long long)sms * occ));
     clear_stale_error();
-    q4_dequant_f16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(qw),
-                                                  reinterpret_cast<const __half *>(scales),
-                                                  reinterpret_cast<uint4 *>(w16), chunks, K / 32, gsh, err);
+    q4_dequant_f16_kernel<<<grid, 256, 0, st>>>(qw, reinterpret_cast<const __half *>(scales),
+                                                  reinterpret_cast<uint4 *>(w16), N, K / 8, gsh, err);
     return launch_status();
 }
 
