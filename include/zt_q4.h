@@ -248,6 +248,17 @@ ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, si
 ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
 
 /*
+ * TEST HOOK for the error path (tests only): zt_q4_pass with CTA 0 not counting
+ * phase 0 done, so every CTA's bounded wait before phase 1 runs out (about 2 s),
+ * sets the error bit, drains its copies and returns; phase 0's outputs are
+ * complete, later phases' are not.  The list must contain a projection with
+ * `wait` set (else ZT_ERR_INVALID_ARG).  Nothing faults or hangs: the wait is
+ * the kernel's own bounded one, and the context stays usable.
+ */
+ZT_API int zt_q4_pass_test_withhold(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes,
+                                    void *stream);
+
+/*
  * BATCHED PREFILL (M > 16 tokens; any M >= 1 is accepted)
  *
  * Zero-TVM write-up, limitations section: the project ships shaders for

@@ -80,6 +80,7 @@ struct PassArgs {
     int g_max;                  // largest G of the list (sizes the activation area)
     unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
+    int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
     PassProj p[PMAX];
 };
 
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             // publish this CTA's outputs of the phase, then count it done
             __threadfence();
             __syncthreads();
-            if (tid == 0) atomicAdd(&a.counters[ph], 1u);
+            if (tid == 0 && !(ph == a.withhold && blockIdx.x == 0)) atomicAdd(&a.counters[ph], 1u);
         }
     }
     cp_async_wait<0>();

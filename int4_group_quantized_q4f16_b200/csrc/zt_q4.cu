@@ -319,6 +319,7 @@ int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out
     a.M = q.M;
     a.counters = nullptr;
     a.error = nullptr;
+    a.withhold = -1;
     PassProj &p = a.p[0];
     p.qw = q.qw;
     p.scales = q.scales;
@@ -725,7 +726,8 @@ size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M)
     return pass_ws_layout(projs, n, M, nullptr, nullptr);
 }
 
-int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream)
+static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream,
+                     int withhold)
 {
     if (!projs || !workspace || n < 1 || n > ZT_Q4_PASS_MAX || M < 1 || M > 16) return ZT_ERR_INVALID_ARG;
     bool cooperative = false;
@@ -774,6 +776,7 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
     a.M = M;
     a.counters = cooperative ? reinterpret_cast<unsigned int *>(ws) : nullptr;
     a.error = reinterpret_cast<unsigned int *>(ws + err_off);
+    a.withhold = cooperative ? withhold : -1;
     size_t lm = lm_off;
     for (int i = 0; i < n; ++i) {
         const zt_q4_proj &q = projs[i];
@@ -846,6 +849,19 @@ int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws
         }
     }
     return ZT_OK;
+}
+
+int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream)
+{
+    return pass_impl(projs, n, M, workspace, ws_bytes, stream, -1);
+}
+
+int zt_q4_pass_test_withhold(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream)
+{
+    bool waits = false;
+    for (int i = 1; projs && i < n && i <= ZT_Q4_PASS_MAX; ++i) waits = waits || projs[i].wait;
+    if (!waits) return ZT_ERR_INVALID_ARG;
+    return pass_impl(projs, n, M, workspace, ws_bytes, stream, 0);
 }
 
 int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out)

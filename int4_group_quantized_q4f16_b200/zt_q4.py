@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_pass.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass.restype = ctypes.c_int
     lib.zt_q4_pass_errors.argtypes = [_P, _I, ctypes.POINTER(ctypes.c_uint)]
+    lib.zt_q4_pass_test_withhold.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
+    lib.zt_q4_pass_test_withhold.restype = ctypes.c_int
     lib.zt_q4_pass_errors.restype = ctypes.c_int
     lib.zt_q4_dequant_f16.argtypes = [_P, _P, _P, _I, _I, _I, _P]
     lib.zt_q4_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
@@ -376,6 +378,12 @@ class Pass:
     def run(self, stream=None):
         _check(lib.zt_q4_pass(self.arr, self.n, self.M, self.workspace.data_ptr(), self.workspace.numel(),
                               _stream_handle(stream)), "zt_q4_pass")
+
+    def run_withholding_phase0(self, stream=None):
+        """Error-path test: the pass with CTA 0's phase-0 arrival withheld (see
+        zt_q4_pass_test_withhold); the next phase's bounded wait runs out."""
+        _check(lib.zt_q4_pass_test_withhold(self.arr, self.n, self.M, self.workspace.data_ptr(),
+                                            self.workspace.numel(), _stream_handle(stream)), "zt_q4_pass_test_withhold")
 
     def errors(self) -> int:
         v = ctypes.c_uint(0)

@@ -275,3 +275,12 @@ def test_dequant_and_gemm_f16w_arguments_rejected(zt):
     out = ctypes.c_uint(0)
     assert zt.lib.zt_q4_gemm_errors(None, 8, 64, ctypes.byref(out)) == zt.ZT_ERR_INVALID_ARG
     assert zt.lib.zt_q4_gemm_f16w_errors(None, ctypes.byref(out)) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_withhold_hook_needs_a_wait(zt):
+    """The error-path test hook refuses a list without waits (nothing to expire)."""
+    P = zt.ZtProj
+    arr = (P * 2)(P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0),
+                  P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0))
+    assert zt.lib.zt_q4_pass_test_withhold(arr, 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_pass_test_withhold(None, 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG

@@ -189,3 +189,31 @@ def test_pass_fewer_rows_than_ctas(zt, oracle, N):
     assert p.errors() == 0
     for d in projs:
         _check_against_oracle(oracle, d)
+
+
+def test_pass_bounded_wait_expires_and_reports(zt, oracle):
+    """Failure detection without a GPU fault: with CTA 0's phase-0 arrival
+    withheld (the test hook), every CTA's bounded wait before phase 1 runs out
+    after about 2 s; the kernel sets the error bit, drains its copies and
+    returns.  Phase 0's output is still right, and the same pass run normally
+    afterwards is clean and correct: the context stayed usable."""
+    import time
+    import torch
+    M = 1
+    a = _proj("gemv", 1024, 2048, M, 70, 0)
+    b = _proj("gemv", 512, 1024, M, 71, 1, scale_shift=2)
+    b["x"] = a["out"]
+    b["wait"] = 1
+    p = zt.Pass([a, b])
+    t0 = time.time()
+    p.run_withholding_phase0()
+    torch.cuda.synchronize()
+    took = time.time() - t0
+    assert p.errors() != 0, "the withheld arrival must surface as an expired wait"
+    assert took >= 1.5, f"the wait gave up after {took:.2f} s, before its limit"
+    _check_against_oracle(oracle, a)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    _check_against_oracle(oracle, a)
+    _check_against_oracle(oracle, b, x_host=host(a["out"]).astype(np.float16))
