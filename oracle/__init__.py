@@ -109,9 +109,10 @@ class Oracle:
         lib.zto_gemv_rope.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, ctypes.c_double, _P, _I]
         lib.zto_dequant_f16.argtypes = [_P, _P, _I, _I, _I, _P]
         lib.zto_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I]
+        lib.zto_gate_up_silu_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I]
         for f in (lib.zto_unpack, lib.zto_pack, lib.zto_gemv,
                   lib.zto_gate_up_silu, lib.zto_lmhead_argmax, lib.zto_add_rmsnorm, lib.zto_gemv_rope,
-                  lib.zto_dequant_f16, lib.zto_gemm_f16w):
+                  lib.zto_dequant_f16, lib.zto_gemm_f16w, lib.zto_gate_up_silu_f16w):
             f.restype = ctypes.c_int
         self._lib = lib
 
@@ -193,6 +194,22 @@ class Oracle:
         if rc:
             raise ValueError("zto_gemm_f16w rejected its arguments")
         return y
+
+    def gate_up_silu_f16w(self, qw, scales, x, rows=None, threads: int = 1) -> np.ndarray:
+        """out[m][i] = SiLU(g) * u with g, u the products of the binary16 gate
+        and up rows (rows [0,N) gate, [N,2N) up) with x[m], in double."""
+        qw = np.ascontiguousarray(qw, dtype=np.uint32)
+        s = _u16(scales)
+        x = _u16(np.atleast_2d(x))
+        N2, K = qw.shape[0], qw.shape[1] * 8
+        N, M = N2 // 2, x.shape[0]
+        r, nr = self._rows(rows)
+        out = np.empty((M, nr if r is not None else N), dtype=np.float64)
+        rc = self._lib.zto_gate_up_silu_f16w(_ptr(qw), _ptr(s), _ptr(x), M, N, K, _group(K, s),
+                                             _ptr(r) if r is not None else None, nr, _ptr(out), threads)
+        if rc:
+            raise ValueError("zto_gate_up_silu_f16w rejected its arguments")
+        return out
 
     def gate_up_silu(self, qw, scales, x, rows=None, threads: int = 1) -> np.ndarray:
         """out[m][i] = SiLU(gate_n . x_m) * (up_n . x_m), rows [0,N) gate, [N,2N) up."""

@@ -361,3 +361,44 @@ int zto_gemm_f16w(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
     }
     return bad ? -1 : 0;
 }
+
+/* Fused gate/up + SiLU on the binary16 weights: qw and scales hold 2N rows
+ * (gate rows 0..N-1, up rows N..2N-1); with g = sum_k w16[n][k] x[m][k] and
+ * u = sum_k w16[N + n][k] x[m][k] (double, plain k order, w16 as
+ * zto_dequant_f16 forms it), out[m][i] = SiLU(g) * u for n = rows[i] (or i). */
+int zto_gate_up_silu_f16w(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
+                          int M, int N, int K, int group, const int32_t *rows, int n_rows,
+                          double *out, int threads)
+{
+    if (!qw || !scales || !x || !out || !zto_shape_ok(M, N, K, group)) return -1;
+    if (!rows) n_rows = N;
+    for (int i = 0; rows && i < n_rows; ++i)
+        if (rows[i] < 0 || rows[i] >= N) return -1;
+    if (threads < 1) threads = 1;
+    int bad = 0;
+#pragma omp parallel for schedule(static) num_threads(threads) reduction(| : bad)
+    for (int i = 0; i < n_rows; ++i) {
+        const int64_t n = rows ? rows[i] : i;
+        double *wg = (double *)malloc(sizeof(double) * 2 * (size_t)K);
+        if (!wg) {
+            bad = 1;
+            continue;
+        }
+        double *wu = wg + K;
+        for (int64_t k = 0; k < K; ++k) {
+            wg[k] = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));
+            wu[k] = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, N + n, k)));
+        }
+        for (int64_t m = 0; m < M; ++m) {
+            double g = 0.0, u = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double xv = zto_half_to_double(x[m * K + k]);
+                g += wg[k] * xv;
+                u += wu[k] * xv;
+            }
+            out[m * n_rows + i] = zto_silu(g) * u;
+        }
+        free(wg);
+    }
+    return bad ? -1 : 0;
+}

@@ -606,4 +606,32 @@ def pin_gemm_f16w_rows_and_tokens(o):
         assert np.array_equal(o.gemm_f16w(qw, s, x[m:m + 1])[0], full[m])
 
 
+def pin_gate_up_f16w_golden(o):
+    with open(GOLDEN_F16) as fh:
+        cases = [raw.split("#", 1)[0].split() for raw in fh]
+    cases = [c for c in cases if c and c[0] == "f"]
+    assert len(cases) == 2
+    for _, K, gc, gs, uc, us, xb, out in cases:
+        K = int(K)
+        qw = np.concatenate([_row_of_codes(int(gc), K), _row_of_codes(int(uc), K)])
+        s = np.array([[int(gs, 16)] * (K // 32), [int(us, 16)] * (K // 32)], dtype=np.uint16).view(np.float16)
+        x = np.full((1, K), int(xb, 16), dtype=np.uint16).view(np.float16)
+        assert o.gate_up_silu_f16w(qw, s, x)[0, 0] == float(out)
+
+
+def pin_gate_up_f16w_exact_when_scales_are_short(o):
+    """7-bit scales make every w16 exact: the fp16-weight fused FFN equals the
+    exact one (whose gate/up order and SiLU are pinned above) bit for bit,
+    for all rows and for a row subset."""
+    rng = np.random.default_rng(45)
+    N, K, M = 12, 128, 3
+    qw = rng.integers(0, 2 ** 32, size=(2 * N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s = (rng.integers(64, 128, size=(2 * N, K // 32)).astype(np.float64) * 2.0 ** -10).astype(np.float16)
+    x = rng.standard_normal((M, K)).astype(np.float16)
+    assert np.array_equal(o.gate_up_silu_f16w(qw, s, x), o.gate_up_silu(qw, s, x))
+    rows = np.array([11, 0, 5], dtype=np.int32)
+    assert np.array_equal(o.gate_up_silu_f16w(qw, s, x, rows=rows), o.gate_up_silu(qw, s, x)[:, rows])
+
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

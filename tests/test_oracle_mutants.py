@@ -57,7 +57,14 @@ MUTANTS = [
     ("dequant_f16_transposed", "w16[n * K + k] = zto_double_to_half", "w16[k * N + n] = zto_double_to_half"),
     ("gemm_f16w_first_token_for_all", "acc += w[k] * zto_half_to_double(x[m * K + k]);",
      "acc += w[k] * zto_half_to_double(x[k]);"),
-    ("gemm_f16w_rows_ignored", "const int64_t n = rows ? rows[i] : i;", "const int64_t n = i;"),
+    ("gemm_f16w_rows_ignored", "const int64_t n = rows ? rows[i] : i;\n        double *w = ",
+     "const int64_t n = i;\n        double *w = "),
+    ("gate_up_f16w_rows_ignored", "const int64_t n = rows ? rows[i] : i;\n        double *wg = ",
+     "const int64_t n = i;\n        double *wg = "),
+    ("gate_up_f16w_up_is_gate", "zto_weight(qw, scales, K, group, N + n, k)", "zto_weight(qw, scales, K, group, n, k)"),
+    ("gate_up_f16w_weights_not_rounded",
+     "wg[k] = zto_half_to_double(zto_double_to_half(zto_weight(qw, scales, K, group, n, k)));",
+     "wg[k] = zto_weight(qw, scales, K, group, n, k);"),
     ("sampled_rows_ignored", "int64_t n = rows ? rows[i] : i;\n        for (int64_t m = 0; m < M; ++m)\n            y[",
      "int64_t n = i;\n        for (int64_t m = 0; m < M; ++m)\n            y["),
 ]
