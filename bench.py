@@ -696,6 +696,7 @@ def run_prefill(args, local):
             stream.synchronize()
         return a.elapsed_time(b) / steps * 1e3
 
+    gate_up_w16 = []
     for M in [int(v) for v in args.prefill_m.split(",")]:
         x = torch.randn((M, K), device=device).half()
         y = torch.empty((M, N), dtype=torch.float16, device=device)
@@ -709,6 +710,21 @@ def run_prefill(args, local):
         deq = timed(lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][2],
                                                 stream=stream), steps)
         assert zt_q4.gemm_f16w_errors(gws) == 0 and all(zt_q4.gemm_errors(c, N, K) == 0 for c in ws)
+        # the fused FFN on the same tokens: Phi-3-mini gate_up 3072 -> 2 x 8192, SiLU(g) u in the epilogue,
+        # on cached binary16 weights (the GEMM alone)
+        ffn = gate_up_w16 if gate_up_w16 else [torch.empty((2 * 8192, K), dtype=torch.float16, device=device)
+                                               for _ in range(copies)]
+        if not gate_up_w16:
+            gp = synth.Proj("gate_up", "gate_up", K, 8192, synth.PROJ_GATE_UP)
+            for c in range(copies):
+                gq, gs, _ = synth.proj_inputs(args.seed, c, gp)
+                zt_q4.dequant_f16(torch.from_numpy(gq.view(np.int32)).to(device), torch.from_numpy(gs).to(device),
+                                  ffn[c], stream=stream)
+            gate_up_w16.extend(ffn)
+        yg = torch.empty((M, 8192), dtype=torch.float16, device=device)
+        gu_ws = torch.empty((256,), dtype=torch.uint8, device=device)
+        gu = timed(lambda i: zt_q4.gemm_f16w_gate_up_silu(ffn[i % copies], x, yg, gu_ws, stream=stream), steps)
+        assert zt_q4.gemm_f16w_errors(gu_ws) == 0
         flops = 2.0 * M * N * K
         deq_bytes = N * K // 2 + N * (K // 32) * 2 + N * K * 2
         g_tf = flops / gemm / 1e6
@@ -723,6 +739,9 @@ def run_prefill(args, local):
                 "dequant_roofline": {"bound": "hbm", "achieved": round(deq_bytes / deq / 1e3, 1), "peak": hbm_peak,
                                      "unit": "GB/s", "frac": round(deq_bytes / deq / 1e3 / hbm_peak, 4)
                                      if hbm_peak else None, "bytes_per_call": deq_bytes},
+                "gate_up_silu": {"us_per_call": round(gu, 2), "TFLOP/s": round(2.0 * M * 2 * 8192 * K / gu / 1e6, 1),
+                                 "what": "fused FFN gate_up 3072 -> 2 x 8192 + SiLU(g) u on the same tokens, "
+                                         "binary16 weights cached"},
                 "config": {"workload": f"Phi-3-mini qkv projection 3072->9216 for {M} tokens, q4 group-32, "
                                        "weights dequantized per call"}}
         print(json.dumps(line), flush=True)

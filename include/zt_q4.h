@@ -302,6 +302,25 @@ ZT_API int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t
 ZT_API int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out);
 
 /*
+ * Batched fused FFN (Zero-TVM write-up, kernel-fusion section: gate, up and
+ * SiLU in one pass) on the prefill reading of the weights: qw / scales hold 2N
+ * rows (gate rows 0..N-1, up rows N..2N-1), w16 likewise [2N][K];
+ *     y[m][n] = fp16(SiLU(g) * u),  g = sum_k w16[n][k] x[m][k],  u = sum_k w16[N+n][k] x[m][k],
+ * g and u in fp32 (tensor-core accumulation), SiLU(g) = g / (1 + e^-g) in fp32.
+ * The 2N-wide intermediate never leaves tensor memory.  Workspace: for
+ * zt_q4_gemm_gate_up_silu zt_q4_gemm_gate_up_workspace_bytes(M, N, K) bytes (w16,
+ * then the error word; read it with zt_q4_gemm_errors(workspace, 2 * N, K, &e));
+ * for zt_q4_gemm_f16w_gate_up_silu at least 256 bytes (the error word, read with
+ * zt_q4_gemm_f16w_errors).  Shapes, alignment and status codes as for zt_q4_gemm,
+ * with 2N in place of N.
+ */
+ZT_API size_t zt_q4_gemm_gate_up_workspace_bytes(int M, int N, int K);
+ZT_API int zt_q4_gemm_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y,
+                                   int M, int N, int K, int group, void *workspace, size_t ws_bytes, void *stream);
+ZT_API int zt_q4_gemm_f16w_gate_up_silu(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K,
+                                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * Host-side layout helpers (HOST pointers, synchronous, no CUDA calls).
  * pack:   q uint8 [N][K] codes 0..15  ->  qw uint32 [N][K/8], low nibble first.
  *         A code above 15 is ZT_ERR_INVALID_ARG (qw is then unspecified).

@@ -218,7 +218,12 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32])
 // Split K (blockIdx.z = split, kb_per k blocks each): with part != null the
 // CTA writes its fp32 partial tile to part[z][M][N] instead of y, and
 // q4_splitk_reduce_kernel sums the splits in order.
-template <int AM, int BN, bool TOKA>
+// SILU (with TOKA, unsplit): the fused FFN (Zero-TVM write-up, kernel-fusion
+// section: gate, up and SiLU in one pass) on the binary16 weights [2N][K],
+// gate rows first.  The B tile is two half boxes -- gate rows n0 .. n0 + BN/2
+// and up rows N + n0 .. -- so TMEM columns c and BN/2 + c hold g and u of the
+// same output, and the epilogue writes y = SiLU(g) u for BN/2 outputs.
+template <int AM, int BN, bool TOKA, bool SILU>
 __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_constant__ CUtensorMap tma_a,
                                                                    const __grid_constant__ CUtensorMap tma_b,
                                                                    __half *__restrict__ y, float *__restrict__ part,
@@ -238,7 +243,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     volatile uint32_t *consumed_s = reinterpret_cast<volatile uint32_t *>(tc_smem + (slot + 8 - raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int a0 = blockIdx.x * AM, b0 = blockIdx.y * BN;
+    static_assert(!SILU || TOKA, "the fused FFN epilogue needs tokens as the A operand");
+    const int a0 = blockIdx.x * AM, b0 = blockIdx.y * (SILU ? BN / 2 : BN);
     const int kb_lo = blockIdx.z * kb_per;
     const int kb_n = min((K + kTcK - 1) / kTcK - kb_lo, kb_per);   // k blocks of this split (>= 1)
 
@@ -275,7 +281,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
                          "r"(C::kStageBytes) : "memory");
             const uint32_t a = ring + s * C::kStageBytes;
             tc_tma_2d(a, &tma_a, (kb_lo + kb) * kTcK, a0, full(s));
-            tc_tma_2d(a + C::kABytes, &tma_b, (kb_lo + kb) * kTcK, b0, full(s));
+            if (SILU) {
+                // gate rows, then the matching up rows N further down the fused weight
+                tc_tma_2d(a + C::kABytes, &tma_b, (kb_lo + kb) * kTcK, b0, full(s));
+                tc_tma_2d(a + C::kABytes + (BN / 2) * kTcK * 2, &tma_b, (kb_lo + kb) * kTcK, N + b0, full(s));
+            } else {
+                tc_tma_2d(a + C::kABytes, &tma_b, (kb_lo + kb) * kTcK, b0, full(s));
+            }
             issued = kb + 1;
         }
     } else if (threadIdx.x == 32) {
@@ -322,6 +334,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
     const bool vec = TOKA && (N % 8) == 0 && ((reinterpret_cast<uintptr_t>(y) & 15) == 0);
     const bool vecp = TOKA && (N % 4) == 0 && ((reinterpret_cast<uintptr_t>(part) & 15) == 0);
     float *pz = part ? part + (size_t)blockIdx.z * M * N : nullptr;
+    if constexpr (SILU) {
+#pragma unroll 1
+        for (int h = 0; h < C::kHalves; ++h) {
+            const int m = a0 + h * kTcMma + warp * 32 + lane;          // this thread's token
+            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(h * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 64; ++c) {
+                uint32_t g[32], u[32];
+                tc_ld32(trow + (uint32_t)(c * 32), g);
+                tc_ld32(trow + (uint32_t)(BN / 2 + c * 32), u);
+                const int n = b0 + c * 32;
+                if (ok && m < M) {   // a block, not a jump: the next aligned loads stay converged
+                float o[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float gv = __uint_as_float(g[j]);
+                    o[j] = gv / (1.0f + expf(-gv)) * __uint_as_float(u[j]);
+                }
+                __half *dst = y + (size_t)m * N + n;
+                if (vec && n + 32 <= N) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v;
+                        uint32_t *pv = reinterpret_cast<uint32_t *>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            __half2 h2 = __floats2half2_rn(o[8 * q + 2 * e], o[8 * q + 2 * e + 1]);
+                            pv[e] = *reinterpret_cast<uint32_t *>(&h2);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + 8 * q) = v;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (n + j < N) dst[j] = __float2half_rn(o[j]);
+                }
+                }
+            }
+        }
+    } else {
 #pragma unroll 1
     for (int h = 0; h < C::kHalves; ++h) {
         const int ra = a0 + h * kTcMma + warp * 32 + lane;           // this thread's A row
@@ -385,6 +437,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
             }
         }
     }
+
+    }   // SILU
 
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();

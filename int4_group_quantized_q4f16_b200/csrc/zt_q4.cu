@@ -558,21 +558,23 @@ int launch_dequant(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, in
     return launch_status();
 }
 
-template <int AM, int BN, bool TOKA>
+template <int AM, int BN, bool TOKA, bool SILU = false>
 int launch_gemm_tc_cfg(const GemmPlan &p, const uint16_t *w16, const uint16_t *x, uint16_t *y, float *part, int M,
                        int N, int K, unsigned int *err, cudaStream_t st)
 {
     using C = TcCfg<AM, BN>;
-    const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<AM, BN, TOKA>);
+    const void *fn = reinterpret_cast<const void *>(&q4_gemm_tc_kernel<AM, BN, TOKA, SILU>);
     int sms = 0;
     if (resident_ctas(fn, kTcThreads, C::kSmem, sms) < 1) return ZT_ERR_DEVICE;
     const uint16_t *a = TOKA ? x : w16, *b = TOKA ? w16 : x;
-    const int ra = TOKA ? M : N, rb = TOKA ? N : M;
+    const int ra = TOKA ? M : N, rb = TOKA ? (SILU ? 2 * N : N) : M;   // rows of the two tensors
+    const int b_out = SILU ? BN / 2 : BN;                              // B rows (outputs) per CTA
+    const int b_rows = TOKA ? N : M;
     CUtensorMap ma, mb;
-    if (!tma_map_f16(&ma, a, K, ra, AM) || !tma_map_f16(&mb, b, K, rb, BN)) return ZT_ERR_DEVICE;
-    const dim3 grid((unsigned)((ra + AM - 1) / AM), (unsigned)((rb + BN - 1) / BN), (unsigned)p.splits);
+    if (!tma_map_f16(&ma, a, K, ra, AM) || !tma_map_f16(&mb, b, K, rb, b_out)) return ZT_ERR_DEVICE;
+    const dim3 grid((unsigned)((ra + AM - 1) / AM), (unsigned)((b_rows + b_out - 1) / b_out), (unsigned)p.splits);
     clear_stale_error();
-    q4_gemm_tc_kernel<AM, BN, TOKA><<<grid, kTcThreads, C::kSmem, st>>>(
+    q4_gemm_tc_kernel<AM, BN, TOKA, SILU><<<grid, kTcThreads, C::kSmem, st>>>(
         ma, mb, reinterpret_cast<__half *>(y), p.splits > 1 ? part : nullptr, M, N, K, p.kb_per, err);
     int rc = launch_status();
     if (rc || p.splits == 1) return rc;
@@ -580,6 +582,37 @@ int launch_gemm_tc_cfg(const GemmPlan &p, const uint16_t *w16, const uint16_t *x
     const int grid_r = (int)std::max(1ll, std::min((mn / 4 + 255) / 256, (long long)sms * 8));
     q4_splitk_reduce_kernel<<<grid_r, 256, 0, st>>>(part, reinterpret_cast<__half *>(y), mn, p.splits);
     return launch_status();
+}
+
+// The fused FFN on binary16 weights [2N][K]: tokens as the A operand (also
+// below 128 tokens: the tile's spare rows read zeros), B = BN/2 gate rows and
+// their BN/2 up rows, never split (SiLU needs whole sums); tile by the same
+// cost estimate over the 2N weight rows.
+GemmPlan gate_up_plan(int M, int N, int K)
+{
+    const long long kb_n = (K + kTcK - 1) / kTcK;
+    static const int tiles[][2] = {{256, 256}, {128, 256}, {128, 128}};
+    GemmPlan best{128, 128, 1, (int)kb_n, true};
+    double best_cost = 1e300;
+    for (const auto &t : tiles) {
+        if (t[0] == 256 && M < 128) continue;
+        const double c = plan_cost(t[0], t[1], 1, M, 2ll * N, kb_n, true);
+        if (c < best_cost) {
+            best_cost = c;
+            best = GemmPlan{t[0], t[1], 1, (int)kb_n, true};
+        }
+    }
+    return best;
+}
+
+int launch_gate_up_tc(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K, void *ws,
+                      cudaStream_t st)
+{
+    const GemmPlan p = gate_up_plan(M, N, K);
+    unsigned int *err = static_cast<unsigned int *>(ws);
+    if (p.am == 256) return launch_gemm_tc_cfg<256, 256, true, true>(p, w16, x, y, nullptr, M, N, K, err, st);
+    if (p.bn == 256) return launch_gemm_tc_cfg<128, 256, true, true>(p, w16, x, y, nullptr, M, N, K, err, st);
+    return launch_gemm_tc_cfg<128, 128, true, true>(p, w16, x, y, nullptr, M, N, K, err, st);
 }
 
 // ws: the GEMM's workspace (error word, then partials), f16w_ws_bytes long.
@@ -949,6 +982,52 @@ int zt_q4_gemm_errors(const void *workspace, int N, int K, unsigned int *out)
 {
     if (!workspace || !out || check_gemm_shapes(1, N, K) != ZT_OK) return ZT_ERR_INVALID_ARG;
     return read_error_word(static_cast<const unsigned char *>(workspace) + w16_bytes(N, K), out);
+}
+
+size_t zt_q4_gemm_gate_up_workspace_bytes(int M, int N, int K)
+{
+    if (N > INT_MAX / 2 || check_gemm_shapes(M, 2 * N, K) != ZT_OK) return 0;
+    return w16_bytes(2 * N, K) + 256;
+}
+
+int zt_q4_gemm_f16w_gate_up_silu(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, int N, int K,
+                                 void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w16 || !x || !y || !workspace) return ZT_ERR_INVALID_ARG;
+    if (N > INT_MAX / 2) return ZT_ERR_INVALID_ARG;
+    int rc = check_gemm_shapes(M, 2 * N, K);
+    if (rc) return rc;
+    if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(workspace, 16)) return ZT_ERR_MISALIGNED;
+    if (ws_bytes < 256) return ZT_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    clear_stale_error();
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);
+    if (e != cudaSuccess) {
+        g_last_cuda_error = e;
+        (void)cudaGetLastError();
+        return ZT_ERR_LAUNCH;
+    }
+    return launch_gate_up_tc(w16, x, y, M, N, K, workspace, st);
+}
+
+int zt_q4_gemm_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M,
+                            int N, int K, int group, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!qw || !scales || !x || !y || !workspace) return ZT_ERR_INVALID_ARG;
+    if (N > INT_MAX / 2) return ZT_ERR_INVALID_ARG;
+    int rc = check_gemm_shapes(M, 2 * N, K);
+    if (rc) return rc;
+    const int gsh = group_shift(K, group);
+    if (gsh < 0) return ZT_ERR_INVALID_ARG;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(scales, 2) || !aligned(y, 2))
+        return ZT_ERR_MISALIGNED;
+    if (ws_bytes < w16_bytes(2 * N, K) + 256) return ZT_ERR_WORKSPACE;
+    uint16_t *w16 = static_cast<uint16_t *>(workspace);
+    void *gws = static_cast<unsigned char *>(workspace) + w16_bytes(2 * N, K);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_dequant(qw, scales, w16, 2 * N, K, gsh, static_cast<unsigned int *>(gws), st);
+    if (rc) return rc;
+    return launch_gate_up_tc(w16, x, y, M, N, K, gws, st);
 }
 
 int zt_q4_pack_host(const uint8_t *q, int N, int K, uint32_t *qw)

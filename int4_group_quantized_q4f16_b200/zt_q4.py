@@ -90,8 +90,12 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_gemm_workspace_bytes.restype = ctypes.c_size_t
     lib.zt_q4_gemm.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_gemm_errors.argtypes = [_P, _I, _I, ctypes.POINTER(ctypes.c_uint)]
+    lib.zt_q4_gemm_gate_up_workspace_bytes.argtypes = [_I, _I, _I]
+    lib.zt_q4_gemm_gate_up_workspace_bytes.restype = ctypes.c_size_t
+    lib.zt_q4_gemm_gate_up_silu.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]
+    lib.zt_q4_gemm_f16w_gate_up_silu.argtypes = [_P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
     for f in (lib.zt_q4_dequant_f16, lib.zt_q4_gemm_f16w, lib.zt_q4_gemm, lib.zt_q4_gemm_errors,
-              lib.zt_q4_gemm_f16w_errors):
+              lib.zt_q4_gemm_f16w_errors, lib.zt_q4_gemm_gate_up_silu, lib.zt_q4_gemm_f16w_gate_up_silu):
         f.restype = ctypes.c_int
     lib.zt_q4_pack_host.argtypes = [_P, _I, _I, _P]
     lib.zt_q4_unpack_host.argtypes = [_P, _I, _I, _P]
@@ -271,6 +275,47 @@ def gemm_errors(workspace, N: int, K: int) -> int:
     out = ctypes.c_uint(0)
     _check(lib.zt_q4_gemm_errors(workspace.data_ptr(), N, K, ctypes.byref(out)), "zt_q4_gemm_errors")
     return int(out.value)
+
+
+def gemm_gate_up_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.zt_q4_gemm_gate_up_workspace_bytes(M, N, K))
+
+
+def gemm_gate_up_silu(qw, scales, x, y=None, workspace=None, stream=None):
+    """Batched fused FFN: y fp16 [M][N] = SiLU(x @ W16_gate^T) * (x @ W16_up^T),
+    qw / scales with 2N rows (gate first), through the binary16 weights."""
+    torch = _torch()
+    two_n, K = qw.shape[0], qw.shape[1] * 8
+    g = _group_of(K, scales)
+    M, N, _ = _dims(qw, scales, x, 2, g)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((gemm_gate_up_workspace_bytes(M, N, K),), dtype=torch.uint8, device=x.device)
+    _check(lib.zt_q4_gemm_gate_up_silu(qw.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, g,
+                                       workspace.data_ptr(), workspace.numel(), _stream_handle(stream)),
+           "zt_q4_gemm_gate_up_silu")
+    return y
+
+
+def gemm_f16w_gate_up_silu(w16, x, y=None, workspace=None, stream=None):
+    """The fused FFN on binary16 weights w16 [2N][K] (gate rows first)."""
+    torch = _torch()
+    for t, name in ((w16, "w16"), (x, "x")):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float16 or t.dim() != 2:
+            raise ValueError(f"{name} must be a contiguous 2-D float16 CUDA tensor")
+    (two_n, K), M = w16.shape, x.shape[0]
+    if x.shape[1] != K or two_n % 2:
+        raise ValueError("w16 must be [2N][K] with x [M][K]")
+    N = two_n // 2
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((256,), dtype=torch.uint8, device=x.device)
+    _check(lib.zt_q4_gemm_f16w_gate_up_silu(w16.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
+                                            workspace.data_ptr(), workspace.numel(), _stream_handle(stream)),
+           "zt_q4_gemm_f16w_gate_up_silu")
+    return y
 
 
 def lmhead_workspace_bytes(M: int, N: int, K: int) -> int:

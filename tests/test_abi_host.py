@@ -284,3 +284,19 @@ def test_withhold_hook_needs_a_wait(zt):
                   P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0))
     assert zt.lib.zt_q4_pass_test_withhold(arr, 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG
     assert zt.lib.zt_q4_pass_test_withhold(None, 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG
+
+
+def test_gemm_gate_up_arguments(zt):
+    f = zt.lib.zt_q4_gemm_gate_up_workspace_bytes
+    assert f(512, 8192, 3072) == ((2 * 8192 * 3072 * 2 + 255) // 256) * 256 + 256
+    assert f(0, 8192, 3072) == 0 and f(8, 0, 3072) == 0 and f(8, 8, 48) == 0 and f(8, 2 ** 30 + 1, 32) == 0
+    g = zt.lib.zt_q4_gemm_gate_up_silu
+    ws = f(40, 256, 512)
+    assert g(None, FAKE, FAKE, FAKE, 40, 256, 512, 32, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, FAKE, FAKE, 40, 256, 512, 48, FAKE, ws, None) == zt.ZT_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, FAKE + 8, FAKE, 40, 256, 512, 32, FAKE, ws, None) == zt.ZT_ERR_MISALIGNED
+    assert g(FAKE, FAKE, FAKE, FAKE, 40, 256, 512, 32, FAKE, ws - 1, None) == zt.ZT_ERR_WORKSPACE
+    h = zt.lib.zt_q4_gemm_f16w_gate_up_silu
+    assert h(FAKE, FAKE, FAKE, 40, 256, 512, None, 256, None) == zt.ZT_ERR_INVALID_ARG
+    assert h(FAKE, FAKE, FAKE, 40, 256, 512, FAKE, 255, None) == zt.ZT_ERR_WORKSPACE
+    assert h(FAKE + 8, FAKE, FAKE, 40, 256, 512, FAKE, 256, None) == zt.ZT_ERR_MISALIGNED

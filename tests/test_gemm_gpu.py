@@ -219,3 +219,41 @@ def test_gemm_tile_plans(zt, oracle, M, N, K):
                                      np.random.default_rng(N).integers(0, N, 40)])).astype(np.int32)
     ref = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
     assert_f16_matches(y[:, rows], ref, f"gemm plan M{M} N{N} K{K}", abs_products_f16w(oracle, qw, s, x, rows=rows))
+
+
+def gate_up_bound_f16w(oracle, qw, s, x, rows):
+    """Element bound for SiLU(g) u on binary16 weights, as for the exact
+    weights: |SiLU'| <= 1.1, accumulation errors 2^-14 sum |w16 x|."""
+    from parity import ACC_BOUND
+    N = qw.shape[0] // 2
+    g = oracle.gemm_f16w(qw, s, x, rows=rows, threads=8)
+    u = oracle.gemm_f16w(qw, s, x, rows=rows + N, threads=8)
+    eg = ACC_BOUND * abs_products_f16w(oracle, qw, s, x, rows=rows)
+    eu = ACC_BOUND * abs_products_f16w(oracle, qw, s, x, rows=rows + N)
+    silu = g / (1.0 + np.exp(-g))
+    return (1.1 * eg * np.abs(u) + np.abs(silu) * eu + eg * eu) / ACC_BOUND
+
+
+@pytest.mark.parametrize("M,N,K,group", [(40, 256, 512, 32), (200, 1000, 1056, 32), (300, 333, 256, 32),
+                                         (512, 8192, 3072, 32), (1100, 2048, 1024, 64), (2048, 8192, 3072, 32)])
+def test_gemm_gate_up_silu(zt, oracle, M, N, K, group):
+    """The fused FFN on the prefill path: gate rows and their up rows in one B
+    tile, SiLU(g) u in the epilogue; Phi-3-mini's gate_up (3072 -> 2 x 8192)
+    at 512 and 2048 tokens among the shapes; sampled rows, every token."""
+    import torch
+    qw, s32, _ = synth.problem(1200 + M, 2 * N, K, M=1, proj=2)
+    s = s32[:, ::group // 32].copy()
+    x = (_prefill_x(M + 7, M, K).astype(np.float32) * 0.5).astype(np.float16)
+    ws = torch.empty((zt.gemm_gate_up_workspace_bytes(M, N, K),), dtype=torch.uint8, device="cuda")
+    qd, sd, xd = dev(qw), dev(s), dev(x)
+    y = host(zt.gemm_gate_up_silu(qd, sd, xd, workspace=ws))
+    w16 = zt.dequant_f16(qd, sd)
+    gws = torch.empty((256,), dtype=torch.uint8, device="cuda")
+    y2 = host(zt.gemm_f16w_gate_up_silu(w16, xd, workspace=gws))
+    torch.cuda.synchronize()
+    assert zt.gemm_errors(ws, 2 * N, K) == 0 and zt.gemm_f16w_errors(gws) == 0
+    assert np.array_equal(y.view(np.uint16), y2.view(np.uint16))
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128, N - 1],
+                                     np.random.default_rng(N + M).integers(0, N, 40)])).astype(np.int32)
+    ref = oracle.gate_up_silu_f16w(qw, s, x, rows=rows, threads=8)
+    assert_f16_matches(y[:, rows], ref, f"gate_up M{M} N{N} K{K}", gate_up_bound_f16w(oracle, qw, s, x, rows))
