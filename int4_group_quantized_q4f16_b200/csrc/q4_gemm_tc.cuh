@@ -349,8 +349,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) q4_gemm_tc_kernel(const __grid_
                 float o[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
+                    // fast exp and divide: their error (a few fp32 ulp) is far below the fp16 output's
+                    // rounding; e^-g overflowing to inf gives SiLU = 0, its limit
                     const float gv = __uint_as_float(g[j]);
-                    o[j] = gv / (1.0f + expf(-gv)) * __uint_as_float(u[j]);
+                    o[j] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[j]);
                 }
                 __half *dst = y + (size_t)m * N + n;
                 if (vec && n + 32 <= N) {
