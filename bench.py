@@ -20,10 +20,14 @@ of the dominant kernel, the CPU oracle baseline, an end-to-end figure with
 host<->device copies, the SM clocks seen, and the launch count.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py --sweep-m        # gate_up single calls at M = 1, 2, 4, 8, 16
+  python bench.py --prefill        # batched prefill: dequant + tensor-core GEMM
 
 --impl reference times the float64 CPU oracle on the same workload (a bounded
 sample per step) on the host cores.  With N > 1 (torchrun) every rank runs
-its own replica (the path does not shard; weak scaling).
+its own replica (the path does not shard; weak scaling).  --prefill prints one
+line per token count with the GEMM against the measured tensor peak, the
+dequant against HBM, and the fused gate_up + SiLU on the same tokens.
 """
 from __future__ import annotations
 
