@@ -288,7 +288,9 @@ ZT_API int zt_q4_pass_test_withhold(const zt_q4_proj *projs, int n, int M, void 
  * The tile plan (and so the workspace size) is a function of (M, N, K) alone.
  * Shapes: 1 <= M <= 2^22, N >= 1, K >= 32, K % 32 == 0, N*K <= 2^40.  Inputs and
  * outputs must not overlap.  Status codes as elsewhere; ZT_ERR_DEVICE also when the
- * TMA descriptor encoder is unavailable.  The *_errors calls are synchronous.
+ * TMA descriptor encoder is unavailable; ZT_ERR_UNSUPPORTED when the plan's weight-row
+ * tiles exceed CUDA's 65535 grid rows (millions of weight rows; checked before any
+ * launch).  The *_errors calls are synchronous.
  */
 ZT_API int zt_q4_dequant_f16(const uint32_t *qw, const uint16_t *scales, uint16_t *w16, int N, int K, int group,
                              void *stream);

@@ -537,6 +537,16 @@ GemmPlan gemm_plan(int M, int N, int K)
     return best;
 }
 
+// CUDA caps grid.y (the weight-row tiles when tokens are the A operand, the
+// token tiles otherwise) at 65535: beyond that the shape is unsupported.
+// Checked on the host before anything is launched.
+bool gemm_grid_ok(const GemmPlan &p, int M, int N, bool silu)
+{
+    const long long b_rows = p.toka ? N : M;
+    const long long b_out = silu ? p.bn / 2 : p.bn;
+    return (b_rows + b_out - 1) / b_out <= 65535 && p.splits <= 65535;
+}
+
 size_t f16w_ws_bytes(int M, int N, int K)
 {
     const GemmPlan p = gemm_plan(M, N, K);
@@ -936,6 +946,7 @@ int zt_q4_gemm_f16w(const uint16_t *w16, const uint16_t *x, uint16_t *y, int M, 
     if (rc) return rc;
     if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(workspace, 16)) return ZT_ERR_MISALIGNED;
     if (ws_bytes < f16w_ws_bytes(M, N, K)) return ZT_ERR_WORKSPACE;
+    if (!gemm_grid_ok(gemm_plan(M, N, K), M, N, false)) return ZT_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     clear_stale_error();
     const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);
@@ -964,6 +975,7 @@ int zt_q4_gemm(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, ui
     if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return ZT_ERR_MISALIGNED;
     if (ws_bytes < w16_bytes(N, K) + f16w_ws_bytes(M, N, K)) return ZT_ERR_WORKSPACE;
+    if (!gemm_grid_ok(gemm_plan(M, N, K), M, N, false)) return ZT_ERR_UNSUPPORTED;
     uint16_t *w16 = static_cast<uint16_t *>(workspace);
     void *gws = static_cast<unsigned char *>(workspace) + w16_bytes(N, K);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -999,6 +1011,7 @@ int zt_q4_gemm_f16w_gate_up_silu(const uint16_t *w16, const uint16_t *x, uint16_
     if (rc) return rc;
     if (!aligned(w16, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(workspace, 16)) return ZT_ERR_MISALIGNED;
     if (ws_bytes < 256) return ZT_ERR_WORKSPACE;
+    if (!gemm_grid_ok(gate_up_plan(M, N, K), M, N, true)) return ZT_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     clear_stale_error();
     const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st);
@@ -1022,6 +1035,7 @@ int zt_q4_gemm_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const ui
     if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(scales, 2) || !aligned(y, 2))
         return ZT_ERR_MISALIGNED;
     if (ws_bytes < w16_bytes(2 * N, K) + 256) return ZT_ERR_WORKSPACE;
+    if (!gemm_grid_ok(gate_up_plan(M, N, K), M, N, true)) return ZT_ERR_UNSUPPORTED;
     uint16_t *w16 = static_cast<uint16_t *>(workspace);
     void *gws = static_cast<unsigned char *>(workspace) + w16_bytes(2 * N, K);
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -300,3 +300,24 @@ def test_gemm_gate_up_arguments(zt):
     assert h(FAKE, FAKE, FAKE, 40, 256, 512, None, 256, None) == zt.ZT_ERR_INVALID_ARG
     assert h(FAKE, FAKE, FAKE, 40, 256, 512, FAKE, 255, None) == zt.ZT_ERR_WORKSPACE
     assert h(FAKE + 8, FAKE, FAKE, 40, 256, 512, FAKE, 256, None) == zt.ZT_ERR_MISALIGNED
+
+
+def test_gemm_grid_limit_rejected_before_launch(zt):
+    """Weight-row tiles beyond CUDA's 65535 grid rows: ZT_ERR_UNSUPPORTED from
+    the host checks (no device needed); a large but legal shape passes them
+    (and only then meets the device: ZT_ERR_DEVICE without a GPU)."""
+    import torch
+    M, K = 128, 32
+    for N in (20_000_000,):            # > 65535 tiles of even 256 weight rows
+        ws = zt.gemm_workspace_bytes(M, N, K)
+        assert zt.lib.zt_q4_gemm(FAKE, FAKE, FAKE, FAKE, M, N, K, 32, FAKE, ws, None) == zt.ZT_ERR_UNSUPPORTED
+        gws = zt.gemm_f16w_workspace_bytes(M, N, K)
+        assert zt.lib.zt_q4_gemm_f16w(FAKE, FAKE, FAKE, M, N, K, FAKE, gws, None) == zt.ZT_ERR_UNSUPPORTED
+    N = 9_000_000
+    ws = zt.gemm_gate_up_workspace_bytes(M, N, K)
+    assert zt.lib.zt_q4_gemm_gate_up_silu(FAKE, FAKE, FAKE, FAKE, M, N, K, 32, FAKE, ws, None) == zt.ZT_ERR_UNSUPPORTED
+    assert zt.lib.zt_q4_gemm_f16w_gate_up_silu(FAKE, FAKE, FAKE, M, N, K, FAKE, 256, None) == zt.ZT_ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        N = 32064                                   # the Phi-3-mini LM head: legal
+        ws = zt.gemm_workspace_bytes(M, N, K)
+        assert zt.lib.zt_q4_gemm(FAKE, FAKE, FAKE, FAKE, M, N, K, 32, FAKE, ws, None) == zt.ZT_ERR_DEVICE
