@@ -548,6 +548,27 @@ def run_ours(args, world, rank, local):
     e2e_ms = dist_max(e0.elapsed_time(e1), world, device)
     e2e_value = total_bytes * world * e2e_steps / (e2e_ms / 1e3) / 1e9
 
+    # ---- a read-only stream probe of this GPU, beside the driver's copy peak:
+    # torch.sum over 2 GiB of fp16 (a library kernel), best of 5 -- context for
+    # the percentages only; any failure leaves it null ----
+    read_probe = None
+    try:
+        buf = torch.ones((1 << 30,), dtype=torch.float16, device=device)
+        best = float("inf")
+        with torch.cuda.stream(stream):
+            for _ in range(6):
+                p0 = torch.cuda.Event(enable_timing=True)
+                p1 = torch.cuda.Event(enable_timing=True)
+                p0.record(stream)
+                torch.sum(buf, dtype=torch.float32)
+                p1.record(stream)
+                stream.synchronize()
+                best = min(best, p0.elapsed_time(p1))
+        read_probe = round(buf.numel() * 2 / (best / 1e3) / 1e9, 1)
+        del buf
+    except Exception:   # noqa: BLE001 -- a context figure must never break the line
+        read_probe = None
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1:
@@ -587,6 +608,8 @@ def run_ours(args, world, rank, local):
             "us_per_pass": round(ms_per_step * 1e3, 2),
             "pct_of_nominal_8TBs": round(value / world / NOMINAL_HBM_GBS * 100, 2),
             "pct_of_measured_peak": round(value / world / peak * 100, 2),
+            "read_stream_probe_gbs": read_probe,
+            "pct_of_read_stream_probe": round(value / world / read_probe * 100, 2) if read_probe else None,
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "kernel": f"q4_pass_kernel (one launch per step over the {len(calls)} projections)",
