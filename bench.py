@@ -574,9 +574,19 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1:
         cores = host_cores()
         nb, secs = cpu_oracle_sample(args.seed, 4, cores)
+        # the same oracle on one thread, on the first layer's o projection (5.3 MB): bounded to ~1 s
+        import oracle as _oracle
+        o1 = _oracle.get()
+        p_o = synth.phi3_mini_layer()[1]
+        qo, so, xo = synth.proj_inputs(args.seed, 0, p_o)
+        t0 = time.perf_counter()
+        o1.gemv(qo, so, xo, threads=1)
+        t1 = time.perf_counter() - t0
         cpu = {"value": round(nb / secs / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"layers 0-3 of the pass (16 projections, {nb / 1e6:.1f} MB), float64 oracle, "
-                         f"OpenMP over rows, {secs:.1f} s"}
+                         f"OpenMP over rows, {secs:.1f} s",
+               "single_thread": {"value": round(alg_bytes(p_o) / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                 "sample": f"layer 0 o projection ({alg_bytes(p_o) / 1e6:.1f} MB), {t1:.2f} s"}}
 
     peaks = {}
     try:
