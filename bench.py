@@ -88,7 +88,7 @@ def alg_bytes(p: synth.Proj, M: int = 1) -> int:
     return p.weight_bytes() + M * p.K * 2 + M * p.n_out * out_bytes + (4 * M if p.kind == "lm_head" else 0)
 
 
-PASS_KERNEL_SOURCES = ("q4_gemv.cuh", "q4_mma.cuh", "q4_pass.cuh", "q4_stream.cuh")
+PASS_KERNEL_SOURCES = ("q4_common.cuh", "q4_mma.cuh", "q4_pass.cuh")
 
 
 def kernel_sources_sha() -> str:

@@ -244,6 +244,19 @@ typedef struct zt_q4_proj {
 ZT_API size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M);
 ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * Launch plan of the decode kernel (every decode entry point and zt_q4_pass run
+ * it), from the shapes alone -- no device is touched, nothing is launched:
+ * M tokens (1..16), K_max the largest K of the list (a multiple of 32), n the
+ * number of projections (1 for a single call).  Writes the CTAs resident per SM
+ * (1 or 2), the ring depth in weight items per warp (2..4), and k_window: 0 when
+ * each projection's activations are staged whole in shared memory, else the
+ * length in k of the windows that projections with K > k_window are staged in
+ * (a multiple of 256; the CTA then walks such a projection's rows in rounds and
+ * stages the windows in turn).  Every legal shape has a plan.  Diagnostics.
+ */
+ZT_API int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window);
+
 /* Synchronous read of a finished pass's error word (0: no bounded wait expired). */
 ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
 

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzt_q4.so")
 SOURCES = ["zt_q4.cu"]
-HEADERS = ["q4_gemv.cuh", "q4_stream.cuh", "q4_mma.cuh", "q4_pass.cuh", "q4_gemm_tc.cuh"]
+HEADERS = ["q4_common.cuh", "q4_mma.cuh", "q4_pass.cuh", "q4_gemm_tc.cuh"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 

@@ -34,6 +34,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "q4_common.cuh"
+
 namespace zt {
 
 __device__ __forceinline__ float4 ldg_stream_f4(const float *p)

@@ -60,7 +60,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "q4_stream.cuh"
+#include "q4_common.cuh"
 
 namespace zt {
 
@@ -166,16 +166,19 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
     }
 }
 
-__device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsigned char *xp, float *x7, int M,
-                                            int K, int G, int NT)
+// x: the first of the Gw groups to stage in row 0; row m starts ldx halves
+// further.  Gs: groups per staged column (the n-stride is Gs * 64 + 32 bytes);
+// the whole K is Gw = Gs = K / 32, a K window fewer groups.
+__device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ldx, unsigned char *xp, float *x7,
+                                            int M, int Gw, int Gs, int NT)
 {
-    const int K8 = K >> 3;                     // a multiple of 4: groups never straddle a column
+    const int K8 = Gw * 4;                     // 8-element pieces per row: groups never straddle a column
     const int total = M * K8;
-    const size_t nstride = (size_t)G * 64 + 32;
+    const size_t nstride = (size_t)Gs * 64 + 32;
     // C entries of the padding columns M .. 8 NT - 1 are zero
     const bool compact = M == 1;
     const int pad = compact ? 0 : 8 * NT - M;
-    for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
+    for (int j = threadIdx.x; j < Gw * pad; j += kMThreads) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
         float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -190,8 +193,8 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, unsign
         const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
         const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
-        if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * K + 8 * k0));
-        if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * K + 8 * k1));
+        if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * ldx + 8 * k0));
+        if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * ldx + 8 * k1));
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
         if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
@@ -275,6 +278,103 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
             xx[j] = __floats2half2_rn(hf.x * r * gf.x, hf.y * r * gf.y);
         }
         if (x_out) *reinterpret_cast<uint4 *>(x_out + (size_t)m * K + 8 * kk) = x;
+        return x;
+    };
+    for (int base = 0; base < total; base += 2 * kMThreads) {
+        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+        const bool v0 = i0 < total, v1 = i1 < total;
+        const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
+        const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
+        uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
+        if (v0) r0 = normalise(m0, k0);
+        if (v1) r1 = normalise(m1, k1);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
+        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+    }
+}
+
+// The same prologue for a projection whose activations are staged in K
+// windows (they do not fit in shared memory whole).  norm_rows takes the sums
+// of squares over all of K once per segment, in exactly stage_x_norm's order
+// (so r is bit-identical), writes h to res_out when non-null and r[m] to rn;
+// stage_x_norm_window then stages groups [g0, g0 + Gw) of x = fp16(h r gamma),
+// recomputing h = fp16(res + dlt) for just those k.  scratch: kMW floats.
+__device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, float eps, __half *res_out,
+                                          float *rn, float *scratch, int M, int K)
+{
+    const int K8 = K >> 3;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int m = 0; m < M; ++m) {
+        float part = 0.f;
+        for (int kk = threadIdx.x; kk < K8; kk += kMThreads) {
+            uint4 h = __ldcg(reinterpret_cast<const uint4 *>(res + (size_t)m * K + 8 * kk));
+            if (dlt) {
+                const uint4 d = __ldcg(reinterpret_cast<const uint4 *>(dlt + (size_t)m * K + 8 * kk));
+                h.x = hadd2_u32(h.x, d.x);
+                h.y = hadd2_u32(h.y, d.y);
+                h.z = hadd2_u32(h.z, d.z);
+                h.w = hadd2_u32(h.w, d.w);
+            }
+            if (res_out) *reinterpret_cast<uint4 *>(res_out + (size_t)m * K + 8 * kk) = h;
+            const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(hh[j]);
+                part = fmaf(f.x, f.x, part);
+                part = fmaf(f.y, f.y, part);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        if (lane == 0) scratch[warp] = part;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float ss = 0.f;
+            for (int w = 0; w < kMW; ++w) ss += scratch[w];
+            rn[m] = 1.0f / sqrtf(ss / (float)K + eps);
+        }
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ void stage_x_norm_window(const __half *res, const __half *dlt, const __half *gamma,
+                                                    __half *x_out, const float *rn, unsigned char *xp, float *x7,
+                                                    int M, int K, int g0, int Gw, int Gs, int NT)
+{
+    const int K8 = Gw * 4, k8_0 = g0 * 4;
+    const int total = M * K8;
+    const size_t nstride = (size_t)Gs * 64 + 32;
+    const bool compact = M == 1;
+    const int pad = compact ? 0 : 8 * NT - M;
+    for (int j = threadIdx.x; j < Gw * pad; j += kMThreads) {
+        const int g = j / pad, m = M + (j - (j / pad) * pad);
+        const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
+        float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
+        cv[e] = 0.f;
+        cv[2 + e] = 0.f;
+    }
+    auto normalise = [&](int m, int kk) {
+        const size_t off = (size_t)m * K + 8 * (size_t)(k8_0 + kk);
+        uint4 h = __ldcg(reinterpret_cast<const uint4 *>(res + off));
+        if (dlt) {
+            const uint4 d = __ldcg(reinterpret_cast<const uint4 *>(dlt + off));
+            h.x = hadd2_u32(h.x, d.x);
+            h.y = hadd2_u32(h.y, d.y);
+            h.z = hadd2_u32(h.z, d.z);
+            h.w = hadd2_u32(h.w, d.w);
+        }
+        const uint4 g = __ldcg(reinterpret_cast<const uint4 *>(gamma + 8 * (size_t)(k8_0 + kk)));
+        const float r = rn[m];
+        const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
+        const __half2 *gg = reinterpret_cast<const __half2 *>(&g);
+        uint4 x;
+        __half2 *xx = reinterpret_cast<__half2 *>(&x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 hf = __half22float2(hh[j]), gf = __half22float2(gg[j]);
+            xx[j] = __floats2half2_rn(hf.x * r * gf.x, hf.y * r * gf.y);
+        }
+        if (x_out) *reinterpret_cast<uint4 *>(x_out + off) = x;
         return x;
     };
     for (int base = 0; base < total; base += 2 * kMThreads) {

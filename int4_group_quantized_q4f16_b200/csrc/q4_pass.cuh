@@ -77,7 +77,8 @@ __device__ __forceinline__ int *pass_ws_idx(const PassProj &P, int M)
 template <int PMAX>
 struct PassArgs {
     int n, M, phases;
-    int g_max;                  // largest G of the list (sizes the activation area)
+    int g_stage;                // groups of K per column the activation area holds: the largest G of
+                                // the list, or (windowed kernel) the K window of longer projections
     unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
     int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
@@ -98,15 +99,16 @@ struct PassSeg {
     int n_tiles, n_chunks, wkl, rout;       // warp tiles, K chunks, log2 of the K-splitting warps
 };
 
-// Shared memory per CTA: rings, permuted activations (n-stride G*64 + 32
-// bytes), C-operand table, WK partials / LM-head maxima, segment list, flags.
-__host__ __device__ inline size_t pass_smem_bytes(int M, int g_max, int stages, int n, int NT)
+// Shared memory per CTA: rings, permuted activations (n-stride g_stage*64 +
+// 32 bytes), C-operand table, WK partials / LM-head maxima, segment list,
+// flags, the RMSNorm factors of a windowed segment (16 floats).
+__host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT)
 {
     const size_t ring = (size_t)kMW * stages * kMStage + 1024;   // + alignment of the code stages
-    const size_t xp = (size_t)M * ((size_t)g_max * 64 + 32);
-    const size_t x7 = M == 1 ? (size_t)g_max * 16 : (size_t)g_max * NT * 64;   // compact C table at M = 1
+    const size_t xp = (size_t)M * ((size_t)g_stage * 64 + 32);
+    const size_t x7 = M == 1 ? (size_t)g_stage * 16 : (size_t)g_stage * NT * 64;   // compact C table at M = 1
     return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT) * 4 + (size_t)n * sizeof(PassSeg) +
-           (kMW + 4) * sizeof(int);
+           (kMW + 4) * sizeof(int) + 16 * sizeof(float);
 }
 
 // Per-segment geometry of one warp.
@@ -120,15 +122,17 @@ static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel
 
 // log2 of the warps splitting K for a segment: minimise the items of the
 // busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
-// K-warps, with the partial buffer bounded (tiles * WK * 16 * 8 NT <= pass_red_floats).
-__device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT)
+// K-warps.  `bounded`: the whole segment's partials meet at once, so the
+// partial buffer bounds them (tiles * WK * 16 * 8 NT <= pass_red_floats); a
+// windowed segment reduces one round of at most 8 / WK tiles at a time.
+__device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool bounded)
 {
     int best = 0, best_cost = -1;
 #pragma unroll
     for (int wkl = 0; wkl <= 3; ++wkl) {
         const int wk = 1 << wkl;
         if (wk > n_chunks) break;
-        if (wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT)) break;
+        if (bounded && wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT)) break;
         const int cost = ((n_tiles + (kMW >> wkl) - 1) >> (3 - wkl)) * ((n_chunks + wk - 1) >> wkl);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
@@ -238,8 +242,13 @@ __device__ __noinline__ void rope_store(__half *out, size_t row_off, int pair, i
 }
 
 // NT: n-tiles of 8 activation columns (M <= 8 NT); ONE: M == 1, so the mma's
-// odd columns are never read and their accumulation is skipped; S: ring depth.
-template <int NT, int PMAX, int S, bool ONE>
+// odd columns are never read and their accumulation is skipped; S: ring depth;
+// WIN: projections with more than g_stage groups stage their activations in
+// K windows of g_stage groups (a multiple of 8): the CTA walks its tiles in
+// rounds of one tile per warp, and each round stages the windows in turn
+// while the warps' accumulators carry over (the weight stream's order is the
+// same as without windows).
+template <int NT, int PMAX, int S, bool ONE, bool WIN>
 __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
@@ -255,20 +264,22 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     unsigned char *ring_c = codes + (size_t)warp * S * kMCodeStage;
     unsigned char *ring_s = codes + (size_t)kMW * S * kMCodeStage + (size_t)warp * S * kMScaleStage;
     unsigned char *xp = codes + (size_t)kMW * S * kMStage;
-    const size_t xp_bytes = ((size_t)M * ((size_t)a.g_max * 64 + 32) + 15) & ~(size_t)15;
+    const size_t xp_bytes = ((size_t)M * ((size_t)a.g_stage * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
-    float *red = x7 + (ONE ? (size_t)a.g_max * 4 : (size_t)a.g_max * NT * 16);
+    float *red = x7 + (ONE ? (size_t)a.g_stage * 4 : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
     PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT));
     int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
     volatile int *abort_flag = wcount + kMW;
+    float *rn = reinterpret_cast<float *>(wcount + kMW + 4);   // RMSNorm factors of a windowed segment
 
     pdl_launch_dependents();
 
     // ---- this CTA's segments: per phase, its byte-balanced share of the
     //      phase's concatenated rows (a row belongs to the CTA whose share
     //      holds the row's first byte).  Thread p looks at projection p. ----
+    bool neutral_max = false;   // an LM head this CTA has no rows of: write a neutral partial maximum
     {
         PassSeg mine{};
         bool has = false;
@@ -289,16 +300,10 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
-                    mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT);
+                    mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
                 }
             }
-            if (!has && P.kind == kEpiLogits) {
-                // an LM head this CTA has no rows of still gets a (neutral) partial maximum
-                for (int m = 0; m < M; ++m) {
-                    P.ws_val[(size_t)blockIdx.x * M + m] = -INFINITY;
-                    pass_ws_idx(P, M)[(size_t)blockIdx.x * M + m] = 0x7fffffff;
-                }
-            }
+            neutral_max = !has && P.kind == kEpiLogits;
         }
         const unsigned ball = __ballot_sync(0xffffffffu, has);
         if (lane == 0) wcount[warp] = __popc(ball);
@@ -409,6 +414,15 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 #pragma unroll
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
+    if (neutral_max) {
+        // written only after the wait: the kernel ahead on the stream may be
+        // the argmax reduction of an earlier call that reads the same scratch
+        const PassProj &P = a.p[tid];
+        for (int m = 0; m < M; ++m) {
+            P.ws_val[(size_t)blockIdx.x * M + m] = -INFINITY;
+            pass_ws_idx(P, M)[(size_t)blockIdx.x * M + m] = 0x7fffffff;
+        }
+    }
 
     // row qg's codes: bits 4..6 of this offset hold qg (the stage bases are
     // multiples of 1024 from a 128-aligned array start), so XOR-ing gl * 16
@@ -435,16 +449,23 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d, gsh = P.gsh;
             const bool sasync = P.scales_async;
             void *const out = P.out;
-            if (P.norm) {
-                const bool writer = sgm.o_begin == 0;   // exactly one CTA holds row 0
-                stage_x_norm(P.res, P.dlt, P.gamma, P.eps, writer ? P.res_out : nullptr,
-                             writer ? P.x_out : nullptr, xp, x7, red, M, P.K, G, NT);
-            } else {
-                stage_x_mma(P.x, xp, x7, M, P.K, G, NT);
+            const bool writer = sgm.o_begin == 0;   // exactly one CTA holds row 0
+            // windowed: the segment's activations exceed the staging area (WIN kernels only)
+            const bool windowed = WIN && G > a.g_stage;
+            if (!windowed) {
+                if (P.norm) {
+                    stage_x_norm(P.res, P.dlt, P.gamma, P.eps, writer ? P.res_out : nullptr,
+                                 writer ? P.x_out : nullptr, xp, x7, red, M, P.K, G, NT);
+                } else {
+                    stage_x_mma(P.x, P.K, xp, x7, M, G, G, NT);
+                }
+                __syncthreads();
+            } else if (P.norm) {
+                norm_rows(P.res, P.dlt, P.eps, writer ? P.res_out : nullptr, rn, red, M, P.K);
             }
-            __syncthreads();
 
-            const uint32_t nstride = (uint32_t)G * 64u + 32u;
+            const int gs = windowed ? a.g_stage : G;   // groups per staged activation column
+            const uint32_t nstride = (uint32_t)gs * 64u + 32u;
             uint32_t xb[NT];   // B-operand column of this lane (columns >= M read column M-1: ignored)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -453,11 +474,52 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             // per chunk: 64 B of staged x per group; the C table 64 NT B per group (16 B compact)
             const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = ONE ? xstep / 4 : xstep * NT;
 
+            // The WK partials of tiles [t0, t0 + tn) meet here in a fixed order
+            // (tile t's partials sit at local index t - t0 of the buffer), and
+            // the epilogue of their outputs runs; best_v / best_i: the LM head's
+            // running maxima of this thread (slot 0: column tid % (8 NT)).
+            auto reduce_tiles = [&](auto log_tag, int t0, int tn, float (&best_v)[2 * NT], int (&best_i)[2 * NT]) {
+                constexpr bool LOG = decltype(log_tag)::value;
+                const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
+                for (int idx = tid; idx < tn * VO; idx += kMThreads) {
+                    const int tt = idx / VO, vo = idx - (idx / VO) * VO;
+                    const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
+                    const int nn = g.o_begin + (t0 + tt) * g.rout + r;
+                    if (nn >= g.o_end || m >= M) continue;
+                    const float *rp = red + (size_t)tt * g.wk * kMTileRows * 8 * NT;
+                    float y = 0.f, u = 0.f;
+                    for (int k2 = 0; k2 < g.wk; ++k2) {
+                        y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
+                        if (kind == kEpiGateUp || kind == kEpiRope)
+                            u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                    }
+                    y *= pow2f(24);
+                    if constexpr (LOG) {
+                        reinterpret_cast<float *>(out)[(size_t)m * ldo + nn] = y;
+                        // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
+                        if (better(y, nn, best_v[0], best_i[0])) {
+                            best_v[0] = isnan(y) ? -INFINITY : y;
+                            best_i[0] = nn;
+                        }
+                    } else if (kind == kEpiF16) {
+                        reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
+                    } else if (kind == kEpiRope) {
+                        rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta, P.pos[m],
+                                   y, u * pow2f(24));
+                    } else {
+                        u *= pow2f(24);
+                        const float silu = y / (1.0f + expf(-y));
+                        reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(silu * u);
+                    }
+                }
+            };
+
             // The segment's tiles; LOG: the LM head's epilogue (f32 logits and
             // running maxima) -- compiled apart so that the other projections'
-            // loop does not carry the maxima.
-            auto run_segment = [&](auto log_tag) {
+            // loop does not carry the maxima.  WS: a windowed segment.
+            auto run_segment = [&](auto log_tag, auto win_tag) {
                 constexpr bool LOG = decltype(log_tag)::value;
+                constexpr bool WS = decltype(win_tag)::value;
                 float best_v[2 * NT];
                 int best_i[2 * NT];
 #pragma unroll
@@ -465,7 +527,12 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     best_v[i] = -INFINITY;
                     best_i[i] = 0x7fffffff;
                 }
-                for (int tl = 0; tl < g.my_tiles; ++tl) {
+                // windowed: rounds of one tile per warp (the same count for all
+                // warps: every round stages the windows with the whole CTA)
+                const int n_rounds = WS ? (g.n_tiles + g.wr_n - 1) / g.wr_n : g.my_tiles;
+                const int n_win = WS ? (G + gs - 1) / gs : 1;
+                for (int tl = 0; tl < n_rounds; ++tl) {
+                    const bool have = !WS || tl < g.my_tiles;
                     const int t = g.my_wr + g.wr_n * tl;
                     const int o0 = g.o_begin + t * g.rout;
                     float acc[NT][4];
@@ -475,94 +542,117 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
                     uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
                     uint32_t coff = ONE ? xoff / 4 : xoff * NT;           // C-table bytes
-                    for (int cl = 0; cl < g.my_chunks; ++cl) {
-                        cp_async_wait<S - 2>();
-                        __syncwarp();
-                        const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
-                        uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
-                        if (sasync) {
-                            const unsigned char *sp = smem + sc_o + (st << 8);
-                            sg = *reinterpret_cast<const uint4 *>(sp);
-                            sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
-                            if (gsh) {
-                                // one scale per 32-block: repeat each of the 4 (or 2) scales 2 (or 4) times
-                                sg = spread_scales(sg, gsh);
-                                sg8 = spread_scales(sg8, gsh);
+                    int cl = 0;
+                    for (int w = 0; w < n_win; ++w) {
+                        int cl_end = g.my_chunks;
+                        if constexpr (WS) {
+                            // stage window w (groups [w gs, w gs + gn)) once every warp is done with w - 1
+                            __syncthreads();
+                            const int g0 = w * gs, gn = min(gs, G - g0);
+                            if (P.norm)
+                                stage_x_norm_window(P.res, P.dlt, P.gamma, (writer && tl == 0) ? P.x_out : nullptr,
+                                                    rn, xp, x7, M, P.K, g0, gn, gs, NT);
+                            else
+                                stage_x_mma(P.x + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT);
+                            __syncthreads();
+                            if (w > 0) {   // the area now starts at group w gs
+                                xoff -= (uint32_t)gs * 64u;
+                                coff -= ONE ? (uint32_t)gs * 16u : (uint32_t)gs * 64u * NT;
                             }
-                        } else {
-                            bool v0, v1;
-                            const int c = g.my_wk + g.wk * cl;
-                            const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
-                            const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
-                            uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                            const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) +
-                                                       (size_t)r0 * (G >> gsh);
-                            const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
-                                                       (size_t)r1 * (G >> gsh);
-                            for (int gl = 0; gl < kc; ++gl) {
-                                const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
-                                u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
-                                u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
-                            }
-                            sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-                            sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
+                            // this warp's chunks c = my_wk + wk cl below the window's end
+                            const int c_end = (w + 1) * (gs / kMChunkG);
+                            cl_end = have ? min(g.my_chunks, (c_end - g.my_wk + g.wk - 1) / g.wk) : 0;
                         }
-                        const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-                        // shared-memory pointers of the item; the unrolled groups add constants
-                        const uint32_t wb = wq_o + (st << 11);
-                        const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
-                        const unsigned char *bp[NT];
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
-                        auto step = [&](int gl) {
-                            const unsigned char *wa = smem + (wb ^ (uint32_t)(gl << 4));
-                            const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wa);
-                            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wa + 1024);
-                            const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                            const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
-                                                    w1s & 0x000F000Fu};
-                            const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
-                                                    w1s & 0x00F000F0u};
-                            const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                            const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                            const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                            const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
-                                const uint4 czu =
-                                    *reinterpret_cast<const uint4 *>(cp + (ONE ? gl * 16 : (gl * NT + nt) * 64));
-                                float d[4];
-                                mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
-                                          __uint_as_float(czu.z), __uint_as_float(czu.w));
-                                mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                                acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                                acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                                if (!ONE) {
-                                    acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                                    acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                        for (; cl < cl_end; ++cl) {
+                            cp_async_wait<S - 2>();
+                            __syncwarp();
+                            const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
+                            uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
+                            if (sasync) {
+                                const unsigned char *sp = smem + sc_o + (st << 8);
+                                sg = *reinterpret_cast<const uint4 *>(sp);
+                                sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
+                                if (gsh) {
+                                    // one scale per 32-block: repeat each of the 4 (or 2) scales 2 (or 4) times
+                                    sg = spread_scales(sg, gsh);
+                                    sg8 = spread_scales(sg8, gsh);
                                 }
+                            } else {
+                                bool v0, v1;
+                                const int c = g.my_wk + g.wk * cl;
+                                const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
+                                const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
+                                uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
+                                const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                           (size_t)r0 * (G >> gsh);
+                                const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                           (size_t)r1 * (G >> gsh);
+                                for (int gl = 0; gl < kc; ++gl) {
+                                    const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
+                                    u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
+                                    u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
+                                }
+                                sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+                                sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
                             }
-                        };
-                        if (kc == kMChunkG) {
+                            const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+                            // shared-memory pointers of the item; the unrolled groups add constants
+                            const uint32_t wb = wq_o + (st << 11);
+                            const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
+                            const unsigned char *bp[NT];
 #pragma unroll
-                            for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
-                        } else {
+                            for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
+                            auto step = [&](int gl) {
+                                const unsigned char *wa = smem + (wb ^ (uint32_t)(gl << 4));
+                                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wa);
+                                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wa + 1024);
+                                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                                const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
+                                                        w1s & 0x000F000Fu};
+                                const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
+                                                        w1s & 0x00F000F0u};
+                                const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+                                const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+                                const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+                                const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
 #pragma unroll
-                            for (int gl = 0; gl < kMChunkG; ++gl)
-                                if (gl < kc) step(gl);
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
+                                    const uint4 czu =
+                                        *reinterpret_cast<const uint4 *>(cp + (ONE ? gl * 16 : (gl * NT + nt) * 64));
+                                    float d[4];
+                                    mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
+                                              __uint_as_float(czu.z), __uint_as_float(czu.w));
+                                    mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                                    acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                                    acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                                    if (!ONE) {
+                                        acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                                        acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                                    }
+                                }
+                            };
+                            if (kc == kMChunkG) {
+#pragma unroll
+                                for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
+                            } else {
+#pragma unroll
+                                for (int gl = 0; gl < kMChunkG; ++gl)
+                                    if (gl < kc) step(gl);
+                            }
+                            __syncwarp();
+                            issue_next();
+                            st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
+                            xoff += xstep;
+                            coff += cstep;
                         }
-                        __syncwarp();
-                        issue_next();
-                        st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
-                        xoff += xstep;
-                        coff += cstep;
                     }
 
                     // ---- tile epilogue ----
-                    if (g.wk > 1) {
-                        // this warp's partial of tile t: [16 rows][8*NT columns]
-                        float *rp = red + ((size_t)t * g.wk + g.my_wk) * kMTileRows * 8 * NT;
+                    if (have && g.wk > 1) {
+                        // this warp's partial of tile t: [16 rows][8*NT columns]; windowed
+                        // rounds number their tiles from the round's first (my_wr)
+                        float *rp = red + ((size_t)(WS ? g.my_wr : t) * g.wk + g.my_wk) * kMTileRows * 8 * NT;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
@@ -570,7 +660,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
                             rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
                         }
-                    } else {
+                    } else if (have) {
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -609,43 +699,19 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             }
                         }
                     }
-                }
-
-                if (g.wk > 1) {
-                    // WK partials of each tile meet here; fixed summation order
-                    __syncthreads();
-                    const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
-                    for (int idx = tid; idx < g.n_tiles * VO; idx += kMThreads) {
-                        const int t = idx / VO, vo = idx - (idx / VO) * VO;
-                        const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
-                        const int nn = g.o_begin + t * g.rout + r;
-                        if (nn >= g.o_end || m >= M) continue;
-                        const float *rp = red + (size_t)t * g.wk * kMTileRows * 8 * NT;
-                        float y = 0.f, u = 0.f;
-                        for (int k2 = 0; k2 < g.wk; ++k2) {
-                            y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
-                            if (kind == kEpiGateUp || kind == kEpiRope)
-                                u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
-                        }
-                        y *= pow2f(24);
-                        if constexpr (LOG) {
-                            reinterpret_cast<float *>(out)[(size_t)m * ldo + nn] = y;
-                            // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
-                            if (better(y, nn, best_v[0], best_i[0])) {
-                                best_v[0] = isnan(y) ? -INFINITY : y;
-                                best_i[0] = nn;
-                            }
-                        } else if (kind == kEpiF16) {
-                            reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
-                        } else if (kind == kEpiRope) {
-                            rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta, P.pos[m],
-                                       y, u * pow2f(24));
-                        } else {
-                            u *= pow2f(24);
-                            const float silu = y / (1.0f + expf(-y));
-                            reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(silu * u);
+                    if constexpr (WS) {
+                        if (g.wk > 1) {
+                            // this round's WK partials meet before the next round writes the buffer
+                            __syncthreads();
+                            reduce_tiles(log_tag, tl * g.wr_n, min(g.wr_n, g.n_tiles - tl * g.wr_n), best_v, best_i);
                         }
                     }
+                }
+
+                if (!WS && g.wk > 1) {
+                    // WK partials of each tile meet here; fixed summation order
+                    __syncthreads();
+                    reduce_tiles(log_tag, 0, g.n_tiles, best_v, best_i);
                 }
 
                 if constexpr (LOG) {
@@ -679,8 +745,18 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     }
                 }
             };
-            if (kind == kEpiLogits) run_segment(std::true_type{});
-            else run_segment(std::false_type{});
+            if constexpr (WIN) {
+                if (windowed) {
+                    if (kind == kEpiLogits) run_segment(std::true_type{}, std::true_type{});
+                    else run_segment(std::false_type{}, std::true_type{});
+                } else {
+                    if (kind == kEpiLogits) run_segment(std::true_type{}, std::false_type{});
+                    else run_segment(std::false_type{}, std::false_type{});
+                }
+            } else {
+                if (kind == kEpiLogits) run_segment(std::true_type{}, std::false_type{});
+                else run_segment(std::false_type{}, std::false_type{});
+            }
             __syncthreads();   // the activation area and partial buffers are free again
         }
         if (ph + 1 < nphase) {

@@ -14,8 +14,7 @@
 #include <mutex>
 #include <unordered_map>
 
-#include "q4_gemv.cuh"
-#include "q4_stream.cuh"
+#include "q4_common.cuh"
 #include "q4_mma.cuh"
 #include "q4_pass.cuh"
 #include "q4_gemm_tc.cuh"
@@ -33,8 +32,6 @@ int check_shapes(int M, int N, int K, int row_mult)
     if ((int64_t)N * row_mult > INT_MAX) return ZT_ERR_INVALID_ARG;
     return ZT_OK;
 }
-
-int smallest_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 
 struct OccKey {
     const void *fn;
@@ -124,116 +121,53 @@ int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
     return nb > 0 ? nb : -1;
 }
 
-template <int R, int MT, int U, int EPI>
-int launch_one(Q4Args a, cudaStream_t st, int *grid_out)
-{
-    constexpr int ROUT = (EPI == kEpiGateUp) ? R / 2 : R;
-    const size_t smem = q4_smem_bytes(a.M, a.G);
-    if (smem > 227 * 1024) return ZT_ERR_UNSUPPORTED;
-    const void *fn = reinterpret_cast<const void *>(&q4_gemv_kernel<R, MT, U, EPI>);
-    int sms = 0;
-    const int occ = resident_ctas(fn, kThreads, smem, sms);
-    if (occ < 1) return ZT_ERR_DEVICE;
-    a.n_tiles = (a.N + ROUT - 1) / ROUT;
-    const int grid = std::max(1, std::min({a.n_tiles, sms * occ, kMaxCtas}));
-    if (grid_out) *grid_out = grid;
-    clear_stale_error();
-    q4_gemv_kernel<R, MT, U, EPI><<<grid, kThreads, smem, st>>>(a);
-    return launch_status();
-}
-
 // shared memory per CTA for 2 and for 1 resident CTA per SM (228 KiB per SM,
 // 1 KiB reserved per CTA)
 constexpr size_t kSmemTwoPerSm = 113 * 1024;
 constexpr size_t kSmemOnePerSm = 227 * 1024;
 
-// Warps splitting K for the streaming kernel: minimise the items of the
-// busiest warp (tiles per row-warp x chunks per K-warp); ties -> smaller WK.
-int pick_wk(int max_tiles, int n_chunks)
-{
-    int best = 1;
-    long best_cost = -1;
-    for (int wk = 1; wk <= kAW; wk *= 2) {
-        if (wk > n_chunks) break;
-        const int wr = kAW / wk;
-        const long cost = (long)((max_tiles + wr - 1) / wr) * ((n_chunks + wk - 1) / wk);
-        if (best_cost < 0 || cost < best_cost) {
-            best_cost = cost;
-            best = wk;
-        }
-    }
-    return best;
-}
+// How a pass launch stages its activations: CTAs per SM, ring depth, the
+// groups of K per column the activation area holds, and whether longer
+// projections go through K windows of that many groups.  A function of
+// (M, the list's largest K, the list length) only.
+struct PassPlan {
+    int cps, stages, g_stage;
+    bool win;
+};
 
-// Launch the streaming kernel; ZT_ERR_UNSUPPORTED if its rings and staged
-// activations do not fit in shared memory.
-template <int MT, int EPI>
-int launch_stream(const Q4Args &q, cudaStream_t st, int *grid_out)
+// Whole-K staging when the rings (2..4 stages) and all of x fit, two CTAs per
+// SM before one; otherwise K windows (a multiple of 8 groups, one item's
+// chunk) as long as fit three stages at two CTAs per SM, else one CTA per SM
+// with four stages.  Always succeeds for M <= 16 and lists of up to
+// kPassMax projections: the smallest window (8 groups) needs 96 KiB.
+PassPlan pass_plan(int M, int g_max, int n, int NT)
 {
-    constexpr int V = kAR * MT;
-    constexpr int ROUT = (EPI == kEpiGateUp) ? kAR / 2 : kAR;
-    const void *fn = reinterpret_cast<const void *>(&q4_stream_kernel<MT, EPI>);
-    int sms = 0;
-    if (resident_ctas(fn, kAThreads, 0, sms) < 1) return ZT_ERR_DEVICE;
-    StreamArgs a;
-    a.qw = q.qw;
-    a.scales = q.scales;
-    a.x = q.x;
-    a.out = q.out;
-    a.ws_val = q.ws_val;
-    a.ws_idx = q.ws_idx;
-    a.M = q.M;
-    a.N = q.N;
-    a.K = q.K;
-    a.G = q.G;
-    a.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
-    const int n_chunks = (q.G + kAChunkG - 1) / kAChunkG;
+    const size_t per_stage = (size_t)kMW * kMStage;
     for (int cps = 2; cps >= 1; --cps) {
-        const int grid = std::max(1, std::min({sms * cps, q.N, kMaxCtas}));
-        const int rows_max = (q.N + grid - 1) / grid;
-        a.max_tiles = (rows_max + ROUT - 1) / ROUT;
-        a.wk = pick_wk(a.max_tiles, n_chunks);
-        const size_t fixed = stream_smem_bytes(q.M, q.G, 0, a.wk, a.max_tiles, kAR, V);
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
-        const size_t per_stage = (size_t)kAW * kAStage;
-        const int stages = budget > fixed ? (int)std::min<size_t>(kAMaxStages, (budget - fixed) / per_stage) : 0;
-        if (stages < 2) continue;
-        a.stages = stages;
-        const size_t smem = stream_smem_bytes(q.M, q.G, stages, a.wk, a.max_tiles, kAR, V);
-        const int occ = resident_ctas(fn, kAThreads, smem, sms);
-        if (occ < cps) continue;
-        if (grid_out) *grid_out = grid;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid);
-        cfg.blockDim = dim3(kAThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        clear_stale_error();
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_stream_kernel<MT, EPI>, a);
-        if (e != cudaSuccess) {
-            g_last_cuda_error = e;
-            (void)cudaGetLastError();
-            return ZT_ERR_LAUNCH;
-        }
-        return ZT_OK;
+        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT);
+        const int stages = budget > fixed ? (int)std::min<size_t>(kPassMaxStages, (budget - fixed) / per_stage) : 0;
+        if (stages >= 2) return PassPlan{cps, stages, g_max, false};
     }
-    return ZT_ERR_UNSUPPORTED;
+    for (int cps = 2; cps >= 1; --cps) {
+        const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
+        const int stages = cps == 2 ? 3 : kPassMaxStages;
+        int best = 0;
+        for (int gw = kMChunkG; gw < g_max; gw += kMChunkG)
+            if (pass_smem_bytes(M, gw, stages, n, NT) <= budget) best = gw;
+        if (best > 0) return PassPlan{cps, stages, best, true};
+    }
+    return PassPlan{0, 0, 0, false};
 }
 
 // Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
 // some projection waits on earlier ones (all CTAs must be co-resident).
-// ZT_ERR_UNSUPPORTED if the rings and staged activations do not fit.
 constexpr int kNotResident = 1;   // launch_pass_s: this shape does not reach the wanted residency
 
-template <int NT, int PMAX, int S, bool ONE>
+template <int NT, int PMAX, int S, bool ONE, bool WIN>
 int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps)
 {
-    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S, ONE>);
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S, ONE, WIN>);
     int sms = 0;
     if (resident_ctas(fn, kMThreads, smem, sms) < cps) return kNotResident;
     cudaLaunchConfig_t cfg = {};
@@ -252,7 +186,7 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     clear_stale_error();
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S, ONE>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S, ONE, WIN>, a);
     if (e != cudaSuccess) {
         g_last_cuda_error = e;
         (void)cudaGetLastError();
@@ -261,19 +195,27 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
     return ZT_OK;
 }
 
-// Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
-// some projection waits on earlier ones (all CTAs must be co-resident).
-// Two CTAs per SM when the rings (2..4 stages) and the staged activations
-// fit in half the SM's shared memory, else one.  ZT_ERR_UNSUPPORTED if
-// neither fits.
+template <int NT, int PMAX, bool ONE, bool WIN>
+int launch_pass_w(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps,
+                  int stages)
+{
+    switch (stages) {
+    case 2: return launch_pass_s<NT, PMAX, 2, ONE, WIN>(a, cooperative, st, grid, smem, cps);
+    case 3: return launch_pass_s<NT, PMAX, 3, ONE, WIN>(a, cooperative, st, grid, smem, cps);
+    default: return launch_pass_s<NT, PMAX, 4, ONE, WIN>(a, cooperative, st, grid, smem, cps);
+    }
+}
+
+// Launch the tensor-core pass kernel over a.p[0 .. a.n) with the plan of
+// pass_plan.  ZT_ERR_DEVICE if the device cannot hold the planned residency.
 template <int NT, int PMAX, bool ONE>
 int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_out)
 {
     int sms = 0;
-    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2, ONE>), kMThreads, 0, sms) < 1)
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2, ONE, false>), kMThreads, 0, sms) < 1)
         return ZT_ERR_DEVICE;
-    a.g_max = 0;
-    for (int i = 0; i < a.n; ++i) a.g_max = std::max(a.g_max, a.p[i].G);
+    int g_max = 0;
+    for (int i = 0; i < a.n; ++i) g_max = std::max(g_max, a.p[i].G);
     // Phases: a new one at every projection that waits.  Each CTA takes a
     // byte-balanced share of each phase's concatenated rows.
     long long rows = 0;      // a CTA with no rows of a list without waits would only idle
@@ -289,103 +231,60 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         rows += p.N;
     }
     for (int i = 0; i < a.n; ++i) a.p[i].phase_bytes = phase_bytes[a.p[i].phase];
-    for (int cps = 2; cps >= 1; --cps) {
+    const PassPlan plan = pass_plan(a.M, g_max, a.n, NT);
+    if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
+    a.g_stage = plan.g_stage;
+    const size_t smem = pass_smem_bytes(a.M, plan.g_stage, plan.stages, a.n, NT);
+    // the planned CTAs per SM, or one if the device holds fewer at this shared memory size
+    for (int cps = plan.cps; cps >= 1; --cps) {
         const int grid = (int)std::max<long long>(
             1, std::min<long long>({(long long)sms * cps, cooperative ? (long long)sms * cps : rows, kMaxCtas}));
-        const size_t fixed = pass_smem_bytes(a.M, a.g_max, 0, a.n, NT);
-        const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
-        const size_t per_stage = (size_t)kMW * kMStage;
-        const int stages = budget > fixed ? (int)std::min<size_t>(kPassMaxStages, (budget - fixed) / per_stage) : 0;
-        if (stages < 2) continue;
-        const size_t smem = pass_smem_bytes(a.M, a.g_max, stages, a.n, NT);
-        int rc;
-        switch (stages) {
-        case 2: rc = launch_pass_s<NT, PMAX, 2, ONE>(a, cooperative, st, grid, smem, cps); break;
-        case 3: rc = launch_pass_s<NT, PMAX, 3, ONE>(a, cooperative, st, grid, smem, cps); break;
-        default: rc = launch_pass_s<NT, PMAX, 4, ONE>(a, cooperative, st, grid, smem, cps); break;
-        }
+        const int rc = plan.win ? launch_pass_w<NT, PMAX, ONE, true>(a, cooperative, st, grid, smem, cps, plan.stages)
+                                : launch_pass_w<NT, PMAX, ONE, false>(a, cooperative, st, grid, smem, cps, plan.stages);
         if (rc == kNotResident) continue;
         if (rc == ZT_OK && grid_out) *grid_out = grid;
         return rc;
     }
-    return ZT_ERR_UNSUPPORTED;
+    return ZT_ERR_DEVICE;
 }
 
 // One projection through the pass kernel (no waits, launched with PDL).
-int launch_single_pass(const Q4Args &q, int kind, cudaStream_t st, int *grid_out)
+// ws_val: the LM head's per-CTA maxima (the arg-max follows at ws_val +
+// kMaxCtas * M), null otherwise.
+template <int EPI>
+int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, void *out, float *ws_val, int M,
+              int N, int K, void *stream, int *grid_out)
 {
     PassArgs<1> a;
     a.n = 1;
-    a.M = q.M;
+    a.M = M;
     a.counters = nullptr;
     a.error = nullptr;
     a.withhold = -1;
     PassProj &p = a.p[0];
-    p.qw = q.qw;
-    p.scales = q.scales;
-    p.x = q.x;
-    p.out = q.out;
-    p.ws_val = q.ws_val;   // the arg-max follows at ws_val + kMaxCtas * M (q.ws_idx)
-    p.N = q.N;
-    p.K = q.K;
-    p.G = q.G;
-    p.kind = kind;
-    p.scales_async = (q.K % 256 == 0) && aligned(q.scales, 16);
+    p.qw = reinterpret_cast<const uint4 *>(qw);
+    p.scales = reinterpret_cast<const __half *>(scales);
+    p.x = reinterpret_cast<const __half *>(x);
+    p.out = out;
+    p.ws_val = ws_val;
+    p.N = N;
+    p.K = K;
+    p.G = K / kGroup;
+    p.kind = EPI;
+    p.scales_async = (K % 256 == 0) && aligned(scales, 16);
     p.wait = 0;
     p.norm = 0;
     p.res = p.dlt = p.gamma = nullptr;
     p.res_out = p.x_out = nullptr;
     p.eps = 0.f;
-    p.ldo = q.N;
+    p.ldo = N;
     p.pos = nullptr;
     p.theta = 0.f;
     p.rope_d = 0;
     p.gsh = 0;
-    if (q.M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
-    return (q.M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
-}
-
-template <int EPI>
-int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, void *out, float *ws_val,
-              int *ws_idx, int M, int N, int K, void *stream, int *grid_out)
-{
-    Q4Args a;
-    a.qw = reinterpret_cast<const uint4 *>(qw);
-    a.scales = reinterpret_cast<const __half *>(scales);
-    a.x = reinterpret_cast<const __half *>(x);
-    a.out = out;
-    a.ws_val = ws_val;
-    a.ws_idx = ws_idx;
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.G = K / kGroup;
-    a.n_tiles = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // The tensor-core kernel whenever its rings and activations fit.
-    {
-        const int rc = launch_single_pass(a, EPI, st, grid_out);
-        if (rc != ZT_ERR_UNSUPPORTED) return rc;
-    }
-    // Small batch: the CUDA-core streaming kernel when its ring fits.
-    if (M <= 4) {
-        int rc = ZT_ERR_UNSUPPORTED;
-        switch (smallest_mt(M)) {
-        case 1: rc = launch_stream<1, EPI>(a, st, grid_out); break;
-        case 2: rc = launch_stream<2, EPI>(a, st, grid_out); break;
-        default: rc = launch_stream<4, EPI>(a, st, grid_out); break;
-        }
-        if (rc != ZT_ERR_UNSUPPORTED) return rc;
-    }
-    // Otherwise the register-pipelined kernel: rows per warp tile R, groups in
-    // flight per lane U, padded batch MT.
-    switch (smallest_mt(M)) {
-    case 1: return launch_one<4, 1, 2, EPI>(a, st, grid_out);
-    case 2: return launch_one<4, 2, 1, EPI>(a, st, grid_out);
-    case 4: return launch_one<4, 4, 1, EPI>(a, st, grid_out);
-    case 8: return launch_one<2, 8, 1, EPI>(a, st, grid_out);
-    default: return launch_one<2, 16, 1, EPI>(a, st, grid_out);
-    }
+    if (M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
+    return (M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
 
 size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + sizeof(int)); }
@@ -672,7 +571,7 @@ const char *zt_q4_strerror(int status)
     case ZT_ERR_MISALIGNED: return "pointer misaligned (qw and x need 16 bytes, workspace 16, logits/argmax 4, scales/y 2)";
     case ZT_ERR_WORKSPACE: return "workspace smaller than zt_q4_lmhead_workspace_bytes()";
     case ZT_ERR_LAUNCH: return "CUDA kernel launch failed";
-    case ZT_ERR_UNSUPPORTED: return "shape is valid but exceeds this build's limits (staged activations must fit in shared memory: M*K*4.125 + 4096 bytes <= 227 KiB)";
+    case ZT_ERR_UNSUPPORTED: return "shape is valid but exceeds this build's limits";
     case ZT_ERR_DEVICE: return "no usable CUDA device, or a device attribute query failed";
     default: return "unknown status";
     }
@@ -685,7 +584,7 @@ int zt_q4_gemv(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, ui
     int rc = check_shapes(M, N, K, 1);
     if (rc) return rc;
     if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(y, 2)) return ZT_ERR_MISALIGNED;
-    return launch_q4<kEpiF16>(qw, scales, x, y, nullptr, nullptr, M, N, K, stream, nullptr);
+    return launch_q4<kEpiF16>(qw, scales, x, y, nullptr, M, N, K, stream, nullptr);
 }
 
 int zt_q4_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, uint16_t *y, int M,
@@ -695,7 +594,7 @@ int zt_q4_gate_up_silu(const uint32_t *qw, const uint16_t *scales, const uint16_
     int rc = check_shapes(M, N, K, 2);
     if (rc) return rc;
     if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(y, 2)) return ZT_ERR_MISALIGNED;
-    return launch_q4<kEpiGateUp>(qw, scales, x, y, nullptr, nullptr, M, N, K, stream, nullptr);
+    return launch_q4<kEpiGateUp>(qw, scales, x, y, nullptr, M, N, K, stream, nullptr);
 }
 
 size_t zt_q4_lmhead_workspace_bytes(int M, int N, int K)
@@ -717,7 +616,7 @@ int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const uint16
     float *ws_val = reinterpret_cast<float *>(workspace);
     int *ws_idx = reinterpret_cast<int *>(ws_val + (size_t)kMaxCtas * M);
     int grid = 0;
-    rc = launch_q4<kEpiLogits>(qw, scales, x, logits, ws_val, ws_idx, M, N, K, stream, &grid);
+    rc = launch_q4<kEpiLogits>(qw, scales, x, logits, ws_val, M, N, K, stream, &grid);
     if (rc) return rc;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(M);
@@ -746,6 +645,8 @@ int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scales, cons
     if (!qw || !scales || !x || !logits || !argmax) return ZT_ERR_INVALID_ARG;
     const int rc = check_shapes(M, N, K, 1);
     if (rc) return rc;
+    if (!aligned(qw, 16) || !aligned(x, 16) || !aligned(scales, 2) || !aligned(logits, 4) || !aligned(argmax, 4))
+        return ZT_ERR_MISALIGNED;
     if (lmhead_ws_bytes(M) > kNoAllocScratchBytes) return ZT_ERR_WORKSPACE;
     void *scratch = noalloc_scratch();
     if (!scratch) return ZT_ERR_DEVICE;
@@ -891,6 +792,18 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
             return ZT_ERR_LAUNCH;
         }
     }
+    return ZT_OK;
+}
+
+int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window)
+{
+    if (!ctas_per_sm || !stages || !k_window) return ZT_ERR_INVALID_ARG;
+    if (M < 1 || M > 16 || n < 1 || n > ZT_Q4_PASS_MAX || K_max < kGroup || K_max % kGroup) return ZT_ERR_INVALID_ARG;
+    const PassPlan plan = pass_plan(M, K_max / kGroup, n, M <= 8 ? 1 : 2);
+    if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
+    *ctas_per_sm = plan.cps;
+    *stages = plan.stages;
+    *k_window = plan.win ? plan.g_stage * kGroup : 0;
     return ZT_OK;
 }
 

@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_pass.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass.restype = ctypes.c_int
     lib.zt_q4_pass_errors.argtypes = [_P, _I, ctypes.POINTER(ctypes.c_uint)]
+    lib.zt_q4_pass_plan.argtypes = [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]
+    lib.zt_q4_pass_plan.restype = ctypes.c_int
     lib.zt_q4_pass_test_withhold.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass_test_withhold.restype = ctypes.c_int
     lib.zt_q4_pass_errors.restype = ctypes.c_int
@@ -351,6 +353,14 @@ def lmhead_argmax_noalloc(qw, scales, x, logits=None, argmax=None, stream=None):
                                            argmax.data_ptr(), M, N, K, _stream_handle(stream)),
            "zt_q4_lmhead_argmax_noalloc")
     return logits, argmax
+
+
+def pass_plan(M: int, K_max: int, n: int = 1) -> Tuple[int, int, int]:
+    """(CTAs per SM, ring stages, k_window) of the decode kernel for these
+    shapes; k_window 0 = activations staged whole (no device needed)."""
+    c, st, kw = _I(0), _I(0), _I(0)
+    _check(lib.zt_q4_pass_plan(M, K_max, n, ctypes.byref(c), ctypes.byref(st), ctypes.byref(kw)), "zt_q4_pass_plan")
+    return c.value, st.value, kw.value
 
 
 class Pass:
