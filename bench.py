@@ -75,11 +75,23 @@ def parse_args():
     return p.parse_args()
 
 
-def projections(layers: int):
+MODELS = {
+    "phi3": (synth.phi3_mini_layer, synth.phi3_mini_lm_head),
+    "llama7b": (synth.llama7b_layer, synth.llama7b_lm_head),
+}
+
+
+def projections(layers: int, model: str = "phi3"):
     """(layer, Proj) for every launch of the pass, LM head last."""
-    out = [(l, p) for l in range(layers) for p in synth.phi3_mini_layer()]
-    out.append((0, synth.phi3_mini_lm_head()))
+    layer, head = MODELS[model]
+    out = [(l, p) for l in range(layers) for p in layer()]
+    out.append((0, head()))
     return out
+
+
+def llama_workload(seed: int) -> str:
+    return ("Llama-7B decode weight pass, M=1: 32 x (qkv 4096->12288, o 4096->4096, gate_up 4096->2x11008 +SiLU*up, "
+            f"down 11008->4096) + LM head 4096->32000 f32+argmax; q4 group-32 weights, seed {seed}")
 
 
 def alg_bytes(p: synth.Proj, M: int = 1) -> int:
@@ -246,13 +258,13 @@ def run_reference(args, world, rank):
 
 
 # ------------------------------------------------------------- GPU side ----
-def build_pass(args, device):
+def build_pass(args, device, model: str = "phi3"):
     """Allocate the pass on the device: weights, activations, outputs.  All
     activations live in one contiguous buffer and all outputs in another, so
     an end-to-end step moves them with one copy each way."""
     import torch
     from int4_group_quantized_q4f16_b200 import zt_q4
-    projs = projections(args.layers)
+    projs = projections(args.layers, model)
     x_bytes = sum(p.K * 2 for _, p in projs)
     y_bytes = sum(p.n_out * (4 if p.kind == "lm_head" else 2) for _, p in projs) + 16
     xbuf = torch.empty((x_bytes,), dtype=torch.uint8, device=device)
@@ -311,7 +323,7 @@ def run_ours(args, world, rank, local):
     # activations are independent inputs, so no projection waits on another;
     # the chained form (each projection waits for all earlier ones, as when
     # every x were an earlier output) is timed below for comparison.
-    def make_pass(chained):
+    def make_pass(chained, calls=calls):
         projs = []
         for i, d in enumerate(calls):
             e = {"kind": d["p"].kind, "qw": d["qw"], "scales": d["s"], "x": d["x"], "out": d["y"],
@@ -569,6 +581,37 @@ def run_ours(args, world, rank, local):
     except Exception:   # noqa: BLE001 -- a context figure must never break the line
         read_probe = None
 
+    # ---- config 4: the Llama-7B decode weight pass (3.72 GB), independent
+    # and chained, each call between its own events on the launching stream ----
+    lcalls, _, _ = build_pass(args, device, "llama7b")
+    lbytes = sum(alg_bytes(d["p"]) for d in lcalls)
+    lpass, lchain = make_pass(False, lcalls), make_pass(True, lcalls)
+    l_steps = max(20, min(args.steps, 200))
+
+    def per_call_mean_us(zp, steps):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                zp.run(stream)
+            for e0_, e1_ in ev:
+                e0_.record(stream)
+                zp.run(stream)
+                e1_.record(stream)
+            stream.synchronize()
+        return statistics.mean(e0_.elapsed_time(e1_) for e0_, e1_ in ev) * 1e3
+
+    l_us = per_call_mean_us(lpass, l_steps)
+    l_chain_us = per_call_mean_us(lchain, max(10, l_steps // 4))
+    assert lpass.errors() == 0 and lchain.errors() == 0, "a bounded wait of the Llama pass expired"
+    del lpass, lchain, lcalls
+    torch.cuda.empty_cache()
+
+    # ---- config 3 (small batch) and the batched prefill, at modest step counts ----
+    sweep = sweep_m_results(args.seed, device, stream, max(64, min(args.steps, 200)), 3,
+                            float(measured_peaks().get("hbm_gbs", 6650.0)))
+    pre_rows, _, _ = prefill_results(args.seed, device, stream, [512, 2048], max(16, min(args.steps, 100)), 3)
+    torch.cuda.empty_cache()
+
     # ---- CPU oracle baseline (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1:
@@ -641,6 +684,16 @@ def run_ours(args, world, rank, local):
                                        "gate_up (96 norms, x computed while staging); calls alternating with "
                                        "the plain pass, each between its own events"},
             "per_call_graph_us_per_pass": round(per_call_us, 2),
+            "llama7b_pass": {"workload": llama_workload(args.seed), "us_per_pass": round(l_us, 2),
+                             "GBps": round(lbytes / l_us / 1e3, 1), "frac": round(lbytes / l_us / 1e3 / peak, 4),
+                             "bytes_per_pass": lbytes, "chained_us_per_pass": round(l_chain_us, 2),
+                             "steps": l_steps, "kernel": "q4_pass_kernel + argmax reduction, one zt_q4_pass call",
+                             "duration": "mean of event-bracketed zt_q4_pass calls"},
+            "small_batch": sweep_summary(sweep),
+            "prefill": {"workload": "Phi-3-mini qkv 3072->9216 (dequant + tcgen05 GEMM) and gate_up 3072->2x8192 "
+                                    "+SiLU (cached binary16 weights), q4 group-32",
+                        "tokens": {str(r["M"]): {k: v for k, v in r.items() if k != "M"} for r in pre_rows},
+                        "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst) and hbm_gbs"},
             "per_projection_us_isolated": per_kind_us,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -652,42 +705,91 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_sweep_m(args, local):
-    """The small-batch configuration: gate_up (K 3072, 2 x 8192 rows, SiLU(g)*u)
-    at M = 1, 2, 4, 8, 16 tokens.  Eight copies of the weights (8 x 28.3 MB,
-    larger than L2) are used in turn, so every call streams from HBM."""
+def _timed_calls(stream, fn, steps: int, warmup: int) -> float:
+    """us per call of fn(i), i = 0 .. steps - 1, after `warmup` untimed calls;
+    one CUDA-event pair on the launching stream around the timed calls."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            fn(i)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(steps):
+            fn(i)
+        b.record(stream)
+        stream.synchronize()
+    return a.elapsed_time(b) / steps * 1e3
+
+
+SWEEP_MS = (1, 2, 4, 8, 16)
+
+
+def sweep_m_results(seed: int, device, stream, steps: int, warmup: int, hbm_peak: float):
+    """The small-batch configuration: gate_up (K 3072, 2 x 8192 rows,
+    SiLU(g)*u) at M = 1, 2, 4, 8, 16 tokens through the decode entry point
+    (codes unpacked in registers into tensor-core mma operands), beside the
+    tcgen05 path of the batched prefill (weights dequantized to binary16 per
+    call; and on cached binary16 weights).  Eight weight copies (8 x 28.3 MB,
+    > L2) in turn, so every call streams its weights from HBM."""
     import torch
     from int4_group_quantized_q4f16_b200 import zt_q4
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
     K, N, copies = 3072, 8192, 8
     p = synth.Proj("gate_up", "gate_up", K, N, synth.PROJ_GATE_UP)
-    w = []
+    w, w16 = [], []
     for c in range(copies):
-        qw, s, _ = synth.proj_inputs(args.seed, c, p)
-        w.append((torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)))
-    stream = torch.cuda.Stream(device=device)
-    for M in (1, 2, 4, 8, 16):
-        x = torch.randn((M, K), device=device).half()
+        qw, s, _ = synth.proj_inputs(seed, c, p)
+        qd, sd = torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)
+        w.append((qd, sd))
+        w16.append(zt_q4.dequant_f16(qd, sd, stream=stream))
+    stream.synchronize()
+    ws = torch.empty((zt_q4.gemm_gate_up_workspace_bytes(16, N, K),), dtype=torch.uint8, device=device)
+    gws = torch.empty((256,), dtype=torch.uint8, device=device)
+    out = []
+    for M in SWEEP_MS:
+        x = torch.randn((M, K), generator=torch.Generator(device=device).manual_seed(M), device=device).half()
         y = torch.empty((M, N), dtype=torch.float16, device=device)
-        steps = max(args.steps, 8 * copies)
-        with torch.cuda.stream(stream):
-            for i in range(max(args.warmup, 3) * copies):
-                zt_q4.gate_up_silu(w[i % copies][0], w[i % copies][1], x, y, stream=stream)
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for i in range(steps):
-                zt_q4.gate_up_silu(w[i % copies][0], w[i % copies][1], x, y, stream=stream)
-            b.record(stream)
-            stream.synchronize()
-        us = a.elapsed_time(b) / steps * 1e3
+        n = max(steps, 8 * copies)
+        dec = _timed_calls(stream, lambda i: zt_q4.gate_up_silu(w[i % copies][0], w[i % copies][1], x, y,
+                                                                stream=stream), n, warmup * copies)
+        tcd = _timed_calls(stream, lambda i: zt_q4.gemm_gate_up_silu(w[i % copies][0], w[i % copies][1], x, y,
+                                                                     workspace=ws, stream=stream), n, warmup * copies)
+        tcc = _timed_calls(stream, lambda i: zt_q4.gemm_f16w_gate_up_silu(w16[i % copies], x, y, workspace=gws,
+                                                                          stream=stream), n, warmup * copies)
+        assert zt_q4.gemm_errors(ws, 2 * N, K) == 0 and zt_q4.gemm_f16w_errors(gws) == 0
         nbytes = alg_bytes(p, M)
-        print(json.dumps({"metric": "q4 gate_up GEMV effective HBM GB/s", "value": round(nbytes / us / 1e3, 1),
-                          "unit": "GB/s", "M": M, "us_per_call": round(us, 3), "bytes_per_call": nbytes,
-                          "flops_per_call": 2 * M * 2 * N * K, "steps": steps, "weight_copies": copies,
-                          "config": {"workload": "gate_up K=3072 N=2x8192 +SiLU*up, q4 group-32, single calls"}}),
+        out.append({"M": M, "decode_us": round(dec, 3), "decode_GBps": round(nbytes / dec / 1e3, 1),
+                    "decode_frac": round(nbytes / dec / 1e3 / hbm_peak, 4), "bytes_per_call": nbytes,
+                    "tcgen05_dequant_per_call_us": round(tcd, 3), "tcgen05_cached_f16_us": round(tcc, 3),
+                    "calls": n})
+    del w16
+    return out
+
+
+def sweep_summary(rows) -> dict:
+    cross = next((r["M"] for r in rows
+                  if min(r["tcgen05_dequant_per_call_us"], r["tcgen05_cached_f16_us"]) < r["decode_us"]), None)
+    return {"workload": "gate_up K=3072 N=2x8192 +SiLU*up, q4 group-32, single calls, 8 weight copies in turn",
+            "M": [r["M"] for r in rows], "decode_us": [r["decode_us"] for r in rows],
+            "decode_GBps": [r["decode_GBps"] for r in rows], "decode_frac": [r["decode_frac"] for r in rows],
+            "tcgen05_dequant_per_call_us": [r["tcgen05_dequant_per_call_us"] for r in rows],
+            "tcgen05_cached_f16_us": [r["tcgen05_cached_f16_us"] for r in rows],
+            "crossover_M": cross,
+            "crossover": "smallest M at which the tcgen05 prefill path beats the decode kernel; null: not up to 16"}
+
+
+def run_sweep_m(args, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=device)
+    rows = sweep_m_results(args.seed, device, stream, args.steps, max(args.warmup, 3),
+                           float(measured_peaks().get("hbm_gbs", 6650.0)))
+    for r in rows:
+        print(json.dumps({"metric": "q4 gate_up GEMV effective HBM GB/s", "value": r["decode_GBps"], "unit": "GB/s",
+                          **r, "config": {"workload": "gate_up K=3072 N=2x8192 +SiLU*up, q4 group-32, single calls"}}),
               flush=True)
+    print(json.dumps({"small_batch": sweep_summary(rows)}), flush=True)
 
 
 def measured_peaks() -> dict:
@@ -698,90 +800,86 @@ def measured_peaks() -> dict:
         return {}
 
 
-def run_prefill(args, local):
+def prefill_results(seed: int, device, stream, Ms, steps: int, warmup: int):
     """Batched prefill (M > 16): zt_q4_gemm = dequant to binary16 (HBM-bound)
-    + tcgen05 GEMM (tensor-bound) on the Phi-3-mini qkv projection.  Four
-    weight copies (4 x 28.3 MB of codes + 56.6 MB of w16 each) rotate so the
-    dequant streams from HBM; each timed region is bracketed by CUDA events on
-    the launching stream."""
+    + tcgen05 GEMM (tensor-bound) on the Phi-3-mini qkv projection, and the
+    fused gate_up + SiLU on cached binary16 weights.  Four weight copies
+    rotate so the dequant streams from HBM; each timed region is bracketed by
+    CUDA events on the launching stream."""
     import torch
     from int4_group_quantized_q4f16_b200 import zt_q4
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
     K, N, copies = 3072, 9216, 4
     p = synth.Proj("qkv", "gemv", K, N, synth.PROJ_QKV)
     w = []
     for c in range(copies):
-        qw, s, _ = synth.proj_inputs(args.seed, c, p)
+        qw, s, _ = synth.proj_inputs(seed, c, p)
         qd, sd = torch.from_numpy(qw.view(np.int32)).to(device), torch.from_numpy(s).to(device)
         w.append((qd, sd, torch.empty((N, K), dtype=torch.float16, device=device)))
     peaks = measured_peaks()
     tc_peak = peaks.get("bf16_tflops")
     hbm_peak = peaks.get("hbm_gbs")
-    stream = torch.cuda.Stream(device=device)
-
-    def timed(fn, steps):
-        with torch.cuda.stream(stream):
-            for i in range(max(args.warmup, 3) * copies):
-                fn(i)
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for i in range(steps):
-                fn(i)
-            b.record(stream)
-            stream.synchronize()
-        return a.elapsed_time(b) / steps * 1e3
-
-    gate_up_w16 = []
-    for M in [int(v) for v in args.prefill_m.split(",")]:
-        x = torch.randn((M, K), device=device).half()
+    gp = synth.Proj("gate_up", "gate_up", K, 8192, synth.PROJ_GATE_UP)
+    ffn = []
+    for c in range(copies):
+        gq, gs, _ = synth.proj_inputs(seed, c, gp)
+        ffn.append(zt_q4.dequant_f16(torch.from_numpy(gq.view(np.int32)).to(device), torch.from_numpy(gs).to(device),
+                                     stream=stream))
+    stream.synchronize()
+    out = []
+    for M in Ms:
+        x = torch.randn((M, K), generator=torch.Generator(device=device).manual_seed(M), device=device).half()
         y = torch.empty((M, N), dtype=torch.float16, device=device)
-        steps = max(min(args.steps, 200), 4 * copies)
+        n = max(steps, 4 * copies)
         ws = [torch.empty((zt_q4.gemm_workspace_bytes(M, N, K),), dtype=torch.uint8, device=device)
               for _ in range(copies)]
         gws = torch.empty((zt_q4.gemm_f16w_workspace_bytes(M, N, K),), dtype=torch.uint8, device=device)
-        both = timed(lambda i: zt_q4.gemm(w[i % copies][0], w[i % copies][1], x, y, ws[i % copies],
-                                          stream=stream), steps)
-        gemm = timed(lambda i: zt_q4.gemm_f16w(w[i % copies][2], x, y, gws, stream=stream), steps)
-        deq = timed(lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][2],
-                                                stream=stream), steps)
+        w_ = warmup * copies
+        both = _timed_calls(stream, lambda i: zt_q4.gemm(w[i % copies][0], w[i % copies][1], x, y, ws[i % copies],
+                                                         stream=stream), n, w_)
+        gemm = _timed_calls(stream, lambda i: zt_q4.gemm_f16w(w[i % copies][2], x, y, gws, stream=stream), n, w_)
+        deq = _timed_calls(stream, lambda i: zt_q4.dequant_f16(w[i % copies][0], w[i % copies][1], w[i % copies][2],
+                                                               stream=stream), n, w_)
         assert zt_q4.gemm_f16w_errors(gws) == 0 and all(zt_q4.gemm_errors(c, N, K) == 0 for c in ws)
-        # the fused FFN on the same tokens: Phi-3-mini gate_up 3072 -> 2 x 8192, SiLU(g) u in the epilogue,
-        # on cached binary16 weights (the GEMM alone)
-        ffn = gate_up_w16 if gate_up_w16 else [torch.empty((2 * 8192, K), dtype=torch.float16, device=device)
-                                               for _ in range(copies)]
-        if not gate_up_w16:
-            gp = synth.Proj("gate_up", "gate_up", K, 8192, synth.PROJ_GATE_UP)
-            for c in range(copies):
-                gq, gs, _ = synth.proj_inputs(args.seed, c, gp)
-                zt_q4.dequant_f16(torch.from_numpy(gq.view(np.int32)).to(device), torch.from_numpy(gs).to(device),
-                                  ffn[c], stream=stream)
-            gate_up_w16.extend(ffn)
         yg = torch.empty((M, 8192), dtype=torch.float16, device=device)
         gu_ws = torch.empty((256,), dtype=torch.uint8, device=device)
-        gu = timed(lambda i: zt_q4.gemm_f16w_gate_up_silu(ffn[i % copies], x, yg, gu_ws, stream=stream), steps)
+        gu = _timed_calls(stream, lambda i: zt_q4.gemm_f16w_gate_up_silu(ffn[i % copies], x, yg, gu_ws,
+                                                                         stream=stream), n, w_)
         assert zt_q4.gemm_f16w_errors(gu_ws) == 0
         flops = 2.0 * M * N * K
         deq_bytes = N * K // 2 + N * (K // 32) * 2 + N * K * 2
         g_tf = flops / gemm / 1e6
-        line = {"metric": "q4 prefill GEMM TFLOP/s (dequant to binary16 + tcgen05 GEMM)",
-                "value": round(flops / both / 1e6, 1), "unit": "TFLOP/s", "higher_is_better": True, "M": M,
-                "us_per_call": round(both, 2), "gemm_us": round(gemm, 2), "dequant_us": round(deq, 2),
-                "dtype": "f16 x f16 -> f32", "steps": steps, "weight_copies": copies,
-                "roofline": {"bound": "tensor", "achieved": round(g_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
-                             "frac": round(g_tf / tc_peak, 4) if tc_peak else None,
-                             "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst; fp16 runs at the bf16 rate)",
-                             "kernel": "q4_gemm_tc_kernel"},
-                "dequant_roofline": {"bound": "hbm", "achieved": round(deq_bytes / deq / 1e3, 1), "peak": hbm_peak,
-                                     "unit": "GB/s", "frac": round(deq_bytes / deq / 1e3 / hbm_peak, 4)
-                                     if hbm_peak else None, "bytes_per_call": deq_bytes},
-                "gate_up_silu": {"us_per_call": round(gu, 2), "TFLOP/s": round(2.0 * M * 2 * 8192 * K / gu / 1e6, 1),
-                                 "what": "fused FFN gate_up 3072 -> 2 x 8192 + SiLU(g) u on the same tokens, "
-                                         "binary16 weights cached"},
-                "config": {"workload": f"Phi-3-mini qkv projection 3072->9216 for {M} tokens, q4 group-32, "
-                                       "weights dequantized per call"}}
-        print(json.dumps(line), flush=True)
+        gu_tf = 2.0 * M * 2 * 8192 * K / gu / 1e6
+        out.append({"M": M, "us_per_call": round(both, 2), "TFLOPs_dequant_and_gemm": round(flops / both / 1e6, 1),
+                    "gemm_us": round(gemm, 2), "gemm_TFLOPs": round(g_tf, 1),
+                    "gemm_frac": round(g_tf / tc_peak, 4) if tc_peak else None,
+                    "dequant_us": round(deq, 2), "dequant_GBps": round(deq_bytes / deq / 1e3, 1),
+                    "dequant_frac": round(deq_bytes / deq / 1e3 / hbm_peak, 4) if hbm_peak else None,
+                    "gate_up_silu_us": round(gu, 2), "gate_up_silu_TFLOPs": round(gu_tf, 1),
+                    "gate_up_silu_frac": round(gu_tf / tc_peak, 4) if tc_peak else None, "calls": n})
+    return out, tc_peak, hbm_peak
+
+
+def run_prefill(args, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=device)
+    rows, tc_peak, hbm_peak = prefill_results(args.seed, device, stream,
+                                              [int(v) for v in args.prefill_m.split(",")],
+                                              max(min(args.steps, 200), 16), max(args.warmup, 3))
+    for r in rows:
+        print(json.dumps({
+            "metric": "q4 prefill GEMM TFLOP/s (dequant to binary16 + tcgen05 GEMM)",
+            "value": r["TFLOPs_dequant_and_gemm"], "unit": "TFLOP/s", "higher_is_better": True,
+            "dtype": "f16 x f16 -> f32", **r,
+            "roofline": {"bound": "tensor", "achieved": r["gemm_TFLOPs"], "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": r["gemm_frac"], "kernel": "q4_gemm_tc_kernel",
+                         "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst; fp16 runs at the bf16 rate)"},
+            "dequant_roofline": {"bound": "hbm", "achieved": r["dequant_GBps"], "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": r["dequant_frac"]},
+            "config": {"workload": f"Phi-3-mini qkv projection 3072->9216 for {r['M']} tokens, q4 group-32, "
+                                   "weights dequantized per call; gate_up_silu: 3072 -> 2 x 8192 on cached binary16 "
+                                   "weights"}}), flush=True)
 
 
 def main():

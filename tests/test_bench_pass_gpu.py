@@ -3,7 +3,10 @@ Phi-3-mini decode weight pass (32 layers of qkv 3072->9216, o 3072->3072,
 gate_up 3072->2x8192 + SiLU*up, down 8192->3072, then the LM head
 3072->32064 with f32 logits and argmax; Zero-TVM write-up, sections
 "完整的推理流水线" and "内核融合") as one zt_q4_pass call over all 129
-projections, built by the same code the benchmark times.
+projections, built by the same code the benchmark times -- and the same for
+the Llama-7B pass (32 layers of qkv 4096->12288, o 4096->4096, gate_up
+4096->2x11008 + SiLU*up, down 11008->4096, LM head 4096->32000; the wgpu-llm
+page's performance table runs Llama-7B at 4 bits).
 
 The oracle computes sampled rows of every projection of three layers one by
 one, and the whole LM head; a second run must reproduce the first bit for
@@ -27,15 +30,15 @@ def _sample_rows(n, seed):
     return np.unique(np.concatenate([[0, 1, n // 2, n - 2, n - 1], g.integers(0, n, 48)])).astype(np.int64)
 
 
-@pytest.fixture(scope="module")
-def full_pass():
+@pytest.fixture(scope="module", params=["phi3", "llama7b"])
+def full_pass(request):
     import torch
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import bench
     from int4_group_quantized_q4f16_b200 import zt_q4
     args = argparse.Namespace(layers=32, seed=0)
-    calls, _, _ = bench.build_pass(args, torch.device("cuda", 0))
+    calls, _, _ = bench.build_pass(args, torch.device("cuda", 0), request.param)
 
     def make(chained):
         projs = []
@@ -61,7 +64,8 @@ def test_full_pass_projection_count(full_pass):
     calls = full_pass[0]
     assert len(calls) == 129
     assert [d["p"].kind for d in calls[:4]] == ["gemv", "gemv", "gate_up", "gemv"]
-    assert calls[-1]["p"].kind == "lm_head" and calls[-1]["p"].n_out == 32064
+    assert calls[-1]["p"].kind == "lm_head" and calls[-1]["p"].n_out in (32064, 32000)
+    assert {d["p"].K for d in calls} in ({3072, 8192}, {4096, 11008})
 
 
 def _check_sampled(oracle, calls, outs, layer, what):
