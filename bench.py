@@ -69,6 +69,9 @@ def parse_args():
                    help="instead of the pass: the batched prefill GEMM (binary16 dequant + tensor-core GEMM) on the "
                         "Phi-3-mini qkv projection (K 3072, N 9216) at M = 128, 512, 2048 tokens, one JSON line per M")
     p.add_argument("--prefill-m", type=str, default="128,512,2048")
+    p.add_argument("--only-pass", action="store_true",
+                   help="time the pass alone and print its line without the comparisons, the CPU baseline and the "
+                        "other configurations (for profiling the pass kernel)")
     p.add_argument("--sweep-m", action="store_true",
                    help="instead of the pass: the fused gate_up projection (K 3072, 2 x 8192 rows) at M = 1, 2, 4, "
                         "8, 16, one JSON line per M")
@@ -369,6 +372,15 @@ def run_ours(args, world, rank, local):
     ms_per_step = ms_max / args.steps
     value = total_bytes * world * args.steps / (ms_max / 1e3) / 1e9
     assert zpass.errors() == 0, "a bounded wait of the pass kernel expired"
+    if args.only_pass:
+        if rank == 0:
+            kms = statistics.mean(launch_ms)
+            print(json.dumps({"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+                              "us_per_launch": round(kms * 1e3, 3), "bytes_per_step": total_bytes,
+                              "config": {"workload": workload(args.layers, args.seed), "only_pass": True},
+                              "clocks": clock_info}), flush=True)
+        return
 
     # ---- the chained form of the pass, for comparison ----
     with torch.cuda.stream(stream):

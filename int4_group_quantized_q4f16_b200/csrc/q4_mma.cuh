@@ -64,8 +64,13 @@
 
 namespace zt {
 
-constexpr int kMW = 8;                              // warps per CTA
+constexpr int kMW = 8;                              // math (consumer) warps per CTA
 constexpr int kMThreads = kMW * 32;
+
+// Barrier among the CTA's math warps (threads 0 .. kMThreads - 1) only: named
+// barrier 1, so that a copy-producer warp (if the kernel has one) need not
+// take part.  With no producer warp it is the same as __syncthreads().
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kMThreads) : "memory"); }
 constexpr int kMTileRows = 16;                      // weight rows per warp tile (mma M)
 constexpr int kMChunkG = 8;                         // groups per item
 // A ring stage holds an item: codes [16 rows][128 B] with the 128-byte XOR
@@ -115,13 +120,39 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
 }
 
+// Single-column (M = 1) staging for the block-diagonal contraction of
+// q4_pass.cuh: the area starts with 64 bytes of zeros (the B operand of the
+// lanes whose mma column is another group's), then group g's four 16-byte
+// pieces at 64 + 80 g (80, not 64: the lanes reading groups 2t and 2t + 1
+// then hit distinct banks); the C table holds one float per group.  Groups
+// are padded with zeros to a multiple of 8 (one item).
+constexpr int kBdZero = 64;
+constexpr int kBdGroup = 80;
+__host__ __device__ constexpr uint32_t bd_piece(int kk) { return kBdZero + (kk >> 2) * kBdGroup + (kk & 3) * 16; }
+__host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
+
+// zero x and C of groups [Gw, round8(Gw)) in the single-column layout
+__device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw)
+{
+    for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += kMThreads) {
+        *reinterpret_cast<uint4 *>(xp + bd_piece(Gw * 4 + j)) = make_uint4(0, 0, 0, 0);
+        if ((j & 3) == 0) x7[Gw + (j >> 2)] = 0.f;
+    }
+}
+
+// Byte offset of piece kk (8 activations) of column m in the staged area.
+__device__ __forceinline__ size_t x_piece(int m, int kk, size_t nstride, bool compact)
+{
+    return compact ? (size_t)bd_piece(kk) : (size_t)m * nstride + (size_t)kk * 16;
+}
+
 // Stage x in mma-B order: for column n and group g, 64 bytes = for t = 0..3:
 // step 0 (x[8t], x[8t+4], x[8t+2], x[8t+6]), step 1 (x[8t+1], x[8t+5],
 // x[8t+3], x[8t+7]) / 16 (k relative to 32g).  The C table holds, for each
 // (g, n-tile, quad thread t), (c, c', c, c') with c = -7 X_g 2^-24 of column
 // 8 nt + 2t and c' of the next column (zero for columns >= M).  With a single
-// column (compact) the table holds one entry (c, 0, c, 0) per group, which
-// every lane reads -- the other lanes' columns are never used.  Thread i of
+// column (compact) the layout is the block-diagonal one above and the table
+// holds c per group.  Thread i of
 // the CTA takes 8 activations of one column per round; the 4 threads of a
 // group are adjacent lanes.  Callers synchronise before reading.
 __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool valid, unsigned char *xp,
@@ -140,7 +171,7 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
         __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
         o.z = *reinterpret_cast<uint32_t *>(&q15);
         o.w = *reinterpret_cast<uint32_t *>(&q37);
-        *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = o;
+        *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, compact)) = o;
         const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
         float v[8];
 #pragma unroll
@@ -156,7 +187,7 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
     if (valid && (kk & 3) == 0) {
         const float c = part * (-7.0f * pow2f(-24));
         if (compact) {
-            *reinterpret_cast<float4 *>(x7 + (size_t)(kk >> 2) * 4) = make_float4(c, 0.f, c, 0.f);
+            x7[kk >> 2] = c;
         } else {
             const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
             float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -198,6 +229,7 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
         if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
+    if (compact) bd_pad(xp, x7, Gw);
 }
 
 // Residual add + RMSNorm ahead of a projection (the pages' add_norm step:
@@ -233,7 +265,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
                 h.z = hadd2_u32(h.z, d.z);
                 h.w = hadd2_u32(h.w, d.w);
             }
-            *reinterpret_cast<uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16) = h;
+            *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, M == 1)) = h;
             if (res_out) *reinterpret_cast<uint4 *>(res_out + (size_t)m * K + 8 * kk) = h;
             const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
 #pragma unroll
@@ -246,13 +278,13 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (lane == 0) scratch[warp] = part;
-        __syncthreads();
+        consumer_sync();
         if (threadIdx.x == 0) {
             float ss = 0.f;
             for (int w = 0; w < kMW; ++w) ss += scratch[w];
             scratch[kMW + m] = 1.0f / sqrtf(ss / (float)K + eps);
         }
-        __syncthreads();
+        consumer_sync();
     }
     const int total = M * K8;
     const bool compact = M == 1;
@@ -265,7 +297,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         cv[2 + e] = 0.f;
     }
     auto normalise = [&](int m, int kk) {
-        const uint4 h = *reinterpret_cast<const uint4 *>(xp + (size_t)m * nstride + (size_t)kk * 16);
+        const uint4 h = *reinterpret_cast<const uint4 *>(xp + x_piece(m, kk, nstride, compact));
         const uint4 g = __ldcg(reinterpret_cast<const uint4 *>(gamma + 8 * kk));
         const float r = scratch[kMW + m];
         const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
@@ -291,6 +323,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
         if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
+    if (compact) bd_pad(xp, x7, G);
 }
 
 // The same prologue for a projection whose activations are staged in K
@@ -327,13 +360,13 @@ __device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, 
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
         if (lane == 0) scratch[warp] = part;
-        __syncthreads();
+        consumer_sync();
         if (threadIdx.x == 0) {
             float ss = 0.f;
             for (int w = 0; w < kMW; ++w) ss += scratch[w];
             rn[m] = 1.0f / sqrtf(ss / (float)K + eps);
         }
-        __syncthreads();
+        consumer_sync();
     }
 }
 
@@ -388,6 +421,7 @@ __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __h
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
         if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
+    if (compact) bd_pad(xp, x7, Gw);
 }
 
 }  // namespace zt

@@ -105,8 +105,9 @@ struct PassSeg {
 __host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT)
 {
     const size_t ring = (size_t)kMW * stages * kMStage + 1024;   // + alignment of the code stages
-    const size_t xp = (size_t)M * ((size_t)g_stage * 64 + 32);
-    const size_t x7 = M == 1 ? (size_t)g_stage * 16 : (size_t)g_stage * NT * 64;   // compact C table at M = 1
+    // M = 1: the block-diagonal layout (a zero block, 80 bytes per group, one C float per group)
+    const size_t xp = M == 1 ? (size_t)kBdZero + (size_t)round8(g_stage) * kBdGroup : (size_t)M * ((size_t)g_stage * 64 + 32);
+    const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 4 : (size_t)g_stage * NT * 64;
     return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT) * 4 + (size_t)n * sizeof(PassSeg) +
            (kMW + 4) * sizeof(int) + 16 * sizeof(float);
 }
@@ -264,9 +265,10 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     unsigned char *ring_c = codes + (size_t)warp * S * kMCodeStage;
     unsigned char *ring_s = codes + (size_t)kMW * S * kMCodeStage + (size_t)warp * S * kMScaleStage;
     unsigned char *xp = codes + (size_t)kMW * S * kMStage;
-    const size_t xp_bytes = ((size_t)M * ((size_t)a.g_stage * 64 + 32) + 15) & ~(size_t)15;
+    const size_t xp_bytes = ONE ? (size_t)kBdZero + (size_t)round8(a.g_stage) * kBdGroup
+                                : ((size_t)M * ((size_t)a.g_stage * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
-    float *red = x7 + (ONE ? (size_t)a.g_stage * 4 : (size_t)a.g_stage * NT * 16);
+    float *red = x7 + (ONE ? (size_t)round8(a.g_stage) : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
     PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT));
@@ -308,6 +310,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         const unsigned ball = __ballot_sync(0xffffffffu, has);
         if (lane == 0) wcount[warp] = __popc(ball);
         if (tid == 0) *abort_flag = 0;
+        if (ONE && tid < kBdZero / 16) reinterpret_cast<uint4 *>(xp)[tid] = make_uint4(0, 0, 0, 0);   // the zero block
         __syncthreads();
         if (has) {
             int idx = __popc(ball & ((1u << lane) - 1u));
@@ -429,7 +432,17 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     // gives the swizzled chunk of group gl; row qg + 8 is 1024 bytes on
     const uint32_t wq_o = (uint32_t)(ring_c - smem) + qg * 128 + qt * 4 + (qg << 4);   // + stage * 2048
     const uint32_t sc_o = (uint32_t)(ring_s - smem) + qg * 16;                          // + stage * 256
-    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? 0 : qt * 16);
+    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? qt * 8 : qt * 16);
+    // M = 1 (block-diagonal): the mma's 8 columns are the item's 8 groups; lane (qg, qt) holds
+    // the codes of groups 2 qt and 2 qt + 1 of rows qg and qg + 8 (16 bytes each), and the B
+    // operand of group 2 qt (2 qt + 1) only if its column qg is that group, else zeros
+    const uint32_t bd_c0 = (uint32_t)(ring_c - smem) + qg * 128 + (((2 * qt) ^ qg) << 4);       // + stage * 2048
+    const uint32_t bd_c1 = (uint32_t)(ring_c - smem) + qg * 128 + (((2 * qt + 1) ^ qg) << 4);
+    const uint32_t xp_o = (uint32_t)(xp - smem);
+    const bool bd_sel0 = qg == 2 * qt, bd_sel1 = qg == 2 * qt + 1;
+    const uint32_t bd_b0 = bd_sel0 ? xp_o + kBdZero + 2 * qt * kBdGroup : xp_o;       // + chunk offset if selected
+    const uint32_t bd_b1 = bd_sel1 ? xp_o + kBdZero + (2 * qt + 1) * kBdGroup : xp_o;
+    const uint32_t bd_m0 = bd_sel0 ? 0xffffffffu : 0u, bd_m1 = bd_sel1 ? 0xffffffffu : 0u;
     uint32_t st = 0;                // ring stage of the next item to compute
     int cs = 0;
 
@@ -439,7 +452,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 atomicOr(a.error, kErrWaitExpired);
                 *abort_flag = 1;
             }
-            __syncthreads();
+            consumer_sync();
             if (*abort_flag) break;
         }
         for (; cs < nseg && segs[cs].phase == ph; ++cs) {
@@ -459,7 +472,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 } else {
                     stage_x_mma(P.x, P.K, xp, x7, M, G, G, NT);
                 }
-                __syncthreads();
+                consumer_sync();
             } else if (P.norm) {
                 norm_rows(P.res, P.dlt, P.eps, writer ? P.res_out : nullptr, rn, red, M, P.K);
             }
@@ -471,8 +484,9 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             for (int nt = 0; nt < NT; ++nt)
                 xb[nt] = (uint32_t)(xp - smem) + (uint32_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
             const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
-            // per chunk: 64 B of staged x per group; the C table 64 NT B per group (16 B compact)
-            const uint32_t xstep = (uint32_t)g.wk * kMChunkG * 64u, cstep = ONE ? xstep / 4 : xstep * NT;
+            // per chunk: XG bytes of staged x per group, CG bytes of the C table per group
+            constexpr uint32_t XG = ONE ? kBdGroup : 64u, CG = ONE ? 4u : 64u * NT;
+            const uint32_t xstep = (uint32_t)g.wk * kMChunkG * XG, cstep = (uint32_t)g.wk * kMChunkG * CG;
 
             // The WK partials of tiles [t0, t0 + tn) meet here in a fixed order
             // (tile t's partials sit at local index t - t0 of the buffer), and
@@ -540,24 +554,24 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-                    uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * 64u;   // B bytes of this warp's first chunk
-                    uint32_t coff = ONE ? xoff / 4 : xoff * NT;           // C-table bytes
+                    uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * XG;   // B bytes of this warp's first chunk
+                    uint32_t coff = (uint32_t)g.my_wk * kMChunkG * CG;   // C-table bytes
                     int cl = 0;
                     for (int w = 0; w < n_win; ++w) {
                         int cl_end = g.my_chunks;
                         if constexpr (WS) {
                             // stage window w (groups [w gs, w gs + gn)) once every warp is done with w - 1
-                            __syncthreads();
+                            consumer_sync();
                             const int g0 = w * gs, gn = min(gs, G - g0);
                             if (P.norm)
                                 stage_x_norm_window(P.res, P.dlt, P.gamma, (writer && tl == 0) ? P.x_out : nullptr,
                                                     rn, xp, x7, M, P.K, g0, gn, gs, NT);
                             else
                                 stage_x_mma(P.x + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT);
-                            __syncthreads();
+                            consumer_sync();
                             if (w > 0) {   // the area now starts at group w gs
-                                xoff -= (uint32_t)gs * 64u;
-                                coff -= ONE ? (uint32_t)gs * 16u : (uint32_t)gs * 64u * NT;
+                                xoff -= (uint32_t)gs * XG;
+                                coff -= (uint32_t)gs * CG;
                             }
                             // this warp's chunks c = my_wk + wk cl below the window's end
                             const int c_end = (w + 1) * (gs / kMChunkG);
@@ -567,78 +581,155 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             cp_async_wait<S - 2>();
                             __syncwarp();
                             const int kc = cl == g.my_chunks - 1 ? kc_last : kMChunkG;
-                            uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
-                            if (sasync) {
-                                const unsigned char *sp = smem + sc_o + (st << 8);
-                                sg = *reinterpret_cast<const uint4 *>(sp);
-                                sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
-                                if (gsh) {
-                                    // one scale per 32-block: repeat each of the 4 (or 2) scales 2 (or 4) times
-                                    sg = spread_scales(sg, gsh);
-                                    sg8 = spread_scales(sg8, gsh);
-                                }
-                            } else {
-                                bool v0, v1;
-                                const int c = g.my_wk + g.wk * cl;
-                                const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
-                                const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
-                                uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
-                                const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) +
-                                                           (size_t)r0 * (G >> gsh);
-                                const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
-                                                           (size_t)r1 * (G >> gsh);
-                                for (int gl = 0; gl < kc; ++gl) {
-                                    const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
-                                    u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
-                                    u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
-                                }
-                                sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
-                                sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
-                            }
-                            const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
-                            // shared-memory pointers of the item; the unrolled groups add constants
-                            const uint32_t wb = wq_o + (st << 11);
-                            const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
-                            const unsigned char *bp[NT];
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
-                            auto step = [&](int gl) {
-                                const unsigned char *wa = smem + (wb ^ (uint32_t)(gl << 4));
-                                const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wa);
-                                const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wa + 1024);
-                                const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
-                                const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
-                                                        w1s & 0x000F000Fu};
-                                const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
-                                                        w1s & 0x00F000F0u};
-                                const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
-                                const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
-                                const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
-                                const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
-                                    const uint4 czu =
-                                        *reinterpret_cast<const uint4 *>(cp + (ONE ? gl * 16 : (gl * NT + nt) * 64));
-                                    float d[4];
-                                    mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
-                                              __uint_as_float(czu.z), __uint_as_float(czu.w));
-                                    mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
-                                    acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
-                                    acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
-                                    if (!ONE) {
-                                        acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
-                                        acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                            if constexpr (ONE) {
+                                // Block-diagonal contraction of the item (M = 1): 16 mma steps, step
+                                // 4 t + p takes pair p of word t of the lane's four 16-byte chunks
+                                // (p: codes {0,4} | {2,6} | 16 {1,5} | 16 {3,7}), so column c of D
+                                // sums group c's 32 products; C starts it at -7 X_c 2^-24.
+                                const unsigned char *cw = smem + (st << 11);
+                                const uint4 qa = *reinterpret_cast<const uint4 *>(cw + bd_c0);          // row qg,     group 2 qt
+                                const uint4 qb = *reinterpret_cast<const uint4 *>(cw + bd_c0 + 1024);   // row qg + 8, group 2 qt
+                                const uint4 qc = *reinterpret_cast<const uint4 *>(cw + bd_c1);          // row qg,     group 2 qt + 1
+                                const uint4 qd = *reinterpret_cast<const uint4 *>(cw + bd_c1 + 1024);   // row qg + 8, group 2 qt + 1
+                                // scales of (row qg, qg + 8) x (group 2 qt, 2 qt + 1)
+                                float s00, s01, s10, s11;
+                                if (sasync) {
+                                    const unsigned char *sp = smem + sc_o + (st << 8);
+                                    if (gsh == 0) {
+                                        const __half2 h0 = *reinterpret_cast<const __half2 *>(sp + 4 * qt);
+                                        const __half2 h1 = *reinterpret_cast<const __half2 *>(sp + 128 + 4 * qt);
+                                        s00 = __low2float(h0);
+                                        s01 = __high2float(h0);
+                                        s10 = __low2float(h1);
+                                        s11 = __high2float(h1);
+                                    } else {
+                                        // 64 or 128 k per scale: both groups read the same one
+                                        const int off = 2 * ((2 * qt) >> gsh);
+                                        s00 = s01 = __half2float(*reinterpret_cast<const __half *>(sp + off));
+                                        s10 = s11 = __half2float(*reinterpret_cast<const __half *>(sp + 128 + off));
                                     }
+                                } else {
+                                    bool v0, v1;
+                                    const int c = g.my_wk + g.wk * cl;
+                                    const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
+                                    const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
+                                    const __half *p0 = P.scales + (size_t)r0 * (G >> gsh);
+                                    const __half *p1 = P.scales + (size_t)r1 * (G >> gsh);
+                                    const int b = c * kMChunkG + 2 * qt;
+                                    s00 = 2 * qt < kc ? __half2float(p0[b >> gsh]) : 0.f;
+                                    s10 = 2 * qt < kc ? __half2float(p1[b >> gsh]) : 0.f;
+                                    s01 = 2 * qt + 1 < kc ? __half2float(p0[(b + 1) >> gsh]) : 0.f;
+                                    s11 = 2 * qt + 1 < kc ? __half2float(p1[(b + 1) >> gsh]) : 0.f;
                                 }
-                            };
-                            if (kc == kMChunkG) {
+                                if (kc < kMChunkG) {
+                                    // the last chunk's missing groups: zero x and C were staged,
+                                    // and their scale slots were not copied (any bits): use 0
+                                    if (2 * qt >= kc) s00 = s10 = 0.f;
+                                    if (2 * qt + 1 >= kc) s01 = s11 = 0.f;
+                                }
+                                const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
+                                float d[4] = {cz.x, cz.y, cz.x, cz.y};
+                                const unsigned char *b0p = smem + bd_b0 + (xoff & bd_m0);
+                                const unsigned char *b1p = smem + bd_b1 + (xoff & bd_m1);
+                                const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
+                                const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
 #pragma unroll
-                                for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
+                                for (int t4 = 0; t4 < 4; ++t4) {
+                                    const uint4 x0 = *reinterpret_cast<const uint4 *>(b0p + 16 * t4);
+                                    const uint4 x1 = *reinterpret_cast<const uint4 *>(b1p + 16 * t4);
+                                    const uint32_t wa = wa4[t4], wb = wb4[t4], wc = wc4[t4], wd = wd4[t4];
+                                    const uint32_t was = wa >> 8, wbs = wb >> 8, wcs = wc >> 8, wds = wd >> 8;
+                                    const uint32_t A0[4] = {wa & 0x000F000Fu, wb & 0x000F000Fu, wc & 0x000F000Fu,
+                                                            wd & 0x000F000Fu};
+                                    mma_16816(d, A0, x0.x, x1.x, d[0], d[1], d[2], d[3]);
+                                    const uint32_t A1[4] = {was & 0x000F000Fu, wbs & 0x000F000Fu, wcs & 0x000F000Fu,
+                                                            wds & 0x000F000Fu};
+                                    mma_16816(d, A1, x0.y, x1.y, d[0], d[1], d[2], d[3]);
+                                    const uint32_t A2[4] = {wa & 0x00F000F0u, wb & 0x00F000F0u, wc & 0x00F000F0u,
+                                                            wd & 0x00F000F0u};
+                                    mma_16816(d, A2, x0.z, x1.z, d[0], d[1], d[2], d[3]);
+                                    const uint32_t A3[4] = {was & 0x00F000F0u, wbs & 0x00F000F0u, wcs & 0x00F000F0u,
+                                                            wds & 0x00F000F0u};
+                                    mma_16816(d, A3, x0.w, x1.w, d[0], d[1], d[2], d[3]);
+                                }
+                                acc[0][0] = fmaf(d[0], s00, acc[0][0]);
+                                acc[0][1] = fmaf(d[1], s01, acc[0][1]);
+                                acc[0][2] = fmaf(d[2], s10, acc[0][2]);
+                                acc[0][3] = fmaf(d[3], s11, acc[0][3]);
                             } else {
-#pragma unroll
-                                for (int gl = 0; gl < kMChunkG; ++gl)
-                                    if (gl < kc) step(gl);
+                                uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
+                                if (sasync) {
+                                    const unsigned char *sp = smem + sc_o + (st << 8);
+                                    sg = *reinterpret_cast<const uint4 *>(sp);
+                                    sg8 = *reinterpret_cast<const uint4 *>(sp + 8 * 16);
+                                    if (gsh) {
+                                        // one scale per 32-block: repeat each of the 4 (or 2) scales 2 (or 4) times
+                                        sg = spread_scales(sg, gsh);
+                                        sg8 = spread_scales(sg8, gsh);
+                                    }
+                                } else {
+                                    bool v0, v1;
+                                    const int c = g.my_wk + g.wk * cl;
+                                    const int r0 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg, v0);
+                                    const int r1 = pass_slot_row(kind, N, rope_d, g.o_end, o0, qg + 8, v1);
+                                    uint32_t u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0};
+                                    const unsigned short *p0 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                               (size_t)r0 * (G >> gsh);
+                                    const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
+                                                               (size_t)r1 * (G >> gsh);
+                                    for (int gl = 0; gl < kc; ++gl) {
+                                        const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
+                                        u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
+                                        u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
+                                    }
+                                    sg = make_uint4(u0[0], u0[1], u0[2], u0[3]);
+                                    sg8 = make_uint4(u1[0], u1[1], u1[2], u1[3]);
+                                }
+                                const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w}, sg8w[4] = {sg8.x, sg8.y, sg8.z, sg8.w};
+                                // shared-memory pointers of the item; the unrolled groups add constants
+                                const uint32_t wb = wq_o + (st << 11);
+                                const unsigned char *cp = smem + x7_o + coff;     // + (gl * NT + nt) * 64, compact: + gl * 16
+                                const unsigned char *bp[NT];
+    #pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) bp[nt] = smem + xb[nt] + xoff;   // + gl * 64
+                                auto step = [&](int gl) {
+                                    const unsigned char *wa = smem + (wb ^ (uint32_t)(gl << 4));
+                                    const uint32_t w0 = *reinterpret_cast<const uint32_t *>(wa);
+                                    const uint32_t w1 = *reinterpret_cast<const uint32_t *>(wa + 1024);
+                                    const uint32_t w0s = w0 >> 8, w1s = w1 >> 8;
+                                    const uint32_t A0[4] = {w0 & 0x000F000Fu, w1 & 0x000F000Fu, w0s & 0x000F000Fu,
+                                                            w1s & 0x000F000Fu};
+                                    const uint32_t A1[4] = {w0 & 0x00F000F0u, w1 & 0x00F000F0u, w0s & 0x00F000F0u,
+                                                            w1s & 0x00F000F0u};
+                                    const __half2 sh0 = *reinterpret_cast<const __half2 *>(&sgw[gl >> 1]);
+                                    const __half2 sh1 = *reinterpret_cast<const __half2 *>(&sg8w[gl >> 1]);
+                                    const float s0 = (gl & 1) ? __high2float(sh0) : __low2float(sh0);
+                                    const float s1 = (gl & 1) ? __high2float(sh1) : __low2float(sh1);
+    #pragma unroll
+                                    for (int nt = 0; nt < NT; ++nt) {
+                                        const uint4 bb = *reinterpret_cast<const uint4 *>(bp[nt] + gl * 64);
+                                        const uint4 czu =
+                                            *reinterpret_cast<const uint4 *>(cp + (ONE ? gl * 16 : (gl * NT + nt) * 64));
+                                        float d[4];
+                                        mma_16816(d, A0, bb.x, bb.y, __uint_as_float(czu.x), __uint_as_float(czu.y),
+                                                  __uint_as_float(czu.z), __uint_as_float(czu.w));
+                                        mma_16816(d, A1, bb.z, bb.w, d[0], d[1], d[2], d[3]);
+                                        acc[nt][0] = fmaf(d[0], s0, acc[nt][0]);
+                                        acc[nt][2] = fmaf(d[2], s1, acc[nt][2]);
+                                        if (!ONE) {
+                                            acc[nt][1] = fmaf(d[1], s0, acc[nt][1]);
+                                            acc[nt][3] = fmaf(d[3], s1, acc[nt][3]);
+                                        }
+                                    }
+                                };
+                                if (kc == kMChunkG) {
+    #pragma unroll
+                                    for (int gl = 0; gl < kMChunkG; ++gl) step(gl);
+                                } else {
+    #pragma unroll
+                                    for (int gl = 0; gl < kMChunkG; ++gl)
+                                        if (gl < kc) step(gl);
+                                }
                             }
                             __syncwarp();
                             issue_next();
@@ -646,6 +737,20 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             xoff += xstep;
                             coff += cstep;
                         }
+                    }
+
+                    if constexpr (ONE) {
+                        // a row's group partials are spread over the quad: sum them (the
+                        // same butterfly on every lane, so the order is fixed) into the
+                        // slots the single-column epilogue reads (quad thread 0, column 0)
+                        float r0 = acc[0][0] + acc[0][1], r1 = acc[0][2] + acc[0][3];
+                        r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+                        r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+                        r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+                        r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+                        acc[0][0] = r0;
+                        acc[0][2] = r1;
+                        acc[0][1] = acc[0][3] = 0.f;
                     }
 
                     // ---- tile epilogue ----
@@ -702,7 +807,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     if constexpr (WS) {
                         if (g.wk > 1) {
                             // this round's WK partials meet before the next round writes the buffer
-                            __syncthreads();
+                            consumer_sync();
                             reduce_tiles(log_tag, tl * g.wr_n, min(g.wr_n, g.n_tiles - tl * g.wr_n), best_v, best_i);
                         }
                     }
@@ -710,18 +815,18 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 
                 if (!WS && g.wk > 1) {
                     // WK partials of each tile meet here; fixed summation order
-                    __syncthreads();
+                    consumer_sync();
                     reduce_tiles(log_tag, 0, g.n_tiles, best_v, best_i);
                 }
 
                 if constexpr (LOG) {
-                    __syncthreads();   // the maxima overwrite the partial buffer
+                    consumer_sync();   // the maxima overwrite the partial buffer
 #pragma unroll
                     for (int i = 0; i < 2 * NT; ++i) {
                         bvs[tid * 2 * NT + i] = best_v[i];
                         bis[tid * 2 * NT + i] = best_i[i];
                     }
-                    __syncthreads();
+                    consumer_sync();
                     if (tid < M) {
                         float bv = -INFINITY;
                         int bi = 0x7fffffff;
@@ -757,12 +862,12 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 if (kind == kEpiLogits) run_segment(std::true_type{}, std::false_type{});
                 else run_segment(std::false_type{}, std::false_type{});
             }
-            __syncthreads();   // the activation area and partial buffers are free again
+            consumer_sync();   // the activation area and partial buffers are free again
         }
         if (ph + 1 < nphase) {
             // publish this CTA's outputs of the phase, then count it done
             __threadfence();
-            __syncthreads();
+            consumer_sync();
             if (tid == 0 && !(ph == a.withhold && blockIdx.x == 0)) atomicAdd(&a.counters[ph], 1u);
         }
     }
