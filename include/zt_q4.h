@@ -140,6 +140,11 @@ ZT_API int zt_q4_lmhead_argmax(const uint32_t *qw, const uint16_t *scales, const
  *     give wrong argmax; serialize them (one stream, or events).
  *   - Nothing in the array needs to start at zero: each call writes every
  *     entry it later reads.
+ *   - Every check (null pointers, shapes, alignment, the array's size) runs
+ *     before the first CUDA call.
+ *   - The array's device address is looked up once per device and kept for
+ *     the life of the process; after cudaDeviceReset the library must be
+ *     reloaded before this entry point is used again.
  */
 ZT_API int zt_q4_lmhead_argmax_noalloc(const uint32_t *qw, const uint16_t *scales, const uint16_t *x,
                                        float *logits, int32_t *argmax, int M, int N, int K, void *stream);
@@ -355,7 +360,7 @@ ZT_API const char *zt_q4_strerror(int status);
  */
 ZT_API const char *zt_q4_last_cuda_error(void);
 
-/* Library ABI version, (major << 16) | minor. */
+/* Library ABI version, (major << 16) | minor.  1.3 added zt_q4_pass_plan. */
 ZT_API int zt_q4_version(void);
 
 #ifdef __cplusplus

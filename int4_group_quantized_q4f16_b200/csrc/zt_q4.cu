@@ -556,7 +556,7 @@ int read_error_word(const void *p, unsigned int *out)
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 2; }
+int zt_q4_version(void) { return (1 << 16) | 3; }
 
 const char *zt_q4_last_cuda_error(void)
 {
