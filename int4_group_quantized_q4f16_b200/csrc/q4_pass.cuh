@@ -731,7 +731,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                                         if (gl < kc) step(gl);
                                 }
                             }
-                            __syncwarp();
+                            // the refill goes to the previous item's stage, which every lane finished
+                            // reading before it passed this item's __syncwarp above
                             issue_next();
                             st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
                             xoff += xstep;
@@ -820,29 +821,49 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                 }
 
                 if constexpr (LOG) {
-                    consumer_sync();   // the maxima overwrite the partial buffer
+                    // The CTA's (maximum, lowest index) per column m under better()'s total order
+                    // (so the reduction order does not matter): within each warp a butterfly over
+                    // the lanes that hold the same column, then the 8 warps' results per column.
+                    // Column of slot i: with WK > 1 only slot 0, column lane % (8 NT); otherwise
+                    // column 8 (i >> 1) + 2 qt + (i & 1), shared by the lanes of equal qt.
+                    auto comb = [&](float &v, int &ix, int mask) {
+                        const float ov = __shfl_xor_sync(0xffffffffu, v, mask);
+                        const int oi = __shfl_xor_sync(0xffffffffu, ix, mask);
+                        if (better(ov, oi, v, ix)) {
+                            v = isnan(ov) ? -INFINITY : ov;
+                            ix = oi;
+                        }
+                    };
+                    if (g.wk > 1) {
+                        for (int mask = 8 * NT; mask < 32; mask <<= 1) comb(best_v[0], best_i[0], mask);
+                    } else {
 #pragma unroll
-                    for (int i = 0; i < 2 * NT; ++i) {
-                        bvs[tid * 2 * NT + i] = best_v[i];
-                        bis[tid * 2 * NT + i] = best_i[i];
+                        for (int i = 0; i < 2 * NT; ++i)
+#pragma unroll
+                            for (int mask = 4; mask < 32; mask <<= 1) comb(best_v[i], best_i[i], mask);
+                    }
+                    consumer_sync();   // the warp results overwrite the partial buffer
+                    if (g.wk > 1) {
+                        if (lane < 8 * NT) {
+                            bvs[warp * 8 * NT + lane] = best_v[0];
+                            bis[warp * 8 * NT + lane] = best_i[0];
+                        }
+                    } else if (qg == 0) {
+#pragma unroll
+                        for (int i = 0; i < 2 * NT; ++i) {
+                            const int m = 8 * (i >> 1) + 2 * qt + (i & 1);
+                            bvs[warp * 8 * NT + m] = best_v[i];
+                            bis[warp * 8 * NT + m] = best_i[i];
+                        }
                     }
                     consumer_sync();
                     if (tid < M) {
                         float bv = -INFINITY;
                         int bi = 0x7fffffff;
-                        for (int th = 0; th < kMThreads; ++th) {
-                            for (int i = 0; i < 2 * NT; ++i) {
-                                int tm;
-                                if (g.wk > 1) {
-                                    if (i != 0) continue;
-                                    tm = th % (8 * NT);
-                                } else {
-                                    tm = 8 * (i >> 1) + 2 * (th & 3) + (i & 1);
-                                }
-                                if (tm == tid && better(bvs[th * 2 * NT + i], bis[th * 2 * NT + i], bv, bi)) {
-                                    bv = bvs[th * 2 * NT + i];
-                                    bi = bis[th * 2 * NT + i];
-                                }
+                        for (int w = 0; w < kMW; ++w) {
+                            if (better(bvs[w * 8 * NT + tid], bis[w * 8 * NT + tid], bv, bi)) {
+                                bv = bvs[w * 8 * NT + tid];
+                                bi = bis[w * 8 * NT + tid];
                             }
                         }
                         P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
