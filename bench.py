@@ -298,6 +298,44 @@ def build_pass(args, device, model: str = "phi3"):
     return calls, xbuf, ybuf
 
 
+def batched_pass_results(seed: int, device, calls, stream, Ms, steps: int, hbm_peak: float):
+    """Batched decode: the same pass (the weights of `calls`) with M tokens per projection -- x [M][K]
+    ~ N(0,1) fp16, outputs [M][N] -- one zt_q4_pass call, each between its own events.  Returns per M
+    (us per pass, GB/s of algorithmic bytes, fraction of the measured copy)."""
+    import torch
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    gen = torch.Generator(device=device).manual_seed(seed)
+    out = []
+    for M in Ms:
+        projs, nbytes = [], 0
+        for d in calls:
+            p = d["p"]
+            e = {"kind": p.kind, "qw": d["qw"], "scales": d["s"],
+                 "x": torch.randn((M, p.K), generator=gen, device=device).half(),
+                 "out": torch.empty((M, p.n_out), dtype=torch.float32 if p.kind == "lm_head" else torch.float16,
+                                    device=device)}
+            if p.kind == "lm_head":
+                e["argmax"] = torch.empty((M,), dtype=torch.int32, device=device)
+            projs.append(e)
+            nbytes += alg_bytes(p, M)
+        zp = zt_q4.Pass(projs)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                zp.run(stream)
+            for a_, b_ in ev:
+                a_.record(stream)
+                zp.run(stream)
+                b_.record(stream)
+            stream.synchronize()
+        assert zp.errors() == 0, "a bounded wait of the pass kernel expired"
+        us = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ev) * 1e3
+        out.append({"M": M, "us": round(us, 2), "GBps": round(nbytes / us / 1e3, 1),
+                    "frac": round(nbytes / us / 1e3 / hbm_peak, 4), "bytes": nbytes})
+        del zp, projs
+    return out
+
+
 def launch(zt_q4, d, stream):
     p = d["p"]
     if p.kind == "gemv":
@@ -681,6 +719,8 @@ def run_ours(args, world, rank, local):
     # ---- config 3 (small batch) and the batched prefill, at modest step counts ----
     sweep = sweep_m_results(args.seed, device, stream, max(64, min(args.steps, 200)), 3,
                             float(measured_peaks().get("hbm_gbs", 6650.0)))
+    batched = batched_pass_results(args.seed, device, calls, stream, (2, 4, 8, 16), max(10, min(args.steps, 50)),
+                                   float(measured_peaks().get("hbm_gbs", 6650.0)))
     pre_rows, _, _ = prefill_results(args.seed, device, stream, [512, 2048], max(16, min(args.steps, 100)), 3)
     torch.cuda.empty_cache()
 
@@ -761,7 +801,11 @@ def run_ours(args, world, rank, local):
                              "bytes_per_pass": lbytes, "chained_us_per_pass": round(l_chain_us, 2),
                              "steps": l_steps, "kernel": "q4_pass_kernel + argmax reduction, one zt_q4_pass call",
                              "duration": "mean of event-bracketed zt_q4_pass calls"},
-            "small_batch": sweep_summary(sweep),
+            "small_batch": {**sweep_summary(sweep),
+                            "pass": {"workload": "the Phi-3-mini decode weight pass (129 projections, one zt_q4_pass "
+                                                 "call) with M tokens per projection",
+                                     "M": [b["M"] for b in batched], "us_per_pass": [b["us"] for b in batched],
+                                     "GBps": [b["GBps"] for b in batched], "frac": [b["frac"] for b in batched]}},
             "prefill": {"workload": "Phi-3-mini qkv 3072->9216 (dequant + tcgen05 GEMM) and gate_up 3072->2x8192 "
                                     "+SiLU (cached binary16 weights), q4 group-32",
                         "tokens": {str(r["M"]): {k: v for k, v in r.items() if k != "M"} for r in pre_rows},
