@@ -82,6 +82,8 @@ struct PassArgs {
     unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
     int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
+    int colsplit;               // M > 8 as two column blocks: CTAs 2s and 2s + 1 take row share s, tokens
+                                // 0 .. ceil(M/2) - 1 and the rest (each an M <= 8 problem of 5..8 tokens)
     PassProj p[PMAX];
 };
 
@@ -255,7 +257,15 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     static_assert(!ONE || NT == 1, "one column fits one n-tile");
     extern __shared__ __align__(1024) unsigned char smem[];
-    const int M = a.M, n = a.n;
+    // this CTA's tokens (columns) and row share: with the column split, tokens m0 .. m0 + M - 1
+    // of the list's Mt (the first ceil(Mt / 2) or the other floor(Mt / 2), so never a single
+    // column: the staging helpers take M == 1 for the block-diagonal layout of ONE), and
+    // share sb of nsb (two CTAs per share)
+    const int Mt = a.M, n = a.n;
+    const int cb = a.colsplit ? (int)(blockIdx.x & 1) : 0, m0 = cb * ((Mt + 1) >> 1);
+    const int M = a.colsplit ? (cb ? Mt >> 1 : (Mt + 1) >> 1) : Mt;
+    const int sb = a.colsplit ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nsb = a.colsplit ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int qg = lane >> 2, qt = lane & 3;       // mma quad row / thread in quad
 
@@ -287,8 +297,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         bool has = false;
         if (tid < n) {
             const PassProj &P = a.p[tid];
-            const long long lo = P.phase_bytes * blockIdx.x / gridDim.x;
-            const long long hi = P.phase_bytes * (blockIdx.x + 1) / gridDim.x;
+            const long long lo = P.phase_bytes * sb / nsb;
+            const long long hi = P.phase_bytes * (sb + 1) / nsb;
             const long long rb = P.row_bytes, end = P.base + (long long)P.N * rb;
             if (hi > P.base && lo < end) {
                 const int o0 = lo > P.base ? (int)((lo - P.base + rb - 1) / rb) : 0;
@@ -421,9 +431,9 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         // written only after the wait: the kernel ahead on the stream may be
         // the argmax reduction of an earlier call that reads the same scratch
         const PassProj &P = a.p[tid];
-        for (int m = 0; m < M; ++m) {
-            P.ws_val[(size_t)blockIdx.x * M + m] = -INFINITY;
-            pass_ws_idx(P, M)[(size_t)blockIdx.x * M + m] = 0x7fffffff;
+        for (int m = 0; m < Mt; ++m) {
+            P.ws_val[(size_t)blockIdx.x * Mt + m] = -INFINITY;
+            pass_ws_idx(P, Mt)[(size_t)blockIdx.x * Mt + m] = 0x7fffffff;
         }
     }
 
@@ -461,20 +471,29 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
             const PassGeo g = pass_geo(sgm, warp);
             const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d, gsh = P.gsh;
             const bool sasync = P.scales_async;
-            void *const out = P.out;
-            const bool writer = sgm.o_begin == 0;   // exactly one CTA holds row 0
+            // this CTA's tokens m0 .. m0 + M - 1 of the [Mt][K] inputs and [Mt][ldo] outputs
+            const size_t xo = (size_t)m0 * P.K;
+            const __half *const px = P.x ? P.x + xo : nullptr;
+            const __half *const pres = P.res ? P.res + xo : nullptr;
+            const __half *const pdlt = P.dlt ? P.dlt + xo : nullptr;
+            __half *const pres_out = P.res_out ? P.res_out + xo : nullptr;
+            __half *const px_out = P.x_out ? P.x_out + xo : nullptr;
+            const int *const ppos = P.pos ? P.pos + m0 : nullptr;
+            void *const out = kind == kEpiLogits ? (void *)(reinterpret_cast<float *>(P.out) + (size_t)m0 * ldo)
+                                                 : (void *)(reinterpret_cast<__half *>(P.out) + (size_t)m0 * ldo);
+            const bool writer = sgm.o_begin == 0;   // the CTA (of each column block) holding row 0
             // windowed: the segment's activations exceed the staging area (WIN kernels only)
             const bool windowed = WIN && G > a.g_stage;
             if (!windowed) {
                 if (P.norm) {
-                    stage_x_norm(P.res, P.dlt, P.gamma, P.eps, writer ? P.res_out : nullptr,
-                                 writer ? P.x_out : nullptr, xp, x7, red, M, P.K, G, NT);
+                    stage_x_norm(pres, pdlt, P.gamma, P.eps, writer ? pres_out : nullptr,
+                                 writer ? px_out : nullptr, xp, x7, red, M, P.K, G, NT);
                 } else {
-                    stage_x_mma(P.x, P.K, xp, x7, M, G, G, NT);
+                    stage_x_mma(px, P.K, xp, x7, M, G, G, NT);
                 }
                 consumer_sync();
             } else if (P.norm) {
-                norm_rows(P.res, P.dlt, P.eps, writer ? P.res_out : nullptr, rn, red, M, P.K);
+                norm_rows(pres, pdlt, P.eps, writer ? pres_out : nullptr, rn, red, M, P.K);
             }
 
             const int gs = windowed ? a.g_stage : G;   // groups per staged activation column
@@ -518,7 +537,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     } else if (kind == kEpiF16) {
                         reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
                     } else if (kind == kEpiRope) {
-                        rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta, P.pos[m],
+                        rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta, ppos[m],
                                    y, u * pow2f(24));
                     } else {
                         u *= pow2f(24);
@@ -564,10 +583,10 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                             consumer_sync();
                             const int g0 = w * gs, gn = min(gs, G - g0);
                             if (P.norm)
-                                stage_x_norm_window(P.res, P.dlt, P.gamma, (writer && tl == 0) ? P.x_out : nullptr,
+                                stage_x_norm_window(pres, pdlt, P.gamma, (writer && tl == 0) ? px_out : nullptr,
                                                     rn, xp, x7, M, P.K, g0, gn, gs, NT);
                             else
-                                stage_x_mma(P.x + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT);
+                                stage_x_mma(px + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT);
                             consumer_sync();
                             if (w > 0) {   // the area now starts at group w gs
                                 xoff -= (uint32_t)gs * XG;
@@ -784,7 +803,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                                     const int nn = o0 + qg;
                                     if (nn < g.o_end)
                                         rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta,
-                                                   P.pos[m], acc[nt][e] * pow2f(24), acc[nt][2 + e] * pow2f(24));
+                                                   ppos[m], acc[nt][e] * pow2f(24), acc[nt][2 + e] * pow2f(24));
                                 } else {
 #pragma unroll
                                     for (int h = 0; h < 2; ++h) {
@@ -866,8 +885,13 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                                 bi = bis[w * 8 * NT + tid];
                             }
                         }
-                        P.ws_val[(size_t)blockIdx.x * M + tid] = bv;
-                        pass_ws_idx(P, M)[(size_t)blockIdx.x * M + tid] = bi;
+                        P.ws_val[(size_t)blockIdx.x * Mt + m0 + tid] = bv;
+                        pass_ws_idx(P, Mt)[(size_t)blockIdx.x * Mt + m0 + tid] = bi;
+                    } else if (tid < Mt) {
+                        // the Mt - M tokens of the other column block: a neutral partial maximum
+                        const int m = (m0 + tid) % Mt;
+                        P.ws_val[(size_t)blockIdx.x * Mt + m] = -INFINITY;
+                        pass_ws_idx(P, Mt)[(size_t)blockIdx.x * Mt + m] = 0x7fffffff;
                     }
                 }
             };

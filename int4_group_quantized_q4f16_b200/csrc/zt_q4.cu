@@ -160,6 +160,13 @@ PassPlan pass_plan(int M, int g_max, int n, int NT)
     return PassPlan{0, 0, 0, false};
 }
 
+// M > 8 runs as two column blocks of ceil(M/2) and floor(M/2) tokens (the
+// kernel's colsplit) when the list's longest K would not fit whole at 16
+// columns: each CTA of a pair then stages its <= 8 columns whole (or in
+// windows twice as long), instead of restaging 16 columns per K window.  The
+// pair shares its rows' weights, the second read of them coming from L2.
+bool pass_colsplit(int M, int g_max, int n) { return M > 8 && pass_plan(M, g_max, n, 2).win; }
+
 // Launch the tensor-core pass kernel over a.p[0 .. a.n).  `cooperative`:
 // some projection waits on earlier ones (all CTAs must be co-resident).
 constexpr int kNotResident = 1;   // launch_pass_s: this shape does not reach the wanted residency
@@ -231,16 +238,24 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         rows += p.N;
     }
     for (int i = 0; i < a.n; ++i) a.p[i].phase_bytes = phase_bytes[a.p[i].phase];
-    const PassPlan plan = pass_plan(a.M, g_max, a.n, NT);
+    const int Mc = a.colsplit ? (a.M + 1) / 2 : a.M;   // columns one CTA stages at most
+    const PassPlan plan = pass_plan(Mc, g_max, a.n, NT);
     if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
     a.g_stage = plan.g_stage;
-    const size_t smem = pass_smem_bytes(a.M, plan.g_stage, plan.stages, a.n, NT);
+    const size_t smem = pass_smem_bytes(Mc, plan.g_stage, plan.stages, a.n, NT);
     // the planned CTAs per SM, or one if the device holds fewer at this shared memory size
+    // (with the column split, an even grid: CTAs 2s and 2s + 1 take the same rows)
+    const long long per_row = a.colsplit ? 2 : 1;
     for (int cps = plan.cps; cps >= 1; --cps) {
-        const int grid = (int)std::max<long long>(
-            1, std::min<long long>({(long long)sms * cps, cooperative ? (long long)sms * cps : rows, kMaxCtas}));
-        const int rc = plan.win ? launch_pass_w<NT, PMAX, ONE, true>(a, cooperative, st, grid, smem, cps, plan.stages)
-                                : launch_pass_w<NT, PMAX, ONE, false>(a, cooperative, st, grid, smem, cps, plan.stages);
+        long long g = std::min<long long>({(long long)sms * cps, cooperative ? (long long)sms * cps : rows * per_row,
+                                           kMaxCtas});
+        if (a.colsplit) g &= ~1LL;
+        const int grid = (int)std::max<long long>(per_row, g);
+        int rc = ZT_ERR_UNSUPPORTED;
+        if (!plan.win)
+            rc = launch_pass_w<NT, PMAX, ONE, false>(a, cooperative, st, grid, smem, cps, plan.stages);
+        else if constexpr (NT == 1)   // 16 columns that would need windows run as two column blocks instead
+            rc = launch_pass_w<NT, PMAX, ONE, true>(a, cooperative, st, grid, smem, cps, plan.stages);
         if (rc == kNotResident) continue;
         if (rc == ZT_OK && grid_out) *grid_out = grid;
         return rc;
@@ -258,6 +273,7 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     PassArgs<1> a;
     a.n = 1;
     a.M = M;
+    a.colsplit = pass_colsplit(M, K / kGroup, 1) ? 1 : 0;
     a.counters = nullptr;
     a.error = nullptr;
     a.withhold = -1;
@@ -284,7 +300,8 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     p.gsh = 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (M == 1) return launch_pass<1, 1, true>(a, false, st, grid_out);
-    return (M <= 8) ? launch_pass<1, 1, false>(a, false, st, grid_out) : launch_pass<2, 1, false>(a, false, st, grid_out);
+    return (M <= 8 || a.colsplit) ? launch_pass<1, 1, false>(a, false, st, grid_out)
+                                  : launch_pass<2, 1, false>(a, false, st, grid_out);
 }
 
 size_t lmhead_ws_bytes(int M) { return (size_t)kMaxCtas * M * (sizeof(float) + sizeof(int)); }
@@ -556,7 +573,7 @@ int read_error_word(const void *p, unsigned int *out)
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 3; }
+int zt_q4_version(void) { return (1 << 16) | 4; }
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -768,10 +785,13 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
         (void)cudaGetLastError();
         return ZT_ERR_LAUNCH;
     }
+    int g_max = 0;
+    for (int i = 0; i < n; ++i) g_max = std::max(g_max, projs[i].K / kGroup);
+    a.colsplit = pass_colsplit(M, g_max, n) ? 1 : 0;
     int grid = 0;
-    const int rc = M == 1   ? launch_pass<1, kPassMax, true>(a, cooperative, st, &grid)
-                   : M <= 8 ? launch_pass<1, kPassMax, false>(a, cooperative, st, &grid)
-                            : launch_pass<2, kPassMax, false>(a, cooperative, st, &grid);
+    const int rc = M == 1                   ? launch_pass<1, kPassMax, true>(a, cooperative, st, &grid)
+                   : (M <= 8 || a.colsplit) ? launch_pass<1, kPassMax, false>(a, cooperative, st, &grid)
+                                            : launch_pass<2, kPassMax, false>(a, cooperative, st, &grid);
     if (rc) return rc;
     for (int i = 0; i < n; ++i) {
         if (projs[i].kind != ZT_Q4_LM_HEAD) continue;
@@ -795,15 +815,17 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
     return ZT_OK;
 }
 
-int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window)
+int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window, int *column_blocks)
 {
-    if (!ctas_per_sm || !stages || !k_window) return ZT_ERR_INVALID_ARG;
+    if (!ctas_per_sm || !stages || !k_window || !column_blocks) return ZT_ERR_INVALID_ARG;
     if (M < 1 || M > 16 || n < 1 || n > ZT_Q4_PASS_MAX || K_max < kGroup || K_max % kGroup) return ZT_ERR_INVALID_ARG;
-    const PassPlan plan = pass_plan(M, K_max / kGroup, n, M <= 8 ? 1 : 2);
+    const bool split = pass_colsplit(M, K_max / kGroup, n);
+    const PassPlan plan = pass_plan(split ? (M + 1) / 2 : M, K_max / kGroup, n, (M <= 8 || split) ? 1 : 2);
     if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
     *ctas_per_sm = plan.cps;
     *stages = plan.stages;
     *k_window = plan.win ? plan.g_stage * kGroup : 0;
+    *column_blocks = split ? 2 : 1;
     return ZT_OK;
 }
 

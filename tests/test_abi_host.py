@@ -327,25 +327,34 @@ def test_gemm_grid_limit_rejected_before_launch(zt):
 def test_decode_plan_covers_every_small_batch_shape(zt):
     """Every decode shape with M <= 16 has a plan, from the shapes alone: the
     activations are staged whole while they fit in shared memory, and in K
-    windows (multiples of one 256-k item) beyond.  No device is touched."""
+    windows (multiples of one 256-k item) beyond; more than 8 tokens that
+    would need windows run as two column blocks.  No device is touched."""
     for M in range(1, 17):
         for K in (32, 256, 1056, 3072, 4096, 8192, 11008, 12320, 16384, 40000, 65536, 131072, 1 << 20):
             for n in (1, 4, 129, 192):
-                cps, stages, kw = zt.pass_plan(M, K, n)
+                cps, stages, kw, cb = zt.pass_plan(M, K, n)
                 assert cps in (1, 2) and 2 <= stages <= 4, (M, K, n)
                 assert kw == 0 or (kw % 256 == 0 and 256 <= kw < K), (M, K, n, kw)
+                assert cb == 1 or (cb == 2 and M > 8), (M, K, n, cb)
+                if M > 8 and cb == 1:
+                    assert kw == 0, (M, K, n)   # 16 columns are never windowed
 
 
 def test_decode_plan_pins(zt):
     """Where the plan switches, on the shapes of the benchmark and its configs."""
     # the benchmark's Phi-3-mini pass at M = 1: x staged whole, two CTAs per SM, 4-deep rings
-    assert zt.pass_plan(1, 8192, 129) == (2, 4, 0)
-    # config 3 (gate_up K = 3072) at M = 16 still fits whole, one CTA per SM
-    assert zt.pass_plan(16, 3072, 1)[2] == 0
-    # Llama-7B down (K = 11008): whole at M = 4, windows from M = 8; Phi-3 down (8192) windows at M = 12
+    assert zt.pass_plan(1, 8192, 129) == (2, 4, 0, 1)
+    # config 3 (gate_up K = 3072) at M = 16 still fits whole, one CTA per SM, one column block
+    assert zt.pass_plan(16, 3072, 1) == (1, 4, 0, 1)
+    # Llama-7B down (K = 11008): whole at M = 4, windows from M = 8, and two column blocks
+    # of windows at M = 16
     assert zt.pass_plan(4, 11008, 1)[2] == 0
-    assert zt.pass_plan(8, 11008, 1)[2] > 0
-    assert zt.pass_plan(12, 8192, 1)[2] > 0 and zt.pass_plan(16, 8192, 1)[2] > 0
+    assert zt.pass_plan(8, 11008, 1)[2:] == (2816, 1)
+    assert zt.pass_plan(16, 11008, 1)[2:] == (2816, 2)
+    # Phi-3 down (8192): 16 columns fit whole up to M = 9; at M = 12 and 16 two column
+    # blocks of at most 8 tokens, each whole
+    assert zt.pass_plan(9, 8192, 1)[2:] == (0, 1)
+    assert zt.pass_plan(12, 8192, 1)[2:] == (0, 2) and zt.pass_plan(16, 8192, 129)[2:] == (0, 2)
     # single token: whole up to K = 65536, windows beyond
     assert zt.pass_plan(1, 65536, 1)[2] == 0
     assert zt.pass_plan(1, 131072, 1)[2] > 0
@@ -356,9 +365,9 @@ def test_decode_plan_pins(zt):
 def test_decode_plan_rejects_bad_shapes(zt):
     c = ctypes.c_int(0)
     for M, K, n in ((0, 256, 1), (17, 256, 1), (1, 16, 1), (1, 100, 1), (1, 256, 0), (1, 256, 193)):
-        assert zt.lib.zt_q4_pass_plan(M, K, n, ctypes.byref(c), ctypes.byref(c), ctypes.byref(c)) == \
-            zt.ZT_ERR_INVALID_ARG
-    assert zt.lib.zt_q4_pass_plan(1, 256, 1, None, ctypes.byref(c), ctypes.byref(c)) == zt.ZT_ERR_INVALID_ARG
+        assert zt.lib.zt_q4_pass_plan(M, K, n, *[ctypes.byref(c)] * 4) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_pass_plan(1, 256, 1, None, *[ctypes.byref(c)] * 3) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_pass_plan(1, 256, 1, *[ctypes.byref(c)] * 3, None) == zt.ZT_ERR_INVALID_ARG
 
 
 def test_noalloc_misaligned_rejected_without_cuda(zt):

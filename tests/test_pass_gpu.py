@@ -177,12 +177,31 @@ def test_pass_batch_sweep(zt, oracle, M):
         _check_against_oracle(oracle, d)
 
 
-@pytest.mark.parametrize("N", [1, 3, 17])
-def test_pass_fewer_rows_than_ctas(zt, oracle, N):
-    """A list smaller than the grid: CTAs without rows still write neutral
-    LM-head partial maxima."""
+@pytest.mark.parametrize("M,K", [(10, 8192), (16, 11008)])
+def test_pass_column_split_mixed(zt, oracle, M, K):
+    """More than 8 tokens with a long K in the list: every projection runs as
+    two column blocks (ceil(M/2) tokens and the rest) sharing each row share, the LM
+    head's per-CTA maxima of both blocks meeting in one reduction."""
     import torch
-    projs = [_proj("gemv", N, 256, 1, 600 + N, 0), _proj("lm_head", N, 256, 1, 601 + N, 1)]
+    assert zt.pass_plan(M, K, 5)[3] == 2
+    shapes = [("gemv", 300, 1024), ("gate_up", 200, 1024), ("lm_head", 777, 512), ("gemv", 64, K),
+              ("lm_head", 1500, K)]
+    projs = [_proj(k, N, KK, M, 540 + i, i) for i, (k, N, KK) in enumerate(shapes)]
+    p = zt.Pass(projs)
+    p.run()
+    torch.cuda.synchronize()
+    assert p.errors() == 0
+    for d in projs:
+        _check_against_oracle(oracle, d)
+
+
+@pytest.mark.parametrize("N,M,K", [(1, 1, 256), (3, 1, 256), (17, 1, 256), (1, 12, 8192), (3, 16, 11008),
+                                   (17, 9, 12288)])
+def test_pass_fewer_rows_than_ctas(zt, oracle, N, M, K):
+    """A list smaller than the grid: CTAs without rows still write neutral
+    LM-head partial maxima (with the column split, for both blocks' tokens)."""
+    import torch
+    projs = [_proj("gemv", N, K, M, 600 + N, 0), _proj("lm_head", N, K, M, 601 + N, 1)]
     p = zt.Pass(projs)
     p.run()
     torch.cuda.synchronize()

@@ -1,15 +1,18 @@
 """GPU parity of the decode kernel at small batch (M = 2..16) on full-size
-shapes, and of its K-windowed staging: projections whose activations do not
-fit in shared memory whole (M x K x 2 bytes beyond ~190 KiB, e.g. the Phi-3
-down projection 8192 -> 3072 from M = 12, Llama-7B's 11008 -> 4096 from
-M = 8) stage them in K windows (Zero-TVM write-up, sections "完整的推理流水线"
-and "内核融合": the int4 dequantizing products of the decoder layer and the
-fused FFN, here with several tokens per call).
+shapes, of its K-windowed staging and of its column split: activations that
+do not fit in shared memory whole (M x K x 2 bytes beyond ~190 KiB) are
+staged in K windows (Llama-7B's down projection 11008 -> 4096 at M = 8), and
+more than 8 tokens that would need windows run as two CTAs per row share,
+the first ceil(M/2) tokens and the rest (Phi-3 down 8192 -> 3072 at M = 12
+and 16: each block whole; Llama-7B down at M = 16: each block in windows)
+(Zero-TVM write-up,
+sections "完整的推理流水线" and "内核融合": the int4 dequantizing products of
+the decoder layer and the fused FFN, here with several tokens per call).
 
 Every output of the full-size calls is compared with the float64 oracle, so
 each CTA's first and last tile is covered whatever the grid; larger cases
-check densely sampled rows.  zt_q4_pass_plan confirms that each windowed case
-really takes the windowed path."""
+check densely sampled rows.  zt_q4_pass_plan confirms the path each case
+takes."""
 import os
 
 import numpy as np
@@ -44,6 +47,10 @@ def _windowed(zt, M, K, n=1):
     return zt.pass_plan(M, K, n)[2] > 0
 
 
+def _split(zt, M, K, n=1):
+    return zt.pass_plan(M, K, n)[3] == 2
+
+
 # ---------------------------------------------- config 3: gate_up at M > 1 --
 @pytest.mark.parametrize("M", [2, 4, 8, 16])
 def test_gate_up_full_size_small_batch(zt, oracle, M):
@@ -57,11 +64,14 @@ def test_gate_up_full_size_small_batch(zt, oracle, M):
 
 
 # ------------------------------------- down projections past whole-K staging --
-@pytest.mark.parametrize("M,N,K", [(12, 3072, 8192), (16, 3072, 8192), (8, 4096, 11008), (16, 4096, 11008)])
-def test_down_full_size_windowed(zt, oracle, M, N, K):
-    """Phi-3 down (8192 -> 3072) at M = 12, 16 and Llama-7B down (11008 ->
-    4096) at M = 8, 16: K windows, every output."""
-    assert _windowed(zt, M, K)
+@pytest.mark.parametrize("M,N,K,win,split", [(12, 3072, 8192, False, True), (16, 3072, 8192, False, True),
+                                             (9, 3072, 8192, False, False), (8, 4096, 11008, True, False),
+                                             (16, 4096, 11008, True, True)])
+def test_down_full_size_beyond_whole(zt, oracle, M, N, K, win, split):
+    """Phi-3 down (8192 -> 3072) at M = 9 (16 columns whole), 12 and 16 (two
+    column blocks, each whole) and Llama-7B down (11008 -> 4096) at M = 8 (K
+    windows) and 16 (two column blocks of windows): every output."""
+    assert (_windowed(zt, M, K), _split(zt, M, K)) == (win, split)
     qw, s, x = synth.problem(400 + M + K, N, K, M=M, proj=synth.PROJ_DOWN)
     got = host(zt.gemv(dev(qw), dev(s), dev(x)))
     ref = oracle.gemv(qw, s, x, threads=THREADS)
@@ -76,11 +86,12 @@ def test_down_m4_whole_k(zt, oracle):
     assert_f16_matches(got, oracle.gemv(qw, s, x, threads=THREADS), "down M4", abs_products(oracle, qw, s, x))
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 1000, 16384), (16, 64, 16384), (9, 333, 12320), (5, 96, 40000)])
+@pytest.mark.parametrize("M,N,K", [(16, 1000, 16384), (16, 64, 16384), (9, 333, 20000), (5, 96, 40000)])
 def test_windowed_ragged(zt, oracle, M, N, K):
     """K = 16384 at M = 16 (the last window ragged), few rows per CTA (K split
     over up to 8 warps inside each window), K not a multiple of 256 (a
-    partial last chunk inside the last window)."""
+    partial last chunk inside the last window; at M = 9 in blocks of 5 + 4
+    tokens)."""
     assert _windowed(zt, M, K)
     qw, s, x = synth.problem(500 + N, N, K, M=M, proj=0)
     got = host(zt.gemv(dev(qw), dev(s), dev(x)))
@@ -111,10 +122,12 @@ def test_windowed_gate_up(zt, oracle):
     assert_f16_matches(got[:, rows], ref, "windowed gate_up", gate_up_bound(oracle, qw, s, x, rows))
 
 
-@pytest.mark.parametrize("M,N,K", [(16, 6000, 8192), (8, 2500, 11008)])
+@pytest.mark.parametrize("M,N,K", [(16, 6000, 8192), (8, 2500, 11008), (15, 2500, 11008), (9, 3001, 11008)])
 def test_windowed_lm_head(zt, oracle, M, N, K):
-    """f32 logits and argmax through windows: every logit, every argmax."""
-    assert _windowed(zt, M, K)
+    """f32 logits and argmax through windows and column blocks (M = 15, 9:
+    blocks of 8 + 7 tokens in windows, 5 + 4 whole; the per-CTA maxima of
+    both blocks meet in one reduction): every logit, every argmax."""
+    assert _windowed(zt, M, K) or _split(zt, M, K)
     qw, s, x = synth.problem(700 + M, N, K, M=M, proj=synth.PROJ_LM_HEAD)
     logits, am = zt.lmhead_argmax(dev(qw), dev(s), dev(x))
     ref, _ = oracle.lmhead_argmax(qw, s, x, threads=THREADS)
@@ -152,13 +165,15 @@ def _norm_inputs(seed, M, K):
     return res, dlt, gamma
 
 
-def test_windowed_norm_prologue(zt, oracle):
-    """Residual add + RMSNorm ahead of a windowed projection (M = 16, K = 8192):
+@pytest.mark.parametrize("M,K", [(16, 8192), (15, 11008)])
+def test_windowed_norm_prologue(zt, oracle, M, K):
+    """Residual add + RMSNorm ahead of a column-split projection (M = 16,
+    K = 8192: each block whole; M = 15, K = 11008: each block in windows):
     h bit-exact, x within one fp16 ulp of the oracle, y against the oracle on
     the kernel's own x; a second call is bit-identical."""
     import torch
-    M, N, K = 16, 1500, 8192
-    assert _windowed(zt, M, K)
+    N = 1500
+    assert _split(zt, M, K)
     qw, s, _ = synth.problem(1001, N, K, M=M, proj=3)
     res, dlt, gamma = _norm_inputs(1001, M, K)
     nm = {"residual": dev(res), "delta": dev(dlt), "gamma": dev(gamma), "eps": EPS}
@@ -183,11 +198,13 @@ def test_windowed_norm_prologue(zt, oracle):
     assert np.array_equal(got.view(np.uint16), host(out).view(np.uint16))
 
 
-def test_windowed_rope_epilogue(zt, oracle):
-    """RoPE on a windowed projection (M = 16, K = 8192, head_dim 128)."""
+@pytest.mark.parametrize("M,K", [(16, 8192), (15, 11008)])
+def test_windowed_rope_epilogue(zt, oracle, M, K):
+    """RoPE on a column-split projection (head_dim 128; each token's own
+    position in both blocks), whole and windowed."""
     import torch
-    M, N, K, d = 16, 1024, 8192, 128
-    assert _windowed(zt, M, K)
+    N, d = 1024, 128
+    assert _split(zt, M, K)
     qw, s, x = synth.problem(1101, N, K, M=M, proj=0)
     pos = np.random.default_rng(5).integers(0, 4096, M).astype(np.int32)
     out = torch.empty((M, N), dtype=torch.float16, device="cuda")
