@@ -52,13 +52,10 @@ struct PassProj {
     // RoPE epilogue (kind kEpiRope): pairs (i, i + d/2) of each head of d rows
     // turned by pos[m] * theta^(-2i/d); N counts pairs
     const int *pos;
-    long long base;             // byte offset of the projection's rows within its phase
-    long long phase_bytes;      // HBM bytes of the whole phase
     int N, K, G, kind;          // kind: kEpiF16 / kEpiGateUp / kEpiLogits / kEpiRope (N: outputs, pairs for RoPE)
     int ldo;                    // elements between output rows
     int row_bytes;              // HBM bytes per output (codes + scales of its weight rows)
     int scales_async;           // scales copied by cp.async (16-byte aligned rows)
-    int phase;                  // index of the projection's phase
     int wait;                   // starts a phase: wait for all earlier projections
     int norm;
     int rope_d;
@@ -84,6 +81,13 @@ struct PassArgs {
     int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
     int colsplit;               // M > 8 as two column blocks: CTAs 2s and 2s + 1 take row share s, tokens
                                 // 0 .. ceil(M/2) - 1 and the rest (each an M <= 8 problem of 5..8 tokens)
+    // What every CTA reads to find its rows, kept apart from p[] in dense arrays: a warp
+    // reading one entry per lane then touches a few consecutive constant-cache lines,
+    // not one line per lane.
+    long long pbeg[PMAX + 1];   // HBM byte offset of projection i's rows in the list; pbeg[n]: the total
+    long long phbeg[PMAX + 1];  // HBM byte offset where phase i starts; phbeg[phases]: the total
+    int pphase[PMAX];           // phase of projection i
+    unsigned lm_bits[(PMAX + 31) / 32];   // bit i: projection i is an LM head
     PassProj p[PMAX];
 };
 
@@ -296,26 +300,28 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         PassSeg mine{};
         bool has = false;
         if (tid < n) {
-            const PassProj &P = a.p[tid];
-            const long long lo = P.phase_bytes * sb / nsb;
-            const long long hi = P.phase_bytes * (sb + 1) / nsb;
-            const long long rb = P.row_bytes, end = P.base + (long long)P.N * rb;
-            if (hi > P.base && lo < end) {
-                const int o0 = lo > P.base ? (int)((lo - P.base + rb - 1) / rb) : 0;
-                const int o1 = hi < end ? (int)((hi - P.base + rb - 1) / rb) : P.N;
+            const int ph = a.pphase[tid];
+            const long long s0 = a.phbeg[ph], len = a.phbeg[ph + 1] - s0;
+            const long long lo = s0 + len * sb / nsb, hi = s0 + len * (sb + 1) / nsb;
+            const long long beg = a.pbeg[tid], end = a.pbeg[tid + 1];
+            if (hi > beg && lo < end) {
+                const PassProj &P = a.p[tid];
+                const long long rb = P.row_bytes;
+                const int o0 = lo > beg ? (int)((lo - beg + rb - 1) / rb) : 0;
+                const int o1 = hi < end ? (int)((hi - beg + rb - 1) / rb) : P.N;
                 if (o1 > o0) {
                     has = true;
                     mine.p = tid;
                     mine.o_begin = o0;
                     mine.o_end = o1;
-                    mine.phase = P.phase;
+                    mine.phase = ph;
                     mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
                     mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
                 }
             }
-            neutral_max = !has && P.kind == kEpiLogits;
+            neutral_max = !has && ((a.lm_bits[tid >> 5] >> (tid & 31)) & 1u);
         }
         const unsigned ball = __ballot_sync(0xffffffffu, has);
         if (lane == 0) wcount[warp] = __popc(ball);

@@ -226,18 +226,21 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
     // Phases: a new one at every projection that waits.  Each CTA takes a
     // byte-balanced share of each phase's concatenated rows.
     long long rows = 0;      // a CTA with no rows of a list without waits would only idle
-    long long phase_bytes[kPassMax];
+    long long off = 0;       // HBM bytes of the projections so far
     a.phases = 0;
+    for (int w = 0; w < (PMAX + 31) / 32; ++w) a.lm_bits[w] = 0;
     for (int i = 0; i < a.n; ++i) {
         PassProj &p = a.p[i];
-        if (i == 0 || p.wait) phase_bytes[a.phases++] = 0;
-        p.phase = a.phases - 1;
+        if (i == 0 || p.wait) a.phbeg[a.phases++] = off;
+        a.pphase[i] = a.phases - 1;
         p.row_bytes = (p.K / 2 + (p.K / 16 >> p.gsh)) * ((p.kind == kEpiGateUp || p.kind == kEpiRope) ? 2 : 1);
-        p.base = phase_bytes[p.phase];
-        phase_bytes[p.phase] += (long long)p.N * p.row_bytes;
+        a.pbeg[i] = off;
+        off += (long long)p.N * p.row_bytes;
         rows += p.N;
+        if (p.kind == kEpiLogits) a.lm_bits[i >> 5] |= 1u << (i & 31);
     }
-    for (int i = 0; i < a.n; ++i) a.p[i].phase_bytes = phase_bytes[a.p[i].phase];
+    a.pbeg[a.n] = off;
+    a.phbeg[a.phases] = off;
     const int Mc = a.colsplit ? (a.M + 1) / 2 : a.M;   // columns one CTA stages at most
     const PassPlan plan = pass_plan(Mc, g_max, a.n, NT);
     if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
