@@ -254,7 +254,8 @@ ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, si
  * it), from the shapes alone -- no device is touched, nothing is launched:
  * M tokens (1..16), K_max the largest K of the list (a multiple of 32), n the
  * number of projections (1 for a single call).  Writes the CTAs resident per SM
- * (1 or 2), the ring depth in weight items per warp (2..4), k_window: 0 when
+ * (1 or 2) and their warps (warps_per_cta: 16 with one CTA per SM, else 8),
+ * the ring depth in weight items per warp (2..4), k_window: 0 when
  * each projection's activations are staged whole in shared memory, else the
  * length in k of the windows that projections with K > k_window are staged in
  * (a multiple of 256; the CTA then walks such a projection's rows in rounds and
@@ -264,7 +265,7 @@ ZT_API int zt_q4_pass(const zt_q4_proj *projs, int n, int M, void *workspace, si
  * tokens).  Every legal shape has a plan.  Diagnostics.
  */
 ZT_API int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window,
-                           int *column_blocks);
+                           int *column_blocks, int *warps_per_cta);
 
 /* Synchronous read of a finished pass's error word (0: no bounded wait expired). */
 ZT_API int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out);
@@ -364,7 +365,8 @@ ZT_API const char *zt_q4_strerror(int status);
  */
 ZT_API const char *zt_q4_last_cuda_error(void);
 
-/* Library ABI version, (major << 16) | minor.  1.3 added zt_q4_pass_plan; 1.4 its column_blocks. */
+/* Library ABI version, (major << 16) | minor.  1.3 added zt_q4_pass_plan; 1.4 its column_blocks; 1.5 its
+ * warps_per_cta. */
 ZT_API int zt_q4_version(void);
 
 #ifdef __cplusplus

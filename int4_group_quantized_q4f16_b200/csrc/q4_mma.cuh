@@ -64,13 +64,14 @@
 
 namespace zt {
 
-constexpr int kMW = 8;                              // math (consumer) warps per CTA
-constexpr int kMThreads = kMW * 32;
+// Math warps per CTA: 16 (one CTA per SM) or 8 (one or two CTAs per SM), a
+// launch-plan choice.  The staging helpers below take the CTA's size from
+// blockDim; kMWMax sizes per-warp tables.
+constexpr int kMWMax = 16;
 
-// Barrier among the CTA's math warps (threads 0 .. kMThreads - 1) only: named
-// barrier 1, so that a copy-producer warp (if the kernel has one) need not
-// take part.  With no producer warp it is the same as __syncthreads().
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kMThreads) : "memory"); }
+// Barrier among all threads of the CTA as named barrier 1 (the same as
+// __syncthreads(), kept apart from barrier 0).
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"r"(blockDim.x) : "memory"); }
 constexpr int kMTileRows = 16;                      // weight rows per warp tile (mma M)
 constexpr int kMChunkG = 8;                         // groups per item
 // A ring stage holds an item: codes [16 rows][128 B] with the 128-byte XOR
@@ -134,7 +135,7 @@ __host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
 // zero x and C of groups [Gw, round8(Gw)) in the single-column layout
 __device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw)
 {
-    for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += kMThreads) {
+    for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += (int)blockDim.x) {
         *reinterpret_cast<uint4 *>(xp + bd_piece(Gw * 4 + j)) = make_uint4(0, 0, 0, 0);
         if ((j & 3) == 0) x7[Gw + (j >> 2)] = 0.f;
     }
@@ -209,7 +210,7 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
     // C entries of the padding columns M .. 8 NT - 1 are zero
     const bool compact = M == 1;
     const int pad = compact ? 0 : 8 * NT - M;
-    for (int j = threadIdx.x; j < Gw * pad; j += kMThreads) {
+    for (int j = threadIdx.x; j < Gw * pad; j += (int)blockDim.x) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
         float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -218,8 +219,8 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
     }
     // two rounds per iteration: both loads in flight before either is used.
     // L2-coherent loads: x may be an output of an earlier phase of the same launch.
-    for (int base = 0; base < total; base += 2 * kMThreads) {
-        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+    for (int base = 0; base < total; base += 2 * (int)blockDim.x) {
+        const int i0 = base + threadIdx.x, i1 = i0 + (int)blockDim.x;
         const bool v0 = i0 < total, v1 = i1 < total;
         const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
         const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
@@ -227,7 +228,7 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
         if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * ldx + 8 * k0));
         if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * ldx + 8 * k1));
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
     if (compact) bd_pad(xp, x7, Gw);
 }
@@ -240,7 +241,7 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
 // (fp32, fixed order: per-thread strided sums, warp butterfly, warps in
 // order); pass 2 turns each thread's own 16 bytes of h into x in the mma-B
 // order.  res_out / x_out (plain [M][K] fp16) are written when non-null.
-// scratch: kMW + M floats of shared memory.  All threads of the CTA call it.
+// scratch: kMWMax + M floats of shared memory.  All threads of the CTA call it.
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
 {
     __half2 r = __hadd2(*reinterpret_cast<const __half2 *>(&a), *reinterpret_cast<const __half2 *>(&b));
@@ -256,7 +257,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int m = 0; m < M; ++m) {
         float part = 0.f;
-        for (int kk = threadIdx.x; kk < K8; kk += kMThreads) {
+        for (int kk = threadIdx.x; kk < K8; kk += (int)blockDim.x) {
             uint4 h = __ldcg(reinterpret_cast<const uint4 *>(res + (size_t)m * K + 8 * kk));
             if (dlt) {
                 const uint4 d = __ldcg(reinterpret_cast<const uint4 *>(dlt + (size_t)m * K + 8 * kk));
@@ -281,15 +282,15 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         consumer_sync();
         if (threadIdx.x == 0) {
             float ss = 0.f;
-            for (int w = 0; w < kMW; ++w) ss += scratch[w];
-            scratch[kMW + m] = 1.0f / sqrtf(ss / (float)K + eps);
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ss += scratch[w];
+            scratch[kMWMax + m] = 1.0f / sqrtf(ss / (float)K + eps);
         }
         consumer_sync();
     }
     const int total = M * K8;
     const bool compact = M == 1;
     const int pad = compact ? 0 : 8 * NT - M;
-    for (int j = threadIdx.x; j < G * pad; j += kMThreads) {
+    for (int j = threadIdx.x; j < G * pad; j += (int)blockDim.x) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
         float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -299,7 +300,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
     auto normalise = [&](int m, int kk) {
         const uint4 h = *reinterpret_cast<const uint4 *>(xp + x_piece(m, kk, nstride, compact));
         const uint4 g = __ldcg(reinterpret_cast<const uint4 *>(gamma + 8 * kk));
-        const float r = scratch[kMW + m];
+        const float r = scratch[kMWMax + m];
         const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
         const __half2 *gg = reinterpret_cast<const __half2 *>(&g);
         uint4 x;
@@ -312,8 +313,8 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         if (x_out) *reinterpret_cast<uint4 *>(x_out + (size_t)m * K + 8 * kk) = x;
         return x;
     };
-    for (int base = 0; base < total; base += 2 * kMThreads) {
-        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+    for (int base = 0; base < total; base += 2 * (int)blockDim.x) {
+        const int i0 = base + threadIdx.x, i1 = i0 + (int)blockDim.x;
         const bool v0 = i0 < total, v1 = i1 < total;
         const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
         const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
@@ -321,7 +322,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         if (v0) r0 = normalise(m0, k0);
         if (v1) r1 = normalise(m1, k1);
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
     if (compact) bd_pad(xp, x7, G);
 }
@@ -331,7 +332,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
 // of squares over all of K once per segment, in exactly stage_x_norm's order
 // (so r is bit-identical), writes h to res_out when non-null and r[m] to rn;
 // stage_x_norm_window then stages groups [g0, g0 + Gw) of x = fp16(h r gamma),
-// recomputing h = fp16(res + dlt) for just those k.  scratch: kMW floats.
+// recomputing h = fp16(res + dlt) for just those k.  scratch: kMWMax floats.
 __device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, float eps, __half *res_out,
                                           float *rn, float *scratch, int M, int K)
 {
@@ -339,7 +340,7 @@ __device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int m = 0; m < M; ++m) {
         float part = 0.f;
-        for (int kk = threadIdx.x; kk < K8; kk += kMThreads) {
+        for (int kk = threadIdx.x; kk < K8; kk += (int)blockDim.x) {
             uint4 h = __ldcg(reinterpret_cast<const uint4 *>(res + (size_t)m * K + 8 * kk));
             if (dlt) {
                 const uint4 d = __ldcg(reinterpret_cast<const uint4 *>(dlt + (size_t)m * K + 8 * kk));
@@ -363,7 +364,7 @@ __device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, 
         consumer_sync();
         if (threadIdx.x == 0) {
             float ss = 0.f;
-            for (int w = 0; w < kMW; ++w) ss += scratch[w];
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ss += scratch[w];
             rn[m] = 1.0f / sqrtf(ss / (float)K + eps);
         }
         consumer_sync();
@@ -379,7 +380,7 @@ __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __h
     const size_t nstride = (size_t)Gs * 64 + 32;
     const bool compact = M == 1;
     const int pad = compact ? 0 : 8 * NT - M;
-    for (int j = threadIdx.x; j < Gw * pad; j += kMThreads) {
+    for (int j = threadIdx.x; j < Gw * pad; j += (int)blockDim.x) {
         const int g = j / pad, m = M + (j - (j / pad) * pad);
         const int nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
         float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -410,8 +411,8 @@ __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __h
         if (x_out) *reinterpret_cast<uint4 *>(x_out + off) = x;
         return x;
     };
-    for (int base = 0; base < total; base += 2 * kMThreads) {
-        const int i0 = base + threadIdx.x, i1 = i0 + kMThreads;
+    for (int base = 0; base < total; base += 2 * (int)blockDim.x) {
+        const int i0 = base + threadIdx.x, i1 = i0 + (int)blockDim.x;
         const bool v0 = i0 < total, v1 = i1 < total;
         const int m0 = v0 ? i0 / K8 : 0, m1 = v1 ? i1 / K8 : 0;
         const int k0 = i0 - m0 * K8, k1 = i1 - m1 * K8;
@@ -419,7 +420,7 @@ __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __h
         if (v0) r0 = normalise(m0, k0);
         if (v1) r1 = normalise(m1, k1);
         stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + kMThreads < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
     }
     if (compact) bd_pad(xp, x7, Gw);
 }

@@ -94,9 +94,9 @@ struct PassArgs {
 // WK > 1 partial buffer: (tiles x WK) warp tiles of 16 rows x 8 NT columns
 // per segment.  The LM head's per-thread maxima reuse it once a segment's
 // partial sums have been read.
-__host__ __device__ constexpr int pass_red_floats(int NT) { return 1024 * NT; }   // 4 KB per n-tile
-static_assert(kMThreads * 2 * 1 * 8 <= pass_red_floats(1) * 4, "LM-head maxima must fit the partial buffer");
-static_assert(kMThreads * 2 * 2 * 8 <= pass_red_floats(2) * 4, "LM-head maxima must fit the partial buffer");
+// 4 KB per n-tile and 8 warps.  The LM head's maxima take 2 x MW x 8 NT words.
+__host__ __device__ constexpr int pass_red_floats(int NT, int MW) { return 128 * MW * NT; }
+static_assert(2 * 8 * 8 <= pass_red_floats(1, 8), "LM-head maxima must fit the partial buffer");
 constexpr int kPassMaxStages = 4;           // ring depths 2..4 are instantiated
 
 // One projection's rows in one CTA, with the CTA's warp layout for them.
@@ -108,14 +108,14 @@ struct PassSeg {
 // Shared memory per CTA: rings, permuted activations (n-stride g_stage*64 +
 // 32 bytes), C-operand table, WK partials / LM-head maxima, segment list,
 // flags, the RMSNorm factors of a windowed segment (16 floats).
-__host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT)
+__host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT, int MW)
 {
-    const size_t ring = (size_t)kMW * stages * kMStage + 1024;   // + alignment of the code stages
+    const size_t ring = (size_t)MW * stages * kMStage + 1024;   // + alignment of the code stages
     // M = 1: the block-diagonal layout (a zero block, 80 bytes per group, one C float per group)
     const size_t xp = M == 1 ? (size_t)kBdZero + (size_t)round8(g_stage) * kBdGroup : (size_t)M * ((size_t)g_stage * 64 + 32);
     const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 4 : (size_t)g_stage * NT * 64;
-    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT) * 4 + (size_t)n * sizeof(PassSeg) +
-           (kMW + 4) * sizeof(int) + 16 * sizeof(float);
+    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT, MW) * 4 + (size_t)n * sizeof(PassSeg) +
+           (MW + 4) * sizeof(int) + 16 * sizeof(float);
 }
 
 // Per-segment geometry of one warp.
@@ -123,24 +123,25 @@ struct PassGeo {
     int o_begin, o_end, rout, n_tiles, n_chunks, wk, wr_n, my_wk, my_wr, my_tiles, my_chunks;
 };
 
-static_assert(kMW == 8, "warp layout below assumes 8 warps");
-static_assert(kPassMax <= kMThreads, "one thread per projection builds the segment list");
+static_assert(kPassMax <= 8 * 32, "one thread per projection builds the segment list");
 static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel parameter block");
 
 // log2 of the warps splitting K for a segment: minimise the items of the
 // busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
-// K-warps.  `bounded`: the whole segment's partials meet at once, so the
-// partial buffer bounds them (tiles * WK * 16 * 8 NT <= pass_red_floats); a
-// windowed segment reduces one round of at most 8 / WK tiles at a time.
+// K-warps.  LW: log2 of the CTA's warps.  `bounded`: the whole segment's
+// partials meet at once, so the partial buffer bounds them (tiles * WK * 16 *
+// 8 NT <= pass_red_floats); a windowed segment reduces one round of at most
+// (warps / WK) tiles at a time.
+template <int LW>
 __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool bounded)
 {
     int best = 0, best_cost = -1;
 #pragma unroll
-    for (int wkl = 0; wkl <= 3; ++wkl) {
+    for (int wkl = 0; wkl <= LW; ++wkl) {
         const int wk = 1 << wkl;
         if (wk > n_chunks) break;
-        if (bounded && wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT)) break;
-        const int cost = ((n_tiles + (kMW >> wkl) - 1) >> (3 - wkl)) * ((n_chunks + wk - 1) >> wkl);
+        if (bounded && wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT, 1 << LW)) break;
+        const int cost = ((n_tiles + ((1 << LW) >> wkl) - 1) >> (LW - wkl)) * ((n_chunks + wk - 1) >> wkl);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = wkl;
@@ -149,6 +150,7 @@ __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool 
     return best;
 }
 
+template <int LW>
 __device__ __forceinline__ PassGeo pass_geo(const PassSeg &sg, int warp)
 {
     PassGeo g;
@@ -158,10 +160,10 @@ __device__ __forceinline__ PassGeo pass_geo(const PassSeg &sg, int warp)
     g.n_tiles = sg.n_tiles;
     g.n_chunks = sg.n_chunks;
     g.wk = 1 << sg.wkl;
-    g.wr_n = kMW >> sg.wkl;
+    g.wr_n = (1 << LW) >> sg.wkl;
     g.my_wk = warp & (g.wk - 1);
     g.my_wr = warp >> sg.wkl;
-    g.my_tiles = g.my_wr < g.n_tiles ? (g.n_tiles - g.my_wr + g.wr_n - 1) >> (3 - sg.wkl) : 0;
+    g.my_tiles = g.my_wr < g.n_tiles ? (g.n_tiles - g.my_wr + g.wr_n - 1) >> (LW - sg.wkl) : 0;
     g.my_chunks = g.my_wk < g.n_chunks ? (g.n_chunks - g.my_wk + g.wk - 1) >> sg.wkl : 0;
     if (g.my_chunks == 0) g.my_tiles = 0;
     return g;
@@ -255,9 +257,11 @@ __device__ __noinline__ void rope_store(__half *out, size_t row_off, int pair, i
 // rounds of one tile per warp, and each round stages the windows in turn
 // while the warps' accumulators carry over (the weight stream's order is the
 // same as without windows).
-template <int NT, int PMAX, int S, bool ONE, bool WIN>
-__global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
+template <int NT, int PMAX, int S, bool ONE, bool WIN, int MW>
+__global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(const __grid_constant__ PassArgs<PMAX> a)
 {
+    static_assert(MW == 8 || MW == 16, "8 or 16 warps per CTA");
+    constexpr int kMW = MW, kMThreads = MW * 32, LW = MW == 16 ? 4 : 3;
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     static_assert(!ONE || NT == 1, "one column fits one n-tile");
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -284,8 +288,8 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
     float *red = x7 + (ONE ? (size_t)round8(a.g_stage) : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
-    int *bis = reinterpret_cast<int *>(bvs + kMThreads * 2 * NT);
-    PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT));
+    int *bis = reinterpret_cast<int *>(bvs + kMW * 8 * NT);
+    PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT, MW));
     int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
     volatile int *abort_flag = wcount + kMW;
     float *rn = reinterpret_cast<float *>(wcount + kMW + 4);   // RMSNorm factors of a windowed segment
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
                     mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
-                    mine.wkl = pick_wkl(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
+                    mine.wkl = pick_wkl<LW>(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
                 }
             }
             neutral_max = !has && ((a.lm_bits[tid >> 5] >> (tid & 31)) & 1u);
@@ -382,23 +386,31 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         is_gsh = P.gsh;
         is_chunks = ig.my_chunks;
     };
-    // move to the next segment that has items for this warp (or end the stream)
-    auto next_segment = [&]() {
-        is_chunks = 0;
-        while (++is_s < nseg) {
-            ig = pass_geo(segs[is_s], warp);
-            if (ig.my_tiles == 0) continue;
-            const PassProj &P = a.p[segs[is_s].p];
+    // this warp's next tile: the current segment's next one, else the first one of the next
+    // segment that has any for this warp (is_chunks 0: the stream has ended).  One place for
+    // every tile change keeps the code small where issue_next is inlined.
+    auto advance = [&]() {
+        if (is_tiles > 0) {
+            --is_tiles;
+            is_o0 += is_rstep;
+        } else {
+            for (;;) {
+                if (++is_s >= nseg) {
+                    is_chunks = 0;
+                    return;
+                }
+                ig = pass_geo<LW>(segs[is_s], warp);
+                if (ig.my_tiles > 0) break;
+            }
             is_tiles = ig.my_tiles - 1;
-            is_kc_last = pass_last_kc(ig, P.G);
+            is_kc_last = pass_last_kc(ig, a.p[segs[is_s].p].G);
             is_step = ig.wk * kMChunkG;
             is_rstep = ig.wr_n * ig.rout;
             is_o0 = ig.o_begin + ig.my_wr * ig.rout;
-            set_tile();
-            return;
         }
+        set_tile();
     };
-    next_segment();
+    advance();
     auto issue_next = [&]() {
         if (is_chunks > 0) {
             const int kc = is_chunks == 1 ? is_kc_last : kMChunkG;
@@ -415,22 +427,14 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 4; ++i) src_w[i] += is_step;
             src_s += is_step >> is_gsh;
-            if (--is_chunks == 0) {
-                if (is_tiles > 0) {
-                    --is_tiles;
-                    is_o0 += is_rstep;
-                    set_tile();
-                } else {
-                    next_segment();
-                }
-            }
+            if (--is_chunks == 0) advance();
         }
         cp_async_commit();     // one group per item slot, so wait counts stay uniform
         is_st = (is_st + 1 == (uint32_t)S) ? 0u : is_st + 1;
     };
 
     // prologue: the first weights stream before the previous kernel has finished
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
     if (neutral_max) {
@@ -474,7 +478,7 @@ __global__ void __launch_bounds__(kMThreads, 2) q4_pass_kernel(const __grid_cons
         for (; cs < nseg && segs[cs].phase == ph; ++cs) {
             const PassSeg sgm = segs[cs];
             const PassProj &P = a.p[sgm.p];
-            const PassGeo g = pass_geo(sgm, warp);
+            const PassGeo g = pass_geo<LW>(sgm, warp);
             const int G = P.G, N = P.N, kind = P.kind, ldo = P.ldo, rope_d = P.rope_d, gsh = P.gsh;
             const bool sasync = P.scales_async;
             // this CTA's tokens m0 .. m0 + M - 1 of the [Mt][K] inputs and [Mt][ldo] outputs

@@ -126,38 +126,49 @@ int resident_ctas(const void *fn, int threads, size_t smem, int &sms)
 constexpr size_t kSmemTwoPerSm = 113 * 1024;
 constexpr size_t kSmemOnePerSm = 227 * 1024;
 
-// How a pass launch stages its activations: CTAs per SM, ring depth, the
-// groups of K per column the activation area holds, and whether longer
-// projections go through K windows of that many groups.  A function of
+// How a pass launch stages its activations: warps per CTA, CTAs per SM, ring
+// depth, the groups of K per column the activation area holds, and whether
+// longer projections go through K windows of that many groups.  A function of
 // (M, the list's largest K, the list length) only.
 struct PassPlan {
-    int cps, stages, g_stage;
+    int mw, cps, stages, g_stage;
     bool win;
 };
 
-// Whole-K staging when the rings (2..4 stages) and all of x fit, two CTAs per
-// SM before one; otherwise K windows (a multiple of 8 groups, one item's
-// chunk) as long as fit three stages at two CTAs per SM, else one CTA per SM
-// with four stages.  Always succeeds for M <= 16 and lists of up to
-// kPassMax projections: the smallest window (8 groups) needs 96 KiB.
-PassPlan pass_plan(int M, int g_max, int n, int NT)
+// Whole-K staging when the rings (2..4 stages) and all of x fit: first one CTA
+// of 16 warps per SM, then two CTAs of 8, then one of 8; otherwise K windows (a
+// multiple of 8 groups, one item's chunk) with 8 warps, as long as fit three
+// stages at two CTAs per SM, else one CTA per SM with four stages.  Always
+// succeeds for M <= 16 and lists of up to kPassMax projections: the smallest
+// window (8 groups) needs 96 KiB.  One CTA of 16 warps beats two of 8 when it
+// fits: two CTAs on an SM do not share its issue slots evenly (the older one
+// runs ahead), and the kernel ends with the slower one.  `wide`: 16 warps may
+// be planned.
+PassPlan pass_plan(int M, int g_max, int n, int NT, bool wide = true)
 {
-    const size_t per_stage = (size_t)kMW * kMStage;
+    if (wide) {
+        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 16);
+        const size_t per_stage = (size_t)16 * kMStage;
+        const int stages =
+            kSmemOnePerSm > fixed ? (int)std::min<size_t>(kPassMaxStages, (kSmemOnePerSm - fixed) / per_stage) : 0;
+        if (stages >= 2) return PassPlan{16, 1, stages, g_max, false};
+    }
+    const size_t per_stage = (size_t)8 * kMStage;
     for (int cps = 2; cps >= 1; --cps) {
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
-        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT);
+        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 8);
         const int stages = budget > fixed ? (int)std::min<size_t>(kPassMaxStages, (budget - fixed) / per_stage) : 0;
-        if (stages >= 2) return PassPlan{cps, stages, g_max, false};
+        if (stages >= 2) return PassPlan{8, cps, stages, g_max, false};
     }
     for (int cps = 2; cps >= 1; --cps) {
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const int stages = cps == 2 ? 3 : kPassMaxStages;
         int best = 0;
         for (int gw = kMChunkG; gw < g_max; gw += kMChunkG)
-            if (pass_smem_bytes(M, gw, stages, n, NT) <= budget) best = gw;
-        if (best > 0) return PassPlan{cps, stages, best, true};
+            if (pass_smem_bytes(M, gw, stages, n, NT, 8) <= budget) best = gw;
+        if (best > 0) return PassPlan{8, cps, stages, best, true};
     }
-    return PassPlan{0, 0, 0, false};
+    return PassPlan{0, 0, 0, 0, false};
 }
 
 // M > 8 runs as two column blocks of ceil(M/2) and floor(M/2) tokens (the
@@ -171,15 +182,15 @@ bool pass_colsplit(int M, int g_max, int n) { return M > 8 && pass_plan(M, g_max
 // some projection waits on earlier ones (all CTAs must be co-resident).
 constexpr int kNotResident = 1;   // launch_pass_s: this shape does not reach the wanted residency
 
-template <int NT, int PMAX, int S, bool ONE, bool WIN>
+template <int NT, int PMAX, int S, bool ONE, bool WIN, int MW>
 int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps)
 {
-    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S, ONE, WIN>);
+    const void *fn = reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, S, ONE, WIN, MW>);
     int sms = 0;
-    if (resident_ctas(fn, kMThreads, smem, sms) < cps) return kNotResident;
+    if (resident_ctas(fn, MW * 32, smem, sms) < cps) return kNotResident;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kMThreads);
+    cfg.blockDim = dim3(MW * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -193,7 +204,7 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     clear_stale_error();
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S, ONE, WIN>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, q4_pass_kernel<NT, PMAX, S, ONE, WIN, MW>, a);
     if (e != cudaSuccess) {
         g_last_cuda_error = e;
         (void)cudaGetLastError();
@@ -202,14 +213,14 @@ int launch_pass_s(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, in
     return ZT_OK;
 }
 
-template <int NT, int PMAX, bool ONE, bool WIN>
+template <int NT, int PMAX, bool ONE, bool WIN, int MW>
 int launch_pass_w(const PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int grid, size_t smem, int cps,
                   int stages)
 {
     switch (stages) {
-    case 2: return launch_pass_s<NT, PMAX, 2, ONE, WIN>(a, cooperative, st, grid, smem, cps);
-    case 3: return launch_pass_s<NT, PMAX, 3, ONE, WIN>(a, cooperative, st, grid, smem, cps);
-    default: return launch_pass_s<NT, PMAX, 4, ONE, WIN>(a, cooperative, st, grid, smem, cps);
+    case 2: return launch_pass_s<NT, PMAX, 2, ONE, WIN, MW>(a, cooperative, st, grid, smem, cps);
+    case 3: return launch_pass_s<NT, PMAX, 3, ONE, WIN, MW>(a, cooperative, st, grid, smem, cps);
+    default: return launch_pass_s<NT, PMAX, 4, ONE, WIN, MW>(a, cooperative, st, grid, smem, cps);
     }
 }
 
@@ -219,7 +230,7 @@ template <int NT, int PMAX, bool ONE>
 int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_out)
 {
     int sms = 0;
-    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2, ONE, false>), kMThreads, 0, sms) < 1)
+    if (resident_ctas(reinterpret_cast<const void *>(&q4_pass_kernel<NT, PMAX, 2, ONE, false, 8>), 8 * 32, 0, sms) < 1)
         return ZT_ERR_DEVICE;
     int g_max = 0;
     for (int i = 0; i < a.n; ++i) g_max = std::max(g_max, a.p[i].G);
@@ -242,26 +253,31 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
     a.pbeg[a.n] = off;
     a.phbeg[a.phases] = off;
     const int Mc = a.colsplit ? (a.M + 1) / 2 : a.M;   // columns one CTA stages at most
-    const PassPlan plan = pass_plan(Mc, g_max, a.n, NT);
-    if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
-    a.g_stage = plan.g_stage;
-    const size_t smem = pass_smem_bytes(Mc, plan.g_stage, plan.stages, a.n, NT);
-    // the planned CTAs per SM, or one if the device holds fewer at this shared memory size
-    // (with the column split, an even grid: CTAs 2s and 2s + 1 take the same rows)
     const long long per_row = a.colsplit ? 2 : 1;
-    for (int cps = plan.cps; cps >= 1; --cps) {
-        long long g = std::min<long long>({(long long)sms * cps, cooperative ? (long long)sms * cps : rows * per_row,
-                                           kMaxCtas});
-        if (a.colsplit) g &= ~1LL;
-        const int grid = (int)std::max<long long>(per_row, g);
-        int rc = ZT_ERR_UNSUPPORTED;
-        if (!plan.win)
-            rc = launch_pass_w<NT, PMAX, ONE, false>(a, cooperative, st, grid, smem, cps, plan.stages);
-        else if constexpr (NT == 1)   // 16 columns that would need windows run as two column blocks instead
-            rc = launch_pass_w<NT, PMAX, ONE, true>(a, cooperative, st, grid, smem, cps, plan.stages);
-        if (rc == kNotResident) continue;
-        if (rc == ZT_OK && grid_out) *grid_out = grid;
-        return rc;
+    // the plan, then (if the device holds fewer CTAs of it) the plan without 16-warp CTAs
+    for (int attempt = 0; attempt < 2; ++attempt) {
+        const PassPlan plan = pass_plan(Mc, g_max, a.n, NT, attempt == 0);
+        if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
+        a.g_stage = plan.g_stage;
+        const size_t smem = pass_smem_bytes(Mc, plan.g_stage, plan.stages, a.n, NT, plan.mw);
+        // the planned CTAs per SM, or one if the device holds fewer at this shared memory size
+        // (with the column split, an even grid: CTAs 2s and 2s + 1 take the same rows)
+        for (int cps = plan.cps; cps >= 1; --cps) {
+            long long g = std::min<long long>(
+                {(long long)sms * cps, cooperative ? (long long)sms * cps : rows * per_row, kMaxCtas});
+            if (a.colsplit) g &= ~1LL;
+            const int grid = (int)std::max<long long>(per_row, g);
+            int rc = ZT_ERR_UNSUPPORTED;
+            if (plan.mw == 16)
+                rc = launch_pass_w<NT, PMAX, ONE, false, 16>(a, cooperative, st, grid, smem, cps, plan.stages);
+            else if (!plan.win)
+                rc = launch_pass_w<NT, PMAX, ONE, false, 8>(a, cooperative, st, grid, smem, cps, plan.stages);
+            else if constexpr (NT == 1)   // 16 columns that would need windows run as two column blocks instead
+                rc = launch_pass_w<NT, PMAX, ONE, true, 8>(a, cooperative, st, grid, smem, cps, plan.stages);
+            if (rc == kNotResident) continue;
+            if (rc == ZT_OK && grid_out) *grid_out = grid;
+            return rc;
+        }
     }
     return ZT_ERR_DEVICE;
 }
@@ -576,7 +592,7 @@ int read_error_word(const void *p, unsigned int *out)
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 4; }
+int zt_q4_version(void) { return (1 << 16) | 5; }
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -818,9 +834,10 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
     return ZT_OK;
 }
 
-int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window, int *column_blocks)
+int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int *k_window, int *column_blocks,
+                    int *warps_per_cta)
 {
-    if (!ctas_per_sm || !stages || !k_window || !column_blocks) return ZT_ERR_INVALID_ARG;
+    if (!ctas_per_sm || !stages || !k_window || !column_blocks || !warps_per_cta) return ZT_ERR_INVALID_ARG;
     if (M < 1 || M > 16 || n < 1 || n > ZT_Q4_PASS_MAX || K_max < kGroup || K_max % kGroup) return ZT_ERR_INVALID_ARG;
     const bool split = pass_colsplit(M, K_max / kGroup, n);
     const PassPlan plan = pass_plan(split ? (M + 1) / 2 : M, K_max / kGroup, n, (M <= 8 || split) ? 1 : 2);
@@ -829,6 +846,7 @@ int zt_q4_pass_plan(int M, int K_max, int n, int *ctas_per_sm, int *stages, int 
     *stages = plan.stages;
     *k_window = plan.win ? plan.g_stage * kGroup : 0;
     *column_blocks = split ? 2 : 1;
+    *warps_per_cta = plan.mw;
     return ZT_OK;
 }
 

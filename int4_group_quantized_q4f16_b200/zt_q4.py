@@ -78,7 +78,7 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_pass.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass.restype = ctypes.c_int
     lib.zt_q4_pass_errors.argtypes = [_P, _I, ctypes.POINTER(ctypes.c_uint)]
-    lib.zt_q4_pass_plan.argtypes = [_I, _I, _I] + [ctypes.POINTER(_I)] * 4
+    lib.zt_q4_pass_plan.argtypes = [_I, _I, _I] + [ctypes.POINTER(_I)] * 5
     lib.zt_q4_pass_plan.restype = ctypes.c_int
     lib.zt_q4_pass_test_withhold.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass_test_withhold.restype = ctypes.c_int
@@ -355,15 +355,15 @@ def lmhead_argmax_noalloc(qw, scales, x, logits=None, argmax=None, stream=None):
     return logits, argmax
 
 
-def pass_plan(M: int, K_max: int, n: int = 1) -> Tuple[int, int, int, int]:
-    """(CTAs per SM, ring stages, k_window, column_blocks) of the decode kernel
-    for these shapes; k_window 0 = activations staged whole; column_blocks 2 =
-    the first ceil(M/2) tokens and the rest in separate CTAs (no device
-    needed)."""
-    c, st, kw, cb = _I(0), _I(0), _I(0), _I(0)
-    _check(lib.zt_q4_pass_plan(M, K_max, n, ctypes.byref(c), ctypes.byref(st), ctypes.byref(kw), ctypes.byref(cb)),
-           "zt_q4_pass_plan")
-    return c.value, st.value, kw.value, cb.value
+def pass_plan(M: int, K_max: int, n: int = 1) -> Tuple[int, int, int, int, int]:
+    """(CTAs per SM, ring stages, k_window, column_blocks, warps per CTA) of
+    the decode kernel for these shapes; k_window 0 = activations staged whole;
+    column_blocks 2 = the first ceil(M/2) tokens and the rest in separate CTAs
+    (no device needed)."""
+    c, st, kw, cb, w = _I(0), _I(0), _I(0), _I(0), _I(0)
+    _check(lib.zt_q4_pass_plan(M, K_max, n, ctypes.byref(c), ctypes.byref(st), ctypes.byref(kw), ctypes.byref(cb),
+                               ctypes.byref(w)), "zt_q4_pass_plan")
+    return c.value, st.value, kw.value, cb.value, w.value
 
 
 class Pass:

@@ -332,8 +332,9 @@ def test_decode_plan_covers_every_small_batch_shape(zt):
     for M in range(1, 17):
         for K in (32, 256, 1056, 3072, 4096, 8192, 11008, 12320, 16384, 40000, 65536, 131072, 1 << 20):
             for n in (1, 4, 129, 192):
-                cps, stages, kw, cb = zt.pass_plan(M, K, n)
+                cps, stages, kw, cb, warps = zt.pass_plan(M, K, n)
                 assert cps in (1, 2) and 2 <= stages <= 4, (M, K, n)
+                assert warps == 8 or (warps == 16 and cps == 1 and kw == 0), (M, K, n, warps)
                 assert kw == 0 or (kw % 256 == 0 and 256 <= kw < K), (M, K, n, kw)
                 assert cb == 1 or (cb == 2 and M > 8), (M, K, n, cb)
                 if M > 8 and cb == 1:
@@ -342,20 +343,22 @@ def test_decode_plan_covers_every_small_batch_shape(zt):
 
 def test_decode_plan_pins(zt):
     """Where the plan switches, on the shapes of the benchmark and its configs."""
-    # the benchmark's Phi-3-mini pass at M = 1: x staged whole, two CTAs per SM, 4-deep rings
-    assert zt.pass_plan(1, 8192, 129) == (2, 4, 0, 1)
-    # config 3 (gate_up K = 3072) at M = 16 still fits whole, one CTA per SM, one column block
-    assert zt.pass_plan(16, 3072, 1) == (1, 4, 0, 1)
+    # the benchmark's Phi-3-mini pass at M = 1: x staged whole, one CTA of 16 warps per SM, 4-deep rings
+    assert zt.pass_plan(1, 8192, 129) == (1, 4, 0, 1, 16)
+    # config 3 (gate_up K = 3072) at M = 16 still fits whole, 16 warps with 2-deep rings, one column block
+    assert zt.pass_plan(16, 3072, 1) == (1, 2, 0, 1, 16)
+    # M = 8 with K = 8192: x (131 KB) leaves no room for 16 warps' rings: 8 warps, 4-deep rings
+    assert zt.pass_plan(8, 8192, 129) == (1, 4, 0, 1, 8)
     # Llama-7B down (K = 11008): whole at M = 4, windows from M = 8, and two column blocks
     # of windows at M = 16
     assert zt.pass_plan(4, 11008, 1)[2] == 0
-    assert zt.pass_plan(8, 11008, 1)[2:] == (2816, 1)
-    assert zt.pass_plan(16, 11008, 1)[2:] == (2816, 2)
+    assert zt.pass_plan(8, 11008, 1)[2:] == (2816, 1, 8)
+    assert zt.pass_plan(16, 11008, 1)[2:] == (2816, 2, 8)
     # Phi-3 down (8192): 16 columns fit whole up to M = 9; at M = 12 and 16 two column
     # blocks of at most 8 tokens, each whole
-    assert zt.pass_plan(9, 8192, 1)[2:] == (0, 1)
-    assert zt.pass_plan(12, 8192, 1)[2:] == (0, 2) and zt.pass_plan(16, 8192, 129)[2:] == (0, 2)
-    # single token: whole up to K = 65536, windows beyond
+    assert zt.pass_plan(9, 8192, 1)[2:4] == (0, 1)
+    assert zt.pass_plan(12, 8192, 1)[2:4] == (0, 2) and zt.pass_plan(16, 8192, 129)[2:4] == (0, 2)
+    # single token: whole up to K = 65536 (8 warps from there), windows beyond
     assert zt.pass_plan(1, 65536, 1)[2] == 0
     assert zt.pass_plan(1, 131072, 1)[2] > 0
     # windows go with two CTAs per SM
@@ -365,9 +368,9 @@ def test_decode_plan_pins(zt):
 def test_decode_plan_rejects_bad_shapes(zt):
     c = ctypes.c_int(0)
     for M, K, n in ((0, 256, 1), (17, 256, 1), (1, 16, 1), (1, 100, 1), (1, 256, 0), (1, 256, 193)):
-        assert zt.lib.zt_q4_pass_plan(M, K, n, *[ctypes.byref(c)] * 4) == zt.ZT_ERR_INVALID_ARG
-    assert zt.lib.zt_q4_pass_plan(1, 256, 1, None, *[ctypes.byref(c)] * 3) == zt.ZT_ERR_INVALID_ARG
-    assert zt.lib.zt_q4_pass_plan(1, 256, 1, *[ctypes.byref(c)] * 3, None) == zt.ZT_ERR_INVALID_ARG
+        assert zt.lib.zt_q4_pass_plan(M, K, n, *[ctypes.byref(c)] * 5) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_pass_plan(1, 256, 1, None, *[ctypes.byref(c)] * 4) == zt.ZT_ERR_INVALID_ARG
+    assert zt.lib.zt_q4_pass_plan(1, 256, 1, *[ctypes.byref(c)] * 4, None) == zt.ZT_ERR_INVALID_ARG
 
 
 def test_noalloc_misaligned_rejected_without_cuda(zt):
