@@ -437,6 +437,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
 #pragma unroll 1
     for (int j = 0; j < S - 1; ++j) issue_next();
     pdl_wait();
+    // a list without waits is launched without clearing its workspace: no wait can expire,
+    // so its error word is simply cleared (after the wait: the kernel ahead may be a pass on
+    // the same workspace)
+    if (!a.counters && a.error && blockIdx.x == 0 && tid == 0) *a.error = 0;
     if (neutral_max) {
         // written only after the wait: the kernel ahead on the stream may be
         // the argmax reduction of an earlier call that reads the same scratch

@@ -798,7 +798,9 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     clear_stale_error();
-    cudaError_t e = cudaMemsetAsync(ws, 0, err_off + 16, st);   // counters + error bits
+    // counters + error bits; a list without waits has no counters and can set no error bit, so
+    // its kernel clears the error word itself (one launch fewer per call)
+    cudaError_t e = cooperative ? cudaMemsetAsync(ws, 0, err_off + 16, st) : cudaSuccess;
     if (e != cudaSuccess) {
         g_last_cuda_error = e;
         (void)cudaGetLastError();

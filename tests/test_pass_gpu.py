@@ -177,6 +177,25 @@ def test_pass_batch_sweep(zt, oracle, M):
         _check_against_oracle(oracle, d)
 
 
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_pass_two_lm_heads(zt, oracle, M):
+    """Two LM heads in one list (and one in a later phase): each gets its own
+    per-CTA maxima and argmax reduction; a second call starts clean."""
+    import torch
+    projs = [_proj("lm_head", 4000, 1024, M, 801, 1), _proj("gemv", 640, 1024, M, 802, 2),
+             _proj("lm_head", 333, 512, M, 803, 3), _proj("lm_head", 2100, 640, M, 804, 4)]
+    projs[3]["x"] = projs[1]["out"]   # reads an earlier output: a second phase
+    projs[3]["wait"] = 1
+    p = zt.Pass(projs)
+    for _ in range(2):   # the counters start from zero again on the second call
+        p.run()
+        torch.cuda.synchronize()
+        assert p.errors() == 0
+        for d in projs[:3]:
+            _check_against_oracle(oracle, d)
+        _check_against_oracle(oracle, projs[3], x_host=host(projs[1]["out"]).astype(np.float16))
+
+
 @pytest.mark.parametrize("M,K", [(10, 8192), (16, 11008)])
 def test_pass_column_split_mixed(zt, oracle, M, K):
     """More than 8 tokens with a long K in the list: every projection runs as
