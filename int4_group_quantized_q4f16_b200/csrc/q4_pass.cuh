@@ -129,18 +129,20 @@ static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel
 // log2 of the warps splitting K for a segment: minimise the items of the
 // busiest warp (tiles per row-warp x chunks per K-warp), ties -> fewer
 // K-warps.  LW: log2 of the CTA's warps.  `bounded`: the whole segment's
-// partials meet at once, so the partial buffer bounds them (tiles * WK * 16 *
-// 8 NT <= pass_red_floats); a windowed segment reduces one round of at most
-// (warps / WK) tiles at a time.
-template <int LW>
+// partials meet at once, so the partial buffer bounds them (tiles * WK * the
+// floats of one partial <= pass_red_floats); a windowed segment reduces one
+// round of at most (warps / WK) tiles at a time.  A partial is 16 rows x 8 NT
+// columns, or 16 row sums with a single column (ONE).
+template <int LW, bool ONE>
 __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool bounded)
 {
+    constexpr int kPart = ONE ? kMTileRows : kMTileRows * 8;
     int best = 0, best_cost = -1;
 #pragma unroll
     for (int wkl = 0; wkl <= LW; ++wkl) {
         const int wk = 1 << wkl;
         if (wk > n_chunks) break;
-        if (bounded && wkl > 0 && n_tiles * wk * kMTileRows * 8 * NT > pass_red_floats(NT, 1 << LW)) break;
+        if (bounded && wkl > 0 && n_tiles * wk * kPart * (ONE ? 1 : NT) > pass_red_floats(NT, 1 << LW)) break;
         const int cost = ((n_tiles + ((1 << LW) >> wkl) - 1) >> (LW - wkl)) * ((n_chunks + wk - 1) >> wkl);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
-                    mine.wkl = pick_wkl<LW>(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
+                    mine.wkl = pick_wkl<LW, ONE>(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
                 }
             }
             neutral_max = !has && ((a.lm_bits[tid >> 5] >> (tid & 31)) & 1u);
@@ -525,25 +527,27 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
             // (tile t's partials sit at local index t - t0 of the buffer), and
             // the epilogue of their outputs runs; best_v / best_i: the LM head's
             // running maxima of this thread (slot 0: column tid % (8 NT)).
+            // a warp's partial of a tile: [16 rows][8 NT columns] floats, or (ONE) the 16 row sums
+            constexpr int PC = ONE ? 1 : 8 * NT, PART = kMTileRows * PC;
             auto reduce_tiles = [&](auto log_tag, int t0, int tn, float (&best_v)[2 * NT], int (&best_i)[2 * NT]) {
                 constexpr bool LOG = decltype(log_tag)::value;
-                const int VO = g.rout * 8 * NT;               // (output row, column) pairs per tile
+                const int VO = g.rout * PC;                   // (output row, column) pairs per tile
                 for (int idx = tid; idx < tn * VO; idx += kMThreads) {
                     const int tt = idx / VO, vo = idx - (idx / VO) * VO;
-                    const int r = vo / (8 * NT), m = vo - (vo / (8 * NT)) * (8 * NT);
+                    const int r = vo / PC, m = vo - (vo / PC) * PC;
                     const int nn = g.o_begin + (t0 + tt) * g.rout + r;
                     if (nn >= g.o_end || m >= M) continue;
-                    const float *rp = red + (size_t)tt * g.wk * kMTileRows * 8 * NT;
+                    const float *rp = red + (size_t)tt * g.wk * PART;
                     float y = 0.f, u = 0.f;
                     for (int k2 = 0; k2 < g.wk; ++k2) {
-                        y += rp[(size_t)k2 * kMTileRows * 8 * NT + r * 8 * NT + m];
+                        y += rp[(size_t)k2 * PART + r * PC + m];
                         if (kind == kEpiGateUp || kind == kEpiRope)
-                            u += rp[(size_t)k2 * kMTileRows * 8 * NT + (r + 8) * 8 * NT + m];
+                            u += rp[(size_t)k2 * PART + (r + 8) * PC + m];
                     }
                     y *= pow2f(24);
                     if constexpr (LOG) {
                         reinterpret_cast<float *>(out)[(size_t)m * ldo + nn] = y;
-                        // thread tid handles m = idx % (8 NT) = tid % (8 NT): slot 0 of its table
+                        // thread tid handles m = idx % PC = tid % PC: slot 0 of its table
                         if (better(y, nn, best_v[0], best_i[0])) {
                             best_v[0] = isnan(y) ? -INFINITY : y;
                             best_i[0] = nn;
@@ -789,15 +793,23 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
 
                     // ---- tile epilogue ----
                     if (have && g.wk > 1) {
-                        // this warp's partial of tile t: [16 rows][8*NT columns]; windowed
-                        // rounds number their tiles from the round's first (my_wr)
-                        float *rp = red + ((size_t)(WS ? g.my_wr : t) * g.wk + g.my_wk) * kMTileRows * 8 * NT;
+                        // this warp's partial of tile t; windowed rounds number their tiles
+                        // from the round's first (my_wr)
+                        float *rp = red + ((size_t)(WS ? g.my_wr : t) * g.wk + g.my_wk) * PART;
+                        if constexpr (ONE) {
+                            // the quad's row sums (slots 0 and 2 of every lane of the quad)
+                            if (qt == 0) {
+                                rp[qg] = acc[0][0];
+                                rp[qg + 8] = acc[0][2];
+                            }
+                        } else {
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
-                            rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
-                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
-                            rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                            for (int nt = 0; nt < NT; ++nt) {
+                                rp[qg * 8 * NT + 8 * nt + 2 * qt] = acc[nt][0];
+                                rp[qg * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][1];
+                                rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt] = acc[nt][2];
+                                rp[(qg + 8) * 8 * NT + 8 * nt + 2 * qt + 1] = acc[nt][3];
+                            }
                         }
                     } else if (have) {
 #pragma unroll
@@ -856,9 +868,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                 if constexpr (LOG) {
                     // The CTA's (maximum, lowest index) per column m under better()'s total order
                     // (so the reduction order does not matter): within each warp a butterfly over
-                    // the lanes that hold the same column, then the 8 warps' results per column.
-                    // Column of slot i: with WK > 1 only slot 0, column lane % (8 NT); otherwise
-                    // column 8 (i >> 1) + 2 qt + (i & 1), shared by the lanes of equal qt.
+                    // the lanes that hold the same column, then the warps' results per column.
+                    // Column of slot i: with WK > 1 only slot 0, column lane % PC (column 0 in
+                    // every lane with ONE); otherwise column 8 (i >> 1) + 2 qt + (i & 1), shared by
+                    // the lanes of equal qt.
                     auto comb = [&](float &v, int &ix, int mask) {
                         const float ov = __shfl_xor_sync(0xffffffffu, v, mask);
                         const int oi = __shfl_xor_sync(0xffffffffu, ix, mask);
@@ -868,7 +881,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                         }
                     };
                     if (g.wk > 1) {
-                        for (int mask = 8 * NT; mask < 32; mask <<= 1) comb(best_v[0], best_i[0], mask);
+                        // slot 0 holds column lane % PC (every lane column 0 with ONE)
+                        for (int mask = PC; mask < 32; mask <<= 1) comb(best_v[0], best_i[0], mask);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 2 * NT; ++i)
