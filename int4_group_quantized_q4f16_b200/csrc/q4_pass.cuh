@@ -79,6 +79,7 @@ struct PassArgs {
     unsigned int *counters;     // [phases - 1], zero at launch (only when phases > 1)
     unsigned int *error;        // error bits
     int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
+    int red_floats;             // size of the WK partial buffer (floats)
     int colsplit;               // M > 8 as two column blocks: CTAs 2s and 2s + 1 take row share s, tokens
                                 // 0 .. ceil(M/2) - 1 and the rest (each an M <= 8 problem of 5..8 tokens)
     // What every CTA reads to find its rows, kept apart from p[] in dense arrays: a warp
@@ -94,9 +95,14 @@ struct PassArgs {
 // WK > 1 partial buffer: (tiles x WK) warp tiles of 16 rows x 8 NT columns
 // per segment.  The LM head's per-thread maxima reuse it once a segment's
 // partial sums have been read.
-// 4 KB per n-tile and 8 warps.  The LM head's maxima take 2 x MW x 8 NT words.
-__host__ __device__ constexpr int pass_red_floats(int NT, int MW) { return 128 * MW * NT; }
-static_assert(2 * 8 * 8 <= pass_red_floats(1, 8), "LM-head maxima must fit the partial buffer");
+// Its size in floats is a launch parameter: 128 per warp and n-tile (16-float partials with
+// one column: 128 per warp), or, where shared memory is short (16 warps, several columns),
+// the least that still holds the LM head's maxima (2 x MW x 8 NT words) with room for some
+// K splitting: 1024 per n-tile.
+__host__ __device__ constexpr int pass_red_floats(int NT, int MW, bool ONE) { return ONE ? 128 * MW : 128 * MW * NT; }
+__host__ __device__ constexpr int pass_red_floats_min(int NT, bool ONE) { return ONE ? 128 * 16 : 1024 * NT; }
+static_assert(2 * 16 * 8 * 2 <= pass_red_floats_min(2, false) && 2 * 16 * 8 <= pass_red_floats_min(1, true),
+              "LM-head maxima must fit the partial buffer");
 constexpr int kPassMaxStages = 4;           // ring depths 2..4 are instantiated
 
 // One projection's rows in one CTA, with the CTA's warp layout for them.
@@ -108,13 +114,14 @@ struct PassSeg {
 // Shared memory per CTA: rings, permuted activations (n-stride g_stage*64 +
 // 32 bytes), C-operand table, WK partials / LM-head maxima, segment list,
 // flags, the RMSNorm factors of a windowed segment (16 floats).
-__host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT, int MW)
+__host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages, int n, int NT, int MW,
+                                                   int red_floats)
 {
     const size_t ring = (size_t)MW * stages * kMStage + 1024;   // + alignment of the code stages
     // M = 1: the block-diagonal layout (a zero block, 80 bytes per group, one C float per group)
     const size_t xp = M == 1 ? (size_t)kBdZero + (size_t)round8(g_stage) * kBdGroup : (size_t)M * ((size_t)g_stage * 64 + 32);
     const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 4 : (size_t)g_stage * NT * 64;
-    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)pass_red_floats(NT, MW) * 4 + (size_t)n * sizeof(PassSeg) +
+    return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)red_floats * 4 + (size_t)n * sizeof(PassSeg) +
            (MW + 4) * sizeof(int) + 16 * sizeof(float);
 }
 
@@ -134,7 +141,7 @@ static_assert(sizeof(PassArgs<kPassMax>) <= 32764, "the list must fit the kernel
 // round of at most (warps / WK) tiles at a time.  A partial is 16 rows x 8 NT
 // columns, or 16 row sums with a single column (ONE).
 template <int LW, bool ONE>
-__device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool bounded)
+__device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool bounded, int red_floats)
 {
     constexpr int kPart = ONE ? kMTileRows : kMTileRows * 8;
     int best = 0, best_cost = -1;
@@ -142,7 +149,7 @@ __device__ __forceinline__ int pick_wkl(int n_tiles, int n_chunks, int NT, bool 
     for (int wkl = 0; wkl <= LW; ++wkl) {
         const int wk = 1 << wkl;
         if (wk > n_chunks) break;
-        if (bounded && wkl > 0 && n_tiles * wk * kPart * (ONE ? 1 : NT) > pass_red_floats(NT, 1 << LW)) break;
+        if (bounded && wkl > 0 && n_tiles * wk * kPart * (ONE ? 1 : NT) > red_floats) break;
         const int cost = ((n_tiles + ((1 << LW) >> wkl) - 1) >> (LW - wkl)) * ((n_chunks + wk - 1) >> wkl);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     float *red = x7 + (ONE ? (size_t)round8(a.g_stage) : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMW * 8 * NT);
-    PassSeg *segs = reinterpret_cast<PassSeg *>(red + pass_red_floats(NT, MW));
+    PassSeg *segs = reinterpret_cast<PassSeg *>(red + a.red_floats);
     int *wcount = reinterpret_cast<int *>(segs + n);           // [kMW] segments per warp
     volatile int *abort_flag = wcount + kMW;
     float *rn = reinterpret_cast<float *>(wcount + kMW + 4);   // RMSNorm factors of a windowed segment
@@ -324,7 +331,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     mine.rout = (P.kind == kEpiGateUp || P.kind == kEpiRope) ? kMTileRows / 2 : kMTileRows;
                     mine.n_tiles = (o1 - o0 + mine.rout - 1) / mine.rout;
                     mine.n_chunks = (P.G + kMChunkG - 1) / kMChunkG;
-                    mine.wkl = pick_wkl<LW, ONE>(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage));
+                    mine.wkl = pick_wkl<LW, ONE>(mine.n_tiles, mine.n_chunks, NT, !(WIN && P.G > a.g_stage), a.red_floats);
                 }
             }
             neutral_max = !has && ((a.lm_bits[tid >> 5] >> (tid & 31)) & 1u);

@@ -133,6 +133,7 @@ constexpr size_t kSmemOnePerSm = 227 * 1024;
 struct PassPlan {
     int mw, cps, stages, g_stage;
     bool win;
+    int red;   // WK partial buffer, floats
 };
 
 // Whole-K staging when the rings (2..4 stages) and all of x fit: first one CTA
@@ -146,29 +147,34 @@ struct PassPlan {
 // be planned.
 PassPlan pass_plan(int M, int g_max, int n, int NT, bool wide = true)
 {
+    const bool one = M == 1;
     if (wide) {
-        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 16);
-        const size_t per_stage = (size_t)16 * kMStage;
-        const int stages =
-            kSmemOnePerSm > fixed ? (int)std::min<size_t>(kPassMaxStages, (kSmemOnePerSm - fixed) / per_stage) : 0;
-        if (stages >= 2) return PassPlan{16, 1, stages, g_max, false};
+        // the full partial buffer, else the least one (room for the rings of 16 warps)
+        for (const int red : {pass_red_floats(NT, 16, one), pass_red_floats_min(NT, one)}) {
+            const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 16, red);
+            const size_t per_stage = (size_t)16 * kMStage;
+            const int stages =
+                kSmemOnePerSm > fixed ? (int)std::min<size_t>(kPassMaxStages, (kSmemOnePerSm - fixed) / per_stage) : 0;
+            if (stages >= 2) return PassPlan{16, 1, stages, g_max, false, red};
+        }
     }
+    const int red8 = pass_red_floats(NT, 8, one);
     const size_t per_stage = (size_t)8 * kMStage;
     for (int cps = 2; cps >= 1; --cps) {
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
-        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 8);
+        const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 8, red8);
         const int stages = budget > fixed ? (int)std::min<size_t>(kPassMaxStages, (budget - fixed) / per_stage) : 0;
-        if (stages >= 2) return PassPlan{8, cps, stages, g_max, false};
+        if (stages >= 2) return PassPlan{8, cps, stages, g_max, false, red8};
     }
     for (int cps = 2; cps >= 1; --cps) {
         const size_t budget = cps == 2 ? kSmemTwoPerSm : kSmemOnePerSm;
         const int stages = cps == 2 ? 3 : kPassMaxStages;
         int best = 0;
         for (int gw = kMChunkG; gw < g_max; gw += kMChunkG)
-            if (pass_smem_bytes(M, gw, stages, n, NT, 8) <= budget) best = gw;
-        if (best > 0) return PassPlan{8, cps, stages, best, true};
+            if (pass_smem_bytes(M, gw, stages, n, NT, 8, red8) <= budget) best = gw;
+        if (best > 0) return PassPlan{8, cps, stages, best, true, red8};
     }
-    return PassPlan{0, 0, 0, 0, false};
+    return PassPlan{0, 0, 0, 0, false, 0};
 }
 
 // M > 8 runs as two column blocks of ceil(M/2) and floor(M/2) tokens (the
@@ -259,7 +265,8 @@ int launch_pass(PassArgs<PMAX> &a, bool cooperative, cudaStream_t st, int *grid_
         const PassPlan plan = pass_plan(Mc, g_max, a.n, NT, attempt == 0);
         if (plan.cps == 0) return ZT_ERR_UNSUPPORTED;
         a.g_stage = plan.g_stage;
-        const size_t smem = pass_smem_bytes(Mc, plan.g_stage, plan.stages, a.n, NT, plan.mw);
+        a.red_floats = plan.red;
+        const size_t smem = pass_smem_bytes(Mc, plan.g_stage, plan.stages, a.n, NT, plan.mw, plan.red);
         // the planned CTAs per SM, or one if the device holds fewer at this shared memory size
         // (with the column split, an even grid: CTAs 2s and 2s + 1 take the same rows)
         for (int cps = plan.cps; cps >= 1; --cps) {

@@ -347,8 +347,10 @@ def test_decode_plan_pins(zt):
     assert zt.pass_plan(1, 8192, 129) == (1, 4, 0, 1, 16)
     # config 3 (gate_up K = 3072) at M = 16 still fits whole, 16 warps with 2-deep rings, one column block
     assert zt.pass_plan(16, 3072, 1) == (1, 2, 0, 1, 16)
-    # M = 8 with K = 8192: x (131 KB) leaves no room for 16 warps' rings: 8 warps, 4-deep rings
-    assert zt.pass_plan(8, 8192, 129) == (1, 4, 0, 1, 8)
+    # M = 8 with K = 8192: x (131 KB) leaves room for 16 warps' rings 2 deep, with the least
+    # partial buffer; M = 9 (16 columns, 262 KB of x at whole K) needs 8 warps
+    assert zt.pass_plan(8, 8192, 129) == (1, 2, 0, 1, 16)
+    assert zt.pass_plan(9, 8192, 1)[4] == 8
     # Llama-7B down (K = 11008): whole at M = 4, windows from M = 8, and two column blocks
     # of windows at M = 16
     assert zt.pass_plan(4, 11008, 1)[2] == 0
