@@ -11,7 +11,8 @@ page's performance table runs Llama-7B at 4 bits).
 The oracle computes sampled rows of every projection of three layers one by
 one, and the whole LM head; a second run must reproduce the first bit for
 bit.  The chained form (every projection waiting for the previous ones) is
-checked the same way."""
+checked the same way, and the same weights with 8 and 16 tokens per
+projection (the benchmark's batched decode)."""
 import argparse
 
 import numpy as np
@@ -145,3 +146,52 @@ def test_full_pass_chained(full_pass, oracle):
     for layer in CHECKED_LAYERS:
         _check_sampled(oracle, calls, one, layer, "chained")
     _check_lm_head(oracle, calls, one, "chained")
+
+
+@pytest.mark.parametrize("M", [8, 16])
+def test_full_pass_batched(full_pass, oracle, M):
+    """The same 129 projections with M tokens each, as the benchmark's batched
+    decode runs them: at M = 8 one 16-warp CTA per SM with 2-deep rings and
+    the least partial buffer (Phi-3) or K windows (Llama-7B's 11008-k down
+    projection), at M = 16 two column blocks of 8 tokens.  Sampled rows of
+    layers 0 and 31, the whole LM head and its argmax."""
+    import torch
+    from int4_group_quantized_q4f16_b200 import zt_q4
+    calls = full_pass[0]
+    rng = np.random.default_rng([M, 77])
+    projs, xs = [], []
+    for d in calls:
+        p = d["p"]
+        x = rng.standard_normal((M, p.K)).astype(np.float16)
+        xs.append(x)
+        e = {"kind": p.kind, "qw": d["qw"], "scales": d["s"], "x": torch.from_numpy(x).cuda(),
+             "out": torch.empty((M, p.n_out), dtype=torch.float32 if p.kind == "lm_head" else torch.float16,
+                                device="cuda")}
+        if p.kind == "lm_head":
+            e["argmax"] = torch.empty((M,), dtype=torch.int32, device="cuda")
+        projs.append(e)
+    zp = zt_q4.Pass(projs)
+    zp.run()
+    torch.cuda.synchronize()
+    assert zp.errors() == 0
+    for i, d in enumerate(calls):
+        p = d["p"]
+        if d["layer"] not in (0, 31) or p.kind == "lm_head":
+            continue
+        qw, s, _ = synth.proj_inputs(0, d["layer"], p)
+        x = xs[i]
+        rows = _sample_rows(p.n_out, 7 * i + M)
+        got = host(projs[i]["out"])
+        if p.kind == "gemv":
+            ref = oracle.gemv(qw, s, x, rows=rows.astype(np.int32), threads=8)
+            bound = abs_products(oracle, qw[rows], s[rows], x)
+        else:
+            ref = oracle.gate_up_silu(qw, s, x, rows=rows.astype(np.int32), threads=8)
+            sub = np.concatenate([rows, rows + p.n_out])
+            bound = gate_up_bound(oracle, qw[sub], s[sub], x, np.arange(len(rows), dtype=np.int32))
+        assert_f16_matches(got[:, rows], ref, f"M{M} layer {d['layer']} {p.name}", bound)
+    d = calls[-1]
+    qw, s, _ = synth.proj_inputs(0, d["layer"], d["p"])
+    ref, _ = oracle.lmhead_argmax(qw, s, xs[-1], threads=8)
+    assert_f32_matches(host(projs[-1]["out"]), ref, f"M{M} lm head")
+    check_argmax(host(projs[-1]["argmax"]), ref)
