@@ -47,8 +47,9 @@
 //     rows of the same outputs, so gate and up of an output meet in one
 //     thread).  K is cut into chunks of 8 groups (256 k).  Item = (tile,
 //     chunk) = 16 x 128 bytes of codes + 16 x 16 bytes of scales.
-//   * Each CTA owns a contiguous, balanced range of outputs; its 8 warps form
-//     WR x WK (WK warps split a tile's chunks when the CTA has few rows).
+//   * Each CTA owns a contiguous, balanced range of outputs; its 16 (or 8)
+//     warps form WR x WK (WK warps split a tile's chunks when the CTA has few
+//     rows).
 //   * Every warp streams its items through a private ring of S stages with
 //     16-byte cp.async copies (hardware waits, no spin loops).  Rows outside
 //     the CTA's range are never copied: a partial tile costs math, not bytes.

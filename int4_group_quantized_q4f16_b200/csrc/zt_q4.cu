@@ -137,7 +137,8 @@ struct PassPlan {
 };
 
 // Whole-K staging when the rings (2..4 stages) and all of x fit: first one CTA
-// of 16 warps per SM, then two CTAs of 8, then one of 8; otherwise K windows (a
+// of 16 warps per SM (with the full WK partial buffer, else the least one),
+// then two CTAs of 8, then one of 8; otherwise K windows (a
 // multiple of 8 groups, one item's chunk) with 8 warps, as long as fit three
 // stages at two CTAs per SM, else one CTA per SM with four stages.  Always
 // succeeds for M <= 16 and lists of up to kPassMax projections: the smallest
