@@ -945,10 +945,13 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
             consumer_sync();   // the activation area and partial buffers are free again
         }
         if (ph + 1 < nphase) {
-            // publish this CTA's outputs of the phase, then count it done
-            __threadfence();
-            consumer_sync();
-            if (tid == 0 && !(ph == a.withhold && blockIdx.x == 0)) atomicAdd(&a.counters[ph], 1u);
+            // publish this CTA's outputs of the phase, then count it done: every output was
+            // written before the CTA barrier that closes each segment, so one fence by the
+            // counting thread orders them all before its count
+            if (tid == 0 && !(ph == a.withhold && blockIdx.x == 0)) {
+                __threadfence();
+                atomicAdd(&a.counters[ph], 1u);
+            }
         }
     }
     cp_async_wait<0>();
