@@ -144,12 +144,14 @@ struct PassPlan {
 // succeeds for M <= 16 and lists of up to kPassMax projections: the smallest
 // window (8 groups) needs 96 KiB.  One CTA of 16 warps beats two of 8 when it
 // fits: two CTAs on an SM do not share its issue slots evenly (the older one
-// runs ahead), and the kernel ends with the slower one.  `wide`: 16 warps may
-// be planned.
+// runs ahead), and the kernel ends with the slower one.  Except for a single
+// projection of one token: there two 8-warp CTAs per SM leave room on each SM
+// for the next call's CTAs to start (programmatic dependent launch) while this
+// one drains, and measured faster alone too.  `wide`: 16 warps may be planned.
 PassPlan pass_plan(int M, int g_max, int n, int NT, bool wide = true)
 {
     const bool one = M == 1;
-    if (wide) {
+    if (wide && !(one && n == 1)) {
         // the full partial buffer, else the least one (room for the rings of 16 warps)
         for (const int red : {pass_red_floats(NT, 16, one), pass_red_floats_min(NT, one)}) {
             const size_t fixed = pass_smem_bytes(M, g_max, 0, n, NT, 16, red);

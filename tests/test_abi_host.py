@@ -343,8 +343,10 @@ def test_decode_plan_covers_every_small_batch_shape(zt):
 
 def test_decode_plan_pins(zt):
     """Where the plan switches, on the shapes of the benchmark and its configs."""
-    # the benchmark's Phi-3-mini pass at M = 1: x staged whole, one CTA of 16 warps per SM, 4-deep rings
+    # the benchmark's Phi-3-mini pass at M = 1: x staged whole, one CTA of 16 warps per SM, 4-deep rings;
+    # a single projection of one token: two CTAs of 8 warps per SM
     assert zt.pass_plan(1, 8192, 129) == (1, 4, 0, 1, 16)
+    assert zt.pass_plan(1, 3072, 1) == (2, 4, 0, 1, 8) and zt.pass_plan(2, 3072, 1)[4] == 16
     # config 3 (gate_up K = 3072) at M = 16 still fits whole, 16 warps with 2-deep rings, one column block
     assert zt.pass_plan(16, 3072, 1) == (1, 2, 0, 1, 16)
     # M = 8 with K = 8192: x (131 KB) leaves room for 16 warps' rings 2 deep, with the least
