@@ -374,6 +374,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     int is_chunks = 0;              // chunks left in the current tile (0: stream ended)
     int is_kc_last = kMChunkG;      // groups of the tile's last chunk
     int is_step = 0;                // uint4 per chunk step (WK chunks of 8 groups)
+    int is_sstep = 0;               // scale elements per chunk step
     uint32_t is_st = 0;             // ring stage of the next item to issue
     int is_o0 = 0, is_rstep = 0;    // current tile's first output, outputs per tile step
     PassGeo ig{};
@@ -381,6 +382,13 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     bool ok_w[4];
     const __half *src_s = nullptr;
     bool ok_s = false;
+    // the tile's last chunk holds only is_kc_last groups (K % 256 != 0): drop the other pieces
+    auto last_chunk = [&]() {
+        if (is_kc_last < kMChunkG) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ok_w[i] = ok_w[i] && pg < is_kc_last;
+        }
+    };
     auto set_tile = [&]() {
         const PassProj &P = a.p[segs[is_s].p];
 #pragma unroll
@@ -393,7 +401,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
         ok_s = ok_s && lane < kMTileRows && P.scales_async;
         src_s = P.scales + (size_t)row * (P.G >> P.gsh) + ((ig.my_wk * kMChunkG) >> P.gsh);
         is_gsh = P.gsh;
+        is_sstep = is_step >> P.gsh;
         is_chunks = ig.my_chunks;
+        if (is_chunks == 1) last_chunk();
     };
     // this warp's next tile: the current segment's next one, else the first one of the next
     // segment that has any for this warp (is_chunks 0: the stream has ended).  One place for
@@ -422,10 +432,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     advance();
     auto issue_next = [&]() {
         if (is_chunks > 0) {
-            const int kc = is_chunks == 1 ? is_kc_last : kMChunkG;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok_w[i] && pg < kc)
+                if (ok_w[i])
                     cp_async16_u32(((i & 1) ? piece_u1 : piece_u0) + (is_st << 11) + (i >> 1) * 1024, src_w[i]);
             if (ok_s) {
                 // the item's 8 blocks of 32 share 8, 4 or 2 scales: 16, 8 or 4 bytes per row
@@ -435,8 +444,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) src_w[i] += is_step;
-            src_s += is_step >> is_gsh;
+            src_s += is_sstep;
             if (--is_chunks == 0) advance();
+            else if (is_chunks == 1) last_chunk();
         }
         cp_async_commit();     // one group per item slot, so wait counts stay uniform
         is_st = (is_st + 1 == (uint32_t)S) ? 0u : is_st + 1;
@@ -665,12 +675,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                     s01 = 2 * qt + 1 < kc ? __half2float(p0[(b + 1) >> gsh]) : 0.f;
                                     s11 = 2 * qt + 1 < kc ? __half2float(p1[(b + 1) >> gsh]) : 0.f;
                                 }
-                                if (kc < kMChunkG) {
-                                    // the last chunk's missing groups: zero x and C were staged,
-                                    // and their scale slots were not copied (any bits): use 0
-                                    if (2 * qt >= kc) s00 = s10 = 0.f;
-                                    if (2 * qt + 1 >= kc) s01 = s11 = 0.f;
-                                }
+                                // (a chunk with missing groups, kc < 8, occurs only when K % 256 != 0, and
+                                // then scales are never copied asynchronously: the loads above give 0)
                                 const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
                                 float d[4] = {cz.x, cz.y, cz.x, cz.y};
                                 const unsigned char *b0p = smem + bd_b0 + (xoff & bd_m0);
