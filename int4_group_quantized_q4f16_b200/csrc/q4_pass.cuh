@@ -610,6 +610,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
                     uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * XG;   // B bytes of this warp's first chunk
                     uint32_t coff = (uint32_t)g.my_wk * kMChunkG * CG;   // C-table bytes
+                    // single column: this lane's two B-operand addresses, stepped per item by
+                    // the chunk step or by 0 (lanes that read the zero block)
+                    uint32_t bo0 = bd_b0 + (xoff & bd_m0), bo1 = bd_b1 + (xoff & bd_m1);
+                    const uint32_t xs0 = xstep & bd_m0, xs1 = xstep & bd_m1;
                     int cl = 0;
                     for (int w = 0; w < n_win; ++w) {
                         int cl_end = g.my_chunks;
@@ -626,6 +630,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             if (w > 0) {   // the area now starts at group w gs
                                 xoff -= (uint32_t)gs * XG;
                                 coff -= (uint32_t)gs * CG;
+                                bo0 -= ((uint32_t)gs * XG) & bd_m0;
+                                bo1 -= ((uint32_t)gs * XG) & bd_m1;
                             }
                             // this warp's chunks c = my_wk + wk cl below the window's end
                             const int c_end = (w + 1) * (gs / kMChunkG);
@@ -679,8 +685,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 // then scales are never copied asynchronously: the loads above give 0)
                                 const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
                                 float d[4] = {cz.x, cz.y, cz.x, cz.y};
-                                const unsigned char *b0p = smem + bd_b0 + (xoff & bd_m0);
-                                const unsigned char *b1p = smem + bd_b1 + (xoff & bd_m1);
+                                const unsigned char *b0p = smem + bo0;
+                                const unsigned char *b1p = smem + bo1;
                                 const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
                                 const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
 #pragma unroll
@@ -787,6 +793,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
                             xoff += xstep;
                             coff += cstep;
+                            bo0 += xs0;
+                            bo1 += xs1;
                         }
                     }
 
