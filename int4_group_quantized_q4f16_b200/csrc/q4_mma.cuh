@@ -123,29 +123,54 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 }
 
 // Single-column (M = 1) staging for the block-diagonal contraction of
-// q4_pass.cuh: the area starts with 64 bytes of zeros (the B operand of the
-// lanes whose mma column is another group's), then group g's four 16-byte
-// pieces at 64 + 80 g (80, not 64: the lanes reading groups 2t and 2t + 1
-// then hit distinct banks); the C table holds one float per group.  Groups
-// are padded with zeros to a multiple of 8 (one item).
-constexpr int kBdZero = 64;
-constexpr int kBdGroup = 80;
-__host__ __device__ constexpr uint32_t bd_piece(int kk) { return kBdZero + (kk >> 2) * kBdGroup + (kk & 3) * 16; }
+// q4_pass.cuh.  A lane's mma B operand is a register pair (b0, b1) of which at
+// most one is non-zero: b0 for a lane whose column is an even group of its
+// pair of groups, b1 for an odd one, neither for the other lanes.  So that one
+// 16-byte load gives two such pairs ready for two mma steps, each word w_s of
+// a group (mma step s) is staged next to a zero: groups 2p and 2p + 1 form a
+// 288-byte block, the even group as [w_0, 0, w_1, 0, ...] (128 bytes), 16
+// bytes apart, the odd one as [0, w_0, 0, w_1, ...].  The area starts with a
+// 224-byte zero region (the other lanes read 128 bytes of it, at 32 bytes per
+// quarter-warp); with these offsets the three addresses a quarter-warp reads
+// fall in distinct 16-byte bank groups.  The C table holds one float per
+// group; groups are padded with zeros to a multiple of 8 (one item).
+constexpr int kBdZero = 224;
+constexpr int kBdPair = 288;
+constexpr int kBdGroup = kBdPair / 2;   // bytes per group, for sizes and chunk steps
+__host__ __device__ constexpr uint32_t bd_slot(int kk)   // the 32 bytes of piece kk (4 words, 4 zeros)
+{
+    return kBdZero + (kk >> 3) * kBdPair + ((kk >> 2) & 1) * (kBdPair / 2) + (kk & 3) * 32;
+}
 __host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
+
+// the four words o of piece kk, each beside a zero (after it in an even group, before it in an odd one)
+__device__ __forceinline__ void bd_store(unsigned char *xp, int kk, uint4 o)
+{
+    uint4 *d = reinterpret_cast<uint4 *>(xp + bd_slot(kk));
+    if ((kk >> 2) & 1) {
+        d[0] = make_uint4(0u, o.x, 0u, o.y);
+        d[1] = make_uint4(0u, o.z, 0u, o.w);
+    } else {
+        d[0] = make_uint4(o.x, 0u, o.y, 0u);
+        d[1] = make_uint4(o.z, 0u, o.w, 0u);
+    }
+}
 
 // zero x and C of groups [Gw, round8(Gw)) in the single-column layout
 __device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw)
 {
     for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += (int)blockDim.x) {
-        *reinterpret_cast<uint4 *>(xp + bd_piece(Gw * 4 + j)) = make_uint4(0, 0, 0, 0);
+        bd_store(xp, Gw * 4 + j, make_uint4(0, 0, 0, 0));
         if ((j & 3) == 0) x7[Gw + (j >> 2)] = 0.f;
     }
 }
 
-// Byte offset of piece kk (8 activations) of column m in the staged area.
+// Byte offset of piece kk (8 activations) of column m in the staged area; with a
+// single column (compact) the first 16 bytes of the piece's slot, where the norm
+// prologue keeps h until the same thread turns it into x.
 __device__ __forceinline__ size_t x_piece(int m, int kk, size_t nstride, bool compact)
 {
-    return compact ? (size_t)bd_piece(kk) : (size_t)m * nstride + (size_t)kk * 16;
+    return compact ? (size_t)bd_slot(kk) : (size_t)m * nstride + (size_t)kk * 16;
 }
 
 // Stage x in mma-B order: for column n and group g, 64 bytes = for t = 0..3:
@@ -173,7 +198,8 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
         __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
         o.z = *reinterpret_cast<uint32_t *>(&q15);
         o.w = *reinterpret_cast<uint32_t *>(&q37);
-        *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, compact)) = o;
+        if (compact) bd_store(xp, kk, o);
+        else *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, false)) = o;
         const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
         float v[8];
 #pragma unroll

@@ -477,15 +477,16 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     const uint32_t sc_o = (uint32_t)(ring_s - smem) + qg * 16;                          // + stage * 256
     const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? qt * 8 : qt * 16);
     // M = 1 (block-diagonal): the mma's 8 columns are the item's 8 groups; lane (qg, qt) holds
-    // the codes of groups 2 qt and 2 qt + 1 of rows qg and qg + 8 (16 bytes each), and the B
-    // operand of group 2 qt (2 qt + 1) only if its column qg is that group, else zeros
+    // the codes of groups 2 qt and 2 qt + 1 of rows qg and qg + 8 (16 bytes each), and as its B
+    // operand pairs group 2 qt's x (as b0) if its column qg is that group, group 2 qt + 1's (as
+    // b1) if it is that one, else zeros: the staged layout gives each pair in one load
     const uint32_t bd_c0 = (uint32_t)(ring_c - smem) + qg * 128 + (((2 * qt) ^ qg) << 4);       // + stage * 2048
     const uint32_t bd_c1 = (uint32_t)(ring_c - smem) + qg * 128 + (((2 * qt + 1) ^ qg) << 4);
     const uint32_t xp_o = (uint32_t)(xp - smem);
     const bool bd_sel0 = qg == 2 * qt, bd_sel1 = qg == 2 * qt + 1;
-    const uint32_t bd_b0 = bd_sel0 ? xp_o + kBdZero + 2 * qt * kBdGroup : xp_o;       // + chunk offset if selected
-    const uint32_t bd_b1 = bd_sel1 ? xp_o + kBdZero + (2 * qt + 1) * kBdGroup : xp_o;
-    const uint32_t bd_m0 = bd_sel0 ? 0xffffffffu : 0u, bd_m1 = bd_sel1 ? 0xffffffffu : 0u;
+    const uint32_t bd_b = (bd_sel0 || bd_sel1) ? xp_o + kBdZero + qt * kBdPair + (bd_sel1 ? kBdPair / 2 : 0)
+                                               : xp_o + 32 * (qg >> 1);   // + chunk offset if selected
+    const uint32_t bd_m = (bd_sel0 || bd_sel1) ? 0xffffffffu : 0u;
     uint32_t st = 0;                // ring stage of the next item to compute
     int cs = 0;
 
@@ -610,10 +611,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
                     uint32_t xoff = (uint32_t)g.my_wk * kMChunkG * XG;   // B bytes of this warp's first chunk
                     uint32_t coff = (uint32_t)g.my_wk * kMChunkG * CG;   // C-table bytes
-                    // single column: this lane's two B-operand addresses, stepped per item by
-                    // the chunk step or by 0 (lanes that read the zero block)
-                    uint32_t bo0 = bd_b0 + (xoff & bd_m0), bo1 = bd_b1 + (xoff & bd_m1);
-                    const uint32_t xs0 = xstep & bd_m0, xs1 = xstep & bd_m1;
+                    // single column: this lane's B-operand address, stepped per item by the
+                    // chunk step or by 0 (lanes that read the zero region)
+                    uint32_t bo = bd_b + (xoff & bd_m);
+                    const uint32_t xs = xstep & bd_m;
                     int cl = 0;
                     for (int w = 0; w < n_win; ++w) {
                         int cl_end = g.my_chunks;
@@ -630,8 +631,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             if (w > 0) {   // the area now starts at group w gs
                                 xoff -= (uint32_t)gs * XG;
                                 coff -= (uint32_t)gs * CG;
-                                bo0 -= ((uint32_t)gs * XG) & bd_m0;
-                                bo1 -= ((uint32_t)gs * XG) & bd_m1;
+                                bo -= ((uint32_t)gs * XG) & bd_m;
                             }
                             // this warp's chunks c = my_wk + wk cl below the window's end
                             const int c_end = (w + 1) * (gs / kMChunkG);
@@ -685,28 +685,28 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 // then scales are never copied asynchronously: the loads above give 0)
                                 const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
                                 float d[4] = {cz.x, cz.y, cz.x, cz.y};
-                                const unsigned char *b0p = smem + bo0;
-                                const unsigned char *b1p = smem + bo1;
+                                const unsigned char *bp = smem + bo;
                                 const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
                                 const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
 #pragma unroll
                                 for (int t4 = 0; t4 < 4; ++t4) {
-                                    const uint4 x0 = *reinterpret_cast<const uint4 *>(b0p + 16 * t4);
-                                    const uint4 x1 = *reinterpret_cast<const uint4 *>(b1p + 16 * t4);
+                                    // (b0, b1) of steps 4 t4 .. 4 t4 + 3: (xa.x, xa.y), (xa.z, xa.w), (xb.x, xb.y), (xb.z, xb.w)
+                                    const uint4 xa = *reinterpret_cast<const uint4 *>(bp + 32 * t4);
+                                    const uint4 xb = *reinterpret_cast<const uint4 *>(bp + 32 * t4 + 16);
                                     const uint32_t wa = wa4[t4], wb = wb4[t4], wc = wc4[t4], wd = wd4[t4];
                                     const uint32_t was = wa >> 8, wbs = wb >> 8, wcs = wc >> 8, wds = wd >> 8;
                                     const uint32_t A0[4] = {wa & 0x000F000Fu, wb & 0x000F000Fu, wc & 0x000F000Fu,
                                                             wd & 0x000F000Fu};
-                                    mma_16816(d, A0, x0.x, x1.x, d[0], d[1], d[2], d[3]);
+                                    mma_16816(d, A0, xa.x, xa.y, d[0], d[1], d[2], d[3]);
                                     const uint32_t A1[4] = {was & 0x000F000Fu, wbs & 0x000F000Fu, wcs & 0x000F000Fu,
                                                             wds & 0x000F000Fu};
-                                    mma_16816(d, A1, x0.y, x1.y, d[0], d[1], d[2], d[3]);
+                                    mma_16816(d, A1, xa.z, xa.w, d[0], d[1], d[2], d[3]);
                                     const uint32_t A2[4] = {wa & 0x00F000F0u, wb & 0x00F000F0u, wc & 0x00F000F0u,
                                                             wd & 0x00F000F0u};
-                                    mma_16816(d, A2, x0.z, x1.z, d[0], d[1], d[2], d[3]);
+                                    mma_16816(d, A2, xb.x, xb.y, d[0], d[1], d[2], d[3]);
                                     const uint32_t A3[4] = {was & 0x00F000F0u, wbs & 0x00F000F0u, wcs & 0x00F000F0u,
                                                             wds & 0x00F000F0u};
-                                    mma_16816(d, A3, x0.w, x1.w, d[0], d[1], d[2], d[3]);
+                                    mma_16816(d, A3, xb.z, xb.w, d[0], d[1], d[2], d[3]);
                                 }
                                 acc[0][0] = fmaf(d[0], s00, acc[0][0]);
                                 acc[0][1] = fmaf(d[1], s01, acc[0][1]);
@@ -793,8 +793,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
                             xoff += xstep;
                             coff += cstep;
-                            bo0 += xs0;
-                            bo1 += xs1;
+                            bo += xs;
                         }
                     }
 

@@ -362,9 +362,9 @@ def test_decode_plan_pins(zt):
     # blocks of at most 8 tokens, each whole
     assert zt.pass_plan(9, 8192, 1)[2:4] == (0, 1)
     assert zt.pass_plan(12, 8192, 1)[2:4] == (0, 2) and zt.pass_plan(16, 8192, 129)[2:4] == (0, 2)
-    # single token: whole up to K = 65536 (8 warps from there), windows beyond
-    assert zt.pass_plan(1, 65536, 1)[2] == 0
-    assert zt.pass_plan(1, 131072, 1)[2] > 0
+    # single token: whole up to K ~ 40000 (144 staged bytes per group of 32), windows beyond
+    assert zt.pass_plan(1, 32768, 1)[2] == 0
+    assert zt.pass_plan(1, 65536, 1)[2] > 0 and zt.pass_plan(1, 131072, 1)[2] > 0
     # windows go with two CTAs per SM
     assert zt.pass_plan(16, 16384, 192)[0] == 2
 
