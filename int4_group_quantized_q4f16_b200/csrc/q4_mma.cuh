@@ -142,6 +142,13 @@ __host__ __device__ constexpr uint32_t bd_slot(int kk)   // the 32 bytes of piec
     return kBdZero + (kk >> 3) * kBdPair + ((kk >> 2) & 1) * (kBdPair / 2) + (kk & 3) * 32;
 }
 __host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
+// The single-column C table: per pair of groups (2p, 2p + 1) four floats (c_2p, c_2p+1, c_2p, c_2p+1), the C
+// operand quad of the lanes that hold that pair, in one 16-byte load; 2 floats per group.
+__device__ __forceinline__ void bd_c(float *x7, int g, float c)
+{
+    x7[(g >> 1) * 4 + (g & 1)] = c;
+    x7[(g >> 1) * 4 + (g & 1) + 2] = c;
+}
 
 // the four words o of piece kk, each beside a zero (after it in an even group, before it in an odd one)
 __device__ __forceinline__ void bd_store(unsigned char *xp, int kk, uint4 o)
@@ -161,7 +168,7 @@ __device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw)
 {
     for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += (int)blockDim.x) {
         bd_store(xp, Gw * 4 + j, make_uint4(0, 0, 0, 0));
-        if ((j & 3) == 0) x7[Gw + (j >> 2)] = 0.f;
+        if ((j & 3) == 0) bd_c(x7, Gw + (j >> 2), 0.f);
     }
 }
 
@@ -215,7 +222,7 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
     if (valid && (kk & 3) == 0) {
         const float c = part * (-7.0f * pow2f(-24));
         if (compact) {
-            x7[kk >> 2] = c;
+            bd_c(x7, kk >> 2, c);
         } else {
             const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
             float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;

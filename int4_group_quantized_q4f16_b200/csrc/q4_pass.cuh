@@ -120,7 +120,7 @@ __host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages
     const size_t ring = (size_t)MW * stages * kMStage + 1024;   // + alignment of the code stages
     // M = 1: the block-diagonal layout (a zero block, 80 bytes per group, one C float per group)
     const size_t xp = M == 1 ? (size_t)kBdZero + (size_t)round8(g_stage) * kBdGroup : (size_t)M * ((size_t)g_stage * 64 + 32);
-    const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 4 : (size_t)g_stage * NT * 64;
+    const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 8 : (size_t)g_stage * NT * 64;
     return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)red_floats * 4 + (size_t)n * sizeof(PassSeg) +
            (MW + 4) * sizeof(int) + 16 * sizeof(float);
 }
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     const size_t xp_bytes = ONE ? (size_t)kBdZero + (size_t)round8(a.g_stage) * kBdGroup
                                 : ((size_t)M * ((size_t)a.g_stage * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
-    float *red = x7 + (ONE ? (size_t)round8(a.g_stage) : (size_t)a.g_stage * NT * 16);
+    float *red = x7 + (ONE ? (size_t)round8(a.g_stage) * 2 : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMW * 8 * NT);
     PassSeg *segs = reinterpret_cast<PassSeg *>(red + a.red_floats);
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     // gives the swizzled chunk of group gl; row qg + 8 is 1024 bytes on
     const uint32_t wq_o = (uint32_t)(ring_c - smem) + qg * 128 + qt * 4 + (qg << 4);   // + stage * 2048
     const uint32_t sc_o = (uint32_t)(ring_s - smem) + qg * 16;                          // + stage * 256
-    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE ? qt * 8 : qt * 16);
+    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
     // M = 1 (block-diagonal): the mma's 8 columns are the item's 8 groups; lane (qg, qt) holds
     // the codes of groups 2 qt and 2 qt + 1 of rows qg and qg + 8 (16 bytes each), and as its B
     // operand pairs group 2 qt's x (as b0) if its column qg is that group, group 2 qt + 1's (as
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                 xb[nt] = (uint32_t)(xp - smem) + (uint32_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
             const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
             // per chunk: XG bytes of staged x per group, CG bytes of the C table per group
-            constexpr uint32_t XG = ONE ? kBdGroup : 64u, CG = ONE ? 4u : 64u * NT;
+            constexpr uint32_t XG = ONE ? kBdGroup : 64u, CG = ONE ? 8u : 64u * NT;
             const uint32_t xstep = (uint32_t)g.wk * kMChunkG * XG, cstep = (uint32_t)g.wk * kMChunkG * CG;
 
             // The WK partials of tiles [t0, t0 + tn) meet here in a fixed order
@@ -683,8 +683,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 }
                                 // (a chunk with missing groups, kc < 8, occurs only when K % 256 != 0, and
                                 // then scales are never copied asynchronously: the loads above give 0)
-                                const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
-                                float d[4] = {cz.x, cz.y, cz.x, cz.y};
+                                const float4 cz = *reinterpret_cast<const float4 *>(smem + x7_o + coff);
+                                float d[4] = {cz.x, cz.y, cz.z, cz.w};
                                 const unsigned char *bp = smem + bo;
                                 const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
                                 const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
