@@ -132,27 +132,50 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 // bytes apart, the odd one as [0, w_0, 0, w_1, ...].  The area starts with a
 // 224-byte zero region (the other lanes read 128 bytes of it, at 32 bytes per
 // quarter-warp); with these offsets the three addresses a quarter-warp reads
-// fall in distinct 16-byte bank groups.  The C table holds one float per
-// group; groups are padded with zeros to a multiple of 8 (one item).
+// fall in distinct 16-byte bank groups.  Groups are padded with zeros to a
+// multiple of 8 (one item).
+// That paired layout serves the 16-warp CTAs of a pass.  The CTAs of single calls (8
+// warps, several per SM, where the staging is a larger share of the call) use the plain
+// one: a 64-byte zero block, then group g's four 16-byte pieces at 64 + 80 g (80, not
+// 64: the lanes reading groups 2t and 2t + 1 then hit distinct banks), and one C float
+// per group; their b0 and b1 come from two loads.
 constexpr int kBdZero = 224;
 constexpr int kBdPair = 288;
 constexpr int kBdGroup = kBdPair / 2;   // bytes per group, for sizes and chunk steps
+constexpr int kBd1Zero = 64;
+constexpr int kBd1Group = 80;
 __host__ __device__ constexpr uint32_t bd_slot(int kk)   // the 32 bytes of piece kk (4 words, 4 zeros)
 {
     return kBdZero + (kk >> 3) * kBdPair + ((kk >> 2) & 1) * (kBdPair / 2) + (kk & 3) * 32;
 }
-__host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
-// The single-column C table: per pair of groups (2p, 2p + 1) four floats (c_2p, c_2p+1, c_2p, c_2p+1), the C
-// operand quad of the lanes that hold that pair, in one 16-byte load; 2 floats per group.
-__device__ __forceinline__ void bd_c(float *x7, int g, float c)
+__host__ __device__ constexpr uint32_t bd1_piece(int kk) { return kBd1Zero + (kk >> 2) * kBd1Group + (kk & 3) * 16; }
+// bytes of the single-column area and of its C table for g_stage groups
+__host__ __device__ constexpr size_t bd_area_bytes(int g8, bool paired)
 {
-    x7[(g >> 1) * 4 + (g & 1)] = c;
-    x7[(g >> 1) * 4 + (g & 1) + 2] = c;
+    return paired ? (size_t)kBdZero + (size_t)g8 * kBdGroup : (size_t)kBd1Zero + (size_t)g8 * kBd1Group;
+}
+__host__ __device__ constexpr size_t bd_ctable_bytes(int g8, bool paired) { return (size_t)g8 * (paired ? 8 : 4); }
+__host__ __device__ constexpr int round8(int g) { return (g + 7) & ~7; }
+// The single-column C table.  Paired layout: per pair of groups (2p, 2p + 1) four floats (c_2p, c_2p+1,
+// c_2p, c_2p+1), the C operand quad of the lanes that hold that pair, in one 16-byte load.  Plain layout:
+// one float per group.
+__device__ __forceinline__ void bd_c(float *x7, int g, float c, bool paired)
+{
+    if (paired) {
+        x7[(g >> 1) * 4 + (g & 1)] = c;
+        x7[(g >> 1) * 4 + (g & 1) + 2] = c;
+    } else {
+        x7[g] = c;
+    }
 }
 
 // the four words o of piece kk, each beside a zero (after it in an even group, before it in an odd one)
-__device__ __forceinline__ void bd_store(unsigned char *xp, int kk, uint4 o)
+__device__ __forceinline__ void bd_store(unsigned char *xp, int kk, uint4 o, bool paired)
 {
+    if (!paired) {
+        *reinterpret_cast<uint4 *>(xp + bd1_piece(kk)) = o;
+        return;
+    }
     uint4 *d = reinterpret_cast<uint4 *>(xp + bd_slot(kk));
     if ((kk >> 2) & 1) {
         d[0] = make_uint4(0u, o.x, 0u, o.y);
@@ -164,20 +187,20 @@ __device__ __forceinline__ void bd_store(unsigned char *xp, int kk, uint4 o)
 }
 
 // zero x and C of groups [Gw, round8(Gw)) in the single-column layout
-__device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw)
+__device__ __forceinline__ void bd_pad(unsigned char *xp, float *x7, int Gw, bool paired)
 {
     for (int j = threadIdx.x; j < (round8(Gw) - Gw) * 4; j += (int)blockDim.x) {
-        bd_store(xp, Gw * 4 + j, make_uint4(0, 0, 0, 0));
-        if ((j & 3) == 0) bd_c(x7, Gw + (j >> 2), 0.f);
+        bd_store(xp, Gw * 4 + j, make_uint4(0, 0, 0, 0), paired);
+        if ((j & 3) == 0) bd_c(x7, Gw + (j >> 2), 0.f, paired);
     }
 }
 
 // Byte offset of piece kk (8 activations) of column m in the staged area; with a
 // single column (compact) the first 16 bytes of the piece's slot, where the norm
 // prologue keeps h until the same thread turns it into x.
-__device__ __forceinline__ size_t x_piece(int m, int kk, size_t nstride, bool compact)
+__device__ __forceinline__ size_t x_piece(int m, int kk, size_t nstride, bool compact, bool paired)
 {
-    return compact ? (size_t)bd_slot(kk) : (size_t)m * nstride + (size_t)kk * 16;
+    return compact ? (size_t)(paired ? bd_slot(kk) : bd1_piece(kk)) : (size_t)m * nstride + (size_t)kk * 16;
 }
 
 // Stage x in mma-B order: for column n and group g, 64 bytes = for t = 0..3:
@@ -190,7 +213,7 @@ __device__ __forceinline__ size_t x_piece(int m, int kk, size_t nstride, bool co
 // the CTA takes 8 activations of one column per round; the 4 threads of a
 // group are adjacent lanes.  Callers synchronise before reading.
 __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool valid, unsigned char *xp,
-                                            float *x7, size_t nstride, int NT, bool compact)
+                                            float *x7, size_t nstride, int NT, bool compact, bool paired)
 {
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     float part = 0.f;
@@ -205,8 +228,8 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
         __half2 q37 = __hmul2(*reinterpret_cast<__half2 *>(&h37), sixteenth);
         o.z = *reinterpret_cast<uint32_t *>(&q15);
         o.w = *reinterpret_cast<uint32_t *>(&q37);
-        if (compact) bd_store(xp, kk, o);
-        else *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, false)) = o;
+        if (compact) bd_store(xp, kk, o, paired);
+        else *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, false, false)) = o;
         const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
         float v[8];
 #pragma unroll
@@ -222,7 +245,7 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
     if (valid && (kk & 3) == 0) {
         const float c = part * (-7.0f * pow2f(-24));
         if (compact) {
-            bd_c(x7, kk >> 2, c);
+            bd_c(x7, kk >> 2, c, paired);
         } else {
             const int g = kk >> 2, nt = m >> 3, t = (m & 7) >> 1, e = m & 1;
             float *cv = x7 + (((size_t)g * NT + nt) * 4 + t) * 4;
@@ -236,7 +259,7 @@ __device__ __forceinline__ void stage_x_one(const uint4 raw, int m, int kk, bool
 // further.  Gs: groups per staged column (the n-stride is Gs * 64 + 32 bytes);
 // the whole K is Gw = Gs = K / 32, a K window fewer groups.
 __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ldx, unsigned char *xp, float *x7,
-                                            int M, int Gw, int Gs, int NT)
+                                            int M, int Gw, int Gs, int NT, bool paired = false)
 {
     const int K8 = Gw * 4;                     // 8-element pieces per row: groups never straddle a column
     const int total = M * K8;
@@ -261,10 +284,10 @@ __device__ __forceinline__ void stage_x_mma(const __half *__restrict__ x, int ld
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
         if (v0) r0 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m0 * ldx + 8 * k0));
         if (v1) r1 = __ldcg(reinterpret_cast<const uint4 *>(x + (size_t)m1 * ldx + 8 * k1));
-        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact, paired);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact, paired);
     }
-    if (compact) bd_pad(xp, x7, Gw);
+    if (compact) bd_pad(xp, x7, Gw, paired);
 }
 
 // Residual add + RMSNorm ahead of a projection (the pages' add_norm step:
@@ -284,7 +307,7 @@ __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
 
 __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dlt, const __half *gamma, float eps,
                                              __half *res_out, __half *x_out, unsigned char *xp, float *x7,
-                                             float *scratch, int M, int K, int G, int NT)
+                                             float *scratch, int M, int K, int G, int NT, bool paired = false)
 {
     const int K8 = K >> 3;
     const size_t nstride = (size_t)G * 64 + 32;
@@ -300,7 +323,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
                 h.z = hadd2_u32(h.z, d.z);
                 h.w = hadd2_u32(h.w, d.w);
             }
-            *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, M == 1)) = h;
+            *reinterpret_cast<uint4 *>(xp + x_piece(m, kk, nstride, M == 1, paired)) = h;
             if (res_out) *reinterpret_cast<uint4 *>(res_out + (size_t)m * K + 8 * kk) = h;
             const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
 #pragma unroll
@@ -332,7 +355,7 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         cv[2 + e] = 0.f;
     }
     auto normalise = [&](int m, int kk) {
-        const uint4 h = *reinterpret_cast<const uint4 *>(xp + x_piece(m, kk, nstride, compact));
+        const uint4 h = *reinterpret_cast<const uint4 *>(xp + x_piece(m, kk, nstride, compact, paired));
         const uint4 g = __ldcg(reinterpret_cast<const uint4 *>(gamma + 8 * kk));
         const float r = scratch[kMWMax + m];
         const __half2 *hh = reinterpret_cast<const __half2 *>(&h);
@@ -355,10 +378,10 @@ __device__ __forceinline__ void stage_x_norm(const __half *res, const __half *dl
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
         if (v0) r0 = normalise(m0, k0);
         if (v1) r1 = normalise(m1, k1);
-        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact, paired);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact, paired);
     }
-    if (compact) bd_pad(xp, x7, G);
+    if (compact) bd_pad(xp, x7, G, paired);
 }
 
 // The same prologue for a projection whose activations are staged in K
@@ -407,7 +430,8 @@ __device__ __forceinline__ void norm_rows(const __half *res, const __half *dlt, 
 
 __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __half *dlt, const __half *gamma,
                                                     __half *x_out, const float *rn, unsigned char *xp, float *x7,
-                                                    int M, int K, int g0, int Gw, int Gs, int NT)
+                                                    int M, int K, int g0, int Gw, int Gs, int NT,
+                                                    bool paired = false)
 {
     const int K8 = Gw * 4, k8_0 = g0 * 4;
     const int total = M * K8;
@@ -453,10 +477,10 @@ __device__ __forceinline__ void stage_x_norm_window(const __half *res, const __h
         uint4 r0 = make_uint4(0, 0, 0, 0), r1 = make_uint4(0, 0, 0, 0);
         if (v0) r0 = normalise(m0, k0);
         if (v1) r1 = normalise(m1, k1);
-        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact);
-        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact);
+        stage_x_one(r0, m0, k0, v0, xp, x7, nstride, NT, compact, paired);
+        if (base + (int)blockDim.x < total) stage_x_one(r1, m1, k1, v1, xp, x7, nstride, NT, compact, paired);
     }
-    if (compact) bd_pad(xp, x7, Gw);
+    if (compact) bd_pad(xp, x7, Gw, paired);
 }
 
 }  // namespace zt

@@ -119,8 +119,8 @@ __host__ __device__ inline size_t pass_smem_bytes(int M, int g_stage, int stages
 {
     const size_t ring = (size_t)MW * stages * kMStage + 1024;   // + alignment of the code stages
     // M = 1: the block-diagonal layout (a zero block, 80 bytes per group, one C float per group)
-    const size_t xp = M == 1 ? (size_t)kBdZero + (size_t)round8(g_stage) * kBdGroup : (size_t)M * ((size_t)g_stage * 64 + 32);
-    const size_t x7 = M == 1 ? (size_t)round8(g_stage) * 8 : (size_t)g_stage * NT * 64;
+    const size_t xp = M == 1 ? bd_area_bytes(round8(g_stage), MW == 16) : (size_t)M * ((size_t)g_stage * 64 + 32);
+    const size_t x7 = M == 1 ? bd_ctable_bytes(round8(g_stage), MW == 16) : (size_t)g_stage * NT * 64;
     return ring + ((xp + 15) & ~(size_t)15) + x7 + (size_t)red_floats * 4 + (size_t)n * sizeof(PassSeg) +
            (MW + 4) * sizeof(int) + 16 * sizeof(float);
 }
@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
 {
     static_assert(MW == 8 || MW == 16, "8 or 16 warps per CTA");
     constexpr int kMW = MW, kMThreads = MW * 32, LW = MW == 16 ? 4 : 3;
+    constexpr bool PAIRED = ONE && MW == 16;   // the paired single-column layout (q4_mma.cuh)
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     static_assert(!ONE || NT == 1, "one column fits one n-tile");
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -292,10 +293,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     unsigned char *ring_c = codes + (size_t)warp * S * kMCodeStage;
     unsigned char *ring_s = codes + (size_t)kMW * S * kMCodeStage + (size_t)warp * S * kMScaleStage;
     unsigned char *xp = codes + (size_t)kMW * S * kMStage;
-    const size_t xp_bytes = ONE ? (size_t)kBdZero + (size_t)round8(a.g_stage) * kBdGroup
+    const size_t xp_bytes = ONE ? bd_area_bytes(round8(a.g_stage), PAIRED)
                                 : ((size_t)M * ((size_t)a.g_stage * 64 + 32) + 15) & ~(size_t)15;
     float *x7 = reinterpret_cast<float *>(xp + xp_bytes);
-    float *red = x7 + (ONE ? (size_t)round8(a.g_stage) * 2 : (size_t)a.g_stage * NT * 16);
+    float *red = x7 + (ONE ? bd_ctable_bytes(round8(a.g_stage), PAIRED) / 4 : (size_t)a.g_stage * NT * 16);
     float *bvs = red;                                           // LM-head maxima reuse red
     int *bis = reinterpret_cast<int *>(bvs + kMW * 8 * NT);
     PassSeg *segs = reinterpret_cast<PassSeg *>(red + a.red_floats);
@@ -339,7 +340,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
         const unsigned ball = __ballot_sync(0xffffffffu, has);
         if (lane == 0) wcount[warp] = __popc(ball);
         if (tid == 0) *abort_flag = 0;
-        if (ONE && tid < kBdZero / 16) reinterpret_cast<uint4 *>(xp)[tid] = make_uint4(0, 0, 0, 0);   // the zero block
+        if (ONE && tid < (PAIRED ? kBdZero : kBd1Zero) / 16)
+            reinterpret_cast<uint4 *>(xp)[tid] = make_uint4(0, 0, 0, 0);   // the zero region
         __syncthreads();
         if (has) {
             int idx = __popc(ball & ((1u << lane) - 1u));
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     // gives the swizzled chunk of group gl; row qg + 8 is 1024 bytes on
     const uint32_t wq_o = (uint32_t)(ring_c - smem) + qg * 128 + qt * 4 + (qg << 4);   // + stage * 2048
     const uint32_t sc_o = (uint32_t)(ring_s - smem) + qg * 16;                          // + stage * 256
-    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + qt * 16;
+    const uint32_t x7_o = (uint32_t)(reinterpret_cast<unsigned char *>(x7) - smem) + (ONE && !PAIRED ? qt * 8 : qt * 16);
     // M = 1 (block-diagonal): the mma's 8 columns are the item's 8 groups; lane (qg, qt) holds
     // the codes of groups 2 qt and 2 qt + 1 of rows qg and qg + 8 (16 bytes each), and as its B
     // operand pairs group 2 qt's x (as b0) if its column qg is that group, group 2 qt + 1's (as
@@ -484,9 +486,13 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     const uint32_t bd_c1 = (uint32_t)(ring_c - smem) + qg * 128 + (((2 * qt + 1) ^ qg) << 4);
     const uint32_t xp_o = (uint32_t)(xp - smem);
     const bool bd_sel0 = qg == 2 * qt, bd_sel1 = qg == 2 * qt + 1;
+    // paired layout: one address per lane; plain layout: one per B half (b0 from group 2 qt, b1 from 2 qt + 1)
     const uint32_t bd_b = (bd_sel0 || bd_sel1) ? xp_o + kBdZero + qt * kBdPair + (bd_sel1 ? kBdPair / 2 : 0)
                                                : xp_o + 32 * (qg >> 1);   // + chunk offset if selected
     const uint32_t bd_m = (bd_sel0 || bd_sel1) ? 0xffffffffu : 0u;
+    const uint32_t bd_b0 = bd_sel0 ? xp_o + kBd1Zero + 2 * qt * kBd1Group : xp_o;
+    const uint32_t bd_b1 = bd_sel1 ? xp_o + kBd1Zero + (2 * qt + 1) * kBd1Group : xp_o;
+    const uint32_t bd_m0 = bd_sel0 ? 0xffffffffu : 0u, bd_m1 = bd_sel1 ? 0xffffffffu : 0u;
     uint32_t st = 0;                // ring stage of the next item to compute
     int cs = 0;
 
@@ -521,9 +527,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
             if (!windowed) {
                 if (P.norm) {
                     stage_x_norm(pres, pdlt, P.gamma, P.eps, writer ? pres_out : nullptr,
-                                 writer ? px_out : nullptr, xp, x7, red, M, P.K, G, NT);
+                                 writer ? px_out : nullptr, xp, x7, red, M, P.K, G, NT, PAIRED);
                 } else {
-                    stage_x_mma(px, P.K, xp, x7, M, G, G, NT);
+                    stage_x_mma(px, P.K, xp, x7, M, G, G, NT, PAIRED);
                 }
                 consumer_sync();
             } else if (P.norm) {
@@ -538,7 +544,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                 xb[nt] = (uint32_t)(xp - smem) + (uint32_t)min(qg + 8 * nt, M - 1) * nstride + qt * 16;
             const int kc_last = g.my_tiles > 0 ? pass_last_kc(g, G) : kMChunkG;
             // per chunk: XG bytes of staged x per group, CG bytes of the C table per group
-            constexpr uint32_t XG = ONE ? kBdGroup : 64u, CG = ONE ? 8u : 64u * NT;
+            constexpr uint32_t XG = ONE ? (PAIRED ? kBdGroup : kBd1Group) : 64u,
+                               CG = ONE ? (PAIRED ? 8u : 4u) : 64u * NT;
             const uint32_t xstep = (uint32_t)g.wk * kMChunkG * XG, cstep = (uint32_t)g.wk * kMChunkG * CG;
 
             // The WK partials of tiles [t0, t0 + tn) meet here in a fixed order
@@ -615,6 +622,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     // chunk step or by 0 (lanes that read the zero region)
                     uint32_t bo = bd_b + (xoff & bd_m);
                     const uint32_t xs = xstep & bd_m;
+                    uint32_t bo0 = bd_b0 + (xoff & bd_m0), bo1 = bd_b1 + (xoff & bd_m1);
+                    const uint32_t xs0 = xstep & bd_m0, xs1 = xstep & bd_m1;
                     int cl = 0;
                     for (int w = 0; w < n_win; ++w) {
                         int cl_end = g.my_chunks;
@@ -624,14 +633,16 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             const int g0 = w * gs, gn = min(gs, G - g0);
                             if (P.norm)
                                 stage_x_norm_window(pres, pdlt, P.gamma, (writer && tl == 0) ? px_out : nullptr,
-                                                    rn, xp, x7, M, P.K, g0, gn, gs, NT);
+                                                    rn, xp, x7, M, P.K, g0, gn, gs, NT, PAIRED);
                             else
-                                stage_x_mma(px + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT);
+                                stage_x_mma(px + (size_t)g0 * kGroup, P.K, xp, x7, M, gn, gs, NT, PAIRED);
                             consumer_sync();
                             if (w > 0) {   // the area now starts at group w gs
                                 xoff -= (uint32_t)gs * XG;
                                 coff -= (uint32_t)gs * CG;
                                 bo -= ((uint32_t)gs * XG) & bd_m;
+                                bo0 -= ((uint32_t)gs * XG) & bd_m0;
+                                bo1 -= ((uint32_t)gs * XG) & bd_m1;
                             }
                             // this warp's chunks c = my_wk + wk cl below the window's end
                             const int c_end = (w + 1) * (gs / kMChunkG);
@@ -683,16 +694,32 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 }
                                 // (a chunk with missing groups, kc < 8, occurs only when K % 256 != 0, and
                                 // then scales are never copied asynchronously: the loads above give 0)
-                                const float4 cz = *reinterpret_cast<const float4 *>(smem + x7_o + coff);
-                                float d[4] = {cz.x, cz.y, cz.z, cz.w};
+                                float d[4];
+                                if constexpr (PAIRED) {
+                                    const float4 cz = *reinterpret_cast<const float4 *>(smem + x7_o + coff);
+                                    d[0] = cz.x; d[1] = cz.y; d[2] = cz.z; d[3] = cz.w;
+                                } else {
+                                    const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
+                                    d[0] = cz.x; d[1] = cz.y; d[2] = cz.x; d[3] = cz.y;
+                                }
                                 const unsigned char *bp = smem + bo;
+                                const unsigned char *b0p = smem + bo0, *b1p = smem + bo1;
                                 const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
                                 const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
 #pragma unroll
                                 for (int t4 = 0; t4 < 4; ++t4) {
-                                    // (b0, b1) of steps 4 t4 .. 4 t4 + 3: (xa.x, xa.y), (xa.z, xa.w), (xb.x, xb.y), (xb.z, xb.w)
-                                    const uint4 xa = *reinterpret_cast<const uint4 *>(bp + 32 * t4);
-                                    const uint4 xb = *reinterpret_cast<const uint4 *>(bp + 32 * t4 + 16);
+                                    // (b0, b1) of steps 4 t4 .. 4 t4 + 3: paired, (xa.x, xa.y), (xa.z, xa.w),
+                                    // (xb.x, xb.y), (xb.z, xb.w); plain, (xa.x, xb.x), (xa.y, xb.y), ...
+                                    uint4 xa, xb;
+                                    if constexpr (PAIRED) {
+                                        xa = *reinterpret_cast<const uint4 *>(bp + 32 * t4);
+                                        xb = *reinterpret_cast<const uint4 *>(bp + 32 * t4 + 16);
+                                    } else {
+                                        const uint4 x0 = *reinterpret_cast<const uint4 *>(b0p + 16 * t4);
+                                        const uint4 x1 = *reinterpret_cast<const uint4 *>(b1p + 16 * t4);
+                                        xa = make_uint4(x0.x, x1.x, x0.y, x1.y);
+                                        xb = make_uint4(x0.z, x1.z, x0.w, x1.w);
+                                    }
                                     const uint32_t wa = wa4[t4], wb = wb4[t4], wc = wc4[t4], wd = wd4[t4];
                                     const uint32_t was = wa >> 8, wbs = wb >> 8, wcs = wc >> 8, wds = wd >> 8;
                                     const uint32_t A0[4] = {wa & 0x000F000Fu, wb & 0x000F000Fu, wc & 0x000F000Fu,
@@ -793,7 +820,11 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                             st = (st + 1 == (uint32_t)S) ? 0u : st + 1;
                             xoff += xstep;
                             coff += cstep;
-                            bo += xs;
+                            if constexpr (PAIRED) bo += xs;
+                            else {
+                                bo0 += xs0;
+                                bo1 += xs1;
+                            }
                         }
                     }
 

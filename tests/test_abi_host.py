@@ -362,9 +362,12 @@ def test_decode_plan_pins(zt):
     # blocks of at most 8 tokens, each whole
     assert zt.pass_plan(9, 8192, 1)[2:4] == (0, 1)
     assert zt.pass_plan(12, 8192, 1)[2:4] == (0, 2) and zt.pass_plan(16, 8192, 129)[2:4] == (0, 2)
-    # single token: whole up to K ~ 40000 (144 staged bytes per group of 32), windows beyond
-    assert zt.pass_plan(1, 32768, 1)[2] == 0
-    assert zt.pass_plan(1, 65536, 1)[2] > 0 and zt.pass_plan(1, 131072, 1)[2] > 0
+    # single token: 16 warps (paired layout, 144 staged bytes per group of 32) up to K ~ 30000,
+    # then 8 warps (plain layout, 80 bytes per group) whole up to K ~ 72000, windows beyond
+    assert zt.pass_plan(1, 16384, 129)[2:] == (0, 1, 16)
+    assert zt.pass_plan(1, 32768, 129)[2:] == (0, 1, 8)
+    assert zt.pass_plan(1, 65536, 1)[2] == 0
+    assert zt.pass_plan(1, 98304, 1)[2] > 0 and zt.pass_plan(1, 131072, 1)[2] > 0
     # windows go with two CTAs per SM
     assert zt.pass_plan(16, 16384, 192)[0] == 2
 
