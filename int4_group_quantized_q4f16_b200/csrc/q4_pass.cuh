@@ -694,7 +694,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 }
                                 // (a chunk with missing groups, kc < 8, occurs only when K % 256 != 0, and
                                 // then scales are never copied asynchronously: the loads above give 0)
-                                float d[4];
+                                // two accumulators (the steps of codes {0,4} and 16 {1,5} -> d, of {2,6} and
+                                // 16 {3,7} -> e): two chains of 8 dependent mma instead of one of 16
+                                float d[4], e[4] = {0.f, 0.f, 0.f, 0.f};
                                 if constexpr (PAIRED) {
                                     const float4 cz = *reinterpret_cast<const float4 *>(smem + x7_o + coff);
                                     d[0] = cz.x; d[1] = cz.y; d[2] = cz.z; d[3] = cz.w;
@@ -727,18 +729,18 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                     mma_16816(d, A0, xa.x, xa.y, d[0], d[1], d[2], d[3]);
                                     const uint32_t A1[4] = {was & 0x000F000Fu, wbs & 0x000F000Fu, wcs & 0x000F000Fu,
                                                             wds & 0x000F000Fu};
-                                    mma_16816(d, A1, xa.z, xa.w, d[0], d[1], d[2], d[3]);
+                                    mma_16816(e, A1, xa.z, xa.w, e[0], e[1], e[2], e[3]);
                                     const uint32_t A2[4] = {wa & 0x00F000F0u, wb & 0x00F000F0u, wc & 0x00F000F0u,
                                                             wd & 0x00F000F0u};
                                     mma_16816(d, A2, xb.x, xb.y, d[0], d[1], d[2], d[3]);
                                     const uint32_t A3[4] = {was & 0x00F000F0u, wbs & 0x00F000F0u, wcs & 0x00F000F0u,
                                                             wds & 0x00F000F0u};
-                                    mma_16816(d, A3, xb.z, xb.w, d[0], d[1], d[2], d[3]);
+                                    mma_16816(e, A3, xb.z, xb.w, e[0], e[1], e[2], e[3]);
                                 }
-                                acc[0][0] = fmaf(d[0], s00, acc[0][0]);
-                                acc[0][1] = fmaf(d[1], s01, acc[0][1]);
-                                acc[0][2] = fmaf(d[2], s10, acc[0][2]);
-                                acc[0][3] = fmaf(d[3], s11, acc[0][3]);
+                                acc[0][0] = fmaf(d[0] + e[0], s00, acc[0][0]);
+                                acc[0][1] = fmaf(d[1] + e[1], s01, acc[0][1]);
+                                acc[0][2] = fmaf(d[2] + e[2], s10, acc[0][2]);
+                                acc[0][3] = fmaf(d[3] + e[3], s11, acc[0][3]);
                             } else {
                                 uint4 sg, sg8;     // scales of rows qg and qg + 8 for the item's 8 groups
                                 if (sasync) {
