@@ -282,6 +282,32 @@ ZT_API int zt_q4_pass_test_withhold(const zt_q4_proj *projs, int n, int M, void 
                                     void *stream);
 
 /*
+ * BOUNDS-CHECKED BUILD.  The same sources compiled with -DZT_Q4_CHECKED
+ * (libzt_q4_checked.so beside libzt_q4.so) compare, in the pass kernel that
+ * serves every decode entry point, each computed global index (weight and
+ * scale copies and loads, output and LM-head workspace stores) and each read
+ * and write of its shared partial buffer with the extent of its buffer.  An
+ * index outside it sets bit ZT_Q4_ERR_BOUNDS (2) of the error word that
+ * zt_q4_pass_errors reads (bit 0 is the expired bounded wait) and the access
+ * is skipped: no assert, no trap, the context stays usable.  The activation
+ * staging (m < M, k < K over x with row stride K) is not instrumented.
+ *
+ * zt_q4_build_flags: ZT_Q4_BUILD_CHECKED when this library is the checked
+ * build, else 0.
+ *
+ * zt_q4_pass_test_cut (TEST HOOK, checked build only; ZT_ERR_UNSUPPORTED in
+ * the default one): zt_q4_pass with the weight extent of every projection
+ * taken `rows` rows short, so that the copies of its last rows fail their
+ * check (and are skipped) while the buffers themselves stay whole: the error
+ * bit is set and nothing out of bounds is read.  rows < 1: ZT_ERR_INVALID_ARG.
+ */
+#define ZT_Q4_BUILD_CHECKED 1
+#define ZT_Q4_ERR_BOUNDS 2u
+ZT_API int zt_q4_build_flags(void);
+ZT_API int zt_q4_pass_test_cut(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes,
+                               void *stream, int rows);
+
+/*
  * BATCHED PREFILL (M > 16 tokens; any M >= 1 is accepted)
  *
  * Zero-TVM write-up, limitations section: the project ships shaders for
@@ -366,7 +392,7 @@ ZT_API const char *zt_q4_strerror(int status);
 ZT_API const char *zt_q4_last_cuda_error(void);
 
 /* Library ABI version, (major << 16) | minor.  1.3 added zt_q4_pass_plan; 1.4 its column_blocks; 1.5 its
- * warps_per_cta. */
+ * warps_per_cta; 1.6 zt_q4_build_flags and zt_q4_pass_test_cut. */
 ZT_API int zt_q4_version(void);
 
 #ifdef __cplusplus

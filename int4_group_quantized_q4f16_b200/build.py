@@ -1,4 +1,5 @@
-"""Build the CUDA library in-tree: nvcc for sm_100a -> libzt_q4.so beside this file.
+"""Build the CUDA library in-tree: nvcc for sm_100a -> libzt_q4.so beside this file,
+and the bounds-checked build of the same sources (-DZT_Q4_CHECKED) -> libzt_q4_checked.so.
 
 Run ``python -m int4_group_quantized_q4f16_b200.build``.  The library links the
 CUDA runtime statically, so it loads on a machine without a GPU (every entry
@@ -15,6 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libzt_q4.so")
+LIB_CHECKED = os.path.join(PKG, "libzt_q4_checked.so")
 SOURCES = ["zt_q4.cu"]
 HEADERS = ["q4_common.cuh", "q4_mma.cuh", "q4_pass.cuh", "q4_gemm_tc.cuh"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
@@ -40,6 +42,10 @@ def stale(lib: str = LIB) -> bool:
     return any(os.path.getmtime(s) > t for s in sources())
 
 
+def build_checked(force: bool = False, verbose: bool = False) -> str:
+    return build(force, verbose, LIB_CHECKED, ["-DZT_Q4_CHECKED"])
+
+
 def build(force: bool = False, verbose: bool = False, out: str = LIB, extra=()) -> str:
     if not force and not stale(out):
         return out
@@ -55,3 +61,4 @@ def build(force: bool = False, verbose: bool = False, out: str = LIB, extra=()) 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_checked(force="--force" in sys.argv, verbose=True))

@@ -37,6 +37,25 @@ namespace zt {
 constexpr int kPassMax = 192;                       // projections per launch
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr unsigned kErrWaitExpired = 1u;
+constexpr unsigned kErrBounds = 2u;
+
+// Bounds-checked build (compiled with -DZT_Q4_CHECKED): before every global access whose
+// address the kernel computes (weight and scale copies and loads, output and workspace
+// stores) and every read of the shared partial buffer, the index is compared with the
+// extent of its buffer; an index outside it sets kErrBounds in the error word and the
+// access is skipped, so a wrong index shows as an error bit, never as a fault.  The
+// default build compiles the comparisons out.
+#ifdef ZT_Q4_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// weight rows of a projection: gate_up and RoPE projections hold two rows per output
+__host__ __device__ constexpr int pass_weight_rows(int kind, int N)
+{
+    return (kind == kEpiGateUp || kind == kEpiRope) ? 2 * N : N;
+}
 
 struct PassProj {
     const uint4 *qw;            // [rows][G] 16-byte chunks
@@ -80,6 +99,8 @@ struct PassArgs {
     unsigned int *error;        // error bits
     int withhold;               // test hook: CTA 0 does not count this phase done (-1: none)
     int red_floats;             // size of the WK partial buffer (floats)
+    int chk_cut;                // test hook of the checked build: weight rows taken off every projection's
+                                // extent, so that the last rows' checks fire (0: none)
     int colsplit;               // M > 8 as two column blocks: CTAs 2s and 2s + 1 take row share s, tokens
                                 // 0 .. ceil(M/2) - 1 and the rest (each an M <= 8 problem of 5..8 tokens)
     // What every CTA reads to find its rows, kept apart from p[] in dense arrays: a warp
@@ -275,6 +296,15 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     static_assert(S >= 2 && S <= kPassMaxStages, "ring depth");
     static_assert(!ONE || NT == 1, "one column fits one n-tile");
     extern __shared__ __align__(1024) unsigned char smem[];
+    // checked build: false (and the error bit) for an index outside its buffer; else always true
+    auto chk = [&](bool in_bounds) -> bool {
+        if constexpr (kChecked) {
+            if (!in_bounds && a.error) atomicOr(a.error, kErrBounds);
+            return in_bounds;
+        } else {
+            return true;
+        }
+    };
     // this CTA's tokens (columns) and row share: with the column split, tokens m0 .. m0 + M - 1
     // of the list's Mt (the first ceil(Mt / 2) or the other floor(Mt / 2), so never a single
     // column: the staging helpers take M == 1 for the block-diagonal layout of ONE), and
@@ -377,6 +407,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
     int is_kc_last = kMChunkG;      // groups of the tile's last chunk
     int is_step = 0;                // uint4 per chunk step (WK chunks of 8 groups)
     int is_sstep = 0;               // scale elements per chunk step
+    const uint4 *is_qlo = nullptr, *is_qhi = nullptr;      // checked build: the weight buffer
+    const __half *is_slo = nullptr, *is_shi = nullptr;     // and the scale buffer of the segment
     uint32_t is_st = 0;             // ring stage of the next item to issue
     int is_o0 = 0, is_rstep = 0;    // current tile's first output, outputs per tile step
     PassGeo ig{};
@@ -402,6 +434,13 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
         const int row = pass_slot_row(P.kind, P.N, P.rope_d, ig.o_end, is_o0, lane & 15, ok_s);
         ok_s = ok_s && lane < kMTileRows && P.scales_async;
         src_s = P.scales + (size_t)row * (P.G >> P.gsh) + ((ig.my_wk * kMChunkG) >> P.gsh);
+        if constexpr (kChecked) {
+            const int rows = pass_weight_rows(P.kind, P.N);
+            is_qlo = P.qw;
+            is_qhi = P.qw + (size_t)max(rows - a.chk_cut, 0) * P.G;
+            is_slo = P.scales;
+            is_shi = P.scales + (size_t)rows * (P.G >> P.gsh);
+        }
         is_gsh = P.gsh;
         is_sstep = is_step >> P.gsh;
         is_chunks = ig.my_chunks;
@@ -436,9 +475,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
         if (is_chunks > 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (ok_w[i])
+                if (ok_w[i] && chk(src_w[i] >= is_qlo && src_w[i] < is_qhi))
                     cp_async16_u32(((i & 1) ? piece_u1 : piece_u0) + (is_st << 11) + (i >> 1) * 1024, src_w[i]);
-            if (ok_s) {
+            if (ok_s && chk(src_s >= is_slo && src_s + (16 >> (1 + is_gsh)) <= is_shi)) {
                 // the item's 8 blocks of 32 share 8, 4 or 2 scales: 16, 8 or 4 bytes per row
                 if (is_gsh == 0) cp_async16_u32(scale_u + (is_st << 8), src_s);
                 else if (is_gsh == 1) cp_async8_u32(scale_u + (is_st << 8), src_s);
@@ -466,7 +505,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
         // written only after the wait: the kernel ahead on the stream may be
         // the argmax reduction of an earlier call that reads the same scratch
         const PassProj &P = a.p[tid];
-        for (int m = 0; m < Mt; ++m) {
+        for (int m = 0; m < Mt && chk(blockIdx.x < (unsigned)kMaxCtas); ++m) {
             P.ws_val[(size_t)blockIdx.x * Mt + m] = -INFINITY;
             pass_ws_idx(P, Mt)[(size_t)blockIdx.x * Mt + m] = 0x7fffffff;
         }
@@ -562,6 +601,7 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     const int r = vo / PC, m = vo - (vo / PC) * PC;
                     const int nn = g.o_begin + (t0 + tt) * g.rout + r;
                     if (nn >= g.o_end || m >= M) continue;
+                    if (!chk(nn < N && (size_t)(tt + 1) * g.wk * PART <= (size_t)a.red_floats)) continue;
                     const float *rp = red + (size_t)tt * g.wk * PART;
                     float y = 0.f, u = 0.f;
                     for (int k2 = 0; k2 < g.wk; ++k2) {
@@ -621,9 +661,9 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     // single column: this lane's B-operand address, stepped per item by the
                     // chunk step or by 0 (lanes that read the zero region)
                     uint32_t bo = bd_b + (xoff & bd_m);
-                    const uint32_t xs = xstep & bd_m;
+                    [[maybe_unused]] const uint32_t xs = xstep & bd_m;
                     uint32_t bo0 = bd_b0 + (xoff & bd_m0), bo1 = bd_b1 + (xoff & bd_m1);
-                    const uint32_t xs0 = xstep & bd_m0, xs1 = xstep & bd_m1;
+                    [[maybe_unused]] const uint32_t xs0 = xstep & bd_m0, xs1 = xstep & bd_m1;
                     int cl = 0;
                     for (int w = 0; w < n_win; ++w) {
                         int cl_end = g.my_chunks;
@@ -687,10 +727,15 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                     const __half *p0 = P.scales + (size_t)r0 * (G >> gsh);
                                     const __half *p1 = P.scales + (size_t)r1 * (G >> gsh);
                                     const int b = c * kMChunkG + 2 * qt;
-                                    s00 = 2 * qt < kc ? __half2float(p0[b >> gsh]) : 0.f;
-                                    s10 = 2 * qt < kc ? __half2float(p1[b >> gsh]) : 0.f;
-                                    s01 = 2 * qt + 1 < kc ? __half2float(p0[(b + 1) >> gsh]) : 0.f;
-                                    s11 = 2 * qt + 1 < kc ? __half2float(p1[(b + 1) >> gsh]) : 0.f;
+                                    const int wr = pass_weight_rows(kind, N), sr = G >> gsh;
+                                    const bool e0 = 2 * qt < kc && chk(r0 >= 0 && r0 < wr && r1 >= 0 && r1 < wr &&
+                                                                      (b >> gsh) < sr);
+                                    const bool e1 = 2 * qt + 1 < kc && chk(r0 >= 0 && r0 < wr && r1 >= 0 &&
+                                                                          r1 < wr && ((b + 1) >> gsh) < sr);
+                                    s00 = e0 ? __half2float(p0[b >> gsh]) : 0.f;
+                                    s10 = e0 ? __half2float(p1[b >> gsh]) : 0.f;
+                                    s01 = e1 ? __half2float(p0[(b + 1) >> gsh]) : 0.f;
+                                    s11 = e1 ? __half2float(p1[(b + 1) >> gsh]) : 0.f;
                                 }
                                 // (a chunk with missing groups, kc < 8, occurs only when K % 256 != 0, and
                                 // then scales are never copied asynchronously: the loads above give 0)
@@ -704,8 +749,6 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                     const float2 cz = *reinterpret_cast<const float2 *>(smem + x7_o + coff);
                                     d[0] = cz.x; d[1] = cz.y; d[2] = cz.x; d[3] = cz.y;
                                 }
-                                const unsigned char *bp = smem + bo;
-                                const unsigned char *b0p = smem + bo0, *b1p = smem + bo1;
                                 const uint32_t wa4[4] = {qa.x, qa.y, qa.z, qa.w}, wb4[4] = {qb.x, qb.y, qb.z, qb.w};
                                 const uint32_t wc4[4] = {qc.x, qc.y, qc.z, qc.w}, wd4[4] = {qd.x, qd.y, qd.z, qd.w};
 #pragma unroll
@@ -714,11 +757,11 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                     // (xb.x, xb.y), (xb.z, xb.w); plain, (xa.x, xb.x), (xa.y, xb.y), ...
                                     uint4 xa, xb;
                                     if constexpr (PAIRED) {
-                                        xa = *reinterpret_cast<const uint4 *>(bp + 32 * t4);
-                                        xb = *reinterpret_cast<const uint4 *>(bp + 32 * t4 + 16);
+                                        xa = *reinterpret_cast<const uint4 *>(smem + bo + 32 * t4);
+                                        xb = *reinterpret_cast<const uint4 *>(smem + bo + 32 * t4 + 16);
                                     } else {
-                                        const uint4 x0 = *reinterpret_cast<const uint4 *>(b0p + 16 * t4);
-                                        const uint4 x1 = *reinterpret_cast<const uint4 *>(b1p + 16 * t4);
+                                        const uint4 x0 = *reinterpret_cast<const uint4 *>(smem + bo0 + 16 * t4);
+                                        const uint4 x1 = *reinterpret_cast<const uint4 *>(smem + bo1 + 16 * t4);
                                         xa = make_uint4(x0.x, x1.x, x0.y, x1.y);
                                         xb = make_uint4(x0.z, x1.z, x0.w, x1.w);
                                     }
@@ -762,8 +805,10 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                                                (size_t)r0 * (G >> gsh);
                                     const unsigned short *p1 = reinterpret_cast<const unsigned short *>(P.scales) +
                                                                (size_t)r1 * (G >> gsh);
+                                    const int wr = pass_weight_rows(kind, N), sr = G >> gsh;
                                     for (int gl = 0; gl < kc; ++gl) {
                                         const int b = (c * kMChunkG + gl) >> gsh;      // the block's scale
+                                        if (!chk(r0 >= 0 && r0 < wr && r1 >= 0 && r1 < wr && b < sr)) continue;
                                         u0[gl >> 1] |= (uint32_t)p0[b] << (16 * (gl & 1));
                                         u1[gl >> 1] |= (uint32_t)p1[b] << (16 * (gl & 1));
                                     }
@@ -845,7 +890,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                     }
 
                     // ---- tile epilogue ----
-                    if (have && g.wk > 1) {
+                    if (have && g.wk > 1 &&
+                        chk(((size_t)(WS ? g.my_wr : t) * g.wk + g.my_wk + 1) * PART <= (size_t)a.red_floats)) {
                         // this warp's partial of tile t; windowed rounds number their tiles
                         // from the round's first (my_wr)
                         float *rp = red + ((size_t)(WS ? g.my_wr : t) * g.wk + g.my_wk) * PART;
@@ -873,21 +919,21 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                                 if (m >= M) continue;
                                 if (kind == kEpiGateUp) {
                                     const int nn = o0 + qg;
-                                    if (nn < g.o_end) {
+                                    if (nn < g.o_end && chk(nn < N)) {
                                         const float gv = acc[nt][e] * pow2f(24), u = acc[nt][2 + e] * pow2f(24);
                                         const float silu = gv / (1.0f + expf(-gv));
                                         reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(silu * u);
                                     }
                                 } else if (!LOG && kind == kEpiRope) {
                                     const int nn = o0 + qg;
-                                    if (nn < g.o_end)
+                                    if (nn < g.o_end && chk(nn < N))
                                         rope_store(reinterpret_cast<__half *>(out), (size_t)m * ldo, nn, rope_d, P.theta,
                                                    ppos[m], acc[nt][e] * pow2f(24), acc[nt][2 + e] * pow2f(24));
                                 } else {
 #pragma unroll
                                     for (int h = 0; h < 2; ++h) {
                                         const int nn = o0 + qg + 8 * h;
-                                        if (nn >= g.o_end) continue;
+                                        if (nn >= g.o_end || !chk(nn < N)) continue;
                                         const float y = acc[nt][2 * h + e] * pow2f(24);
                                         if constexpr (!LOG) {
                                             reinterpret_cast<__half *>(out)[(size_t)m * ldo + nn] = __float2half_rn(y);
@@ -957,7 +1003,8 @@ __global__ void __launch_bounds__(MW * 32, MW == 16 ? 1 : 2) q4_pass_kernel(cons
                         }
                     }
                     consumer_sync();
-                    if (tid < M) {
+                    if (!chk(blockIdx.x < (unsigned)kMaxCtas && m0 + M <= Mt)) {
+                    } else if (tid < M) {
                         float bv = -INFINITY;
                         int bi = 0x7fffffff;
                         for (int w = 0; w < kMW; ++w) {

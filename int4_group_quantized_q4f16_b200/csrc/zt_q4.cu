@@ -306,6 +306,7 @@ int launch_q4(const uint32_t *qw, const uint16_t *scales, const uint16_t *x, voi
     a.counters = nullptr;
     a.error = nullptr;
     a.withhold = -1;
+    a.chk_cut = 0;
     PassProj &p = a.p[0];
     p.qw = reinterpret_cast<const uint4 *>(qw);
     p.scales = reinterpret_cast<const __half *>(scales);
@@ -602,7 +603,7 @@ int read_error_word(const void *p, unsigned int *out)
 
 extern "C" {
 
-int zt_q4_version(void) { return (1 << 16) | 5; }
+int zt_q4_version(void) { return (1 << 16) | 6; }
 
 const char *zt_q4_last_cuda_error(void)
 {
@@ -717,7 +718,7 @@ size_t zt_q4_pass_workspace_bytes(const zt_q4_proj *projs, int n, int M)
 }
 
 static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream,
-                     int withhold)
+                     int withhold, int chk_cut = 0)
 {
     if (!projs || !workspace || n < 1 || n > ZT_Q4_PASS_MAX || M < 1 || M > 16) return ZT_ERR_INVALID_ARG;
     bool cooperative = false;
@@ -767,6 +768,7 @@ static int pass_impl(const zt_q4_proj *projs, int n, int M, void *workspace, siz
     a.counters = cooperative ? reinterpret_cast<unsigned int *>(ws) : nullptr;
     a.error = reinterpret_cast<unsigned int *>(ws + err_off);
     a.withhold = cooperative ? withhold : -1;
+    a.chk_cut = chk_cut;
     size_t lm = lm_off;
     for (int i = 0; i < n; ++i) {
         const zt_q4_proj &q = projs[i];
@@ -874,6 +876,16 @@ int zt_q4_pass_test_withhold(const zt_q4_proj *projs, int n, int M, void *worksp
     if (!waits) return ZT_ERR_INVALID_ARG;
     return pass_impl(projs, n, M, workspace, ws_bytes, stream, 0);
 }
+
+int zt_q4_pass_test_cut(const zt_q4_proj *projs, int n, int M, void *workspace, size_t ws_bytes, void *stream,
+                        int rows)
+{
+    if (!kChecked) return ZT_ERR_UNSUPPORTED;
+    if (rows < 1) return ZT_ERR_INVALID_ARG;
+    return pass_impl(projs, n, M, workspace, ws_bytes, stream, -1, rows);
+}
+
+int zt_q4_build_flags(void) { return kChecked ? ZT_Q4_BUILD_CHECKED : 0; }
 
 int zt_q4_pass_errors(const void *workspace, int n, unsigned int *out)
 {

@@ -14,7 +14,11 @@ from typing import Optional, Tuple
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libzt_q4.so")
+# ZT_Q4_LIB names another build of the same library to load instead, e.g. the
+# bounds-checked libzt_q4_checked.so beside this file
+LIB_PATH = os.environ.get("ZT_Q4_LIB") or os.path.join(_PKG, "libzt_q4.so")
+CHECKED_LIB_PATH = os.path.join(_PKG, "libzt_q4_checked.so")
+ZT_Q4_ERR_BOUNDS = 2
 
 ZT_OK = 0
 ZT_ERR_INVALID_ARG = -1
@@ -82,6 +86,10 @@ def _load() -> ctypes.CDLL:
     lib.zt_q4_pass_plan.restype = ctypes.c_int
     lib.zt_q4_pass_test_withhold.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P]
     lib.zt_q4_pass_test_withhold.restype = ctypes.c_int
+    lib.zt_q4_pass_test_cut.argtypes = [ctypes.POINTER(ZtProj), _I, _I, _P, ctypes.c_size_t, _P, _I]
+    lib.zt_q4_pass_test_cut.restype = ctypes.c_int
+    lib.zt_q4_build_flags.argtypes = []
+    lib.zt_q4_build_flags.restype = ctypes.c_int
     lib.zt_q4_pass_errors.restype = ctypes.c_int
     lib.zt_q4_dequant_f16.argtypes = [_P, _P, _P, _I, _I, _I, _P]
     lib.zt_q4_gemm_f16w.argtypes = [_P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P]
@@ -122,6 +130,11 @@ def strerror(status: int) -> str:
 def version() -> Tuple[int, int]:
     v = lib.zt_q4_version()
     return v >> 16, v & 0xFFFF
+
+
+def is_checked_build() -> bool:
+    """True when the loaded library is the bounds-checked build (-DZT_Q4_CHECKED)."""
+    return bool(lib.zt_q4_build_flags() & 1)
 
 
 def _check(rc: int, what: str) -> None:
@@ -442,6 +455,12 @@ class Pass:
         zt_q4_pass_test_withhold); the next phase's bounded wait runs out."""
         _check(lib.zt_q4_pass_test_withhold(self.arr, self.n, self.M, self.workspace.data_ptr(),
                                             self.workspace.numel(), _stream_handle(stream)), "zt_q4_pass_test_withhold")
+
+    def run_with_cut_extent(self, rows: int, stream=None):
+        """Checked-build test: the pass with every weight extent ``rows`` rows short (see
+        zt_q4_pass_test_cut); the copies of the last rows fail their check and are skipped."""
+        _check(lib.zt_q4_pass_test_cut(self.arr, self.n, self.M, self.workspace.data_ptr(),
+                                       self.workspace.numel(), _stream_handle(stream), rows), "zt_q4_pass_test_cut")
 
     def errors(self) -> int:
         v = ctypes.c_uint(0)

@@ -286,6 +286,25 @@ def test_withhold_hook_needs_a_wait(zt):
     assert zt.lib.zt_q4_pass_test_withhold(None, 2, 1, FAKE, 1 << 20, None) == zt.ZT_ERR_INVALID_ARG
 
 
+def test_checked_build_hooks(zt):
+    """The default library is not the checked build and refuses its test hook before any
+    CUDA call; the checked library (where built) says so, loads, and exports the same ABI."""
+    import ctypes
+    P = zt.ZtProj
+    arr = (P * 1)(P(FAKE, FAKE, FAKE, FAKE, None, zt.ZT_Q4_GEMV, 64, 64, 0))
+    assert not zt.is_checked_build()
+    assert zt.lib.zt_q4_pass_test_cut(arr, 1, 1, FAKE, 1 << 20, None, 3) == zt.ZT_ERR_UNSUPPORTED
+    if not os.path.exists(zt.CHECKED_LIB_PATH):
+        pytest.skip("libzt_q4_checked.so not built")
+    lib = ctypes.CDLL(zt.CHECKED_LIB_PATH)
+    assert lib.zt_q4_build_flags() == 1
+    for sym in declared_symbols(HEADER):
+        assert hasattr(lib, sym), sym
+    lib.zt_q4_pass_test_cut.argtypes = [ctypes.POINTER(P), ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int]
+    assert lib.zt_q4_pass_test_cut(arr, 1, 1, FAKE, 1 << 20, None, 0) == zt.ZT_ERR_INVALID_ARG
+
+
 def test_gemm_gate_up_arguments(zt):
     f = zt.lib.zt_q4_gemm_gate_up_workspace_bytes
     assert f(512, 8192, 3072) == ((2 * 8192 * 3072 * 2 + 255) // 256) * 256 + 256
