@@ -117,5 +117,6 @@ def test_cut_extent_sets_the_error_bit(both, oracle, M):
     for d in projs:
         _check_against_oracle(oracle, d)
     # the default build refuses the hook
-    assert zt.lib.zt_q4_pass_test_cut(p.arr, p.n, p.M, p.workspace.data_ptr(), p.workspace.numel(),
+    pz = zt.Pass(projs)
+    assert zt.lib.zt_q4_pass_test_cut(pz.arr, pz.n, pz.M, pz.workspace.data_ptr(), pz.workspace.numel(),
                                       None, 3) == zt.ZT_ERR_UNSUPPORTED
